@@ -1,0 +1,100 @@
+"""Seeded synthetic inputs for the factorised linear: signs, scales, activations.
+
+This module draws random numbers and converts them to the storage dtypes; it holds none
+of the layer's arithmetic (no packing, no products, no sums).  Both the CUDA path and the
+CPU oracle are fed from it, so neither produces the other's inputs.
+
+Value distributions (the workloads of the factorised-linear benchmarks):
+  * sign entries of U and V: i.i.d. Bernoulli(0.5) -> {+1, -1}
+  * scale vectors s1, s2: U(0.5, 1.5) * 0.02, rounded to fp16
+  * activations x: N(0, 1), rounded to bfloat16 (round to nearest even)
+Every draw is keyed by an integer seed plus a tuple of tags (layer, tensor name, ...)
+through numpy's SeedSequence, so any single tensor can be regenerated alone.
+"""
+from __future__ import annotations
+
+import zlib
+
+import numpy as np
+
+
+def _rng(seed: int, *tags) -> np.random.Generator:
+    words = [int(seed) & 0xFFFFFFFF]
+    for t in tags:
+        if isinstance(t, str):
+            words.append(zlib.crc32(t.encode()))
+        else:
+            words.append(int(t) & 0xFFFFFFFF)
+    return np.random.default_rng(np.random.SeedSequence(words))
+
+
+def signs(rows: int, cols: int, seed: int, *tags) -> np.ndarray:
+    """rows x cols int8 in {+1, -1}, each entry +1 with probability 1/2."""
+    bits = _rng(seed, "signs", rows, cols, *tags).integers(0, 2, size=(rows, cols), dtype=np.int8)
+    return (2 * bits - 1).astype(np.int8)
+
+
+def random_words(rows: int, words: int, seed: int, *tags) -> np.ndarray:
+    """rows x words uint32 of independent fair random bits.
+
+    Under the one-bit-per-sign storage (bit 1 = +1) these are exactly the stored form of
+    i.i.d. Bernoulli(0.5) sign matrices; large benchmark weights are drawn this way to
+    avoid materialising billions of int8 signs on the host.
+    """
+    g = _rng(seed, "words", rows, words, *tags)
+    return g.integers(0, 1 << 32, size=(rows, words), dtype=np.uint64).astype(np.uint32)
+
+
+def scales_f16(length: int, seed: int, *tags) -> np.ndarray:
+    """length fp16 values U(0.5, 1.5) * 0.02, returned as their uint16 bit patterns."""
+    u = _rng(seed, "scales", length, *tags).uniform(0.5, 1.5, size=length) * 0.02
+    return u.astype(np.float16).view(np.uint16)
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float32 -> bfloat16 bit patterns, round to nearest, ties to even (finite inputs)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """bfloat16 bit patterns -> float32 (exact)."""
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def activations_bf16(batch: int, n: int, seed: int, *tags) -> np.ndarray:
+    """batch x n bfloat16 N(0, 1) activations, as uint16 bit patterns."""
+    z = _rng(seed, "x", batch, n, *tags).standard_normal(size=(batch, n)).astype(np.float32)
+    return f32_to_bf16_bits(z)
+
+
+def f16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float32)
+
+
+# Layer shapes of the benchmark workloads: (name, m_out, n_in, rank).
+LLAMA2_7B_LAYERS = [
+    ("q", 4096, 4096, 1664),
+    ("k", 4096, 4096, 1664),
+    ("v", 4096, 4096, 1664),
+    ("o", 4096, 4096, 1664),
+    ("gate", 11008, 4096, 2432),
+    ("up", 11008, 4096, 2432),
+    ("down", 4096, 11008, 2432),
+]
+
+LLAMA2_70B_LAYERS = [
+    ("q", 8192, 8192, 2432),
+    ("k", 1024, 8192, 384),
+    ("v", 1024, 8192, 384),
+    ("o", 8192, 8192, 2432),
+    ("gate", 28672, 8192, 3840),
+    ("up", 28672, 8192, 3840),
+    ("down", 8192, 28672, 3840),
+]
+
+SMALL_LAYER = ("single", 512, 512, 128)
+
+PREFILL_SHAPE = ("gate", 11008, 4096, 2432)
+PREFILL_BATCHES = (16, 128, 1024, 4096)

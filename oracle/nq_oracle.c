@@ -1,0 +1,210 @@
+/*
+ * nq_oracle.c -- plain CPU fp64 oracle for the low-rank binary factorised linear.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the CUDA library and its
+ * Python binding) includes, links or calls this file; only the tests, the smoke check
+ * and the CPU-baseline leg of the benchmark do.  It shares no code, header, table or
+ * helper with the CUDA sources: its own bit reader, its own bf16/fp16 decoders.
+ *
+ * What it computes, and where that is defined:
+ *
+ *  - The weight of a factorised linear layer is a product of +1/-1 matrices and
+ *    diagonal scaling vectors (hardwired.dev, "NanoQuant jednoduse: 70B model na herni
+ *    grafice", section "Jak NanoQuant funguje"; rapidrecap.app "Nanoquant: Efficient
+ *    Sub-1-Bit Quantization of Large Language Models", section "Quantization Technique":
+ *    U and V binary matrices plus scaling factors).  Read here as
+ *        W = diag(s1) . U . V^T . diag(s2),   U in {+1,-1}^{m x r},  V in {+1,-1}^{n x r},
+ *    s1 (m) and s2 (n) fp16, and the layer output
+ *        y = s1 (.) ( U . ( V^T . ( s2 (.) x ) ) ).
+ *  - The sign matrices are stored one bit per entry (same section of hardwired.dev:
+ *    r*(m+n) binary values plus the scales).  Storage bit 1 stands for +1, bit 0 for -1;
+ *    32 entries per uint32, least significant bit first, words contiguous along the
+ *    reduction dimension:  bit b of word w of a row = column 32*w + b.
+ *    U is stored as its m rows (reduction over r), V as the r rows of V^T (reduction
+ *    over n).  A row of `cols` entries takes ceil(cols/32) words; unused high bits of
+ *    the last word are zero.
+ *  - sign(0) is taken as +1 (the sign projection of the ADMM step, hardwired.dev section
+ *    "Krok 2", does not say; this is the reading used throughout).
+ *  - Bits per weight = (r*(m+n) + 16*(m+n)) / (m*n): r(m+n) one-bit entries plus two
+ *    fp16 scale vectors (hardwired.dev sections "Jak NanoQuant funguje" and
+ *    "Co znamena sub-1-bit").
+ *
+ * Arithmetic: every input is decoded exactly into double; x' = s2*x is exact in double
+ * (8-bit by 11-bit significands); sums run in increasing index order in double.  The
+ * optional OpenMP pragma only spreads independent output rows over threads; it does not
+ * change any sum.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_OK 0
+#define ORC_ERR_ARG (-1)
+#define ORC_ERR_VALUE (-5)
+
+/* ---- exact decoders, written from the IEEE 754 binary16 / bfloat16 bit layouts ---- */
+
+/* bfloat16: 1 sign bit, 8 exponent bits (bias 127), 7 fraction bits.  It is the upper
+ * half of an IEEE binary32, so the value is that binary32 with 16 zero bits appended.
+ * Decoded here from the fields, without type punning, so it is checkable by eye. */
+double orc_bf16_to_double(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int expo = (h >> 7) & 0xFF;
+    int frac = h & 0x7F;
+    double v;
+    if (expo == 0xFF) {
+        v = frac ? NAN : INFINITY;
+    } else if (expo == 0) {
+        v = ldexp((double)frac, -126 - 7);           /* subnormal: 0.frac * 2^-126 */
+    } else {
+        v = ldexp((double)(frac | 0x80), expo - 127 - 7); /* 1.frac * 2^(e-127) */
+    }
+    return sign ? -v : v;
+}
+
+/* binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+double orc_f16_to_double(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int expo = (h >> 10) & 0x1F;
+    int frac = h & 0x3FF;
+    double v;
+    if (expo == 0x1F) {
+        v = frac ? NAN : INFINITY;
+    } else if (expo == 0) {
+        v = ldexp((double)frac, -14 - 10);            /* subnormal: 0.frac * 2^-14 */
+    } else {
+        v = ldexp((double)(frac | 0x400), expo - 15 - 10);
+    }
+    return sign ? -v : v;
+}
+
+/* ---- storage of the sign matrices ---- */
+
+static int64_t words_per_row(int64_t cols) { return (cols + 31) / 32; }
+
+/* The entry (row, col) of a packed sign matrix, as +1 or -1. */
+static int orc_sign_at(const uint32_t *packed, int64_t wpr, int64_t row, int64_t col) {
+    uint32_t word = packed[row * wpr + col / 32];
+    return ((word >> (col % 32)) & 1u) ? +1 : -1;
+}
+
+/* Pack a rows x cols matrix of int8 signs (row-major) into rows x ceil(cols/32) words.
+ * Entries must be -1, 0 or +1; 0 packs as +1.  Any other value: ORC_ERR_VALUE and the
+ * output is left untouched. */
+int orc_pack_signs(const int8_t *signs, int64_t rows, int64_t cols, uint32_t *out) {
+    if (rows < 0 || cols < 0 || (rows * cols > 0 && (!signs || !out))) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < rows * cols; ++i)
+        if (signs[i] < -1 || signs[i] > 1) return ORC_ERR_VALUE;
+    int64_t wpr = words_per_row(cols);
+    for (int64_t row = 0; row < rows; ++row) {
+        for (int64_t w = 0; w < wpr; ++w) {
+            uint32_t word = 0;
+            for (int b = 0; b < 32; ++b) {
+                int64_t col = 32 * w + b;
+                if (col < cols && signs[row * cols + col] >= 0) word |= (1u << b);
+            }
+            out[row * wpr + w] = word;
+        }
+    }
+    return ORC_OK;
+}
+
+/* Inverse of orc_pack_signs: rows x cols int8 in {-1, +1}. */
+int orc_unpack_signs(const uint32_t *packed, int64_t rows, int64_t cols, int8_t *out) {
+    if (rows < 0 || cols < 0 || (rows * cols > 0 && (!packed || !out))) return ORC_ERR_ARG;
+    int64_t wpr = words_per_row(cols);
+    for (int64_t row = 0; row < rows; ++row)
+        for (int64_t col = 0; col < cols; ++col)
+            out[row * cols + col] = (int8_t)orc_sign_at(packed, wpr, row, col);
+    return ORC_OK;
+}
+
+/* ---- the forward pass ----
+ *
+ * x   : batch x n bfloat16 bit patterns, row-major (one token per row)
+ * Upk : m rows of ceil(r/32) words   (row i holds U[i][0..r))
+ * Vpk : r rows of ceil(n/32) words   (row k holds V^T[k][0..n) = V[0..n)[k])
+ * s1  : m fp16 bit patterns;  s2 : n fp16 bit patterns
+ * y   : batch x m doubles (written)
+ */
+int orc_lowrank_linear_fwd(const uint16_t *x, const uint32_t *Upk, const uint32_t *Vpk,
+                           const uint16_t *s1, const uint16_t *s2, int64_t m, int64_t n,
+                           int64_t r, int64_t batch, double *y) {
+    if (m <= 0 || n <= 0 || r <= 0 || batch < 0) return ORC_ERR_ARG;
+    if (batch == 0) return ORC_OK;
+    if (!x || !Upk || !Vpk || !s1 || !s2 || !y) return ORC_ERR_ARG;
+    const int64_t wpr_u = words_per_row(r), wpr_v = words_per_row(n);
+    double *xs = (double *)malloc(sizeof(double) * (size_t)(n * batch));
+    double *t = (double *)malloc(sizeof(double) * (size_t)(r * batch));
+    if (!xs || !t) { free(xs); free(t); return ORC_ERR_ARG; }
+
+    /* step 1: x' = s2 (.) x, exact in double */
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t j = 0; j < n; ++j)
+            xs[b * n + j] = orc_f16_to_double(s2[j]) * orc_bf16_to_double(x[b * n + j]);
+
+    /* step 2: t_k = sum_j V[j][k] * x'_j, increasing j */
+#pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k < r; ++k) {
+        for (int64_t b = 0; b < batch; ++b) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < n; ++j)
+                acc += orc_sign_at(Vpk, wpr_v, k, j) * xs[b * n + j];
+            t[b * r + k] = acc;
+        }
+    }
+
+    /* step 3: y_i = s1_i * sum_k U[i][k] * t_k, increasing k */
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < m; ++i) {
+        double si = orc_f16_to_double(s1[i]);
+        for (int64_t b = 0; b < batch; ++b) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < r; ++k)
+                acc += orc_sign_at(Upk, wpr_u, i, k) * t[b * r + k];
+            y[b * m + i] = si * acc;
+        }
+    }
+    free(xs);
+    free(t);
+    return ORC_OK;
+}
+
+/* The intermediate t = V^T (s2 (.) x) alone (batch x r doubles), for tests that look
+ * at the rank bottleneck. */
+int orc_stage1(const uint16_t *x, const uint32_t *Vpk, const uint16_t *s2, int64_t n,
+               int64_t r, int64_t batch, double *t) {
+    if (n <= 0 || r <= 0 || batch < 0) return ORC_ERR_ARG;
+    if (batch == 0) return ORC_OK;
+    if (!x || !Vpk || !s2 || !t) return ORC_ERR_ARG;
+    const int64_t wpr_v = words_per_row(n);
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t k = 0; k < r; ++k) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < n; ++j)
+                acc += orc_sign_at(Vpk, wpr_v, k, j) *
+                       (orc_f16_to_double(s2[j]) * orc_bf16_to_double(x[b * n + j]));
+            t[b * r + k] = acc;
+        }
+    return ORC_OK;
+}
+
+/* Storage accounting: (r(m+n) + 16(m+n)) / (mn); -1.0 if any argument is <= 0. */
+double orc_bits_per_weight(int64_t m, int64_t n, int64_t r) {
+    if (m <= 0 || n <= 0 || r <= 0) return -1.0;
+    double num = (double)r * (double)(m + n) + 16.0 * (double)(m + n);
+    return num / ((double)m * (double)n);
+}
+
+/* Number of threads the parallel loops above use (1 without OpenMP). */
+int orc_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,245 @@
+"""Checks that tie the CPU oracle to facts fixed outside itself.
+
+Each function takes an ``oracle.Oracle`` and raises AssertionError on a mismatch, so the
+same checks run on the real oracle (they must pass) and on deliberately broken copies of
+it (each copy must fail at least one).  Sources of truth, none of them the oracle:
+  * hand-worked numbers in tests/golden/ (each file states its derivation and passage);
+  * the materialised weight diag(s1) U V^T diag(s2) built with numpy from the int8
+    signs, then one numpy matrix-vector product (a different order of operations and a
+    different reader of the signs than the oracle's bit reader);
+  * closed forms (all-(+1) signs, rank 1), invariances (negating column k of both U and
+    V), linearity, and numpy's / torch's own fp16 and bf16 conversions.
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+
+from binary_rank_linear_02_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden_kv(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            out[key] = vals
+    return out
+
+
+def load_pack_patterns():
+    rows = []
+    with open(os.path.join(GOLDEN, "pack_patterns.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            name, cols, pattern, words = [p.strip() for p in line.split("|")]
+            cols = int(cols)
+            kind, arg = pattern.split(":")
+            if kind == "all":
+                s = np.full(cols, int(arg), dtype=np.int8)
+            elif kind == "alt":
+                first = int(arg)
+                s = np.array([first if c % 2 == 0 else -first for c in range(cols)], dtype=np.int8)
+            elif kind == "one":
+                s = np.full(cols, -1, dtype=np.int8)
+                s[int(arg)] = 1
+            else:
+                raise ValueError(kind)
+            expected = np.array([int(w, 16) for w in words.split()], dtype=np.uint32)
+            rows.append((name, s.reshape(1, cols), expected.reshape(1, -1)))
+    return rows
+
+
+def load_bits_per_weight():
+    out = []
+    with open(os.path.join(GOLDEN, "bits_per_weight.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            m, n, r, num, den = (int(v) for v in line.split())
+            out.append((m, n, r, num, den))
+    return out
+
+
+def dense_reference(x_bits, U, V, s1_bits, s2_bits):
+    """y = x W^T with W = diag(s1) U V^T diag(s2), materialised with numpy in float64."""
+    x = synth.bf16_bits_to_f32(x_bits).astype(np.float64)
+    s1 = synth.f16_bits_to_f32(s1_bits).astype(np.float64)
+    s2 = synth.f16_bits_to_f32(s2_bits).astype(np.float64)
+    W = (s1[:, None] * (U.astype(np.float64) @ V.astype(np.float64).T)) * s2[None, :]
+    return x @ W.T
+
+
+def rel_err(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-300))
+
+
+# ---------------------------------------------------------------- individual pins
+
+def pin_decoders(o):
+    """Every finite fp16 / bf16 bit pattern decodes to numpy's / the IEEE value."""
+    allbits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):
+        f16 = allbits.view(np.float16).astype(np.float64)
+        bf16 = synth.bf16_bits_to_f32(allbits).astype(np.float64)
+    for b in range(0, 1 << 16, 7):  # a stride that visits every exponent and both signs
+        if np.isfinite(f16[b]):
+            assert o.f16_to_double(b) == f16[b], f"fp16 {b:#06x}"
+        if np.isfinite(bf16[b]):
+            assert o.bf16_to_double(b) == bf16[b], f"bf16 {b:#06x}"
+    for b in (0x0001, 0x03FF, 0x0400, 0x3C00, 0x7BFF, 0x8001, 0xFBFF):
+        assert o.f16_to_double(b) == f16[b]
+    for b in (0x0001, 0x007F, 0x0080, 0x3F80, 0x7F7F, 0x8001, 0xC000):
+        assert o.bf16_to_double(b) == bf16[b]
+
+
+def pin_pack_patterns(o):
+    for name, signs, expected in load_pack_patterns():
+        got = o.pack_signs(signs)
+        assert got.shape == expected.shape and np.array_equal(got, expected), name
+        back = o.unpack_signs(got, signs.shape[1])
+        assert np.array_equal(back, np.where(signs >= 0, 1, -1)), name
+
+
+def pin_pack_roundtrip(o):
+    for rows, cols, seed in ((3, 70, 1), (17, 128, 2), (5, 33, 3)):
+        s = synth.signs(rows, cols, seed)
+        p = o.pack_signs(s)
+        assert p.shape == (rows, (cols + 31) // 32)
+        assert np.array_equal(o.unpack_signs(p, cols), s)
+        # the words count the +1 entries: popcount of each row = number of +1 in it
+        pc = np.array([sum(bin(int(w)).count("1") for w in row) for row in p])
+        assert np.array_equal(pc, (s > 0).sum(axis=1))
+
+
+def pin_handworked(o):
+    g = _golden_kv("handworked_small.txt")
+    m, n, r, batch = (int(g[k][0]) for k in ("m", "n", "r", "batch"))
+    x = np.array([int(v, 16) for v in g["x_bf16"]], dtype=np.uint16).reshape(batch, n)
+    s1 = np.array([int(v, 16) for v in g["s1_f16"]], dtype=np.uint16)
+    s2 = np.array([int(v, 16) for v in g["s2_f16"]], dtype=np.uint16)
+    U = np.array([int(v) for v in g["U_signs"]], dtype=np.int8).reshape(m, r)
+    V = np.array([int(v) for v in g["V_signs"]], dtype=np.int8).reshape(n, r)
+    Upk = np.array([int(v, 16) for v in g["Upk"]], dtype=np.uint32).reshape(m, 1)
+    Vpk = np.array([int(v, 16) for v in g["Vpk"]], dtype=np.uint32).reshape(r, 1)
+    assert np.array_equal(o.pack_signs(U), Upk)
+    assert np.array_equal(o.pack_signs(np.ascontiguousarray(V.T)), Vpk)
+    t = o.stage1(x, Vpk, s2, n, r)
+    assert np.array_equal(t, np.array([float(v) for v in g["t"]]).reshape(batch, r))
+    y = o.lowrank_linear_fwd(x, Upk, Vpk, s1, s2, m, n, r)
+    assert np.array_equal(y, np.array([float(v) for v in g["y"]]).reshape(batch, m))
+
+
+def _case(m, n, r, batch, seed):
+    U = synth.signs(m, r, seed, "U")
+    V = synth.signs(n, r, seed, "V")
+    s1 = synth.scales_f16(m, seed, "s1")
+    s2 = synth.scales_f16(n, seed, "s2")
+    x = synth.activations_bf16(batch, n, seed)
+    return x, U, V, s1, s2
+
+
+def _fwd(o, x, U, V, s1, s2):
+    m, r = U.shape
+    n = V.shape[0]
+    return o.lowrank_linear_fwd(x, o.pack_signs(U), o.pack_signs(np.ascontiguousarray(V.T)), s1, s2, m, n, r)
+
+
+def pin_dense_materialised(o):
+    """Factorised evaluation equals the materialised dense product (fp64, 1e-12)."""
+    for (m, n, r, batch, seed) in ((8, 12, 3, 2, 11), (33, 40, 7, 3, 12), (64, 64, 64, 2, 13), (5, 70, 40, 1, 14)):
+        x, U, V, s1, s2 = _case(m, n, r, batch, seed)
+        y = _fwd(o, x, U, V, s1, s2)
+        y_ref = dense_reference(x, U, V, s1, s2)
+        assert y.shape == (batch, m)
+        assert rel_err(y, y_ref) <= 1e-12, (m, n, r, rel_err(y, y_ref))
+
+
+def pin_column_negation(o):
+    """Negating column k of both U and V leaves y bit-identical (t_k and U_ik flip together)."""
+    x, U, V, s1, s2 = _case(48, 64, 9, 2, 21)
+    y0 = _fwd(o, x, U, V, s1, s2)
+    for k in (0, 4, 8):
+        U2, V2 = U.copy(), V.copy()
+        U2[:, k] *= -1
+        V2[:, k] *= -1
+        assert np.array_equal(_fwd(o, x, U2, V2, s1, s2), y0), k
+    # negating only one factor's column changes y (so the check above has teeth)
+    U3 = U.copy()
+    U3[:, 4] *= -1
+    assert not np.array_equal(_fwd(o, x, U3, V, s1, s2), y0)
+
+
+def pin_closed_forms(o):
+    m, n, batch = 24, 40, 2
+    x, _, _, s1, s2 = _case(m, n, 1, batch, 31)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    s1f = synth.f16_bits_to_f32(s1).astype(np.float64)
+    s2f = synth.f16_bits_to_f32(s2).astype(np.float64)
+    # all signs +1: y_i = s1_i * r * sum_j s2_j x_j
+    for r in (1, 5, 32):
+        U = np.ones((m, r), dtype=np.int8)
+        V = np.ones((n, r), dtype=np.int8)
+        y = _fwd(o, x, U, V, s1, s2)
+        expect = s1f[None, :] * r * (xf @ s2f)[:, None]
+        assert rel_err(y, expect) <= 1e-13
+    # rank 1: y = s1 * u * (v . (s2 * x))
+    u = synth.signs(m, 1, 32)
+    v = synth.signs(n, 1, 33)
+    y = _fwd(o, x, u, v, s1, s2)
+    expect = (s1f * u[:, 0])[None, :] * ((xf * s2f[None, :]) @ v[:, 0].astype(np.float64))[:, None]
+    assert rel_err(y, expect) <= 1e-13
+
+
+def pin_linearity(o):
+    m, n, r = 20, 48, 6
+    _, U, V, s1, s2 = _case(m, n, r, 1, 41)
+    rng = np.random.default_rng(41)
+    # small-integer activations: x1, x2 and x1 + x2 are all exact in bfloat16
+    x1 = rng.integers(-8, 9, size=(2, n)).astype(np.float32)
+    x2 = rng.integers(-8, 9, size=(2, n)).astype(np.float32)
+    b = synth.f32_to_bf16_bits
+    y1 = _fwd(o, b(x1), U, V, s1, s2)
+    y2 = _fwd(o, b(x2), U, V, s1, s2)
+    y12 = _fwd(o, b(x1 + x2), U, V, s1, s2)
+    assert rel_err(y12, y1 + y2) <= 1e-12
+    y3 = _fwd(o, b(-2 * x1), U, V, s1, s2)
+    assert np.array_equal(y3, -2 * y1)
+    # y is linear in s1: doubling every s1 (exact in fp16) doubles y exactly
+    s1d = (synth.f16_bits_to_f32(s1) * 2).astype(np.float16).view(np.uint16)
+    assert np.array_equal(_fwd(o, b(x1), U, V, s1d, s2), 2 * y1)
+
+
+def pin_bits_per_weight(o):
+    for (m, n, r, num, den) in load_bits_per_weight():
+        assert o.bits_per_weight(m, n, r) == num / den, (m, n, r)
+        # the same figure from the sizes of the stored buffers
+        packed_bytes = m * ((r + 31) // 32) * 4 + r * ((n + 31) // 32) * 4
+        scale_bytes = 2 * (m + n)
+        assert 8 * (packed_bytes + scale_bytes) / (m * n) == num / den
+    for bad in ((0, 4, 4), (4, -1, 4), (4, 4, 0)):
+        assert o.bits_per_weight(*bad) == -1.0
+
+
+ALL_PINS = [
+    pin_decoders,
+    pin_pack_patterns,
+    pin_pack_roundtrip,
+    pin_handworked,
+    pin_dense_materialised,
+    pin_column_negation,
+    pin_closed_forms,
+    pin_linearity,
+    pin_bits_per_weight,
+]

@@ -1,0 +1,51 @@
+"""Each plausible mistake planted in a copy of the oracle must be caught by a pin.
+
+The copy is the oracle's own C source with one textual change, compiled to a temporary
+library on the CPU; the real oracle is not touched.  Every mutant keeps all memory
+accesses in bounds for the shapes the pins use (square-safe index swaps are avoided).
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "nq_oracle.c")
+
+MUTANTS = {
+    "drop_s2": ("orc_f16_to_double(s2[j]) * orc_bf16_to_double(x[b * n + j]);\n\n    /* step 2",
+                "orc_bf16_to_double(x[b * n + j]);\n\n    /* step 2"),
+    "drop_s1": ("y[b * m + i] = si * acc;", "y[b * m + i] = acc;"),
+    "sign_flip": ("& 1u) ? +1 : -1;", "& 1u) ? -1 : +1;"),
+    "msb_first": ("(word >> (col % 32))", "(word >> (31 - col % 32))"),
+    "pack_zero_as_minus": ("signs[row * cols + col] >= 0", "signs[row * cols + col] > 0"),
+    "t_skips_last": ("acc += orc_sign_at(Vpk, wpr_v, k, j) * xs[b * n + j];",
+                     "if (j + 1 < n) acc += orc_sign_at(Vpk, wpr_v, k, j) * xs[b * n + j];"),
+    "bpw_no_scales": ("+ 16.0 * (double)(m + n)", "+ 0.0 * (double)(m + n)"),
+    "f16_bias": ("expo - 15 - 10", "expo - 16 - 10"),
+    "bf16_subnormal": ("-126 - 7", "-127 - 7"),
+    "t_wrong_token": ("orc_sign_at(Vpk, wpr_v, k, j) * xs[b * n + j];", "orc_sign_at(Vpk, wpr_v, k, j) * xs[j];"),
+    "y_wrong_t_index": ("acc += orc_sign_at(Upk, wpr_u, i, k) * t[b * r + k];",
+                        "acc += orc_sign_at(Upk, wpr_u, i, k) * t[b * r + (k + 1) % r];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    before, after = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, f"mutation site for {name} not unique"
+    mutated = tmp_path / "mut.c"
+    mutated.write_text(src.replace(before, after))
+    lib = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O1", "-fPIC", "-shared", "-std=c11", "-o", str(lib), str(mutated), "-lm"])
+    o = oracle.Oracle(str(lib))
+    failures = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(o)
+        except (AssertionError, ValueError):
+            failures.append(pin.__name__)
+    assert failures, f"mutant {name} passed every pin"
