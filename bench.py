@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Benchmark of the factorised binary low-rank linear, y = s1 * (U (V^T (s2 * x))).
+
+Default workload (one "step"): the seven linears of a Llama-2-7B-shaped block
+(q/k/v/o 4096x4096 r=1664, gate/up 11008x4096 r=2432, down 4096x11008 r=2432) at decode
+batch 1, each layer with its own seeded input, all through the C ABI
+(nq_lowrank_linear_fwd) on one stream, the whole run captured in CUDA graphs.
+Metric: packed-weight HBM GB/s = (packed sign bytes of the seven layers) x steps / time.
+The weights rotate over enough seeded copies (> 2x the 126 MB L2) that every step
+streams its signs from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...   (independent replicas, one per GPU)
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead
+(rank 0 only) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from binary_rank_linear_02_b200 import synth  # noqa: E402
+
+METRIC = "packed-weight HBM GB/s (decode) & TFLOP/s (prefill), binary low-rank linear"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def packed_bytes(m, n, r):
+    return r * (m + n) // 8
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks during the timed region
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="nq_clocks_", suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons, n = [], [], set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                n += 1
+                for name, flag in zip(names, parts[5:9]):
+                    if flag.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": n}
+
+
+# ------------------------------------------------------------------ the decode workload on the GPU
+
+class DecodeWorkload:
+    """Seven factorised linears per step, weights rotating over `copies` seeded sets."""
+
+    def __init__(self, layers, batch, seed, device, min_bytes=2 * L2_BYTES):
+        import torch
+
+        from binary_rank_linear_02_b200 import nq
+
+        self.nq = nq
+        self.layers = layers
+        self.batch = batch
+        self.step_bytes = sum(packed_bytes(m, n, r) for _, m, n, r in layers)
+        self.copies = max(1, -(-min_bytes // self.step_bytes))
+        gen = torch.Generator(device=device)
+        gen.manual_seed(seed)
+        self.sets = []
+        for c in range(self.copies):
+            per = []
+            for li, (name, m, n, r) in enumerate(layers):
+                Upk = torch.randint(-(1 << 31), 1 << 31, (m, r // 32), dtype=torch.int64, device=device,
+                                    generator=gen).to(torch.int32)
+                Vpk = torch.randint(-(1 << 31), 1 << 31, (r, n // 32), dtype=torch.int64, device=device,
+                                    generator=gen).to(torch.int32)
+                s1 = torch.from_numpy(synth.scales_f16(m, seed, c, li, "s1").view(np.int16)).to(device)
+                s2 = torch.from_numpy(synth.scales_f16(n, seed, c, li, "s2").view(np.int16)).to(device)
+                per.append((Upk, Vpk, s1, s2))
+            self.sets.append(per)
+        self.x = [torch.from_numpy(synth.activations_bf16(batch, n, seed, li, "x").view(np.int16)).to(device)
+                  for li, (_, m, n, r) in enumerate(layers)]
+        self.y = [torch.empty((batch, m), dtype=torch.float32, device=device) for (_, m, n, r) in layers]
+        for (_, m, n, r) in layers:
+            nq.workspace_reserve(m, n, r, batch)
+
+    def step(self, i, stream_handle, layer_filter=None):
+        per = self.sets[i % self.copies]
+        fwd = self.nq.lib().nq_lowrank_linear_fwd
+        for li, (name, m, n, r) in enumerate(self.layers):
+            if layer_filter is not None and li != layer_filter:
+                continue
+            Upk, Vpk, s1, s2 = per[li]
+            st = fwd(self.x[li].data_ptr(), Upk.data_ptr(), Vpk.data_ptr(), s1.data_ptr(), s2.data_ptr(),
+                     m, n, r, self.batch, self.y[li].data_ptr(), stream_handle)
+            if st != 0:
+                raise RuntimeError(f"nq_lowrank_linear_fwd: {self.nq.nq_status_string(st)}")
+
+
+def capture(fn, stream):
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        fn(torch.cuda.current_stream().cuda_stream)
+    return g
+
+
+def timed_graphs(work, steps, warmup, stream, layer_filter=None, dist=None):
+    """Capture graphs covering `steps` steps (rotating copies) and time them with events."""
+    import torch
+
+    full = capture(lambda h: [work.step(i, h, layer_filter) for i in range(work.copies)], stream)
+    rem = steps % work.copies
+    part = capture(lambda h: [work.step(i, h, layer_filter) for i in range(rem)], stream) if rem else None
+    reps = steps // work.copies
+    for _ in range(max(1, -(-warmup // work.copies))):
+        full.replay()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(reps):
+            full.replay()
+        if part is not None:
+            part.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    if dist is not None:
+        dist.barrier()
+    del full, part
+    return ms
+
+
+def run_ours(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+        dist = tdist
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    from binary_rank_linear_02_b200 import nq
+
+    peaks = load_peaks()
+    layers = synth.LLAMA2_7B_LAYERS
+    batch = args.batch
+    work = DecodeWorkload(layers, batch, seed=1234 + rank, device=device)
+    stream = torch.cuda.Stream(device)
+    # first calls outside capture (kernel attributes, workspace)
+    with torch.cuda.stream(stream):
+        work.step(0, stream.cuda_stream)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    sampler.start()
+    ms = timed_graphs(work, args.steps, args.warmup, stream, dist=dist)
+    clocks = sampler.stop()
+    ms_max = ms
+    if dist is not None:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    total_bytes = work.step_bytes * args.steps * world
+    value = total_bytes / (ms_max * 1e-3) / 1e9
+    tokens_per_s = batch * args.steps * world / (ms_max * 1e-3)
+
+    # roofline: the largest layer (gate) alone, back to back over its own rotating copies
+    gate = [l for l in layers if l[0] == "gate"][0]
+    _, gm, gn, gr = gate
+    gwork = DecodeWorkload([gate], batch, seed=777 + rank, device=device)
+    with torch.cuda.stream(stream):
+        gwork.step(0, stream.cuda_stream)
+    torch.cuda.synchronize()
+    r_steps = max(gwork.copies * 10, 500)
+    ms_gate = timed_graphs(gwork, r_steps, args.warmup, stream)
+    del gwork
+    gate_bytes = packed_bytes(gm, gn, gr)
+    achieved = gate_bytes * r_steps / (ms_gate * 1e-3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get("gate_b%d_dram_bytes_per_call" % batch)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "kernel": f"decode layer {gm}x{gn} r={gr} batch {batch} (stage-1 + stage-2 kernels)",
+                "peak_source": peaks["source"]}
+
+    # end to end through the public API with host buffers (pinned), synchronous per call
+    e2e = run_e2e(work, stream, min(args.steps, 100), device)
+
+    # secondary: batch 8 decode on the same shapes
+    secondary = {}
+    if args.secondary and batch == 1 and world == 1:
+        w8 = DecodeWorkload(layers, 8, seed=99, device=device)
+        with torch.cuda.stream(stream):
+            w8.step(0, stream.cuda_stream)
+        torch.cuda.synchronize()
+        ms8 = timed_graphs(w8, args.steps, args.warmup, stream)
+        secondary["decode_b8_gbs"] = round(w8.step_bytes * args.steps / (ms8 * 1e-3) / 1e9, 1)
+        secondary["decode_b8_tokens_per_s"] = round(8 * args.steps / (ms8 * 1e-3), 1)
+        del w8
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = run_cpu_baseline(layers, batch, budget_s=args.cpu_seconds)
+
+    launches = args.steps * len(layers) * 2
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in; int8x2-limb tensor-core products, int32/fp32 acc",
+            "data": "synthetic",
+            "config": {"workload": f"llama2-7b-shaped decode, batch {batch}: 7 factorised linears per step "
+                                   "(q/k/v/o 4096x4096 r1664, gate/up 11008x4096 r2432, down 4096x11008 r2432)",
+                       "batch": batch, "packed_bytes_per_step": work.step_bytes,
+                       "l2": f"weights rotate over {work.copies} seeded copies "
+                             f"({work.copies * work.step_bytes / 1e6:.0f} MB > 2x L2)",
+                       "graphs": "CUDA graphs of the C-ABI calls", "parallelism": f"replicas x{world}"},
+            "tokens_per_s": round(tokens_per_s, 1),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+            "secondary": secondary,
+        }
+        print(json.dumps(line), flush=True)
+    del work
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(work, stream, steps, device):
+    import torch
+
+    nq = work.nq
+    xs = [x.cpu().pin_memory() for x in work.x]
+    ys = [torch.empty(y.shape, dtype=torch.float32).pin_memory() for y in work.y]
+    fwd = nq.lib().nq_lowrank_linear_fwd
+    h = stream.cuda_stream
+
+    def one(i):
+        per = work.sets[i % work.copies]
+        for li, (name, m, n, r) in enumerate(work.layers):
+            Upk, Vpk, s1, s2 = per[li]
+            st = fwd(xs[li].data_ptr(), Upk.data_ptr(), Vpk.data_ptr(), s1.data_ptr(), s2.data_ptr(), m, n, r,
+                     work.batch, ys[li].data_ptr(), h)
+            if st != 0:
+                raise RuntimeError(nq.nq_status_string(st))
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(steps):
+        one(i)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    h2d = sum(x.numel() * 2 for x in xs)
+    d2h = sum(y.numel() * 4 for y in ys)
+    return {"value": round(work.step_bytes * steps / dt / 1e9, 2), "unit": "GB/s", "steps": steps,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "how": "nq_lowrank_linear_fwd with pinned host x and y per layer (copy in, both kernels, copy out, "
+                   "stream sync), wall clock"}
+
+
+# ------------------------------------------------------------------ the oracle on the host
+
+def run_cpu_baseline(layers, batch, budget_s):
+    import oracle
+
+    o = oracle.default()
+    data = []
+    for li, (name, m, n, r) in enumerate(layers):
+        Upk = synth.random_words(m, r // 32, 5, li, "U")
+        Vpk = synth.random_words(r, n // 32, 5, li, "V")
+        data.append((Upk, Vpk, synth.scales_f16(m, 5, li), synth.scales_f16(n, 6, li),
+                     synth.activations_bf16(batch, n, 5, li), m, n, r))
+    step_bytes = sum(packed_bytes(m, n, r) for _, m, n, r in layers)
+    steps = 0
+    t0 = time.perf_counter()
+    while True:
+        for (Upk, Vpk, s1, s2, x, m, n, r) in data:
+            o.lowrank_linear_fwd(x, Upk, Vpk, s1, s2, m, n, r)
+        steps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(step_bytes * steps / dt / 1e9, 4), "unit": "GB/s", "cores": o.num_threads(),
+            "kind": "oracle",
+            "sample": f"{steps} step(s) of the 7-layer batch-{batch} workload on the fp64 C oracle ({dt:.1f} s)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cpu = run_cpu_baseline(synth.LLAMA2_7B_LAYERS, args.batch, budget_s=args.cpu_seconds)
+    steps_done = int(cpu["sample"].split()[0])
+    value = cpu["value"]
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "impl": "reference",
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"llama2-7b-shaped decode, batch {args.batch}: 7 factorised linears per step",
+                       "batch": args.batch, "steps_sampled": steps_done},
+            "cpu_baseline": cpu, "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                                          "d2h_bytes_per_step": 0},
+            "vs_baseline": None}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", dest="secondary", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

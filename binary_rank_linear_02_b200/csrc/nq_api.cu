@@ -1,0 +1,277 @@
+// nq_api.cu -- the C ABI of libnq (declared in include/nq.h): argument checks, the
+// per-device workspace, host-memory staging and the decode / prefill dispatch.
+#include <mutex>
+#include <string.h>
+
+#include "nq_internal.cuh"
+
+namespace nq {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxDim = int64_t(1) << 20;
+constexpr int64_t kMaxRank = 65536;
+constexpr int kMaxSplits = 64;
+
+std::mutex g_mutex;
+Workspace g_ws[kMaxDevices];
+int g_sm_count[kMaxDevices];
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Memory kind of a pointer: 1 = device-accessible (device or managed), 0 = host.
+// Without a usable device every pointer is a host pointer.
+int pointer_kind(const void* p) {
+    cudaPointerAttributes attr;
+    cudaError_t err = cudaPointerGetAttributes(&attr, p);
+    if (err != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) ? 1 : 0;
+}
+
+}  // namespace
+
+int sm_count() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (g_sm_count[dev] == 0) {
+        int c = 0;
+        cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev);
+        g_sm_count[dev] = c > 0 ? c : 148;
+    }
+    return g_sm_count[dev];
+}
+
+Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, int* status) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        *status = NQ_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    Workspace& w = g_ws[dev];
+    const int64_t pbatch = batch > 8 ? batch : 0;  // prefill buffers only for prefill batches
+    if (w.base && r <= w.r_cap && n <= w.n_cap && m <= w.m_cap && pbatch <= w.batch_cap) {
+        *status = NQ_OK;
+        return &w;
+    }
+    // grow: keep the larger of old and new capacities
+    int64_t r_cap = r > w.r_cap ? r : w.r_cap;
+    int64_t n_cap = n > w.n_cap ? n : w.n_cap;
+    int64_t m_cap = m > w.m_cap ? m : w.m_cap;
+    int64_t b_cap = pbatch > w.batch_cap ? pbatch : w.batch_cap;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(0, &cs);  // legacy stream: errors if a global capture is active
+    if (cudaGetLastError() != cudaSuccess) {
+        *status = NQ_ERR_NOMEM;
+        return nullptr;
+    }
+    if (w.base) cudaDeviceSynchronize();  // old buffers may still be in use
+    size_t off = 0;
+    const size_t o_t = off;        off = align_up(off + sizeof(float) * 8 * r_cap, 256);
+    const size_t o_tgmax = off;    off = align_up(off + sizeof(float) * 8 * (r_cap / 128 + 1), 256);
+    const size_t o_part = off;     off = align_up(off + sizeof(float) * (size_t)kMaxSplits * 8 * r_cap, 256);
+    const size_t o_cnt = off;      off = align_up(off + sizeof(int) * (r_cap / 128 + 1), 256);
+    const size_t o_status = off;   off = align_up(off + sizeof(unsigned) * 64, 256);
+    const size_t o_xp = off;       off = align_up(off + sizeof(uint16_t) * (size_t)b_cap * n_cap, 256);
+    const size_t o_T = off;        off = align_up(off + sizeof(uint16_t) * (size_t)b_cap * r_cap, 256);
+    char* base = nullptr;
+    if (cudaMalloc(&base, off) != cudaSuccess) {
+        cudaGetLastError();
+        *status = NQ_ERR_NOMEM;
+        return nullptr;
+    }
+    if (cudaMemset(base, 0, off) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(base);
+        *status = NQ_ERR_CUDA;
+        return nullptr;
+    }
+    if (w.base) cudaFree(w.base);
+    w.device = dev;
+    w.bytes = off;
+    w.base = base;
+    w.t = reinterpret_cast<float*>(base + o_t);
+    w.tgmax = reinterpret_cast<float*>(base + o_tgmax);
+    w.partials = reinterpret_cast<float*>(base + o_part);
+    w.counters = reinterpret_cast<int*>(base + o_cnt);
+    w.status = reinterpret_cast<unsigned*>(base + o_status);
+    w.xprime = reinterpret_cast<uint16_t*>(base + o_xp);
+    w.T = reinterpret_cast<uint16_t*>(base + o_T);
+    w.r_cap = r_cap;
+    w.n_cap = n_cap;
+    w.m_cap = m_cap;
+    w.batch_cap = b_cap;
+    w.split_cap = kMaxSplits;
+    *status = NQ_OK;
+    return &w;
+}
+
+// Host-memory x / y are staged through device buffers of the workspace.
+static int ensure_staging(Workspace* w, size_t xbytes, size_t ybytes) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (xbytes > w->xstage_bytes) {
+        if (w->xstage) { cudaDeviceSynchronize(); cudaFree(w->xstage); w->xstage = nullptr; w->xstage_bytes = 0; }
+        if (cudaMalloc(&w->xstage, xbytes) != cudaSuccess) { cudaGetLastError(); return NQ_ERR_NOMEM; }
+        w->xstage_bytes = xbytes;
+    }
+    if (ybytes > w->ystage_bytes) {
+        if (w->ystage) { cudaDeviceSynchronize(); cudaFree(w->ystage); w->ystage = nullptr; w->ystage_bytes = 0; }
+        void* p = nullptr;
+        if (cudaMalloc(&p, ybytes) != cudaSuccess) { cudaGetLastError(); return NQ_ERR_NOMEM; }
+        w->ystage = static_cast<float*>(p);
+        w->ystage_bytes = ybytes;
+    }
+    return NQ_OK;
+}
+
+}  // namespace nq
+
+using namespace nq;
+
+extern "C" {
+
+int nq_version(void) { return 100; }
+
+const char* nq_status_string(int status) {
+    switch (status) {
+        case NQ_OK: return "NQ_OK";
+        case NQ_ERR_NULL: return "NQ_ERR_NULL: a required pointer is NULL";
+        case NQ_ERR_SHAPE: return "NQ_ERR_SHAPE: a size is out of range or not a supported multiple";
+        case NQ_ERR_ALIGN: return "NQ_ERR_ALIGN: a pointer is not 16-byte aligned";
+        case NQ_ERR_BATCH: return "NQ_ERR_BATCH: batch is negative";
+        case NQ_ERR_VALUE: return "NQ_ERR_VALUE: an input value is outside its domain";
+        case NQ_ERR_CUDA: return "NQ_ERR_CUDA: a CUDA call or kernel launch failed";
+        case NQ_ERR_TIMEOUT: return "NQ_ERR_TIMEOUT: a bounded device-side wait gave up";
+        case NQ_ERR_NOMEM: return "NQ_ERR_NOMEM: workspace allocation failed (or was needed during stream capture)";
+        case NQ_ERR_PTRKIND: return "NQ_ERR_PTRKIND: pointers of mixed or unsupported memory kinds";
+        default: return "unknown nq status";
+    }
+}
+
+double nq_bits_per_weight(int64_t m, int64_t n, int64_t r) {
+    if (m <= 0 || n <= 0 || r <= 0) return -1.0;
+    // r(m+n) one-bit sign entries + 16(m+n) bits of fp16 scales, over the m*n dense weights
+    return ((double)r * (double)(m + n) + 16.0 * (double)(m + n)) / ((double)m * (double)n);
+}
+
+int nq_pack_signs(const int8_t* signs, int64_t rows, int64_t cols, uint32_t* out, void* stream) {
+    if (rows < 0 || cols < 0) return NQ_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return NQ_OK;
+    if (!signs || !out) return NQ_ERR_NULL;
+    if (rows > (int64_t(1) << 40) / cols) return NQ_ERR_SHAPE;
+    const int ks = pointer_kind(signs), ko = pointer_kind(out);
+    if (ks != ko) return NQ_ERR_PTRKIND;
+    const int64_t wpr = (cols + 31) / 32;
+    if (ks == 0) {
+        for (int64_t i = 0; i < rows * cols; ++i)
+            if (signs[i] < -1 || signs[i] > 1) return NQ_ERR_VALUE;
+        for (int64_t row = 0; row < rows; ++row) {
+            const int8_t* src = signs + row * cols;
+            for (int64_t w = 0; w < wpr; ++w) {
+                uint32_t word = 0;
+                const int64_t c0 = 32 * w;
+                const int nb = (int)((cols - c0) < 32 ? (cols - c0) : 32);
+                for (int b = 0; b < nb; ++b) word |= (src[c0 + b] >= 0 ? 1u : 0u) << b;
+                out[row * wpr + w] = word;
+            }
+        }
+        return NQ_OK;
+    }
+    int st = NQ_OK;
+    Workspace* ws = workspace_for(128, 128, 128, 0, &st);
+    if (!ws) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws->status, 0, sizeof(unsigned), s) != cudaSuccess) return NQ_ERR_CUDA;
+    st = pack_device(signs, rows, cols, out, ws->status, s);
+    if (st != NQ_OK) return st;
+    unsigned flag = 0;
+    if (cudaMemcpyAsync(&flag, ws->status, sizeof(unsigned), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return NQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NQ_ERR_CUDA;
+    return flag ? NQ_ERR_VALUE : NQ_OK;
+}
+
+int nq_unpack_signs(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* out, void* stream) {
+    if (rows < 0 || cols < 0) return NQ_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return NQ_OK;
+    if (!packed || !out) return NQ_ERR_NULL;
+    if (rows > (int64_t(1) << 40) / cols) return NQ_ERR_SHAPE;
+    const int kp = pointer_kind(packed), ko = pointer_kind(out);
+    if (kp != ko) return NQ_ERR_PTRKIND;
+    const int64_t wpr = (cols + 31) / 32;
+    if (kp == 0) {
+        for (int64_t row = 0; row < rows; ++row)
+            for (int64_t c = 0; c < cols; ++c)
+                out[row * cols + c] = ((packed[row * wpr + c / 32] >> (c % 32)) & 1u) ? 1 : -1;
+        return NQ_OK;
+    }
+    return unpack_device(packed, rows, cols, out, static_cast<cudaStream_t>(stream));
+}
+
+int nq_workspace_reserve(int64_t m, int64_t n, int64_t r, int64_t batch) {
+    if (m <= 0 || n <= 0 || r <= 0 || m % 128 || n % 128 || r % 128 || m > kMaxDim || n > kMaxDim ||
+        r > kMaxRank)
+        return NQ_ERR_SHAPE;
+    if (batch < 0) return NQ_ERR_BATCH;
+    int st = NQ_OK;
+    Workspace* ws = workspace_for(m, n, r, batch, &st);
+    return ws ? NQ_OK : st;
+}
+
+int nq_lowrank_linear_fwd(const void* x, const uint32_t* Upk, const uint32_t* Vpk, const void* s1,
+                          const void* s2, int64_t m, int64_t n, int64_t r, int64_t batch, float* y,
+                          void* stream) {
+    if (batch < 0) return NQ_ERR_BATCH;
+    if (m <= 0 || n <= 0 || r <= 0 || m % 128 || n % 128 || r % 128 || m > kMaxDim || n > kMaxDim ||
+        r > kMaxRank)
+        return NQ_ERR_SHAPE;
+    if (batch > (int64_t(1) << 40) / (m > n ? m : n)) return NQ_ERR_SHAPE;
+    if (batch == 0) return NQ_OK;
+    if (!x || !Upk || !Vpk || !s1 || !s2 || !y) return NQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(Upk) || !aligned16(Vpk) || !aligned16(s1) || !aligned16(s2) ||
+        !aligned16(y))
+        return NQ_ERR_ALIGN;
+    if (!pointer_kind(Upk) || !pointer_kind(Vpk) || !pointer_kind(s1) || !pointer_kind(s2))
+        return NQ_ERR_PTRKIND;
+    const bool x_host = pointer_kind(x) == 0, y_host = pointer_kind(y) == 0;
+
+    int st = NQ_OK;
+    Workspace* ws = workspace_for(m, n, r, batch, &st);
+    if (!ws) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t xbytes = sizeof(uint16_t) * (size_t)batch * n, ybytes = sizeof(float) * (size_t)batch * m;
+    if (x_host || y_host) {
+        st = ensure_staging(ws, x_host ? xbytes : 0, y_host ? ybytes : 0);
+        if (st != NQ_OK) return st;
+    }
+    const uint16_t* xd = static_cast<const uint16_t*>(x);
+    float* yd = y;
+    if (x_host) {
+        if (cudaMemcpyAsync(ws->xstage, x, xbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return NQ_ERR_CUDA;
+        xd = static_cast<const uint16_t*>(ws->xstage);
+    }
+    if (y_host) yd = ws->ystage;
+
+    const uint16_t* s1h = static_cast<const uint16_t*>(s1);
+    const uint16_t* s2h = static_cast<const uint16_t*>(s2);
+    if (batch <= NQ_DECODE_MAX_BATCH)
+        st = decode_forward(xd, Upk, Vpk, s1h, s2h, m, n, r, batch, yd, ws, s);
+    else
+        st = prefill_forward(xd, Upk, Vpk, s1h, s2h, m, n, r, batch, yd, ws, s);
+    if (st != NQ_OK) return st;
+
+    if (y_host) {
+        if (cudaMemcpyAsync(y, ws->ystage, ybytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return NQ_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return NQ_ERR_CUDA;
+    }
+    return NQ_OK;
+}
+
+}  // extern "C"

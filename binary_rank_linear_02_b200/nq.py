@@ -1,0 +1,182 @@
+"""ctypes binding of libnq (include/nq.h): argument marshalling only.
+
+Every step of the factorised linear runs in the CUDA library; this module turns torch
+tensors / numpy arrays into the plain pointers, sizes and stream handle of the C ABI and
+raises ``NQError`` on a non-zero status.  There is no fallback: if ``libnq.so`` is
+missing or cannot be loaded, importing this module raises.
+
+Same names as the C entry points: ``nq_pack_signs``, ``nq_unpack_signs``,
+``nq_lowrank_linear_fwd``, ``nq_bits_per_weight``, ``nq_status_string``,
+``nq_workspace_reserve``; plus tensor-level conveniences ``pack_signs``,
+``unpack_signs`` and ``lowrank_linear_fwd``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnq.so")
+
+NQ_OK = 0
+NQ_ERR_NULL = -1
+NQ_ERR_SHAPE = -2
+NQ_ERR_ALIGN = -3
+NQ_ERR_BATCH = -4
+NQ_ERR_VALUE = -5
+NQ_ERR_CUDA = -6
+NQ_ERR_TIMEOUT = -7
+NQ_ERR_NOMEM = -8
+NQ_ERR_PTRKIND = -9
+NQ_DECODE_MAX_BATCH = 8
+
+
+class NQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {nq_status_string(status)} ({status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m binary_rank_linear_02_b200.build` "
+            "(this package has no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    p, i64 = ctypes.c_void_p, ctypes.c_int64
+    L.nq_pack_signs.argtypes = [p, i64, i64, p, p]
+    L.nq_pack_signs.restype = ctypes.c_int
+    L.nq_unpack_signs.argtypes = [p, i64, i64, p, p]
+    L.nq_unpack_signs.restype = ctypes.c_int
+    L.nq_lowrank_linear_fwd.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p]
+    L.nq_lowrank_linear_fwd.restype = ctypes.c_int
+    L.nq_bits_per_weight.argtypes = [i64, i64, i64]
+    L.nq_bits_per_weight.restype = ctypes.c_double
+    L.nq_status_string.argtypes = [ctypes.c_int]
+    L.nq_status_string.restype = ctypes.c_char_p
+    L.nq_workspace_reserve.argtypes = [i64, i64, i64, i64]
+    L.nq_workspace_reserve.restype = ctypes.c_int
+    L.nq_version.restype = ctypes.c_int
+    return L
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+# ------------------------------------------------------------------ raw C names
+
+def nq_pack_signs(signs_ptr: int, rows: int, cols: int, out_ptr: int, stream: int = 0) -> int:
+    return _lib.nq_pack_signs(signs_ptr, rows, cols, out_ptr, stream)
+
+
+def nq_unpack_signs(packed_ptr: int, rows: int, cols: int, out_ptr: int, stream: int = 0) -> int:
+    return _lib.nq_unpack_signs(packed_ptr, rows, cols, out_ptr, stream)
+
+
+def nq_lowrank_linear_fwd(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n, r, batch, y_ptr, stream=0) -> int:
+    return _lib.nq_lowrank_linear_fwd(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n, r, batch, y_ptr, stream)
+
+
+def nq_bits_per_weight(m: int, n: int, r: int) -> float:
+    return _lib.nq_bits_per_weight(m, n, r)
+
+
+def nq_status_string(status: int) -> str:
+    return _lib.nq_status_string(status).decode()
+
+
+def nq_workspace_reserve(m: int, n: int, r: int, batch: int) -> int:
+    return _lib.nq_workspace_reserve(m, n, r, batch)
+
+
+def nq_version() -> int:
+    return _lib.nq_version()
+
+
+# ------------------------------------------------------------------ tensor conveniences
+
+def _ptr(a) -> int:
+    if a is None:
+        return 0
+    if isinstance(a, np.ndarray):
+        assert a.flags["C_CONTIGUOUS"], "array must be C-contiguous"
+        return a.ctypes.data
+    assert a.is_contiguous(), "tensor must be contiguous"
+    return a.data_ptr()
+
+
+def _stream(stream, *tensors) -> int:
+    if stream is not None:
+        return int(stream)
+    import torch
+
+    for t in tensors:
+        if isinstance(t, torch.Tensor) and t.is_cuda:
+            return torch.cuda.current_stream(t.device).cuda_stream
+    return 0
+
+
+def _check(status: int, where: str) -> None:
+    if status != NQ_OK:
+        raise NQError(status, where)
+
+
+def pack_signs(signs, out=None, stream=None):
+    """rows x cols int8 signs (torch tensor or numpy array) -> rows x ceil(cols/32) words."""
+    rows, cols = signs.shape
+    wpr = (cols + 31) // 32
+    if out is None:
+        if isinstance(signs, np.ndarray):
+            out = np.empty((rows, wpr), dtype=np.uint32)
+        else:
+            import torch
+
+            out = torch.empty((rows, wpr), dtype=torch.int32, device=signs.device)
+    _check(_lib.nq_pack_signs(_ptr(signs), rows, cols, _ptr(out), _stream(stream, signs)), "nq_pack_signs")
+    return out
+
+
+def unpack_signs(packed, cols: int, out=None, stream=None):
+    rows = packed.shape[0]
+    if out is None:
+        if isinstance(packed, np.ndarray):
+            out = np.empty((rows, cols), dtype=np.int8)
+        else:
+            import torch
+
+            out = torch.empty((rows, cols), dtype=torch.int8, device=packed.device)
+    _check(_lib.nq_unpack_signs(_ptr(packed), rows, cols, _ptr(out), _stream(stream, packed)), "nq_unpack_signs")
+    return out
+
+
+def lowrank_linear_fwd(x, Upk, Vpk, s1, s2, m: int, n: int, r: int, y=None, stream=None):
+    """y (batch x m, float32) = s1 * (U (V^T (s2 * x))).
+
+    x: batch x n bfloat16 (device or host); Upk: m x r/32 and Vpk: r x n/32 packed words
+    (device); s1: m and s2: n fp16 (device).  y defaults to a new float32 tensor on x's
+    device.
+    """
+    batch = x.shape[0] if x.dim() == 2 else 1
+    if y is None:
+        import torch
+
+        y = torch.empty((batch, m), dtype=torch.float32, device=x.device,
+                        pin_memory=(not x.is_cuda and torch.cuda.is_available()))
+    st = _lib.nq_lowrank_linear_fwd(_ptr(x), _ptr(Upk), _ptr(Vpk), _ptr(s1), _ptr(s2), m, n, r, batch,
+                                    _ptr(y), _stream(stream, x, Upk, y))
+    _check(st, "nq_lowrank_linear_fwd")
+    return y
+
+
+def bits_per_weight(m: int, n: int, r: int) -> float:
+    return _lib.nq_bits_per_weight(m, n, r)
+
+
+def workspace_reserve(m: int, n: int, r: int, batch: int) -> None:
+    _check(_lib.nq_workspace_reserve(m, n, r, batch), "nq_workspace_reserve")

@@ -1,0 +1,132 @@
+/*
+ * nq.h -- C ABI of libnq: the forward pass of a linear layer whose weight is stored as a
+ * low-rank binary factorisation,
+ *
+ *     W ~= diag(s1) . U . V^T . diag(s2),   U in {+1,-1}^{m x r},  V in {+1,-1}^{n x r},
+ *     y  = s1 (.) ( U . ( V^T . ( s2 (.) x ) ) ),
+ *
+ * with U and V stored one bit per entry and s1 (m), s2 (n) fp16 scale vectors.
+ * The method is NanoQuant's (hardwired.dev, "NanoQuant jednoduse: 70B model na herni
+ * grafice", section "Jak NanoQuant funguje": the weight matrix as a product of +1/-1
+ * matrices and diagonal scaling vectors, r*(m+n) binary values plus the scales;
+ * rapidrecap.app, "Nanoquant: Efficient Sub-1-Bit Quantization of Large Language
+ * Models", section "Quantization Technique": binary U and V plus scaling factors,
+ * evaluated by custom CUDA kernels; hardwired.dev section "Cisla": binary GEMV/GEMM
+ * kernels).  The pages publish no kernel and no interface; this ABI is this library's.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Plain pointers and sizes; no ownership transfer: every buffer is owned by the caller.
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy default stream.
+ *  - Return value: an nq_status (0 = NQ_OK, negative = error).  Argument errors are
+ *    detected on the host before anything is enqueued; in that case nothing is launched
+ *    and no output is written.
+ *  - Stored form of a sign matrix ("packed"): row-major rows of ceil(cols/32) uint32
+ *    words; bit b of word w of a row is the entry in column 32*w + b; bit 1 = +1,
+ *    bit 0 = -1; unused high bits of a partial last word are 0.
+ *      Upk: U as m rows of r/32 words         (row i = U[i][0..r))
+ *      Vpk: V^T as r rows of n/32 words       (row k = V[0..n)[k])
+ *  - x, s1, s2 hold IEEE bit patterns: x bfloat16, s1 and s2 binary16 (fp16).
+ *  - The library keeps one workspace per device (intermediate t = V^T (s2 (.) x) and
+ *    a few counters).  It is allocated on the first call on a device and grown when a
+ *    larger shape arrives; call nq_workspace_reserve() beforehand to keep allocation out
+ *    of a CUDA-graph capture.  Calls that use the same device's workspace must not run
+ *    concurrently on different streams.
+ */
+#ifndef NQ_H_
+#define NQ_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NQ_OK = 0,
+    NQ_ERR_NULL = -1,      /* a required pointer is NULL */
+    NQ_ERR_SHAPE = -2,     /* a size is out of range or not a supported multiple */
+    NQ_ERR_ALIGN = -3,     /* a pointer is not 16-byte aligned */
+    NQ_ERR_BATCH = -4,     /* batch < 0 */
+    NQ_ERR_VALUE = -5,     /* an input value is outside its domain (e.g. a sign of 2) */
+    NQ_ERR_CUDA = -6,      /* a CUDA runtime/driver call or a launch failed */
+    NQ_ERR_TIMEOUT = -7,   /* a bounded device-side wait gave up */
+    NQ_ERR_NOMEM = -8,     /* workspace allocation failed */
+    NQ_ERR_PTRKIND = -9    /* pointers of mixed or unsupported memory kinds */
+} nq_status;
+
+/* Largest decode batch: calls with 1 <= batch <= NQ_DECODE_MAX_BATCH run the two-stage
+ * binary GEMV; larger batches run the tensor-core path. */
+#define NQ_DECODE_MAX_BATCH 8
+
+/*
+ * nq_pack_signs -- store a sign matrix one bit per entry (the sign projection of the
+ * ADMM step, hardwired.dev section "Krok 2", followed by the one-bit storage of section
+ * "Jak NanoQuant funguje").
+ *   signs : rows x cols int8, row-major; each entry -1, 0 or +1 (0 is stored as +1).
+ *   out   : rows x ceil(cols/32) uint32 (layout above).
+ *   rows, cols >= 0; rows*cols == 0 is a no-op returning NQ_OK.
+ * Both pointers on the device: a kernel runs on `stream`, then the call synchronises
+ * `stream` to read back the value check (packing is an offline step).  Both pointers in
+ * host memory: packed on the calling thread, `stream` unused.  Mixed: NQ_ERR_PTRKIND.
+ * An entry outside {-1, 0, +1} returns NQ_ERR_VALUE; `out` is then unspecified.
+ */
+int nq_pack_signs(const int8_t* signs, int64_t rows, int64_t cols, uint32_t* out, void* stream);
+
+/*
+ * nq_unpack_signs -- inverse of nq_pack_signs: rows x cols int8 in {-1, +1}.
+ * Same pointer-kind rules; the device path does not synchronise.
+ */
+int nq_unpack_signs(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* out, void* stream);
+
+/*
+ * nq_lowrank_linear_fwd -- y = s1 (.) (U (V^T (s2 (.) x))) for `batch` tokens.
+ *   x    : batch x n bfloat16, row-major (one token per row)
+ *   Upk  : m x (r/32) uint32, device memory
+ *   Vpk  : r x (n/32) uint32, device memory
+ *   s1   : m fp16, device memory;  s2 : n fp16, device memory
+ *   y    : batch x m float32, row-major (written)
+ *   m, n, r : positive multiples of 128, each at most 1<<20
+ *   batch   : >= 0; 0 is a no-op returning NQ_OK
+ * x and y may be device memory, or host memory (pageable or pinned): host x is copied
+ * to the device on `stream` first, host y is copied back and the call then synchronises
+ * `stream` before returning.  Device buffers are used asynchronously on `stream`.
+ * Every pointer must be 16-byte aligned.
+ * Path: batch <= NQ_DECODE_MAX_BATCH runs the decode path (two binary GEMV stages on the
+ * CUDA cores and integer tensor-core instructions, t kept in the workspace); larger
+ * batches run the prefill path (two tcgen05 tensor-core GEMMs with the +1/-1 operands
+ * expanded on chip, fp16 operands, fp32 accumulation).
+ * Accuracy: max|y - y_exact| / max|y_exact| <= 2e-3 for the documented input ranges
+ * (|s2_j x_j| and |t_k| below 6.0e4).
+ * Weights (Upk, Vpk, s1, s2) may be read before the work enqueued earlier on `stream`
+ * has finished (programmatic dependent launch), so they must not be produced by the
+ * kernel enqueued immediately before this call on the same stream; x may be.
+ */
+int nq_lowrank_linear_fwd(const void* x, const uint32_t* Upk, const uint32_t* Vpk,
+                          const void* s1, const void* s2, int64_t m, int64_t n, int64_t r,
+                          int64_t batch, float* y, void* stream);
+
+/*
+ * nq_bits_per_weight -- storage cost of the factorised layer in bits per weight of the
+ * dense m x n matrix it replaces: (r*(m+n) + 16*(m+n)) / (m*n)  (hardwired.dev sections
+ * "Jak NanoQuant funguje" and "Co znamena sub-1-bit").  -1.0 if any argument is <= 0.
+ */
+double nq_bits_per_weight(int64_t m, int64_t n, int64_t r);
+
+/* A static, human-readable name for a status code. */
+const char* nq_status_string(int status);
+
+/*
+ * nq_workspace_reserve -- allocate (or grow) the current device's workspace so that
+ * later calls with these or smaller sizes allocate nothing.  Synchronises the device.
+ */
+int nq_workspace_reserve(int64_t m, int64_t n, int64_t r, int64_t batch);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int nq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NQ_H_ */

@@ -1,0 +1,103 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/nq.h declares, rejects bad arguments on the host before touching a device, and
+its host-memory pack / unpack path and storage accounting agree with the oracle and
+the golden values."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import pins
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def nq():
+    from binary_rank_linear_02_b200 import build
+
+    build.build()
+    from binary_rank_linear_02_b200 import nq as mod
+
+    return mod
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "nq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nq_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(nq):
+    names = declared_functions()
+    assert {"nq_pack_signs", "nq_unpack_signs", "nq_lowrank_linear_fwd", "nq_bits_per_weight"} <= set(names)
+    lib = ctypes.CDLL(nq.LIB_PATH)
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(nq):
+    for code in range(0, -10, -1):
+        s = nq.nq_status_string(code)
+        assert s.startswith("NQ_")
+    assert "unknown" in nq.nq_status_string(-99)
+
+
+def test_bits_per_weight_golden(nq):
+    for (m, n, r, num, den) in pins.load_bits_per_weight():
+        assert nq.bits_per_weight(m, n, r) == num / den
+    assert nq.bits_per_weight(0, 1, 1) == -1.0
+    assert nq.bits_per_weight(1, 1, -3) == -1.0
+
+
+def test_host_pack_matches_oracle_and_golden(nq, orc):
+    for name, signs, expected in pins.load_pack_patterns():
+        got = nq.pack_signs(signs)
+        assert np.array_equal(got, expected), name
+    from binary_rank_linear_02_b200 import synth
+
+    for rows, cols, seed in ((7, 64, 5), (3, 100, 6), (1, 1, 7), (4, 31, 8)):
+        s = synth.signs(rows, cols, seed)
+        s[0, 0] = 0
+        got = nq.pack_signs(s)
+        assert np.array_equal(got, orc.pack_signs(s))
+        back = nq.unpack_signs(got, cols)
+        assert np.array_equal(back, np.where(s >= 0, 1, -1).astype(np.int8))
+
+
+def test_host_pack_rejects_bad_values(nq):
+    bad = np.array([[1, -1, 3, 0]], dtype=np.int8)
+    out = np.zeros((1, 1), dtype=np.uint32)
+    assert nq.nq_pack_signs(bad.ctypes.data, 1, 4, out.ctypes.data, 0) == nq.NQ_ERR_VALUE
+
+
+def test_pack_argument_errors(nq):
+    out = np.zeros((1, 1), dtype=np.uint32)
+    s = np.ones((1, 4), dtype=np.int8)
+    assert nq.nq_pack_signs(0, 1, 4, out.ctypes.data, 0) == nq.NQ_ERR_NULL
+    assert nq.nq_pack_signs(s.ctypes.data, -1, 4, out.ctypes.data, 0) == nq.NQ_ERR_SHAPE
+    assert nq.nq_pack_signs(s.ctypes.data, 0, 4, out.ctypes.data, 0) == nq.NQ_OK
+    assert nq.nq_unpack_signs(0, 1, 4, s.ctypes.data, 0) == nq.NQ_ERR_NULL
+
+
+def test_forward_argument_errors(nq):
+    buf = np.zeros(1 << 16, dtype=np.uint8)
+    base = (buf.ctypes.data + 255) // 256 * 256
+    p = [base + 1024 * i for i in range(6)]
+    f = nq.nq_lowrank_linear_fwd
+    assert f(p[0], p[1], p[2], p[3], p[4], 128, 128, 128, -1, p[5], 0) == nq.NQ_ERR_BATCH
+    assert f(p[0], p[1], p[2], p[3], p[4], 100, 128, 128, 1, p[5], 0) == nq.NQ_ERR_SHAPE
+    assert f(p[0], p[1], p[2], p[3], p[4], 128, 0, 128, 1, p[5], 0) == nq.NQ_ERR_SHAPE
+    assert f(p[0], p[1], p[2], p[3], p[4], 128, 128, 64, 1, p[5], 0) == nq.NQ_ERR_SHAPE
+    assert f(p[0], p[1], p[2], p[3], p[4], 128, 128, 1 << 17, 1, p[5], 0) == nq.NQ_ERR_SHAPE
+    assert f(p[0], p[1], p[2], p[3], p[4], 128, 128, 128, 0, p[5], 0) == nq.NQ_OK
+    assert f(0, p[1], p[2], p[3], p[4], 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_NULL
+    assert f(p[0], p[1], p[2], p[3], p[4], 128, 128, 128, 1, 0, 0) == nq.NQ_ERR_NULL
+    assert f(p[0] + 2, p[1], p[2], p[3], p[4], 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_ALIGN
+    assert f(p[0], p[1], p[2] + 8, p[3], p[4], 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_ALIGN
+    # weights in host memory are refused (they must live on the device)
+    assert f(p[0], p[1], p[2], p[3], p[4], 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_PTRKIND
+    assert nq.nq_workspace_reserve(128, 100, 128, 1) == nq.NQ_ERR_SHAPE
+    assert nq.nq_workspace_reserve(128, 128, 128, -2) == nq.NQ_ERR_BATCH

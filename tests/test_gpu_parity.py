@@ -1,0 +1,197 @@
+"""CUDA path against the CPU oracle, through the C ABI, on seeded synthetic inputs.
+
+Bar: packing bit-exact; the forward within max|y - y_ref| / max|y_ref| <= 2e-3 (the
+tolerance the factorised-linear benchmarks state for bf16 inputs with fp32
+accumulation).  Small cases are compared element by element; at full benchmark sizes
+the oracle computes every output of the decode configurations, and a sample of token
+rows of the large prefill batches.
+"""
+import numpy as np
+import pytest
+
+from binary_rank_linear_02_b200 import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def nq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from binary_rank_linear_02_b200 import nq as mod
+
+    return mod
+
+
+def rel_err(y, y_ref):
+    y = np.asarray(y, dtype=np.float64)
+    return float(np.max(np.abs(y - y_ref)) / np.max(np.abs(y_ref)))
+
+
+class Case:
+    """One factorised layer: signs, scales and activations from the seeded generators,
+    stored once by the oracle and once by the CUDA packer."""
+
+    def __init__(self, orc, nq, m, n, r, batch, seed, U=None, V=None, x=None):
+        self.m, self.n, self.r, self.batch = m, n, r, batch
+        self.U = synth.signs(m, r, seed, "U") if U is None else U
+        self.V = synth.signs(n, r, seed, "V") if V is None else V
+        self.s1 = synth.scales_f16(m, seed, "s1")
+        self.s2 = synth.scales_f16(n, seed, "s2")
+        self.x = synth.activations_bf16(batch, n, seed) if x is None else x
+        self.Upk_o = orc.pack_signs(self.U)
+        self.Vpk_o = orc.pack_signs(np.ascontiguousarray(self.V.T))
+        dev = torch.device("cuda")
+        self.Upk = nq.pack_signs(torch.from_numpy(self.U).to(dev))
+        self.Vpk = nq.pack_signs(torch.from_numpy(np.ascontiguousarray(self.V.T)).to(dev))
+        self.s1_d = torch.from_numpy(self.s1.view(np.int16)).to(dev)
+        self.s2_d = torch.from_numpy(self.s2.view(np.int16)).to(dev)
+        self.x_d = torch.from_numpy(self.x.view(np.int16)).to(dev)
+
+    def gpu(self, x_d=None):
+        x_d = self.x_d if x_d is None else x_d
+        y = nq_mod().lowrank_linear_fwd(x_d, self.Upk, self.Vpk, self.s1_d, self.s2_d, self.m, self.n, self.r)
+        torch.cuda.synchronize()
+        return y.cpu().numpy()
+
+    def oracle(self, orc, rows=None):
+        x = self.x if rows is None else self.x[rows]
+        return orc.lowrank_linear_fwd(x, self.Upk_o, self.Vpk_o, self.s1, self.s2, self.m, self.n, self.r)
+
+
+def nq_mod():
+    from binary_rank_linear_02_b200 import nq as mod
+
+    return mod
+
+
+# ------------------------------------------------------------------ packing
+
+@pytest.mark.parametrize("rows,cols", [(1, 32), (7, 100), (128, 4096), (3, 33), (64, 1)])
+def test_pack_device_bit_exact(nq, orc, rows, cols):
+    s = synth.signs(rows, cols, 3, rows, cols)
+    s[0, 0] = 0
+    got = nq.pack_signs(torch.from_numpy(s).cuda()).cpu().numpy().view(np.uint32)
+    assert np.array_equal(got, orc.pack_signs(s))
+    back = nq.unpack_signs(torch.from_numpy(got.view(np.int32)).cuda(), cols).cpu().numpy()
+    assert np.array_equal(back, np.where(s >= 0, 1, -1))
+
+
+def test_pack_device_golden_patterns(nq):
+    import pins
+
+    for name, signs, expected in pins.load_pack_patterns():
+        got = nq.pack_signs(torch.from_numpy(signs).cuda()).cpu().numpy().view(np.uint32)
+        assert np.array_equal(got, expected), name
+
+
+def test_pack_device_rejects_bad_values(nq):
+    s = torch.ones((4, 64), dtype=torch.int8, device="cuda")
+    s[2, 17] = 5
+    out = torch.empty((4, 2), dtype=torch.int32, device="cuda")
+    st = nq.nq_pack_signs(s.data_ptr(), 4, 64, out.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert st == nq.NQ_ERR_VALUE
+
+
+# ------------------------------------------------------------------ forward, small and ragged
+
+SMALL = [
+    (512, 512, 128, 1),     # the single-layer workload
+    (512, 512, 128, 2),
+    (512, 512, 128, 4),
+    (512, 512, 128, 5),
+    (512, 512, 128, 8),
+    (384, 640, 256, 3),
+    (128, 128, 128, 1),     # one tile everywhere
+    (256, 2176, 2176, 2),   # 17 column blocks: a full chunk plus a ragged one, both stages
+    (1152, 384, 1664, 7),
+    (512, 512, 128, 9),     # first prefill batches
+    (512, 512, 128, 16),
+    (640, 384, 256, 33),
+]
+
+
+@pytest.mark.parametrize("m,n,r,batch", SMALL)
+def test_forward_small(nq, orc, m, n, r, batch):
+    c = Case(orc, nq, m, n, r, batch, seed=1000 + m + n + r + batch)
+    y = c.gpu()
+    y_ref = c.oracle(orc)
+    assert y.shape == (batch, m)
+    assert rel_err(y, y_ref) <= TOL
+
+
+def test_forward_deterministic(nq, orc):
+    c = Case(orc, nq, 1024, 4096, 1664, 3, seed=7)
+    a, b = c.gpu(), c.gpu()
+    assert np.array_equal(a, b)
+
+
+def test_forward_special_signs(nq, orc):
+    m, n, r = 256, 512, 128
+    ones_u = np.ones((m, r), np.int8)
+    ones_v = np.ones((n, r), np.int8)
+    for U, V in ((ones_u, ones_v), (-ones_u, ones_v), (ones_u, -ones_v)):
+        c = Case(orc, nq, m, n, r, 2, seed=11, U=U, V=V)
+        assert rel_err(c.gpu(), c.oracle(orc)) <= TOL
+
+
+def test_forward_column_negation(nq, orc):
+    m, n, r = 512, 1024, 256
+    base = Case(orc, nq, m, n, r, 2, seed=21)
+    U2, V2 = base.U.copy(), base.V.copy()
+    U2[:, 5] *= -1
+    V2[:, 5] *= -1
+    U2[:, 200] *= -1
+    V2[:, 200] *= -1
+    neg = Case(orc, nq, m, n, r, 2, seed=21, U=U2, V=V2)
+    assert np.array_equal(neg.oracle(orc), base.oracle(orc))
+    y_ref = base.oracle(orc)
+    assert rel_err(base.gpu(), y_ref) <= TOL
+    assert rel_err(neg.gpu(), y_ref) <= TOL
+
+
+def test_forward_zero_input(nq, orc):
+    c = Case(orc, nq, 256, 256, 128, 2, seed=5, x=np.zeros((2, 256), np.uint16))
+    assert np.all(c.gpu() == 0.0)
+
+
+def test_forward_host_buffers(nq, orc):
+    c = Case(orc, nq, 512, 512, 128, 3, seed=9)
+    x_host = torch.from_numpy(c.x.view(np.int16)).pin_memory()
+    y_dev = c.gpu()
+    y_host = nq.lowrank_linear_fwd(x_host, c.Upk, c.Vpk, c.s1_d, c.s2_d, c.m, c.n, c.r)
+    assert not y_host.is_cuda
+    assert np.array_equal(y_host.numpy(), y_dev)
+    x_pageable = torch.from_numpy(c.x.view(np.int16).copy())
+    y_out = torch.empty((3, 512), dtype=torch.float32)
+    nq.lowrank_linear_fwd(x_pageable, c.Upk, c.Vpk, c.s1_d, c.s2_d, c.m, c.n, c.r, y=y_out)
+    assert np.array_equal(y_out.numpy(), y_dev)
+
+
+# ------------------------------------------------------------------ full benchmark shapes
+
+@pytest.mark.parametrize("name,m,n,r", synth.LLAMA2_7B_LAYERS[3:])
+@pytest.mark.parametrize("batch", [1, 8])
+def test_forward_llama2_7b_shapes(nq, orc, name, m, n, r, batch):
+    c = Case(orc, nq, m, n, r, batch, seed=sum(map(ord, name)))
+    assert rel_err(c.gpu(), c.oracle(orc)) <= TOL
+
+
+@pytest.mark.parametrize("name,m,n,r", [synth.LLAMA2_70B_LAYERS[i] for i in (0, 1, 4, 6)])
+@pytest.mark.parametrize("batch", [1, 4])
+def test_forward_llama2_70b_shapes(nq, orc, name, m, n, r, batch):
+    c = Case(orc, nq, m, n, r, batch, seed=70 + len(name))
+    assert rel_err(c.gpu(), c.oracle(orc)) <= TOL
+
+
+@pytest.mark.parametrize("batch", list(synth.PREFILL_BATCHES))
+def test_forward_prefill_sweep_sampled(nq, orc, batch):
+    _, m, n, r = synth.PREFILL_SHAPE
+    c = Case(orc, nq, m, n, r, batch, seed=400 + batch)
+    y = c.gpu()
+    rng = np.random.default_rng(batch)
+    rows = np.unique(np.concatenate([[0, batch - 1], rng.choice(batch, size=min(batch, 14), replace=False)]))
+    assert rel_err(y[rows], c.oracle(orc, rows)) <= TOL
