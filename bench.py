@@ -18,6 +18,7 @@ Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instea
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -76,6 +77,14 @@ class ClockSampler:
                  "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        # wait (up to 3 s) for the first sample, so the timed region is covered
+        t0 = time.time()
+        while time.time() - t0 < 3.0:
+            self.fh.flush()
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
 
     def stop(self):
         if self.proc is None:
@@ -142,9 +151,21 @@ class DecodeWorkload:
         self.y = [torch.empty((batch, m), dtype=torch.float32, device=device) for (_, m, n, r) in layers]
         for (_, m, n, r) in layers:
             nq.workspace_reserve(m, n, r, batch)
+        # one grouped descriptor array per weight copy (kept alive for graph replays)
+        self.descs = [nq.make_descs([(self.x[li], *per[li][:2], *per[li][2:], self.y[li], m, n, r)
+                                     for li, (_, m, n, r) in enumerate(layers)]) for per in self.sets]
+        self.grouped = True
 
     def step(self, i, stream_handle, layer_filter=None):
+        """One pass over the layers: one grouped call, or one call per layer."""
         per = self.sets[i % self.copies]
+        if self.grouped and layer_filter is None:
+            arr = self.descs[i % self.copies]
+            st = self.nq.lib().nq_lowrank_linear_fwd_grouped(ctypes.addressof(arr), len(self.layers), self.batch,
+                                                               stream_handle)
+            if st != 0:
+                raise RuntimeError(f"nq_lowrank_linear_fwd_grouped: {self.nq.nq_status_string(st)}")
+            return
         fwd = self.nq.lib().nq_lowrank_linear_fwd
         for li, (name, m, n, r) in enumerate(self.layers):
             if layer_filter is not None and li != layer_filter:
@@ -261,8 +282,13 @@ def run_ours(args):
     # end to end through the public API with host buffers (pinned), synchronous per call
     e2e = run_e2e(work, stream, min(args.steps, 100), device)
 
-    # secondary: batch 8 decode on the same shapes
+    # secondary: the same step as seven separate nq_lowrank_linear_fwd calls; batch 8
     secondary = {}
+    if args.secondary and world == 1:
+        work.grouped = False
+        ms1 = timed_graphs(work, args.steps, args.warmup, stream)
+        work.grouped = True
+        secondary["decode_b%d_per_layer_calls_gbs" % batch] = round(work.step_bytes * args.steps / (ms1 * 1e-3) / 1e9, 1)
     if args.secondary and batch == 1 and world == 1:
         w8 = DecodeWorkload(layers, 8, seed=99, device=device)
         with torch.cuda.stream(stream):
@@ -273,11 +299,14 @@ def run_ours(args):
         secondary["decode_b8_tokens_per_s"] = round(8 * args.steps / (ms8 * 1e-3), 1)
         del w8
 
+    if args.secondary and world == 1:
+        secondary["prefill_11008x4096_r2432"] = run_prefill_sweep(device, stream, args.warmup, peaks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = run_cpu_baseline(layers, batch, budget_s=args.cpu_seconds)
 
-    launches = args.steps * len(layers) * 2
+    launches = args.steps * 2  # stage-1 and stage-2 kernels of one grouped call per step
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -285,7 +314,8 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in; int8x2-limb tensor-core products, int32/fp32 acc",
             "data": "synthetic",
             "config": {"workload": f"llama2-7b-shaped decode, batch {batch}: 7 factorised linears per step "
-                                   "(q/k/v/o 4096x4096 r1664, gate/up 11008x4096 r2432, down 4096x11008 r2432)",
+                                   "(q/k/v/o 4096x4096 r1664, gate/up 11008x4096 r2432, down 4096x11008 r2432), "
+                                   "one nq_lowrank_linear_fwd_grouped call per step",
                        "batch": batch, "packed_bytes_per_step": work.step_bytes,
                        "l2": f"weights rotate over {work.copies} seeded copies "
                              f"({work.copies * work.step_bytes / 1e6:.0f} MB > 2x L2)",
@@ -299,6 +329,58 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_prefill_sweep(device, stream, warmup, peaks, calls=20):
+    """Config-4 sweep: the 11008x4096 r=2432 layer at token batches 16..4096 (tcgen05 path)."""
+    import torch
+
+    from binary_rank_linear_02_b200 import nq
+
+    _, m, n, r = synth.PREFILL_SHAPE
+    gen = torch.Generator(device=device)
+    gen.manual_seed(4242)
+    Upk = torch.randint(-(1 << 31), 1 << 31, (m, r // 32), dtype=torch.int64, device=device, generator=gen).to(torch.int32)
+    Vpk = torch.randint(-(1 << 31), 1 << 31, (r, n // 32), dtype=torch.int64, device=device, generator=gen).to(torch.int32)
+    s1 = torch.from_numpy(synth.scales_f16(m, 4242, "s1").view(np.int16)).to(device)
+    s2 = torch.from_numpy(synth.scales_f16(n, 4242, "s2").view(np.int16)).to(device)
+    out = {}
+    for b in synth.PREFILL_BATCHES:
+        x = torch.from_numpy(synth.activations_bf16(b, n, 4242, b).view(np.int16)).to(device)
+        y = torch.empty((b, m), dtype=torch.float32, device=device)
+        nq.workspace_reserve(m, n, r, b)
+        fwd = nq.lib().nq_lowrank_linear_fwd
+
+        def one(h):
+            st = fwd(x.data_ptr(), Upk.data_ptr(), Vpk.data_ptr(), s1.data_ptr(), s2.data_ptr(), m, n, r, b,
+                     y.data_ptr(), h)
+            if st != 0:
+                raise RuntimeError(nq.nq_status_string(st))
+
+        with torch.cuda.stream(stream):
+            one(stream.cuda_stream)
+        torch.cuda.synchronize()
+        g = capture(lambda h: [one(h) for _ in range(calls)], stream)
+        for _ in range(max(1, warmup // calls)):
+            g.replay()
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(reps):
+                g.replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+        nq.device_status(stream.cuda_stream)
+        ms = start.elapsed_time(end) / (reps * calls)
+        flops = 2.0 * b * r * (m + n)
+        tf = flops / (ms * 1e-3) / 1e12
+        out[str(b)] = {"tflops": round(tf, 1), "us_per_call": round(ms * 1e3, 2),
+                       "frac_of_bf16_burst": round(tf / peaks["bf16_tflops"], 4),
+                       "tokens_per_s": round(b / (ms * 1e-3), 1)}
+        del g, x, y
+    return out
 
 
 def run_e2e(work, stream, steps, device):

@@ -12,7 +12,6 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxDim = int64_t(1) << 20;
 constexpr int64_t kMaxRank = 65536;
-constexpr int kMaxSplits = 64;
 
 std::mutex g_mutex;
 Workspace g_ws[kMaxDevices];
@@ -47,7 +46,7 @@ int sm_count() {
     return g_sm_count[dev];
 }
 
-Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, int* status) {
+Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, const DecodeNeed& dec, int* status) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         cudaGetLastError();
@@ -56,16 +55,23 @@ Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, int* st
     }
     std::lock_guard<std::mutex> lock(g_mutex);
     Workspace& w = g_ws[dev];
-    const int64_t pbatch = batch > 8 ? batch : 0;  // prefill buffers only for prefill batches
-    if (w.base && r <= w.r_cap && n <= w.n_cap && m <= w.m_cap && pbatch <= w.batch_cap) {
+    const int64_t pbatch = batch > NQ_DECODE_MAX_BATCH ? batch : 0;  // prefill buffers only for prefill
+    auto fits = [&](const Workspace& c) {
+        return c.base && r <= c.r_cap && n <= c.n_cap && m <= c.m_cap && pbatch <= c.batch_cap &&
+               (size_t)dec.t <= c.t_cap && (size_t)dec.tgmax <= c.tgmax_cap && (size_t)dec.partials <= c.partial_cap &&
+               (size_t)dec.counters <= c.counter_cap;
+    };
+    if (fits(w)) {
         *status = NQ_OK;
         return &w;
     }
     // grow: keep the larger of old and new capacities
-    int64_t r_cap = r > w.r_cap ? r : w.r_cap;
-    int64_t n_cap = n > w.n_cap ? n : w.n_cap;
-    int64_t m_cap = m > w.m_cap ? m : w.m_cap;
-    int64_t b_cap = pbatch > w.batch_cap ? pbatch : w.batch_cap;
+    auto mx = [](int64_t a, int64_t b) { return a > b ? a : b; };
+    const int64_t r_cap = mx(r, w.r_cap), n_cap = mx(n, w.n_cap), m_cap = mx(m, w.m_cap);
+    const int64_t b_cap = mx(pbatch, w.batch_cap);
+    const size_t t_cap = (size_t)mx(dec.t, (int64_t)w.t_cap), g_cap = (size_t)mx(dec.tgmax, (int64_t)w.tgmax_cap);
+    const size_t p_cap = (size_t)mx(dec.partials, (int64_t)w.partial_cap);
+    const size_t c_cap = (size_t)mx(dec.counters, (int64_t)w.counter_cap);
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     cudaStreamIsCapturing(0, &cs);  // legacy stream: errors if a global capture is active
     if (cudaGetLastError() != cudaSuccess) {
@@ -74,10 +80,10 @@ Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, int* st
     }
     if (w.base) cudaDeviceSynchronize();  // old buffers may still be in use
     size_t off = 0;
-    const size_t o_t = off;        off = align_up(off + sizeof(float) * 8 * r_cap, 256);
-    const size_t o_tgmax = off;    off = align_up(off + sizeof(float) * 8 * (r_cap / 128 + 1), 256);
-    const size_t o_part = off;     off = align_up(off + sizeof(float) * (size_t)kMaxSplits * 8 * r_cap, 256);
-    const size_t o_cnt = off;      off = align_up(off + sizeof(int) * (r_cap / 128 + 1), 256);
+    const size_t o_t = off;        off = align_up(off + sizeof(float) * (t_cap + 1), 256);
+    const size_t o_tgmax = off;    off = align_up(off + sizeof(float) * (g_cap + 1), 256);
+    const size_t o_part = off;     off = align_up(off + sizeof(float) * (p_cap + 1), 256);
+    const size_t o_cnt = off;      off = align_up(off + sizeof(int) * (c_cap + 1), 256);
     const size_t o_status = off;   off = align_up(off + sizeof(unsigned) * 64, 256);
     const size_t o_xp = off;       off = align_up(off + sizeof(uint16_t) * (size_t)b_cap * n_cap, 256);
     const size_t o_T = off;        off = align_up(off + sizeof(uint16_t) * (size_t)b_cap * r_cap, 256);
@@ -104,13 +110,23 @@ Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, int* st
     w.status = reinterpret_cast<unsigned*>(base + o_status);
     w.xprime = reinterpret_cast<uint16_t*>(base + o_xp);
     w.T = reinterpret_cast<uint16_t*>(base + o_T);
+    w.t_cap = t_cap;
+    w.tgmax_cap = g_cap;
+    w.partial_cap = p_cap;
+    w.counter_cap = c_cap;
     w.r_cap = r_cap;
     w.n_cap = n_cap;
     w.m_cap = m_cap;
     w.batch_cap = b_cap;
-    w.split_cap = kMaxSplits;
     *status = NQ_OK;
     return &w;
+}
+
+DecodeNeed decode_need(const DecodeCall* calls, int count, int64_t batch) {
+    DecodeNeed d;
+    if (batch >= 1 && batch <= NQ_DECODE_MAX_BATCH)
+        decode_workspace_need(calls, count, batch, &d.t, &d.tgmax, &d.partials, &d.counters);
+    return d;
 }
 
 // Host-memory x / y are staged through device buffers of the workspace.
@@ -185,7 +201,7 @@ int nq_pack_signs(const int8_t* signs, int64_t rows, int64_t cols, uint32_t* out
         return NQ_OK;
     }
     int st = NQ_OK;
-    Workspace* ws = workspace_for(128, 128, 128, 0, &st);
+    Workspace* ws = workspace_for(128, 128, 128, 0, DecodeNeed(), &st);
     if (!ws) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(ws->status, 0, sizeof(unsigned), s) != cudaSuccess) return NQ_ERR_CUDA;
@@ -215,13 +231,79 @@ int nq_unpack_signs(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* 
     return unpack_device(packed, rows, cols, out, static_cast<cudaStream_t>(stream));
 }
 
+int nq_lowrank_linear_fwd_grouped(const nq_linear_desc* layers, int count, int64_t batch, void* stream) {
+    if (batch < 0) return NQ_ERR_BATCH;
+    if (count < 0) return NQ_ERR_SHAPE;
+    if (count == 0 || batch == 0) return NQ_OK;
+    if (!layers) return NQ_ERR_NULL;
+    int64_t m_max = 0, n_max = 0, r_max = 0;
+    for (int i = 0; i < count; ++i) {
+        const nq_linear_desc& L = layers[i];
+        if (L.m <= 0 || L.n <= 0 || L.r <= 0 || L.m % 128 || L.n % 128 || L.r % 128 || L.m > kMaxDim ||
+            L.n > kMaxDim || L.r > kMaxRank)
+            return NQ_ERR_SHAPE;
+        if (batch > (int64_t(1) << 40) / (L.m > L.n ? L.m : L.n)) return NQ_ERR_SHAPE;
+        if (!L.x || !L.Upk || !L.Vpk || !L.s1 || !L.s2 || !L.y) return NQ_ERR_NULL;
+        if (!aligned16(L.x) || !aligned16(L.Upk) || !aligned16(L.Vpk) || !aligned16(L.s1) || !aligned16(L.s2) ||
+            !aligned16(L.y))
+            return NQ_ERR_ALIGN;
+        m_max = L.m > m_max ? L.m : m_max;
+        n_max = L.n > n_max ? L.n : n_max;
+        r_max = L.r > r_max ? L.r : r_max;
+    }
+    for (int i = 0; i < count; ++i) {
+        const nq_linear_desc& L = layers[i];
+        if (!pointer_kind(L.x) || !pointer_kind(L.Upk) || !pointer_kind(L.Vpk) || !pointer_kind(L.s1) ||
+            !pointer_kind(L.s2) || !pointer_kind(L.y))
+            return NQ_ERR_PTRKIND;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int st = NQ_OK;
+    if (batch > NQ_DECODE_MAX_BATCH) {
+        Workspace* ws = workspace_for(m_max, n_max, r_max, batch, DecodeNeed(), &st);
+        if (!ws) return st;
+        for (int i = 0; i < count && st == NQ_OK; ++i) {
+            const nq_linear_desc& L = layers[i];
+            st = prefill_forward(static_cast<const uint16_t*>(L.x), L.Upk, L.Vpk, static_cast<const uint16_t*>(L.s1),
+                                 static_cast<const uint16_t*>(L.s2), L.m, L.n, L.r, batch, L.y, ws, s);
+        }
+        return st;
+    }
+    for (int i0 = 0; i0 < count && st == NQ_OK; i0 += kMaxGroup) {
+        const int cnt = count - i0 < kMaxGroup ? count - i0 : kMaxGroup;
+        DecodeCall calls[kMaxGroup];
+        for (int i = 0; i < cnt; ++i) {
+            const nq_linear_desc& L = layers[i0 + i];
+            calls[i] = DecodeCall{static_cast<const uint16_t*>(L.x), L.Upk, L.Vpk, static_cast<const uint16_t*>(L.s1),
+                                  static_cast<const uint16_t*>(L.s2), L.y, L.m, L.n, L.r};
+        }
+        Workspace* ws = workspace_for(m_max, n_max, r_max, batch, decode_need(calls, cnt, batch), &st);
+        if (!ws) return st;
+        st = decode_forward_group(calls, cnt, batch, ws, s);
+    }
+    return st;
+}
+
+int nq_device_status(void* stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NQ_ERR_CUDA;
+    int st = NQ_OK;
+    Workspace* ws = workspace_for(128, 128, 128, 0, DecodeNeed(), &st);
+    if (!ws) return st;
+    unsigned word = 0;
+    if (cudaMemcpy(&word, ws->status + 1, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) return NQ_ERR_CUDA;
+    if (word != 0 && cudaMemset(ws->status + 1, 0, sizeof(unsigned)) != cudaSuccess) return NQ_ERR_CUDA;
+    return word == 0 ? NQ_OK : -(int)word;
+}
+
 int nq_workspace_reserve(int64_t m, int64_t n, int64_t r, int64_t batch) {
     if (m <= 0 || n <= 0 || r <= 0 || m % 128 || n % 128 || r % 128 || m > kMaxDim || n > kMaxDim ||
         r > kMaxRank)
         return NQ_ERR_SHAPE;
     if (batch < 0) return NQ_ERR_BATCH;
     int st = NQ_OK;
-    Workspace* ws = workspace_for(m, n, r, batch, &st);
+    const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, m, n, r};
+    Workspace* ws = workspace_for(m, n, r, batch, decode_need(&c, 1, batch), &st);
     return ws ? NQ_OK : st;
 }
 
@@ -243,7 +325,8 @@ int nq_lowrank_linear_fwd(const void* x, const uint32_t* Upk, const uint32_t* Vp
     const bool x_host = pointer_kind(x) == 0, y_host = pointer_kind(y) == 0;
 
     int st = NQ_OK;
-    Workspace* ws = workspace_for(m, n, r, batch, &st);
+    const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, m, n, r};
+    Workspace* ws = workspace_for(m, n, r, batch, decode_need(&c, 1, batch), &st);
     if (!ws) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t xbytes = sizeof(uint16_t) * (size_t)batch * n, ybytes = sizeof(float) * (size_t)batch * m;

@@ -1,33 +1,40 @@
-// nq_decode.cu -- decode path (1 <= batch <= 8): two binary GEMV stages.
+// nq_decode.cu -- decode path (1 <= batch <= 8): two binary GEMV stages per layer.
 //
 //   stage 1:  t_k = sum_j V[j][k] * (s2_j x_j)          (rows k of V^T, r of them)
 //   stage 2:  y_i = s1_i * sum_k U[i][k] * t_k          (rows i of U, m of them)
 //
 // The product with a +1/-1 row is the binary GEMV of hardwired.dev section "Cisla"
 // (custom binary GEMV/GEMM kernels) for the factorised weight of section "Jak
-// NanoQuant funguje".  Both stages run the same core: a row of signs against a vector.
+// NanoQuant funguje".  Both stages run the same core: 16 rows of signs against a vector.
 //
 // Why integer tensor-core instructions.  At HBM speed a B200 SM must retire ~190 packed
-// sign bits per clock but can issue only 4 warp instructions per clock, so unpacking a
-// bit and adding +/-x on the CUDA cores (shift, sign flip, add: >= 3 ops per bit per
-// token) caps a GEMV at a fraction of the bandwidth.  Here one LOP3 turns a word into
-// four bytes that are 0 or 2^s (s = bit position inside each byte, a mask selects the
-// bits s, s+8, s+16, s+24), and mma.sync m16n8k32 (u8 x s8 -> s32) multiplies 16 rows
-// x 32 such bytes against the activation, which is quantised per column range to 14
-// bits and split into two int8 limbs (hi, lo) that sit in the MMA's N dimension next to
-// up to four tokens.  Integer accumulation is exact; the only rounding is the 14-bit
-// quantisation of the activation (relative step 2^-14 of the range's largest entry).
+// sign bits per clock but issues only 4 warp instructions per clock (and logic ops at
+// half that rate), so unpacking a bit and adding +/-x on the CUDA cores (shift, sign
+// flip, add: >= 3 ops per bit per token) caps a GEMV at a fraction of the bandwidth.
+// Here one LOP3 turns a word into four bytes that are 0 or 2^s (a mask selects bits s,
+// s+8, s+16, s+24), and mma.sync m16n8k32 (u8 x s8 -> s32) multiplies 16 rows x 32 such
+// bytes against the activation, which is quantised per column chunk to 14 bits and split
+// into two int8 limbs (hi, lo) that sit in the MMA's N dimension beside up to four
+// tokens.  Integer accumulation is exact; the only rounding is the 14-bit quantisation of
+// the activation (relative step 2^-14 of the chunk's largest entry).
 //
 // Since the A bytes are 0/1 (times 2^s), the MMA yields sum_j b_j q_j; the signed sum is
 // sum_j (2 b_j - 1) q_j = 2 * sum_j b_j q_j - sum_j q_j, with sum_j q_j counted while
 // quantising.
 //
-// Layout in one column block (CB) of 128 columns = 4 words per row: lane (g, t) of a
-// warp (g = lane/4, t = lane%4) reads word t of rows g and g+8 of a 16-row tile.  For s
-// in 0..3, A = { w & M_s, w(g+8) & M_s, (w>>4) & M_s, (w(g+8)>>4) & M_s } with
-// M_s = 0x01010101 << s.  MMA K column 4t+c maps to column 32t + s + 8c of the CB and K
-// column 16+4t+c to column 32t + s + 4 + 8c; the B fragments are built in that order.
-// N column n = 2*token + limb (limb 0 = hi, 1 = lo), four tokens per "token group".
+// Fragment layout in one column block (CB) of 128 columns = 4 words per row: lane (g, t)
+// of a warp (g = lane/4, t = lane%4) takes word t of rows g and g+8 of a 16-row tile.
+// For s in 0..3, A = { w & M_s, w(g+8) & M_s, (w>>4) & M_s, (w(g+8)>>4) & M_s } with
+// M_s = 0x01010101 << s.  MMA K column 4t+c is column 32t + s + 8c of the CB and K column
+// 16+4t+c is column 32t + s + 4 + 8c; the B fragments are built in that order.  N column
+// n = 2*token + limb (limb 0 = hi, 1 = lo), four tokens per token group.
+//
+// Latency.  A decode layer moves 0.4-18 MB, a few microseconds at HBM speed, so the
+// fixed costs decide: each CTA copies its weight rows into shared memory with cp.async
+// (and prefetches the rest into L2) before it waits on the previous kernel
+// (programmatic dependent launch), and it lets the next kernel launch at once, so weight
+// streaming overlaps the dependency chain.  Stage-1 CTAs own whole rows (no cross-CTA
+// reduction), and several independent layers can share one launch pair.
 #include <cuda_fp16.h>
 #include <math.h>
 
@@ -36,12 +43,15 @@
 namespace nq {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;          // 4 warps
 constexpr int kWarps = kThreads / 32;
-constexpr int kCB = 128;           // columns per column block
-constexpr int kChunk = 2048;       // columns quantised and staged per pass
+constexpr int kCB = 128;               // columns per column block
+constexpr int kChunk = 1024;           // columns staged per pass
 constexpr int kChunkCB = kChunk / kCB;
-constexpr int kQBits = 14;         // |q| < 2^14
+constexpr int kChunkWords = kChunk / 32;
+constexpr int kQBits = 14;             // |q| < 2^14
+constexpr int kRowsS1 = 64;            // stage-1 rows per CTA (4 warps x 16)
+constexpr int kRowPad = 4;             // words of padding per staged row (bank spread)
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 __device__ __forceinline__ float f16_to_f32(uint16_t h) { return __half2float(__ushort_as_half(h)); }
@@ -55,83 +65,170 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Exponent E with max < 2^E (0 for max == 0): values are quantised as rint(v * 2^(14-E)).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Quantisation exponent E of a range whose largest |value| is max_abs: max_abs < 2^E,
+// clamped to [-100, 113] so that both 2^(14-E) and 2^(E-14) are normal floats.  Values
+// are quantised as q = rint(v * 2^(14-E)), |q| < 2^14, and dequantised by 2^(E-14); both
+// scalings are exact.  (Inputs whose largest magnitude is below 2^-100 lose precision.)
 __device__ __forceinline__ int range_exponent(float max_abs) {
     int e = 0;
     if (max_abs > 0.f) frexpf(max_abs, &e);
-    return e;
+    return min(max(e, -100), 113);
 }
 
-__device__ __forceinline__ int quantise(float v, int e) {
-    float q = rintf(scalbnf(v, kQBits - e));
-    q = fminf(fmaxf(q, -16384.f), 16383.f);
-    return (int)q;
+__device__ __forceinline__ float pow2f(int k) { return __int_as_float((k + 127) << 23); }  // k in [-126, 127]
+
+__device__ __forceinline__ int quantise(float v, float up) {
+    const int q = __float2int_rn(v * up);
+    return min(max(q, -16384), 16383);
 }
 
-// Shared-memory staging of one chunk: q values (int16) and the B fragments.
-struct ChunkSmem {
-    int16_t q[8][kChunk];                  // 32 KB
-    uint4 frag[kChunkCB][2][2][32];        // [cb][token group][half][lane] = 32 KB
+__device__ __forceinline__ float warp_max(float v) {
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// One layer of a decode launch (device view).
+struct DecLayer {
+    const uint16_t* x;
+    const uint32_t* Upk;
+    const uint32_t* Vpk;
+    const uint16_t* s1;
+    const uint16_t* s2;
+    float* y;
+    float* t;        // workspace: batch x r
+    float* tgmax;    // workspace: batch x r/64 (max |t| per 64-row block)
+    float* partials; // workspace: nsplit x batch x r (stage-1 column splits)
+    int* counters;   // workspace: r/64 arrival counters, zero between calls
+    int m, n, r;
+    int nsplit;      // stage-1 column splits (CTAs per 64-row block)
+    int cps;         // column blocks per split
+    int rt;          // stage-2 row tiles per CTA (4/rt k-parts per tile)
 };
 
-// Build the B fragments of `ncb` column blocks from sq (tokens >= batch are zero).
-__device__ void build_fragments(ChunkSmem& sm, int ncb, int batch, int ntg) {
-    const int total = ncb * ntg * 32 * 8;  // fragment words
-    for (int idx = threadIdx.x; idx < total; idx += kThreads) {
-        const int j = idx & 7;             // 2*s + h
-        const int lane = (idx >> 3) & 31;
-        const int tg = (idx >> 8) % ntg;
-        const int cb = (idx >> 8) / ntg;
-        const int s = j >> 1, h = j & 1;
-        const int t = lane & 3, tok = 4 * tg + (lane >> 3), limb = (lane >> 2) & 1;
-        uint32_t word = 0;
-        if (tok < batch) {
-            const int16_t* qrow = sm.q[tok] + cb * kCB + 32 * t + s + 4 * h;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                int q = qrow[8 * c];
-                uint32_t byte = limb == 0 ? (uint32_t)((q >> 7) & 0xFF) : (uint32_t)(q & 0x7F);
-                word |= byte << (8 * c);
-            }
-        }
-        reinterpret_cast<uint32_t*>(&sm.frag[cb][tg][j >> 2][lane])[j & 3] = word;
+struct DecGroup {
+    DecLayer L[kMaxGroup];
+    int count;
+    int batch;
+    int s1_start[kMaxGroup + 1];
+    int s2_start[kMaxGroup + 1];
+};
+
+__device__ __forceinline__ int find_layer(const int* start, int count, int block) {
+    int l = 0;
+    while (l + 1 < count && block >= start[l + 1]) ++l;
+    return l;
+}
+
+// Shared memory of both stages; NT = 4 * NTG token slots.
+template <int NTG>
+struct DecSmem {
+    static constexpr int NT = 4 * NTG;
+    uint32_t w[2][kRowsS1][kChunkWords + kRowPad];  // weight rows of two chunks (18 KB)
+    union {
+        float t[2][NT][kChunk];                      // stage 2: two chunks of t
+        struct {
+            uint16_t x[2][NT][kChunk];               // stage 1: two chunks of x
+            uint16_t s2[2][kChunk];                  //          and of s2
+        } s1;
+    } act;
+    uint4 frag[kChunkCB][NTG][2][32];               // [cb][token group][half][lane]
+    float red[kWarps][8];
+    int e[8];
+    float up[8];                                    // 2^(14 - e): quantisation factor per token
+    int qsum[8];
+    int bq[64][8];                                  // stage 2: per (row, token) across k-parts
+    float res[8][kRowsS1];                          // stage 1: sums of the CTA's rows
+    int last;
+};
+
+// Copy `rows` weight rows, words [w0, w0 + nw) of each, into buffer `buf` (cp.async).
+template <int NTG>
+__device__ __forceinline__ void stage_weights(DecSmem<NTG>& sm, int buf, const uint32_t* W, int64_t wpr, int rows,
+                                              int64_t w0, int nw) {
+    const int per_row = nw / 4;  // 16-byte pieces
+    const int total = rows * per_row;
+    for (int i = threadIdx.x; i < total; i += kThreads) {
+        const int row = i / per_row, p = i % per_row;
+        cp_async16(&sm.w[buf][row][4 * p], W + (int64_t)row * wpr + w0 + 4 * p);
     }
 }
 
-// Accumulate one 16-row tile against column blocks [cb0, cb1) of the staged chunk.
-// W points at word 0 of the tile's row 0 for the chunk; wpr = words per row.
-template <int NTG>
-__device__ __forceinline__ void tile_mma(const uint32_t* __restrict__ W, int64_t wpr, const ChunkSmem& sm,
-                                         int cb0, int cb1, int cbstep, int (&acc)[NTG][4][4]) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const uint32_t* rg = W + (int64_t)g * wpr + t;
-    const uint32_t* rg8 = rg + 8 * wpr;
-    int cb = cb0;
-    for (; cb + 3 * cbstep < cb1; cb += 4 * cbstep) {
-        uint32_t wa[4], wb[4];
+// B fragments of `ncb` column blocks from values v(tok, col) (col relative to the chunk),
+// quantised with sm.up[tok]; adds each token's sum of q to sm.qsum.  One task =
+// (cb, token, word t of the CB, half h): the 16 columns 32t + s + 4h + 8c (s, c in 0..3)
+// feed fragment words j = 2s + h of two lanes, the hi-limb lane 8*tok' + t and the
+// lo-limb lane 8*tok' + 4 + t (tok' = token within its group).  Slots of tokens >= batch
+// are never written and stay zero (zero_fragments at kernel start).
+template <int NTG, typename ValueFn>
+__device__ __forceinline__ void build_fragments(DecSmem<NTG>& sm, int ncb, int batch, ValueFn value) {
+    const int tasks = ncb * batch * 8;
+    for (int task = threadIdx.x; task < tasks; task += kThreads) {
+        const int h = task & 1, t = (task >> 1) & 3;
+        const int tok = (task >> 3) % batch, cb = (task >> 3) / batch;
+        const float up = sm.up[tok];
+        const int c0 = cb * kCB + 32 * t + 4 * h;
+        uint32_t hi[4], lo[4];
+        int qs = 0;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            wa[u] = __ldg(rg + 4 * (cb + u * cbstep));
-            wb[u] = __ldg(rg8 + 4 * (cb + u * cbstep));
-        }
+        for (int s4 = 0; s4 < 4; ++s4) {
+            uint32_t wh = 0, wl = 0;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int c = cb + u * cbstep;
-            const uint32_t a4 = wa[u] >> 4, b4 = wb[u] >> 4;
-#pragma unroll
-            for (int tg = 0; tg < NTG; ++tg) {
-                const uint4 f0 = sm.frag[c][tg][0][lane], f1 = sm.frag[c][tg][1][lane];
-                const uint32_t bf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const uint32_t M = 0x01010101u << s;
-                    mma_u8s8(acc[tg][s], wa[u] & M, wb[u] & M, a4 & M, b4 & M, bf[2 * s], bf[2 * s + 1]);
-                }
+            for (int c = 0; c < 4; ++c) {
+                const int q = quantise(value(tok, c0 + s4 + 8 * c), up);
+                qs += q;
+                wh |= (uint32_t)((q >> 7) & 0xFF) << (8 * c);
+                wl |= (uint32_t)(q & 0x7F) << (8 * c);
             }
+            hi[s4] = wh;
+            lo[s4] = wl;
         }
+        atomicAdd(&sm.qsum[tok], qs);
+        const int tg = tok >> 2, ti = tok & 3;
+        uint32_t* fh0 = reinterpret_cast<uint32_t*>(&sm.frag[cb][tg][0][8 * ti + t]);
+        uint32_t* fh1 = reinterpret_cast<uint32_t*>(&sm.frag[cb][tg][1][8 * ti + t]);
+        uint32_t* fl0 = reinterpret_cast<uint32_t*>(&sm.frag[cb][tg][0][8 * ti + 4 + t]);
+        uint32_t* fl1 = reinterpret_cast<uint32_t*>(&sm.frag[cb][tg][1][8 * ti + 4 + t]);
+        // word j = 2*s4 + h lives in half j >> 2 at component j & 3
+        fh0[h] = hi[0];
+        fh0[2 + h] = hi[1];
+        fh1[h] = hi[2];
+        fh1[2 + h] = hi[3];
+        fl0[h] = lo[0];
+        fl0[2 + h] = lo[1];
+        fl1[h] = lo[2];
+        fl1[2 + h] = lo[3];
     }
-    for (; cb < cb1; cb += cbstep) {
-        const uint32_t wa = __ldg(rg + 4 * cb), wb = __ldg(rg8 + 4 * cb);
+}
+
+template <int NTG>
+__device__ __forceinline__ void zero_fragments(DecSmem<NTG>& sm) {
+    uint4* f = &sm.frag[0][0][0][0];
+    for (int i = threadIdx.x; i < kChunkCB * NTG * 2 * 32; i += kThreads) f[i] = make_uint4(0, 0, 0, 0);
+}
+
+// Accumulate one 16-row tile (rows r0.., staged in sm.w[buf]) against column blocks
+// cb0, cb0 + step, ... < cb1 of the staged chunk.
+template <int NTG>
+__device__ __forceinline__ void tile_mma(const DecSmem<NTG>& sm, int buf, int r0, int cb0, int cb1, int step,
+                                         int (&acc)[NTG][4][4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const uint32_t* wa_row = sm.w[buf][r0 + g];
+    const uint32_t* wb_row = sm.w[buf][r0 + g + 8];
+#pragma unroll 2
+    for (int cb = cb0; cb < cb1; cb += step) {
+        const uint32_t wa = wa_row[4 * cb + t], wb = wb_row[4 * cb + t];
         const uint32_t a4 = wa >> 4, b4 = wb >> 4;
 #pragma unroll
         for (int tg = 0; tg < NTG; ++tg) {
@@ -146,7 +243,7 @@ __device__ __forceinline__ void tile_mma(const uint32_t* __restrict__ W, int64_t
     }
 }
 
-// sum_j b_j q_j for (row g, token 4tg+t) and (row g+8, same token) from the accumulators.
+// sum_j b_j q_j for (row g, token 4tg+t) and (row g+8, same token).
 template <int NTG>
 __device__ __forceinline__ void combine(const int (&acc)[NTG][4][4], int tg, int& row_g, int& row_g8) {
     int hi0 = 0, lo0 = 0, hi8 = 0, lo8 = 0;
@@ -161,107 +258,102 @@ __device__ __forceinline__ void combine(const int (&acc)[NTG][4][4], int tg, int
     row_g8 = hi8 * 128 + lo8;
 }
 
-__device__ __forceinline__ float block_max_token(float v, float* sred) {
-    // max over the block of v for one token; sred has kWarps floats
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) sred[threadIdx.x >> 5] = v;
-    __syncthreads();
-    float m = sred[0];
-    for (int w = 1; w < kWarps; ++w) m = fmaxf(m, sred[w]);
-    return m;
+template <int NTG>
+__device__ __forceinline__ void zero_acc(int (&acc)[NTG][4][4]) {
+#pragma unroll
+    for (int tg = 0; tg < NTG; ++tg)
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[tg][s][i] = 0;
 }
 
-struct Stage1Smem {
-    ChunkSmem chunk;
-    float v[8][kChunk];                    // 64 KB: s2 * x of the chunk
-    float res[8][128];                     // finished sums of the CTA's 128 rows
-    float red[kWarps];
-    int e[8];
-    int qsum[8];
-    int last;
-};
-
-struct Stage2Smem {
-    ChunkSmem chunk;
-    int bq[128][8];                        // per (row of the CTA, token) sum_k b q
-    int e[8];
-    int qsum[8];
-};
-
 // ------------------------------------------------------------------ stage 1
-// grid = (r/128 row groups, nsplit).  CTA (rg, sp) handles rows [128 rg, 128 rg + 128)
-// of V^T against column blocks [sp*cps, (sp+1)*cps), staged kChunk columns at a time;
-// warp w owns rows
-// 128 rg + 16 w .. +16.  Each chunk has its own quantisation exponent per token, so
-// the warp converts its integer sums to fp32 after every chunk.  With nsplit > 1 the
-// CTAs of a row group leave fp32 partials; the last to arrive adds them in split order
-// (deterministic) and writes t and the row group's max |t| per token.
+// CTA = 64 rows of V^T of one layer x one column split (cps column blocks, staged kChunk
+// columns at a time); warp w owns rows 16w..16w+15.  Each chunk has its own quantisation
+// exponent per token, so the warp converts its integer sums to fp32 after every chunk.
+// With several splits, the CTAs of a row block leave fp32 partials and the last to arrive
+// adds them in split order (deterministic), then writes t and the block's max |t| per
+// token (stage 2 builds its exponent from those maxima).
 template <int NTG>
-__global__ void __launch_bounds__(kThreads) stage1_kernel(const uint16_t* __restrict__ x,
-                                                          const uint32_t* __restrict__ Vpk,
-                                                          const uint16_t* __restrict__ s2, int64_t n, int64_t r,
-                                                          int batch, int nsplit, int cps, float* __restrict__ t,
-                                                          float* __restrict__ tgmax, float* __restrict__ partials,
-                                                          int* __restrict__ counters) {
+__device__ __forceinline__ void stage1_fetch_x(DecSmem<NTG>& sm, int buf, const DecLayer& L, int batch, int col0,
+                                               int ccols) {
+    const int per_tok = ccols / 8;  // 16-byte pieces
+    for (int i = threadIdx.x; i < (batch + 1) * per_tok; i += kThreads) {
+        const int tok = i / per_tok, p = i % per_tok;
+        if (tok < batch)
+            cp_async16(&sm.act.s1.x[buf][tok][8 * p], L.x + (int64_t)tok * L.n + col0 + 8 * p);
+        else
+            cp_async16(&sm.act.s1.s2[buf][8 * p], L.s2 + col0 + 8 * p);
+    }
+}
+
+template <int NTG>
+__global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant__ DecGroup grp) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    Stage1Smem& sm = *reinterpret_cast<Stage1Smem*>(smem_raw);
-    const int rg = blockIdx.x, sp = blockIdx.y;
+    DecSmem<NTG>& sm = *reinterpret_cast<DecSmem<NTG>*>(smem_raw);
+    const int li = find_layer(grp.s1_start, grp.count, blockIdx.x);
+    const DecLayer& L = grp.L[li];
+    const int local = blockIdx.x - grp.s1_start[li];
+    const int rb = local / L.nsplit, sp = local % L.nsplit;
+    const int batch = grp.batch;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    const int n = L.n, r = L.r;
     const int64_t wpr = n / 32;
-    const int64_t row0 = (int64_t)rg * 128 + 16 * warp;
-    const int ncb_total = (int)(n / kCB);
-    const int cbA = sp * cps, cbB = min(ncb_total, cbA + cps);
+    const int64_t row0 = (int64_t)rb * kRowsS1;
+    const uint32_t* W = L.Vpk + row0 * wpr;
+    const int cbA = sp * L.cps, cbB = min(n / kCB, cbA + L.cps);
+    const int nchunks = (cbB - cbA + kChunkCB - 1) / kChunkCB;
+    auto chunk_cb = [&](int ch) { return min(kChunkCB, cbB - cbA - ch * kChunkCB); };
+
+    // weights first: they do not depend on the previous kernel
+    stage_weights(sm, 0, W, wpr, kRowsS1, (int64_t)cbA * 4, chunk_cb(0) * 4);
+    cp_async_commit();
+    if (nchunks > 1) stage_weights(sm, 1, W, wpr, kRowsS1, (int64_t)(cbA + kChunkCB) * 4, chunk_cb(1) * 4);
+    cp_async_commit();
+    if (nchunks > 2 && threadIdx.x < kRowsS1)
+        prefetch_l2(W + threadIdx.x * wpr + (cbA + 2 * kChunkCB) * 4, (uint32_t)((cbB - cbA - 2 * kChunkCB) * 16));
+    zero_fragments(sm);
+    pdl_trigger();
+    pdl_wait();  // x may come from the previous kernel on the stream
+    stage1_fetch_x(sm, 0, L, batch, cbA * kCB, chunk_cb(0) * kCB);
+    cp_async_commit();
+    if (nchunks > 1) stage1_fetch_x(sm, 1, L, batch, (cbA + kChunkCB) * kCB, chunk_cb(1) * kCB);
+    cp_async_commit();
 
     float part[NTG][2];
 #pragma unroll
     for (int tg = 0; tg < NTG; ++tg) part[tg][0] = part[tg][1] = 0.f;
 
-    pdl_wait();  // x may come from the previous kernel on the stream
-
-    for (int cbc = cbA; cbc < cbB; cbc += kChunkCB) {
-        const int ncb = min(kChunkCB, cbB - cbc);
-        const int64_t col0 = (int64_t)cbc * kCB;
+    for (int ch = 0; ch < nchunks; ++ch) {
+        const int buf = ch & 1;
+        const int ncb = chunk_cb(ch);
         const int ccols = ncb * kCB;
-        // stage s2 * x (exact in fp32) and its per-token max
-        for (int tok = 0; tok < batch; ++tok) {
+        if (ch + 1 < nchunks) cp_async_wait<1>(); else cp_async_wait<0>();
+        __syncthreads();
+        // per-token max of s2 * x over the chunk
+        const uint16_t* xs = &sm.act.s1.x[buf][0][0];
+        const uint16_t* ss = sm.act.s1.s2[buf];
+        for (int tok = warp; tok < batch; tok += kWarps) {
             float mx = 0.f;
-            for (int c = threadIdx.x; c < ccols; c += kThreads) {
-                float v = bf16_to_f32(x[(int64_t)tok * n + col0 + c]) * f16_to_f32(s2[col0 + c]);
-                sm.v[tok][c] = v;
-                mx = fmaxf(mx, fabsf(v));
-            }
-            mx = block_max_token(mx, sm.red);
-            if (threadIdx.x == 0) {
-                sm.e[tok] = range_exponent(mx);
+            for (int c = lane; c < ccols; c += 32) mx = fmaxf(mx, fabsf(bf16_to_f32(xs[tok * kChunk + c]) * f16_to_f32(ss[c])));
+            mx = warp_max(mx);
+            if (lane == 0) {
+                const int e = range_exponent(mx);
+                sm.e[tok] = e;
+                sm.up[tok] = pow2f(kQBits - e);
                 sm.qsum[tok] = 0;
             }
         }
         __syncthreads();
-        for (int tok = 0; tok < batch; ++tok) {
-            const int e = sm.e[tok];
-            int qs = 0;
-            for (int c = threadIdx.x; c < ccols; c += kThreads) {
-                int q = quantise(sm.v[tok][c], e);
-                sm.chunk.q[tok][c] = (int16_t)q;
-                qs += q;
-            }
-            for (int o = 16; o > 0; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
-            if (lane == 0) atomicAdd(&sm.qsum[tok], qs);
-        }
-        __syncthreads();
-        build_fragments(sm.chunk, ncb, batch, NTG);
+        build_fragments(sm, ncb, batch, [&](int tok, int c) {
+            return bf16_to_f32(xs[tok * kChunk + c]) * f16_to_f32(ss[c]);
+        });
         __syncthreads();
 
         int acc[NTG][4][4];
-#pragma unroll
-        for (int tg = 0; tg < NTG; ++tg)
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[tg][s][i] = 0;
-        tile_mma<NTG>(Vpk + row0 * wpr + col0 / 32, wpr, sm.chunk, 0, ncb, 1, acc);
-
+        zero_acc<NTG>(acc);
+        tile_mma<NTG>(sm, buf, 16 * warp, 0, ncb, 1, acc);
 #pragma unroll
         for (int tg = 0; tg < NTG; ++tg) {
             const int tok = 4 * tg + tq;
@@ -269,15 +361,21 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const uint16_t* __rest
                 int bq0, bq8;
                 combine<NTG>(acc, tg, bq0, bq8);
                 const int64_t qs = sm.qsum[tok];
-                const int e = sm.e[tok] - kQBits;
-                part[tg][0] += scalbnf((float)(2 * (int64_t)bq0 - qs), e);
-                part[tg][1] += scalbnf((float)(2 * (int64_t)bq8 - qs), e);
+                const float down = pow2f(sm.e[tok] - kQBits);
+                part[tg][0] += (float)(2 * (int64_t)bq0 - qs) * down;
+                part[tg][1] += (float)(2 * (int64_t)bq8 - qs) * down;
             }
         }
-        __syncthreads();  // before the next chunk overwrites the staging
+        __syncthreads();  // buffers are free again
+        if (ch + 2 < nchunks) {
+            const int cb2 = cbA + (ch + 2) * kChunkCB;
+            stage_weights(sm, buf, W, wpr, kRowsS1, (int64_t)cb2 * 4, chunk_cb(ch + 2) * 4);
+            stage1_fetch_x(sm, buf, L, batch, cb2 * kCB, chunk_cb(ch + 2) * kCB);
+            cp_async_commit();
+        }
     }
-    pdl_trigger();
 
+    // this CTA's sums for its 64 rows, into shared memory
 #pragma unroll
     for (int tg = 0; tg < NTG; ++tg) {
         const int tok = 4 * tg + tq;
@@ -287,203 +385,260 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const uint16_t* __rest
         }
     }
     __syncthreads();
-
-    const int ngroups = (int)(r / 128);
-    if (nsplit == 1) {
-        for (int tok = 0; tok < batch; ++tok) {
-            float mx = 0.f;
-            for (int i = threadIdx.x; i < 128; i += kThreads) {
-                float v = sm.res[tok][i];
-                t[(int64_t)tok * r + (int64_t)rg * 128 + i] = v;
-                mx = fmaxf(mx, fabsf(v));
-            }
-            mx = block_max_token(mx, sm.red);
-            if (threadIdx.x == 0) tgmax[(int64_t)tok * ngroups + rg] = mx;
+    const int nrb = r / kRowsS1;
+    if (L.nsplit > 1) {
+        for (int i = threadIdx.x; i < batch * kRowsS1; i += kThreads) {
+            const int tok = i / kRowsS1, k = i % kRowsS1;
+            L.partials[((int64_t)sp * batch + tok) * r + row0 + k] = sm.res[tok][k];
         }
-        return;
-    }
-
-    for (int idx = threadIdx.x; idx < batch * 128; idx += kThreads) {
-        const int tok = idx / 128, i = idx % 128;
-        partials[((int64_t)sp * 8 + tok) * r + (int64_t)rg * 128 + i] = sm.res[tok][i];
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
         __threadfence();
-        int prev = atomicAdd(&counters[rg], 1);
-        sm.last = (prev == nsplit - 1);
-    }
-    __syncthreads();
-    if (!sm.last) return;
-    __threadfence();
-    for (int tok = 0; tok < batch; ++tok) {
-        float mx = 0.f;
-        for (int i = threadIdx.x; i < 128; i += kThreads) {
+        __syncthreads();
+        if (threadIdx.x == 0) sm.last = (atomicAdd(&L.counters[rb], 1) == L.nsplit - 1);
+        __syncthreads();
+        if (!sm.last) return;
+        __threadfence();
+        for (int i = threadIdx.x; i < batch * kRowsS1; i += kThreads) {
+            const int tok = i / kRowsS1, k = i % kRowsS1;
+            const float* pp = L.partials + (int64_t)tok * r + row0 + k;
+            const int64_t stride = (int64_t)batch * r;
             float sum = 0.f;
-            for (int s = 0; s < nsplit; ++s)
-                sum += __ldcg(&partials[((int64_t)s * 8 + tok) * r + (int64_t)rg * 128 + i]);
-            t[(int64_t)tok * r + (int64_t)rg * 128 + i] = sum;
-            mx = fmaxf(mx, fabsf(sum));
+            int q = 0;
+            for (; q + 4 <= L.nsplit; q += 4) {  // four independent loads in flight
+                const float a = __ldcg(pp + q * stride), b = __ldcg(pp + (q + 1) * stride);
+                const float c = __ldcg(pp + (q + 2) * stride), d = __ldcg(pp + (q + 3) * stride);
+                sum = (((sum + a) + b) + c) + d;
+            }
+            for (; q < L.nsplit; ++q) sum += __ldcg(pp + q * stride);
+            sm.res[tok][k] = sum;
         }
-        mx = block_max_token(mx, sm.red);
-        if (threadIdx.x == 0) tgmax[(int64_t)tok * ngroups + rg] = mx;
+        if (threadIdx.x == 0) L.counters[rb] = 0;
+        __syncthreads();
     }
-    if (threadIdx.x == 0) counters[rg] = 0;
+    // t and the block's max |t| per token (one warp per token)
+    for (int tok = warp; tok < batch; tok += kWarps) {
+        const float a = sm.res[tok][lane], b = sm.res[tok][lane + 32];
+        L.t[(int64_t)tok * r + row0 + lane] = a;
+        L.t[(int64_t)tok * r + row0 + lane + 32] = b;
+        const float v = warp_max(fmaxf(fabsf(a), fabsf(b)));
+        if (lane == 0) L.tgmax[(int64_t)tok * nrb + rb] = v;
+    }
 }
 
 // ------------------------------------------------------------------ stage 2
-// CTA = RT row tiles x KS k-parts (RT * KS = 8 warps), rows [RT*16*blockIdx.x, +RT*16).
-// One quantisation exponent per token for the whole of t (from the row-group maxima of
-// stage 1), so integer sums run across all chunks and k-parts and are converted once.
-template <int NTG, int RT>
-__global__ void __launch_bounds__(kThreads) stage2_kernel(const float* __restrict__ t,
-                                                          const float* __restrict__ tgmax,
-                                                          const uint32_t* __restrict__ Upk,
-                                                          const uint16_t* __restrict__ s1, int64_t m, int64_t r,
-                                                          int batch, float* __restrict__ y) {
-    constexpr int KS = kWarps / RT;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    Stage2Smem& sm = *reinterpret_cast<Stage2Smem*>(smem_raw);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-    const int rt = warp / KS, kp = warp % KS;
-    const int64_t wpr = r / 32;
-    const int64_t rowc = (int64_t)blockIdx.x * RT * 16;
-    const int64_t row0 = rowc + 16 * rt;
-    const int ngroups = (int)(r / 128);
-    const int nchunks = (int)((r + kChunk - 1) / kChunk);
-
-    for (int i = threadIdx.x; i < 128 * 8; i += kThreads) (&sm.bq[0][0])[i] = 0;
-
-    pdl_wait();  // t and tgmax come from stage 1
-
-    if (threadIdx.x < 8) {
-        const int tok = threadIdx.x;
-        float mx = 0.f;
-        if (tok < batch)
-            for (int gi = 0; gi < ngroups; ++gi) mx = fmaxf(mx, tgmax[(int64_t)tok * ngroups + gi]);
-        sm.e[tok] = range_exponent(mx);
-        sm.qsum[tok] = 0;
-    }
-    __syncthreads();
-
-    int acc[NTG][4][4];
-#pragma unroll
-    for (int tg = 0; tg < NTG; ++tg)
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[tg][s][i] = 0;
-
-    for (int ch = 0; ch < nchunks; ++ch) {
-        const int64_t col0 = (int64_t)ch * kChunk;
-        const int ccols = (int)min((int64_t)kChunk, r - col0);
-        const int ncb = ccols / kCB;
-        for (int tok = 0; tok < batch; ++tok) {
-            const int e = sm.e[tok];
-            int qs = 0;
-            for (int c = threadIdx.x; c < ccols; c += kThreads) {
-                int q = quantise(t[(int64_t)tok * r + col0 + c], e);
-                sm.chunk.q[tok][c] = (int16_t)q;
-                qs += q;
-            }
-            for (int o = 16; o > 0; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
-            if (lane == 0) atomicAdd(&sm.qsum[tok], qs);
-        }
-        __syncthreads();
-        build_fragments(sm.chunk, ncb, batch, NTG);
-        __syncthreads();
-        if (row0 < m) tile_mma<NTG>(Upk + row0 * wpr + col0 / 32, wpr, sm.chunk, kp, ncb, KS, acc);
-        __syncthreads();
-    }
-    pdl_trigger();
-
-    if (row0 < m) {
-#pragma unroll
-        for (int tg = 0; tg < NTG; ++tg) {
-            const int tok = 4 * tg + tq;
-            if (tok < batch) {
-                int bq0, bq8;
-                combine<NTG>(acc, tg, bq0, bq8);
-                atomicAdd(&sm.bq[16 * rt + g][tok], bq0);
-                atomicAdd(&sm.bq[16 * rt + g + 8][tok], bq8);
-            }
-        }
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < RT * 16 * batch; idx += kThreads) {
-        const int tok = idx / (RT * 16), i = idx % (RT * 16);
-        const int64_t row = rowc + i;
-        if (row < m) {
-            const float v = scalbnf((float)(2 * (int64_t)sm.bq[i][tok] - sm.qsum[tok]), sm.e[tok] - kQBits);
-            y[(int64_t)tok * m + row] = f16_to_f32(s1[row]) * v;
-        }
+// CTA = RT row tiles x KS = 4/RT k-parts of one layer.  One quantisation exponent per
+// token for the whole of t (from stage 1's maxima), so integer sums run across all
+// chunks and k-parts and are converted once, in the epilogue.
+template <int NTG>
+__device__ __forceinline__ void stage2_fetch_t(DecSmem<NTG>& sm, int buf, const DecLayer& L, int batch, int col0,
+                                               int ccols) {
+    const int per_tok = ccols / 4;  // 16-byte pieces
+    for (int i = threadIdx.x; i < batch * per_tok; i += kThreads) {
+        const int tok = i / per_tok, p = i % per_tok;
+        cp_async16(&sm.act.t[buf][tok][4 * p], L.t + (int64_t)tok * L.r + col0 + 4 * p);
     }
 }
-
-template <typename K>
-cudaError_t set_smem(K kernel, size_t bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-}
-
-}  // namespace
-
-// Column split of stage 1: about two CTAs per SM over the r/128 row groups; returns the
-// number of column blocks per split (cps) and the split count.
-void decode_split(int64_t n, int64_t r, int* nsplit, int* cps) {
-    const int64_t ncb = n / kCB;
-    const int64_t groups = r / 128;
-    int64_t want = (2 * (int64_t)sm_count() + groups - 1) / groups;
-    if (want > 64) want = 64;
-    if (want > ncb) want = ncb;
-    if (want < 1) want = 1;
-    int64_t c = (ncb + want - 1) / want;
-    *cps = (int)c;
-    *nsplit = (int)((ncb + c - 1) / c);
-}
-
-namespace {
 
 template <int NTG>
-int decode_launch(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const uint16_t* s1,
-                  const uint16_t* s2, int64_t m, int64_t n, int64_t r, int batch, float* y, Workspace* ws,
-                  cudaStream_t stream) {
+__global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant__ DecGroup grp) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    DecSmem<NTG>& sm = *reinterpret_cast<DecSmem<NTG>*>(smem_raw);
+    const int li = find_layer(grp.s2_start, grp.count, blockIdx.x);
+    const DecLayer& L = grp.L[li];
+    const int blk = blockIdx.x - grp.s2_start[li];
+    const int batch = grp.batch;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    const int RT = L.rt, KS = kWarps / RT;
+    const int rt = warp / KS, kp = warp % KS;
+    const int m = L.m, r = L.r;
+    const int64_t wpr = r / 32;
+    const int rows = 16 * RT;
+    const int64_t row0 = (int64_t)blk * rows;
+    const uint32_t* W = L.Upk + row0 * wpr;
+    const int nchunks = (r + kChunk - 1) / kChunk;
+    auto chunk_cols = [&](int ch) { return min(kChunk, r - ch * kChunk); };
+
+    stage_weights(sm, 0, W, wpr, rows, 0, chunk_cols(0) / 32);
+    cp_async_commit();
+    if (nchunks > 1) stage_weights(sm, 1, W, wpr, rows, kChunkWords, chunk_cols(1) / 32);
+    cp_async_commit();
+    if (nchunks > 2 && threadIdx.x < rows)
+        prefetch_l2(W + threadIdx.x * wpr + 2 * kChunkWords, (uint32_t)((r - 2 * kChunk) / 8));
+    for (int i = threadIdx.x; i < 64 * 8; i += kThreads) (&sm.bq[0][0])[i] = 0;
+    zero_fragments(sm);
+    pdl_trigger();
+    pdl_wait();  // t and its maxima come from stage 1
+    stage2_fetch_t(sm, 0, L, batch, 0, chunk_cols(0));
+    cp_async_commit();
+    if (nchunks > 1) stage2_fetch_t(sm, 1, L, batch, kChunk, chunk_cols(1));
+    cp_async_commit();
+
+    // global max |t| per token from the per-block maxima (one warp per token)
+    const int nrb = r / kRowsS1;
+    for (int tok = warp; tok < batch; tok += kWarps) {
+        float mx = 0.f;
+        for (int gi = lane; gi < nrb; gi += 32) mx = fmaxf(mx, L.tgmax[(int64_t)tok * nrb + gi]);
+        mx = warp_max(mx);
+        if (lane == 0) {
+            const int e = range_exponent(mx);
+            sm.e[tok] = e;
+            sm.up[tok] = pow2f(kQBits - e);
+            sm.qsum[tok] = 0;
+        }
+    }
+
+    int acc[NTG][4][4];
+    zero_acc<NTG>(acc);
+    for (int ch = 0; ch < nchunks; ++ch) {
+        const int buf = ch & 1;
+        const int ccols = chunk_cols(ch);
+        const int ncb = ccols / kCB;
+        if (ch + 1 < nchunks) cp_async_wait<1>(); else cp_async_wait<0>();
+        __syncthreads();
+        const float* ts = &sm.act.t[buf][0][0];
+        build_fragments(sm, ncb, batch, [&](int tok, int c) { return ts[tok * kChunk + c]; });
+        __syncthreads();
+        tile_mma<NTG>(sm, buf, 16 * rt, kp, ncb, KS, acc);
+        __syncthreads();
+        if (ch + 2 < nchunks) {
+            stage_weights(sm, buf, W, wpr, rows, (int64_t)(ch + 2) * kChunkWords, chunk_cols(ch + 2) / 32);
+            stage2_fetch_t(sm, buf, L, batch, (ch + 2) * kChunk, chunk_cols(ch + 2));
+            cp_async_commit();
+        }
+    }
+
+#pragma unroll
+    for (int tg = 0; tg < NTG; ++tg) {
+        const int tok = 4 * tg + tq;
+        if (tok < batch) {
+            int bq0, bq8;
+            combine<NTG>(acc, tg, bq0, bq8);
+            atomicAdd(&sm.bq[16 * rt + g][tok], bq0);
+            atomicAdd(&sm.bq[16 * rt + g + 8][tok], bq8);
+        }
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < rows * batch; idx += kThreads) {
+        const int tok = idx / rows, i = idx % rows;
+        const int64_t row = row0 + i;
+        const float v = (float)(2 * (int64_t)sm.bq[i][tok] - sm.qsum[tok]) * pow2f(sm.e[tok] - kQBits);
+        L.y[(int64_t)tok * m + row] = f16_to_f32(L.s1[row]) * v;
+    }
+}
+
+template <int NTG>
+int launch_group(DecGroup& grp, cudaStream_t stream, int device) {
     static unsigned long long init_mask = 0;  // devices whose kernel attributes are set
-    const size_t smem1 = sizeof(Stage1Smem), smem2 = sizeof(Stage2Smem);
-    const unsigned long long bit = 1ull << (ws->device & 63);
+    const unsigned long long bit = 1ull << (device & 63);
+    const size_t smem = sizeof(DecSmem<NTG>);
     if (!(__atomic_load_n(&init_mask, __ATOMIC_ACQUIRE) & bit)) {
-        if (set_smem(stage1_kernel<NTG>, smem1) != cudaSuccess || set_smem(stage2_kernel<NTG, 1>, smem2) != cudaSuccess ||
-            set_smem(stage2_kernel<NTG, 2>, smem2) != cudaSuccess || set_smem(stage2_kernel<NTG, 4>, smem2) != cudaSuccess)
+        if (cudaFuncSetAttribute(stage1_kernel<NTG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(stage2_kernel<NTG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+                cudaSuccess)
             return NQ_ERR_CUDA;
         __atomic_fetch_or(&init_mask, bit, __ATOMIC_RELEASE);
     }
-    int nsplit = 1, cps = 1;
-    decode_split(n, r, &nsplit, &cps);
-    dim3 grid1((unsigned)(r / 128), (unsigned)nsplit);
-    cudaError_t err = launch_pdl(stage1_kernel<NTG>, grid1, dim3(kThreads), smem1, stream, x, Vpk, s2, n, r, batch,
-                                 nsplit, cps, ws->t, ws->tgmax, ws->partials, ws->counters);
-    if (err != cudaSuccess) return NQ_ERR_CUDA;
-    // stage 2: fewer rows (more k-parts) per CTA when m is small
-    const int64_t tiles = m / 16, sms = sm_count();
-    const int rt = tiles >= 8 * sms ? 4 : (tiles >= 2 * sms ? 2 : 1);
-    dim3 grid2((unsigned)((m + 16 * rt - 1) / (16 * rt)));
-    const float* t = ws->t;
-    const float* tgmax = ws->tgmax;
-    if (rt == 1)
-        err = launch_pdl(stage2_kernel<NTG, 1>, grid2, dim3(kThreads), smem2, stream, t, tgmax, Upk, s1, m, r, batch, y);
-    else if (rt == 2)
-        err = launch_pdl(stage2_kernel<NTG, 2>, grid2, dim3(kThreads), smem2, stream, t, tgmax, Upk, s1, m, r, batch, y);
-    else
-        err = launch_pdl(stage2_kernel<NTG, 4>, grid2, dim3(kThreads), smem2, stream, t, tgmax, Upk, s1, m, r, batch, y);
-    return err == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
+    if (launch_pdl(stage1_kernel<NTG>, dim3((unsigned)grp.s1_start[grp.count]), dim3(kThreads), smem, stream, grp) !=
+        cudaSuccess)
+        return NQ_ERR_CUDA;
+    if (launch_pdl(stage2_kernel<NTG>, dim3((unsigned)grp.s2_start[grp.count]), dim3(kThreads), smem, stream, grp) !=
+        cudaSuccess)
+        return NQ_ERR_CUDA;
+    return NQ_OK;
 }
 
 }  // namespace
+
+// Stage-2 row tiles per CTA: fewer rows (more k-parts) when the launch has few rows.
+static int stage2_rt(int64_t total_tiles) {
+    const int64_t sms = sm_count();
+    return total_tiles >= 12 * sms ? 4 : (total_tiles >= 4 * sms ? 2 : 1);
+}
+
+// Column blocks per stage-1 split: about two CTAs per SM over the whole launch, at least
+// 4 and (while the split count stays <= 64) at most 16 column blocks per CTA.
+static int stage1_cps(const DecodeCall* calls, int count) {
+    int64_t units = 0, max_ncb = 0;
+    for (int i = 0; i < count; ++i) {
+        units += (calls[i].r / kRowsS1) * (calls[i].n / kCB);
+        max_ncb = calls[i].n / kCB > max_ncb ? calls[i].n / kCB : max_ncb;
+    }
+    const int64_t target = 2 * (int64_t)sm_count();
+    int64_t cps = (units + target - 1) / target;
+    if (cps < 4) cps = 4;
+    if (cps > kChunkCB) cps = kChunkCB;
+    if ((max_ncb + cps - 1) / cps > 64) cps = (max_ncb + 63) / 64;
+    return (int)cps;
+}
+
+void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, int64_t* t_floats,
+                           int64_t* tgmax_floats, int64_t* partial_floats, int64_t* counter_ints) {
+    const int cps = stage1_cps(calls, count);
+    int64_t t = 0, gm = 0, pf = 0, ci = 0;
+    for (int i = 0; i < count; ++i) {
+        const int64_t ncb = calls[i].n / kCB, nsplit = (ncb + cps - 1) / cps;
+        t += batch * calls[i].r;
+        gm += batch * (calls[i].r / kRowsS1);
+        if (nsplit > 1) pf += nsplit * batch * calls[i].r;
+        ci += calls[i].r / kRowsS1;
+    }
+    *t_floats = t;
+    *tgmax_floats = gm;
+    *partial_floats = pf;
+    *counter_ints = ci;
+}
+
+int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Workspace* ws, cudaStream_t stream) {
+    if (count < 1 || count > kMaxGroup) return NQ_ERR_SHAPE;
+    int64_t need_t, need_g, need_p, need_c;
+    decode_workspace_need(calls, count, batch, &need_t, &need_g, &need_p, &need_c);
+    if ((size_t)need_t > ws->t_cap || (size_t)need_g > ws->tgmax_cap || (size_t)need_p > ws->partial_cap ||
+        (size_t)need_c > ws->counter_cap)
+        return NQ_ERR_NOMEM;
+    DecGroup grp;
+    grp.count = count;
+    grp.batch = (int)batch;
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) tiles += calls[i].m / 16;
+    const int rt = stage2_rt(tiles);
+    const int cps = stage1_cps(calls, count);
+    size_t toff = 0, goff = 0, poff = 0, coff = 0;
+    grp.s1_start[0] = grp.s2_start[0] = 0;
+    for (int i = 0; i < count; ++i) {
+        const DecodeCall& c = calls[i];
+        DecLayer& L = grp.L[i];
+        L.x = c.x;
+        L.Upk = c.Upk;
+        L.Vpk = c.Vpk;
+        L.s1 = c.s1;
+        L.s2 = c.s2;
+        L.y = c.y;
+        L.m = (int)c.m;
+        L.n = (int)c.n;
+        L.r = (int)c.r;
+        L.rt = rt;
+        L.cps = cps;
+        L.nsplit = (int)((c.n / kCB + cps - 1) / cps);
+        L.t = ws->t + toff;
+        L.tgmax = ws->tgmax + goff;
+        L.partials = ws->partials + poff;
+        L.counters = ws->counters + coff;
+        toff += (size_t)batch * c.r;
+        goff += (size_t)batch * (c.r / kRowsS1);
+        if (L.nsplit > 1) poff += (size_t)L.nsplit * batch * c.r;
+        coff += (size_t)(c.r / kRowsS1);
+        grp.s1_start[i + 1] = grp.s1_start[i] + (int)(c.r / kRowsS1) * L.nsplit;
+        grp.s2_start[i + 1] = grp.s2_start[i] + (int)(c.m / (16 * rt));
+    }
+    if (batch <= 4) return launch_group<1>(grp, stream, ws->device);
+    return launch_group<2>(grp, stream, ws->device);
+}
 
 int decode_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const uint16_t* s1,
                    const uint16_t* s2, int64_t m, int64_t n, int64_t r, int64_t batch, float* y,
                    Workspace* ws, cudaStream_t stream) {
-    if (batch <= 4) return decode_launch<1>(x, Upk, Vpk, s1, s2, m, n, r, (int)batch, y, ws, stream);
-    return decode_launch<2>(x, Upk, Vpk, s1, s2, m, n, r, (int)batch, y, ws, stream);
+    DecodeCall c{x, Upk, Vpk, s1, s2, y, m, n, r};
+    return decode_forward_group(&c, 1, batch, ws, stream);
 }
 
 }  // namespace nq

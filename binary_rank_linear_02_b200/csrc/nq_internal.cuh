@@ -8,31 +8,51 @@
 
 namespace nq {
 
+constexpr int kMaxGroup = 16;  // layers per decode launch
+
 // ---------------------------------------------------------------- workspace
-// One per device.  Decode keeps t (batch x r fp32), the split partials of stage 1 and a
-// per-row-group arrival counter; prefill keeps x' (batch x n fp16) and T (batch x r
-// fp16); host-memory x / y are staged through xstage / ystage.
+// One per device.  Decode keeps t (batch x r fp32 per layer) and the max |t| of each
+// 64-row block; prefill keeps x' (batch x n fp16) and T (batch x r fp16); host-memory
+// x / y are staged through xstage / ystage.
 struct Workspace {
     int device = -1;
     size_t bytes = 0;
     char* base = nullptr;
     // carved regions
-    float* t = nullptr;            // [8][r_cap] (decode)
-    float* tgmax = nullptr;        // [8][r_cap/128] max |t| per 128-row group (decode)
-    float* partials = nullptr;     // [split_cap][8][r_cap]
-    int* counters = nullptr;       // [r_cap/128], zero between calls
-    unsigned* status = nullptr;    // device status word(s)
+    float* t = nullptr;            // [t_cap] (decode: sum over a launch's layers of batch x r)
+    float* tgmax = nullptr;        // [tgmax_cap] (decode: batch x r/64 per layer)
+    float* partials = nullptr;     // [partial_cap] (decode: stage-1 column-split partial sums)
+    int* counters = nullptr;       // [counter_cap] (decode: arrival counters, zero between calls)
+    unsigned* status = nullptr;    // [0]: pack value check, [1]: device wait timeout
     uint16_t* xprime = nullptr;    // [batch_cap][n_cap] fp16 (prefill)
     uint16_t* T = nullptr;         // [batch_cap][r_cap] fp16 (prefill)
     void* xstage = nullptr;        // staged host x
     float* ystage = nullptr;       // staged host y
     size_t xstage_bytes = 0, ystage_bytes = 0;
-    int64_t r_cap = 0, n_cap = 0, m_cap = 0, batch_cap = 0, split_cap = 0;
+    size_t t_cap = 0, tgmax_cap = 0, partial_cap = 0, counter_cap = 0;
+    int64_t r_cap = 0, n_cap = 0, m_cap = 0, batch_cap = 0, rsum_cap = 0;
 };
 
-// Returns the current device's workspace, grown to fit (m, n, r, batch).  nullptr on
-// allocation failure (status set to NQ_ERR_NOMEM / NQ_ERR_CUDA).
-Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, int* status);
+// What a decode launch needs from the workspace, in elements.
+struct DecodeNeed {
+    int64_t t = 0, tgmax = 0, partials = 0, counters = 0;
+};
+
+// Returns the current device's workspace, grown to fit a prefill layer of at most
+// (m, n, r) and `batch` tokens and a decode launch needing `dec`.  nullptr on failure
+// (status set to NQ_ERR_NOMEM / NQ_ERR_CUDA).
+Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, const DecodeNeed& dec, int* status);
+
+// One factorised layer of a decode launch.
+struct DecodeCall {
+    const uint16_t* x;
+    const uint32_t* Upk;
+    const uint32_t* Vpk;
+    const uint16_t* s1;
+    const uint16_t* s2;
+    float* y;
+    int64_t m, n, r;
+};
 
 int sm_count();
 
@@ -60,6 +80,10 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------- entry points of the kernels
+int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Workspace* ws, cudaStream_t stream);
+void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, int64_t* t_floats,
+                           int64_t* tgmax_floats, int64_t* partial_floats, int64_t* counter_ints);
+
 int decode_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const uint16_t* s1,
                    const uint16_t* s2, int64_t m, int64_t n, int64_t r, int64_t batch, float* y,
                    Workspace* ws, cudaStream_t stream);

@@ -33,6 +33,14 @@ NQ_ERR_PTRKIND = -9
 NQ_DECODE_MAX_BATCH = 8
 
 
+class nq_linear_desc(ctypes.Structure):
+    """One layer of nq_lowrank_linear_fwd_grouped (see include/nq.h)."""
+
+    _fields_ = [("x", ctypes.c_void_p), ("Upk", ctypes.c_void_p), ("Vpk", ctypes.c_void_p),
+                ("s1", ctypes.c_void_p), ("s2", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("m", ctypes.c_int64), ("n", ctypes.c_int64), ("r", ctypes.c_int64)]
+
+
 class NQError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -59,6 +67,10 @@ def _load() -> ctypes.CDLL:
     L.nq_workspace_reserve.argtypes = [i64, i64, i64, i64]
     L.nq_workspace_reserve.restype = ctypes.c_int
     L.nq_version.restype = ctypes.c_int
+    L.nq_lowrank_linear_fwd_grouped.argtypes = [p, ctypes.c_int, i64, p]
+    L.nq_lowrank_linear_fwd_grouped.restype = ctypes.c_int
+    L.nq_device_status.argtypes = [p]
+    L.nq_device_status.restype = ctypes.c_int
     return L
 
 
@@ -83,6 +95,10 @@ def nq_lowrank_linear_fwd(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n, r, batc
     return _lib.nq_lowrank_linear_fwd(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n, r, batch, y_ptr, stream)
 
 
+def nq_lowrank_linear_fwd_grouped(descs_ptr, count, batch, stream=0) -> int:
+    return _lib.nq_lowrank_linear_fwd_grouped(descs_ptr, count, batch, stream)
+
+
 def nq_bits_per_weight(m: int, n: int, r: int) -> float:
     return _lib.nq_bits_per_weight(m, n, r)
 
@@ -93,6 +109,18 @@ def nq_status_string(status: int) -> str:
 
 def nq_workspace_reserve(m: int, n: int, r: int, batch: int) -> int:
     return _lib.nq_workspace_reserve(m, n, r, batch)
+
+
+def nq_device_status(stream: int = 0) -> int:
+    return _lib.nq_device_status(stream)
+
+
+def device_status(stream=None) -> None:
+    """Synchronise and raise NQError if a kernel recorded a timed-out device wait."""
+    import torch
+
+    h = int(stream) if stream is not None else torch.cuda.current_stream().cuda_stream
+    _check(_lib.nq_device_status(h), "nq_device_status")
 
 
 def nq_version() -> int:
@@ -172,6 +200,22 @@ def lowrank_linear_fwd(x, Upk, Vpk, s1, s2, m: int, n: int, r: int, y=None, stre
                                     _ptr(y), _stream(stream, x, Upk, y))
     _check(st, "nq_lowrank_linear_fwd")
     return y
+
+
+def make_descs(layers):
+    """ctypes array of nq_linear_desc from (x, Upk, Vpk, s1, s2, y, m, n, r) tuples."""
+    arr = (nq_linear_desc * len(layers))()
+    for i, (x, Upk, Vpk, s1, s2, y, m, n, r) in enumerate(layers):
+        arr[i] = nq_linear_desc(_ptr(x), _ptr(Upk), _ptr(Vpk), _ptr(s1), _ptr(s2), _ptr(y), m, n, r)
+    return arr
+
+
+def lowrank_linear_fwd_grouped(layers, batch: int, stream=None):
+    """Run independent layers [(x, Upk, Vpk, s1, s2, y, m, n, r), ...] in one grouped call."""
+    arr = make_descs(layers)
+    h = _stream(stream, *(l[0] for l in layers))
+    _check(_lib.nq_lowrank_linear_fwd_grouped(ctypes.addressof(arr), len(layers), batch, h),
+           "nq_lowrank_linear_fwd_grouped")
 
 
 def bits_per_weight(m: int, n: int, r: int) -> float:

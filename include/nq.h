@@ -106,6 +106,29 @@ int nq_lowrank_linear_fwd(const void* x, const uint32_t* Upk, const uint32_t* Vp
                           const void* s1, const void* s2, int64_t m, int64_t n, int64_t r,
                           int64_t batch, float* y, void* stream);
 
+/* One factorised layer of a grouped call (same meaning and rules as the arguments of
+ * nq_lowrank_linear_fwd; every pointer in device memory, 16-byte aligned). */
+typedef struct nq_linear_desc {
+    const void* x;          /* batch x n bfloat16 */
+    const uint32_t* Upk;    /* m x (r/32) */
+    const uint32_t* Vpk;    /* r x (n/32) */
+    const void* s1;         /* m fp16 */
+    const void* s2;         /* n fp16 */
+    float* y;               /* batch x m float32 (written) */
+    int64_t m, n, r;
+} nq_linear_desc;
+
+/*
+ * nq_lowrank_linear_fwd_grouped -- `count` independent factorised layers with the same
+ * batch, e.g. the projections of one transformer block that read the same or different
+ * activations.  The result of every layer equals nq_lowrank_linear_fwd on it; the
+ * decode path (batch <= NQ_DECODE_MAX_BATCH) runs up to 16 layers per launch pair, so
+ * small layers share the launch and dependency latency.  No layer's y may overlap
+ * another layer's inputs.  Argument checks as nq_lowrank_linear_fwd, plus count >= 0
+ * (0 is a no-op) and `layers` non-NULL; host-memory buffers are refused (NQ_ERR_PTRKIND).
+ */
+int nq_lowrank_linear_fwd_grouped(const nq_linear_desc* layers, int count, int64_t batch, void* stream);
+
 /*
  * nq_bits_per_weight -- storage cost of the factorised layer in bits per weight of the
  * dense m x n matrix it replaces: (r*(m+n) + 16*(m+n)) / (m*n)  (hardwired.dev sections
@@ -121,6 +144,13 @@ const char* nq_status_string(int status);
  * later calls with these or smaller sizes allocate nothing.  Synchronises the device.
  */
 int nq_workspace_reserve(int64_t m, int64_t n, int64_t r, int64_t batch);
+
+/*
+ * nq_device_status -- synchronise `stream`, then read and clear the current device's
+ * status word, in which kernels record a bounded device-side wait that gave up.
+ * Returns NQ_OK, NQ_ERR_TIMEOUT, or NQ_ERR_CUDA if the synchronisation itself failed.
+ */
+int nq_device_status(void* stream);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int nq_version(void);

@@ -101,3 +101,28 @@ def test_forward_argument_errors(nq):
     assert f(p[0], p[1], p[2], p[3], p[4], 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_PTRKIND
     assert nq.nq_workspace_reserve(128, 100, 128, 1) == nq.NQ_ERR_SHAPE
     assert nq.nq_workspace_reserve(128, 128, 128, -2) == nq.NQ_ERR_BATCH
+
+
+def test_grouped_argument_errors(nq):
+    buf = np.zeros(1 << 16, dtype=np.uint8)
+    base = (buf.ctypes.data + 255) // 256 * 256
+    ptr = [base + 1024 * i for i in range(6)]
+    good = nq.nq_linear_desc(ptr[0], ptr[1], ptr[2], ptr[3], ptr[4], ptr[5], 128, 128, 128)
+    arr = (nq.nq_linear_desc * 2)(good, good)
+    f = nq.nq_lowrank_linear_fwd_grouped
+    a = ctypes.addressof(arr)
+    assert f(a, 2, -1, 0) == nq.NQ_ERR_BATCH
+    assert f(a, -1, 1, 0) == nq.NQ_ERR_SHAPE
+    assert f(a, 0, 1, 0) == nq.NQ_OK
+    assert f(a, 2, 0, 0) == nq.NQ_OK
+    assert f(0, 2, 1, 0) == nq.NQ_ERR_NULL
+    arr[1].n = 96
+    assert f(a, 2, 1, 0) == nq.NQ_ERR_SHAPE
+    arr[1].n = 128
+    arr[1].Vpk = ptr[2] + 4
+    assert f(a, 2, 1, 0) == nq.NQ_ERR_ALIGN
+    arr[1].Vpk = ptr[2]
+    arr[0].s1 = 0
+    assert f(a, 2, 1, 0) == nq.NQ_ERR_NULL
+    arr[0].s1 = ptr[3]
+    assert f(a, 2, 1, 0) == nq.NQ_ERR_PTRKIND  # host memory is refused

@@ -195,3 +195,65 @@ def test_forward_prefill_sweep_sampled(nq, orc, batch):
     rng = np.random.default_rng(batch)
     rows = np.unique(np.concatenate([[0, batch - 1], rng.choice(batch, size=min(batch, 14), replace=False)]))
     assert rel_err(y[rows], c.oracle(orc, rows)) <= TOL
+
+
+# ------------------------------------------------------------------ tensor-core prefill tiles
+
+@pytest.mark.parametrize("m,n,r,batch", [
+    (128, 128, 128, 9),       # one M tile, one N tile of 64, ragged
+    (256, 384, 256, 64),      # exact N tile of 64
+    (384, 256, 384, 65),      # N tile of 128, ragged
+    (256, 512, 128, 300),     # three N tiles of 128, ragged tail
+    (128, 256, 256, 1025),    # N tiles of 256, one token in the last
+    (1408, 640, 896, 517),    # several M tiles in both GEMMs
+])
+def test_prefill_tiles(nq, orc, m, n, r, batch):
+    c = Case(orc, nq, m, n, r, batch, seed=m * 7 + batch)
+    y = c.gpu()
+    nq.device_status()
+    assert rel_err(y, c.oracle(orc)) <= TOL
+
+
+def test_prefill_deterministic_and_status(nq, orc):
+    c = Case(orc, nq, 512, 1024, 384, 200, seed=3)
+    a, b = c.gpu(), c.gpu()
+    nq.device_status()
+    assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------------ grouped calls
+
+@pytest.mark.parametrize("batch", [1, 3, 8, 20])
+def test_grouped_matches_single_calls(nq, orc, batch):
+    shapes = [(512, 512, 128), (384, 640, 256), (1024, 256, 384), (256, 2176, 128)]
+    cases = [Case(orc, nq, m, n, r, batch, seed=900 + i) for i, (m, n, r) in enumerate(shapes)]
+    ys = [torch.empty((batch, c.m), dtype=torch.float32, device="cuda") for c in cases]
+    nq.lowrank_linear_fwd_grouped([(c.x_d, c.Upk, c.Vpk, c.s1_d, c.s2_d, y, c.m, c.n, c.r)
+                                   for c, y in zip(cases, ys)], batch)
+    torch.cuda.synchronize()
+    for c, y in zip(cases, ys):
+        single = c.gpu()
+        assert np.array_equal(y.cpu().numpy(), single)
+        assert rel_err(single, c.oracle(orc)) <= TOL
+
+
+def test_grouped_more_than_one_launch(nq, orc):
+    batch = 2
+    cases = [Case(orc, nq, 256, 256, 128, batch, seed=950 + i) for i in range(19)]
+    ys = [torch.empty((batch, 256), dtype=torch.float32, device="cuda") for _ in cases]
+    nq.lowrank_linear_fwd_grouped([(c.x_d, c.Upk, c.Vpk, c.s1_d, c.s2_d, y, c.m, c.n, c.r)
+                                   for c, y in zip(cases, ys)], batch)
+    torch.cuda.synchronize()
+    for c, y in zip(cases, ys):
+        assert rel_err(y.cpu().numpy(), c.oracle(orc)) <= TOL
+
+
+def test_grouped_llama2_7b_block(nq, orc):
+    batch = 1
+    cases = [Case(orc, nq, m, n, r, batch, seed=960 + i) for i, (_, m, n, r) in enumerate(synth.LLAMA2_7B_LAYERS)]
+    ys = [torch.empty((batch, c.m), dtype=torch.float32, device="cuda") for c in cases]
+    nq.lowrank_linear_fwd_grouped([(c.x_d, c.Upk, c.Vpk, c.s1_d, c.s2_d, y, c.m, c.n, c.r)
+                                   for c, y in zip(cases, ys)], batch)
+    torch.cuda.synchronize()
+    for c, y in zip(cases, ys):
+        assert rel_err(y.cpu().numpy(), c.oracle(orc)) <= TOL
