@@ -125,7 +125,7 @@ Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, const D
 DecodeNeed decode_need(const DecodeCall* calls, int count, int64_t batch) {
     DecodeNeed d;
     if (batch >= 1 && batch <= NQ_DECODE_MAX_BATCH)
-        decode_workspace_need(calls, count, batch, &d.t, &d.tgmax, &d.partials, &d.counters);
+        decode_workspace_need(calls, count, batch, kDecodeMaxSplits, &d.t, &d.tgmax, &d.partials, &d.counters);
     return d;
 }
 
@@ -167,6 +167,9 @@ const char* nq_status_string(int status) {
         case NQ_ERR_TIMEOUT: return "NQ_ERR_TIMEOUT: a bounded device-side wait gave up";
         case NQ_ERR_NOMEM: return "NQ_ERR_NOMEM: workspace allocation failed (or was needed during stream capture)";
         case NQ_ERR_PTRKIND: return "NQ_ERR_PTRKIND: pointers of mixed or unsupported memory kinds";
+        case NQ_ERR_NOALLOC_LIMIT:
+            return "NQ_ERR_NOALLOC_LIMIT: nq_lowrank_linear_fwd_noalloc takes 1 <= batch <= 8 and r <= 4096 "
+                   "(its scratch is a fixed array)";
         default: return "unknown nq status";
     }
 }

@@ -38,6 +38,8 @@
 #include <cuda_fp16.h>
 #include <math.h>
 
+#include <mutex>
+
 #include "nq_internal.cuh"
 
 namespace nq {
@@ -556,8 +558,8 @@ static int stage2_rt(int64_t total_tiles) {
 }
 
 // Column blocks per stage-1 split: about two CTAs per SM over the whole launch, at least
-// 4 and (while the split count stays <= 64) at most 16 column blocks per CTA.
-static int stage1_cps(const DecodeCall* calls, int count) {
+// 4 and (while the split count stays <= max_splits) at most kChunkCB column blocks per CTA.
+static int stage1_cps(const DecodeCall* calls, int count, int max_splits) {
     int64_t units = 0, max_ncb = 0;
     for (int i = 0; i < count; ++i) {
         units += (calls[i].r / kRowsS1) * (calls[i].n / kCB);
@@ -567,13 +569,13 @@ static int stage1_cps(const DecodeCall* calls, int count) {
     int64_t cps = (units + target - 1) / target;
     if (cps < 4) cps = 4;
     if (cps > kChunkCB) cps = kChunkCB;
-    if ((max_ncb + cps - 1) / cps > 64) cps = (max_ncb + 63) / 64;
+    if ((max_ncb + cps - 1) / cps > max_splits) cps = (max_ncb + max_splits - 1) / max_splits;
     return (int)cps;
 }
 
-void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, int64_t* t_floats,
+void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, int max_splits, int64_t* t_floats,
                            int64_t* tgmax_floats, int64_t* partial_floats, int64_t* counter_ints) {
-    const int cps = stage1_cps(calls, count);
+    const int cps = stage1_cps(calls, count, max_splits);
     int64_t t = 0, gm = 0, pf = 0, ci = 0;
     for (int i = 0; i < count; ++i) {
         const int64_t ncb = calls[i].n / kCB, nsplit = (ncb + cps - 1) / cps;
@@ -588,10 +590,11 @@ void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, in
     *counter_ints = ci;
 }
 
-int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Workspace* ws, cudaStream_t stream) {
+int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Workspace* ws, cudaStream_t stream,
+                         int max_splits) {
     if (count < 1 || count > kMaxGroup) return NQ_ERR_SHAPE;
     int64_t need_t, need_g, need_p, need_c;
-    decode_workspace_need(calls, count, batch, &need_t, &need_g, &need_p, &need_c);
+    decode_workspace_need(calls, count, batch, max_splits, &need_t, &need_g, &need_p, &need_c);
     if ((size_t)need_t > ws->t_cap || (size_t)need_g > ws->tgmax_cap || (size_t)need_p > ws->partial_cap ||
         (size_t)need_c > ws->counter_cap)
         return NQ_ERR_NOMEM;
@@ -601,7 +604,7 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
     int64_t tiles = 0;
     for (int i = 0; i < count; ++i) tiles += calls[i].m / 16;
     const int rt = stage2_rt(tiles);
-    const int cps = stage1_cps(calls, count);
+    const int cps = stage1_cps(calls, count, max_splits);
     size_t toff = 0, goff = 0, poff = 0, coff = 0;
     grp.s1_start[0] = grp.s2_start[0] = 0;
     for (int i = 0; i < count; ++i) {
@@ -638,7 +641,118 @@ int decode_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, 
                    const uint16_t* s2, int64_t m, int64_t n, int64_t r, int64_t batch, float* y,
                    Workspace* ws, cudaStream_t stream) {
     DecodeCall c{x, Upk, Vpk, s1, s2, y, m, n, r};
-    return decode_forward_group(&c, 1, batch, ws, stream);
+    return decode_forward_group(&c, 1, batch, ws, stream, kDecodeMaxSplits);
 }
 
 }  // namespace nq
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free decode entry point.
+//
+// Some callers cannot allocate device memory at the moment they run a layer: an inference
+// engine that sized and froze its memory pool at start-up, a process whose allocator is
+// owned by another framework, or code running under a stream capture that must not call
+// cudaMalloc.  For them nq_lowrank_linear_fwd_noalloc keeps the decode path's scratch
+// (t, per-block maxima, stage-1 split partials, arrival counters) in one fixed array of
+// device memory that is part of this library's module, so a call allocates nothing.
+//
+// The array is a file-scope __device__ variable: every GPU that loads the library holds
+// it until the process exits.  Host code may not use its name as an address (on the host
+// the name is a stand-in, not device memory), so the first call on each device resolves
+// the device address with cudaGetSymbolAddress, with that device current, and caches it.
+// All calls share the one array: calls whose kernels overlap on the GPU (different
+// streams, or different host threads on one device) race and must be serialised by the
+// caller.  The arrival counters must start at zero; each call clears them on its stream
+// before its kernels run.
+namespace nq {
+namespace {
+
+constexpr int64_t kNoAllocMaxRank = 4096;   // largest r
+constexpr int kNoAllocMaxSplits = 8;        // stage-1 column splits
+constexpr size_t kNoAllocT = (size_t)NQ_DECODE_MAX_BATCH * kNoAllocMaxRank;
+constexpr size_t kNoAllocG = (size_t)NQ_DECODE_MAX_BATCH * (kNoAllocMaxRank / kRowsS1);
+constexpr size_t kNoAllocP = (size_t)kNoAllocMaxSplits * NQ_DECODE_MAX_BATCH * kNoAllocMaxRank;
+constexpr size_t kNoAllocC = kNoAllocMaxRank / kRowsS1;
+constexpr size_t kNoAllocBytes = 4 * (kNoAllocT + kNoAllocG + kNoAllocP + kNoAllocC);  // 1.16 MB
+
+}  // namespace
+}  // namespace nq
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[nq::kNoAllocBytes];
+
+namespace nq {
+namespace {
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[64];  // device address of g_noalloc_scratch, per device
+
+int noalloc_scratch(int dev, void** out) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return NQ_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return NQ_OK;
+}
+
+bool is_device_memory(const void* p) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+}
+
+}  // namespace
+}  // namespace nq
+
+extern "C" int nq_lowrank_linear_fwd_noalloc(const void* x, const uint32_t* Upk, const uint32_t* Vpk, const void* s1,
+                                             const void* s2, int64_t m, int64_t n, int64_t r, int64_t batch, float* y,
+                                             void* stream) {
+    using namespace nq;
+    if (batch < 0) return NQ_ERR_BATCH;
+    if (m <= 0 || n <= 0 || r <= 0 || m % 128 || n % 128 || r % 128 || m > (int64_t(1) << 20) ||
+        n > (int64_t(1) << 20))
+        return NQ_ERR_SHAPE;
+    if (r > kNoAllocMaxRank || batch > NQ_DECODE_MAX_BATCH) return NQ_ERR_NOALLOC_LIMIT;
+    if (batch == 0) return NQ_OK;
+    if (!x || !Upk || !Vpk || !s1 || !s2 || !y) return NQ_ERR_NULL;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(Upk) |
+                        reinterpret_cast<uintptr_t>(Vpk) | reinterpret_cast<uintptr_t>(s1) |
+                        reinterpret_cast<uintptr_t>(s2) | reinterpret_cast<uintptr_t>(y);
+    if (a & 15u) return NQ_ERR_ALIGN;
+    if (!is_device_memory(x) || !is_device_memory(Upk) || !is_device_memory(Vpk) || !is_device_memory(s1) ||
+        !is_device_memory(s2) || !is_device_memory(y))
+        return NQ_ERR_PTRKIND;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return NQ_ERR_CUDA;
+    }
+    void* scratch = nullptr;
+    int st = noalloc_scratch(dev, &scratch);
+    if (st != NQ_OK) return st;
+
+    // a workspace view over the fixed array (nothing here is allocated)
+    Workspace ws;
+    ws.device = dev;
+    ws.t = static_cast<float*>(scratch);
+    ws.tgmax = ws.t + kNoAllocT;
+    ws.partials = ws.tgmax + kNoAllocG;
+    ws.counters = reinterpret_cast<int*>(ws.partials + kNoAllocP);
+    ws.t_cap = kNoAllocT;
+    ws.tgmax_cap = kNoAllocG;
+    ws.partial_cap = kNoAllocP;
+    ws.counter_cap = kNoAllocC;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws.counters, 0, sizeof(int) * kNoAllocC, s) != cudaSuccess) return NQ_ERR_CUDA;
+    DecodeCall c{static_cast<const uint16_t*>(x), Upk, Vpk, static_cast<const uint16_t*>(s1),
+                 static_cast<const uint16_t*>(s2), y, m, n, r};
+    return decode_forward_group(&c, 1, batch, &ws, s, kNoAllocMaxSplits);
+}

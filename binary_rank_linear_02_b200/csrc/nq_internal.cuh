@@ -8,7 +8,8 @@
 
 namespace nq {
 
-constexpr int kMaxGroup = 16;  // layers per decode launch
+constexpr int kMaxGroup = 16;         // layers per decode launch
+constexpr int kDecodeMaxSplits = 64;  // stage-1 column splits per layer
 
 // ---------------------------------------------------------------- workspace
 // One per device.  Decode keeps t (batch x r fp32 per layer) and the max |t| of each
@@ -80,8 +81,9 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------- entry points of the kernels
-int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Workspace* ws, cudaStream_t stream);
-void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, int64_t* t_floats,
+int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Workspace* ws, cudaStream_t stream,
+                         int max_splits = kDecodeMaxSplits);
+void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, int max_splits, int64_t* t_floats,
                            int64_t* tgmax_floats, int64_t* partial_floats, int64_t* counter_ints);
 
 int decode_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const uint16_t* s1,

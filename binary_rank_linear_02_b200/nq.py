@@ -30,7 +30,9 @@ NQ_ERR_CUDA = -6
 NQ_ERR_TIMEOUT = -7
 NQ_ERR_NOMEM = -8
 NQ_ERR_PTRKIND = -9
+NQ_ERR_NOALLOC_LIMIT = -10
 NQ_DECODE_MAX_BATCH = 8
+NQ_NOALLOC_MAX_RANK = 4096
 
 
 class nq_linear_desc(ctypes.Structure):
@@ -67,6 +69,8 @@ def _load() -> ctypes.CDLL:
     L.nq_workspace_reserve.argtypes = [i64, i64, i64, i64]
     L.nq_workspace_reserve.restype = ctypes.c_int
     L.nq_version.restype = ctypes.c_int
+    L.nq_lowrank_linear_fwd_noalloc.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p]
+    L.nq_lowrank_linear_fwd_noalloc.restype = ctypes.c_int
     L.nq_lowrank_linear_fwd_grouped.argtypes = [p, ctypes.c_int, i64, p]
     L.nq_lowrank_linear_fwd_grouped.restype = ctypes.c_int
     L.nq_device_status.argtypes = [p]
@@ -93,6 +97,10 @@ def nq_unpack_signs(packed_ptr: int, rows: int, cols: int, out_ptr: int, stream:
 
 def nq_lowrank_linear_fwd(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n, r, batch, y_ptr, stream=0) -> int:
     return _lib.nq_lowrank_linear_fwd(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n, r, batch, y_ptr, stream)
+
+
+def nq_lowrank_linear_fwd_noalloc(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n, r, batch, y_ptr, stream=0) -> int:
+    return _lib.nq_lowrank_linear_fwd_noalloc(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n, r, batch, y_ptr, stream)
 
 
 def nq_lowrank_linear_fwd_grouped(descs_ptr, count, batch, stream=0) -> int:

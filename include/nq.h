@@ -52,7 +52,8 @@ typedef enum {
     NQ_ERR_CUDA = -6,      /* a CUDA runtime/driver call or a launch failed */
     NQ_ERR_TIMEOUT = -7,   /* a bounded device-side wait gave up */
     NQ_ERR_NOMEM = -8,     /* workspace allocation failed */
-    NQ_ERR_PTRKIND = -9    /* pointers of mixed or unsupported memory kinds */
+    NQ_ERR_PTRKIND = -9,   /* pointers of mixed or unsupported memory kinds */
+    NQ_ERR_NOALLOC_LIMIT = -10 /* size beyond nq_lowrank_linear_fwd_noalloc's fixed scratch */
 } nq_status;
 
 /* Largest decode batch: calls with 1 <= batch <= NQ_DECODE_MAX_BATCH run the two-stage
@@ -128,6 +129,32 @@ typedef struct nq_linear_desc {
  * (0 is a no-op) and `layers` non-NULL; host-memory buffers are refused (NQ_ERR_PTRKIND).
  */
 int nq_lowrank_linear_fwd_grouped(const nq_linear_desc* layers, int count, int64_t batch, void* stream);
+
+/* Limits of nq_lowrank_linear_fwd_noalloc. */
+#define NQ_NOALLOC_MAX_RANK 4096
+#define NQ_NOALLOC_MAX_BATCH NQ_DECODE_MAX_BATCH
+
+/*
+ * nq_lowrank_linear_fwd_noalloc -- the decode path of nq_lowrank_linear_fwd for callers
+ * that cannot allocate device memory when they run a layer (an engine whose memory pool
+ * is fixed at start-up, a host framework that owns the allocator, work recorded while
+ * allocation is off limits).  It has no counterpart in the NanoQuant pages: it is a
+ * property of this library, not of the method.
+ *   Same arguments, layout and result as nq_lowrank_linear_fwd, restricted to
+ *   1 <= batch <= NQ_NOALLOC_MAX_BATCH and r <= NQ_NOALLOC_MAX_RANK (larger sizes return
+ *   NQ_ERR_NOALLOC_LIMIT; batch 0 is a no-op).  Every pointer must be device memory.
+ *   Scratch: a fixed 1.16 MB array compiled into the library's device code, held by every
+ *   GPU that loads the library until the process exits.  The call allocates and frees
+ *   nothing, on the host or the device.
+ *   The first call on each device resolves the array's device address (with that device
+ *   current); make that first call before any stream capture that includes this entry.
+ *   All calls share the one array and each call overwrites it: calls whose kernels could
+ *   overlap on the GPU (other streams, other host threads on the same device) race, and
+ *   must be ordered by the caller.
+ */
+int nq_lowrank_linear_fwd_noalloc(const void* x, const uint32_t* Upk, const uint32_t* Vpk,
+                                  const void* s1, const void* s2, int64_t m, int64_t n, int64_t r,
+                                  int64_t batch, float* y, void* stream);
 
 /*
  * nq_bits_per_weight -- storage cost of the factorised layer in bits per weight of the
