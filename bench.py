@@ -177,6 +177,24 @@ class DecodeWorkload:
                 raise RuntimeError(f"nq_lowrank_linear_fwd: {self.nq.nq_status_string(st)}")
 
 
+def aggregate(ms_local: float, units_local: float, dist=None, device=None):
+    """Whole-job numbers of independent replicas: (max time over ranks, units of all ranks).
+
+    Each rank timed its own K steps on its own device; the job took as long as the slowest
+    rank, and did the work of all of them.  Works over NCCL (device tensors) or gloo.
+    """
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return ms_local, units_local
+    import torch
+
+    t = torch.tensor([ms_local, units_local], dtype=torch.float64, device=device)
+    ms = t[:1].clone()
+    units = t[1:].clone()
+    dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    dist.all_reduce(units, op=dist.ReduceOp.SUM)
+    return float(ms.item()), float(units.item())
+
+
 def capture(fn, stream):
     import torch
 
@@ -248,12 +266,7 @@ def run_ours(args):
     sampler.start()
     ms = timed_graphs(work, args.steps, args.warmup, stream, dist=dist)
     clocks = sampler.stop()
-    ms_max = ms
-    if dist is not None:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-    total_bytes = work.step_bytes * args.steps * world
+    ms_max, total_bytes = aggregate(ms, float(work.step_bytes * args.steps), dist, device)
     value = total_bytes / (ms_max * 1e-3) / 1e9
     tokens_per_s = batch * args.steps * world / (ms_max * 1e-3)
 

@@ -123,6 +123,7 @@ struct DecGroup {
     DecLayer L[kMaxGroup];
     int count;
     int batch;
+    int depth1, depth2;  // chunk ring depth of stage 1 / stage 2 (1 or 2)
     int s1_start[kMaxGroup + 1];
     int s2_start[kMaxGroup + 1];
 };
@@ -133,53 +134,84 @@ __device__ __forceinline__ int find_layer(const int* start, int count, int block
     return l;
 }
 
-// Shared memory of both stages; NT = 4 * NTG token slots.
-template <int NTG>
-struct DecSmem {
-    static constexpr int NT = 4 * NTG;
-    uint32_t w[2][kRowsS1][kChunkWords + kRowPad];  // weight rows of two chunks (18 KB)
-    union {
-        float t[2][NT][kChunk];                      // stage 2: two chunks of t
-        struct {
-            uint16_t x[2][NT][kChunk];               // stage 1: two chunks of x
-            uint16_t s2[2][kChunk];                  //          and of s2
-        } s1;
-    } act;
-    uint4 frag[kChunkCB][NTG][2][32];               // [cb][token group][half][lane]
+// Shared memory.  The layout is sized per launch (ring depth, batch), so a CTA holds only
+// what it uses and more CTAs fit on an SM:
+//   w    : depth x 64 rows x (32 + 4) words         weight rows of the staged chunks
+//   act  : stage 1 depth x (batch x kChunk bf16 x + kChunk fp16 s2); stage 2 depth x batch x kChunk fp32 t
+//   frag : kChunkCB x NTG x 2 x 32 uint4             B fragments of one chunk
+//   misc : reductions and per-token quantisation state
+struct DecMisc {
     float red[kWarps][8];
     int e[8];
-    float up[8];                                    // 2^(14 - e): quantisation factor per token
+    float up[8];      // 2^(14 - e): quantisation factor per token
     int qsum[8];
-    int bq[64][8];                                  // stage 2: per (row, token) across k-parts
-    float res[8][kRowsS1];                          // stage 1: sums of the CTA's rows
+    int bq[64][8];    // stage 2: per (row, token) across k-parts
+    float res[8][kRowsS1];  // stage 1: sums of the CTA's rows
     int last;
+};
+
+constexpr int kWRow = kChunkWords + kRowPad;
+
+__host__ __device__ inline size_t smem_w_bytes(int depth) { return (size_t)depth * kRowsS1 * kWRow * 4; }
+__host__ __device__ inline size_t smem_act_bytes(int stage, int depth, int batch) {
+    return stage == 1 ? (size_t)depth * ((size_t)batch * kChunk * 2 + kChunk * 2) : (size_t)depth * batch * kChunk * 4;
+}
+__host__ __device__ inline size_t smem_frag_bytes(int ntg) { return (size_t)kChunkCB * ntg * 2 * 32 * 16; }
+__host__ __device__ inline size_t smem_bytes(int stage, int depth, int batch, int ntg) {
+    return smem_w_bytes(depth) + smem_act_bytes(stage, depth, batch) + smem_frag_bytes(ntg) + sizeof(DecMisc);
+}
+
+template <int NTG>
+struct Sm {
+    uint32_t* w;
+    uint16_t* x;
+    uint16_t* s2;
+    float* t;
+    uint4* frag;
+    DecMisc* misc;
+    int batch;
+
+    __device__ Sm(unsigned char* base, int stage, int depth, int batch_) : batch(batch_) {
+        w = reinterpret_cast<uint32_t*>(base);
+        unsigned char* act = base + smem_w_bytes(depth);
+        x = reinterpret_cast<uint16_t*>(act);
+        s2 = x + (size_t)depth * batch * kChunk;
+        t = reinterpret_cast<float*>(act);
+        frag = reinterpret_cast<uint4*>(act + smem_act_bytes(stage, depth, batch));
+        misc = reinterpret_cast<DecMisc*>(reinterpret_cast<unsigned char*>(frag) + smem_frag_bytes(NTG));
+    }
+    __device__ uint32_t* wrow(int buf, int row) const { return w + ((size_t)buf * kRowsS1 + row) * kWRow; }
+    __device__ uint16_t* xrow(int buf, int tok) const { return x + ((size_t)buf * batch + tok) * kChunk; }
+    __device__ uint16_t* s2row(int buf) const { return s2 + (size_t)buf * kChunk; }
+    __device__ float* trow(int buf, int tok) const { return t + ((size_t)buf * batch + tok) * kChunk; }
+    __device__ uint4& fr(int cb, int tg, int half, int lane) const { return frag[((cb * NTG + tg) * 2 + half) * 32 + lane]; }
 };
 
 // Copy `rows` weight rows, words [w0, w0 + nw) of each, into buffer `buf` (cp.async).
 template <int NTG>
-__device__ __forceinline__ void stage_weights(DecSmem<NTG>& sm, int buf, const uint32_t* W, int64_t wpr, int rows,
+__device__ __forceinline__ void stage_weights(const Sm<NTG>& sm, int buf, const uint32_t* W, int64_t wpr, int rows,
                                               int64_t w0, int nw) {
     const int per_row = nw / 4;  // 16-byte pieces
     const int total = rows * per_row;
     for (int i = threadIdx.x; i < total; i += kThreads) {
         const int row = i / per_row, p = i % per_row;
-        cp_async16(&sm.w[buf][row][4 * p], W + (int64_t)row * wpr + w0 + 4 * p);
+        cp_async16(sm.wrow(buf, row) + 4 * p, W + (int64_t)row * wpr + w0 + 4 * p);
     }
 }
 
 // B fragments of `ncb` column blocks from values v(tok, col) (col relative to the chunk),
-// quantised with sm.up[tok]; adds each token's sum of q to sm.qsum.  One task =
+// quantised with up[tok]; adds each token's sum of q to qsum.  One task =
 // (cb, token, word t of the CB, half h): the 16 columns 32t + s + 4h + 8c (s, c in 0..3)
 // feed fragment words j = 2s + h of two lanes, the hi-limb lane 8*tok' + t and the
 // lo-limb lane 8*tok' + 4 + t (tok' = token within its group).  Slots of tokens >= batch
 // are never written and stay zero (zero_fragments at kernel start).
 template <int NTG, typename ValueFn>
-__device__ __forceinline__ void build_fragments(DecSmem<NTG>& sm, int ncb, int batch, ValueFn value) {
+__device__ __forceinline__ void build_fragments(const Sm<NTG>& sm, int ncb, int batch, ValueFn value) {
     const int tasks = ncb * batch * 8;
     for (int task = threadIdx.x; task < tasks; task += kThreads) {
         const int h = task & 1, t = (task >> 1) & 3;
         const int tok = (task >> 3) % batch, cb = (task >> 3) / batch;
-        const float up = sm.up[tok];
+        const float up = sm.misc->up[tok];
         const int c0 = cb * kCB + 32 * t + 4 * h;
         uint32_t hi[4], lo[4];
         int qs = 0;
@@ -196,12 +228,12 @@ __device__ __forceinline__ void build_fragments(DecSmem<NTG>& sm, int ncb, int b
             hi[s4] = wh;
             lo[s4] = wl;
         }
-        atomicAdd(&sm.qsum[tok], qs);
+        atomicAdd(&sm.misc->qsum[tok], qs);
         const int tg = tok >> 2, ti = tok & 3;
-        uint32_t* fh0 = reinterpret_cast<uint32_t*>(&sm.frag[cb][tg][0][8 * ti + t]);
-        uint32_t* fh1 = reinterpret_cast<uint32_t*>(&sm.frag[cb][tg][1][8 * ti + t]);
-        uint32_t* fl0 = reinterpret_cast<uint32_t*>(&sm.frag[cb][tg][0][8 * ti + 4 + t]);
-        uint32_t* fl1 = reinterpret_cast<uint32_t*>(&sm.frag[cb][tg][1][8 * ti + 4 + t]);
+        uint32_t* fh0 = reinterpret_cast<uint32_t*>(&sm.fr(cb, tg, 0, 8 * ti + t));
+        uint32_t* fh1 = reinterpret_cast<uint32_t*>(&sm.fr(cb, tg, 1, 8 * ti + t));
+        uint32_t* fl0 = reinterpret_cast<uint32_t*>(&sm.fr(cb, tg, 0, 8 * ti + 4 + t));
+        uint32_t* fl1 = reinterpret_cast<uint32_t*>(&sm.fr(cb, tg, 1, 8 * ti + 4 + t));
         // word j = 2*s4 + h lives in half j >> 2 at component j & 3
         fh0[h] = hi[0];
         fh0[2 + h] = hi[1];
@@ -215,34 +247,57 @@ __device__ __forceinline__ void build_fragments(DecSmem<NTG>& sm, int ncb, int b
 }
 
 template <int NTG>
-__device__ __forceinline__ void zero_fragments(DecSmem<NTG>& sm) {
-    uint4* f = &sm.frag[0][0][0][0];
-    for (int i = threadIdx.x; i < kChunkCB * NTG * 2 * 32; i += kThreads) f[i] = make_uint4(0, 0, 0, 0);
+__device__ __forceinline__ void zero_fragments(const Sm<NTG>& sm) {
+    for (int i = threadIdx.x; i < kChunkCB * NTG * 2 * 32; i += kThreads) sm.frag[i] = make_uint4(0, 0, 0, 0);
 }
 
-// Accumulate one 16-row tile (rows r0.., staged in sm.w[buf]) against column blocks
-// cb0, cb0 + step, ... < cb1 of the staged chunk.
+// One column block of a 16-row tile into accumulator set `acc`.
 template <int NTG>
-__device__ __forceinline__ void tile_mma(const DecSmem<NTG>& sm, int buf, int r0, int cb0, int cb1, int step,
-                                         int (&acc)[NTG][4][4]) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const uint32_t* wa_row = sm.w[buf][r0 + g];
-    const uint32_t* wb_row = sm.w[buf][r0 + g + 8];
-#pragma unroll 2
-    for (int cb = cb0; cb < cb1; cb += step) {
-        const uint32_t wa = wa_row[4 * cb + t], wb = wb_row[4 * cb + t];
-        const uint32_t a4 = wa >> 4, b4 = wb >> 4;
+__device__ __forceinline__ void cb_mma(const Sm<NTG>& sm, uint32_t wa, uint32_t wb, int cb, int lane,
+                                       int (&acc)[NTG][4][4]) {
+    const uint32_t a4 = wa >> 4, b4 = wb >> 4;
 #pragma unroll
-        for (int tg = 0; tg < NTG; ++tg) {
-            const uint4 f0 = sm.frag[cb][tg][0][lane], f1 = sm.frag[cb][tg][1][lane];
-            const uint32_t bf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+    for (int tg = 0; tg < NTG; ++tg) {
+        const uint4 f0 = sm.fr(cb, tg, 0, lane), f1 = sm.fr(cb, tg, 1, lane);
+        const uint32_t bf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const uint32_t M = 0x01010101u << s;
-                mma_u8s8(acc[tg][s], wa & M, wb & M, a4 & M, b4 & M, bf[2 * s], bf[2 * s + 1]);
-            }
+        for (int s = 0; s < 4; ++s) {
+            const uint32_t M = 0x01010101u << s;
+            mma_u8s8(acc[tg][s], wa & M, wb & M, a4 & M, b4 & M, bf[2 * s], bf[2 * s + 1]);
         }
     }
+}
+
+// Accumulate one 16-row tile (rows r0.., staged in buffer `buf`) against column blocks
+// cb0, cb0 + step, ... < cb1 of the staged chunk.  Two accumulator sets alternate between
+// consecutive column blocks so that dependent MMAs are two blocks apart.
+template <int NTG>
+__device__ __forceinline__ void tile_mma(const Sm<NTG>& sm, int buf, int r0, int cb0, int cb1, int step,
+                                         int (&acc)[NTG][4][4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const uint32_t* wa_row = sm.wrow(buf, r0 + g);
+    const uint32_t* wb_row = sm.wrow(buf, r0 + g + 8);
+    int acc2[NTG][4][4];
+#pragma unroll
+    for (int tg = 0; tg < NTG; ++tg)
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc2[tg][s][i] = 0;
+    int cb = cb0;
+    for (; cb + step < cb1; cb += 2 * step) {
+        const uint32_t wa0 = wa_row[4 * cb + t], wb0 = wb_row[4 * cb + t];
+        const uint32_t wa1 = wa_row[4 * (cb + step) + t], wb1 = wb_row[4 * (cb + step) + t];
+        cb_mma<NTG>(sm, wa0, wb0, cb, lane, acc);
+        cb_mma<NTG>(sm, wa1, wb1, cb + step, lane, acc2);
+    }
+    if (cb < cb1) cb_mma<NTG>(sm, wa_row[4 * cb + t], wb_row[4 * cb + t], cb, lane, acc);
+#pragma unroll
+    for (int tg = 0; tg < NTG; ++tg)
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[tg][s][i] += acc2[tg][s][i];
 }
 
 // sum_j b_j q_j for (row g, token 4tg+t) and (row g+8, same token).
@@ -278,22 +333,23 @@ __device__ __forceinline__ void zero_acc(int (&acc)[NTG][4][4]) {
 // adds them in split order (deterministic), then writes t and the block's max |t| per
 // token (stage 2 builds its exponent from those maxima).
 template <int NTG>
-__device__ __forceinline__ void stage1_fetch_x(DecSmem<NTG>& sm, int buf, const DecLayer& L, int batch, int col0,
+__device__ __forceinline__ void stage1_fetch_x(const Sm<NTG>& sm, int buf, const DecLayer& L, int batch, int col0,
                                                int ccols) {
     const int per_tok = ccols / 8;  // 16-byte pieces
     for (int i = threadIdx.x; i < (batch + 1) * per_tok; i += kThreads) {
         const int tok = i / per_tok, p = i % per_tok;
         if (tok < batch)
-            cp_async16(&sm.act.s1.x[buf][tok][8 * p], L.x + (int64_t)tok * L.n + col0 + 8 * p);
+            cp_async16(sm.xrow(buf, tok) + 8 * p, L.x + (int64_t)tok * L.n + col0 + 8 * p);
         else
-            cp_async16(&sm.act.s1.s2[buf][8 * p], L.s2 + col0 + 8 * p);
+            cp_async16(sm.s2row(buf) + 8 * p, L.s2 + col0 + 8 * p);
     }
 }
 
 template <int NTG>
 __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant__ DecGroup grp) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    DecSmem<NTG>& sm = *reinterpret_cast<DecSmem<NTG>*>(smem_raw);
+    const Sm<NTG> sm(smem_raw, 1, grp.depth1, grp.batch);
+    DecMisc& mi = *sm.misc;
     const int li = find_layer(grp.s1_start, grp.count, blockIdx.x);
     const DecLayer& L = grp.L[li];
     const int local = blockIdx.x - grp.s1_start[li];
@@ -334,17 +390,17 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
         if (ch + 1 < nchunks) cp_async_wait<1>(); else cp_async_wait<0>();
         __syncthreads();
         // per-token max of s2 * x over the chunk
-        const uint16_t* xs = &sm.act.s1.x[buf][0][0];
-        const uint16_t* ss = sm.act.s1.s2[buf];
+        const uint16_t* xs = sm.xrow(buf, 0);
+        const uint16_t* ss = sm.s2row(buf);
         for (int tok = warp; tok < batch; tok += kWarps) {
             float mx = 0.f;
             for (int c = lane; c < ccols; c += 32) mx = fmaxf(mx, fabsf(bf16_to_f32(xs[tok * kChunk + c]) * f16_to_f32(ss[c])));
             mx = warp_max(mx);
             if (lane == 0) {
                 const int e = range_exponent(mx);
-                sm.e[tok] = e;
-                sm.up[tok] = pow2f(kQBits - e);
-                sm.qsum[tok] = 0;
+                mi.e[tok] = e;
+                mi.up[tok] = pow2f(kQBits - e);
+                mi.qsum[tok] = 0;
             }
         }
         __syncthreads();
@@ -362,8 +418,8 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
             if (tok < batch) {
                 int bq0, bq8;
                 combine<NTG>(acc, tg, bq0, bq8);
-                const int64_t qs = sm.qsum[tok];
-                const float down = pow2f(sm.e[tok] - kQBits);
+                const int64_t qs = mi.qsum[tok];
+                const float down = pow2f(mi.e[tok] - kQBits);
                 part[tg][0] += (float)(2 * (int64_t)bq0 - qs) * down;
                 part[tg][1] += (float)(2 * (int64_t)bq8 - qs) * down;
             }
@@ -382,8 +438,8 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
     for (int tg = 0; tg < NTG; ++tg) {
         const int tok = 4 * tg + tq;
         if (tok < batch) {
-            sm.res[tok][16 * warp + g] = part[tg][0];
-            sm.res[tok][16 * warp + g + 8] = part[tg][1];
+            mi.res[tok][16 * warp + g] = part[tg][0];
+            mi.res[tok][16 * warp + g + 8] = part[tg][1];
         }
     }
     __syncthreads();
@@ -391,14 +447,16 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
     if (L.nsplit > 1) {
         for (int i = threadIdx.x; i < batch * kRowsS1; i += kThreads) {
             const int tok = i / kRowsS1, k = i % kRowsS1;
-            L.partials[((int64_t)sp * batch + tok) * r + row0 + k] = sm.res[tok][k];
+            L.partials[((int64_t)sp * batch + tok) * r + row0 + k] = mi.res[tok][k];
         }
-        __threadfence();
         __syncthreads();
-        if (threadIdx.x == 0) sm.last = (atomicAdd(&L.counters[rb], 1) == L.nsplit - 1);
+        if (threadIdx.x == 0) {
+            __threadfence();  // the CTA's partials (ordered before by the barrier) are visible first
+            mi.last = (atomicAdd(&L.counters[rb], 1) == L.nsplit - 1);
+            if (mi.last) __threadfence();
+        }
         __syncthreads();
-        if (!sm.last) return;
-        __threadfence();
+        if (!mi.last) return;
         for (int i = threadIdx.x; i < batch * kRowsS1; i += kThreads) {
             const int tok = i / kRowsS1, k = i % kRowsS1;
             const float* pp = L.partials + (int64_t)tok * r + row0 + k;
@@ -411,14 +469,14 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
                 sum = (((sum + a) + b) + c) + d;
             }
             for (; q < L.nsplit; ++q) sum += __ldcg(pp + q * stride);
-            sm.res[tok][k] = sum;
+            mi.res[tok][k] = sum;
         }
         if (threadIdx.x == 0) L.counters[rb] = 0;
         __syncthreads();
     }
     // t and the block's max |t| per token (one warp per token)
     for (int tok = warp; tok < batch; tok += kWarps) {
-        const float a = sm.res[tok][lane], b = sm.res[tok][lane + 32];
+        const float a = mi.res[tok][lane], b = mi.res[tok][lane + 32];
         L.t[(int64_t)tok * r + row0 + lane] = a;
         L.t[(int64_t)tok * r + row0 + lane + 32] = b;
         const float v = warp_max(fmaxf(fabsf(a), fabsf(b)));
@@ -431,19 +489,20 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
 // token for the whole of t (from stage 1's maxima), so integer sums run across all
 // chunks and k-parts and are converted once, in the epilogue.
 template <int NTG>
-__device__ __forceinline__ void stage2_fetch_t(DecSmem<NTG>& sm, int buf, const DecLayer& L, int batch, int col0,
+__device__ __forceinline__ void stage2_fetch_t(const Sm<NTG>& sm, int buf, const DecLayer& L, int batch, int col0,
                                                int ccols) {
     const int per_tok = ccols / 4;  // 16-byte pieces
     for (int i = threadIdx.x; i < batch * per_tok; i += kThreads) {
         const int tok = i / per_tok, p = i % per_tok;
-        cp_async16(&sm.act.t[buf][tok][4 * p], L.t + (int64_t)tok * L.r + col0 + 4 * p);
+        cp_async16(sm.trow(buf, tok) + 4 * p, L.t + (int64_t)tok * L.r + col0 + 4 * p);
     }
 }
 
 template <int NTG>
 __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant__ DecGroup grp) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    DecSmem<NTG>& sm = *reinterpret_cast<DecSmem<NTG>*>(smem_raw);
+    const Sm<NTG> sm(smem_raw, 2, grp.depth2, grp.batch);
+    DecMisc& mi = *sm.misc;
     const int li = find_layer(grp.s2_start, grp.count, blockIdx.x);
     const DecLayer& L = grp.L[li];
     const int blk = blockIdx.x - grp.s2_start[li];
@@ -465,7 +524,7 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
     cp_async_commit();
     if (nchunks > 2 && threadIdx.x < rows)
         prefetch_l2(W + threadIdx.x * wpr + 2 * kChunkWords, (uint32_t)((r - 2 * kChunk) / 8));
-    for (int i = threadIdx.x; i < 64 * 8; i += kThreads) (&sm.bq[0][0])[i] = 0;
+    for (int i = threadIdx.x; i < 64 * 8; i += kThreads) (&mi.bq[0][0])[i] = 0;
     zero_fragments(sm);
     pdl_trigger();
     pdl_wait();  // t and its maxima come from stage 1
@@ -482,9 +541,9 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
         mx = warp_max(mx);
         if (lane == 0) {
             const int e = range_exponent(mx);
-            sm.e[tok] = e;
-            sm.up[tok] = pow2f(kQBits - e);
-            sm.qsum[tok] = 0;
+            mi.e[tok] = e;
+            mi.up[tok] = pow2f(kQBits - e);
+            mi.qsum[tok] = 0;
         }
     }
 
@@ -496,7 +555,7 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
         const int ncb = ccols / kCB;
         if (ch + 1 < nchunks) cp_async_wait<1>(); else cp_async_wait<0>();
         __syncthreads();
-        const float* ts = &sm.act.t[buf][0][0];
+        const float* ts = sm.trow(buf, 0);
         build_fragments(sm, ncb, batch, [&](int tok, int c) { return ts[tok * kChunk + c]; });
         __syncthreads();
         tile_mma<NTG>(sm, buf, 16 * rt, kp, ncb, KS, acc);
@@ -514,15 +573,15 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
         if (tok < batch) {
             int bq0, bq8;
             combine<NTG>(acc, tg, bq0, bq8);
-            atomicAdd(&sm.bq[16 * rt + g][tok], bq0);
-            atomicAdd(&sm.bq[16 * rt + g + 8][tok], bq8);
+            atomicAdd(&mi.bq[16 * rt + g][tok], bq0);
+            atomicAdd(&mi.bq[16 * rt + g + 8][tok], bq8);
         }
     }
     __syncthreads();
     for (int idx = threadIdx.x; idx < rows * batch; idx += kThreads) {
         const int tok = idx / rows, i = idx % rows;
         const int64_t row = row0 + i;
-        const float v = (float)(2 * (int64_t)sm.bq[i][tok] - sm.qsum[tok]) * pow2f(sm.e[tok] - kQBits);
+        const float v = (float)(2 * (int64_t)mi.bq[i][tok] - mi.qsum[tok]) * pow2f(mi.e[tok] - kQBits);
         L.y[(int64_t)tok * m + row] = f16_to_f32(L.s1[row]) * v;
     }
 }
@@ -531,19 +590,18 @@ template <int NTG>
 int launch_group(DecGroup& grp, cudaStream_t stream, int device) {
     static unsigned long long init_mask = 0;  // devices whose kernel attributes are set
     const unsigned long long bit = 1ull << (device & 63);
-    const size_t smem = sizeof(DecSmem<NTG>);
     if (!(__atomic_load_n(&init_mask, __ATOMIC_ACQUIRE) & bit)) {
-        if (cudaFuncSetAttribute(stage1_kernel<NTG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(stage2_kernel<NTG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-                cudaSuccess)
+        const int most = (int)smem_bytes(2, 2, 4 * NTG, NTG);  // the largest layout either stage uses
+        if (cudaFuncSetAttribute(stage1_kernel<NTG>, cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess ||
+            cudaFuncSetAttribute(stage2_kernel<NTG>, cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess)
             return NQ_ERR_CUDA;
         __atomic_fetch_or(&init_mask, bit, __ATOMIC_RELEASE);
     }
-    if (launch_pdl(stage1_kernel<NTG>, dim3((unsigned)grp.s1_start[grp.count]), dim3(kThreads), smem, stream, grp) !=
+    const size_t smem1 = smem_bytes(1, grp.depth1, grp.batch, NTG), smem2 = smem_bytes(2, grp.depth2, grp.batch, NTG);
+    if (launch_pdl(stage1_kernel<NTG>, dim3((unsigned)grp.s1_start[grp.count]), dim3(kThreads), smem1, stream, grp) !=
         cudaSuccess)
         return NQ_ERR_CUDA;
-    if (launch_pdl(stage2_kernel<NTG>, dim3((unsigned)grp.s2_start[grp.count]), dim3(kThreads), smem, stream, grp) !=
+    if (launch_pdl(stage2_kernel<NTG>, dim3((unsigned)grp.s2_start[grp.count]), dim3(kThreads), smem2, stream, grp) !=
         cudaSuccess)
         return NQ_ERR_CUDA;
     return NQ_OK;
@@ -633,6 +691,15 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
         grp.s1_start[i + 1] = grp.s1_start[i] + (int)(c.r / kRowsS1) * L.nsplit;
         grp.s2_start[i + 1] = grp.s2_start[i] + (int)(c.m / (16 * rt));
     }
+    int max_c1 = 1, max_c2 = 1;
+    for (int i = 0; i < count; ++i) {
+        const int c1 = (cps + kChunkCB - 1) / kChunkCB;
+        const int c2 = (int)((calls[i].r + kChunk - 1) / kChunk);
+        max_c1 = c1 > max_c1 ? c1 : max_c1;
+        max_c2 = c2 > max_c2 ? c2 : max_c2;
+    }
+    grp.depth1 = max_c1 > 1 ? 2 : 1;
+    grp.depth2 = max_c2 > 1 ? 2 : 1;
     if (batch <= 4) return launch_group<1>(grp, stream, ws->device);
     return launch_group<2>(grp, stream, ws->device);
 }
