@@ -30,11 +30,12 @@
 // n = 2*token + limb (limb 0 = hi, 1 = lo), four tokens per token group.
 //
 // Latency.  A decode layer moves 0.4-18 MB, a few microseconds at HBM speed, so the
-// fixed costs decide: each CTA copies its weight rows into shared memory with cp.async
-// (and prefetches the rest into L2) before it waits on the previous kernel
-// (programmatic dependent launch), and it lets the next kernel launch at once, so weight
-// streaming overlaps the dependency chain.  Stage-1 CTAs own whole rows (no cross-CTA
-// reduction), and several independent layers can share one launch pair.
+// fixed costs decide.  Every CTA copies its weight rows into shared memory (cp.async)
+// before it waits on the previous kernel (programmatic dependent launch) and lets the next
+// kernel launch at once, so weight streaming overlaps the dependency chain.  Stage 1
+// splits each 64-row block's columns so that every CTA stages one chunk; the last CTA of a
+// block adds the partial sums in a fixed order (deterministic).  Stage 2 holds its whole
+// row block and the whole of t on chip.  Several independent layers can share one launch.
 #include <cuda_fp16.h>
 #include <math.h>
 
@@ -48,12 +49,12 @@ namespace {
 constexpr int kThreads = 128;          // 4 warps
 constexpr int kWarps = kThreads / 32;
 constexpr int kCB = 128;               // columns per column block
-constexpr int kChunk = 1024;           // columns staged per pass
+constexpr int kChunk = 1024;           // columns per fragment chunk
 constexpr int kChunkCB = kChunk / kCB;
 constexpr int kChunkWords = kChunk / 32;
 constexpr int kQBits = 14;             // |q| < 2^14
 constexpr int kRowsS1 = 64;            // stage-1 rows per CTA (4 warps x 16)
-constexpr int kRowPad = 4;             // words of padding per staged row (bank spread)
+constexpr int kS1Stride = kChunkWords + 4;  // words per staged stage-1 row (36: bank-spread)
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 __device__ __forceinline__ float f16_to_f32(uint16_t h) { return __half2float(__ushort_as_half(h)); }
@@ -81,7 +82,7 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 
 // Quantisation exponent E of a range whose largest |value| is max_abs: max_abs < 2^E,
 // clamped to [-100, 113] so that both 2^(14-E) and 2^(E-14) are normal floats.  Values
-// are quantised as q = rint(v * 2^(14-E)), |q| < 2^14, and dequantised by 2^(E-14); both
+// are quantised as q = rint(v * 2^(14-E)), |q| <= 2^14, and dequantised by 2^(E-14); both
 // scalings are exact.  (Inputs whose largest magnitude is below 2^-100 lose precision.)
 __device__ __forceinline__ int range_exponent(float max_abs) {
     int e = 0;
@@ -91,10 +92,8 @@ __device__ __forceinline__ int range_exponent(float max_abs) {
 
 __device__ __forceinline__ float pow2f(int k) { return __int_as_float((k + 127) << 23); }  // k in [-126, 127]
 
-__device__ __forceinline__ int quantise(float v, float up) {
-    const int q = __float2int_rn(v * up);
-    return min(max(q, -16384), 16383);
-}
+// |v * up| < 2^14 by the choice of E, so rounding gives at most 2^14: clamp the top only.
+__device__ __forceinline__ int quantise(float v, float up) { return min(__float2int_rn(v * up), 16383); }
 
 __device__ __forceinline__ float warp_max(float v) {
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -114,16 +113,18 @@ struct DecLayer {
     float* partials; // workspace: nsplit x batch x r (stage-1 column splits)
     int* counters;   // workspace: r/64 arrival counters, zero between calls
     int m, n, r;
-    int nsplit;      // stage-1 column splits (CTAs per 64-row block)
-    int cps;         // column blocks per split
-    int rt;          // stage-2 row tiles per CTA (4/rt k-parts per tile)
+    int nsplit;      // stage 1: CTAs per 64-row block (column splits)
+    int cps;         // stage 1: column blocks per split
+    int rt;          // stage 2: row tiles per CTA (4/rt k-parts per tile)
 };
 
 struct DecGroup {
     DecLayer L[kMaxGroup];
     int count;
     int batch;
-    int depth1, depth2;  // chunk ring depth of stage 1 / stage 2 (1 or 2)
+    int depth1;       // stage-1 chunk ring depth (1 or 2)
+    int r2;           // stage-2 columns held on chip at a time (a multiple of kCB)
+    int w2stride;     // stage-2 words per staged row
     int s1_start[kMaxGroup + 1];
     int s2_start[kMaxGroup + 1];
 };
@@ -134,131 +135,86 @@ __device__ __forceinline__ int find_layer(const int* start, int count, int block
     return l;
 }
 
-// Shared memory.  The layout is sized per launch (ring depth, batch), so a CTA holds only
-// what it uses and more CTAs fit on an SM:
-//   w    : depth x 64 rows x (32 + 4) words         weight rows of the staged chunks
-//   act  : stage 1 depth x (batch x kChunk bf16 x + kChunk fp16 s2); stage 2 depth x batch x kChunk fp32 t
-//   frag : kChunkCB x NTG x 2 x 32 uint4             B fragments of one chunk
-//   misc : reductions and per-token quantisation state
-struct DecMisc {
+// ------------------------------------------------------------------ shared memory
+// Sized per launch (ring depth, batch, ranks), so a CTA holds only what it uses.
+struct Misc {
     float red[kWarps][8];
     int e[8];
-    float up[8];      // 2^(14 - e): quantisation factor per token
+    float up[8];             // 2^(14 - e): quantisation factor per token
     int qsum[8];
-    int bq[64][8];    // stage 2: per (row, token) across k-parts
-    float res[8][kRowsS1];  // stage 1: sums of the CTA's rows
+    int bq[64][8];           // stage 2: per (row, token) across k-parts
+    float res[8][kRowsS1];   // stage 1: the CTA's partial sums of its 64 rows
     int last;
 };
 
-constexpr int kWRow = kChunkWords + kRowPad;
+__host__ __device__ inline size_t frag_bytes(int ntg) { return (size_t)kChunkCB * ntg * 2 * 32 * 16; }
 
-__host__ __device__ inline size_t smem_w_bytes(int depth) { return (size_t)depth * kRowsS1 * kWRow * 4; }
-__host__ __device__ inline size_t smem_act_bytes(int stage, int depth, int batch) {
-    return stage == 1 ? (size_t)depth * ((size_t)batch * kChunk * 2 + kChunk * 2) : (size_t)depth * batch * kChunk * 4;
+// stage 1: w [depth][64][36] | x [depth][batch + 1][1024] bf16 (slot batch = s2) | v [batch][1024] f32 | frag | misc
+__host__ __device__ inline size_t s1_w_bytes(int depth) { return (size_t)depth * kRowsS1 * kS1Stride * 4; }
+__host__ __device__ inline size_t s1_x_bytes(int depth, int batch) { return (size_t)depth * (batch + 1) * kChunk * 2; }
+__host__ __device__ inline size_t s1_v_bytes(int batch) { return (size_t)batch * kChunk * 4; }
+__host__ __device__ inline size_t s1_bytes(int depth, int batch, int ntg) {
+    return s1_w_bytes(depth) + s1_x_bytes(depth, batch) + s1_v_bytes(batch) + frag_bytes(ntg) + sizeof(Misc);
 }
-__host__ __device__ inline size_t smem_frag_bytes(int ntg) { return (size_t)kChunkCB * ntg * 2 * 32 * 16; }
-__host__ __device__ inline size_t smem_bytes(int stage, int depth, int batch, int ntg) {
-    return smem_w_bytes(depth) + smem_act_bytes(stage, depth, batch) + smem_frag_bytes(ntg) + sizeof(DecMisc);
+// stage 2: w [64][w2stride] | t [batch][r2] f32 | frag | misc
+__host__ __device__ inline size_t s2_w_bytes(int w2stride) { return (size_t)kRowsS1 * w2stride * 4; }
+__host__ __device__ inline size_t s2_t_bytes(int batch, int r2) { return (size_t)batch * r2 * 4; }
+__host__ __device__ inline size_t s2_bytes(int w2stride, int batch, int r2, int ntg) {
+    return s2_w_bytes(w2stride) + s2_t_bytes(batch, r2) + frag_bytes(ntg) + sizeof(Misc);
 }
 
 template <int NTG>
-struct Sm {
-    uint32_t* w;
-    uint16_t* x;
-    uint16_t* s2;
-    float* t;
-    uint4* frag;
-    DecMisc* misc;
-    int batch;
-
-    __device__ Sm(unsigned char* base, int stage, int depth, int batch_) : batch(batch_) {
-        w = reinterpret_cast<uint32_t*>(base);
-        unsigned char* act = base + smem_w_bytes(depth);
-        x = reinterpret_cast<uint16_t*>(act);
-        s2 = x + (size_t)depth * batch * kChunk;
-        t = reinterpret_cast<float*>(act);
-        frag = reinterpret_cast<uint4*>(act + smem_act_bytes(stage, depth, batch));
-        misc = reinterpret_cast<DecMisc*>(reinterpret_cast<unsigned char*>(frag) + smem_frag_bytes(NTG));
-    }
-    __device__ uint32_t* wrow(int buf, int row) const { return w + ((size_t)buf * kRowsS1 + row) * kWRow; }
-    __device__ uint16_t* xrow(int buf, int tok) const { return x + ((size_t)buf * batch + tok) * kChunk; }
-    __device__ uint16_t* s2row(int buf) const { return s2 + (size_t)buf * kChunk; }
-    __device__ float* trow(int buf, int tok) const { return t + ((size_t)buf * batch + tok) * kChunk; }
-    __device__ uint4& fr(int cb, int tg, int half, int lane) const { return frag[((cb * NTG + tg) * 2 + half) * 32 + lane]; }
-};
-
-// Copy `rows` weight rows, words [w0, w0 + nw) of each, into buffer `buf` (cp.async).
-template <int NTG>
-__device__ __forceinline__ void stage_weights(const Sm<NTG>& sm, int buf, const uint32_t* W, int64_t wpr, int rows,
-                                              int64_t w0, int nw) {
-    const int per_row = nw / 4;  // 16-byte pieces
-    const int total = rows * per_row;
-    for (int i = threadIdx.x; i < total; i += kThreads) {
-        const int row = i / per_row, p = i % per_row;
-        cp_async16(sm.wrow(buf, row) + 4 * p, W + (int64_t)row * wpr + w0 + 4 * p);
-    }
+__device__ __forceinline__ uint4& frag_at(uint4* frag, int cb, int tg, int half, int lane) {
+    return frag[((cb * NTG + tg) * 2 + half) * 32 + lane];
 }
 
-// B fragments of `ncb` column blocks from values v(tok, col) (col relative to the chunk),
-// quantised with up[tok]; adds each token's sum of q to qsum.  One task =
-// (cb, token, word t of the CB, half h): the 16 columns 32t + s + 4h + 8c (s, c in 0..3)
-// feed fragment words j = 2s + h of two lanes, the hi-limb lane 8*tok' + t and the
-// lo-limb lane 8*tok' + 4 + t (tok' = token within its group).  Slots of tokens >= batch
-// are never written and stay zero (zero_fragments at kernel start).
-template <int NTG, typename ValueFn>
-__device__ __forceinline__ void build_fragments(const Sm<NTG>& sm, int ncb, int batch, ValueFn value) {
-    const int tasks = ncb * batch * 8;
+template <int NTG>
+__device__ __forceinline__ void zero_fragments(uint4* frag) {
+    for (int i = threadIdx.x; i < kChunkCB * NTG * 2 * 32; i += kThreads) frag[i] = make_uint4(0, 0, 0, 0);
+}
+
+// B fragments of `ncb` column blocks from fp32 values vals[tok * vstride + col] (col from
+// the chunk's first column), quantised with up[tok]; adds each token's sum of q to qsum.
+// One task = (cb, token, word t of the CB, fragment word j = 2s + h): the 4 columns
+// 32t + s + 4h + 8c (c in 0..3) give word j of two lanes, the hi-limb lane 8*tok' + t and
+// the lo-limb lane 8*tok' + 4 + t (tok' = token within its group).  The 32 tasks of a
+// warp step share one token, so the warp adds its q's with a shuffle reduction.  Slots of
+// tokens >= batch are never written and stay zero (zero_fragments at kernel start).
+template <int NTG>
+__device__ __forceinline__ void build_fragments(uint4* frag, Misc& mi, const float* vals, int vstride, int ncb,
+                                                int batch) {
+    const int tasks = ncb * batch * 32;  // a multiple of 32: whole warps take part in every step
     for (int task = threadIdx.x; task < tasks; task += kThreads) {
-        const int h = task & 1, t = (task >> 1) & 3;
-        const int tok = (task >> 3) % batch, cb = (task >> 3) / batch;
-        const float up = sm.misc->up[tok];
-        const int c0 = cb * kCB + 32 * t + 4 * h;
-        uint32_t hi[4], lo[4];
+        const int j = task & 7, t = (task >> 3) & 3;
+        const int tok = (task >> 5) % batch, cb = (task >> 5) / batch;
+        const int s4 = j >> 1, h = j & 1;
+        const float up = mi.up[tok];
+        const float* v = vals + tok * vstride + cb * kCB + 32 * t + s4 + 4 * h;
+        uint32_t wh = 0, wl = 0;
         int qs = 0;
 #pragma unroll
-        for (int s4 = 0; s4 < 4; ++s4) {
-            uint32_t wh = 0, wl = 0;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int q = quantise(value(tok, c0 + s4 + 8 * c), up);
-                qs += q;
-                wh |= (uint32_t)((q >> 7) & 0xFF) << (8 * c);
-                wl |= (uint32_t)(q & 0x7F) << (8 * c);
-            }
-            hi[s4] = wh;
-            lo[s4] = wl;
+        for (int c = 0; c < 4; ++c) {
+            const int q = quantise(v[8 * c], up);
+            qs += q;
+            wh |= (uint32_t)((q >> 7) & 0xFF) << (8 * c);
+            wl |= (uint32_t)(q & 0x7F) << (8 * c);
         }
-        atomicAdd(&sm.misc->qsum[tok], qs);
+        for (int o = 16; o > 0; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+        if ((threadIdx.x & 31) == 0) atomicAdd(&mi.qsum[tok], qs);
         const int tg = tok >> 2, ti = tok & 3;
-        uint32_t* fh0 = reinterpret_cast<uint32_t*>(&sm.fr(cb, tg, 0, 8 * ti + t));
-        uint32_t* fh1 = reinterpret_cast<uint32_t*>(&sm.fr(cb, tg, 1, 8 * ti + t));
-        uint32_t* fl0 = reinterpret_cast<uint32_t*>(&sm.fr(cb, tg, 0, 8 * ti + 4 + t));
-        uint32_t* fl1 = reinterpret_cast<uint32_t*>(&sm.fr(cb, tg, 1, 8 * ti + 4 + t));
-        // word j = 2*s4 + h lives in half j >> 2 at component j & 3
-        fh0[h] = hi[0];
-        fh0[2 + h] = hi[1];
-        fh1[h] = hi[2];
-        fh1[2 + h] = hi[3];
-        fl0[h] = lo[0];
-        fl0[2 + h] = lo[1];
-        fl1[h] = lo[2];
-        fl1[2 + h] = lo[3];
+        // word j lives in half j >> 2 at component j & 3
+        reinterpret_cast<uint32_t*>(&frag_at<NTG>(frag, cb, tg, j >> 2, 8 * ti + t))[j & 3] = wh;
+        reinterpret_cast<uint32_t*>(&frag_at<NTG>(frag, cb, tg, j >> 2, 8 * ti + 4 + t))[j & 3] = wl;
     }
-}
-
-template <int NTG>
-__device__ __forceinline__ void zero_fragments(const Sm<NTG>& sm) {
-    for (int i = threadIdx.x; i < kChunkCB * NTG * 2 * 32; i += kThreads) sm.frag[i] = make_uint4(0, 0, 0, 0);
 }
 
 // One column block of a 16-row tile into accumulator set `acc`.
 template <int NTG>
-__device__ __forceinline__ void cb_mma(const Sm<NTG>& sm, uint32_t wa, uint32_t wb, int cb, int lane,
-                                       int (&acc)[NTG][4][4]) {
+__device__ __forceinline__ void cb_mma(uint4* frag, uint32_t wa, uint32_t wb, int cb, int lane, int (&acc)[NTG][4][4]) {
     const uint32_t a4 = wa >> 4, b4 = wb >> 4;
 #pragma unroll
     for (int tg = 0; tg < NTG; ++tg) {
-        const uint4 f0 = sm.fr(cb, tg, 0, lane), f1 = sm.fr(cb, tg, 1, lane);
+        const uint4 f0 = frag_at<NTG>(frag, cb, tg, 0, lane), f1 = frag_at<NTG>(frag, cb, tg, 1, lane);
         const uint32_t bf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
@@ -268,15 +224,16 @@ __device__ __forceinline__ void cb_mma(const Sm<NTG>& sm, uint32_t wa, uint32_t 
     }
 }
 
-// Accumulate one 16-row tile (rows r0.., staged in buffer `buf`) against column blocks
-// cb0, cb0 + step, ... < cb1 of the staged chunk.  Two accumulator sets alternate between
-// consecutive column blocks so that dependent MMAs are two blocks apart.
+// Accumulate one 16-row tile against column blocks cb0, cb0 + step, ... < cb1 of the
+// chunk's fragments.  wrow points at the tile's row 0, word 0 of the chunk; rows are
+// `stride` words apart.  Two accumulator sets alternate between consecutive column blocks
+// so that dependent MMAs are two blocks apart.
 template <int NTG>
-__device__ __forceinline__ void tile_mma(const Sm<NTG>& sm, int buf, int r0, int cb0, int cb1, int step,
+__device__ __forceinline__ void tile_mma(uint4* frag, const uint32_t* wrow, int stride, int cb0, int cb1, int step,
                                          int (&acc)[NTG][4][4]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const uint32_t* wa_row = sm.wrow(buf, r0 + g);
-    const uint32_t* wb_row = sm.wrow(buf, r0 + g + 8);
+    const uint32_t* wa_row = wrow + g * stride + t;
+    const uint32_t* wb_row = wa_row + 8 * stride;
     int acc2[NTG][4][4];
 #pragma unroll
     for (int tg = 0; tg < NTG; ++tg)
@@ -286,12 +243,12 @@ __device__ __forceinline__ void tile_mma(const Sm<NTG>& sm, int buf, int r0, int
             for (int i = 0; i < 4; ++i) acc2[tg][s][i] = 0;
     int cb = cb0;
     for (; cb + step < cb1; cb += 2 * step) {
-        const uint32_t wa0 = wa_row[4 * cb + t], wb0 = wb_row[4 * cb + t];
-        const uint32_t wa1 = wa_row[4 * (cb + step) + t], wb1 = wb_row[4 * (cb + step) + t];
-        cb_mma<NTG>(sm, wa0, wb0, cb, lane, acc);
-        cb_mma<NTG>(sm, wa1, wb1, cb + step, lane, acc2);
+        const uint32_t wa0 = wa_row[4 * cb], wb0 = wb_row[4 * cb];
+        const uint32_t wa1 = wa_row[4 * (cb + step)], wb1 = wb_row[4 * (cb + step)];
+        cb_mma<NTG>(frag, wa0, wb0, cb, lane, acc);
+        cb_mma<NTG>(frag, wa1, wb1, cb + step, lane, acc2);
     }
-    if (cb < cb1) cb_mma<NTG>(sm, wa_row[4 * cb + t], wb_row[4 * cb + t], cb, lane, acc);
+    if (cb < cb1) cb_mma<NTG>(frag, wa_row[4 * cb], wb_row[4 * cb], cb, lane, acc);
 #pragma unroll
     for (int tg = 0; tg < NTG; ++tg)
 #pragma unroll
@@ -333,50 +290,62 @@ __device__ __forceinline__ void zero_acc(int (&acc)[NTG][4][4]) {
 // adds them in split order (deterministic), then writes t and the block's max |t| per
 // token (stage 2 builds its exponent from those maxima).
 template <int NTG>
-__device__ __forceinline__ void stage1_fetch_x(const Sm<NTG>& sm, int buf, const DecLayer& L, int batch, int col0,
-                                               int ccols) {
-    const int per_tok = ccols / 8;  // 16-byte pieces
-    for (int i = threadIdx.x; i < (batch + 1) * per_tok; i += kThreads) {
-        const int tok = i / per_tok, p = i % per_tok;
-        if (tok < batch)
-            cp_async16(sm.xrow(buf, tok) + 8 * p, L.x + (int64_t)tok * L.n + col0 + 8 * p);
-        else
-            cp_async16(sm.s2row(buf) + 8 * p, L.s2 + col0 + 8 * p);
-    }
-}
-
-template <int NTG>
 __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant__ DecGroup grp) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    const Sm<NTG> sm(smem_raw, 1, grp.depth1, grp.batch);
-    DecMisc& mi = *sm.misc;
+    const int batch = grp.batch, depth = grp.depth1;
+    uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem_raw);
+    uint16_t* xbuf = reinterpret_cast<uint16_t*>(smem_raw + s1_w_bytes(depth));  // [depth][batch + 1][kChunk]
+    float* vbuf = reinterpret_cast<float*>(smem_raw + s1_w_bytes(depth) + s1_x_bytes(depth, batch));
+    uint4* frag = reinterpret_cast<uint4*>(smem_raw + s1_w_bytes(depth) + s1_x_bytes(depth, batch) + s1_v_bytes(batch));
+    Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(frag) + frag_bytes(NTG));
+
     const int li = find_layer(grp.s1_start, grp.count, blockIdx.x);
     const DecLayer& L = grp.L[li];
     const int local = blockIdx.x - grp.s1_start[li];
     const int rb = local / L.nsplit, sp = local % L.nsplit;
-    const int batch = grp.batch;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
     const int n = L.n, r = L.r;
     const int64_t wpr = n / 32;
     const int64_t row0 = (int64_t)rb * kRowsS1;
     const uint32_t* W = L.Vpk + row0 * wpr;
-    const int cbA = sp * L.cps, cbB = min(n / kCB, cbA + L.cps);
+    const int cbA = min(n / kCB, sp * L.cps), cbB = min(n / kCB, cbA + L.cps);
     const int nchunks = (cbB - cbA + kChunkCB - 1) / kChunkCB;
     auto chunk_cb = [&](int ch) { return min(kChunkCB, cbB - cbA - ch * kChunkCB); };
+    auto wchunk = [&](int buf) { return wbuf + (size_t)buf * kRowsS1 * kS1Stride; };
+    auto xchunk = [&](int buf, int tok) { return xbuf + ((size_t)buf * (batch + 1) + tok) * kChunk; };
+
+    auto fetch_w = [&](int ch) {  // weight rows of chunk ch into buffer ch % depth
+        const int per_row = chunk_cb(ch);  // 16-byte pieces (one per column block)
+        uint32_t* dst = wchunk(ch % depth);
+        const uint32_t* src = W + (int64_t)(cbA + ch * kChunkCB) * 4;
+        for (int i = threadIdx.x; i < kRowsS1 * per_row; i += kThreads) {
+            const int row = i / per_row, p = i % per_row;
+            cp_async16(dst + row * kS1Stride + 4 * p, src + row * wpr + 4 * p);
+        }
+    };
+    auto fetch_x = [&](int ch) {  // x rows (batch of them) and s2 of chunk ch; s2 goes in slot `batch`
+        const int per_tok = chunk_cb(ch) * kCB / 8;
+        const int col0 = (cbA + ch * kChunkCB) * kCB;
+        for (int i = threadIdx.x; i < (batch + 1) * per_tok; i += kThreads) {
+            const int tok = i / per_tok, p = i % per_tok;
+            const uint16_t* src = tok < batch ? L.x + (int64_t)tok * n + col0 + 8 * p : L.s2 + col0 + 8 * p;
+            cp_async16(xchunk(ch % depth, tok) + 8 * p, src);
+        }
+    };
 
     // weights first: they do not depend on the previous kernel
-    stage_weights(sm, 0, W, wpr, kRowsS1, (int64_t)cbA * 4, chunk_cb(0) * 4);
+    if (nchunks > 0) fetch_w(0);
     cp_async_commit();
-    if (nchunks > 1) stage_weights(sm, 1, W, wpr, kRowsS1, (int64_t)(cbA + kChunkCB) * 4, chunk_cb(1) * 4);
+    if (nchunks > 1) fetch_w(1);
     cp_async_commit();
     if (nchunks > 2 && threadIdx.x < kRowsS1)
         prefetch_l2(W + threadIdx.x * wpr + (cbA + 2 * kChunkCB) * 4, (uint32_t)((cbB - cbA - 2 * kChunkCB) * 16));
-    zero_fragments(sm);
+    zero_fragments<NTG>(frag);
     pdl_trigger();
     pdl_wait();  // x may come from the previous kernel on the stream
-    stage1_fetch_x(sm, 0, L, batch, cbA * kCB, chunk_cb(0) * kCB);
+    if (nchunks > 0) fetch_x(0);
     cp_async_commit();
-    if (nchunks > 1) stage1_fetch_x(sm, 1, L, batch, (cbA + kChunkCB) * kCB, chunk_cb(1) * kCB);
+    if (nchunks > 1) fetch_x(1);
     cp_async_commit();
 
     float part[NTG][2];
@@ -384,34 +353,43 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
     for (int tg = 0; tg < NTG; ++tg) part[tg][0] = part[tg][1] = 0.f;
 
     for (int ch = 0; ch < nchunks; ++ch) {
-        const int buf = ch & 1;
+        const int buf = ch % depth;
         const int ncb = chunk_cb(ch);
         const int ccols = ncb * kCB;
         if (ch + 1 < nchunks) cp_async_wait<1>(); else cp_async_wait<0>();
         __syncthreads();
-        // per-token max of s2 * x over the chunk
-        const uint16_t* xs = sm.xrow(buf, 0);
-        const uint16_t* ss = sm.s2row(buf);
-        for (int tok = warp; tok < batch; tok += kWarps) {
+        // v = s2 * x (exact in fp32) and its per-token max: every thread takes a column
+        // stripe of every token, then the four warps' maxima are combined
+        const uint16_t* ss = xchunk(buf, batch);
+        for (int tok = 0; tok < batch; ++tok) {
+            const uint16_t* xs = xchunk(buf, tok);
+            float* vs = vbuf + tok * kChunk;
             float mx = 0.f;
-            for (int c = lane; c < ccols; c += 32) mx = fmaxf(mx, fabsf(bf16_to_f32(xs[tok * kChunk + c]) * f16_to_f32(ss[c])));
-            mx = warp_max(mx);
-            if (lane == 0) {
-                const int e = range_exponent(mx);
-                mi.e[tok] = e;
-                mi.up[tok] = pow2f(kQBits - e);
-                mi.qsum[tok] = 0;
+            for (int c = threadIdx.x; c < ccols; c += kThreads) {
+                const float v = bf16_to_f32(xs[c]) * f16_to_f32(ss[c]);
+                vs[c] = v;
+                mx = fmaxf(mx, fabsf(v));
             }
+            mx = warp_max(mx);
+            if (lane == 0) mi.red[warp][tok] = mx;
         }
         __syncthreads();
-        build_fragments(sm, ncb, batch, [&](int tok, int c) {
-            return bf16_to_f32(xs[tok * kChunk + c]) * f16_to_f32(ss[c]);
-        });
+        if (threadIdx.x < batch) {
+            const int tok = threadIdx.x;
+            float mx = mi.red[0][tok];
+            for (int w = 1; w < kWarps; ++w) mx = fmaxf(mx, mi.red[w][tok]);
+            const int e = range_exponent(mx);
+            mi.e[tok] = e;
+            mi.up[tok] = pow2f(kQBits - e);
+            mi.qsum[tok] = 0;
+        }
+        __syncthreads();
+        build_fragments<NTG>(frag, mi, vbuf, kChunk, ncb, batch);
         __syncthreads();
 
         int acc[NTG][4][4];
         zero_acc<NTG>(acc);
-        tile_mma<NTG>(sm, buf, 16 * warp, 0, ncb, 1, acc);
+        tile_mma<NTG>(frag, wchunk(buf) + 16 * warp * kS1Stride, kS1Stride, 0, ncb, 1, acc);
 #pragma unroll
         for (int tg = 0; tg < NTG; ++tg) {
             const int tok = 4 * tg + tq;
@@ -426,9 +404,8 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
         }
         __syncthreads();  // buffers are free again
         if (ch + 2 < nchunks) {
-            const int cb2 = cbA + (ch + 2) * kChunkCB;
-            stage_weights(sm, buf, W, wpr, kRowsS1, (int64_t)cb2 * 4, chunk_cb(ch + 2) * 4);
-            stage1_fetch_x(sm, buf, L, batch, cb2 * kCB, chunk_cb(ch + 2) * kCB);
+            fetch_w(ch + 2);
+            fetch_x(ch + 2);
             cp_async_commit();
         }
     }
@@ -485,28 +462,22 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
 }
 
 // ------------------------------------------------------------------ stage 2
-// CTA = RT row tiles x KS = 4/RT k-parts of one layer.  One quantisation exponent per
-// token for the whole of t (from stage 1's maxima), so integer sums run across all
-// chunks and k-parts and are converted once, in the epilogue.
-template <int NTG>
-__device__ __forceinline__ void stage2_fetch_t(const Sm<NTG>& sm, int buf, const DecLayer& L, int batch, int col0,
-                                               int ccols) {
-    const int per_tok = ccols / 4;  // 16-byte pieces
-    for (int i = threadIdx.x; i < batch * per_tok; i += kThreads) {
-        const int tok = i / per_tok, p = i % per_tok;
-        cp_async16(sm.trow(buf, tok) + 4 * p, L.t + (int64_t)tok * L.r + col0 + 4 * p);
-    }
-}
-
+// CTA = RT row tiles x KS = 4/RT k-parts of one layer.  The CTA's weight rows for up to
+// r2 columns are copied on chip before the dependency wait, and t for those columns right
+// after it.  One quantisation exponent per token for the whole of t (from stage 1's
+// maxima), so integer sums run across all chunks and k-parts and are converted once.
 template <int NTG>
 __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant__ DecGroup grp) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    const Sm<NTG> sm(smem_raw, 2, grp.depth2, grp.batch);
-    DecMisc& mi = *sm.misc;
+    const int batch = grp.batch, r2 = grp.r2, ws = grp.w2stride;
+    uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem_raw);
+    float* tbuf = reinterpret_cast<float*>(smem_raw + s2_w_bytes(ws));
+    uint4* frag = reinterpret_cast<uint4*>(smem_raw + s2_w_bytes(ws) + s2_t_bytes(batch, r2));
+    Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(frag) + frag_bytes(NTG));
+
     const int li = find_layer(grp.s2_start, grp.count, blockIdx.x);
     const DecLayer& L = grp.L[li];
     const int blk = blockIdx.x - grp.s2_start[li];
-    const int batch = grp.batch;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
     const int RT = L.rt, KS = kWarps / RT;
     const int rt = warp / KS, kp = warp % KS;
@@ -515,22 +486,34 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
     const int rows = 16 * RT;
     const int64_t row0 = (int64_t)blk * rows;
     const uint32_t* W = L.Upk + row0 * wpr;
-    const int nchunks = (r + kChunk - 1) / kChunk;
-    auto chunk_cols = [&](int ch) { return min(kChunk, r - ch * kChunk); };
+    const int nsc = (r + r2 - 1) / r2;  // column spans held on chip one after the other
 
-    stage_weights(sm, 0, W, wpr, rows, 0, chunk_cols(0) / 32);
+    auto fetch_w = [&](int sc) {
+        const int cols = min(r2, r - sc * r2);
+        const int per_row = cols / 128;  // 16-byte pieces
+        for (int i = threadIdx.x; i < rows * per_row; i += kThreads) {
+            const int row = i / per_row, p = i % per_row;
+            cp_async16(wbuf + row * ws + 4 * p, W + row * wpr + sc * (r2 / 32) + 4 * p);
+        }
+    };
+    auto fetch_t = [&](int sc) {
+        const int cols = min(r2, r - sc * r2);
+        const int per_tok = cols / 4;
+        for (int i = threadIdx.x; i < batch * per_tok; i += kThreads) {
+            const int tok = i / per_tok, p = i % per_tok;
+            cp_async16(tbuf + tok * r2 + 4 * p, L.t + (int64_t)tok * r + sc * r2 + 4 * p);
+        }
+    };
+
+    fetch_w(0);
     cp_async_commit();
-    if (nchunks > 1) stage_weights(sm, 1, W, wpr, rows, kChunkWords, chunk_cols(1) / 32);
-    cp_async_commit();
-    if (nchunks > 2 && threadIdx.x < rows)
-        prefetch_l2(W + threadIdx.x * wpr + 2 * kChunkWords, (uint32_t)((r - 2 * kChunk) / 8));
+    if (nsc > 1 && threadIdx.x < rows)
+        prefetch_l2(W + threadIdx.x * wpr + r2 / 32, (uint32_t)((r - r2) / 8));
     for (int i = threadIdx.x; i < 64 * 8; i += kThreads) (&mi.bq[0][0])[i] = 0;
-    zero_fragments(sm);
+    zero_fragments<NTG>(frag);
     pdl_trigger();
     pdl_wait();  // t and its maxima come from stage 1
-    stage2_fetch_t(sm, 0, L, batch, 0, chunk_cols(0));
-    cp_async_commit();
-    if (nchunks > 1) stage2_fetch_t(sm, 1, L, batch, kChunk, chunk_cols(1));
+    fetch_t(0);
     cp_async_commit();
 
     // global max |t| per token from the per-block maxima (one warp per token)
@@ -549,21 +532,22 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
 
     int acc[NTG][4][4];
     zero_acc<NTG>(acc);
-    for (int ch = 0; ch < nchunks; ++ch) {
-        const int buf = ch & 1;
-        const int ccols = chunk_cols(ch);
-        const int ncb = ccols / kCB;
-        if (ch + 1 < nchunks) cp_async_wait<1>(); else cp_async_wait<0>();
-        __syncthreads();
-        const float* ts = sm.trow(buf, 0);
-        build_fragments(sm, ncb, batch, [&](int tok, int c) { return ts[tok * kChunk + c]; });
-        __syncthreads();
-        tile_mma<NTG>(sm, buf, 16 * rt, kp, ncb, KS, acc);
-        __syncthreads();
-        if (ch + 2 < nchunks) {
-            stage_weights(sm, buf, W, wpr, rows, (int64_t)(ch + 2) * kChunkWords, chunk_cols(ch + 2) / 32);
-            stage2_fetch_t(sm, buf, L, batch, (ch + 2) * kChunk, chunk_cols(ch + 2));
+    for (int sc = 0; sc < nsc; ++sc) {
+        if (sc > 0) {
+            __syncthreads();  // the previous span is consumed
+            fetch_w(sc);
+            fetch_t(sc);
             cp_async_commit();
+        }
+        cp_async_wait<0>();
+        __syncthreads();
+        const int cols = min(r2, r - sc * r2);
+        for (int c0 = 0; c0 < cols; c0 += kChunk) {
+            const int ncb = min(kChunk, cols - c0) / kCB;
+            build_fragments<NTG>(frag, mi, tbuf + c0, r2, ncb, batch);
+            __syncthreads();
+            tile_mma<NTG>(frag, wbuf + 16 * rt * ws + c0 / 32, ws, kp, ncb, KS, acc);
+            __syncthreads();
         }
     }
 
@@ -591,13 +575,15 @@ int launch_group(DecGroup& grp, cudaStream_t stream, int device) {
     static unsigned long long init_mask = 0;  // devices whose kernel attributes are set
     const unsigned long long bit = 1ull << (device & 63);
     if (!(__atomic_load_n(&init_mask, __ATOMIC_ACQUIRE) & bit)) {
-        const int most = (int)smem_bytes(2, 2, 4 * NTG, NTG);  // the largest layout either stage uses
+        const int most = 200 * 1024;
         if (cudaFuncSetAttribute(stage1_kernel<NTG>, cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess ||
             cudaFuncSetAttribute(stage2_kernel<NTG>, cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess)
             return NQ_ERR_CUDA;
         __atomic_fetch_or(&init_mask, bit, __ATOMIC_RELEASE);
     }
-    const size_t smem1 = smem_bytes(1, grp.depth1, grp.batch, NTG), smem2 = smem_bytes(2, grp.depth2, grp.batch, NTG);
+    const size_t smem1 = s1_bytes(grp.depth1, grp.batch, NTG);
+    const size_t smem2 = s2_bytes(grp.w2stride, grp.batch, grp.r2, NTG);
+
     if (launch_pdl(stage1_kernel<NTG>, dim3((unsigned)grp.s1_start[grp.count]), dim3(kThreads), smem1, stream, grp) !=
         cudaSuccess)
         return NQ_ERR_CUDA;
@@ -615,8 +601,20 @@ static int stage2_rt(int64_t total_tiles) {
     return total_tiles >= 12 * sms ? 4 : (total_tiles >= 4 * sms ? 2 : 1);
 }
 
+// Stage-2 columns held on chip at a time: all of r when it fits (up to 4096 columns, less
+// for larger batches since t takes batch x r2 x 4 bytes), else spans of a multiple of kChunk.
+static int stage2_span(int64_t r_max, int64_t batch) {
+    int64_t span = 8192 / batch;
+    span = span / kChunk * kChunk;
+    if (span > 4096) span = 4096;
+    if (span < kChunk) span = kChunk;
+    const int64_t need = (r_max + kCB - 1) / kCB * kCB;
+    return (int)(need < span ? need : span);
+}
+
 // Column blocks per stage-1 split: about two CTAs per SM over the whole launch, at least
-// 4 and (while the split count stays <= max_splits) at most kChunkCB column blocks per CTA.
+// 4 and (while the split count stays <= max_splits) at most kChunkCB column blocks per CTA,
+// so that every CTA does one chunk.
 static int stage1_cps(const DecodeCall* calls, int count, int max_splits) {
     int64_t units = 0, max_ncb = 0;
     for (int i = 0; i < count; ++i) {
@@ -659,10 +657,17 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
     DecGroup grp;
     grp.count = count;
     grp.batch = (int)batch;
-    int64_t tiles = 0;
-    for (int i = 0; i < count; ++i) tiles += calls[i].m / 16;
+    int64_t tiles = 0, r_max = 0;
+    for (int i = 0; i < count; ++i) {
+        tiles += calls[i].m / 16;
+        r_max = calls[i].r > r_max ? calls[i].r : r_max;
+    }
     const int rt = stage2_rt(tiles);
     const int cps = stage1_cps(calls, count, max_splits);
+    grp.r2 = stage2_span(r_max, batch);
+    // an odd number of 4-word groups per row spreads the 8 rows a warp reads over all 32 banks
+    grp.w2stride = grp.r2 / 32 + (((grp.r2 / 128) % 2) ? 0 : 4);
+    grp.depth1 = cps > kChunkCB ? 2 : 1;
     size_t toff = 0, goff = 0, poff = 0, coff = 0;
     grp.s1_start[0] = grp.s2_start[0] = 0;
     for (int i = 0; i < count; ++i) {
@@ -691,15 +696,6 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
         grp.s1_start[i + 1] = grp.s1_start[i] + (int)(c.r / kRowsS1) * L.nsplit;
         grp.s2_start[i + 1] = grp.s2_start[i] + (int)(c.m / (16 * rt));
     }
-    int max_c1 = 1, max_c2 = 1;
-    for (int i = 0; i < count; ++i) {
-        const int c1 = (cps + kChunkCB - 1) / kChunkCB;
-        const int c2 = (int)((calls[i].r + kChunk - 1) / kChunk);
-        max_c1 = c1 > max_c1 ? c1 : max_c1;
-        max_c2 = c2 > max_c2 ? c2 : max_c2;
-    }
-    grp.depth1 = max_c1 > 1 ? 2 : 1;
-    grp.depth2 = max_c2 > 1 ? 2 : 1;
     if (batch <= 4) return launch_group<1>(grp, stream, ws->device);
     return launch_group<2>(grp, stream, ws->device);
 }
@@ -720,8 +716,9 @@ int decode_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, 
 // engine that sized and froze its memory pool at start-up, a process whose allocator is
 // owned by another framework, or code running under a stream capture that must not call
 // cudaMalloc.  For them nq_lowrank_linear_fwd_noalloc keeps the decode path's scratch
-// (t, per-block maxima, stage-1 split partials, arrival counters) in one fixed array of
-// device memory that is part of this library's module, so a call allocates nothing.
+// (t, the per-block maxima of |t|, the stage-1 split partials and arrival counters) in one
+// fixed array of device memory that is part of this library's module, so a call allocates
+// nothing.
 //
 // The array is a file-scope __device__ variable: every GPU that loads the library holds
 // it until the process exits.  Host code may not use its name as an address (on the host
