@@ -253,7 +253,10 @@ def run_ours(args):
     from binary_rank_linear_02_b200 import nq
 
     peaks = load_peaks()
-    layers = synth.LLAMA2_7B_LAYERS
+    if args.workload == "prefill":
+        return run_prefill_only(args, device, peaks)
+    layers = synth.LLAMA2_70B_LAYERS if args.workload == "decode70b" else synth.LLAMA2_7B_LAYERS
+    model = "llama2-70b" if args.workload == "decode70b" else "llama2-7b"
     batch = args.batch
     work = DecodeWorkload(layers, batch, seed=1234 + rank, device=device)
     stream = torch.cuda.Stream(device)
@@ -270,7 +273,27 @@ def run_ours(args):
     value = total_bytes / (ms_max * 1e-3) / 1e9
     tokens_per_s = batch * args.steps * world / (ms_max * 1e-3)
 
-    # roofline: the largest layer (gate) alone, back to back over its own rotating copies
+    # roofline: the kernels of the headline step (the stage-1 and stage-2 kernels of one
+    # grouped call, timed live above), against the measured HBM copy bandwidth
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if os.path.exists(tpath) and batch == 1 and args.workload == "decode7b":
+        import hashlib
+
+        with open(tpath) as f:
+            rec = json.load(f)
+        with open(os.path.join(ROOT, rec["kernel_source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        if sha == rec["kernel_source_sha256_16"]:  # counters are only valid for the kernel they came from
+            traffic = rec["dram_bytes_per_step_b1"]
+    achieved = value / world
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "kernel": f"stage1_kernel + stage2_kernel of one grouped call ({work.step_bytes} packed bytes "
+                          "per launch pair), per-GPU",
+                "peak_source": peaks["source"]}
+
+    # the largest layer (gate) alone, back to back over its own rotating copies
     gate = [l for l in layers if l[0] == "gate"][0]
     _, gm, gn, gr = gate
     gwork = DecodeWorkload([gate], batch, seed=777 + rank, device=device)
@@ -280,29 +303,29 @@ def run_ours(args):
     r_steps = max(gwork.copies * 10, 500)
     ms_gate = timed_graphs(gwork, r_steps, args.warmup, stream)
     del gwork
-    gate_bytes = packed_bytes(gm, gn, gr)
-    achieved = gate_bytes * r_steps / (ms_gate * 1e-3) / 1e9
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            traffic = json.load(f).get("gate_b%d_dram_bytes_per_call" % batch)
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-                "kernel": f"decode layer {gm}x{gn} r={gr} batch {batch} (stage-1 + stage-2 kernels)",
-                "peak_source": peaks["source"]}
+    gate_gbs = packed_bytes(gm, gn, gr) * r_steps / (ms_gate * 1e-3) / 1e9
 
     # end to end through the public API with host buffers (pinned), synchronous per call
     e2e = run_e2e(work, stream, min(args.steps, 100), device)
 
     # secondary: the same step as seven separate nq_lowrank_linear_fwd calls; batch 8
-    secondary = {}
+    secondary = {"decode_%s_gate_alone_b%d_gbs" % (model, batch): round(gate_gbs, 1)}
     if args.secondary and world == 1:
         work.grouped = False
         ms1 = timed_graphs(work, args.steps, args.warmup, stream)
         work.grouped = True
         secondary["decode_b%d_per_layer_calls_gbs" % batch] = round(work.step_bytes * args.steps / (ms1 * 1e-3) / 1e9, 1)
-    if args.secondary and batch == 1 and world == 1:
+    if args.secondary and batch == 1 and world == 1 and args.workload == "decode7b":
+        for b70 in (1, 4):  # the Llama-2-70B-shaped block, batch 1 and 4
+            w70 = DecodeWorkload(synth.LLAMA2_70B_LAYERS, b70, seed=70 + b70, device=device)
+            with torch.cuda.stream(stream):
+                w70.step(0, stream.cuda_stream)
+            torch.cuda.synchronize()
+            st70 = max(w70.copies, min(args.steps, 400) // w70.copies * w70.copies)
+            ms70 = timed_graphs(w70, st70, args.warmup, stream)
+            secondary["decode70b_b%d_gbs" % b70] = round(w70.step_bytes * st70 / (ms70 * 1e-3) / 1e9, 1)
+            secondary["decode70b_b%d_tokens_per_s" % b70] = round(b70 * st70 / (ms70 * 1e-3), 1)
+            del w70
         w8 = DecodeWorkload(layers, 8, seed=99, device=device)
         with torch.cuda.stream(stream):
             w8.step(0, stream.cuda_stream)
@@ -326,8 +349,8 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in; int8x2-limb tensor-core products, int32/fp32 acc",
             "data": "synthetic",
-            "config": {"workload": f"llama2-7b-shaped decode, batch {batch}: 7 factorised linears per step "
-                                   "(q/k/v/o 4096x4096 r1664, gate/up 11008x4096 r2432, down 4096x11008 r2432), "
+            "config": {"workload": f"{model}-shaped decode, batch {batch}: 7 factorised linears per step "
+                                   f"({', '.join(f'{nm} {m}x{n} r{r}' for nm, m, n, r in layers)}), "
                                    "one nq_lowrank_linear_fwd_grouped call per step",
                        "batch": batch, "packed_bytes_per_step": work.step_bytes,
                        "l2": f"weights rotate over {work.copies} seeded copies "
@@ -344,7 +367,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_prefill_sweep(device, stream, warmup, peaks, calls=20):
+def run_prefill_sweep(device, stream, warmup, peaks, calls=20, batches=synth.PREFILL_BATCHES):
     """Config-4 sweep: the 11008x4096 r=2432 layer at token batches 16..4096 (tcgen05 path)."""
     import torch
 
@@ -358,7 +381,7 @@ def run_prefill_sweep(device, stream, warmup, peaks, calls=20):
     s1 = torch.from_numpy(synth.scales_f16(m, 4242, "s1").view(np.int16)).to(device)
     s2 = torch.from_numpy(synth.scales_f16(n, 4242, "s2").view(np.int16)).to(device)
     out = {}
-    for b in synth.PREFILL_BATCHES:
+    for b in batches:
         x = torch.from_numpy(synth.activations_bf16(b, n, 4242, b).view(np.int16)).to(device)
         y = torch.empty((b, m), dtype=torch.float32, device=device)
         nq.workspace_reserve(m, n, r, b)
@@ -394,6 +417,21 @@ def run_prefill_sweep(device, stream, warmup, peaks, calls=20):
                        "tokens_per_s": round(b / (ms * 1e-3), 1)}
         del g, x, y
     return out
+
+
+def run_prefill_only(args, device, peaks):
+    """--workload prefill: the config-4 sweep alone (or one batch), one JSON line, TFLOP/s."""
+    import torch
+
+    stream = torch.cuda.Stream(device)
+    sweep = run_prefill_sweep(device, stream, args.warmup, peaks, calls=max(1, args.steps),
+                              batches=(args.prefill_batch,) if args.prefill_batch else synth.PREFILL_BATCHES)
+    top = str(max(int(b) for b in sweep))
+    line = {"metric": METRIC, "value": sweep[top]["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp16 tcgen05 operands, fp32 accumulate", "data": "synthetic",
+            "config": {"workload": f"prefill 11008x4096 r=2432, token batch {top}"}, "prefill": sweep}
+    print(json.dumps(line), flush=True)
 
 
 def run_e2e(work, stream, steps, device):
@@ -485,6 +523,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", dest="secondary", action="store_false")
+    ap.add_argument("--workload", choices=["decode7b", "decode70b", "prefill"], default="decode7b")
+    ap.add_argument("--prefill-batch", type=int, default=0)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
