@@ -46,14 +46,14 @@
 namespace nq {
 namespace {
 
-constexpr int kThreads = 128;          // 4 warps
+constexpr int kThreads = 256;          // 8 warps
 constexpr int kWarps = kThreads / 32;
 constexpr int kCB = 128;               // columns per column block
 constexpr int kChunk = 1024;           // columns per fragment chunk
 constexpr int kChunkCB = kChunk / kCB;
 constexpr int kChunkWords = kChunk / 32;
 constexpr int kQBits = 14;             // |q| < 2^14
-constexpr int kRowsS1 = 64;            // stage-1 rows per CTA (4 warps x 16)
+constexpr int kRowsS1 = 128;           // stage-1 rows per CTA (8 warps x 16)
 constexpr int kS1Stride = kChunkWords + 4;  // words per staged stage-1 row (36: bank-spread)
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
@@ -109,13 +109,13 @@ struct DecLayer {
     const uint16_t* s2;
     float* y;
     float* t;        // workspace: batch x r
-    float* tgmax;    // workspace: batch x r/64 (max |t| per 64-row block)
+    float* tgmax;    // workspace: batch x r/128 (max |t| per 128-row block)
     float* partials; // workspace: nsplit x batch x r (stage-1 column splits)
-    int* counters;   // workspace: r/64 arrival counters, zero between calls
+    int* counters;   // workspace: r/128 arrival counters, zero between calls
     int m, n, r;
-    int nsplit;      // stage 1: CTAs per 64-row block (column splits)
+    int nsplit;      // stage 1: CTAs per 128-row block (column splits)
     int cps;         // stage 1: column blocks per split
-    int rt;          // stage 2: row tiles per CTA (4/rt k-parts per tile)
+    int rt;          // stage 2: row tiles per CTA (8/rt k-parts per tile)
 };
 
 struct DecGroup {
@@ -142,25 +142,27 @@ struct Misc {
     int e[8];
     float up[8];             // 2^(14 - e): quantisation factor per token
     int qsum[8];
-    int bq[64][8];           // stage 2: per (row, token) across k-parts
-    float res[8][kRowsS1];   // stage 1: the CTA's partial sums of its 64 rows
+    union {
+        int bq[kRowsS1][8];      // stage 2: per (row, token) across k-parts
+        float res[8][kRowsS1];   // stage 1: the CTA's partial sums of its rows
+    };
     int last;
 };
 
-__host__ __device__ inline size_t frag_bytes(int ntg) { return (size_t)kChunkCB * ntg * 2 * 32 * 16; }
+__host__ __device__ inline size_t frag_bytes(int ncb, int ntg) { return (size_t)ncb * ntg * 2 * 32 * 16; }
 
-// stage 1: w [depth][64][36] | x [depth][batch + 1][1024] bf16 (slot batch = s2) | v [batch][1024] f32 | frag | misc
+// stage 1: w [depth][128][36] | x [depth][batch + 1][1024] bf16 (slot batch = s2) | v [batch][1024] f32 | frag (8 CBs) | misc
 __host__ __device__ inline size_t s1_w_bytes(int depth) { return (size_t)depth * kRowsS1 * kS1Stride * 4; }
 __host__ __device__ inline size_t s1_x_bytes(int depth, int batch) { return (size_t)depth * (batch + 1) * kChunk * 2; }
 __host__ __device__ inline size_t s1_v_bytes(int batch) { return (size_t)batch * kChunk * 4; }
 __host__ __device__ inline size_t s1_bytes(int depth, int batch, int ntg) {
-    return s1_w_bytes(depth) + s1_x_bytes(depth, batch) + s1_v_bytes(batch) + frag_bytes(ntg) + sizeof(Misc);
+    return s1_w_bytes(depth) + s1_x_bytes(depth, batch) + s1_v_bytes(batch) + frag_bytes(kChunkCB, ntg) + sizeof(Misc);
 }
-// stage 2: w [64][w2stride] | t [batch][r2] f32 | frag | misc
+// stage 2: w [128][w2stride] | t [batch][r2] f32 | frag (all r2/128 CBs) | misc
 __host__ __device__ inline size_t s2_w_bytes(int w2stride) { return (size_t)kRowsS1 * w2stride * 4; }
 __host__ __device__ inline size_t s2_t_bytes(int batch, int r2) { return (size_t)batch * r2 * 4; }
 __host__ __device__ inline size_t s2_bytes(int w2stride, int batch, int r2, int ntg) {
-    return s2_w_bytes(w2stride) + s2_t_bytes(batch, r2) + frag_bytes(ntg) + sizeof(Misc);
+    return s2_w_bytes(w2stride) + s2_t_bytes(batch, r2) + frag_bytes(r2 / kCB, ntg) + sizeof(Misc);
 }
 
 template <int NTG>
@@ -169,8 +171,8 @@ __device__ __forceinline__ uint4& frag_at(uint4* frag, int cb, int tg, int half,
 }
 
 template <int NTG>
-__device__ __forceinline__ void zero_fragments(uint4* frag) {
-    for (int i = threadIdx.x; i < kChunkCB * NTG * 2 * 32; i += kThreads) frag[i] = make_uint4(0, 0, 0, 0);
+__device__ __forceinline__ void zero_fragments(uint4* frag, int ncb) {
+    for (int i = threadIdx.x; i < ncb * NTG * 2 * 32; i += kThreads) frag[i] = make_uint4(0, 0, 0, 0);
 }
 
 // B fragments of `ncb` column blocks from fp32 values vals[tok * vstride + col] (col from
@@ -297,7 +299,7 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
     uint16_t* xbuf = reinterpret_cast<uint16_t*>(smem_raw + s1_w_bytes(depth));  // [depth][batch + 1][kChunk]
     float* vbuf = reinterpret_cast<float*>(smem_raw + s1_w_bytes(depth) + s1_x_bytes(depth, batch));
     uint4* frag = reinterpret_cast<uint4*>(smem_raw + s1_w_bytes(depth) + s1_x_bytes(depth, batch) + s1_v_bytes(batch));
-    Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(frag) + frag_bytes(NTG));
+    Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(frag) + frag_bytes(kChunkCB, NTG));
 
     const int li = find_layer(grp.s1_start, grp.count, blockIdx.x);
     const DecLayer& L = grp.L[li];
@@ -340,7 +342,7 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
     cp_async_commit();
     if (nchunks > 2 && threadIdx.x < kRowsS1)
         prefetch_l2(W + threadIdx.x * wpr + (cbA + 2 * kChunkCB) * 4, (uint32_t)((cbB - cbA - 2 * kChunkCB) * 16));
-    zero_fragments<NTG>(frag);
+    zero_fragments<NTG>(frag, kChunkCB);
     pdl_trigger();
     pdl_wait();  // x may come from the previous kernel on the stream
     if (nchunks > 0) fetch_x(0);
@@ -453,16 +455,20 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
     }
     // t and the block's max |t| per token (one warp per token)
     for (int tok = warp; tok < batch; tok += kWarps) {
-        const float a = mi.res[tok][lane], b = mi.res[tok][lane + 32];
-        L.t[(int64_t)tok * r + row0 + lane] = a;
-        L.t[(int64_t)tok * r + row0 + lane + 32] = b;
-        const float v = warp_max(fmaxf(fabsf(a), fabsf(b)));
+        float v = 0.f;
+#pragma unroll
+        for (int q = 0; q < kRowsS1 / 32; ++q) {
+            const float a = mi.res[tok][lane + 32 * q];
+            L.t[(int64_t)tok * r + row0 + lane + 32 * q] = a;
+            v = fmaxf(v, fabsf(a));
+        }
+        v = warp_max(v);
         if (lane == 0) L.tgmax[(int64_t)tok * nrb + rb] = v;
     }
 }
 
 // ------------------------------------------------------------------ stage 2
-// CTA = RT row tiles x KS = 4/RT k-parts of one layer.  The CTA's weight rows for up to
+// CTA = RT row tiles x KS = 8/RT k-parts of one layer.  The CTA's weight rows for up to
 // r2 columns are copied on chip before the dependency wait, and t for those columns right
 // after it.  One quantisation exponent per token for the whole of t (from stage 1's
 // maxima), so integer sums run across all chunks and k-parts and are converted once.
@@ -473,7 +479,7 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
     uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem_raw);
     float* tbuf = reinterpret_cast<float*>(smem_raw + s2_w_bytes(ws));
     uint4* frag = reinterpret_cast<uint4*>(smem_raw + s2_w_bytes(ws) + s2_t_bytes(batch, r2));
-    Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(frag) + frag_bytes(NTG));
+    Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(frag) + frag_bytes(r2 / kCB, NTG));
 
     const int li = find_layer(grp.s2_start, grp.count, blockIdx.x);
     const DecLayer& L = grp.L[li];
@@ -509,8 +515,8 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
     cp_async_commit();
     if (nsc > 1 && threadIdx.x < rows)
         prefetch_l2(W + threadIdx.x * wpr + r2 / 32, (uint32_t)((r - r2) / 8));
-    for (int i = threadIdx.x; i < 64 * 8; i += kThreads) (&mi.bq[0][0])[i] = 0;
-    zero_fragments<NTG>(frag);
+    for (int i = threadIdx.x; i < kRowsS1 * 8; i += kThreads) (&mi.bq[0][0])[i] = 0;
+    zero_fragments<NTG>(frag, r2 / kCB);
     pdl_trigger();
     pdl_wait();  // t and its maxima come from stage 1
     fetch_t(0);
@@ -541,14 +547,11 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
         }
         cp_async_wait<0>();
         __syncthreads();
-        const int cols = min(r2, r - sc * r2);
-        for (int c0 = 0; c0 < cols; c0 += kChunk) {
-            const int ncb = min(kChunk, cols - c0) / kCB;
-            build_fragments<NTG>(frag, mi, tbuf + c0, r2, ncb, batch);
-            __syncthreads();
-            tile_mma<NTG>(frag, wbuf + 16 * rt * ws + c0 / 32, ws, kp, ncb, KS, acc);
-            __syncthreads();
-        }
+        // every column block of the span at once: one barrier, then an uninterrupted MMA loop
+        const int ncb = min(r2, r - sc * r2) / kCB;
+        build_fragments<NTG>(frag, mi, tbuf, r2, ncb, batch);
+        __syncthreads();
+        tile_mma<NTG>(frag, wbuf + 16 * rt * ws, ws, kp, ncb, KS, acc);
     }
 
 #pragma unroll
@@ -595,10 +598,12 @@ int launch_group(DecGroup& grp, cudaStream_t stream, int device) {
 
 }  // namespace
 
-// Stage-2 row tiles per CTA: fewer rows (more k-parts) when the launch has few rows.
+// Stage-2 row tiles per CTA: the most rows per CTA that still leaves about two CTAs per SM.
 static int stage2_rt(int64_t total_tiles) {
-    const int64_t sms = sm_count();
-    return total_tiles >= 12 * sms ? 4 : (total_tiles >= 4 * sms ? 2 : 1);
+    const int64_t want = 2 * (int64_t)sm_count();
+    for (int rt = kWarps; rt > 1; rt /= 2)
+        if (total_tiles / rt >= want) return rt;
+    return 1;
 }
 
 // Stage-2 columns held on chip at a time: all of r when it fits (up to 4096 columns, less
