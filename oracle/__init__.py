@@ -53,6 +53,10 @@ def _load(path: str) -> ctypes.CDLL:
     L.orc_f16_to_double.argtypes = [ctypes.c_uint16]
     L.orc_f16_to_double.restype = ctypes.c_double
     L.orc_num_threads.restype = ctypes.c_int
+    L.orc_round_to_bf16.argtypes = [ctypes.c_double]
+    L.orc_round_to_bf16.restype = ctypes.c_uint16
+    L.orc_round_array_bf16.argtypes = [p, i64, p]
+    L.orc_rms_normalize_bf16.argtypes = [p, i64, i64, p]
     return L
 
 
@@ -136,6 +140,51 @@ class Oracle:
 
     def num_threads(self) -> int:
         return self.lib.orc_num_threads()
+
+    # ---------------------------------------------------------------- decode chain
+
+    def round_to_bf16(self, v) -> np.ndarray:
+        """Nearest bfloat16 bit patterns (ties to even) of an array of doubles."""
+        a = np.ascontiguousarray(v, dtype=np.float64)
+        out = np.zeros(a.shape, dtype=np.uint16)
+        st = self.lib.orc_round_array_bf16(_ptr(a), a.size, _ptr(out))
+        if st != ORC_OK:
+            raise ValueError(f"orc_round_array_bf16 failed with status {st}")
+        return out
+
+    def rms_normalize_bf16(self, y) -> np.ndarray:
+        """bf16(y / rms(y)) row by row, rms over the last axis."""
+        a = np.ascontiguousarray(y, dtype=np.float64)
+        a2 = a.reshape(-1, a.shape[-1])
+        out = np.zeros(a2.shape, dtype=np.uint16)
+        st = self.lib.orc_rms_normalize_bf16(_ptr(a2), a2.shape[0], a2.shape[1], _ptr(out))
+        if st != ORC_OK:
+            raise ValueError(f"orc_rms_normalize_bf16 failed with status {st}")
+        return out.reshape(a.shape)
+
+    def chain_block(self, h_bits, w) -> dict:
+        """One block of the decode chain (the reading stated in nq_oracle.c).
+
+        h_bits: batch x n bf16 patterns; w: {name: (Upk, Vpk, s1_bits, s2_bits, m, n, r)}
+        for q, k, v, o, gate, up, down.  Returns every layer's y (float64), the bf16 inputs
+        of o and down, and the next block's input "h_next".
+        """
+        out = {}
+        for name in ("q", "k", "v", "gate", "up"):
+            out[name] = self.lowrank_linear_fwd(h_bits, *w[name])
+        out["x_o"] = self.round_to_bf16(out["v"])
+        out["x_down"] = self.round_to_bf16(out["up"])
+        out["o"] = self.lowrank_linear_fwd(out["x_o"], *w["o"])
+        out["down"] = self.lowrank_linear_fwd(out["x_down"], *w["down"])
+        out["h_next"] = self.rms_normalize_bf16(out["down"])
+        return out
+
+    def decode_chain(self, h0_bits, blocks) -> np.ndarray:
+        """The whole chain: the input of each block is the previous block's h_next."""
+        h = h0_bits
+        for w in blocks:
+            h = self.chain_block(h, w)["h_next"]
+        return h
 
 
 _default = None

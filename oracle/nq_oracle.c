@@ -208,3 +208,59 @@ int orc_num_threads(void) {
     return 1;
 #endif
 }
+
+/* ---- helpers of the decode chain ----
+ *
+ * A decode step runs a decoder's linear layers one after the other (hardwired.dev,
+ * section "Cisla", reports decode tokens/s of a whole quantised 70B model).  The pages
+ * print neither the layers between the linears nor any normalisation, so the chain used
+ * here is a reading: each block's input h is a bfloat16 vector of unit root-mean-square;
+ * q, k, v, gate and up read h; o reads bf16(v's output); down reads bf16(up's output);
+ * the next block's h is bf16(down's output / rms(down's output)).  The two helpers
+ * below are that rounding and that normalisation. */
+
+/* Nearest bfloat16 of v, ties to even (the IEEE 754 default rounding), written from the
+ * bfloat16 layout: 1 sign, 8 exponent (bias 127) and 7 fraction bits; normal numbers
+ * 1.f x 2^E with -126 <= E <= 127, subnormals 0.f x 2^-126.  Overflow gives infinity,
+ * NaN the quiet NaN 0x7FC0. */
+uint16_t orc_round_to_bf16(double v) {
+    if (isnan(v)) return 0x7FC0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return sign | 0x7F80;
+    int e;
+    frexp(a, &e);                      /* a = f * 2^e with 0.5 <= f < 1: a = 1.x * 2^(e-1) */
+    int E = e - 1;
+    if (E < -126) E = -126;            /* below the normal range the quantum stays 2^-133 */
+    double q = rint(ldexp(a, 7 - E));  /* a in units of the quantum 2^(E-7), ties to even */
+    if (q >= 256.0) {                  /* rounded up into the next binade */
+        E += 1;
+        q = 128.0;
+    }
+    if (E > 127) return sign | 0x7F80;
+    if (q < 128.0) return sign | (uint16_t)q;  /* subnormal: exponent field 0 */
+    return sign | (uint16_t)(((uint32_t)(E + 127) << 7) | ((uint32_t)q - 128u));
+}
+
+int orc_round_array_bf16(const double *v, int64_t count, uint16_t *out) {
+    if (count < 0 || (count > 0 && (!v || !out))) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < count; ++i) out[i] = orc_round_to_bf16(v[i]);
+    return ORC_OK;
+}
+
+/* out[row][j] = bf16( y[row][j] / sqrt( (1/cols) * sum_j y[row][j]^2 ) ), the sum in
+ * increasing j in double.  A row whose sum of squares is 0 is copied as bf16(y) (signed
+ * zeros): there is nothing to normalise. */
+int orc_rms_normalize_bf16(const double *y, int64_t rows, int64_t cols, uint16_t *out) {
+    if (rows < 0 || cols <= 0 || (rows > 0 && (!y || !out))) return ORC_ERR_ARG;
+    for (int64_t row = 0; row < rows; ++row) {
+        const double *yr = y + row * cols;
+        double acc = 0.0;
+        for (int64_t j = 0; j < cols; ++j) acc += yr[j] * yr[j];
+        double rms = sqrt(acc / (double)cols);
+        for (int64_t j = 0; j < cols; ++j)
+            out[row * cols + j] = orc_round_to_bf16(rms > 0.0 ? yr[j] / rms : yr[j]);
+    }
+    return ORC_OK;
+}

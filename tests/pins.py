@@ -232,6 +232,126 @@ def pin_bits_per_weight(o):
         assert o.bits_per_weight(*bad) == -1.0
 
 
+def load_bf16_rounding():
+    rows = []
+    with open(os.path.join(GOLDEN, "bf16_rounding.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            mant, expo, hexbits = line.split()[:3]
+            rows.append((int(mant), int(expo), int(hexbits, 16)))
+    return rows
+
+
+def pin_bf16_rounding(o):
+    """Hand-worked roundings, then torch's own float32 -> bfloat16 cast (round to nearest
+    even) on float32 values that cover normals, subnormals and exact half-way points."""
+    import math
+
+    import torch
+
+    for mant, expo, want in load_bf16_rounding():
+        v = math.ldexp(mant, expo)
+        got = int(o.round_to_bf16(np.array([v]))[0])
+        assert got == want, (mant, expo, hex(got), hex(want))
+    rng = np.random.default_rng(11)
+    bits = rng.integers(0, 1 << 32, size=20000, dtype=np.uint64).astype(np.uint32)
+    bits = bits[(bits & 0x7F800000) != 0x7F800000]              # finite values only
+    halfway = (rng.integers(0, 1 << 16, size=4000, dtype=np.uint64).astype(np.uint32) << 16) | 0x8000
+    halfway = halfway[(halfway & 0x7F800000) != 0x7F800000]
+    f32 = np.concatenate([bits, halfway]).view(np.float32)
+    want = torch.from_numpy(f32.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = o.round_to_bf16(f32.astype(np.float64))
+    assert np.array_equal(got, want)
+    assert int(o.round_to_bf16(np.array([float("inf")]))[0]) == 0x7F80
+    assert int(o.round_to_bf16(np.array([-0.0]))[0]) == 0x8000
+
+
+def pin_rms_normalize(o):
+    """Closed forms of y / sqrt(mean(y^2)) and its invariances."""
+    # a constant row normalises to exactly 1.0; negative constants to -1.0
+    c = np.full((2, 96), 0.37)
+    c[1] = -5.25
+    out = o.rms_normalize_bf16(c)
+    assert np.all(out[0] == 0x3F80) and np.all(out[1] == 0xBF80)
+    # (3, 4): mean square 12.5, so 3/sqrt(12.5) = 0.8485... -> 217/256 and
+    # 4/sqrt(12.5) = 1.1314 -> 145/128, by hand from the bfloat16 spacing
+    assert o.rms_normalize_bf16(np.array([[3.0, 4.0]])).tolist() == [[0x3F59, 0x3F91]]
+    # one non-zero entry among n: it becomes +-sqrt(n) (n = 64 -> 8.0 exactly)
+    e = np.zeros((1, 64))
+    e[0, 5] = -0.001
+    out = o.rms_normalize_bf16(e)
+    assert out[0, 5] == 0xC100 and np.all(np.delete(out[0], 5) == 0)
+    # scaling by a power of two and negation change nothing / flip the sign bit only
+    rng = np.random.default_rng(12)
+    y = rng.standard_normal((3, 4096)) * 1.7
+    base = o.rms_normalize_bf16(y)
+    assert np.array_equal(o.rms_normalize_bf16(y * 2.0 ** 9), base)
+    assert np.array_equal(o.rms_normalize_bf16(-y), base ^ 0x8000)
+    # the output has unit root-mean-square up to the bfloat16 rounding (relative 2^-9)
+    vals = torch_bf16_to_f64(base)
+    assert np.all(np.abs(np.sqrt(np.mean(vals ** 2, axis=1)) - 1.0) < 2.0 ** -8)
+    # a zero row stays zero (signed zeros kept)
+    z = np.array([[0.0, -0.0, 0.0]])
+    assert o.rms_normalize_bf16(z).tolist() == [[0x0000, 0x8000, 0x0000]]
+
+
+def _tiny_chain_weights(seed, d=64, f=96, ra=32, rf=48):
+    shapes = {"q": (d, d, ra), "k": (d, d, ra), "v": (d, d, ra), "o": (d, d, ra),
+              "gate": (f, d, rf), "up": (f, d, rf), "down": (d, f, rf)}
+    w, dense = {}, {}
+    for name, (m, n, r) in shapes.items():
+        U = synth.signs(m, r, seed, name, "U")
+        V = synth.signs(n, r, seed, name, "V")
+        s1 = synth.scales_f16(m, seed, name, "s1")
+        s2 = synth.scales_f16(n, seed, name, "s2")
+        dense[name] = (U, V, s1, s2)
+        w[name] = (None, None, s1, s2, m, n, r)
+    return w, dense
+
+
+def pin_chain_block(o):
+    """One block of the decode chain against the same wiring built from materialised
+    dense layers (numpy), torch's bfloat16 cast and a numpy root-mean-square."""
+    import torch
+
+    w, dense = _tiny_chain_weights(31)
+    for name, (U, V, s1, s2) in dense.items():
+        _, _, _, _, m, n, r = w[name]
+        w[name] = (o.pack_signs(U), o.pack_signs(np.ascontiguousarray(V.T)), s1, s2, m, n, r)
+    h = synth.activations_bf16(2, 64, 31, "h")
+
+    def ref(x_bits, name):
+        return dense_reference(x_bits, *dense[name])
+
+    def to_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64)).to(torch.float32).to(
+            torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+    out = o.chain_block(h, w)
+    for name in ("q", "k", "v", "gate", "up"):
+        assert rel_err(out[name], ref(h, name)) <= 1e-12, name
+    assert np.array_equal(out["x_o"], to_bf16(out["v"]))
+    assert np.array_equal(out["x_down"], to_bf16(out["up"]))
+    assert rel_err(out["o"], ref(out["x_o"], "o")) <= 1e-12
+    assert rel_err(out["down"], ref(out["x_down"], "down")) <= 1e-12
+    y = out["down"]
+    want = y / np.sqrt(np.mean(y * y, axis=1, keepdims=True))
+    got = torch_bf16_to_f64(out["h_next"])
+    assert np.all(np.abs(got - want) <= 2.0 ** -8 * np.abs(want))
+    # the chain feeds each block's h_next to the next block
+    w2 = dict(w)
+    h2 = o.decode_chain(h, [w, w2])
+    assert np.array_equal(h2, o.chain_block(out["h_next"], w2)["h_next"])
+
+
+def torch_bf16_to_f64(bits):
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
 ALL_PINS = [
     pin_decoders,
     pin_pack_patterns,
@@ -242,4 +362,7 @@ ALL_PINS = [
     pin_closed_forms,
     pin_linearity,
     pin_bits_per_weight,
+    pin_bf16_rounding,
+    pin_rms_normalize,
+    pin_chain_block,
 ]

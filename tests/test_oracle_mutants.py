@@ -29,6 +29,11 @@ MUTANTS = {
     "t_wrong_token": ("orc_sign_at(Vpk, wpr_v, k, j) * xs[b * n + j];", "orc_sign_at(Vpk, wpr_v, k, j) * xs[j];"),
     "y_wrong_t_index": ("acc += orc_sign_at(Upk, wpr_u, i, k) * t[b * r + k];",
                         "acc += orc_sign_at(Upk, wpr_u, i, k) * t[b * r + (k + 1) % r];"),
+    "bf16_truncates": ("double q = rint(ldexp(a, 7 - E));", "double q = floor(ldexp(a, 7 - E));"),
+    "bf16_no_carry": ("if (q >= 256.0) {", "if (q > 256.0) {"),
+    "bf16_subnormal_quantum": ("if (E < -126) E = -126;", "if (E < -127) E = -127;"),
+    "rms_sum_not_mean": ("sqrt(acc / (double)cols)", "sqrt(acc)"),
+    "rms_no_sqrt": ("double rms = sqrt(acc / (double)cols);", "double rms = acc / (double)cols;"),
 }
 
 
@@ -49,3 +54,30 @@ def test_mutant_is_caught(name, tmp_path):
         except (AssertionError, ValueError):
             failures.append(pin.__name__)
     assert failures, f"mutant {name} passed every pin"
+
+
+# Wiring mistakes planted in a copy of the oracle's Python chain composition.
+CHAIN_MUTANTS = {
+    "o_reads_h": ('out["o"] = self.lowrank_linear_fwd(out["x_o"], *w["o"])',
+                  'out["o"] = self.lowrank_linear_fwd(h_bits, *w["o"])'),
+    "down_reads_gate": ('out["x_down"] = self.round_to_bf16(out["up"])',
+                        'out["x_down"] = self.round_to_bf16(out["gate"])'),
+    "next_from_o": ('out["h_next"] = self.rms_normalize_bf16(out["down"])',
+                    'out["h_next"] = self.rms_normalize_bf16(out["o"])'),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CHAIN_MUTANTS))
+def test_chain_mutant_is_caught(name):
+    import types
+
+    before, after = CHAIN_MUTANTS[name]
+    path = os.path.join(os.path.dirname(oracle.__file__), "__init__.py")
+    src = open(path).read()
+    assert src.count(before) == 1, f"mutation site for {name} not unique"
+    mod = types.ModuleType("oracle_mutant")
+    mod.__file__ = path
+    exec(compile(src.replace(before, after), "oracle_mutant", "exec"), mod.__dict__)
+    o = mod.Oracle(oracle.build())
+    with pytest.raises(AssertionError):
+        pins.pin_chain_block(o)
