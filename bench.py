@@ -255,6 +255,8 @@ def run_ours(args):
     peaks = load_peaks()
     if args.workload == "prefill":
         return run_prefill_only(args, device, peaks)
+    if args.workload == "chain7b":
+        return run_chain_only(args, device, peaks)
     layers = synth.LLAMA2_70B_LAYERS if args.workload == "decode70b" else synth.LLAMA2_7B_LAYERS
     model = "llama2-70b" if args.workload == "decode70b" else "llama2-7b"
     batch = args.batch
@@ -337,6 +339,8 @@ def run_ours(args):
 
     if args.secondary and world == 1:
         secondary["prefill_11008x4096_r2432"] = run_prefill_sweep(device, stream, args.warmup, peaks)
+    if args.secondary and world == 1 and batch == 1 and args.workload == "decode7b":
+        secondary["chain_llama2-7b_32_blocks_b1"] = run_chain(device, stream, args.warmup, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -417,6 +421,79 @@ def run_prefill_sweep(device, stream, warmup, peaks, calls=20, batches=synth.PRE
                        "tokens_per_s": round(b / (ms * 1e-3), 1)}
         del g, x, y
     return out
+
+
+def run_chain(device, stream, warmup, peaks, passes=20, batch=1, nblocks=synth.CHAIN_7B_BLOCKS):
+    """The decode chain: 32 Llama-2-7B-shaped blocks x 7 factorised linears at batch 1, per
+    block two grouped forward calls, one cast and one RMS normalisation (6 kernels).  659 MB
+    of packed weights per pass (> 5x L2), so every pass streams its weights from HBM."""
+    import torch
+
+    from binary_rank_linear_02_b200 import chain
+
+    gen = torch.Generator(device=device)
+    gen.manual_seed(5150)
+    blocks = []
+    for b in range(nblocks):
+        w = {}
+        for li, (name, m, n, r) in enumerate(synth.LLAMA2_7B_LAYERS):
+            Upk = torch.randint(-(1 << 31), 1 << 31, (m, r // 32), dtype=torch.int64, device=device,
+                                generator=gen).to(torch.int32)
+            Vpk = torch.randint(-(1 << 31), 1 << 31, (r, n // 32), dtype=torch.int64, device=device,
+                                generator=gen).to(torch.int32)
+            s1 = torch.from_numpy(synth.scales_f16(m, 5150, b, li, "s1").view(np.int16)).to(device)
+            s2 = torch.from_numpy(synth.scales_f16(n, 5150, b, li, "s2").view(np.int16)).to(device)
+            w[name] = (Upk, Vpk, s1, s2, m, n, r)
+        blocks.append(w)
+    ch = chain.DecodeChain(blocks, batch)
+    h0 = torch.from_numpy(synth.activations_bf16(batch, ch.d, 5150, "h0").view(np.int16)).to(device)
+    ch.h[0].copy_(h0)
+    with torch.cuda.stream(stream):
+        ch.run(stream=stream.cuda_stream)
+    torch.cuda.synchronize()
+    g = capture(lambda h: ch.run(stream=h), stream)
+    for _ in range(max(3, warmup // 10)):
+        g.replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(passes):
+            g.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / passes
+    pb = ch.packed_bytes()
+    gbs = pb / (ms * 1e-3) / 1e9
+    out = {"tokens_per_s": round(batch / (ms * 1e-3), 1), "us_per_pass": round(ms * 1e3, 1),
+           "packed_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+           "packed_bytes_per_pass": pb, "blocks": nblocks, "batch": batch,
+           "kernels_per_pass": nblocks * chain.DecodeChain.launches_per_step_per_block,
+           "roofline_tokens_per_s": round(batch * peaks["hbm_gbs"] * 1e9 / pb, 1)}
+    del g, ch, blocks
+    return out
+
+
+def run_chain_only(args, device, peaks):
+    """--workload chain7b: the decode chain alone, one JSON line (tokens/s of the chain)."""
+    import torch
+
+    stream = torch.cuda.Stream(device)
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    c = run_chain(device, stream, args.warmup, peaks, passes=max(1, args.steps), batch=args.batch)
+    clocks = sampler.stop()
+    line = {"metric": METRIC, "value": c["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(c["us_per_pass"] / 1e3, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 in; int8x2-limb tensor-core products, int32/fp32 acc", "data": "synthetic",
+            "config": {"workload": f"decode chain: {c['blocks']} llama2-7b-shaped blocks x 7 factorised linears, "
+                                   f"batch {c['batch']}, per-block RMS re-normalisation",
+                       "l2": "659 MB of packed weights per pass (> 5x L2)", "graphs": "one CUDA graph per pass"},
+            "roofline": {"bound": "hbm", "achieved": c["packed_gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": c["frac_of_hbm"], "traffic": None, "peak_source": peaks["source"]},
+            "gpu_launches": c["kernels_per_pass"] * max(1, args.steps), "clocks": clocks, "chain": c}
+    print(json.dumps(line), flush=True)
 
 
 def run_prefill_only(args, device, peaks):
@@ -523,7 +600,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", dest="secondary", action="store_false")
-    ap.add_argument("--workload", choices=["decode7b", "decode70b", "prefill"], default="decode7b")
+    ap.add_argument("--workload", choices=["decode7b", "decode70b", "prefill", "chain7b"], default="decode7b")
     ap.add_argument("--prefill-batch", type=int, default=0)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -12,6 +12,8 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxDim = int64_t(1) << 20;
 constexpr int64_t kMaxRank = 65536;
+constexpr int64_t kMaxElems = int64_t(1) << 40;  // element-wise helpers: elements per call
+constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1;  // one CTA per row
 
 std::mutex g_mutex;
 Workspace g_ws[kMaxDevices];
@@ -232,6 +234,24 @@ int nq_unpack_signs(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* 
         return NQ_OK;
     }
     return unpack_device(packed, rows, cols, out, static_cast<cudaStream_t>(stream));
+}
+
+int nq_cast_f32_to_bf16(const float* src, int64_t count, void* dst, void* stream) {
+    if (count < 0 || count > kMaxElems) return NQ_ERR_SHAPE;
+    if (count == 0) return NQ_OK;
+    if (!src || !dst) return NQ_ERR_NULL;
+    if (!aligned16(src) || !aligned16(dst)) return NQ_ERR_ALIGN;
+    if (!pointer_kind(src) || !pointer_kind(dst)) return NQ_ERR_PTRKIND;
+    return cast_f32_bf16_device(src, count, static_cast<uint16_t*>(dst), static_cast<cudaStream_t>(stream));
+}
+
+int nq_rms_normalize_bf16(const float* src, int64_t rows, int64_t cols, void* dst, void* stream) {
+    if (rows < 0 || cols <= 0 || rows > kMaxRows || cols > kMaxElems / (rows > 0 ? rows : 1)) return NQ_ERR_SHAPE;
+    if (rows == 0) return NQ_OK;
+    if (!src || !dst) return NQ_ERR_NULL;
+    if (!aligned16(src) || !aligned16(dst)) return NQ_ERR_ALIGN;
+    if (!pointer_kind(src) || !pointer_kind(dst)) return NQ_ERR_PTRKIND;
+    return rms_normalize_bf16_device(src, rows, cols, static_cast<uint16_t*>(dst), static_cast<cudaStream_t>(stream));
 }
 
 int nq_lowrank_linear_fwd_grouped(const nq_linear_desc* layers, int count, int64_t batch, void* stream) {

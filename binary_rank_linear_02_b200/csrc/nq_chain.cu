@@ -1,0 +1,117 @@
+// nq_chain.cu -- the two small element-wise steps between the factorised layers of a
+// decode chain: rounding a layer's fp32 output to the bfloat16 input of the next layer,
+// and re-normalising a block's output to unit root-mean-square before the next block.
+//
+// A decoder runs its quantised linear layers one after the other (hardwired.dev,
+// "NanoQuant jednoduse: 70B model na herni grafice", section "Cisla": decode tokens/s of
+// a whole quantised 70B model).  The pages print neither what sits between the layers
+// nor any normalisation; these two kernels are the library's helpers for chaining its
+// own forward calls (each layer takes bfloat16 x and returns fp32 y).
+//
+// Both kernels are memory-trivial (tens of KB per call at decode sizes) and sit on the
+// chain's critical path, so they are shaped for latency: launched with programmatic
+// dependent launch, they let the next kernel start its weight prefetch early and read
+// their input only after the producing kernel has finished.
+#include <cuda_bf16.h>
+
+#include "nq_internal.cuh"
+
+namespace nq {
+namespace {
+
+constexpr int kCastThreads = 256;
+constexpr int kNormThreads = 512;
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+// dst[i] = bf16(src[i]) (round to nearest, ties to even); 8 elements per thread step.
+__global__ void __launch_bounds__(kCastThreads) cast_kernel(const float* __restrict__ src, int64_t count,
+                                                            uint16_t* __restrict__ dst) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t groups = count / 8;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < groups; g += stride) {
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(src) + 2 * g);
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(src) + 2 * g + 1);
+        reinterpret_cast<uint4*>(dst)[g] =
+            make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+    }
+    for (int64_t i = groups * 8 + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count; i += stride)
+        dst[i] = __bfloat16_as_ushort(__float2bfloat16_rn(__ldcg(src + i)));
+}
+
+// One CTA per row: dst[row][j] = bf16(src[row][j] * (1 / sqrt(sum_j src^2 / cols))).
+// A row whose sum of squares is 0 is rounded as it is (signed zeros kept).
+__global__ void __launch_bounds__(kNormThreads, 1) rms_norm_kernel(const float* __restrict__ src, int64_t cols,
+                                                                uint16_t* __restrict__ dst) {
+    __shared__ float warp_sums[kNormThreads / 32];
+    __shared__ float inv_rms;
+    pdl_wait();
+    pdl_trigger();
+    const float* row = src + (int64_t)blockIdx.x * cols;
+    uint16_t* out = dst + (int64_t)blockIdx.x * cols;
+    const bool vec = (cols % 8) == 0;  // rows then start on 32-byte (src) and 16-byte (dst) boundaries
+    float ss = 0.f;
+    if (vec) {
+        for (int64_t g = threadIdx.x; g < cols / 4; g += blockDim.x) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(row) + g);
+            ss = fmaf(v.x, v.x, ss);
+            ss = fmaf(v.y, v.y, ss);
+            ss = fmaf(v.z, v.z, ss);
+            ss = fmaf(v.w, v.w, ss);
+        }
+    } else {
+        for (int64_t j = threadIdx.x; j < cols; j += blockDim.x) {
+            const float v = __ldcg(row + j);
+            ss = fmaf(v, v, ss);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float s = threadIdx.x < (blockDim.x >> 5) ? warp_sums[threadIdx.x] : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (threadIdx.x == 0) inv_rms = s > 0.f ? 1.0f / sqrtf(s / (float)cols) : 1.0f;
+    }
+    __syncthreads();
+    const float k = inv_rms;
+    if (vec) {
+        for (int64_t g = threadIdx.x; g < cols / 8; g += blockDim.x) {
+            const float4 a = __ldcg(reinterpret_cast<const float4*>(row) + 2 * g);
+            const float4 b = __ldcg(reinterpret_cast<const float4*>(row) + 2 * g + 1);
+            reinterpret_cast<uint4*>(out)[g] = make_uint4(pack_bf16x2(a.x * k, a.y * k), pack_bf16x2(a.z * k, a.w * k),
+                                                          pack_bf16x2(b.x * k, b.y * k), pack_bf16x2(b.z * k, b.w * k));
+        }
+    } else {
+        for (int64_t j = threadIdx.x; j < cols; j += blockDim.x)
+            out[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__ldcg(row + j) * k));
+    }
+}
+
+}  // namespace
+
+int cast_f32_bf16_device(const float* src, int64_t count, uint16_t* dst, cudaStream_t stream) {
+    int64_t blocks = (count / 8 + kCastThreads - 1) / kCastThreads;
+    if (blocks < 1) blocks = 1;
+    if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
+    return launch_pdl(cast_kernel, dim3((unsigned)blocks), dim3(kCastThreads), 0, stream, src, count, dst) ==
+                   cudaSuccess
+               ? NQ_OK
+               : NQ_ERR_CUDA;
+}
+
+int rms_normalize_bf16_device(const float* src, int64_t rows, int64_t cols, uint16_t* dst, cudaStream_t stream) {
+    return launch_pdl(rms_norm_kernel, dim3((unsigned)rows), dim3(kNormThreads), 0, stream, src, cols, dst) ==
+                   cudaSuccess
+               ? NQ_OK
+               : NQ_ERR_CUDA;
+}
+
+}  // namespace nq

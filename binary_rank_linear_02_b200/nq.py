@@ -7,8 +7,9 @@ missing or cannot be loaded, importing this module raises.
 
 Same names as the C entry points: ``nq_pack_signs``, ``nq_unpack_signs``,
 ``nq_lowrank_linear_fwd``, ``nq_bits_per_weight``, ``nq_status_string``,
-``nq_workspace_reserve``; plus tensor-level conveniences ``pack_signs``,
-``unpack_signs`` and ``lowrank_linear_fwd``.
+``nq_workspace_reserve``, ``nq_cast_f32_to_bf16``, ``nq_rms_normalize_bf16``; plus
+tensor-level conveniences ``pack_signs``, ``unpack_signs``, ``lowrank_linear_fwd``,
+``lowrank_linear_fwd_grouped``, ``cast_f32_to_bf16`` and ``rms_normalize_bf16``.
 """
 from __future__ import annotations
 
@@ -75,6 +76,10 @@ def _load() -> ctypes.CDLL:
     L.nq_lowrank_linear_fwd_grouped.restype = ctypes.c_int
     L.nq_device_status.argtypes = [p]
     L.nq_device_status.restype = ctypes.c_int
+    L.nq_cast_f32_to_bf16.argtypes = [p, i64, p, p]
+    L.nq_cast_f32_to_bf16.restype = ctypes.c_int
+    L.nq_rms_normalize_bf16.argtypes = [p, i64, i64, p, p]
+    L.nq_rms_normalize_bf16.restype = ctypes.c_int
     return L
 
 
@@ -109,6 +114,14 @@ def nq_lowrank_linear_fwd_grouped(descs_ptr, count, batch, stream=0) -> int:
 
 def nq_bits_per_weight(m: int, n: int, r: int) -> float:
     return _lib.nq_bits_per_weight(m, n, r)
+
+
+def nq_cast_f32_to_bf16(src_ptr, count, dst_ptr, stream=0) -> int:
+    return _lib.nq_cast_f32_to_bf16(src_ptr, count, dst_ptr, stream)
+
+
+def nq_rms_normalize_bf16(src_ptr, rows, cols, dst_ptr, stream=0) -> int:
+    return _lib.nq_rms_normalize_bf16(src_ptr, rows, cols, dst_ptr, stream)
 
 
 def nq_status_string(status: int) -> str:
@@ -224,6 +237,28 @@ def lowrank_linear_fwd_grouped(layers, batch: int, stream=None):
     h = _stream(stream, *(l[0] for l in layers))
     _check(_lib.nq_lowrank_linear_fwd_grouped(ctypes.addressof(arr), len(layers), batch, h),
            "nq_lowrank_linear_fwd_grouped")
+
+
+def cast_f32_to_bf16(src, dst=None, stream=None):
+    """bf16 bit patterns (int16 tensor of src's shape) of a float32 device tensor."""
+    import torch
+
+    if dst is None:
+        dst = torch.empty(src.shape, dtype=torch.int16, device=src.device)
+    _check(_lib.nq_cast_f32_to_bf16(_ptr(src), src.numel(), _ptr(dst), _stream(stream, src)), "nq_cast_f32_to_bf16")
+    return dst
+
+
+def rms_normalize_bf16(src, dst=None, stream=None):
+    """Row-wise bf16(src / rms(src)) of a 2-D float32 device tensor (int16 patterns)."""
+    import torch
+
+    rows, cols = src.shape
+    if dst is None:
+        dst = torch.empty((rows, cols), dtype=torch.int16, device=src.device)
+    _check(_lib.nq_rms_normalize_bf16(_ptr(src), rows, cols, _ptr(dst), _stream(stream, src)),
+           "nq_rms_normalize_bf16")
+    return dst
 
 
 def bits_per_weight(m: int, n: int, r: int) -> float:

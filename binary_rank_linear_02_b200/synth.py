@@ -98,3 +98,33 @@ SMALL_LAYER = ("single", 512, 512, 128)
 
 PREFILL_SHAPE = ("gate", 11008, 4096, 2432)
 PREFILL_BATCHES = (16, 128, 1024, 4096)
+
+
+# Decode chain of 32 Llama-2-7B-shaped blocks (7 factorised linears each), and a small
+# chain with the same wiring for quick checks (hidden 256, MLP 384, ranks 128).
+CHAIN_7B_BLOCKS = 32
+CHAIN_SMALL_LAYERS = [
+    ("q", 256, 256, 128),
+    ("k", 256, 256, 128),
+    ("v", 256, 256, 128),
+    ("o", 256, 256, 128),
+    ("gate", 384, 256, 128),
+    ("up", 384, 256, 128),
+    ("down", 256, 384, 128),
+]
+
+
+def chain_weights(nblocks: int, layers, seed: int):
+    """Stored weights of a decode chain on the host: one dict per block,
+    {name: (Upk uint32, Vpk uint32, s1 uint16, s2 uint16, m, n, r)}, signs as fair random
+    words (the stored form of Bernoulli(0.5) signs), scales as ``scales_f16``."""
+    blocks = []
+    for b in range(nblocks):
+        w = {}
+        for (name, m, n, r) in layers:
+            w[name] = (random_words(m, (r + 31) // 32, seed, "chain", b, name, "U"),
+                       random_words(r, (n + 31) // 32, seed, "chain", b, name, "V"),
+                       scales_f16(m, seed, "chain", b, name, "s1"),
+                       scales_f16(n, seed, "chain", b, name, "s2"), m, n, r)
+        blocks.append(w)
+    return blocks

@@ -130,6 +130,32 @@ typedef struct nq_linear_desc {
  */
 int nq_lowrank_linear_fwd_grouped(const nq_linear_desc* layers, int count, int64_t batch, void* stream);
 
+/*
+ * Helpers for running factorised layers one after another (a decode chain).  A decoder
+ * runs its quantised linear layers in sequence (hardwired.dev section "Cisla": decode
+ * tokens/s of a whole quantised model); the pages print nothing about what sits between
+ * the layers, so these are the library's own glue, not steps of the method: each
+ * forward call takes bfloat16 x and returns fp32 y, and these turn one layer's y into the
+ * next layer's x.  Both pointers in device memory, 16-byte aligned; the kernels are
+ * asynchronous on `stream` and, like the forward call, may start before the kernel
+ * enqueued just before them has finished: they read `src` only after it has.
+ *
+ * nq_cast_f32_to_bf16 -- dst[i] = bf16(src[i]) for 0 <= i < count, round to nearest,
+ *   ties to even (overflow to infinity, NaN stays NaN).  count >= 0 (0 is a no-op).
+ *   dst: count bfloat16 (uint16 patterns), written; it must not overlap src.
+ */
+int nq_cast_f32_to_bf16(const float* src, int64_t count, void* dst, void* stream);
+
+/*
+ * nq_rms_normalize_bf16 -- re-normalise each row to unit root-mean-square:
+ *   dst[i][j] = bf16( src[i][j] / sqrt( (1/cols) * sum_j src[i][j]^2 ) ),
+ *   computed in fp32 (sum of squares, one reciprocal square root per row, one product
+ *   per element) and rounded to nearest, ties to even.  A row whose sum of squares is 0
+ *   is rounded unchanged.  src: rows x cols float32 row-major; dst: rows x cols bfloat16,
+ *   written, not overlapping src.  rows >= 0 (0 is a no-op), cols >= 1.
+ */
+int nq_rms_normalize_bf16(const float* src, int64_t rows, int64_t cols, void* dst, void* stream);
+
 /* Limits of nq_lowrank_linear_fwd_noalloc. */
 #define NQ_NOALLOC_MAX_RANK 4096
 #define NQ_NOALLOC_MAX_BATCH NQ_DECODE_MAX_BATCH

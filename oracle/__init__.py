@@ -219,3 +219,19 @@ def bits_per_weight(m, n, r):
 
 def num_threads():
     return default().num_threads()
+
+
+def round_to_bf16(v):
+    return default().round_to_bf16(v)
+
+
+def rms_normalize_bf16(y):
+    return default().rms_normalize_bf16(y)
+
+
+def chain_block(h_bits, w):
+    return default().chain_block(h_bits, w)
+
+
+def decode_chain(h0_bits, blocks):
+    return default().decode_chain(h0_bits, blocks)

@@ -126,3 +126,41 @@ def test_grouped_argument_errors(nq):
     assert f(a, 2, 1, 0) == nq.NQ_ERR_NULL
     arr[0].s1 = ptr[3]
     assert f(a, 2, 1, 0) == nq.NQ_ERR_PTRKIND  # host memory is refused
+
+
+def test_chain_helper_argument_errors(nq):
+    buf = np.zeros(1 << 14, dtype=np.uint8)
+    base = (buf.ctypes.data + 255) // 256 * 256
+    src, dst = base, base + 4096
+    cast, norm = nq.nq_cast_f32_to_bf16, nq.nq_rms_normalize_bf16
+    assert cast(src, -1, dst, 0) == nq.NQ_ERR_SHAPE
+    assert cast(src, 0, dst, 0) == nq.NQ_OK
+    assert cast(0, 8, dst, 0) == nq.NQ_ERR_NULL
+    assert cast(src, 8, 0, 0) == nq.NQ_ERR_NULL
+    assert cast(src + 4, 8, dst, 0) == nq.NQ_ERR_ALIGN
+    assert cast(src, 8, dst + 2, 0) == nq.NQ_ERR_ALIGN
+    assert cast(src, 8, dst, 0) == nq.NQ_ERR_PTRKIND  # host memory is refused
+    assert norm(src, -1, 8, dst, 0) == nq.NQ_ERR_SHAPE
+    assert norm(src, 2, 0, dst, 0) == nq.NQ_ERR_SHAPE
+    assert norm(src, 1 << 31, 8, dst, 0) == nq.NQ_ERR_SHAPE
+    assert norm(src, 0, 8, dst, 0) == nq.NQ_OK
+    assert norm(0, 2, 8, dst, 0) == nq.NQ_ERR_NULL
+    assert norm(src, 2, 8, dst + 8, 0) == nq.NQ_ERR_ALIGN
+    assert norm(src, 2, 8, dst, 0) == nq.NQ_ERR_PTRKIND
+
+
+def test_chain_module_checks_shapes(nq):
+    """The chain driver refuses blocks whose layers do not fit the wiring (host-side check,
+    before any device work)."""
+    import torch
+
+    from binary_rank_linear_02_b200 import chain
+
+    t = torch.zeros(4, dtype=torch.int32)
+    w = {name: (t, t, t, t, m, n, r) for (name, m, n, r) in
+         [("q", 256, 256, 128), ("k", 256, 256, 128), ("v", 256, 256, 128), ("o", 256, 256, 128),
+          ("gate", 384, 256, 128), ("up", 384, 256, 128), ("down", 384, 256, 128)]}
+    with pytest.raises(ValueError, match="down"):
+        chain.DecodeChain([w], 1)
+    with pytest.raises(ValueError):
+        chain.DecodeChain([], 1)
