@@ -11,10 +11,11 @@ library's reading of a decoder's linear chain:
   * o reads bf16(v's output), down reads bf16(up's output);
   * the next block's input is bf16(down's output / rms(down's output)).
 
-Per block this issues four libnq calls: the grouped forward of the five layers that read
-h, one cast of v's and up's outputs (kept adjacent in memory so one call covers both),
-the grouped forward of o and down, and the RMS normalisation.  This module only lays out
-buffers and passes pointers; every step runs in libnq's kernels.
+Per block this issues two libnq calls (``nq_lowrank_linear_fwd_grouped_ex``): the
+five layers that read h, with v and up also writing their bf16 copies (the inputs of o
+and down), then o and down, with down also writing its RMS-normalised bf16 copy (the next
+block's h).  On the decode path each call is two kernels, so a block is four.  This module
+only lays out buffers and passes pointers; every step runs in libnq's kernels.
 """
 from __future__ import annotations
 
@@ -57,7 +58,7 @@ class DecodeChain:
         self.h = torch.zeros((nb + 1, batch, d), dtype=torch.int16, device=dev)
         self.y = {name: torch.empty((nb, batch, want[name][0]), dtype=torch.float32, device=dev)
                   for name in ("q", "k", "gate", "o", "down")}
-        # v's and up's outputs side by side, so one cast call turns both into bf16
+        # v's and up's outputs side by side (and their bf16 copies)
         self._y_vu = torch.empty((nb, batch * (d + f)), dtype=torch.float32, device=dev)
         self._x_vu = torch.empty((nb, batch * (d + f)), dtype=torch.int16, device=dev)
         self.y["v"] = self._y_vu[:, : batch * d].view(nb, batch, d)
@@ -65,12 +66,14 @@ class DecodeChain:
         self.x_o = self._x_vu[:, : batch * d].view(nb, batch, d)
         self.x_down = self._x_vu[:, batch * d:].view(nb, batch, f)
         self._first, self._second = [], []
+        bf16_out = {"v": self.x_o, "up": self.x_down}
         for i, w in enumerate(blocks):
-            first = [(self.h[i], *w[name][:4], self.y[name][i], *w[name][4:]) for name in FIRST]
-            second = [(self.x_o[i], *w["o"][:4], self.y["o"][i], *w["o"][4:]),
-                      (self.x_down[i], *w["down"][:4], self.y["down"][i], *w["down"][4:])]
-            self._first.append(nq.make_descs(first))
-            self._second.append(nq.make_descs(second))
+            first = [(self.h[i], *w[name][:4], self.y[name][i], *w[name][4:],
+                      bf16_out[name][i] if name in bf16_out else None, None) for name in FIRST]
+            second = [(self.x_o[i], *w["o"][:4], self.y["o"][i], *w["o"][4:], None, None),
+                      (self.x_down[i], *w["down"][:4], self.y["down"][i], *w["down"][4:], None, self.h[i + 1])]
+            self._first.append(nq.make_descs_ex(first))
+            self._second.append(nq.make_descs_ex(second))
         self._keep = blocks
         for name in LAYERS:
             m, n, r = blocks[0][name][4:]
@@ -88,16 +91,12 @@ class DecodeChain:
             self.h[0].copy_(h0.view(self.batch, self.d))
         s = int(stream) if stream is not None else torch.cuda.current_stream(self.h.device).cuda_stream
         L = nq.lib()
-        b, d, f = self.batch, self.d, self.f
+        b = self.batch
         for i in range(self.nblocks):
-            nq._check(L.nq_lowrank_linear_fwd_grouped(ctypes.addressof(self._first[i]), len(FIRST), b, s),
-                      "nq_lowrank_linear_fwd_grouped")
-            nq._check(L.nq_cast_f32_to_bf16(self._y_vu[i].data_ptr(), b * (d + f), self._x_vu[i].data_ptr(), s),
-                      "nq_cast_f32_to_bf16")
-            nq._check(L.nq_lowrank_linear_fwd_grouped(ctypes.addressof(self._second[i]), len(SECOND), b, s),
-                      "nq_lowrank_linear_fwd_grouped")
-            nq._check(L.nq_rms_normalize_bf16(self.y["down"][i].data_ptr(), b, d, self.h[i + 1].data_ptr(), s),
-                      "nq_rms_normalize_bf16")
+            nq._check(L.nq_lowrank_linear_fwd_grouped_ex(ctypes.addressof(self._first[i]), len(FIRST), b, s),
+                      "nq_lowrank_linear_fwd_grouped_ex")
+            nq._check(L.nq_lowrank_linear_fwd_grouped_ex(ctypes.addressof(self._second[i]), len(SECOND), b, s),
+                      "nq_lowrank_linear_fwd_grouped_ex")
         return self.h[self.nblocks]
 
-    launches_per_step_per_block = 6  # 2 + 1 + 2 + 1 kernels
+    launches_per_step_per_block = 4  # two grouped calls of two kernels each (decode path)

@@ -153,6 +153,78 @@ static int ensure_staging(Workspace* w, size_t xbytes, size_t ybytes) {
 
 using namespace nq;
 
+// The grouped forward over `count` descriptors `stride` bytes apart; `ex` (may be NULL)
+// adds the optional bf16 outputs of nq_linear_desc_ex.
+static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_linear_desc_ex* ex, int count,
+                       int64_t batch, void* stream) {
+    auto desc = [&](int i) -> const nq_linear_desc& {
+        return *reinterpret_cast<const nq_linear_desc*>(reinterpret_cast<const char*>(first) + stride * i);
+    };
+    if (batch < 0) return NQ_ERR_BATCH;
+    if (count < 0) return NQ_ERR_SHAPE;
+    if (count == 0 || batch == 0) return NQ_OK;
+    if (!first) return NQ_ERR_NULL;
+    int64_t m_max = 0, n_max = 0, r_max = 0;
+    for (int i = 0; i < count; ++i) {
+        const nq_linear_desc& L = desc(i);
+        if (L.m <= 0 || L.n <= 0 || L.r <= 0 || L.m % 128 || L.n % 128 || L.r % 128 || L.m > kMaxDim ||
+            L.n > kMaxDim || L.r > kMaxRank)
+            return NQ_ERR_SHAPE;
+        if (batch > (int64_t(1) << 40) / (L.m > L.n ? L.m : L.n)) return NQ_ERR_SHAPE;
+        if (!L.x || !L.Upk || !L.Vpk || !L.s1 || !L.s2 || !L.y) return NQ_ERR_NULL;
+        if (!aligned16(L.x) || !aligned16(L.Upk) || !aligned16(L.Vpk) || !aligned16(L.s1) || !aligned16(L.s2) ||
+            !aligned16(L.y))
+            return NQ_ERR_ALIGN;
+        if (ex && (!aligned16(ex[i].y_bf16) || !aligned16(ex[i].y_rmsnorm_bf16))) return NQ_ERR_ALIGN;
+        m_max = L.m > m_max ? L.m : m_max;
+        n_max = L.n > n_max ? L.n : n_max;
+        r_max = L.r > r_max ? L.r : r_max;
+    }
+    for (int i = 0; i < count; ++i) {
+        const nq_linear_desc& L = desc(i);
+        if (!pointer_kind(L.x) || !pointer_kind(L.Upk) || !pointer_kind(L.Vpk) || !pointer_kind(L.s1) ||
+            !pointer_kind(L.s2) || !pointer_kind(L.y))
+            return NQ_ERR_PTRKIND;
+        if (ex && ((ex[i].y_bf16 && !pointer_kind(ex[i].y_bf16)) ||
+                   (ex[i].y_rmsnorm_bf16 && !pointer_kind(ex[i].y_rmsnorm_bf16))))
+            return NQ_ERR_PTRKIND;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int st = NQ_OK;
+    if (batch > NQ_DECODE_MAX_BATCH) {
+        Workspace* ws = workspace_for(m_max, n_max, r_max, batch, DecodeNeed(), &st);
+        if (!ws) return st;
+        for (int i = 0; i < count && st == NQ_OK; ++i) {
+            const nq_linear_desc& L = desc(i);
+            st = prefill_forward(static_cast<const uint16_t*>(L.x), L.Upk, L.Vpk, static_cast<const uint16_t*>(L.s1),
+                                 static_cast<const uint16_t*>(L.s2), L.m, L.n, L.r, batch, L.y, ws, s);
+            // the optional outputs by the stand-alone kernels, after the layer
+            if (st == NQ_OK && ex && ex[i].y_bf16)
+                st = cast_f32_bf16_device(L.y, batch * L.m, static_cast<uint16_t*>(ex[i].y_bf16), s);
+            if (st == NQ_OK && ex && ex[i].y_rmsnorm_bf16)
+                st = rms_normalize_bf16_device(L.y, batch, L.m, static_cast<uint16_t*>(ex[i].y_rmsnorm_bf16), s);
+        }
+        return st;
+    }
+    for (int i0 = 0; i0 < count && st == NQ_OK; i0 += kMaxGroup) {
+        const int cnt = count - i0 < kMaxGroup ? count - i0 : kMaxGroup;
+        DecodeCall calls[kMaxGroup];
+        for (int i = 0; i < cnt; ++i) {
+            const nq_linear_desc& L = desc(i0 + i);
+            calls[i] = DecodeCall{static_cast<const uint16_t*>(L.x), L.Upk, L.Vpk, static_cast<const uint16_t*>(L.s1),
+                                  static_cast<const uint16_t*>(L.s2), L.y, L.m, L.n, L.r};
+            if (ex) {
+                calls[i].y_bf16 = static_cast<uint16_t*>(ex[i0 + i].y_bf16);
+                calls[i].y_norm = static_cast<uint16_t*>(ex[i0 + i].y_rmsnorm_bf16);
+            }
+        }
+        Workspace* ws = workspace_for(m_max, n_max, r_max, batch, decode_need(calls, cnt, batch), &st);
+        if (!ws) return st;
+        st = decode_forward_group(calls, cnt, batch, ws, s);
+    }
+    return st;
+}
+
 extern "C" {
 
 int nq_version(void) { return 100; }
@@ -255,56 +327,11 @@ int nq_rms_normalize_bf16(const float* src, int64_t rows, int64_t cols, void* ds
 }
 
 int nq_lowrank_linear_fwd_grouped(const nq_linear_desc* layers, int count, int64_t batch, void* stream) {
-    if (batch < 0) return NQ_ERR_BATCH;
-    if (count < 0) return NQ_ERR_SHAPE;
-    if (count == 0 || batch == 0) return NQ_OK;
-    if (!layers) return NQ_ERR_NULL;
-    int64_t m_max = 0, n_max = 0, r_max = 0;
-    for (int i = 0; i < count; ++i) {
-        const nq_linear_desc& L = layers[i];
-        if (L.m <= 0 || L.n <= 0 || L.r <= 0 || L.m % 128 || L.n % 128 || L.r % 128 || L.m > kMaxDim ||
-            L.n > kMaxDim || L.r > kMaxRank)
-            return NQ_ERR_SHAPE;
-        if (batch > (int64_t(1) << 40) / (L.m > L.n ? L.m : L.n)) return NQ_ERR_SHAPE;
-        if (!L.x || !L.Upk || !L.Vpk || !L.s1 || !L.s2 || !L.y) return NQ_ERR_NULL;
-        if (!aligned16(L.x) || !aligned16(L.Upk) || !aligned16(L.Vpk) || !aligned16(L.s1) || !aligned16(L.s2) ||
-            !aligned16(L.y))
-            return NQ_ERR_ALIGN;
-        m_max = L.m > m_max ? L.m : m_max;
-        n_max = L.n > n_max ? L.n : n_max;
-        r_max = L.r > r_max ? L.r : r_max;
-    }
-    for (int i = 0; i < count; ++i) {
-        const nq_linear_desc& L = layers[i];
-        if (!pointer_kind(L.x) || !pointer_kind(L.Upk) || !pointer_kind(L.Vpk) || !pointer_kind(L.s1) ||
-            !pointer_kind(L.s2) || !pointer_kind(L.y))
-            return NQ_ERR_PTRKIND;
-    }
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    int st = NQ_OK;
-    if (batch > NQ_DECODE_MAX_BATCH) {
-        Workspace* ws = workspace_for(m_max, n_max, r_max, batch, DecodeNeed(), &st);
-        if (!ws) return st;
-        for (int i = 0; i < count && st == NQ_OK; ++i) {
-            const nq_linear_desc& L = layers[i];
-            st = prefill_forward(static_cast<const uint16_t*>(L.x), L.Upk, L.Vpk, static_cast<const uint16_t*>(L.s1),
-                                 static_cast<const uint16_t*>(L.s2), L.m, L.n, L.r, batch, L.y, ws, s);
-        }
-        return st;
-    }
-    for (int i0 = 0; i0 < count && st == NQ_OK; i0 += kMaxGroup) {
-        const int cnt = count - i0 < kMaxGroup ? count - i0 : kMaxGroup;
-        DecodeCall calls[kMaxGroup];
-        for (int i = 0; i < cnt; ++i) {
-            const nq_linear_desc& L = layers[i0 + i];
-            calls[i] = DecodeCall{static_cast<const uint16_t*>(L.x), L.Upk, L.Vpk, static_cast<const uint16_t*>(L.s1),
-                                  static_cast<const uint16_t*>(L.s2), L.y, L.m, L.n, L.r};
-        }
-        Workspace* ws = workspace_for(m_max, n_max, r_max, batch, decode_need(calls, cnt, batch), &st);
-        if (!ws) return st;
-        st = decode_forward_group(calls, cnt, batch, ws, s);
-    }
-    return st;
+    return grouped_run(layers, sizeof(nq_linear_desc), nullptr, count, batch, stream);
+}
+
+int nq_lowrank_linear_fwd_grouped_ex(const nq_linear_desc_ex* layers, int count, int64_t batch, void* stream) {
+    return grouped_run(layers ? &layers[0].base : nullptr, sizeof(nq_linear_desc_ex), layers, count, batch, stream);
 }
 
 int nq_device_status(void* stream) {

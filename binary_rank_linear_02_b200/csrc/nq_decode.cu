@@ -33,9 +33,10 @@
 // fixed costs decide.  Every CTA copies its weight rows into shared memory (cp.async)
 // before it waits on the previous kernel (programmatic dependent launch) and lets the next
 // kernel launch at once, so weight streaming overlaps the dependency chain.  Stage 1
-// splits each 64-row block's columns so that every CTA stages one chunk; the last CTA of a
+// splits each 128-row block's columns so that every CTA stages one chunk; the last CTA of a
 // block adds the partial sums in a fixed order (deterministic).  Stage 2 holds its whole
 // row block and the whole of t on chip.  Several independent layers can share one launch.
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
 
@@ -112,6 +113,10 @@ struct DecLayer {
     float* tgmax;    // workspace: batch x r/128 (max |t| per 128-row block)
     float* partials; // workspace: nsplit x batch x r (stage-1 column splits)
     int* counters;   // workspace: r/128 arrival counters, zero between calls
+    uint16_t* y_bf16;     // optional bf16(y)
+    uint16_t* y_norm;     // optional bf16(y / rms(y)) per token
+    float* norm_partials; // workspace: batch x (stage-2 CTAs of the layer), sums of y^2
+    int* norm_counter;    // workspace: stage-2 arrivals of the layer, zero between calls
     int m, n, r;
     int nsplit;      // stage 1: CTAs per 128-row block (column splits)
     int cps;         // stage 1: column blocks per split
@@ -472,6 +477,56 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
 // r2 columns are copied on chip before the dependency wait, and t for those columns right
 // after it.  One quantisation exponent per token for the whole of t (from stage 1's
 // maxima), so integer sums run across all chunks and k-parts and are converted once.
+// Row-wise RMS normalisation of a layer's whole output, folded into stage 2: every CTA
+// adds up y^2 over its rows per token (fixed order) into the workspace, and the CTA that
+// arrives last adds those partial sums in CTA order (deterministic), then rounds
+// y * (1 / sqrt(sum / m)) to bf16 for the whole layer.  Same result as rms_norm_kernel up
+// to the order of the sum of squares.
+template <typename YAt>
+__device__ void rms_norm_epilogue(const DecLayer& L, int batch, int rows, int blk, Misc& mi, YAt y_at) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nblk = L.m / rows;
+    if (warp < batch) {  // one warp per token (batch <= 8 = warps)
+        float ss = 0.f;
+        for (int i = lane; i < rows; i += 32) {
+            const float yv = y_at(warp, i);
+            ss = fmaf(yv, yv, ss);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) L.norm_partials[(int64_t)warp * nblk + blk] = ss;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        mi.last = atomicAdd(L.norm_counter, 1) == nblk - 1;
+    }
+    __syncthreads();
+    if (!mi.last) return;
+    __threadfence();
+    if (warp < batch) {
+        float ss = 0.f;
+        for (int b = lane; b < nblk; b += 32) ss += __ldcg(L.norm_partials + (int64_t)warp * nblk + b);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) mi.up[warp] = ss > 0.f ? 1.0f / sqrtf(ss / (float)L.m) : 1.0f;
+    }
+    if (threadIdx.x == 0) *L.norm_counter = 0;  // ready for the next call
+    __syncthreads();
+    const int64_t m = L.m;
+    for (int tok = 0; tok < batch; ++tok) {
+        const float k = mi.up[tok];
+        const float4* src = reinterpret_cast<const float4*>(L.y + tok * m);
+        uint2* dst = reinterpret_cast<uint2*>(L.y_norm + tok * m);
+        for (int64_t g = threadIdx.x; g < m / 4; g += kThreads) {
+            const float4 v = __ldcg(src + g);
+            const __nv_bfloat162 a = __floats2bfloat162_rn(v.x * k, v.y * k);
+            const __nv_bfloat162 b = __floats2bfloat162_rn(v.z * k, v.w * k);
+            dst[g] = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+        }
+    }
+}
+
 template <int NTG>
 __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant__ DecGroup grp) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -565,12 +620,17 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
         }
     }
     __syncthreads();
+    auto y_at = [&](int tok, int i) {
+        const float v = (float)(2 * (int64_t)mi.bq[i][tok] - mi.qsum[tok]) * pow2f(mi.e[tok] - kQBits);
+        return f16_to_f32(L.s1[row0 + i]) * v;
+    };
     for (int idx = threadIdx.x; idx < rows * batch; idx += kThreads) {
         const int tok = idx / rows, i = idx % rows;
-        const int64_t row = row0 + i;
-        const float v = (float)(2 * (int64_t)mi.bq[i][tok] - mi.qsum[tok]) * pow2f(mi.e[tok] - kQBits);
-        L.y[(int64_t)tok * m + row] = f16_to_f32(L.s1[row]) * v;
+        const float yv = y_at(tok, i);
+        L.y[(int64_t)tok * m + row0 + i] = yv;
+        if (L.y_bf16) L.y_bf16[(int64_t)tok * m + row0 + i] = __bfloat16_as_ushort(__float2bfloat16_rn(yv));
     }
+    if (L.y_norm) rms_norm_epilogue(L, batch, rows, blk, mi, y_at);
 }
 
 template <int NTG>
@@ -637,6 +697,9 @@ static int stage1_cps(const DecodeCall* calls, int count, int max_splits) {
 void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, int max_splits, int64_t* t_floats,
                            int64_t* tgmax_floats, int64_t* partial_floats, int64_t* counter_ints) {
     const int cps = stage1_cps(calls, count, max_splits);
+    int64_t tiles = 0;
+    for (int i = 0; i < count; ++i) tiles += calls[i].m / 16;
+    const int rt = stage2_rt(tiles);
     int64_t t = 0, gm = 0, pf = 0, ci = 0;
     for (int i = 0; i < count; ++i) {
         const int64_t ncb = calls[i].n / kCB, nsplit = (ncb + cps - 1) / cps;
@@ -644,6 +707,10 @@ void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, in
         gm += batch * (calls[i].r / kRowsS1);
         if (nsplit > 1) pf += nsplit * batch * calls[i].r;
         ci += calls[i].r / kRowsS1;
+        if (calls[i].y_norm) {  // per-CTA sums of y^2 and one arrival counter
+            pf += batch * (calls[i].m / (16 * rt));
+            ci += 1;
+        }
     }
     *t_floats = t;
     *tgmax_floats = gm;
@@ -675,6 +742,13 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
     grp.depth1 = cps > kChunkCB ? 2 : 1;
     size_t toff = 0, goff = 0, poff = 0, coff = 0;
     grp.s1_start[0] = grp.s2_start[0] = 0;
+    // the normalisation's sums and counters go after every layer's stage-1 scratch
+    size_t npoff = 0, ncoff = 0;
+    for (int i = 0; i < count; ++i) {
+        const int64_t nsplit = (calls[i].n / kCB + cps - 1) / cps;
+        if (nsplit > 1) npoff += (size_t)nsplit * batch * calls[i].r;
+        ncoff += (size_t)(calls[i].r / kRowsS1);
+    }
     for (int i = 0; i < count; ++i) {
         const DecodeCall& c = calls[i];
         DecLayer& L = grp.L[i];
@@ -684,6 +758,16 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
         L.s1 = c.s1;
         L.s2 = c.s2;
         L.y = c.y;
+        L.y_bf16 = c.y_bf16;
+        L.y_norm = c.y_norm;
+        L.norm_partials = nullptr;
+        L.norm_counter = nullptr;
+        if (c.y_norm) {
+            L.norm_partials = ws->partials + npoff;
+            L.norm_counter = ws->counters + ncoff;
+            npoff += (size_t)batch * (c.m / (16 * rt));
+            ncoff += 1;
+        }
         L.m = (int)c.m;
         L.n = (int)c.n;
         L.r = (int)c.r;

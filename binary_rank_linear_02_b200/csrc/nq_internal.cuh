@@ -53,6 +53,8 @@ struct DecodeCall {
     const uint16_t* s2;
     float* y;
     int64_t m, n, r;
+    uint16_t* y_bf16 = nullptr;  // optional: bf16(y), batch x m
+    uint16_t* y_norm = nullptr;  // optional: bf16(y / rms(y)) per token, batch x m
 };
 
 int sm_count();

@@ -44,6 +44,12 @@ class nq_linear_desc(ctypes.Structure):
                 ("m", ctypes.c_int64), ("n", ctypes.c_int64), ("r", ctypes.c_int64)]
 
 
+class nq_linear_desc_ex(ctypes.Structure):
+    """One layer of nq_lowrank_linear_fwd_grouped_ex: the layer plus optional bf16 outputs."""
+
+    _fields_ = [("base", nq_linear_desc), ("y_bf16", ctypes.c_void_p), ("y_rmsnorm_bf16", ctypes.c_void_p)]
+
+
 class NQError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -74,6 +80,8 @@ def _load() -> ctypes.CDLL:
     L.nq_lowrank_linear_fwd_noalloc.restype = ctypes.c_int
     L.nq_lowrank_linear_fwd_grouped.argtypes = [p, ctypes.c_int, i64, p]
     L.nq_lowrank_linear_fwd_grouped.restype = ctypes.c_int
+    L.nq_lowrank_linear_fwd_grouped_ex.argtypes = [p, ctypes.c_int, i64, p]
+    L.nq_lowrank_linear_fwd_grouped_ex.restype = ctypes.c_int
     L.nq_device_status.argtypes = [p]
     L.nq_device_status.restype = ctypes.c_int
     L.nq_cast_f32_to_bf16.argtypes = [p, i64, p, p]
@@ -110,6 +118,10 @@ def nq_lowrank_linear_fwd_noalloc(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n,
 
 def nq_lowrank_linear_fwd_grouped(descs_ptr, count, batch, stream=0) -> int:
     return _lib.nq_lowrank_linear_fwd_grouped(descs_ptr, count, batch, stream)
+
+
+def nq_lowrank_linear_fwd_grouped_ex(descs_ptr, count, batch, stream=0) -> int:
+    return _lib.nq_lowrank_linear_fwd_grouped_ex(descs_ptr, count, batch, stream)
 
 
 def nq_bits_per_weight(m: int, n: int, r: int) -> float:
@@ -229,6 +241,25 @@ def make_descs(layers):
     for i, (x, Upk, Vpk, s1, s2, y, m, n, r) in enumerate(layers):
         arr[i] = nq_linear_desc(_ptr(x), _ptr(Upk), _ptr(Vpk), _ptr(s1), _ptr(s2), _ptr(y), m, n, r)
     return arr
+
+
+def make_descs_ex(layers):
+    """ctypes array of nq_linear_desc_ex from (x, Upk, Vpk, s1, s2, y, m, n, r, y_bf16, y_norm)
+    tuples; the last two may be None."""
+    arr = (nq_linear_desc_ex * len(layers))()
+    for i, (x, Upk, Vpk, s1, s2, y, m, n, r, yb, yn) in enumerate(layers):
+        arr[i] = nq_linear_desc_ex(nq_linear_desc(_ptr(x), _ptr(Upk), _ptr(Vpk), _ptr(s1), _ptr(s2), _ptr(y), m, n, r),
+                                   _ptr(yb), _ptr(yn))
+    return arr
+
+
+def lowrank_linear_fwd_grouped_ex(layers, batch: int, stream=None):
+    """Grouped forward with optional bf16 outputs: layers are (x, Upk, Vpk, s1, s2, y, m, n, r,
+    y_bf16 or None, y_rmsnorm_bf16 or None)."""
+    arr = make_descs_ex(layers)
+    h = _stream(stream, *(l[0] for l in layers))
+    _check(_lib.nq_lowrank_linear_fwd_grouped_ex(ctypes.addressof(arr), len(layers), batch, h),
+           "nq_lowrank_linear_fwd_grouped_ex")
 
 
 def lowrank_linear_fwd_grouped(layers, batch: int, stream=None):

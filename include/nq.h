@@ -156,6 +156,28 @@ int nq_cast_f32_to_bf16(const float* src, int64_t count, void* dst, void* stream
  */
 int nq_rms_normalize_bf16(const float* src, int64_t rows, int64_t cols, void* dst, void* stream);
 
+/* A layer of nq_lowrank_linear_fwd_grouped_ex: the layer plus two optional outputs that
+ * feed the next layer of a chain (see nq_cast_f32_to_bf16 / nq_rms_normalize_bf16 above;
+ * like them, these have no counterpart in the NanoQuant pages). */
+typedef struct nq_linear_desc_ex {
+    nq_linear_desc base;     /* the layer, as for nq_lowrank_linear_fwd_grouped */
+    void* y_bf16;            /* NULL, or batch x m bfloat16 written with bf16(y) */
+    void* y_rmsnorm_bf16;    /* NULL, or batch x m bfloat16 written with
+                              * bf16(y[b][i] / sqrt((1/m) sum_i y[b][i]^2)) per token b */
+} nq_linear_desc_ex;
+
+/*
+ * nq_lowrank_linear_fwd_grouped_ex -- nq_lowrank_linear_fwd_grouped, plus per layer the
+ * optional bfloat16 copies of y that the next layer of a decode chain reads.  y is always
+ * written.  y_bf16 equals nq_cast_f32_to_bf16 of y bit for bit; y_rmsnorm_bf16 equals
+ * nq_rms_normalize_bf16 of y (batch rows of m) up to the order of the fp32 sum of squares.
+ * On the decode path both are produced by the forward's own kernels (no extra launch); on
+ * the prefill path by the stand-alone kernels after the layer.  Optional pointers are
+ * device memory, 16-byte aligned, and overlap no other buffer of the call.  Errors as
+ * nq_lowrank_linear_fwd_grouped.
+ */
+int nq_lowrank_linear_fwd_grouped_ex(const nq_linear_desc_ex* layers, int count, int64_t batch, void* stream);
+
 /* Limits of nq_lowrank_linear_fwd_noalloc. */
 #define NQ_NOALLOC_MAX_RANK 4096
 #define NQ_NOALLOC_MAX_BATCH NQ_DECODE_MAX_BATCH

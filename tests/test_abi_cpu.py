@@ -164,3 +164,26 @@ def test_chain_module_checks_shapes(nq):
         chain.DecodeChain([w], 1)
     with pytest.raises(ValueError):
         chain.DecodeChain([], 1)
+
+
+def test_grouped_ex_argument_errors(nq):
+    buf = np.zeros(1 << 16, dtype=np.uint8)
+    base = (buf.ctypes.data + 255) // 256 * 256
+    ptr = [base + 1024 * i for i in range(8)]
+    good = nq.nq_linear_desc(ptr[0], ptr[1], ptr[2], ptr[3], ptr[4], ptr[5], 128, 128, 128)
+    arr = (nq.nq_linear_desc_ex * 2)(nq.nq_linear_desc_ex(good, 0, 0), nq.nq_linear_desc_ex(good, ptr[6], ptr[7]))
+    f = nq.nq_lowrank_linear_fwd_grouped_ex
+    a = ctypes.addressof(arr)
+    assert f(a, 2, -1, 0) == nq.NQ_ERR_BATCH
+    assert f(a, 0, 1, 0) == nq.NQ_OK
+    assert f(0, 2, 1, 0) == nq.NQ_ERR_NULL
+    arr[1].base.m = 100
+    assert f(a, 2, 1, 0) == nq.NQ_ERR_SHAPE
+    arr[1].base.m = 128
+    arr[1].y_bf16 = ptr[6] + 2
+    assert f(a, 2, 1, 0) == nq.NQ_ERR_ALIGN
+    arr[1].y_bf16 = ptr[6]
+    arr[1].y_rmsnorm_bf16 = ptr[7] + 8
+    assert f(a, 2, 1, 0) == nq.NQ_ERR_ALIGN
+    arr[1].y_rmsnorm_bf16 = ptr[7]
+    assert f(a, 2, 1, 0) == nq.NQ_ERR_PTRKIND  # host memory is refused

@@ -214,3 +214,52 @@ def test_chain_in_cuda_graph(nq, chain_mod):
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(ch.h, eager)
+
+
+# ---------------------------------------------------------------------- grouped_ex
+
+@pytest.mark.parametrize("batch", [1, 3, 8, 16])
+def test_grouped_ex_optional_outputs(nq, orc, batch):
+    """y of every layer is the plain grouped call's y; y_bf16 is bf16(y) bit for bit;
+    y_rmsnorm_bf16 is within one unit of the oracle's normalisation of the same y.  Two
+    calls in a row give the same bits (the arrival counters reset themselves)."""
+    dev = torch.device("cuda")
+    shapes = [(512, 256, 128), (384, 512, 256), (1024, 384, 128)]
+    layers, plain = [], []
+    keep = []
+    for li, (m, n, r) in enumerate(shapes):
+        U = synth.random_words(m, r // 32, 90 + batch, li, "U")
+        V = synth.random_words(r, n // 32, 90 + batch, li, "V")
+        s1 = synth.scales_f16(m, 90 + batch, li, "s1")
+        s2 = synth.scales_f16(n, 90 + batch, li, "s2")
+        x = synth.activations_bf16(batch, n, 90 + batch, li)
+        t = [torch.from_numpy(a.view(v)).to(dev) for a, v in ((x, np.int16), (U, np.int32), (V, np.int32),
+                                                              (s1, np.int16), (s2, np.int16))]
+        y = torch.empty((batch, m), dtype=torch.float32, device=dev)
+        y2 = torch.empty_like(y)
+        yb = torch.empty((batch, m), dtype=torch.int16, device=dev) if li != 1 else None
+        yn = torch.empty((batch, m), dtype=torch.int16, device=dev) if li != 0 else None
+        keep += [t, y, y2, yb, yn]
+        layers.append((t[0], t[1], t[2], t[3], t[4], y, m, n, r, yb, yn))
+        plain.append((t[0], t[1], t[2], t[3], t[4], y2, m, n, r))
+    nq.lowrank_linear_fwd_grouped(plain, batch)
+    nq.lowrank_linear_fwd_grouped_ex(layers, batch)
+    torch.cuda.synchronize()
+    first = [(l[9].clone() if l[9] is not None else None, l[10].clone() if l[10] is not None else None)
+             for l in layers]
+    nq.lowrank_linear_fwd_grouped_ex(layers, batch)
+    torch.cuda.synchronize()
+    for li, l in enumerate(layers):
+        y = l[5]
+        assert torch.equal(y, plain[li][5]), li
+        y64 = y.cpu().numpy().astype(np.float64)
+        if l[9] is not None:
+            got = l[9].cpu().numpy().view(np.uint16)
+            assert np.array_equal(got, orc.round_to_bf16(y64)), li
+            assert torch.equal(l[9], first[li][0])
+        if l[10] is not None:
+            got = l[10].cpu().numpy().view(np.uint16)
+            want = orc.rms_normalize_bf16(y64)
+            assert within_one_ulp(got, want).all(), li
+            assert np.mean(got != want) <= 0.01, li
+            assert torch.equal(l[10], first[li][1])
