@@ -124,10 +124,20 @@ Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, const D
     return &w;
 }
 
+// Scratch a call needs: the decode launch's (batch <= 8), or the largest of the prefill
+// layers' split-K partials and counters.
 DecodeNeed decode_need(const DecodeCall* calls, int count, int64_t batch) {
     DecodeNeed d;
-    if (batch >= 1 && batch <= NQ_DECODE_MAX_BATCH)
+    if (batch >= 1 && batch <= NQ_DECODE_MAX_BATCH) {
         decode_workspace_need(calls, count, batch, kDecodeMaxSplits, &d.t, &d.tgmax, &d.partials, &d.counters);
+    } else if (batch > NQ_DECODE_MAX_BATCH) {
+        for (int i = 0; i < count; ++i) {
+            int64_t pf = 0, ci = 0;
+            prefill_workspace_need(calls[i].m, calls[i].n, calls[i].r, batch, &pf, &ci);
+            d.partials = pf > d.partials ? pf : d.partials;
+            d.counters = ci > d.counters ? ci : d.counters;
+        }
+    }
     return d;
 }
 
@@ -192,7 +202,15 @@ static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_line
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int st = NQ_OK;
     if (batch > NQ_DECODE_MAX_BATCH) {
-        Workspace* ws = workspace_for(m_max, n_max, r_max, batch, DecodeNeed(), &st);
+        DecodeNeed need;
+        for (int i = 0; i < count; ++i) {
+            const nq_linear_desc& L = desc(i);
+            const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, L.m, L.n, L.r};
+            const DecodeNeed d = decode_need(&c, 1, batch);
+            need.partials = d.partials > need.partials ? d.partials : need.partials;
+            need.counters = d.counters > need.counters ? d.counters : need.counters;
+        }
+        Workspace* ws = workspace_for(m_max, n_max, r_max, batch, need, &st);
         if (!ws) return st;
         for (int i = 0; i < count && st == NQ_OK; ++i) {
             const nq_linear_desc& L = desc(i);
@@ -343,6 +361,9 @@ int nq_device_status(void* stream) {
     unsigned word = 0;
     if (cudaMemcpy(&word, ws->status + 1, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) return NQ_ERR_CUDA;
     if (word != 0 && cudaMemset(ws->status + 1, 0, sizeof(unsigned)) != cudaSuccess) return NQ_ERR_CUDA;
+    // a kernel that gave up may have left arrival counters part-way: start them from zero again
+    if (word != 0 && cudaMemset(ws->counters, 0, sizeof(int) * (ws->counter_cap + 1)) != cudaSuccess)
+        return NQ_ERR_CUDA;
     return word == 0 ? NQ_OK : -(int)word;
 }
 

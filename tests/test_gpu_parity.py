@@ -206,12 +206,25 @@ def test_forward_prefill_sweep_sampled(nq, orc, batch):
     (256, 512, 128, 300),     # three N tiles of 128, ragged tail
     (128, 256, 256, 1025),    # N tiles of 256, one token in the last
     (1408, 640, 896, 517),    # several M tiles in both GEMMs
+    (256, 4096, 128, 9),      # split K: one row block in GEMM 1, two in GEMM 2, 9 tokens
+    (512, 2048, 384, 40),     # split K with a partial last 16-token group
+    (2432, 512, 1280, 64),    # split K in GEMM 1, 19 row blocks in GEMM 2
+    (128, 8192, 128, 17),     # one row block each: the most splits
 ])
 def test_prefill_tiles(nq, orc, m, n, r, batch):
     c = Case(orc, nq, m, n, r, batch, seed=m * 7 + batch)
     y = c.gpu()
     nq.device_status()
     assert rel_err(y, c.oracle(orc)) <= TOL
+
+
+def test_prefill_split_k_deterministic(nq, orc):
+    # few row blocks: K is split over many CTAs and the partials are added in split order
+    c = Case(orc, nq, 384, 4096, 256, 16, seed=31)
+    a, b = c.gpu(), c.gpu()
+    nq.device_status()
+    assert np.array_equal(a, b)
+    assert rel_err(a, c.oracle(orc)) <= TOL
 
 
 def test_prefill_deterministic_and_status(nq, orc):
