@@ -810,8 +810,11 @@ struct Plan {
     int64_t units;
 };
 
-// Estimated SM clocks of one k-block step of a tile of n tokens: the MMAs (4 x 128 x n x 16
-// at 8192 flop per clock: 2 clocks per token) or the sign expansion (~160 clocks).
+// Relative cost of one k-block step of a tile of n tokens: the MMAs (4 x 128 x n x 16 at
+// 8192 flop per clock: 2 clocks per token) or the sign expansion (~160 clocks).  (Scaling
+// the floor to the ~1000 clocks a step measures at 16 tokens made the plan choose more
+// splits, which measured slower: the split items' partials and reduction cost more than
+// the model's estimate, so the low floor stands in for both.)
 double step_clk(int64_t n) {
     const double mma = 2.0 * (double)((n + 15) & ~15ll);
     return mma > 160.0 ? mma : 160.0;
