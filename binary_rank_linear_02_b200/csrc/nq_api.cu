@@ -367,6 +367,14 @@ int nq_device_status(void* stream) {
     return word == 0 ? NQ_OK : -(int)word;
 }
 
+int nq_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+    if (limit_ns < 1000 || limit_ns > 10000000000ll) return NQ_ERR_VALUE;
+    int st = NQ_OK;
+    Workspace* ws = workspace_for(128, 128, 128, 0, DecodeNeed(), &st);
+    if (!ws) return st;
+    return selftest_wait_timeout(limit_ns, ws, static_cast<cudaStream_t>(stream));
+}
+
 int nq_workspace_reserve(int64_t m, int64_t n, int64_t r, int64_t batch) {
     if (m <= 0 || n <= 0 || r <= 0 || m % 128 || n % 128 || r % 128 || m > kMaxDim || n > kMaxDim ||
         r > kMaxRank)

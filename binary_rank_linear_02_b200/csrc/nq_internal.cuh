@@ -95,6 +95,8 @@ int decode_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, 
 // Scratch of the prefill path's split-K items (fp32 partial tiles and arrival counters).
 void prefill_workspace_need(int64_t m, int64_t n, int64_t r, int64_t batch, int64_t* partial_floats,
                             int64_t* counter_ints);
+// Runs the bounded device wait on a barrier nothing arrives on (failure-path self-test).
+int selftest_wait_timeout(int64_t limit_ns, Workspace* ws, cudaStream_t stream);
 int prefill_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const uint16_t* s1,
                     const uint16_t* s2, int64_t m, int64_t n, int64_t r, int64_t batch, float* y,
                     Workspace* ws, cudaStream_t stream);

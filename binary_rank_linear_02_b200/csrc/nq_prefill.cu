@@ -73,13 +73,13 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 
 // Bounded wait: false if the CTA aborted or the limit expired (then the CTA aborts).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned* status) {
+                                          unsigned* status, unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (true) {
         if (mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit_ns) {
             *abort_flag = 1;
             atomicExch(status, (unsigned)(-NQ_ERR_TIMEOUT));
             return false;
@@ -739,6 +739,21 @@ tile_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint32_t* __res
     }
 }
 
+// Self-test of the failure path: the GEMMs' bounded mbarrier wait on a barrier that
+// nothing arrives on, with a short limit; it gives up, records NQ_ERR_TIMEOUT in the
+// status word exactly as a GEMM would, and the kernel exits.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns, unsigned* status) {
+    __shared__ unsigned long long bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, status, limit_ns);
+}
+
 // x'[b][perm(j)] = fp16(bf16 x[b][j] * fp16 s2[j]); one thread per 32-column group.
 __global__ void prescale_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ s2, int64_t n,
                                 int64_t batch, uint16_t* __restrict__ xp) {
@@ -952,6 +967,11 @@ int run_gemms(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const
 }
 
 }  // namespace
+
+int selftest_wait_timeout(int64_t limit_ns, Workspace* ws, cudaStream_t stream) {
+    wait_selftest_kernel<<<1, 32, 0, stream>>>((unsigned long long)limit_ns, ws->status + 1);
+    return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
+}
 
 void prefill_workspace_need(int64_t m, int64_t n, int64_t r, int64_t batch, int64_t* partial_floats,
                             int64_t* counter_ints) {

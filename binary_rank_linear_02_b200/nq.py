@@ -84,6 +84,8 @@ def _load() -> ctypes.CDLL:
     L.nq_lowrank_linear_fwd_grouped_ex.restype = ctypes.c_int
     L.nq_device_status.argtypes = [p]
     L.nq_device_status.restype = ctypes.c_int
+    L.nq_selftest_wait_timeout.argtypes = [i64, p]
+    L.nq_selftest_wait_timeout.restype = ctypes.c_int
     L.nq_cast_f32_to_bf16.argtypes = [p, i64, p, p]
     L.nq_cast_f32_to_bf16.restype = ctypes.c_int
     L.nq_rms_normalize_bf16.argtypes = [p, i64, i64, p, p]
@@ -154,6 +156,10 @@ def device_status(stream=None) -> None:
 
     h = int(stream) if stream is not None else torch.cuda.current_stream().cuda_stream
     _check(_lib.nq_device_status(h), "nq_device_status")
+
+
+def nq_selftest_wait_timeout(limit_ns: int, stream: int = 0) -> int:
+    return _lib.nq_selftest_wait_timeout(limit_ns, stream)
 
 
 def nq_version() -> int:

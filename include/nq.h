@@ -227,6 +227,16 @@ int nq_workspace_reserve(int64_t m, int64_t n, int64_t r, int64_t batch);
  */
 int nq_device_status(void* stream);
 
+/*
+ * nq_selftest_wait_timeout -- exercise the failure path of the device-side waits: a kernel
+ * runs the same bounded wait the tensor-core kernels use, on a barrier that nothing ever
+ * arrives on, gives up after `limit_ns` nanoseconds of GPU time and records NQ_ERR_TIMEOUT
+ * in the device status word.  The next nq_device_status then returns NQ_ERR_TIMEOUT (and
+ * clears it); the device stays usable.  No counterpart in the pages: a property of this
+ * library.  1000 <= limit_ns <= 1e10, else NQ_ERR_VALUE.  Asynchronous on `stream`.
+ */
+int nq_selftest_wait_timeout(int64_t limit_ns, void* stream);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int nq_version(void);
 

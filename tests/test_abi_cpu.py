@@ -187,3 +187,8 @@ def test_grouped_ex_argument_errors(nq):
     assert f(a, 2, 1, 0) == nq.NQ_ERR_ALIGN
     arr[1].y_rmsnorm_bf16 = ptr[7]
     assert f(a, 2, 1, 0) == nq.NQ_ERR_PTRKIND  # host memory is refused
+
+
+def test_selftest_argument_errors(nq):
+    assert nq.nq_selftest_wait_timeout(10, 0) == nq.NQ_ERR_VALUE
+    assert nq.nq_selftest_wait_timeout(10**11, 0) == nq.NQ_ERR_VALUE

@@ -270,3 +270,22 @@ def test_grouped_llama2_7b_block(nq, orc):
     torch.cuda.synchronize()
     for c, y in zip(cases, ys):
         assert rel_err(y.cpu().numpy(), c.oracle(orc)) <= TOL
+
+
+# ------------------------------------------------------------------ failure path
+
+def test_device_wait_timeout_is_reported_and_cleared(nq, orc):
+    """A bounded device wait that runs out (a barrier nothing arrives on, 2 ms limit) is
+    reported once by nq_device_status as NQ_ERR_TIMEOUT, then cleared, and the context
+    keeps working."""
+    s = torch.cuda.current_stream().cuda_stream
+    assert nq.nq_selftest_wait_timeout(2_000_000, s) == nq.NQ_OK
+    assert nq.nq_device_status(s) == nq.NQ_ERR_TIMEOUT
+    assert nq.nq_device_status(s) == nq.NQ_OK
+    with pytest.raises(nq.NQError):
+        nq.nq_selftest_wait_timeout(2_000_000, s)
+        nq.device_status(s)
+    nq.device_status(s)
+    c = Case(orc, nq, 256, 512, 128, 20, seed=5)
+    assert rel_err(c.gpu(), c.oracle(orc)) <= TOL
+    assert nq.nq_selftest_wait_timeout(10, s) == nq.NQ_ERR_VALUE
