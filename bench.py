@@ -512,15 +512,28 @@ def run_prefill_only(args, device, peaks):
 
 
 def run_e2e(work, stream, steps, device):
+    """End to end through the public API: one nq_lowrank_linear_fwd_grouped call per step
+    with every layer's x and y in pinned host memory (the call copies x in, runs the launch
+    pair, copies y out and synchronises); wall clock around the steps.  Also the same with
+    seven nq_lowrank_linear_fwd calls per step (one copy-in, launch pair, copy-out and sync
+    each)."""
     import torch
 
     nq = work.nq
     xs = [x.cpu().pin_memory() for x in work.x]
     ys = [torch.empty(y.shape, dtype=torch.float32).pin_memory() for y in work.y]
-    fwd = nq.lib().nq_lowrank_linear_fwd
     h = stream.cuda_stream
+    descs = [nq.make_descs([(xs[li], *per[li][:2], *per[li][2:], ys[li], m, n, r)
+                            for li, (_, m, n, r) in enumerate(work.layers)]) for per in work.sets]
+    grouped = nq.lib().nq_lowrank_linear_fwd_grouped
+    fwd = nq.lib().nq_lowrank_linear_fwd
 
-    def one(i):
+    def one_grouped(i):
+        st = grouped(ctypes.addressof(descs[i % work.copies]), len(work.layers), work.batch, h)
+        if st != 0:
+            raise RuntimeError(nq.nq_status_string(st))
+
+    def one_per_layer(i):
         per = work.sets[i % work.copies]
         for li, (name, m, n, r) in enumerate(work.layers):
             Upk, Vpk, s1, s2 = per[li]
@@ -529,20 +542,26 @@ def run_e2e(work, stream, steps, device):
             if st != 0:
                 raise RuntimeError(nq.nq_status_string(st))
 
-    for i in range(3):
-        one(i)
-    torch.cuda.synchronize()
-    t0 = time.perf_counter()
-    for i in range(steps):
-        one(i)
-    torch.cuda.synchronize()
-    dt = time.perf_counter() - t0
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for i in range(steps):
+            fn(i)
+        torch.cuda.synchronize()
+        return time.perf_counter() - t0
+
+    dt = timed(one_grouped)
+    dt_layers = timed(one_per_layer)
     h2d = sum(x.numel() * 2 for x in xs)
     d2h = sum(y.numel() * 4 for y in ys)
     return {"value": round(work.step_bytes * steps / dt / 1e9, 2), "unit": "GB/s", "steps": steps,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "how": "nq_lowrank_linear_fwd with pinned host x and y per layer (copy in, both kernels, copy out, "
-                   "stream sync), wall clock"}
+            "us_per_step": round(dt / steps * 1e6, 2),
+            "per_layer_calls_gbs": round(work.step_bytes * steps / dt_layers / 1e9, 2),
+            "how": "one nq_lowrank_linear_fwd_grouped call per step with pinned host x and y (copy in, "
+                   "launch pair, copy out, stream sync inside the call), wall clock"}
 
 
 # ------------------------------------------------------------------ the oracle on the host

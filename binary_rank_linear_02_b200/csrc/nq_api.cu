@@ -1,6 +1,8 @@
 // nq_api.cu -- the C ABI of libnq (declared in include/nq.h): argument checks, the
 // per-device workspace, host-memory staging and the decode / prefill dispatch.
+#include <algorithm>
 #include <mutex>
+#include <vector>
 #include <string.h>
 
 #include "nq_internal.cuh"
@@ -33,6 +35,17 @@ int pointer_kind(const void* p) {
         return 0;
     }
     return (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) ? 1 : 0;
+}
+
+// Host memory the device can address: the device address of page-locked (pinned) host
+// memory, nullptr for pageable memory or anything else.
+void* pinned_device_ptr(const void* p) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return attr.type == cudaMemoryTypeHost ? attr.devicePointer : nullptr;
 }
 
 }  // namespace
@@ -164,7 +177,9 @@ static int ensure_staging(Workspace* w, size_t xbytes, size_t ybytes) {
 using namespace nq;
 
 // The grouped forward over `count` descriptors `stride` bytes apart; `ex` (may be NULL)
-// adds the optional bf16 outputs of nq_linear_desc_ex.
+// adds the optional bf16 outputs of nq_linear_desc_ex.  Without `ex`, a layer's x and y may
+// be host memory: they are staged through the workspace (one copy per buffer), the layers
+// run as usual, host y are copied back and the call synchronises the stream.
 static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_linear_desc_ex* ex, int count,
                        int64_t batch, void* stream) {
     auto desc = [&](int i) -> const nq_linear_desc& {
@@ -190,19 +205,35 @@ static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_line
         n_max = L.n > n_max ? L.n : n_max;
         r_max = L.r > r_max ? L.r : r_max;
     }
+    // memory kinds: weights on the device; x and y on the device, or (plain call) on the host.
+    // Pinned host x are gathered into the workspace by one kernel; pinned host y are written
+    // by the kernels through their device address; pageable x / y go through copies.
+    std::vector<char> x_host(count, 0), y_host(count, 0);
+    std::vector<void*> x_pin(count, nullptr), y_pin(count, nullptr);
+    size_t xbytes = 0, ybytes = 0;
     for (int i = 0; i < count; ++i) {
         const nq_linear_desc& L = desc(i);
-        if (!pointer_kind(L.x) || !pointer_kind(L.Upk) || !pointer_kind(L.Vpk) || !pointer_kind(L.s1) ||
-            !pointer_kind(L.s2) || !pointer_kind(L.y))
+        if (!pointer_kind(L.Upk) || !pointer_kind(L.Vpk) || !pointer_kind(L.s1) || !pointer_kind(L.s2))
             return NQ_ERR_PTRKIND;
-        if (ex && ((ex[i].y_bf16 && !pointer_kind(ex[i].y_bf16)) ||
+        x_host[i] = pointer_kind(L.x) == 0;
+        y_host[i] = pointer_kind(L.y) == 0;
+        if (ex && (x_host[i] || y_host[i] || (ex[i].y_bf16 && !pointer_kind(ex[i].y_bf16)) ||
                    (ex[i].y_rmsnorm_bf16 && !pointer_kind(ex[i].y_rmsnorm_bf16))))
             return NQ_ERR_PTRKIND;
+        if (x_host[i]) {
+            x_pin[i] = pinned_device_ptr(L.x);
+            xbytes += align_up(sizeof(uint16_t) * (size_t)batch * L.n, 256);
+        }
+        if (y_host[i]) {
+            y_pin[i] = pinned_device_ptr(L.y);
+            if (!y_pin[i]) ybytes += align_up(sizeof(float) * (size_t)batch * L.m, 256);
+        }
     }
+    const bool any_host = xbytes || std::find(y_host.begin(), y_host.end(), 1) != y_host.end();
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int st = NQ_OK;
+    DecodeNeed need;
     if (batch > NQ_DECODE_MAX_BATCH) {
-        DecodeNeed need;
         for (int i = 0; i < count; ++i) {
             const nq_linear_desc& L = desc(i);
             const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, L.m, L.n, L.r};
@@ -210,37 +241,94 @@ static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_line
             need.partials = d.partials > need.partials ? d.partials : need.partials;
             need.counters = d.counters > need.counters ? d.counters : need.counters;
         }
-        Workspace* ws = workspace_for(m_max, n_max, r_max, batch, need, &st);
+    }
+    Workspace* ws = nullptr;
+    std::vector<const void*> xs(count);
+    std::vector<float*> ys(count);
+    if (xbytes || ybytes) {
+        ws = workspace_for(m_max, n_max, r_max, batch, need, &st);
+        if (!ws) return st;
+        st = ensure_staging(ws, xbytes, ybytes);
+        if (st != NQ_OK) return st;
+    }
+    size_t xo = 0, yo = 0;
+    GatherList gl;
+    gl.count = 0;
+    for (int i = 0; i < count; ++i) {
+        const nq_linear_desc& L = desc(i);
+        xs[i] = L.x;
+        ys[i] = L.y;
+        if (x_host[i]) {
+            const size_t b = sizeof(uint16_t) * (size_t)batch * L.n;
+            char* dst = static_cast<char*>(ws->xstage) + xo;
+            if (x_pin[i]) {
+                gl.seg[gl.count++] = GatherSeg{x_pin[i], dst, b};
+                if (gl.count == kMaxGather) {
+                    if (gather_device(gl, s) != NQ_OK) return NQ_ERR_CUDA;
+                    gl.count = 0;
+                }
+            } else if (cudaMemcpyAsync(dst, L.x, b, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+                return NQ_ERR_CUDA;
+            }
+            xs[i] = dst;
+            xo += align_up(b, 256);
+        }
+        if (y_host[i]) {
+            if (y_pin[i]) {
+                ys[i] = static_cast<float*>(y_pin[i]);
+            } else {
+                ys[i] = reinterpret_cast<float*>(reinterpret_cast<char*>(ws->ystage) + yo);
+                yo += align_up(sizeof(float) * (size_t)batch * L.m, 256);
+            }
+        }
+    }
+    if (gl.count > 0 && gather_device(gl, s) != NQ_OK) return NQ_ERR_CUDA;
+    if (batch > NQ_DECODE_MAX_BATCH) {
+        if (!ws) ws = workspace_for(m_max, n_max, r_max, batch, need, &st);
         if (!ws) return st;
         for (int i = 0; i < count && st == NQ_OK; ++i) {
             const nq_linear_desc& L = desc(i);
-            st = prefill_forward(static_cast<const uint16_t*>(L.x), L.Upk, L.Vpk, static_cast<const uint16_t*>(L.s1),
-                                 static_cast<const uint16_t*>(L.s2), L.m, L.n, L.r, batch, L.y, ws, s);
+            st = prefill_forward(static_cast<const uint16_t*>(xs[i]), L.Upk, L.Vpk, static_cast<const uint16_t*>(L.s1),
+                                 static_cast<const uint16_t*>(L.s2), L.m, L.n, L.r, batch, ys[i], ws, s);
             // the optional outputs by the stand-alone kernels, after the layer
             if (st == NQ_OK && ex && ex[i].y_bf16)
-                st = cast_f32_bf16_device(L.y, batch * L.m, static_cast<uint16_t*>(ex[i].y_bf16), s);
+                st = cast_f32_bf16_device(ys[i], batch * L.m, static_cast<uint16_t*>(ex[i].y_bf16), s);
             if (st == NQ_OK && ex && ex[i].y_rmsnorm_bf16)
-                st = rms_normalize_bf16_device(L.y, batch, L.m, static_cast<uint16_t*>(ex[i].y_rmsnorm_bf16), s);
+                st = rms_normalize_bf16_device(ys[i], batch, L.m, static_cast<uint16_t*>(ex[i].y_rmsnorm_bf16), s);
         }
-        return st;
-    }
-    for (int i0 = 0; i0 < count && st == NQ_OK; i0 += kMaxGroup) {
-        const int cnt = count - i0 < kMaxGroup ? count - i0 : kMaxGroup;
-        DecodeCall calls[kMaxGroup];
-        for (int i = 0; i < cnt; ++i) {
-            const nq_linear_desc& L = desc(i0 + i);
-            calls[i] = DecodeCall{static_cast<const uint16_t*>(L.x), L.Upk, L.Vpk, static_cast<const uint16_t*>(L.s1),
-                                  static_cast<const uint16_t*>(L.s2), L.y, L.m, L.n, L.r};
-            if (ex) {
-                calls[i].y_bf16 = static_cast<uint16_t*>(ex[i0 + i].y_bf16);
-                calls[i].y_norm = static_cast<uint16_t*>(ex[i0 + i].y_rmsnorm_bf16);
+    } else {
+        for (int i0 = 0; i0 < count && st == NQ_OK; i0 += kMaxGroup) {
+            const int cnt = count - i0 < kMaxGroup ? count - i0 : kMaxGroup;
+            DecodeCall calls[kMaxGroup];
+            for (int i = 0; i < cnt; ++i) {
+                const nq_linear_desc& L = desc(i0 + i);
+                calls[i] = DecodeCall{static_cast<const uint16_t*>(xs[i0 + i]), L.Upk, L.Vpk,
+                                      static_cast<const uint16_t*>(L.s1), static_cast<const uint16_t*>(L.s2),
+                                      ys[i0 + i], L.m, L.n, L.r};
+                if (ex) {
+                    calls[i].y_bf16 = static_cast<uint16_t*>(ex[i0 + i].y_bf16);
+                    calls[i].y_norm = static_cast<uint16_t*>(ex[i0 + i].y_rmsnorm_bf16);
+                }
             }
+            ws = workspace_for(m_max, n_max, r_max, batch, decode_need(calls, cnt, batch), &st);
+            if (!ws) return st;
+            st = decode_forward_group(calls, cnt, batch, ws, s);
         }
-        Workspace* ws = workspace_for(m_max, n_max, r_max, batch, decode_need(calls, cnt, batch), &st);
-        if (!ws) return st;
-        st = decode_forward_group(calls, cnt, batch, ws, s);
     }
-    return st;
+    if (st != NQ_OK) return st;
+    if (ybytes) {
+        for (int i = 0; i < count; ++i) {
+            if (!y_host[i] || y_pin[i]) continue;
+            const nq_linear_desc& L = desc(i);
+            if (cudaMemcpyAsync(L.y, ys[i], sizeof(float) * (size_t)batch * L.m, cudaMemcpyDeviceToHost, s) !=
+                cudaSuccess)
+                return NQ_ERR_CUDA;
+        }
+    }
+    if (any_host) {
+        if (cudaStreamSynchronize(s) != cudaSuccess) return NQ_ERR_CUDA;
+    }
+    return NQ_OK;
 }
 
 extern "C" {
@@ -401,39 +489,18 @@ int nq_lowrank_linear_fwd(const void* x, const uint32_t* Upk, const uint32_t* Vp
         return NQ_ERR_ALIGN;
     if (!pointer_kind(Upk) || !pointer_kind(Vpk) || !pointer_kind(s1) || !pointer_kind(s2))
         return NQ_ERR_PTRKIND;
-    const bool x_host = pointer_kind(x) == 0, y_host = pointer_kind(y) == 0;
-
-    int st = NQ_OK;
-    const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, m, n, r};
-    Workspace* ws = workspace_for(m, n, r, batch, decode_need(&c, 1, batch), &st);
-    if (!ws) return st;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t xbytes = sizeof(uint16_t) * (size_t)batch * n, ybytes = sizeof(float) * (size_t)batch * m;
-    if (x_host || y_host) {
-        st = ensure_staging(ws, x_host ? xbytes : 0, y_host ? ybytes : 0);
-        if (st != NQ_OK) return st;
-    }
-    const uint16_t* xd = static_cast<const uint16_t*>(x);
-    float* yd = y;
-    if (x_host) {
-        if (cudaMemcpyAsync(ws->xstage, x, xbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return NQ_ERR_CUDA;
-        xd = static_cast<const uint16_t*>(ws->xstage);
-    }
-    if (y_host) yd = ws->ystage;
-
-    const uint16_t* s1h = static_cast<const uint16_t*>(s1);
-    const uint16_t* s2h = static_cast<const uint16_t*>(s2);
-    if (batch <= NQ_DECODE_MAX_BATCH)
-        st = decode_forward(xd, Upk, Vpk, s1h, s2h, m, n, r, batch, yd, ws, s);
-    else
-        st = prefill_forward(xd, Upk, Vpk, s1h, s2h, m, n, r, batch, yd, ws, s);
-    if (st != NQ_OK) return st;
-
-    if (y_host) {
-        if (cudaMemcpyAsync(y, ws->ystage, ybytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return NQ_ERR_CUDA;
-        if (cudaStreamSynchronize(s) != cudaSuccess) return NQ_ERR_CUDA;
-    }
-    return NQ_OK;
+    // one layer of the grouped path, which also handles host x / y
+    nq_linear_desc d;
+    d.x = x;
+    d.Upk = Upk;
+    d.Vpk = Vpk;
+    d.s1 = s1;
+    d.s2 = s2;
+    d.y = y;
+    d.m = m;
+    d.n = n;
+    d.r = r;
+    return grouped_run(&d, sizeof(d), nullptr, 1, batch, stream);
 }
 
 }  // extern "C"

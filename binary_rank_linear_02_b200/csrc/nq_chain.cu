@@ -95,7 +95,31 @@ __global__ void __launch_bounds__(kNormThreads, 1) rms_norm_kernel(const float* 
     }
 }
 
+// Copies up to kMaxGather buffers (16-byte multiples, 16-byte aligned), one per grid row;
+// used to bring the x of a call from pinned host memory (read through its device
+// address) into the device staging buffer in one launch instead of one copy per layer.
+__global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ GatherList list) {
+    if ((int)blockIdx.y >= list.count) return;
+    const GatherSeg& g = list.seg[blockIdx.y];
+    const uint4* src = static_cast<const uint4*>(g.src);
+    uint4* dst = static_cast<uint4*>(g.dst);
+    const int64_t n = (int64_t)(g.bytes / 16);
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = src[i];
+}
+
 }  // namespace
+
+int gather_device(const GatherList& list, cudaStream_t stream) {
+    if (list.count <= 0) return NQ_OK;
+    size_t most = 0;
+    for (int i = 0; i < list.count; ++i) most = list.seg[i].bytes > most ? list.seg[i].bytes : most;
+    int gx = (int)((most / 16 + 255) / 256);
+    if (gx < 1) gx = 1;
+    if (gx > 32) gx = 32;
+    gather_kernel<<<dim3((unsigned)gx, (unsigned)list.count), 256, 0, stream>>>(list);
+    return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
+}
 
 int cast_f32_bf16_device(const float* src, int64_t count, uint16_t* dst, cudaStream_t stream) {
     int64_t blocks = (count / 8 + kCastThreads - 1) / kCastThreads;

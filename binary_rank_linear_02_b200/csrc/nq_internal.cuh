@@ -104,6 +104,17 @@ int prefill_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk,
 int pack_device(const int8_t* signs, int64_t rows, int64_t cols, uint32_t* out, unsigned* flag,
                 cudaStream_t stream);
 int unpack_device(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* out, cudaStream_t stream);
+constexpr int kMaxGather = 16;
+struct GatherSeg {
+    const void* src;
+    void* dst;
+    size_t bytes;  // a multiple of 16
+};
+struct GatherList {
+    GatherSeg seg[kMaxGather];
+    int count;
+};
+int gather_device(const GatherList& list, cudaStream_t stream);
 int cast_f32_bf16_device(const float* src, int64_t count, uint16_t* dst, cudaStream_t stream);
 int rms_normalize_bf16_device(const float* src, int64_t rows, int64_t cols, uint16_t* dst, cudaStream_t stream);
 

@@ -89,9 +89,11 @@ int nq_unpack_signs(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* 
  *   y    : batch x m float32, row-major (written)
  *   m, n, r : positive multiples of 128, each at most 1<<20
  *   batch   : >= 0; 0 is a no-op returning NQ_OK
- * x and y may be device memory, or host memory (pageable or pinned): host x is copied
- * to the device on `stream` first, host y is copied back and the call then synchronises
- * `stream` before returning.  Device buffers are used asynchronously on `stream`.
+ * x and y may be device memory, or host memory (pageable or pinned): host x is brought to
+ * the device on `stream` first (pinned x by a copy kernel that reads it through its device
+ * address, pageable x by a copy), pinned host y is written by the kernels directly and
+ * pageable host y copied back; with any host buffer the call then synchronises `stream`
+ * before returning.  Device buffers are used asynchronously on `stream`.
  * Every pointer must be 16-byte aligned.
  * Path: batch <= NQ_DECODE_MAX_BATCH runs the decode path (two binary GEMV stages on the
  * CUDA cores and integer tensor-core instructions, t kept in the workspace); larger
@@ -126,7 +128,11 @@ typedef struct nq_linear_desc {
  * decode path (batch <= NQ_DECODE_MAX_BATCH) runs up to 16 layers per launch pair, so
  * small layers share the launch and dependency latency.  No layer's y may overlap
  * another layer's inputs.  Argument checks as nq_lowrank_linear_fwd, plus count >= 0
- * (0 is a no-op) and `layers` non-NULL; host-memory buffers are refused (NQ_ERR_PTRKIND).
+ * (0 is a no-op) and `layers` non-NULL.  Weights (Upk, Vpk, s1, s2) must be device memory
+ * (else NQ_ERR_PTRKIND).  Each layer's x and y may be device or host memory, handled as
+ * in nq_lowrank_linear_fwd (pinned x gathered by one kernel for all layers, pinned y
+ * written directly, pageable buffers copied); with any host buffer the call synchronises
+ * `stream` before returning, with only device buffers it is asynchronous.
  */
 int nq_lowrank_linear_fwd_grouped(const nq_linear_desc* layers, int count, int64_t batch, void* stream);
 
@@ -174,7 +180,8 @@ typedef struct nq_linear_desc_ex {
  * On the decode path both are produced by the forward's own kernels (no extra launch); on
  * the prefill path by the stand-alone kernels after the layer.  Optional pointers are
  * device memory, 16-byte aligned, and overlap no other buffer of the call.  Errors as
- * nq_lowrank_linear_fwd_grouped.
+ * nq_lowrank_linear_fwd_grouped, except that every buffer, x and y included, must be
+ * device memory (else NQ_ERR_PTRKIND).
  */
 int nq_lowrank_linear_fwd_grouped_ex(const nq_linear_desc_ex* layers, int count, int64_t batch, void* stream);
 

@@ -289,3 +289,33 @@ def test_device_wait_timeout_is_reported_and_cleared(nq, orc):
     c = Case(orc, nq, 256, 512, 128, 20, seed=5)
     assert rel_err(c.gpu(), c.oracle(orc)) <= TOL
     assert nq.nq_selftest_wait_timeout(10, s) == nq.NQ_ERR_VALUE
+
+
+@pytest.mark.parametrize("batch", [1, 5, 20])
+def test_grouped_host_buffers(nq, orc, batch):
+    """Grouped call with x and y in host memory (pinned and pageable mixed, one layer's
+    buffers on the device): same bits as the device-buffer call."""
+    shapes = [(512, 512, 128), (384, 640, 256), (1024, 256, 384)]
+    cases = [Case(orc, nq, m, n, r, batch, seed=950 + i) for i, (m, n, r) in enumerate(shapes)]
+    dev_layers, host_layers, host_ys = [], [], []
+    for i, c in enumerate(cases):
+        y_dev = torch.empty((batch, c.m), dtype=torch.float32, device="cuda")
+        dev_layers.append((c.x_d, c.Upk, c.Vpk, c.s1_d, c.s2_d, y_dev, c.m, c.n, c.r))
+        if i == 2:  # device buffers in a call that also has host ones
+            xh, yh = c.x_d, torch.empty((batch, c.m), dtype=torch.float32, device="cuda")
+        elif i == 1:  # pageable host memory
+            xh = np.ascontiguousarray(c.x)
+            yh = np.zeros((batch, c.m), dtype=np.float32)
+        else:  # pinned host memory
+            xh = torch.from_numpy(c.x.view(np.int16)).pin_memory()
+            yh = torch.empty((batch, c.m), dtype=torch.float32).pin_memory()
+        host_layers.append((xh, c.Upk, c.Vpk, c.s1_d, c.s2_d, yh, c.m, c.n, c.r))
+        host_ys.append(yh)
+    nq.lowrank_linear_fwd_grouped(dev_layers, batch)
+    nq.lowrank_linear_fwd_grouped(host_layers, batch, stream=torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    for i, c in enumerate(cases):
+        want = dev_layers[i][5].cpu().numpy()
+        got = host_ys[i].cpu().numpy() if isinstance(host_ys[i], torch.Tensor) else host_ys[i]
+        assert np.array_equal(got, want), i
+        assert rel_err(got, c.oracle(orc)) <= TOL
