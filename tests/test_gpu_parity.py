@@ -261,9 +261,24 @@ def test_grouped_more_than_one_launch(nq, orc):
         assert rel_err(y.cpu().numpy(), c.oracle(orc)) <= TOL
 
 
-def test_grouped_llama2_7b_block(nq, orc):
-    batch = 1
+@pytest.mark.parametrize("batch", [1, 8])
+def test_grouped_llama2_7b_block(nq, orc, batch):
+    """The benchmark's decode step: the seven Llama-2-7B-shaped layers in one grouped call
+    (the launch configuration bench.py times), every output checked."""
     cases = [Case(orc, nq, m, n, r, batch, seed=960 + i) for i, (_, m, n, r) in enumerate(synth.LLAMA2_7B_LAYERS)]
+    ys = [torch.empty((batch, c.m), dtype=torch.float32, device="cuda") for c in cases]
+    nq.lowrank_linear_fwd_grouped([(c.x_d, c.Upk, c.Vpk, c.s1_d, c.s2_d, y, c.m, c.n, c.r)
+                                   for c, y in zip(cases, ys)], batch)
+    torch.cuda.synchronize()
+    for c, y in zip(cases, ys):
+        assert rel_err(y.cpu().numpy(), c.oracle(orc)) <= TOL
+
+
+@pytest.mark.parametrize("batch", [1, 4])
+def test_grouped_llama2_70b_block(nq, orc, batch):
+    """The Llama-2-70B-shaped block in one grouped call (up to 28 column splits per layer,
+    a 3840-column stage-2 span), every output checked."""
+    cases = [Case(orc, nq, m, n, r, batch, seed=980 + i) for i, (_, m, n, r) in enumerate(synth.LLAMA2_70B_LAYERS)]
     ys = [torch.empty((batch, c.m), dtype=torch.float32, device="cuda") for c in cases]
     nq.lowrank_linear_fwd_grouped([(c.x_d, c.Upk, c.Vpk, c.s1_d, c.s2_d, y, c.m, c.n, c.r)
                                    for c, y in zip(cases, ys)], batch)
