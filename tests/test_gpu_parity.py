@@ -114,6 +114,18 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("m,n,r,batch", [
+    (128, 131072, 128, 1),   # 1024 column blocks: 16 per stage-1 CTA, two chunks through the ring
+    (256, 98304, 256, 5),    # 768 column blocks: 12 per CTA, a full chunk and a ragged one
+    (384, 70144, 128, 2),    # just past 64 splits of 8 column blocks
+])
+def test_forward_wide_input(nq, orc, m, n, r, batch):
+    """Very wide layers, where a stage-1 CTA takes several 1024-column chunks (the split
+    count is capped), exercising the chunk ring."""
+    c = Case(orc, nq, m, n, r, batch, seed=77 + n)
+    assert rel_err(c.gpu(), c.oracle(orc)) <= TOL
+
+
 @pytest.mark.parametrize("m,n,r,batch", SMALL)
 def test_forward_small(nq, orc, m, n, r, batch):
     c = Case(orc, nq, m, n, r, batch, seed=1000 + m + n + r + batch)
