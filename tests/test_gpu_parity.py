@@ -118,10 +118,13 @@ SMALL = [
     (128, 131072, 128, 1),   # 1024 column blocks: 16 per stage-1 CTA, two chunks through the ring
     (256, 98304, 256, 5),    # 768 column blocks: 12 per CTA, a full chunk and a ragged one
     (384, 70144, 128, 2),    # just past 64 splits of 8 column blocks
+    (256, 512, 16384, 8),    # deep rank: 128 stage-1 row blocks, 16 stage-2 column spans
+    (262144, 128, 128, 1),   # tall output: 2048 stage-2 row tiles
 ])
 def test_forward_wide_input(nq, orc, m, n, r, batch):
-    """Very wide layers, where a stage-1 CTA takes several 1024-column chunks (the split
-    count is capped), exercising the chunk ring."""
+    """Extreme shapes: very wide layers, where a stage-1 CTA takes several 1024-column
+    chunks (the split count is capped) through its ring; a deep rank that stage 2 holds on
+    chip in many spans; a very tall output."""
     c = Case(orc, nq, m, n, r, batch, seed=77 + n)
     assert rel_err(c.gpu(), c.oracle(orc)) <= TOL
 
