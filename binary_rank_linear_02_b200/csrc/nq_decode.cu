@@ -290,7 +290,7 @@ __device__ __forceinline__ void zero_acc(int (&acc)[NTG][4][4]) {
 }
 
 // ------------------------------------------------------------------ stage 1
-// CTA = 64 rows of V^T of one layer x one column split (cps column blocks, staged kChunk
+// CTA = 128 rows of V^T of one layer x one column split (cps column blocks, staged kChunk
 // columns at a time); warp w owns rows 16w..16w+15.  Each chunk has its own quantisation
 // exponent per token, so the warp converts its integer sums to fp32 after every chunk.
 // With several splits, the CTAs of a row block leave fp32 partials and the last to arrive
@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
         if (ch + 1 < nchunks) cp_async_wait<1>(); else cp_async_wait<0>();
         __syncthreads();
         // v = s2 * x (exact in fp32) and its per-token max: every thread takes a column
-        // stripe of every token, then the four warps' maxima are combined
+        // stripe of every token, then the warps' maxima are combined
         const uint16_t* ss = xchunk(buf, batch);
         for (int tok = 0; tok < batch; ++tok) {
             const uint16_t* xs = xchunk(buf, tok);
@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
         }
     }
 
-    // this CTA's sums for its 64 rows, into shared memory
+    // this CTA's sums for its 128 rows, into shared memory
 #pragma unroll
     for (int tg = 0; tg < NTG; ++tg) {
         const int tok = 4 * tg + tq;

@@ -13,8 +13,9 @@ constexpr int kDecodeMaxSplits = 64;  // stage-1 column splits per layer
 
 // ---------------------------------------------------------------- workspace
 // One per device.  Decode keeps t (batch x r fp32 per layer) and the max |t| of each
-// 64-row block; prefill keeps x' (batch x n fp16) and T (batch x r fp16); host-memory
-// x / y are staged through xstage / ystage.
+// 128-row block; prefill keeps x' (batch x n fp16) and T (batch x r fp16); both use
+// `partials` and `counters` for split reductions; host-memory x go through xstage (pinned
+// x by a gather kernel, pageable x by a copy) and pageable host y through ystage.
 struct Workspace {
     int device = -1;
     size_t bytes = 0;
@@ -22,8 +23,8 @@ struct Workspace {
     // carved regions
     float* t = nullptr;            // [t_cap] (decode: sum over a launch's layers of batch x r)
     float* tgmax = nullptr;        // [tgmax_cap] (decode: batch x r/64 per layer)
-    float* partials = nullptr;     // [partial_cap] (decode: stage-1 column-split partial sums)
-    int* counters = nullptr;       // [counter_cap] (decode: arrival counters, zero between calls)
+    float* partials = nullptr;     // [partial_cap] (stage-1 column splits; prefill K splits; norm sums)
+    int* counters = nullptr;       // [counter_cap] (arrival counters, zero between calls)
     unsigned* status = nullptr;    // [0]: pack value check, [1]: device wait timeout
     uint16_t* xprime = nullptr;    // [batch_cap][n_cap] fp16 (prefill)
     uint16_t* T = nullptr;         // [batch_cap][r_cap] fp16 (prefill)
