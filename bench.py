@@ -21,6 +21,7 @@ import argparse
 import ctypes
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -284,9 +285,13 @@ def run_ours(args):
 
         with open(tpath) as f:
             rec = json.load(f)
-        with open(os.path.join(ROOT, rec["kernel_source"]), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
-        if sha == rec["kernel_source_sha256_16"]:  # counters are only valid for the kernel they came from
+        with open(os.path.join(ROOT, rec["kernel_source"])) as f:
+            code = f.read()
+        # the source with comments and white space removed: counters are only valid for the
+        # kernel code they were taken from
+        code = re.sub(r"/\*.*?\*/", "", code, flags=re.S)
+        code = "".join(re.sub(r"//[^\n]*", "", code).split())
+        if hashlib.sha256(code.encode()).hexdigest()[:16] == rec["kernel_code_sha256_16"]:
             traffic = rec["dram_bytes_per_step_b1"]
     achieved = value / world
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
