@@ -541,10 +541,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ Ge
 }
 
 constexpr int kTileThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 expand + epilogue
-// Two CTAs per SM (98 KB each: 3 stages at BN = 128, 2 at BN = 256), so that one CTA's
-// epilogue runs while the other's MMAs do.  Measured against one CTA per SM with twice the
-// stages: 103 vs 129 us at 1024 tokens, 49 vs 57 us at 256, 268 vs 272 us at 4096.
-constexpr int kTileSmemBudget = 100 * 1024;
+// Two CTAs per SM (up to 104 KB each: 4 stages at BN = 64, 3 at 128 and 144, 2 at 176 and
+// 256), so that one CTA's epilogue runs while the other's MMAs do.  Measured against one
+// CTA per SM with twice the stages: 103 vs 129 us at 1024 tokens, 49 vs 57 us at 256.
+constexpr int kTileSmemBudget = 112 * 1024;
 
 template <int BN>
 struct Geometry {
@@ -553,7 +553,7 @@ struct Geometry {
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = (kTileSmemBudget - 2048) / kStageBytes > 8 ? 8 : (kTileSmemBudget - 2048) / kStageBytes;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*alignment slack*/;
-    static constexpr int kTmemCols = BN < 32 ? 32 : BN;
+    static constexpr int kTmemCols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;  // a power of 2
 };
 
 struct TileBarriers {
@@ -719,7 +719,7 @@ tile_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint32_t* __res
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int64_t b = n0 + c0 + j;
-                    if (b < batch) {
+                    if (c0 + j < BN && b < batch) {  // BN need not be a multiple of 32
                         const float d = __uint_as_float(v[j]);
                         if (EPI == 0)
                             T_out[b * mdim + tcol] = __half_as_ushort(__float2half_rn(d));
@@ -935,35 +935,71 @@ cudaError_t launch_prescale(const uint16_t* x, const uint16_t* s2, int64_t n, in
     return launch_pdl(prescale_kernel, dim3(pblocks), dim3(256), 0, stream, x, s2, n, batch, ws->xprime);
 }
 
-template <int BN>
-int run_gemms(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const uint16_t* s1, const uint16_t* s2,
-              int64_t m, int64_t n, int64_t r, int64_t batch, float* y, Workspace* ws, cudaStream_t stream) {
+template <int BN, int EPI>
+int launch_tile_gemm(const void* bsrc, int64_t K, const uint32_t* Wpk, int64_t M, int64_t batch, uint16_t* T_out,
+                     float* y_out, const uint16_t* s1, Workspace* ws, cudaStream_t stream) {
     using G = Geometry<BN>;
     static unsigned long long init_mask = 0;
     const unsigned long long bit = 1ull << (ws->device & 63);
     if (!(__atomic_load_n(&init_mask, __ATOMIC_ACQUIRE) & bit)) {
-        if (cudaFuncSetAttribute(tile_gemm_kernel<BN, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmemBytes) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(tile_gemm_kernel<BN, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::kSmemBytes) !=
-                cudaSuccess)
+        if (cudaFuncSetAttribute(tile_gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 G::kSmemBytes) != cudaSuccess)
             return NQ_ERR_CUDA;
         __atomic_fetch_or(&init_mask, bit, __ATOMIC_RELEASE);
     }
-    CUtensorMap map_x, map_t;
-    if (!make_map(&map_x, ws->xprime, batch, n, kBK, BN, false, true) ||
-        !make_map(&map_t, ws->T, batch, r, kBK, BN, false, true))
-        return NQ_ERR_CUDA;
-
-    if (launch_prescale(x, s2, n, batch, ws, stream) != cudaSuccess) return NQ_ERR_CUDA;
+    CUtensorMap map;
+    if (!make_map(&map, bsrc, batch, K, kBK, BN, false, true)) return NQ_ERR_CUDA;
     const unsigned ntiles = (unsigned)((batch + BN - 1) / BN);
-    if (launch_pdl(tile_gemm_kernel<BN, 0>, dim3((unsigned)(r / kBM), ntiles), dim3(kTileThreads), (size_t)G::kSmemBytes,
-                   stream, map_x, Vpk, n, r, batch, ws->T, (float*)nullptr, (const uint16_t*)nullptr,
-                   ws->status + 1) != cudaSuccess)
-        return NQ_ERR_CUDA;
-    if (launch_pdl(tile_gemm_kernel<BN, 1>, dim3((unsigned)(m / kBM), ntiles), dim3(kTileThreads), (size_t)G::kSmemBytes,
-                   stream, map_t, Upk, r, m, batch, (uint16_t*)nullptr, y, s1, ws->status + 1) != cudaSuccess)
-        return NQ_ERR_CUDA;
-    return NQ_OK;
+    return launch_pdl(tile_gemm_kernel<BN, EPI>, dim3((unsigned)(M / kBM), ntiles), dim3(kTileThreads),
+                      (size_t)G::kSmemBytes, stream, map, Wpk, K, M, batch, T_out, y_out, s1,
+                      ws->status + 1) == cudaSuccess
+               ? NQ_OK
+               : NQ_ERR_CUDA;
+}
+
+// Token-tile width of one GEMM (M rows of A, `batch` tokens): the candidate with the least
+// estimated time, (tiles per SM, rounded up) x (BN + 200), the 200 standing for the
+// per-k-block cost that does not shrink with the tile (sign expansion, ring hand-offs).
+// Fitted to a sweep of all width pairs on the 11008 x 4096, r = 2432 layer on a B200
+// (within 3 % of the best pair from 128 to 4096 tokens); e.g. 517 tokens: GEMM 2 at 176
+// wide, 59 us against 71 us at 128; 2048 tokens: GEMM 1 at 144, 144 us against 151 us.
+int choose_bn(int64_t M, int64_t batch, int sms) {
+    if (batch <= 256) return 128;  // measured best for both GEMMs up to 256 tokens
+    static const int cand[] = {64, 128, 144, 176, 256};
+    int best = 256;
+    double best_t = 1e300;
+    for (int bn : cand) {
+        const int64_t tiles = (M / kBM) * ((batch + bn - 1) / bn);
+        const double t = (double)((tiles + sms - 1) / sms) * (bn + 200);
+        if (t < best_t - 1e-9) {
+            best_t = t;
+            best = bn;
+        }
+    }
+    return best;
+}
+
+template <int EPI>
+int launch_tile_gemm_bn(int bn, const void* bsrc, int64_t K, const uint32_t* Wpk, int64_t M, int64_t batch,
+                        uint16_t* T_out, float* y_out, const uint16_t* s1, Workspace* ws, cudaStream_t stream) {
+    switch (bn) {
+        case 64: return launch_tile_gemm<64, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream);
+        case 128: return launch_tile_gemm<128, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream);
+        case 144: return launch_tile_gemm<144, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream);
+        case 176: return launch_tile_gemm<176, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream);
+        default: return launch_tile_gemm<256, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream);
+    }
+}
+
+int run_tile_gemms(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const uint16_t* s1,
+                   const uint16_t* s2, int64_t m, int64_t n, int64_t r, int64_t batch, float* y, Workspace* ws,
+                   cudaStream_t stream) {
+    if (launch_prescale(x, s2, n, batch, ws, stream) != cudaSuccess) return NQ_ERR_CUDA;
+    const int sms = sm_count();
+    int st = launch_tile_gemm_bn<0>(choose_bn(r, batch, sms), ws->xprime, n, Vpk, r, batch, ws->T, nullptr, nullptr,
+                                    ws, stream);
+    if (st != NQ_OK) return st;
+    return launch_tile_gemm_bn<1>(choose_bn(m, batch, sms), ws->T, r, Upk, m, batch, nullptr, y, s1, ws, stream);
 }
 
 }  // namespace
@@ -997,9 +1033,7 @@ void prefill_workspace_need(int64_t m, int64_t n, int64_t r, int64_t batch, int6
 int prefill_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const uint16_t* s1,
                     const uint16_t* s2, int64_t m, int64_t n, int64_t r, int64_t batch, float* y,
                     Workspace* ws, cudaStream_t stream) {
-    if (batch > kPersistentMaxBatch)
-        return batch <= 1024 ? run_gemms<128>(x, Upk, Vpk, s1, s2, m, n, r, batch, y, ws, stream)
-                             : run_gemms<256>(x, Upk, Vpk, s1, s2, m, n, r, batch, y, ws, stream);
+    if (batch > kPersistentMaxBatch) return run_tile_gemms(x, Upk, Vpk, s1, s2, m, n, r, batch, y, ws, stream);
     static unsigned long long init_mask = 0;
     const unsigned long long bit = 1ull << (ws->device & 63);
     if (!(__atomic_load_n(&init_mask, __ATOMIC_ACQUIRE) & bit)) {

@@ -225,6 +225,8 @@ def test_forward_prefill_sweep_sampled(nq, orc, batch):
     (512, 2048, 384, 40),     # split K with a partial last 16-token group
     (2432, 512, 1280, 64),    # split K in GEMM 1, 19 row blocks in GEMM 2
     (128, 8192, 128, 17),     # one row block each: the most splits
+    (128, 512, 128, 300),     # 64-wide token tiles in both GEMMs
+    (1024, 256, 896, 3000),   # 144-wide tiles in GEMM 1, 176-wide in GEMM 2 (not multiples of 32)
 ])
 def test_prefill_tiles(nq, orc, m, n, r, batch):
     c = Case(orc, nq, m, n, r, batch, seed=m * 7 + batch)
