@@ -40,6 +40,7 @@
 #include <cuda_fp16.h>
 #include <math.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "nq_internal.cuh"
@@ -47,15 +48,20 @@
 namespace nq {
 namespace {
 
-constexpr int kThreads = 256;          // 8 warps
+constexpr int kThreads = 256;          // stage 2: 8 warps
 constexpr int kWarps = kThreads / 32;
 constexpr int kCB = 128;               // columns per column block
 constexpr int kChunk = 1024;           // columns per fragment chunk
 constexpr int kChunkCB = kChunk / kCB;
 constexpr int kChunkWords = kChunk / 32;
 constexpr int kQBits = 14;             // |q| < 2^14
-constexpr int kRowsS1 = 128;           // stage-1 rows per CTA (8 warps x 16)
+constexpr int kRowsS1 = 128;           // stage-1 rows per CTA (8 warps x 1 tile or 4 warps x 2 tiles of 16)
 constexpr int kS1Stride = kChunkWords + 4;  // words per staged stage-1 row (36: bank-spread)
+constexpr int kSumBatch = 16;          // stage-1 split partials loaded at once by the reducing CTA
+constexpr int kMaxK2 = 8;              // stage-2 CTAs per SM tried for a launch that fits in one wave
+constexpr size_t kSmemPerSM = 228 * 1024;  // shared memory of one SM
+constexpr size_t kSmemReserve = 1024;      // taken by the system from it for every resident CTA
+constexpr int kWaveTiles2 = 8;         // stage-2 tiles per CTA of a launch that needs several waves
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 __device__ __forceinline__ float f16_to_f32(uint16_t h) { return __half2float(__ushort_as_half(h)); }
@@ -120,7 +126,7 @@ struct DecLayer {
     int m, n, r;
     int nsplit;      // stage 1: CTAs per 128-row block (column splits)
     int cps;         // stage 1: column blocks per split
-    int rt;          // stage 2: row tiles per CTA (8/rt k-parts per tile)
+    int s2_ctas;     // stage 2: CTAs of the layer, each an even share of its 16-row tiles
 };
 
 struct DecGroup {
@@ -129,15 +135,22 @@ struct DecGroup {
     int batch;
     int depth1;       // stage-1 chunk ring depth (1 or 2)
     int r2;           // stage-2 columns held on chip at a time (a multiple of kCB)
-    int w2stride;     // stage-2 words per staged row
+    int w2words;      // stage-2 weight buffer: the most rows x words per row of one CTA
+    int rows2;        // stage-2 rows held on chip: 16 x the most tiles of one CTA
+    int per_sm2;      // stage-2 CTAs per SM of a one-wave plan (no more may share an SM), else 0
+    // CTA ranges in launch order: range k holds CTAs s1_start[k] .. s1_start[k+1]-1 of layer
+    // s1_layer[k] (likewise for stage 2); the host puts the slowest layers first
     int s1_start[kMaxGroup + 1];
     int s2_start[kMaxGroup + 1];
+    unsigned char s1_layer[kMaxGroup];
+    unsigned char s2_layer[kMaxGroup];
 };
 
-__device__ __forceinline__ int find_layer(const int* start, int count, int block) {
-    int l = 0;
-    while (l + 1 < count && block >= start[l + 1]) ++l;
-    return l;
+// The range of `block` (an index into start[]).
+__device__ __forceinline__ int find_range(const int* start, int count, int block) {
+    int k = 0;
+    while (k + 1 < count && block >= start[k + 1]) ++k;
+    return k;
 }
 
 // ------------------------------------------------------------------ shared memory
@@ -147,61 +160,67 @@ struct Misc {
     int e[8];
     float up[8];             // 2^(14 - e): quantisation factor per token
     int qsum[8];
-    union {
-        int bq[kRowsS1][8];      // stage 2: per (row, token) across k-parts
-        float res[8][kRowsS1];   // stage 1: the CTA's partial sums of its rows
-    };
     int last;
 };
 
+// B fragments: per (column block, token group, half) one uint4 for each of the 32 lanes.
+// (Storing only the lanes that hold tokens, and loading under a lane predicate, measured
+// slower: the unconditional 16-byte loads keep the MMA loop free of branches.)
 __host__ __device__ inline size_t frag_bytes(int ncb, int ntg) { return (size_t)ncb * ntg * 2 * 32 * 16; }
 
-// stage 1: w [depth][128][36] | x [depth][batch + 1][1024] bf16 (slot batch = s2) | v [batch][1024] f32 | frag (8 CBs) | misc
+// stage 1: w [depth][128][36] | x [depth][batch + 1][1024] bf16 (slot batch = s2; after the
+// last chunk its start holds res [batch][128] f32, the CTA's sums of its rows) | frag (8 CBs) | misc
 __host__ __device__ inline size_t s1_w_bytes(int depth) { return (size_t)depth * kRowsS1 * kS1Stride * 4; }
 __host__ __device__ inline size_t s1_x_bytes(int depth, int batch) { return (size_t)depth * (batch + 1) * kChunk * 2; }
-__host__ __device__ inline size_t s1_v_bytes(int batch) { return (size_t)batch * kChunk * 4; }
 __host__ __device__ inline size_t s1_bytes(int depth, int batch, int ntg) {
-    return s1_w_bytes(depth) + s1_x_bytes(depth, batch) + s1_v_bytes(batch) + frag_bytes(kChunkCB, ntg) + sizeof(Misc);
+    return s1_w_bytes(depth) + s1_x_bytes(depth, batch) + frag_bytes(kChunkCB, ntg) + sizeof(Misc);
 }
-// stage 2: w [128][w2stride] | t [batch][r2] f32 | frag (all r2/128 CBs) | misc
-__host__ __device__ inline size_t s2_w_bytes(int w2stride) { return (size_t)kRowsS1 * w2stride * 4; }
+// stage 2: w [rows][stride(r)] | t [batch][r2] f32 | frag (all r2/128 CBs) | bq [rows2][batch] | misc
+// Words per staged row of a layer of rank r: the first span's words, plus 4 when that is an
+// even number of 4-word groups (an odd number spreads the 8 rows a warp reads over all
+// 32 banks).
+__host__ __device__ inline int s2_stride(int r, int r2) {
+    const int cols = r < r2 ? r : r2;
+    return cols / 32 + (((cols / 128) % 2) ? 0 : 4);
+}
 __host__ __device__ inline size_t s2_t_bytes(int batch, int r2) { return (size_t)batch * r2 * 4; }
-__host__ __device__ inline size_t s2_bytes(int w2stride, int batch, int r2, int ntg) {
-    return s2_w_bytes(w2stride) + s2_t_bytes(batch, r2) + frag_bytes(r2 / kCB, ntg) + sizeof(Misc);
+__host__ __device__ inline size_t s2_bq_bytes(int rows2, int batch) { return ((size_t)rows2 * batch * 4 + 15) / 16 * 16; }
+__host__ __device__ inline size_t s2_bytes(int w2words, int rows2, int batch, int r2, int ntg) {
+    return (size_t)w2words * 4 + s2_t_bytes(batch, r2) + frag_bytes(r2 / kCB, ntg) +
+           s2_bq_bytes(rows2, batch) + sizeof(Misc);
 }
 
 template <int NTG>
-__device__ __forceinline__ uint4& frag_at(uint4* frag, int cb, int tg, int half, int lane) {
-    return frag[((cb * NTG + tg) * 2 + half) * 32 + lane];
+__device__ __forceinline__ uint4* frag_ptr(uint4* frag, int cb, int tg, int half, int lane) {
+    return frag + ((cb * NTG + tg) * 2 + half) * 32 + lane;
 }
 
-template <int NTG>
+// Zero every slot: those of lanes without a token (tokens >= batch) are never written.
+template <int NTG, int NT>
 __device__ __forceinline__ void zero_fragments(uint4* frag, int ncb) {
-    for (int i = threadIdx.x; i < ncb * NTG * 2 * 32; i += kThreads) frag[i] = make_uint4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < ncb * NTG * 2 * 32; i += NT) frag[i] = make_uint4(0, 0, 0, 0);
 }
 
-// B fragments of `ncb` column blocks from fp32 values vals[tok * vstride + col] (col from
-// the chunk's first column), quantised with up[tok]; adds each token's sum of q to qsum.
-// One task = (cb, token, word t of the CB, fragment word j = 2s + h): the 4 columns
-// 32t + s + 4h + 8c (c in 0..3) give word j of two lanes, the hi-limb lane 8*tok' + t and
-// the lo-limb lane 8*tok' + 4 + t (tok' = token within its group).  The 32 tasks of a
-// warp step share one token, so the warp adds its q's with a shuffle reduction.  Slots of
-// tokens >= batch are never written and stay zero (zero_fragments at kernel start).
-template <int NTG>
-__device__ __forceinline__ void build_fragments(uint4* frag, Misc& mi, const float* vals, int vstride, int ncb,
-                                                int batch) {
+// B fragments of `ncb` column blocks from the fp32 values val(tok, col) (col from the span's
+// first column), quantised with up[tok]; adds each token's sum of q to qsum.  One task =
+// (cb, token, word t of the CB, fragment word j = 2s + h): the 4 columns 32t + s + 4h + 8c
+// (c in 0..3) give word j of two lanes, the hi-limb lane 8*tok' + t and the lo-limb lane
+// 8*tok' + 4 + t (tok' = token within its group).  The 32 tasks of a warp step share one
+// token, so the warp adds its q's with a shuffle reduction.
+template <int NTG, int NT, typename Val>
+__device__ __forceinline__ void build_fragments(uint4* frag, Misc& mi, Val val, int ncb, int batch) {
     const int tasks = ncb * batch * 32;  // a multiple of 32: whole warps take part in every step
-    for (int task = threadIdx.x; task < tasks; task += kThreads) {
+    for (int task = threadIdx.x; task < tasks; task += NT) {
         const int j = task & 7, t = (task >> 3) & 3;
         const int tok = (task >> 5) % batch, cb = (task >> 5) / batch;
         const int s4 = j >> 1, h = j & 1;
         const float up = mi.up[tok];
-        const float* v = vals + tok * vstride + cb * kCB + 32 * t + s4 + 4 * h;
+        const int col = cb * kCB + 32 * t + s4 + 4 * h;
         uint32_t wh = 0, wl = 0;
         int qs = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            const int q = quantise(v[8 * c], up);
+            const int q = quantise(val(tok, col + 8 * c), up);
             qs += q;
             wh |= (uint32_t)((q >> 7) & 0xFF) << (8 * c);
             wl |= (uint32_t)(q & 0x7F) << (8 * c);
@@ -210,18 +229,20 @@ __device__ __forceinline__ void build_fragments(uint4* frag, Misc& mi, const flo
         if ((threadIdx.x & 31) == 0) atomicAdd(&mi.qsum[tok], qs);
         const int tg = tok >> 2, ti = tok & 3;
         // word j lives in half j >> 2 at component j & 3
-        reinterpret_cast<uint32_t*>(&frag_at<NTG>(frag, cb, tg, j >> 2, 8 * ti + t))[j & 3] = wh;
-        reinterpret_cast<uint32_t*>(&frag_at<NTG>(frag, cb, tg, j >> 2, 8 * ti + 4 + t))[j & 3] = wl;
+        reinterpret_cast<uint32_t*>(frag_ptr<NTG>(frag, cb, tg, j >> 2, 8 * ti + t))[j & 3] = wh;
+        reinterpret_cast<uint32_t*>(frag_ptr<NTG>(frag, cb, tg, j >> 2, 8 * ti + 4 + t))[j & 3] = wl;
     }
 }
 
 // One column block of a 16-row tile into accumulator set `acc`.
 template <int NTG>
-__device__ __forceinline__ void cb_mma(uint4* frag, uint32_t wa, uint32_t wb, int cb, int lane, int (&acc)[NTG][4][4]) {
+__device__ __forceinline__ void cb_mma(const uint4* frag, uint32_t wa, uint32_t wb, int cb, int lane,
+                                       int (&acc)[NTG][4][4]) {
     const uint32_t a4 = wa >> 4, b4 = wb >> 4;
 #pragma unroll
     for (int tg = 0; tg < NTG; ++tg) {
-        const uint4 f0 = frag_at<NTG>(frag, cb, tg, 0, lane), f1 = frag_at<NTG>(frag, cb, tg, 1, lane);
+        const uint4 f0 = *frag_ptr<NTG>(const_cast<uint4*>(frag), cb, tg, 0, lane);
+        const uint4 f1 = *frag_ptr<NTG>(const_cast<uint4*>(frag), cb, tg, 1, lane);
         const uint32_t bf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
@@ -231,12 +252,12 @@ __device__ __forceinline__ void cb_mma(uint4* frag, uint32_t wa, uint32_t wb, in
     }
 }
 
-// Accumulate one 16-row tile against column blocks cb0, cb0 + step, ... < cb1 of the
-// chunk's fragments.  wrow points at the tile's row 0, word 0 of the chunk; rows are
-// `stride` words apart.  Two accumulator sets alternate between consecutive column blocks
-// so that dependent MMAs are two blocks apart.
+// Accumulate one 16-row tile against column blocks cb0 .. cb1-1 of the span's fragments.
+// wrow points at the tile's row 0, word 0 of the span; rows are `stride` words apart.  Two
+// accumulator sets alternate between consecutive column blocks so that dependent MMAs are
+// two blocks apart.
 template <int NTG>
-__device__ __forceinline__ void tile_mma(uint4* frag, const uint32_t* wrow, int stride, int cb0, int cb1, int step,
+__device__ __forceinline__ void tile_mma(const uint4* frag, const uint32_t* wrow, int stride, int cb0, int cb1,
                                          int (&acc)[NTG][4][4]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const uint32_t* wa_row = wrow + g * stride + t;
@@ -249,11 +270,11 @@ __device__ __forceinline__ void tile_mma(uint4* frag, const uint32_t* wrow, int 
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc2[tg][s][i] = 0;
     int cb = cb0;
-    for (; cb + step < cb1; cb += 2 * step) {
+    for (; cb + 1 < cb1; cb += 2) {
         const uint32_t wa0 = wa_row[4 * cb], wb0 = wb_row[4 * cb];
-        const uint32_t wa1 = wa_row[4 * (cb + step)], wb1 = wb_row[4 * (cb + step)];
+        const uint32_t wa1 = wa_row[4 * (cb + 1)], wb1 = wb_row[4 * (cb + 1)];
         cb_mma<NTG>(frag, wa0, wb0, cb, lane, acc);
-        cb_mma<NTG>(frag, wa1, wb1, cb + step, lane, acc2);
+        cb_mma<NTG>(frag, wa1, wb1, cb + 1, lane, acc2);
     }
     if (cb < cb1) cb_mma<NTG>(frag, wa_row[4 * cb], wb_row[4 * cb], cb, lane, acc);
 #pragma unroll
@@ -262,6 +283,35 @@ __device__ __forceinline__ void tile_mma(uint4* frag, const uint32_t* wrow, int 
         for (int s = 0; s < 4; ++s)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[tg][s][i] += acc2[tg][s][i];
+}
+
+// Two 16-row tiles (rows wrow0.., wrow1..) against column blocks cb0 .. cb1-1 at once: each
+// column block's B fragments are loaded once for both tiles, and the tiles' accumulators
+// give eight independent MMA chains per column block.
+template <int NTG>
+__device__ __forceinline__ void tile_pair_mma(const uint4* frag, const uint32_t* wrow0, const uint32_t* wrow1,
+                                              int stride, int cb0, int cb1, int (&acc0)[NTG][4][4],
+                                              int (&acc1)[NTG][4][4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const uint32_t* a0 = wrow0 + g * stride + t;
+    const uint32_t* a1 = wrow1 + g * stride + t;
+    for (int cb = cb0; cb < cb1; ++cb) {
+        const uint32_t wa0 = a0[4 * cb], wb0 = a0[8 * stride + 4 * cb];
+        const uint32_t wa1 = a1[4 * cb], wb1 = a1[8 * stride + 4 * cb];
+        const uint32_t x0 = wa0 >> 4, y0 = wb0 >> 4, x1 = wa1 >> 4, y1 = wb1 >> 4;
+#pragma unroll
+        for (int tg = 0; tg < NTG; ++tg) {
+            const uint4 f0 = *frag_ptr<NTG>(const_cast<uint4*>(frag), cb, tg, 0, lane);
+            const uint4 f1 = *frag_ptr<NTG>(const_cast<uint4*>(frag), cb, tg, 1, lane);
+            const uint32_t bf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const uint32_t M = 0x01010101u << s;
+                mma_u8s8(acc0[tg][s], wa0 & M, wb0 & M, x0 & M, y0 & M, bf[2 * s], bf[2 * s + 1]);
+                mma_u8s8(acc1[tg][s], wa1 & M, wb1 & M, x1 & M, y1 & M, bf[2 * s], bf[2 * s + 1]);
+            }
+        }
+    }
 }
 
 // sum_j b_j q_j for (row g, token 4tg+t) and (row g+8, same token).
@@ -291,24 +341,33 @@ __device__ __forceinline__ void zero_acc(int (&acc)[NTG][4][4]) {
 
 // ------------------------------------------------------------------ stage 1
 // CTA = 128 rows of V^T of one layer x one column split (cps column blocks, staged kChunk
-// columns at a time); warp w owns rows 16w..16w+15.  Each chunk has its own quantisation
-// exponent per token, so the warp converts its integer sums to fp32 after every chunk.
-// With several splits, the CTAs of a row block leave fp32 partials and the last to arrive
-// adds them in split order (deterministic), then writes t and the block's max |t| per
-// token (stage 2 builds its exponent from those maxima).
-template <int NTG>
-__global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant__ DecGroup grp) {
+// columns at a time).  TPW = 1: eight warps, warp w owns the 16-row tile 16w..16w+15 (the
+// launch fits in one wave at four CTAs per SM).  TPW = 2: four warps of fewer registers,
+// warp w owns rows 32w..32w+31 as two tiles multiplied together, sharing each column
+// block's B fragments (more CTAs per SM for launches of several waves, and for two token
+// groups, where one tile per warp would need twice the registers).  Each chunk has its own
+// quantisation exponent per token, so the warp converts its integer sums to fp32 after
+// every chunk.  With several splits, the CTAs of a row block leave fp32 partials and the
+// last to arrive adds them in split order (deterministic), then writes t and the block's
+// max |t| per token (stage 2 builds its exponent from those maxima).
+template <int TPW>
+__host__ __device__ constexpr int s1_threads() { return 32 * kRowsS1 / (16 * TPW); }
+
+template <int NTG, int TPW>
+__global__ void __launch_bounds__(s1_threads<TPW>(), TPW == 1 ? 4 : (NTG == 1 ? 8 : 4))
+stage1_kernel(const __grid_constant__ DecGroup grp) {
+    constexpr int kThreads1 = s1_threads<TPW>(), kWarps1 = kThreads1 / 32;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int batch = grp.batch, depth = grp.depth1;
     uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem_raw);
     uint16_t* xbuf = reinterpret_cast<uint16_t*>(smem_raw + s1_w_bytes(depth));  // [depth][batch + 1][kChunk]
-    float* vbuf = reinterpret_cast<float*>(smem_raw + s1_w_bytes(depth) + s1_x_bytes(depth, batch));
-    uint4* frag = reinterpret_cast<uint4*>(smem_raw + s1_w_bytes(depth) + s1_x_bytes(depth, batch) + s1_v_bytes(batch));
+    uint4* frag = reinterpret_cast<uint4*>(smem_raw + s1_w_bytes(depth) + s1_x_bytes(depth, batch));
     Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(frag) + frag_bytes(kChunkCB, NTG));
+    float(*res)[kRowsS1] = reinterpret_cast<float(*)[kRowsS1]>(xbuf);  // after the last chunk
 
-    const int li = find_layer(grp.s1_start, grp.count, blockIdx.x);
-    const DecLayer& L = grp.L[li];
-    const int local = blockIdx.x - grp.s1_start[li];
+    const int rk = find_range(grp.s1_start, grp.count, blockIdx.x);
+    const DecLayer& L = grp.L[grp.s1_layer[rk]];
+    const int local = blockIdx.x - grp.s1_start[rk];
     const int rb = local / L.nsplit, sp = local % L.nsplit;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
     const int n = L.n, r = L.r;
@@ -321,22 +380,21 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
     auto wchunk = [&](int buf) { return wbuf + (size_t)buf * kRowsS1 * kS1Stride; };
     auto xchunk = [&](int buf, int tok) { return xbuf + ((size_t)buf * (batch + 1) + tok) * kChunk; };
 
-    auto fetch_w = [&](int ch) {  // weight rows of chunk ch into buffer ch % depth
-        const int per_row = chunk_cb(ch);  // 16-byte pieces (one per column block)
+    auto fetch_w = [&](int ch) {  // weight rows of chunk ch into buffer ch % depth: lane p of a warp takes piece p of a row
+        const int per_row = chunk_cb(ch);  // 16-byte pieces (one per column block), at most 8
         uint32_t* dst = wchunk(ch % depth);
         const uint32_t* src = W + (int64_t)(cbA + ch * kChunkCB) * 4;
-        for (int i = threadIdx.x; i < kRowsS1 * per_row; i += kThreads) {
-            const int row = i / per_row, p = i % per_row;
-            cp_async16(dst + row * kS1Stride + 4 * p, src + row * wpr + 4 * p);
-        }
+        const int p = threadIdx.x & 7;
+        if (p < per_row)
+            for (int row = threadIdx.x >> 3; row < kRowsS1; row += kThreads1 / 8)
+                cp_async16(dst + row * kS1Stride + 4 * p, src + row * wpr + 4 * p);
     };
     auto fetch_x = [&](int ch) {  // x rows (batch of them) and s2 of chunk ch; s2 goes in slot `batch`
         const int per_tok = chunk_cb(ch) * kCB / 8;
         const int col0 = (cbA + ch * kChunkCB) * kCB;
-        for (int i = threadIdx.x; i < (batch + 1) * per_tok; i += kThreads) {
-            const int tok = i / per_tok, p = i % per_tok;
-            const uint16_t* src = tok < batch ? L.x + (int64_t)tok * n + col0 + 8 * p : L.s2 + col0 + 8 * p;
-            cp_async16(xchunk(ch % depth, tok) + 8 * p, src);
+        for (int tok = 0; tok <= batch; ++tok) {
+            const uint16_t* src = tok < batch ? L.x + (int64_t)tok * n + col0 : L.s2 + col0;
+            for (int p = threadIdx.x; p < per_tok; p += kThreads1) cp_async16(xchunk(ch % depth, tok) + 8 * p, src + 8 * p);
         }
     };
 
@@ -347,7 +405,7 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
     cp_async_commit();
     if (nchunks > 2 && threadIdx.x < kRowsS1)
         prefetch_l2(W + threadIdx.x * wpr + (cbA + 2 * kChunkCB) * 4, (uint32_t)((cbB - cbA - 2 * kChunkCB) * 16));
-    zero_fragments<NTG>(frag, kChunkCB);
+    zero_fragments<NTG, kThreads1>(frag, kChunkCB);
     pdl_trigger();
     pdl_wait();  // x may come from the previous kernel on the stream
     if (nchunks > 0) fetch_x(0);
@@ -355,9 +413,11 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
     if (nchunks > 1) fetch_x(1);
     cp_async_commit();
 
-    float part[NTG][2];
+    float part[TPW][NTG][2];  // [tile][token group][row g / g+8]
 #pragma unroll
-    for (int tg = 0; tg < NTG; ++tg) part[tg][0] = part[tg][1] = 0.f;
+    for (int tl = 0; tl < TPW; ++tl)
+#pragma unroll
+        for (int tg = 0; tg < NTG; ++tg) part[tl][tg][0] = part[tl][tg][1] = 0.f;
 
     for (int ch = 0; ch < nchunks; ++ch) {
         const int buf = ch % depth;
@@ -365,18 +425,14 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
         const int ccols = ncb * kCB;
         if (ch + 1 < nchunks) cp_async_wait<1>(); else cp_async_wait<0>();
         __syncthreads();
-        // v = s2 * x (exact in fp32) and its per-token max: every thread takes a column
-        // stripe of every token, then the warps' maxima are combined
+        // v = s2 * x (exact in fp32, formed again when the fragments are built) and its
+        // per-token max: every thread takes a column stripe of every token, then the warps'
+        // maxima are combined
         const uint16_t* ss = xchunk(buf, batch);
+        auto val = [&](int tok, int c) { return bf16_to_f32(xchunk(buf, tok)[c]) * f16_to_f32(ss[c]); };
         for (int tok = 0; tok < batch; ++tok) {
-            const uint16_t* xs = xchunk(buf, tok);
-            float* vs = vbuf + tok * kChunk;
             float mx = 0.f;
-            for (int c = threadIdx.x; c < ccols; c += kThreads) {
-                const float v = bf16_to_f32(xs[c]) * f16_to_f32(ss[c]);
-                vs[c] = v;
-                mx = fmaxf(mx, fabsf(v));
-            }
+            for (int c = threadIdx.x; c < ccols; c += kThreads1) mx = fmaxf(mx, fabsf(val(tok, c)));
             mx = warp_max(mx);
             if (lane == 0) mi.red[warp][tok] = mx;
         }
@@ -384,29 +440,38 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
         if (threadIdx.x < batch) {
             const int tok = threadIdx.x;
             float mx = mi.red[0][tok];
-            for (int w = 1; w < kWarps; ++w) mx = fmaxf(mx, mi.red[w][tok]);
+            for (int w = 1; w < kWarps1; ++w) mx = fmaxf(mx, mi.red[w][tok]);
             const int e = range_exponent(mx);
             mi.e[tok] = e;
             mi.up[tok] = pow2f(kQBits - e);
             mi.qsum[tok] = 0;
         }
         __syncthreads();
-        build_fragments<NTG>(frag, mi, vbuf, kChunk, ncb, batch);
+        build_fragments<NTG, kThreads1>(frag, mi, val, ncb, batch);
         __syncthreads();
 
-        int acc[NTG][4][4];
-        zero_acc<NTG>(acc);
-        tile_mma<NTG>(frag, wchunk(buf) + 16 * warp * kS1Stride, kS1Stride, 0, ncb, 1, acc);
+        int acc[TPW][NTG][4][4];
+        const uint32_t* wt = wchunk(buf) + 16 * TPW * warp * kS1Stride;  // the warp's first tile
+        zero_acc<NTG>(acc[0]);
+        if constexpr (TPW == 1) {
+            tile_mma<NTG>(frag, wt, kS1Stride, 0, ncb, acc[0]);
+        } else {
+            zero_acc<NTG>(acc[1]);
+            tile_pair_mma<NTG>(frag, wt, wt + 16 * kS1Stride, kS1Stride, 0, ncb, acc[0], acc[1]);
+        }
 #pragma unroll
-        for (int tg = 0; tg < NTG; ++tg) {
-            const int tok = 4 * tg + tq;
-            if (tok < batch) {
-                int bq0, bq8;
-                combine<NTG>(acc, tg, bq0, bq8);
-                const int64_t qs = mi.qsum[tok];
-                const float down = pow2f(mi.e[tok] - kQBits);
-                part[tg][0] += (float)(2 * (int64_t)bq0 - qs) * down;
-                part[tg][1] += (float)(2 * (int64_t)bq8 - qs) * down;
+        for (int tl = 0; tl < TPW; ++tl) {
+#pragma unroll
+            for (int tg = 0; tg < NTG; ++tg) {
+                const int tok = 4 * tg + tq;
+                if (tok < batch) {
+                    int bq0, bq8;
+                    combine<NTG>(acc[tl], tg, bq0, bq8);
+                    const int64_t qs = mi.qsum[tok];
+                    const float down = pow2f(mi.e[tok] - kQBits);
+                    part[tl][tg][0] += (float)(2 * (int64_t)bq0 - qs) * down;
+                    part[tl][tg][1] += (float)(2 * (int64_t)bq8 - qs) * down;
+                }
             }
         }
         __syncthreads();  // buffers are free again
@@ -417,21 +482,23 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
         }
     }
 
-    // this CTA's sums for its 128 rows, into shared memory
+    // this CTA's sums for its 128 rows, into shared memory (over the x buffer, no longer read)
 #pragma unroll
-    for (int tg = 0; tg < NTG; ++tg) {
-        const int tok = 4 * tg + tq;
-        if (tok < batch) {
-            mi.res[tok][16 * warp + g] = part[tg][0];
-            mi.res[tok][16 * warp + g + 8] = part[tg][1];
+    for (int tl = 0; tl < TPW; ++tl)
+#pragma unroll
+        for (int tg = 0; tg < NTG; ++tg) {
+            const int tok = 4 * tg + tq;
+            if (tok < batch) {
+                res[tok][16 * (TPW * warp + tl) + g] = part[tl][tg][0];
+                res[tok][16 * (TPW * warp + tl) + g + 8] = part[tl][tg][1];
+            }
         }
-    }
     __syncthreads();
     const int nrb = r / kRowsS1;
     if (L.nsplit > 1) {
-        for (int i = threadIdx.x; i < batch * kRowsS1; i += kThreads) {
+        for (int i = threadIdx.x; i < batch * kRowsS1; i += kThreads1) {
             const int tok = i / kRowsS1, k = i % kRowsS1;
-            L.partials[((int64_t)sp * batch + tok) * r + row0 + k] = mi.res[tok][k];
+            L.partials[((int64_t)sp * batch + tok) * r + row0 + k] = res[tok][k];
         }
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -441,29 +508,30 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
         }
         __syncthreads();
         if (!mi.last) return;
-        for (int i = threadIdx.x; i < batch * kRowsS1; i += kThreads) {
+        for (int i = threadIdx.x; i < batch * kRowsS1; i += kThreads1) {
             const int tok = i / kRowsS1, k = i % kRowsS1;
             const float* pp = L.partials + (int64_t)tok * r + row0 + k;
             const int64_t stride = (int64_t)batch * r;
             float sum = 0.f;
-            int q = 0;
-            for (; q + 4 <= L.nsplit; q += 4) {  // four independent loads in flight
-                const float a = __ldcg(pp + q * stride), b = __ldcg(pp + (q + 1) * stride);
-                const float c = __ldcg(pp + (q + 2) * stride), d = __ldcg(pp + (q + 3) * stride);
-                sum = (((sum + a) + b) + c) + d;
+            for (int q0 = 0; q0 < L.nsplit; q0 += kSumBatch) {  // up to kSumBatch loads in flight
+                float pv[kSumBatch];
+#pragma unroll
+                for (int q = 0; q < kSumBatch; ++q) pv[q] = q0 + q < L.nsplit ? __ldcg(pp + (q0 + q) * stride) : 0.f;
+#pragma unroll
+                for (int q = 0; q < kSumBatch; ++q)
+                    if (q0 + q < L.nsplit) sum += pv[q];
             }
-            for (; q < L.nsplit; ++q) sum += __ldcg(pp + q * stride);
-            mi.res[tok][k] = sum;
+            res[tok][k] = sum;
         }
         if (threadIdx.x == 0) L.counters[rb] = 0;
         __syncthreads();
     }
     // t and the block's max |t| per token (one warp per token)
-    for (int tok = warp; tok < batch; tok += kWarps) {
+    for (int tok = warp; tok < batch; tok += kWarps1) {
         float v = 0.f;
 #pragma unroll
         for (int q = 0; q < kRowsS1 / 32; ++q) {
-            const float a = mi.res[tok][lane + 32 * q];
+            const float a = res[tok][lane + 32 * q];
             L.t[(int64_t)tok * r + row0 + lane + 32 * q] = a;
             v = fmaxf(v, fabsf(a));
         }
@@ -473,10 +541,13 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
 }
 
 // ------------------------------------------------------------------ stage 2
-// CTA = RT row tiles x KS = 8/RT k-parts of one layer.  The CTA's weight rows for up to
-// r2 columns are copied on chip before the dependency wait, and t for those columns right
-// after it.  One quantisation exponent per token for the whole of t (from stage 1's
-// maxima), so integer sums run across all chunks and k-parts and are converted once.
+// The launch has about k CTAs per SM (k = 2 when they fit); each layer gets CTAs in
+// proportion to its work (16-row tiles x column blocks) and each CTA an even share of its
+// layer's tiles, so that every CTA, and every SM, has about the same work.  The CTA's weight
+// rows for up to r2 columns are copied on chip before the dependency wait, and t for those
+// columns right after it; the warps split the CTA's (tile, column block) units into even
+// runs.  One quantisation exponent per token for the whole of t (from stage 1's maxima), so
+// integer sums run across all column blocks and warps and are converted once.
 // Row-wise RMS normalisation of a layer's whole output, folded into stage 2: every CTA
 // adds up y^2 over its rows per token (fixed order) into the workspace, and the CTA that
 // arrives last adds those partial sums in CTA order (deterministic), then rounds
@@ -485,7 +556,7 @@ __global__ void __launch_bounds__(kThreads) stage1_kernel(const __grid_constant_
 template <typename YAt>
 __device__ void rms_norm_epilogue(const DecLayer& L, int batch, int rows, int blk, Misc& mi, YAt y_at) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nblk = L.m / rows;
+    const int nblk = L.s2_ctas;
     if (warp < batch) {  // one warp per token (batch <= 8 = warps)
         float ss = 0.f;
         for (int i = lane; i < rows; i += 32) {
@@ -528,24 +599,27 @@ __device__ void rms_norm_epilogue(const DecLayer& L, int batch, int rows, int bl
 }
 
 template <int NTG>
-__global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant__ DecGroup grp) {
+__global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(const __grid_constant__ DecGroup grp) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int batch = grp.batch, r2 = grp.r2, ws = grp.w2stride;
+    const int batch = grp.batch, r2 = grp.r2, rows2 = grp.rows2;
     uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem_raw);
-    float* tbuf = reinterpret_cast<float*>(smem_raw + s2_w_bytes(ws));
-    uint4* frag = reinterpret_cast<uint4*>(smem_raw + s2_w_bytes(ws) + s2_t_bytes(batch, r2));
-    Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(frag) + frag_bytes(r2 / kCB, NTG));
+    float* tbuf = reinterpret_cast<float*>(smem_raw + (size_t)grp.w2words * 4);
+    uint4* frag = reinterpret_cast<uint4*>(smem_raw + (size_t)grp.w2words * 4 + s2_t_bytes(batch, r2));
+    int* bq = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(frag) + frag_bytes(r2 / kCB, NTG));
+    Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(bq) + s2_bq_bytes(rows2, batch));
 
-    const int li = find_layer(grp.s2_start, grp.count, blockIdx.x);
-    const DecLayer& L = grp.L[li];
-    const int blk = blockIdx.x - grp.s2_start[li];
+    const int rk = find_range(grp.s2_start, grp.count, blockIdx.x);
+    const DecLayer& L = grp.L[grp.s2_layer[rk]];
+    const int blk = blockIdx.x - grp.s2_start[rk];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-    const int RT = L.rt, KS = kWarps / RT;
-    const int rt = warp / KS, kp = warp % KS;
     const int m = L.m, r = L.r;
+    const int ws = s2_stride(r, r2);
+    // this CTA's share of the layer's 16-row tiles
+    const int ntl = m / 16;
+    const int tile0 = (int)((int64_t)blk * ntl / L.s2_ctas), tile1 = (int)((int64_t)(blk + 1) * ntl / L.s2_ctas);
+    const int ntiles = tile1 - tile0, rows = 16 * ntiles;
     const int64_t wpr = r / 32;
-    const int rows = 16 * RT;
-    const int64_t row0 = (int64_t)blk * rows;
+    const int64_t row0 = (int64_t)tile0 * 16;
     const uint32_t* W = L.Upk + row0 * wpr;
     const int nsc = (r + r2 - 1) / r2;  // column spans held on chip one after the other
 
@@ -568,10 +642,11 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
 
     fetch_w(0);
     cp_async_commit();
-    if (nsc > 1 && threadIdx.x < rows)
-        prefetch_l2(W + threadIdx.x * wpr + r2 / 32, (uint32_t)((r - r2) / 8));
-    for (int i = threadIdx.x; i < kRowsS1 * 8; i += kThreads) (&mi.bq[0][0])[i] = 0;
-    zero_fragments<NTG>(frag, r2 / kCB);
+    if (nsc > 1)
+        for (int row = threadIdx.x; row < rows; row += kThreads)
+            prefetch_l2(W + row * wpr + r2 / 32, (uint32_t)((r - r2) / 8));
+    for (int i = threadIdx.x; i < rows * batch; i += kThreads) bq[i] = 0;  // [row][batch]
+    zero_fragments<NTG, kThreads>(frag, r2 / kCB);
     pdl_trigger();
     pdl_wait();  // t and its maxima come from stage 1
     fetch_t(0);
@@ -591,8 +666,6 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
         }
     }
 
-    int acc[NTG][4][4];
-    zero_acc<NTG>(acc);
     for (int sc = 0; sc < nsc; ++sc) {
         if (sc > 0) {
             __syncthreads();  // the previous span is consumed
@@ -604,24 +677,34 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
         __syncthreads();
         // every column block of the span at once: one barrier, then an uninterrupted MMA loop
         const int ncb = min(r2, r - sc * r2) / kCB;
-        build_fragments<NTG>(frag, mi, tbuf, r2, ncb, batch);
+        build_fragments<NTG, kThreads>(frag, mi, [&](int tok, int c) { return tbuf[tok * r2 + c]; }, ncb, batch);
         __syncthreads();
-        tile_mma<NTG>(frag, wbuf + 16 * rt * ws, ws, kp, ncb, KS, acc);
-    }
-
+        // the span's units (tile, column block) in tile-major order, an even run per warp;
+        // a run covers the ends of up to a few tiles, each added into bq when done
+        const int units = ntiles * ncb;
+        const int u1 = (warp + 1) * units / kWarps;
+        for (int u = warp * units / kWarps; u < u1;) {
+            const int ti = u / ncb, cb0 = u % ncb;
+            const int cb1 = min(ncb, cb0 + (u1 - u));
+            int acc[NTG][4][4];
+            zero_acc<NTG>(acc);
+            tile_mma<NTG>(frag, wbuf + 16 * ti * ws, ws, cb0, cb1, acc);
 #pragma unroll
-    for (int tg = 0; tg < NTG; ++tg) {
-        const int tok = 4 * tg + tq;
-        if (tok < batch) {
-            int bq0, bq8;
-            combine<NTG>(acc, tg, bq0, bq8);
-            atomicAdd(&mi.bq[16 * rt + g][tok], bq0);
-            atomicAdd(&mi.bq[16 * rt + g + 8][tok], bq8);
+            for (int tg = 0; tg < NTG; ++tg) {
+                const int tok = 4 * tg + tq;
+                if (tok < batch) {
+                    int bq0, bq8;
+                    combine<NTG>(acc, tg, bq0, bq8);
+                    atomicAdd(&bq[(16 * ti + g) * batch + tok], bq0);
+                    atomicAdd(&bq[(16 * ti + g + 8) * batch + tok], bq8);
+                }
+            }
+            u += cb1 - cb0;
         }
     }
     __syncthreads();
     auto y_at = [&](int tok, int i) {
-        const float v = (float)(2 * (int64_t)mi.bq[i][tok] - mi.qsum[tok]) * pow2f(mi.e[tok] - kQBits);
+        const float v = (float)(2 * (int64_t)bq[i * batch + tok] - mi.qsum[tok]) * pow2f(mi.e[tok] - kQBits);
         return f16_to_f32(L.s1[row0 + i]) * v;
     };
     for (int idx = threadIdx.x; idx < rows * batch; idx += kThreads) {
@@ -633,23 +716,44 @@ __global__ void __launch_bounds__(kThreads) stage2_kernel(const __grid_constant_
     if (L.y_norm) rms_norm_epilogue(L, batch, rows, blk, mi, y_at);
 }
 
+template <typename K>
+static bool set_kernel_attributes(K kernel) {
+    // the largest shared-memory carveout for every decode kernel, so that CTAs of the two
+    // stages (and of consecutive calls) can share an SM
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) == cudaSuccess &&
+           cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+}
+
 template <int NTG>
 int launch_group(DecGroup& grp, cudaStream_t stream, int device) {
     static unsigned long long init_mask = 0;  // devices whose kernel attributes are set
     const unsigned long long bit = 1ull << (device & 63);
     if (!(__atomic_load_n(&init_mask, __ATOMIC_ACQUIRE) & bit)) {
-        const int most = 200 * 1024;
-        if (cudaFuncSetAttribute(stage1_kernel<NTG>, cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess ||
-            cudaFuncSetAttribute(stage2_kernel<NTG>, cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess)
+        if (!set_kernel_attributes(stage1_kernel<NTG, 2>) || !set_kernel_attributes(stage2_kernel<NTG>))
             return NQ_ERR_CUDA;
+        if constexpr (NTG == 1)
+            if (!set_kernel_attributes(stage1_kernel<1, 1>)) return NQ_ERR_CUDA;
         __atomic_fetch_or(&init_mask, bit, __ATOMIC_RELEASE);
     }
     const size_t smem1 = s1_bytes(grp.depth1, grp.batch, NTG);
-    const size_t smem2 = s2_bytes(grp.w2stride, grp.batch, grp.r2, NTG);
-
-    if (launch_pdl(stage1_kernel<NTG>, dim3((unsigned)grp.s1_start[grp.count]), dim3(kThreads), smem1, stream, grp) !=
-        cudaSuccess)
-        return NQ_ERR_CUDA;
+    size_t smem2 = s2_bytes(grp.w2words, grp.rows2, grp.batch, grp.r2, NTG);
+    // a one-wave stage-2 plan gives every SM the same work only if no SM takes more than
+    // per_sm2 of its CTAs: ask for enough shared memory that one more does not fit
+    if (grp.per_sm2 > 0) smem2 = std::max(smem2, kSmemPerSM / (grp.per_sm2 + 1) - kSmemReserve + 16);
+    const unsigned grid1 = (unsigned)grp.s1_start[grp.count];
+    // one tile per warp (one token group only) when the launch fits in one wave of four
+    // 8-warp CTAs per SM
+    cudaError_t err;
+    if constexpr (NTG == 1) {
+        if (grid1 <= 4u * (unsigned)sm_count())
+            err = launch_pdl(stage1_kernel<1, 1>, dim3(grid1), dim3(s1_threads<1>()), smem1, stream, grp);
+        else
+            err = launch_pdl(stage1_kernel<1, 2>, dim3(grid1), dim3(s1_threads<2>()), smem1, stream, grp);
+    } else {
+        err = launch_pdl(stage1_kernel<NTG, 2>, dim3(grid1), dim3(s1_threads<2>()), smem1, stream, grp);
+    }
+    if (err != cudaSuccess) return NQ_ERR_CUDA;
     if (launch_pdl(stage2_kernel<NTG>, dim3((unsigned)grp.s2_start[grp.count]), dim3(kThreads), smem2, stream, grp) !=
         cudaSuccess)
         return NQ_ERR_CUDA;
@@ -657,14 +761,6 @@ int launch_group(DecGroup& grp, cudaStream_t stream, int device) {
 }
 
 }  // namespace
-
-// Stage-2 row tiles per CTA: the most rows per CTA that still leaves about two CTAs per SM.
-static int stage2_rt(int64_t total_tiles) {
-    const int64_t want = 2 * (int64_t)sm_count();
-    for (int rt = kWarps; rt > 1; rt /= 2)
-        if (total_tiles / rt >= want) return rt;
-    return 1;
-}
 
 // Stage-2 columns held on chip at a time: all of r when it fits (up to 4096 columns, less
 // for larger batches since t takes batch x r2 x 4 bytes), else spans of a multiple of kChunk.
@@ -675,6 +771,70 @@ static int stage2_span(int64_t r_max, int64_t batch) {
     if (span < kChunk) span = kChunk;
     const int64_t need = (r_max + kCB - 1) / kCB * kCB;
     return (int)(need < span ? need : span);
+}
+
+// Stage-2 CTAs per layer (ctas[i]), the largest weight buffer (words) and the most rows
+// of one CTA.  A launch that fits in one wave gets k CTAs per SM in all, the smallest
+// k = 2 .. kMaxK2 for which k of them fit on an SM (shared memory): layer i gets CTAs in
+// proportion to its work, tiles_i x column blocks_i (largest remainders, at least one and at
+// most one per tile), and each CTA an even share of the layer's tiles, so that all CTAs
+// carry about the same work.  A larger launch takes CTAs of kWaveTiles2 tiles (several waves).
+static void stage2_plan(const DecodeCall* calls, int count, int64_t batch, int* ctas, int* w2words, int* rows2,
+                        int* per_sm) {
+    int64_t work = 0, tiles_all = 0, r_max = 0;
+    for (int i = 0; i < count; ++i) {
+        work += (calls[i].m / 16) * (calls[i].r / kCB);
+        tiles_all += calls[i].m / 16;
+        r_max = calls[i].r > r_max ? calls[i].r : r_max;
+    }
+    const int r2 = stage2_span(r_max, batch);
+    const int ntg = batch <= 4 ? 1 : 2;
+    const int sms = sm_count();
+    auto measure = [&]() {  // buffer sizes of the current ctas[]
+        int64_t words = 0, rows = 0;
+        for (int i = 0; i < count; ++i) {
+            const int64_t tl = (calls[i].m / 16 + ctas[i] - 1) / ctas[i];
+            words = std::max(words, 16 * tl * s2_stride((int)calls[i].r, r2));
+            rows = std::max(rows, 16 * tl);
+        }
+        *w2words = (int)words;
+        *rows2 = (int)rows;
+        return s2_bytes(*w2words, *rows2, (int)batch, r2, ntg) + kSmemReserve;
+    };
+    for (int k = 2; k <= kMaxK2; ++k) {
+        const int64_t total = std::min<int64_t>((int64_t)k * sms, tiles_all);
+        int64_t given = 0;
+        double frac[kMaxGroup];
+        for (int i = 0; i < count; ++i) {
+            const int64_t ti = calls[i].m / 16;
+            const double share = (double)total * (double)(ti * (calls[i].r / kCB)) / (double)work;
+            const int64_t c = std::max<int64_t>(1, std::min<int64_t>((int64_t)share, ti));
+            ctas[i] = (int)c;
+            frac[i] = share - (double)c;
+            given += c;
+        }
+        while (given < total) {  // largest remainders first, never past one CTA per tile
+            int best = -1;
+            for (int i = 0; i < count; ++i)
+                if (ctas[i] < calls[i].m / 16 && (best < 0 || frac[i] > frac[best])) best = i;
+            if (best < 0) break;
+            ++ctas[best];
+            frac[best] -= 1.0;
+            ++given;
+        }
+        const size_t need = measure();
+        if (total == tiles_all) {  // one tile per CTA: no smaller CTAs exist, and no cap is needed
+            *per_sm = 0;
+            return;
+        }
+        if ((size_t)k * need <= kSmemPerSM) {
+            *per_sm = k;
+            return;
+        }
+    }
+    for (int i = 0; i < count; ++i) ctas[i] = (int)((calls[i].m / 16 + kWaveTiles2 - 1) / kWaveTiles2);
+    *per_sm = 0;
+    measure();
 }
 
 // Column blocks per stage-1 split: about two CTAs per SM over the whole launch, at least
@@ -697,9 +857,8 @@ static int stage1_cps(const DecodeCall* calls, int count, int max_splits) {
 void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, int max_splits, int64_t* t_floats,
                            int64_t* tgmax_floats, int64_t* partial_floats, int64_t* counter_ints) {
     const int cps = stage1_cps(calls, count, max_splits);
-    int64_t tiles = 0;
-    for (int i = 0; i < count; ++i) tiles += calls[i].m / 16;
-    const int rt = stage2_rt(tiles);
+    int ctas[kMaxGroup], w2words = 0, rows2 = 0, per_sm = 0;
+    stage2_plan(calls, count, batch, ctas, &w2words, &rows2, &per_sm);
     int64_t t = 0, gm = 0, pf = 0, ci = 0;
     for (int i = 0; i < count; ++i) {
         const int64_t ncb = calls[i].n / kCB, nsplit = (ncb + cps - 1) / cps;
@@ -708,7 +867,7 @@ void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, in
         if (nsplit > 1) pf += nsplit * batch * calls[i].r;
         ci += calls[i].r / kRowsS1;
         if (calls[i].y_norm) {  // per-CTA sums of y^2 and one arrival counter
-            pf += batch * (calls[i].m / (16 * rt));
+            pf += batch * ctas[i];
             ci += 1;
         }
     }
@@ -729,16 +888,12 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
     DecGroup grp;
     grp.count = count;
     grp.batch = (int)batch;
-    int64_t tiles = 0, r_max = 0;
-    for (int i = 0; i < count; ++i) {
-        tiles += calls[i].m / 16;
-        r_max = calls[i].r > r_max ? calls[i].r : r_max;
-    }
-    const int rt = stage2_rt(tiles);
+    int64_t r_max = 0;
+    for (int i = 0; i < count; ++i) r_max = calls[i].r > r_max ? calls[i].r : r_max;
+    int ctas[kMaxGroup];
+    stage2_plan(calls, count, batch, ctas, &grp.w2words, &grp.rows2, &grp.per_sm2);
     const int cps = stage1_cps(calls, count, max_splits);
     grp.r2 = stage2_span(r_max, batch);
-    // an odd number of 4-word groups per row spreads the 8 rows a warp reads over all 32 banks
-    grp.w2stride = grp.r2 / 32 + (((grp.r2 / 128) % 2) ? 0 : 4);
     grp.depth1 = cps > kChunkCB ? 2 : 1;
     size_t toff = 0, goff = 0, poff = 0, coff = 0;
     grp.s1_start[0] = grp.s2_start[0] = 0;
@@ -765,13 +920,13 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
         if (c.y_norm) {
             L.norm_partials = ws->partials + npoff;
             L.norm_counter = ws->counters + ncoff;
-            npoff += (size_t)batch * (c.m / (16 * rt));
+            npoff += (size_t)batch * ctas[i];
             ncoff += 1;
         }
         L.m = (int)c.m;
         L.n = (int)c.n;
         L.r = (int)c.r;
-        L.rt = rt;
+        L.s2_ctas = ctas[i];
         L.cps = cps;
         L.nsplit = (int)((c.n / kCB + cps - 1) / cps);
         L.t = ws->t + toff;
@@ -782,8 +937,22 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
         goff += (size_t)batch * (c.r / kRowsS1);
         if (L.nsplit > 1) poff += (size_t)L.nsplit * batch * c.r;
         coff += (size_t)(c.r / kRowsS1);
-        grp.s1_start[i + 1] = grp.s1_start[i] + (int)(c.r / kRowsS1) * L.nsplit;
-        grp.s2_start[i + 1] = grp.s2_start[i] + (int)(c.m / (16 * rt));
+    }
+    // Launch order of the layers' CTA ranges: the layers with the longest path through a
+    // stage go first, so that their CTAs are the first resident and the first scheduled
+    // (stage 1: most column splits, i.e. the longest hand-off; stage 2: largest rank, i.e.
+    // the most fragments to build per CTA).  Ties keep the caller's order.
+    int o1[kMaxGroup], o2[kMaxGroup];
+    for (int i = 0; i < count; ++i) o1[i] = o2[i] = i;
+    std::stable_sort(o1, o1 + count, [&](int a, int b) { return grp.L[a].nsplit > grp.L[b].nsplit; });
+    std::stable_sort(o2, o2 + count, [&](int a, int b) { return grp.L[a].r > grp.L[b].r; });
+    for (int k = 0; k < count; ++k) {
+        const DecLayer& L1 = grp.L[o1[k]];
+        const DecLayer& L2 = grp.L[o2[k]];
+        grp.s1_layer[k] = (unsigned char)o1[k];
+        grp.s2_layer[k] = (unsigned char)o2[k];
+        grp.s1_start[k + 1] = grp.s1_start[k] + (L1.r / kRowsS1) * L1.nsplit;
+        grp.s2_start[k + 1] = grp.s2_start[k] + L2.s2_ctas;
     }
     if (batch <= 4) return launch_group<1>(grp, stream, ws->device);
     return launch_group<2>(grp, stream, ws->device);
