@@ -175,7 +175,7 @@ __host__ __device__ inline size_t s1_x_bytes(int depth, int batch) { return (siz
 __host__ __device__ inline size_t s1_bytes(int depth, int batch, int ntg) {
     return s1_w_bytes(depth) + s1_x_bytes(depth, batch) + frag_bytes(kChunkCB, ntg) + sizeof(Misc);
 }
-// stage 2: w [rows][stride(r)] | t [batch][r2] f32 | frag (all r2/128 CBs) | bq [rows2][batch] | misc
+// stage 2: w [rows][stride(r)] | t [batch][r2] f32 | frag (all r2/128 CBs) | bq [rows2][batch] | s1 [rows2] | misc
 // Words per staged row of a layer of rank r: the first span's words, plus 4 when that is an
 // even number of 4-word groups (an odd number spreads the 8 rows a warp reads over all
 // 32 banks).
@@ -185,9 +185,10 @@ __host__ __device__ inline int s2_stride(int r, int r2) {
 }
 __host__ __device__ inline size_t s2_t_bytes(int batch, int r2) { return (size_t)batch * r2 * 4; }
 __host__ __device__ inline size_t s2_bq_bytes(int rows2, int batch) { return ((size_t)rows2 * batch * 4 + 15) / 16 * 16; }
+__host__ __device__ inline size_t s2_s1_bytes(int rows2) { return ((size_t)rows2 * 2 + 15) / 16 * 16; }
 __host__ __device__ inline size_t s2_bytes(int w2words, int rows2, int batch, int r2, int ntg) {
     return (size_t)w2words * 4 + s2_t_bytes(batch, r2) + frag_bytes(r2 / kCB, ntg) +
-           s2_bq_bytes(rows2, batch) + sizeof(Misc);
+           s2_bq_bytes(rows2, batch) + s2_s1_bytes(rows2) + sizeof(Misc);
 }
 
 template <int NTG>
@@ -389,19 +390,29 @@ stage1_kernel(const __grid_constant__ DecGroup grp) {
             for (int row = threadIdx.x >> 3; row < kRowsS1; row += kThreads1 / 8)
                 cp_async16(dst + row * kS1Stride + 4 * p, src + row * wpr + 4 * p);
     };
-    auto fetch_x = [&](int ch) {  // x rows (batch of them) and s2 of chunk ch; s2 goes in slot `batch`
+    // x rows (batch of them) of chunk ch, and (a weight, fetched with the sign words) s2 of
+    // chunk ch in slot `batch`
+    auto fetch_xs = [&](int ch, const uint16_t* base, int64_t tok_stride, int tok0, int tok1) {
         const int per_tok = chunk_cb(ch) * kCB / 8;
         const int col0 = (cbA + ch * kChunkCB) * kCB;
-        for (int tok = 0; tok <= batch; ++tok) {
-            const uint16_t* src = tok < batch ? L.x + (int64_t)tok * n + col0 : L.s2 + col0;
+        for (int tok = tok0; tok < tok1; ++tok) {
+            const uint16_t* src = base + (int64_t)(tok - tok0) * tok_stride + col0;
             for (int p = threadIdx.x; p < per_tok; p += kThreads1) cp_async16(xchunk(ch % depth, tok) + 8 * p, src + 8 * p);
         }
     };
+    auto fetch_x = [&](int ch) { fetch_xs(ch, L.x, n, 0, batch); };
+    auto fetch_s2 = [&](int ch) { fetch_xs(ch, L.s2, 0, batch, batch + 1); };
 
     // weights first: they do not depend on the previous kernel
-    if (nchunks > 0) fetch_w(0);
+    if (nchunks > 0) {
+        fetch_w(0);
+        fetch_s2(0);
+    }
     cp_async_commit();
-    if (nchunks > 1) fetch_w(1);
+    if (nchunks > 1) {
+        fetch_w(1);
+        fetch_s2(1);
+    }
     cp_async_commit();
     if (nchunks > 2 && threadIdx.x < kRowsS1)
         prefetch_l2(W + threadIdx.x * wpr + (cbA + 2 * kChunkCB) * 4, (uint32_t)((cbB - cbA - 2 * kChunkCB) * 16));
@@ -477,6 +488,7 @@ stage1_kernel(const __grid_constant__ DecGroup grp) {
         __syncthreads();  // buffers are free again
         if (ch + 2 < nchunks) {
             fetch_w(ch + 2);
+            fetch_s2(ch + 2);
             fetch_x(ch + 2);
             cp_async_commit();
         }
@@ -606,7 +618,8 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
     float* tbuf = reinterpret_cast<float*>(smem_raw + (size_t)grp.w2words * 4);
     uint4* frag = reinterpret_cast<uint4*>(smem_raw + (size_t)grp.w2words * 4 + s2_t_bytes(batch, r2));
     int* bq = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(frag) + frag_bytes(r2 / kCB, NTG));
-    Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(bq) + s2_bq_bytes(rows2, batch));
+    uint16_t* s1buf = reinterpret_cast<uint16_t*>(reinterpret_cast<unsigned char*>(bq) + s2_bq_bytes(rows2, batch));
+    Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(s1buf) + s2_s1_bytes(rows2));
 
     const int rk = find_range(grp.s2_start, grp.count, blockIdx.x);
     const DecLayer& L = grp.L[grp.s2_layer[rk]];
@@ -623,6 +636,8 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
     const uint32_t* W = L.Upk + row0 * wpr;
     const int nsc = (r + r2 - 1) / r2;  // column spans held on chip one after the other
 
+    // consecutive threads take consecutive 16-byte pieces of the CTA's rows (whole warps per
+    // instruction: measured faster than one row per warp)
     auto fetch_w = [&](int sc) {
         const int cols = min(r2, r - sc * r2);
         const int per_row = cols / 128;  // 16-byte pieces
@@ -641,6 +656,7 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
     };
 
     fetch_w(0);
+    for (int p = threadIdx.x; p < rows / 8; p += kThreads) cp_async16(s1buf + 8 * p, L.s1 + row0 + 8 * p);  // s1 of the rows
     cp_async_commit();
     if (nsc > 1)
         for (int row = threadIdx.x; row < rows; row += kThreads)
@@ -705,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
     __syncthreads();
     auto y_at = [&](int tok, int i) {
         const float v = (float)(2 * (int64_t)bq[i * batch + tok] - mi.qsum[tok]) * pow2f(mi.e[tok] - kQBits);
-        return f16_to_f32(L.s1[row0 + i]) * v;
+        return f16_to_f32(s1buf[i]) * v;
     };
     for (int idx = threadIdx.x; idx < rows * batch; idx += kThreads) {
         const int tok = idx / rows, i = idx % rows;
