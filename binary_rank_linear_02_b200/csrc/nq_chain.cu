@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(kNormThreads, 1) rms_norm_kernel(const float* 
 // used to bring the x of a call from pinned host memory (read through its device
 // address) into the device staging buffer in one launch instead of one copy per layer.
 __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ GatherList list) {
+    pdl_trigger();  // the decode kernels may launch and stage their weights during the copy
     if ((int)blockIdx.y >= list.count) return;
     const GatherSeg& g = list.seg[blockIdx.y];
     const uint4* src = static_cast<const uint4*>(g.src);
