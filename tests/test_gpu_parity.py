@@ -291,6 +291,36 @@ def test_grouped_llama2_7b_block(nq, orc, batch):
         assert rel_err(y.cpu().numpy(), c.oracle(orc)) <= TOL
 
 
+@pytest.mark.parametrize("batch", [2, 3, 5])
+def test_grouped_llama2_7b_block_other_batches(nq, orc, batch):
+    """The seven-layer decode step at the batch sizes between the benchmarked ones: one
+    token group with two and three tokens (one wave of the balanced stage-2 plan), and the
+    first batch that needs two token groups."""
+    cases = [Case(orc, nq, m, n, r, batch, seed=1960 + 10 * batch + i)
+             for i, (_, m, n, r) in enumerate(synth.LLAMA2_7B_LAYERS)]
+    ys = [torch.empty((batch, c.m), dtype=torch.float32, device="cuda") for c in cases]
+    nq.lowrank_linear_fwd_grouped([(c.x_d, c.Upk, c.Vpk, c.s1_d, c.s2_d, y, c.m, c.n, c.r)
+                                   for c, y in zip(cases, ys)], batch)
+    torch.cuda.synchronize()
+    for c, y in zip(cases, ys):
+        assert rel_err(y.cpu().numpy(), c.oracle(orc)) <= TOL
+
+
+@pytest.mark.parametrize("batch", [1, 4])
+def test_grouped_mixed_sizes(nq, orc, batch):
+    """A large layer grouped with small ones: the stage-2 plan gives each small layer a
+    single CTA (at least one per layer) and the large one the rest; stage 1 mixes one-split
+    and many-split layers."""
+    shapes = [(11008, 4096, 2432), (128, 128, 128), (256, 2176, 128), (384, 640, 256)]
+    cases = [Case(orc, nq, m, n, r, batch, seed=2900 + i) for i, (m, n, r) in enumerate(shapes)]
+    ys = [torch.empty((batch, c.m), dtype=torch.float32, device="cuda") for c in cases]
+    nq.lowrank_linear_fwd_grouped([(c.x_d, c.Upk, c.Vpk, c.s1_d, c.s2_d, y, c.m, c.n, c.r)
+                                   for c, y in zip(cases, ys)], batch)
+    torch.cuda.synchronize()
+    for c, y in zip(cases, ys):
+        assert rel_err(y.cpu().numpy(), c.oracle(orc)) <= TOL
+
+
 @pytest.mark.parametrize("batch", [1, 4])
 def test_grouped_llama2_70b_block(nq, orc, batch):
     """The Llama-2-70B-shaped block in one grouped call (up to 28 column splits per layer,
