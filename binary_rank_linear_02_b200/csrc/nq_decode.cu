@@ -183,7 +183,10 @@ __host__ __device__ inline int s2_stride(int r, int r2) {
     const int cols = r < r2 ? r : r2;
     return cols / 32 + (((cols / 128) % 2) ? 0 : 4);
 }
-__host__ __device__ inline size_t s2_t_bytes(int batch, int r2) { return (size_t)batch * r2 * 4; }
+// t is staged with 8 floats of padding after every 32, so that the four columns 32 apart
+// that a fragment task reads fall in different banks
+__host__ __device__ inline int s2_t_row(int r2) { return r2 + r2 / 4; }
+__host__ __device__ inline size_t s2_t_bytes(int batch, int r2) { return (size_t)batch * s2_t_row(r2) * 4; }
 __host__ __device__ inline size_t s2_bq_bytes(int rows2, int batch) { return ((size_t)rows2 * batch * 4 + 15) / 16 * 16; }
 __host__ __device__ inline size_t s2_s1_bytes(int rows2) { return ((size_t)rows2 * 2 + 15) / 16 * 16; }
 __host__ __device__ inline size_t s2_bytes(int w2words, int rows2, int batch, int r2, int ntg) {
@@ -203,35 +206,36 @@ __device__ __forceinline__ void zero_fragments(uint4* frag, int ncb) {
 }
 
 // B fragments of `ncb` column blocks from the fp32 values val(tok, col) (col from the span's
-// first column), quantised with up[tok]; adds each token's sum of q to qsum.  One task =
-// (cb, token, word t of the CB, fragment word j = 2s + h): the 4 columns 32t + s + 4h + 8c
-// (c in 0..3) give word j of two lanes, the hi-limb lane 8*tok' + t and the lo-limb lane
-// 8*tok' + 4 + t (tok' = token within its group).  The 32 tasks of a warp step share one
-// token, so the warp adds its q's with a shuffle reduction.
+// first column), quantised with up[tok]; adds each token's sum of q to qsum.  Per token,
+// one task = (cb, word t of the CB, fragment word j = 2s + h): the 4 columns
+// 32t + s + 4h + 8c (c in 0..3) give word j of two lanes, the hi-limb lane 8*tok' + t and
+// the lo-limb lane 8*tok' + 4 + t (tok' = token within its group).  Each thread adds up its
+// q's of the token; one warp reduction per token and warp.
 template <int NTG, int NT, typename Val>
 __device__ __forceinline__ void build_fragments(uint4* frag, Misc& mi, Val val, int ncb, int batch) {
-    const int tasks = ncb * batch * 32;  // a multiple of 32: whole warps take part in every step
-    for (int task = threadIdx.x; task < tasks; task += NT) {
-        const int j = task & 7, t = (task >> 3) & 3;
-        const int tok = (task >> 5) % batch, cb = (task >> 5) / batch;
-        const int s4 = j >> 1, h = j & 1;
+    const int tasks = ncb * 32;
+    for (int tok = 0; tok < batch; ++tok) {
         const float up = mi.up[tok];
-        const int col = cb * kCB + 32 * t + s4 + 4 * h;
-        uint32_t wh = 0, wl = 0;
+        const int tg = tok >> 2, ti = tok & 3;
         int qs = 0;
+        for (int task = threadIdx.x; task < tasks; task += NT) {
+            const int j = task & 7, t = (task >> 3) & 3, cb = task >> 5;
+            const int s4 = j >> 1, h = j & 1;
+            const int col = cb * kCB + 32 * t + s4 + 4 * h;
+            uint32_t wh = 0, wl = 0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int q = quantise(val(tok, col + 8 * c), up);
-            qs += q;
-            wh |= (uint32_t)((q >> 7) & 0xFF) << (8 * c);
-            wl |= (uint32_t)(q & 0x7F) << (8 * c);
+            for (int c = 0; c < 4; ++c) {
+                const int q = quantise(val(tok, col + 8 * c), up);
+                qs += q;
+                wh |= (uint32_t)((q >> 7) & 0xFF) << (8 * c);
+                wl |= (uint32_t)(q & 0x7F) << (8 * c);
+            }
+            // word j lives in half j >> 2 at component j & 3
+            reinterpret_cast<uint32_t*>(frag_ptr<NTG>(frag, cb, tg, j >> 2, 8 * ti + t))[j & 3] = wh;
+            reinterpret_cast<uint32_t*>(frag_ptr<NTG>(frag, cb, tg, j >> 2, 8 * ti + 4 + t))[j & 3] = wl;
         }
         for (int o = 16; o > 0; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
-        if ((threadIdx.x & 31) == 0) atomicAdd(&mi.qsum[tok], qs);
-        const int tg = tok >> 2, ti = tok & 3;
-        // word j lives in half j >> 2 at component j & 3
-        reinterpret_cast<uint32_t*>(frag_ptr<NTG>(frag, cb, tg, j >> 2, 8 * ti + t))[j & 3] = wh;
-        reinterpret_cast<uint32_t*>(frag_ptr<NTG>(frag, cb, tg, j >> 2, 8 * ti + 4 + t))[j & 3] = wl;
+        if ((threadIdx.x & 31) == 0 && qs != 0) atomicAdd(&mi.qsum[tok], qs);
     }
 }
 
@@ -651,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
         const int per_tok = cols / 4;
         for (int i = threadIdx.x; i < batch * per_tok; i += kThreads) {
             const int tok = i / per_tok, p = i % per_tok;
-            cp_async16(tbuf + tok * r2 + 4 * p, L.t + (int64_t)tok * r + sc * r2 + 4 * p);
+            cp_async16(tbuf + tok * s2_t_row(r2) + 4 * p + 8 * (p >> 3), L.t + (int64_t)tok * r + sc * r2 + 4 * p);
         }
     };
 
@@ -693,7 +697,8 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
         __syncthreads();
         // every column block of the span at once: one barrier, then an uninterrupted MMA loop
         const int ncb = min(r2, r - sc * r2) / kCB;
-        build_fragments<NTG, kThreads>(frag, mi, [&](int tok, int c) { return tbuf[tok * r2 + c]; }, ncb, batch);
+        build_fragments<NTG, kThreads>(
+            frag, mi, [&](int tok, int c) { return tbuf[tok * s2_t_row(r2) + c + 8 * (c >> 5)]; }, ncb, batch);
         __syncthreads();
         // the span's units (tile, column block) in tile-major order, an even run per warp;
         // a run covers the ends of up to a few tiles, each added into bq when done
