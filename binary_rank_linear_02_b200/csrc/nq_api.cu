@@ -37,15 +37,18 @@ int pointer_kind(const void* p) {
     return (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) ? 1 : 0;
 }
 
-// Host memory the device can address: the device address of page-locked (pinned) host
-// memory, nullptr for pageable memory or anything else.
-void* pinned_device_ptr(const void* p) {
+// One query for x or y: the kind as pointer_kind, and for page-locked (pinned) host memory
+// the device address of it in *pinned (nullptr for pageable memory or anything else).
+int pointer_kind_pinned(const void* p, void** pinned) {
+    *pinned = nullptr;
     cudaPointerAttributes attr;
     if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
         cudaGetLastError();
-        return nullptr;
+        return 0;
     }
-    return attr.type == cudaMemoryTypeHost ? attr.devicePointer : nullptr;
+    if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) return 1;
+    if (attr.type == cudaMemoryTypeHost) *pinned = attr.devicePointer;
+    return 0;
 }
 
 }  // namespace
@@ -215,17 +218,18 @@ static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_line
         const nq_linear_desc& L = desc(i);
         if (!pointer_kind(L.Upk) || !pointer_kind(L.Vpk) || !pointer_kind(L.s1) || !pointer_kind(L.s2))
             return NQ_ERR_PTRKIND;
-        x_host[i] = pointer_kind(L.x) == 0;
-        y_host[i] = pointer_kind(L.y) == 0;
+        void *xp = nullptr, *yp = nullptr;
+        x_host[i] = pointer_kind_pinned(L.x, &xp) == 0;
+        y_host[i] = pointer_kind_pinned(L.y, &yp) == 0;
         if (ex && (x_host[i] || y_host[i] || (ex[i].y_bf16 && !pointer_kind(ex[i].y_bf16)) ||
                    (ex[i].y_rmsnorm_bf16 && !pointer_kind(ex[i].y_rmsnorm_bf16))))
             return NQ_ERR_PTRKIND;
         if (x_host[i]) {
-            x_pin[i] = pinned_device_ptr(L.x);
+            x_pin[i] = xp;
             xbytes += align_up(sizeof(uint16_t) * (size_t)batch * L.n, 256);
         }
         if (y_host[i]) {
-            y_pin[i] = pinned_device_ptr(L.y);
+            y_pin[i] = yp;
             if (!y_pin[i]) ybytes += align_up(sizeof(float) * (size_t)batch * L.m, 256);
         }
     }
