@@ -46,6 +46,8 @@ def _load(path: str) -> ctypes.CDLL:
     L.orc_unpack_signs.argtypes = [p, i64, i64, p]
     L.orc_lowrank_linear_fwd.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p]
     L.orc_stage1.argtypes = [p, p, p, i64, i64, i64, p]
+    L.orc_lowrank_linear_bwd_input.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p]
+    L.orc_transpose_signs.argtypes = [p, i64, i64, p]
     L.orc_bits_per_weight.argtypes = [i64, i64, i64]
     L.orc_bits_per_weight.restype = ctypes.c_double
     L.orc_bf16_to_double.argtypes = [ctypes.c_uint16]
@@ -93,6 +95,40 @@ class Oracle:
         st = self.lib.orc_unpack_signs(_ptr(p), rows, cols, _ptr(out))
         if st != ORC_OK:
             raise ValueError(f"orc_unpack_signs failed with status {st}")
+        return out
+
+    def lowrank_linear_bwd_input(self, dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r) -> np.ndarray:
+        """dx (batch x n, float64) = s2 * (V (U^T (s1 * dy))): the gradient of the layer's
+        output with respect to its input, for the same packings as the forward pass.
+
+        dy_bits: batch x m uint16 bfloat16 patterns; the other arguments as in
+        ``lowrank_linear_fwd``.
+        """
+        dy = np.ascontiguousarray(dy_bits, dtype=np.uint16).reshape(-1, m)
+        batch = dy.shape[0]
+        U = np.ascontiguousarray(Upk, dtype=np.uint32)
+        V = np.ascontiguousarray(Vpk, dtype=np.uint32)
+        a = np.ascontiguousarray(s1_bits, dtype=np.uint16)
+        b = np.ascontiguousarray(s2_bits, dtype=np.uint16)
+        assert U.shape == (m, words_per_row(r)) and V.shape == (r, words_per_row(n))
+        assert a.shape == (m,) and b.shape == (n,)
+        dx = np.zeros((batch, n), dtype=np.float64)
+        if batch == 0:
+            return dx
+        st = self.lib.orc_lowrank_linear_bwd_input(
+            _ptr(dy), _ptr(U), _ptr(V), _ptr(a), _ptr(b), m, n, r, batch, _ptr(dx))
+        if st != ORC_OK:
+            raise ValueError(f"orc_lowrank_linear_bwd_input failed with status {st}")
+        return dx
+
+    def transpose_signs(self, packed: np.ndarray, rows: int, cols: int) -> np.ndarray:
+        """rows x ceil(cols/32) packed words -> cols x ceil(rows/32) words of the transpose."""
+        p = np.ascontiguousarray(packed, dtype=np.uint32)
+        assert p.shape == (rows, words_per_row(cols))
+        out = np.zeros((cols, words_per_row(rows)), dtype=np.uint32)
+        st = self.lib.orc_transpose_signs(_ptr(p), rows, cols, _ptr(out))
+        if st != ORC_OK:
+            raise ValueError(f"orc_transpose_signs failed with status {st}")
         return out
 
     def lowrank_linear_fwd(self, x_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r) -> np.ndarray:
@@ -235,3 +271,11 @@ def chain_block(h_bits, w):
 
 def decode_chain(h0_bits, blocks):
     return default().decode_chain(h0_bits, blocks)
+
+
+def lowrank_linear_bwd_input(dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r):
+    return default().lowrank_linear_bwd_input(dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r)
+
+
+def transpose_signs(packed, rows, cols):
+    return default().transpose_signs(packed, rows, cols)

@@ -174,6 +174,77 @@ int orc_lowrank_linear_fwd(const uint16_t *x, const uint32_t *Upk, const uint32_
     return ORC_OK;
 }
 
+/* ---- the input gradient ----
+ *
+ * The refinement step fine-tunes the factorised components with straight-through
+ * estimators (hardwired.dev, section "Krok 3": the gradient of the sign function is taken
+ * as the identity on the backward pass), so every step back-propagates through the layer.
+ * With the signs and scales held fixed the layer is the linear map W x, and the gradient
+ * with respect to its input is the transpose applied to the output gradient:
+ *     dx = W^T dy = s2 (.) ( V . ( U^T . ( s1 (.) dy ) ) ).
+ *
+ * dy  : batch x m bfloat16 bit patterns, row-major (one token per row)
+ * Upk, Vpk, s1, s2 : exactly as in the forward pass (this routine reads the same packings)
+ * dx  : batch x n doubles (written)
+ */
+int orc_lowrank_linear_bwd_input(const uint16_t *dy, const uint32_t *Upk, const uint32_t *Vpk,
+                                 const uint16_t *s1, const uint16_t *s2, int64_t m, int64_t n,
+                                 int64_t r, int64_t batch, double *dx) {
+    if (m <= 0 || n <= 0 || r <= 0 || batch < 0) return ORC_ERR_ARG;
+    if (batch == 0) return ORC_OK;
+    if (!dy || !Upk || !Vpk || !s1 || !s2 || !dx) return ORC_ERR_ARG;
+    const int64_t wpr_u = words_per_row(r), wpr_v = words_per_row(n);
+    double *g = (double *)malloc(sizeof(double) * (size_t)(m * batch));
+    double *u = (double *)malloc(sizeof(double) * (size_t)(r * batch));
+    if (!g || !u) { free(g); free(u); return ORC_ERR_ARG; }
+
+    /* step 1: g = s1 (.) dy, exact in double */
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t i = 0; i < m; ++i)
+            g[b * m + i] = orc_f16_to_double(s1[i]) * orc_bf16_to_double(dy[b * m + i]);
+
+    /* step 2: u_k = sum_i U[i][k] * g_i, increasing i */
+#pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k < r; ++k) {
+        for (int64_t b = 0; b < batch; ++b) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < m; ++i)
+                acc += orc_sign_at(Upk, wpr_u, i, k) * g[b * m + i];
+            u[b * r + k] = acc;
+        }
+    }
+
+    /* step 3: dx_j = s2_j * sum_k V[j][k] * u_k, increasing k (V[j][k] is entry (k, j) of V^T) */
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < n; ++j) {
+        double sj = orc_f16_to_double(s2[j]);
+        for (int64_t b = 0; b < batch; ++b) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < r; ++k)
+                acc += orc_sign_at(Vpk, wpr_v, k, j) * u[b * r + k];
+            dx[b * n + j] = sj * acc;
+        }
+    }
+    free(g);
+    free(u);
+    return ORC_OK;
+}
+
+/* Transpose of a packed sign matrix: `in` holds rows x cols entries in rows x ceil(cols/32)
+ * words, `out` receives the cols x rows transpose in cols x ceil(rows/32) words (same bit
+ * convention, unused high bits zero). */
+int orc_transpose_signs(const uint32_t *in, int64_t rows, int64_t cols, uint32_t *out) {
+    if (rows < 0 || cols < 0) return ORC_ERR_ARG;
+    if (rows == 0 || cols == 0) return ORC_OK;
+    if (!in || !out) return ORC_ERR_ARG;
+    const int64_t wpr_in = words_per_row(cols), wpr_out = words_per_row(rows);
+    memset(out, 0, sizeof(uint32_t) * (size_t)(cols * wpr_out));
+    for (int64_t i = 0; i < rows; ++i)
+        for (int64_t j = 0; j < cols; ++j)
+            if (orc_sign_at(in, wpr_in, i, j) > 0) out[j * wpr_out + i / 32] |= 1u << (i % 32);
+    return ORC_OK;
+}
+
 /* The intermediate t = V^T (s2 (.) x) alone (batch x r doubles), for tests that look
  * at the rank bottleneck. */
 int orc_stage1(const uint16_t *x, const uint32_t *Vpk, const uint16_t *s2, int64_t n,

@@ -346,6 +346,57 @@ def pin_chain_block(o):
     assert np.array_equal(h2, o.chain_block(out["h_next"], w2)["h_next"])
 
 
+def dense_input_gradient(dy_bits, U, V, s1_bits, s2_bits):
+    """dx = dy W with W = diag(s1) U V^T diag(s2), materialised with numpy in float64."""
+    dy = synth.bf16_bits_to_f32(dy_bits).astype(np.float64)
+    s1 = synth.f16_bits_to_f32(s1_bits).astype(np.float64)
+    s2 = synth.f16_bits_to_f32(s2_bits).astype(np.float64)
+    W = (s1[:, None] * (U.astype(np.float64) @ V.astype(np.float64).T)) * s2[None, :]
+    return dy @ W
+
+
+def _bwd(o, dy, U, V, s1, s2):
+    m, r = U.shape
+    n = V.shape[0]
+    return o.lowrank_linear_bwd_input(dy, o.pack_signs(U), o.pack_signs(np.ascontiguousarray(V.T)), s1, s2, m, n, r)
+
+
+def pin_bwd_input_dense(o):
+    """The input gradient equals dy W for the materialised dense weight (fp64, 1e-12), on
+    shapes where m, n and r all differ (a swapped operand cannot line up)."""
+    for (m, n, r, batch, seed) in ((8, 12, 3, 2, 51), (33, 40, 7, 3, 52), (5, 70, 40, 1, 53)):
+        _, U, V, s1, s2 = _case(m, n, r, batch, seed)
+        dy = synth.activations_bf16(batch, m, seed, "dy")
+        dx = _bwd(o, dy, U, V, s1, s2)
+        assert dx.shape == (batch, n)
+        assert rel_err(dx, dense_input_gradient(dy, U, V, s1, s2)) <= 1e-12, (m, n, r)
+
+
+def pin_bwd_input_adjoint(o):
+    """The adjoint identity <y(x), dy> = <x, dx(dy)> ties the input gradient to the forward
+    pass: both sides are the bilinear form dy^T W x (fp64, 1e-12 relative)."""
+    for (m, n, r, batch, seed) in ((24, 40, 9, 3, 61), (64, 32, 17, 2, 62)):
+        x, U, V, s1, s2 = _case(m, n, r, batch, seed)
+        dy = synth.activations_bf16(batch, m, seed, "dy")
+        y = _fwd(o, x, U, V, s1, s2)
+        dx = _bwd(o, dy, U, V, s1, s2)
+        lhs = float(np.sum(y * synth.bf16_bits_to_f32(dy).astype(np.float64)))
+        rhs = float(np.sum(synth.bf16_bits_to_f32(x).astype(np.float64) * dx))
+        assert abs(lhs - rhs) <= 1e-12 * max(abs(lhs), 1.0), (m, n, r, lhs, rhs)
+
+
+def pin_transpose_signs(o):
+    """The packed transpose is numpy's transpose of the unpacked signs (ragged shapes
+    included), and transposing twice gives the original words back."""
+    for (rows, cols, seed) in ((70, 45, 71), (32, 32, 72), (1, 100, 73), (129, 3, 74)):
+        s = synth.signs(rows, cols, seed)
+        p = o.pack_signs(s)
+        t = o.transpose_signs(p, rows, cols)
+        assert t.shape == (cols, (rows + 31) // 32)
+        assert np.array_equal(o.unpack_signs(t, rows), s.T)
+        assert np.array_equal(o.transpose_signs(t, cols, rows), p)
+
+
 def torch_bf16_to_f64(bits):
     import torch
 
@@ -365,4 +416,7 @@ ALL_PINS = [
     pin_bf16_rounding,
     pin_rms_normalize,
     pin_chain_block,
+    pin_bwd_input_dense,
+    pin_bwd_input_adjoint,
+    pin_transpose_signs,
 ]

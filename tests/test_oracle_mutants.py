@@ -34,6 +34,14 @@ MUTANTS = {
     "bf16_subnormal_quantum": ("if (E < -126) E = -126;", "if (E < -127) E = -127;"),
     "rms_sum_not_mean": ("sqrt(acc / (double)cols)", "sqrt(acc)"),
     "rms_no_sqrt": ("double rms = sqrt(acc / (double)cols);", "double rms = acc / (double)cols;"),
+    "bwd_drop_s1": ("g[b * m + i] = orc_f16_to_double(s1[i]) * orc_bf16_to_double(dy[b * m + i]);",
+                    "g[b * m + i] = orc_bf16_to_double(dy[b * m + i]);"),
+    "bwd_s1_for_s2": ("double sj = orc_f16_to_double(s2[j]);", "double sj = orc_f16_to_double(s1[j % m]);"),
+    "bwd_u_from_v": ("acc += orc_sign_at(Upk, wpr_u, i, k) * g[b * m + i];",
+                     "acc += orc_sign_at(Upk, wpr_u, i % m, (k + i) % r) * g[b * m + i];"),
+    "bwd_dx_wrong_u": ("acc += orc_sign_at(Vpk, wpr_v, k, j) * u[b * r + k];",
+                       "acc += orc_sign_at(Vpk, wpr_v, k, j) * u[k];"),
+    "transpose_msb": ("out[j * wpr_out + i / 32] |= 1u << (i % 32);", "out[j * wpr_out + i / 32] |= 1u << (31 - i % 32);"),
 }
 
 
