@@ -418,6 +418,31 @@ int nq_unpack_signs(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* 
     return unpack_device(packed, rows, cols, out, static_cast<cudaStream_t>(stream));
 }
 
+int nq_transpose_signs(const uint32_t* packed, int64_t rows, int64_t cols, uint32_t* out, void* stream) {
+    if (rows < 0 || cols < 0) return NQ_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return NQ_OK;
+    if (!packed || !out) return NQ_ERR_NULL;
+    if (rows > (int64_t(1) << 40) / cols) return NQ_ERR_SHAPE;
+    const int kp = pointer_kind(packed), ko = pointer_kind(out);
+    if (kp != ko) return NQ_ERR_PTRKIND;
+    const int64_t wpr_in = (cols + 31) / 32, wpr_out = (rows + 31) / 32;
+    if (kp == 0) {
+        memset(out, 0, sizeof(uint32_t) * (size_t)(cols * wpr_out));
+        for (int64_t row = 0; row < rows; ++row)
+            for (int64_t c = 0; c < cols; ++c)
+                if ((packed[row * wpr_in + c / 32] >> (c % 32)) & 1u) out[c * wpr_out + row / 32] |= 1u << (row % 32);
+        return NQ_OK;
+    }
+    return transpose_device(packed, rows, cols, out, static_cast<cudaStream_t>(stream));
+}
+
+int nq_lowrank_linear_bwd_input(const void* dy, const uint32_t* UpkT, const uint32_t* VpkT, const void* s1,
+                                const void* s2, int64_t m, int64_t n, int64_t r, int64_t batch, float* dx,
+                                void* stream) {
+    // the forward pass with the factors' roles exchanged: dx = s2 (.) (V (U^T (s1 (.) dy)))
+    return nq_lowrank_linear_fwd(dy, VpkT, UpkT, s2, s1, n, m, r, batch, dx, stream);
+}
+
 int nq_cast_f32_to_bf16(const float* src, int64_t count, void* dst, void* stream) {
     if (count < 0 || count > kMaxElems) return NQ_ERR_SHAPE;
     if (count == 0) return NQ_OK;

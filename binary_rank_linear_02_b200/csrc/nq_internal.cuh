@@ -105,6 +105,7 @@ int prefill_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk,
 int pack_device(const int8_t* signs, int64_t rows, int64_t cols, uint32_t* out, unsigned* flag,
                 cudaStream_t stream);
 int unpack_device(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* out, cudaStream_t stream);
+int transpose_device(const uint32_t* packed, int64_t rows, int64_t cols, uint32_t* out, cudaStream_t stream);
 constexpr int kMaxGather = 16;
 struct GatherSeg {
     const void* src;

@@ -1,4 +1,5 @@
-// nq_pack.cu -- one-bit storage of sign matrices on the device.
+// nq_pack.cu -- one-bit storage of sign matrices on the device: packing, unpacking and
+// the transpose of a packed matrix (the backward pass reads U and V along the other axis).
 //
 // The stored form (one bit per +1/-1 entry, hardwired.dev section "Jak NanoQuant
 // funguje"; bit 1 = +1, least significant bit = lowest column, sign(0) = +1) is the
@@ -58,6 +59,30 @@ __global__ void unpack_kernel(const uint32_t* __restrict__ packed, int64_t rows,
     }
 }
 
+// Transpose of a packed sign matrix, one warp per 32 x 32 tile: lane l holds the word of
+// input row 32*tr + l for column block tc; ballot c collects bit c of the 32 words, i.e. the
+// word of output row 32*tc + c for row block tr, and lane c keeps it.  Rows beyond the
+// matrix read as zero words, so the unused high bits of the output stay zero.
+__global__ void transpose_kernel(const uint32_t* __restrict__ in, int64_t rows, int64_t cols, int64_t wpr_in,
+                                 int64_t wpr_out, uint32_t* __restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t tiles_c = wpr_in, tiles = ((rows + 31) / 32) * tiles_c;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    for (int64_t tile = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); tile < tiles; tile += warps) {
+        const int64_t tr = tile / tiles_c, tc = tile % tiles_c;
+        const int64_t row = 32 * tr + lane;
+        const uint32_t w = row < rows ? in[row * wpr_in + tc] : 0u;
+        uint32_t mine = 0;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+            const uint32_t b = __ballot_sync(0xffffffffu, (w >> c) & 1u);
+            if (lane == c) mine = b;
+        }
+        const int64_t col = 32 * tc + lane;
+        if (col < cols) out[col * wpr_out + tr] = mine;
+    }
+}
+
 int grid_for(int64_t items, int threads) {
     int64_t blocks = (items + threads - 1) / threads;
     int64_t cap = (int64_t)sm_count() * 16;
@@ -79,6 +104,14 @@ int unpack_device(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* ou
     const int64_t wpr = (cols + 31) / 32;
     const int threads = 256;
     unpack_kernel<<<grid_for(rows * cols, threads), threads, 0, stream>>>(packed, rows, cols, wpr, out);
+    return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
+}
+
+int transpose_device(const uint32_t* packed, int64_t rows, int64_t cols, uint32_t* out, cudaStream_t stream) {
+    const int64_t wpr_in = (cols + 31) / 32, wpr_out = (rows + 31) / 32;
+    const int threads = 256;
+    const int64_t tiles = ((rows + 31) / 32) * wpr_in;
+    transpose_kernel<<<grid_for(tiles * 32, threads), threads, 0, stream>>>(packed, rows, cols, wpr_in, wpr_out, out);
     return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
 }
 

@@ -66,6 +66,8 @@ def _load() -> ctypes.CDLL:
     L.nq_pack_signs.argtypes = [p, i64, i64, p, p]
     L.nq_pack_signs.restype = ctypes.c_int
     L.nq_unpack_signs.argtypes = [p, i64, i64, p, p]
+    L.nq_transpose_signs.argtypes = [p, i64, i64, p, p]
+    L.nq_lowrank_linear_bwd_input.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p]
     L.nq_unpack_signs.restype = ctypes.c_int
     L.nq_lowrank_linear_fwd.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p]
     L.nq_lowrank_linear_fwd.restype = ctypes.c_int
@@ -108,6 +110,14 @@ def nq_pack_signs(signs_ptr: int, rows: int, cols: int, out_ptr: int, stream: in
 
 def nq_unpack_signs(packed_ptr: int, rows: int, cols: int, out_ptr: int, stream: int = 0) -> int:
     return _lib.nq_unpack_signs(packed_ptr, rows, cols, out_ptr, stream)
+
+
+def nq_transpose_signs(packed_ptr: int, rows: int, cols: int, out_ptr: int, stream: int = 0) -> int:
+    return _lib.nq_transpose_signs(packed_ptr, rows, cols, out_ptr, stream)
+
+
+def nq_lowrank_linear_bwd_input(dy_ptr, UpkT_ptr, VpkT_ptr, s1_ptr, s2_ptr, m, n, r, batch, dx_ptr, stream=0) -> int:
+    return _lib.nq_lowrank_linear_bwd_input(dy_ptr, UpkT_ptr, VpkT_ptr, s1_ptr, s2_ptr, m, n, r, batch, dx_ptr, stream)
 
 
 def nq_lowrank_linear_fwd(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n, r, batch, y_ptr, stream=0) -> int:
@@ -220,6 +230,40 @@ def unpack_signs(packed, cols: int, out=None, stream=None):
             out = torch.empty((rows, cols), dtype=torch.int8, device=packed.device)
     _check(_lib.nq_unpack_signs(_ptr(packed), rows, cols, _ptr(out), _stream(stream, packed)), "nq_unpack_signs")
     return out
+
+
+def transpose_signs(packed, rows: int, cols: int, out=None, stream=None):
+    """rows x ceil(cols/32) packed words -> cols x ceil(rows/32) words of the transpose."""
+    wpr_out = (rows + 31) // 32
+    if out is None:
+        if isinstance(packed, np.ndarray):
+            out = np.empty((cols, wpr_out), dtype=np.uint32)
+        else:
+            import torch
+
+            out = torch.empty((cols, wpr_out), dtype=torch.int32, device=packed.device)
+    _check(_lib.nq_transpose_signs(_ptr(packed), rows, cols, _ptr(out), _stream(stream, packed)),
+           "nq_transpose_signs")
+    return out
+
+
+def lowrank_linear_bwd_input(dy, UpkT, VpkT, s1, s2, m: int, n: int, r: int, dx=None, stream=None):
+    """dx (batch x n, float32) = s2 * (V (U^T (s1 * dy))), the gradient of the layer's
+    output with respect to its input.
+
+    dy: batch x m bfloat16 (device or host); UpkT: r x m/32 = transpose_signs(Upk, m, r) and
+    VpkT: n x r/32 = transpose_signs(Vpk, r, n) (device); s1: m and s2: n fp16 (device).
+    """
+    batch = dy.shape[0] if dy.dim() == 2 else 1
+    if dx is None:
+        import torch
+
+        dx = torch.empty((batch, n), dtype=torch.float32, device=dy.device,
+                         pin_memory=(not dy.is_cuda and torch.cuda.is_available()))
+    st = _lib.nq_lowrank_linear_bwd_input(_ptr(dy), _ptr(UpkT), _ptr(VpkT), _ptr(s1), _ptr(s2), m, n, r, batch,
+                                          _ptr(dx), _stream(stream, dy, UpkT, dx))
+    _check(st, "nq_lowrank_linear_bwd_input")
+    return dx
 
 
 def lowrank_linear_fwd(x, Upk, Vpk, s1, s2, m: int, n: int, r: int, y=None, stream=None):

@@ -109,6 +109,37 @@ int nq_lowrank_linear_fwd(const void* x, const uint32_t* Upk, const uint32_t* Vp
                           const void* s1, const void* s2, int64_t m, int64_t n, int64_t r,
                           int64_t batch, float* y, void* stream);
 
+/*
+ * nq_transpose_signs -- the transpose of a packed sign matrix: `packed` holds rows x cols
+ * entries as rows x ceil(cols/32) uint32 (the layout of nq_pack_signs), `out` receives the
+ * cols x rows transpose as cols x ceil(rows/32) uint32 in the same layout (unused high bits
+ * of each row's last word zero).  rows, cols >= 0; rows*cols == 0 is a no-op returning
+ * NQ_OK.  Both pointers on the device (a kernel on `stream`, no synchronisation) or both
+ * in host memory (on the calling thread); mixed: NQ_ERR_PTRKIND.  Used to give the
+ * backward pass its packings: UpkT = transpose of Upk (m x r -> r x m), VpkT = transpose of
+ * Vpk (r x n -> n x r).  `out` must not overlap `packed`.
+ */
+int nq_transpose_signs(const uint32_t* packed, int64_t rows, int64_t cols, uint32_t* out, void* stream);
+
+/*
+ * nq_lowrank_linear_bwd_input -- the gradient of the layer's output with respect to its
+ * input, dx = W^T dy = s2 (.) (V (U^T (s1 (.) dy))), for `batch` tokens: the step of the
+ * straight-through refinement of the factorised components (hardwired.dev, "Krok 3")
+ * that passes the gradient on to the layer before.
+ *   dy   : batch x m bfloat16, row-major (one token per row)
+ *   UpkT : r x (m/32) uint32, device memory (rows of U^T: nq_transpose_signs(Upk, m, r))
+ *   VpkT : n x (r/32) uint32, device memory (rows of V: nq_transpose_signs(Vpk, r, n))
+ *   s1   : m fp16, s2 : n fp16, device memory (the layer's scales)
+ *   dx   : batch x n float32, row-major (written)
+ * It is the forward pass of the layer with the roles of the factors exchanged (U' = V,
+ * V' = U, s1' = s2, s2' = s1, m' = n, n' = m), so every rule, path and accuracy statement
+ * of nq_lowrank_linear_fwd applies with those names; dy and dx may be host memory as x
+ * and y there.
+ */
+int nq_lowrank_linear_bwd_input(const void* dy, const uint32_t* UpkT, const uint32_t* VpkT, const void* s1,
+                                const void* s2, int64_t m, int64_t n, int64_t r, int64_t batch, float* dx,
+                                void* stream);
+
 /* One factorised layer of a grouped call (same meaning and rules as the arguments of
  * nq_lowrank_linear_fwd; every pointer in device memory, 16-byte aligned). */
 typedef struct nq_linear_desc {

@@ -103,6 +103,40 @@ def test_forward_argument_errors(nq):
     assert nq.nq_workspace_reserve(128, 128, 128, -2) == nq.NQ_ERR_BATCH
 
 
+def test_host_transpose_matches_oracle(nq, orc):
+    """The host-memory transpose (calling thread) equals the oracle's, ragged shapes included."""
+    from binary_rank_linear_02_b200 import synth
+
+    for (rows, cols, seed) in ((70, 45, 81), (1, 100, 82), (129, 3, 83), (64, 96, 84)):
+        packed = orc.pack_signs(synth.signs(rows, cols, seed))
+        got = nq.transpose_signs(packed, rows, cols)
+        assert np.array_equal(got, orc.transpose_signs(packed, rows, cols)), (rows, cols)
+
+
+def test_transpose_and_backward_argument_errors(nq):
+    out = np.zeros((4, 1), dtype=np.uint32)
+    packed = np.zeros((1, 1), dtype=np.uint32)
+    t = nq.nq_transpose_signs
+    assert t(0, 1, 4, out.ctypes.data, 0) == nq.NQ_ERR_NULL
+    assert t(packed.ctypes.data, 1, 4, 0, 0) == nq.NQ_ERR_NULL
+    assert t(packed.ctypes.data, -1, 4, out.ctypes.data, 0) == nq.NQ_ERR_SHAPE
+    assert t(packed.ctypes.data, 1, -4, out.ctypes.data, 0) == nq.NQ_ERR_SHAPE
+    assert t(packed.ctypes.data, 0, 4, out.ctypes.data, 0) == nq.NQ_OK
+    # the input gradient is the forward with the factors exchanged: the same checks, the
+    # shape rules applying to (m' = n, n' = m)
+    buf = np.zeros(1 << 16, dtype=np.uint8)
+    base = (buf.ctypes.data + 255) // 256 * 256
+    p = [base + 1024 * i for i in range(6)]
+    b = nq.nq_lowrank_linear_bwd_input
+    assert b(p[0], p[1], p[2], p[3], p[4], 128, 128, 128, -1, p[5], 0) == nq.NQ_ERR_BATCH
+    assert b(p[0], p[1], p[2], p[3], p[4], 100, 128, 128, 1, p[5], 0) == nq.NQ_ERR_SHAPE
+    assert b(p[0], p[1], p[2], p[3], p[4], 128, 128, 64, 1, p[5], 0) == nq.NQ_ERR_SHAPE
+    assert b(p[0], p[1], p[2], p[3], p[4], 128, 128, 128, 0, p[5], 0) == nq.NQ_OK
+    assert b(0, p[1], p[2], p[3], p[4], 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_NULL
+    assert b(p[0] + 2, p[1], p[2], p[3], p[4], 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_ALIGN
+    assert b(p[0], p[1], p[2], p[3], p[4], 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_PTRKIND
+
+
 def test_grouped_argument_errors(nq):
     buf = np.zeros(1 << 16, dtype=np.uint8)
     base = (buf.ctypes.data + 255) // 256 * 256
