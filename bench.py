@@ -178,6 +178,36 @@ class DecodeWorkload:
                 raise RuntimeError(f"nq_lowrank_linear_fwd: {self.nq.nq_status_string(st)}")
 
 
+def backward_workload(layers, batch, seed, device):
+    """The input gradient of the same layers, one grouped call per step: each layer's
+    forward packings are transposed on the device (nq_transpose_signs) and the grouped
+    forward call runs with the factors' roles exchanged (U' = V, V' = U, s1' = s2,
+    s2' = s1, m' = n, n' = m), which is what nq_lowrank_linear_bwd_input does per layer."""
+    import torch
+
+    work = DecodeWorkload(layers, batch, seed, device)
+    nq = work.nq
+    work.dy = [torch.from_numpy(synth.activations_bf16(batch, m, seed, li, "dy").view(np.int16)).to(device)
+               for li, (_, m, n, r) in enumerate(layers)]
+    work.dx = [torch.empty((batch, n), dtype=torch.float32, device=device) for (_, m, n, r) in layers]
+    work.transposed = []  # kept alive for graph replays
+    descs = []
+    for per in work.sets:
+        entries = []
+        for li, (_, m, n, r) in enumerate(layers):
+            Upk, Vpk, s1, s2 = per[li]
+            UpkT = nq.transpose_signs(Upk, m, r)
+            VpkT = nq.transpose_signs(Vpk, r, n)
+            work.transposed += [UpkT, VpkT]
+            entries.append((work.dy[li], VpkT, UpkT, s2, s1, work.dx[li], n, m, r))
+        descs.append(nq.make_descs(entries))
+    for (_, m, n, r) in layers:
+        nq.workspace_reserve(n, m, r, batch)
+    torch.cuda.synchronize()
+    work.descs = descs
+    return work
+
+
 def aggregate(ms_local: float, units_local: float, dist=None, device=None):
     """Whole-job numbers of independent replicas: (max time over ranks, units of all ranks).
 
@@ -341,6 +371,15 @@ def run_ours(args):
         secondary["decode_b8_gbs"] = round(w8.step_bytes * args.steps / (ms8 * 1e-3) / 1e9, 1)
         secondary["decode_b8_tokens_per_s"] = round(8 * args.steps / (ms8 * 1e-3), 1)
         del w8
+        # the input gradient dx = W^T dy of the same block (backward of the layers)
+        for bb in (1, 8):
+            wb = backward_workload(layers, bb, seed=123 + bb, device=device)
+            with torch.cuda.stream(stream):
+                wb.step(0, stream.cuda_stream)
+            torch.cuda.synchronize()
+            msb = timed_graphs(wb, args.steps, args.warmup, stream)
+            secondary["backward_input_b%d_gbs" % bb] = round(wb.step_bytes * args.steps / (msb * 1e-3) / 1e9, 1)
+            del wb
 
     if args.secondary and world == 1:
         secondary["prefill_11008x4096_r2432"] = run_prefill_sweep(device, stream, args.warmup, peaks)
