@@ -34,8 +34,10 @@
 // before it waits on the previous kernel (programmatic dependent launch) and lets the next
 // kernel launch at once, so weight streaming overlaps the dependency chain.  Stage 1
 // splits each 128-row block's columns so that every CTA stages one chunk; the last CTA of a
-// block adds the partial sums in a fixed order (deterministic).  Stage 2 holds its whole
-// row block and the whole of t on chip.  Several independent layers can share one launch.
+// block adds the partial sums in a fixed order (deterministic).  Stage 2 runs as one even
+// wave where it fits: each layer gets CTAs in proportion to its work, each CTA holds its
+// rows of U and the whole of t on chip.  Several independent layers share one launch, the
+// slowest first in the grid.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
