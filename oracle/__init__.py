@@ -48,6 +48,7 @@ def _load(path: str) -> ctypes.CDLL:
     L.orc_stage1.argtypes = [p, p, p, i64, i64, i64, p]
     L.orc_lowrank_linear_bwd_input.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p]
     L.orc_transpose_signs.argtypes = [p, i64, i64, p]
+    L.orc_lowrank_linear_bwd_scales.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p, p]
     L.orc_bits_per_weight.argtypes = [i64, i64, i64]
     L.orc_bits_per_weight.restype = ctypes.c_double
     L.orc_bf16_to_double.argtypes = [ctypes.c_uint16]
@@ -120,6 +121,25 @@ class Oracle:
         if st != ORC_OK:
             raise ValueError(f"orc_lowrank_linear_bwd_input failed with status {st}")
         return dx
+
+    def lowrank_linear_bwd_scales(self, x_bits, dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r):
+        """(ds1 (m,), ds2 (n,)) float64: the gradients with respect to the scale vectors for
+        input x (batch x n bf16 patterns) and output gradient dy (batch x m bf16 patterns)."""
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1, n)
+        dy = np.ascontiguousarray(dy_bits, dtype=np.uint16).reshape(-1, m)
+        assert x.shape[0] == dy.shape[0]
+        U = np.ascontiguousarray(Upk, dtype=np.uint32)
+        V = np.ascontiguousarray(Vpk, dtype=np.uint32)
+        a = np.ascontiguousarray(s1_bits, dtype=np.uint16)
+        b = np.ascontiguousarray(s2_bits, dtype=np.uint16)
+        assert U.shape == (m, words_per_row(r)) and V.shape == (r, words_per_row(n))
+        ds1 = np.zeros(m, dtype=np.float64)
+        ds2 = np.zeros(n, dtype=np.float64)
+        st = self.lib.orc_lowrank_linear_bwd_scales(
+            _ptr(x), _ptr(dy), _ptr(U), _ptr(V), _ptr(a), _ptr(b), m, n, r, x.shape[0], _ptr(ds1), _ptr(ds2))
+        if st != ORC_OK:
+            raise ValueError(f"orc_lowrank_linear_bwd_scales failed with status {st}")
+        return ds1, ds2
 
     def transpose_signs(self, packed: np.ndarray, rows: int, cols: int) -> np.ndarray:
         """rows x ceil(cols/32) packed words -> cols x ceil(rows/32) words of the transpose."""
@@ -279,3 +299,7 @@ def lowrank_linear_bwd_input(dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r):
 
 def transpose_signs(packed, rows, cols):
     return default().transpose_signs(packed, rows, cols)
+
+
+def lowrank_linear_bwd_scales(x_bits, dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r):
+    return default().lowrank_linear_bwd_scales(x_bits, dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r)

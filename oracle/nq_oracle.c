@@ -230,6 +230,60 @@ int orc_lowrank_linear_bwd_input(const uint16_t *dy, const uint32_t *Upk, const 
     return ORC_OK;
 }
 
+/* ---- the scale gradients ----
+ *
+ * The refinement step tunes the scaling factors together with the binary factors
+ * (hardwired.dev, section "Krok 3").  For a loss with output gradient dy, y is linear in
+ * each scale vector, so
+ *     ds1_i = sum_b dy[b][i] * z[b][i],   z = U (V^T (s2 (.) x))      (y = s1 (.) z)
+ *     ds2_j = sum_b x[b][j]  * w[b][j],   w = V (U^T (s1 (.) dy))     (dx = s2 (.) w)
+ * x: batch x n and dy: batch x m bfloat16 bit patterns; Upk, Vpk, s1, s2 as in the
+ * forward pass; ds1 (m) and ds2 (n) doubles (written).  The sums over b run in increasing
+ * b after z and w are complete.
+ */
+int orc_lowrank_linear_bwd_scales(const uint16_t *x, const uint16_t *dy, const uint32_t *Upk,
+                                  const uint32_t *Vpk, const uint16_t *s1, const uint16_t *s2,
+                                  int64_t m, int64_t n, int64_t r, int64_t batch, double *ds1,
+                                  double *ds2) {
+    if (m <= 0 || n <= 0 || r <= 0 || batch < 0) return ORC_ERR_ARG;
+    if (!ds1 || !ds2) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < m; ++i) ds1[i] = 0.0;
+    for (int64_t j = 0; j < n; ++j) ds2[j] = 0.0;
+    if (batch == 0) return ORC_OK;
+    if (!x || !dy || !Upk || !Vpk || !s1 || !s2) return ORC_ERR_ARG;
+    const int64_t wpr_u = words_per_row(r), wpr_v = words_per_row(n);
+    double *t = (double *)malloc(sizeof(double) * (size_t)(r * batch));
+    double *u = (double *)malloc(sizeof(double) * (size_t)(r * batch));
+    if (!t || !u) { free(t); free(u); return ORC_ERR_ARG; }
+    /* t = V^T (s2 (.) x) and u = U^T (s1 (.) dy), sums in increasing index */
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t k = 0; k < r; ++k) {
+            double at = 0.0, au = 0.0;
+            for (int64_t j = 0; j < n; ++j)
+                at += orc_sign_at(Vpk, wpr_v, k, j) * (orc_f16_to_double(s2[j]) * orc_bf16_to_double(x[b * n + j]));
+            for (int64_t i = 0; i < m; ++i)
+                au += orc_sign_at(Upk, wpr_u, i, k) * (orc_f16_to_double(s1[i]) * orc_bf16_to_double(dy[b * m + i]));
+            t[b * r + k] = at;
+            u[b * r + k] = au;
+        }
+    /* ds1_i = sum_b dy_bi * (U t_b)_i ;  ds2_j = sum_b x_bj * (V u_b)_j */
+    for (int64_t i = 0; i < m; ++i)
+        for (int64_t b = 0; b < batch; ++b) {
+            double z = 0.0;
+            for (int64_t k = 0; k < r; ++k) z += orc_sign_at(Upk, wpr_u, i, k) * t[b * r + k];
+            ds1[i] += orc_bf16_to_double(dy[b * m + i]) * z;
+        }
+    for (int64_t j = 0; j < n; ++j)
+        for (int64_t b = 0; b < batch; ++b) {
+            double w = 0.0;
+            for (int64_t k = 0; k < r; ++k) w += orc_sign_at(Vpk, wpr_v, k, j) * u[b * r + k];
+            ds2[j] += orc_bf16_to_double(x[b * n + j]) * w;
+        }
+    free(t);
+    free(u);
+    return ORC_OK;
+}
+
 /* Transpose of a packed sign matrix: `in` holds rows x cols entries in rows x ceil(cols/32)
  * words, `out` receives the cols x rows transpose in cols x ceil(rows/32) words (same bit
  * convention, unused high bits zero). */

@@ -385,6 +385,59 @@ def pin_bwd_input_adjoint(o):
         assert abs(lhs - rhs) <= 1e-12 * max(abs(lhs), 1.0), (m, n, r, lhs, rhs)
 
 
+def _bwd_scales(o, x, dy, U, V, s1, s2):
+    m, r = U.shape
+    n = V.shape[0]
+    return o.lowrank_linear_bwd_scales(x, dy, o.pack_signs(U), o.pack_signs(np.ascontiguousarray(V.T)), s1, s2,
+                                       m, n, r)
+
+
+def pin_bwd_scales_linear_in_scale(o):
+    """L = sum(dy * y) is linear in every scale entry, so dL/ds1_i = (L(s1) - L(s1 with
+    entry i set to 0)) / s1_i, and likewise for s2_j; L taken from the forward oracle."""
+    m, n, r, batch = 12, 20, 5, 3
+    x, U, V, s1, s2 = _case(m, n, r, batch, 81)
+    dy = synth.activations_bf16(batch, m, 81, "dy")
+    dyf = synth.bf16_bits_to_f32(dy).astype(np.float64)
+    ds1, ds2 = _bwd_scales(o, x, dy, U, V, s1, s2)
+    assert ds1.shape == (m,) and ds2.shape == (n,)
+
+    def loss(a, b):
+        return float(np.sum(dyf * _fwd(o, x, U, V, a, b)))
+
+    L0 = loss(s1, s2)
+    s1f = synth.f16_bits_to_f32(s1).astype(np.float64)
+    s2f = synth.f16_bits_to_f32(s2).astype(np.float64)
+    for i in (0, 5, m - 1):
+        a = s1.copy()
+        a[i] = 0
+        fd = (L0 - loss(a, s2)) / s1f[i]
+        assert abs(fd - ds1[i]) <= 1e-11 * max(1.0, abs(fd)), (i, fd, ds1[i])
+    for j in (0, 7, n - 1):
+        b = s2.copy()
+        b[j] = 0
+        fd = (L0 - loss(s1, b)) / s2f[j]
+        assert abs(fd - ds2[j]) <= 1e-11 * max(1.0, abs(fd)), (j, fd, ds2[j])
+
+
+def pin_bwd_scales_dense(o):
+    """ds1 = sum_b dy_b (.) (U V^T diag(s2) x_b) and ds2 = sum_b x_b (.) (V U^T diag(s1) dy_b),
+    with the factors materialised by numpy (fp64, 1e-12)."""
+    for (m, n, r, batch, seed) in ((9, 14, 4, 2, 82), (40, 24, 11, 3, 83)):
+        x, U, V, s1, s2 = _case(m, n, r, batch, seed)
+        dy = synth.activations_bf16(batch, m, seed, "dy")
+        ds1, ds2 = _bwd_scales(o, x, dy, U, V, s1, s2)
+        xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+        dyf = synth.bf16_bits_to_f32(dy).astype(np.float64)
+        s1f = synth.f16_bits_to_f32(s1).astype(np.float64)
+        s2f = synth.f16_bits_to_f32(s2).astype(np.float64)
+        UV = U.astype(np.float64) @ V.astype(np.float64).T  # m x n
+        z = (xf * s2f[None, :]) @ UV.T                      # batch x m
+        w = (dyf * s1f[None, :]) @ UV                       # batch x n
+        assert rel_err(ds1, np.sum(dyf * z, axis=0)) <= 1e-12
+        assert rel_err(ds2, np.sum(xf * w, axis=0)) <= 1e-12
+
+
 def pin_transpose_signs(o):
     """The packed transpose is numpy's transpose of the unpacked signs (ragged shapes
     included), and transposing twice gives the original words back."""
@@ -419,4 +472,6 @@ ALL_PINS = [
     pin_bwd_input_dense,
     pin_bwd_input_adjoint,
     pin_transpose_signs,
+    pin_bwd_scales_linear_in_scale,
+    pin_bwd_scales_dense,
 ]

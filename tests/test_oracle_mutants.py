@@ -41,6 +41,12 @@ MUTANTS = {
                      "acc += orc_sign_at(Upk, wpr_u, i % m, (k + i) % r) * g[b * m + i];"),
     "bwd_dx_wrong_u": ("acc += orc_sign_at(Vpk, wpr_v, k, j) * u[b * r + k];",
                        "acc += orc_sign_at(Vpk, wpr_v, k, j) * u[k];"),
+    "scales_ds1_uses_s1": ("ds1[i] += orc_bf16_to_double(dy[b * m + i]) * z;",
+                           "ds1[i] += orc_f16_to_double(s1[i]) * orc_bf16_to_double(dy[b * m + i]) * z;"),
+    "scales_ds2_from_t": ("for (int64_t k = 0; k < r; ++k) w += orc_sign_at(Vpk, wpr_v, k, j) * u[b * r + k];",
+                          "for (int64_t k = 0; k < r; ++k) w += orc_sign_at(Vpk, wpr_v, k, j) * t[b * r + k];"),
+    "scales_u_no_s1": ("au += orc_sign_at(Upk, wpr_u, i, k) * (orc_f16_to_double(s1[i]) * orc_bf16_to_double(dy[b * m + i]));",
+                       "au += orc_sign_at(Upk, wpr_u, i, k) * orc_bf16_to_double(dy[b * m + i]);"),
     "transpose_msb": ("out[j * wpr_out + i / 32] |= 1u << (i % 32);", "out[j * wpr_out + i / 32] |= 1u << (31 - i % 32);"),
 }
 
