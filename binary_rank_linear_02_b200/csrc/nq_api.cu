@@ -175,6 +175,28 @@ static int ensure_staging(Workspace* w, size_t xbytes, size_t ybytes) {
     return NQ_OK;
 }
 
+// Scratch of the scale gradients: a vector of fp16 ones (the layer evaluated without one
+// of its scales) and the batch x max(m, n) fp32 output of that evaluation.
+static int ensure_grad_scratch(Workspace* w, size_t ones, size_t outs_bytes, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (ones > w->ones_count) {
+        if (w->ones) { cudaDeviceSynchronize(); cudaFree(w->ones); w->ones = nullptr; w->ones_count = 0; }
+        void* p = nullptr;
+        if (cudaMalloc(&p, sizeof(uint16_t) * ones) != cudaSuccess) { cudaGetLastError(); return NQ_ERR_NOMEM; }
+        w->ones = static_cast<uint16_t*>(p);
+        if (fill_u16_device(w->ones, (int64_t)ones, 0x3C00, stream) != NQ_OK) return NQ_ERR_CUDA;  // fp16 1.0
+        w->ones_count = ones;
+    }
+    if (outs_bytes > w->gstage_bytes) {
+        if (w->gstage) { cudaDeviceSynchronize(); cudaFree(w->gstage); w->gstage = nullptr; w->gstage_bytes = 0; }
+        void* p = nullptr;
+        if (cudaMalloc(&p, outs_bytes) != cudaSuccess) { cudaGetLastError(); return NQ_ERR_NOMEM; }
+        w->gstage = static_cast<float*>(p);
+        w->gstage_bytes = outs_bytes;
+    }
+    return NQ_OK;
+}
+
 }  // namespace nq
 
 using namespace nq;
@@ -441,6 +463,49 @@ int nq_lowrank_linear_bwd_input(const void* dy, const uint32_t* UpkT, const uint
                                 void* stream) {
     // the forward pass with the factors' roles exchanged: dx = s2 (.) (V (U^T (s1 (.) dy)))
     return nq_lowrank_linear_fwd(dy, VpkT, UpkT, s2, s1, n, m, r, batch, dx, stream);
+}
+
+int nq_lowrank_linear_bwd_scales(const void* x, const void* dy, const uint32_t* Upk, const uint32_t* Vpk,
+                                 const uint32_t* UpkT, const uint32_t* VpkT, const void* s1, const void* s2,
+                                 int64_t m, int64_t n, int64_t r, int64_t batch, float* ds1, float* ds2,
+                                 void* stream) {
+    if (batch < 0) return NQ_ERR_BATCH;
+    if (m <= 0 || n <= 0 || r <= 0 || m % 128 || n % 128 || r % 128 || m > kMaxDim || n > kMaxDim ||
+        r > kMaxRank)
+        return NQ_ERR_SHAPE;
+    if (batch > (int64_t(1) << 40) / (m > n ? m : n)) return NQ_ERR_SHAPE;
+    if (!ds1 && !ds2) return NQ_OK;
+    if (!x || !dy || !Upk || !Vpk || !UpkT || !VpkT || !s1 || !s2) return NQ_ERR_NULL;
+    const void* ptrs[] = {x, dy, Upk, Vpk, UpkT, VpkT, s1, s2, ds1, ds2};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return NQ_ERR_ALIGN;
+    for (const void* p : ptrs)
+        if (p && !pointer_kind(p)) return NQ_ERR_PTRKIND;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (batch == 0) {  // empty sums
+        if (ds1 && cudaMemsetAsync(ds1, 0, sizeof(float) * (size_t)m, s) != cudaSuccess) return NQ_ERR_CUDA;
+        if (ds2 && cudaMemsetAsync(ds2, 0, sizeof(float) * (size_t)n, s) != cudaSuccess) return NQ_ERR_CUDA;
+        return NQ_OK;
+    }
+    int st = NQ_OK;
+    const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, m > n ? m : n, m > n ? m : n, r};
+    Workspace* ws = workspace_for(m > n ? m : n, m > n ? m : n, r, batch, decode_need(&c, 1, batch), &st);
+    if (!ws) return st;
+    st = ensure_grad_scratch(ws, (size_t)(m > n ? m : n), sizeof(float) * (size_t)batch * (size_t)(m > n ? m : n), s);
+    if (st != NQ_OK) return st;
+    if (ds1) {  // z = U (V^T (s2 (.) x)): the forward with s1 = 1; ds1 = sum_b dy (.) z
+        st = nq_lowrank_linear_fwd(x, Upk, Vpk, ws->ones, s2, m, n, r, batch, ws->gstage, stream);
+        if (st != NQ_OK) return st;
+        st = col_dot_device(static_cast<const uint16_t*>(dy), ws->gstage, batch, m, ds1, s);
+        if (st != NQ_OK) return st;
+    }
+    if (ds2) {  // w = V (U^T (s1 (.) dy)): the input gradient with s2 = 1; ds2 = sum_b x (.) w
+        st = nq_lowrank_linear_fwd(dy, VpkT, UpkT, ws->ones, s1, n, m, r, batch, ws->gstage, stream);
+        if (st != NQ_OK) return st;
+        st = col_dot_device(static_cast<const uint16_t*>(x), ws->gstage, batch, n, ds2, s);
+        if (st != NQ_OK) return st;
+    }
+    return NQ_OK;
 }
 
 int nq_cast_f32_to_bf16(const float* src, int64_t count, void* dst, void* stream) {

@@ -12,6 +12,9 @@
 // chain's critical path, so they are shaped for latency: launched with programmatic
 // dependent launch, they let the next kernel start its weight prefetch early and read
 // their input only after the producing kernel has finished.
+//
+// Also here: the gather of pinned host inputs, and the per-column dot products over the
+// tokens that finish the scale gradients of the backward pass.
 #include <cuda_bf16.h>
 
 #include "nq_internal.cuh"
@@ -109,6 +112,25 @@ __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ Gat
         dst[i] = src[i];
 }
 
+// Scale gradients: out[i] = sum_b bf16(a[b][i]) * z[b][i], one thread per i, the tokens in
+// increasing order (deterministic).  z comes from the kernel before (programmatic wait).
+__global__ void __launch_bounds__(256) col_dot_kernel(const uint16_t* __restrict__ a, const float* __restrict__ z,
+                                                      int64_t batch, int64_t len, float* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < len; i += (int64_t)gridDim.x * blockDim.x) {
+        float acc = 0.f;
+        for (int64_t b = 0; b < batch; ++b)
+            acc = fmaf(__uint_as_float((uint32_t)a[b * len + i] << 16), z[b * len + i], acc);
+        out[i] = acc;
+    }
+}
+
+__global__ void fill_u16_kernel(uint16_t* p, int64_t count, uint16_t value) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x)
+        p[i] = value;
+}
+
 }  // namespace
 
 int gather_device(const GatherList& list, cudaStream_t stream) {
@@ -137,6 +159,23 @@ int rms_normalize_bf16_device(const float* src, int64_t rows, int64_t cols, uint
                    cudaSuccess
                ? NQ_OK
                : NQ_ERR_CUDA;
+}
+
+int col_dot_device(const uint16_t* a, const float* z, int64_t batch, int64_t len, float* out, cudaStream_t stream) {
+    int64_t blocks = (len + 255) / 256;
+    if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
+    return launch_pdl(col_dot_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, a, z, batch, len, out) ==
+                   cudaSuccess
+               ? NQ_OK
+               : NQ_ERR_CUDA;
+}
+
+int fill_u16_device(uint16_t* p, int64_t count, uint16_t value, cudaStream_t stream) {
+    int64_t blocks = (count + 255) / 256;
+    if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
+    if (blocks < 1) blocks = 1;
+    fill_u16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(p, count, value);
+    return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
 }
 
 }  // namespace nq

@@ -22,7 +22,7 @@ struct Workspace {
     char* base = nullptr;
     // carved regions
     float* t = nullptr;            // [t_cap] (decode: sum over a launch's layers of batch x r)
-    float* tgmax = nullptr;        // [tgmax_cap] (decode: batch x r/64 per layer)
+    float* tgmax = nullptr;        // [tgmax_cap] (decode: batch x r/128 per layer)
     float* partials = nullptr;     // [partial_cap] (stage-1 column splits; prefill K splits; norm sums)
     int* counters = nullptr;       // [counter_cap] (arrival counters, zero between calls)
     unsigned* status = nullptr;    // [0]: pack value check, [1]: device wait timeout
@@ -31,6 +31,9 @@ struct Workspace {
     void* xstage = nullptr;        // staged host x
     float* ystage = nullptr;       // staged host y
     size_t xstage_bytes = 0, ystage_bytes = 0;
+    uint16_t* ones = nullptr;      // [ones_count] fp16 1.0 (scale gradients: the layer without a scale)
+    float* gstage = nullptr;       // scale gradients: batch x max(m, n) outputs of the layer without a scale
+    size_t ones_count = 0, gstage_bytes = 0;
     size_t t_cap = 0, tgmax_cap = 0, partial_cap = 0, counter_cap = 0;
     int64_t r_cap = 0, n_cap = 0, m_cap = 0, batch_cap = 0, rsum_cap = 0;
 };
@@ -106,6 +109,9 @@ int pack_device(const int8_t* signs, int64_t rows, int64_t cols, uint32_t* out, 
                 cudaStream_t stream);
 int unpack_device(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* out, cudaStream_t stream);
 int transpose_device(const uint32_t* packed, int64_t rows, int64_t cols, uint32_t* out, cudaStream_t stream);
+// out[i] = sum over b (increasing) of bf16(a[b][i]) * z[b][i], for i < len
+int col_dot_device(const uint16_t* a, const float* z, int64_t batch, int64_t len, float* out, cudaStream_t stream);
+int fill_u16_device(uint16_t* p, int64_t count, uint16_t value, cudaStream_t stream);
 constexpr int kMaxGather = 16;
 struct GatherSeg {
     const void* src;

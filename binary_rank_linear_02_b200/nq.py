@@ -68,6 +68,7 @@ def _load() -> ctypes.CDLL:
     L.nq_unpack_signs.argtypes = [p, i64, i64, p, p]
     L.nq_transpose_signs.argtypes = [p, i64, i64, p, p]
     L.nq_lowrank_linear_bwd_input.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p]
+    L.nq_lowrank_linear_bwd_scales.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p]
     L.nq_unpack_signs.restype = ctypes.c_int
     L.nq_lowrank_linear_fwd.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p]
     L.nq_lowrank_linear_fwd.restype = ctypes.c_int
@@ -118,6 +119,12 @@ def nq_transpose_signs(packed_ptr: int, rows: int, cols: int, out_ptr: int, stre
 
 def nq_lowrank_linear_bwd_input(dy_ptr, UpkT_ptr, VpkT_ptr, s1_ptr, s2_ptr, m, n, r, batch, dx_ptr, stream=0) -> int:
     return _lib.nq_lowrank_linear_bwd_input(dy_ptr, UpkT_ptr, VpkT_ptr, s1_ptr, s2_ptr, m, n, r, batch, dx_ptr, stream)
+
+
+def nq_lowrank_linear_bwd_scales(x_ptr, dy_ptr, Upk_ptr, Vpk_ptr, UpkT_ptr, VpkT_ptr, s1_ptr, s2_ptr, m, n, r, batch,
+                                 ds1_ptr, ds2_ptr, stream=0) -> int:
+    return _lib.nq_lowrank_linear_bwd_scales(x_ptr, dy_ptr, Upk_ptr, Vpk_ptr, UpkT_ptr, VpkT_ptr, s1_ptr, s2_ptr, m, n,
+                                             r, batch, ds1_ptr, ds2_ptr, stream)
 
 
 def nq_lowrank_linear_fwd(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n, r, batch, y_ptr, stream=0) -> int:
@@ -264,6 +271,20 @@ def lowrank_linear_bwd_input(dy, UpkT, VpkT, s1, s2, m: int, n: int, r: int, dx=
                                           _ptr(dx), _stream(stream, dy, UpkT, dx))
     _check(st, "nq_lowrank_linear_bwd_input")
     return dx
+
+
+def lowrank_linear_bwd_scales(x, dy, Upk, Vpk, UpkT, VpkT, s1, s2, m: int, n: int, r: int, stream=None):
+    """(ds1 (m,), ds2 (n,)) float32 device tensors: the gradients with respect to s1 and s2
+    for input x (batch x n bf16) and output gradient dy (batch x m bf16), all on the device."""
+    import torch
+
+    batch = x.shape[0] if x.dim() == 2 else 1
+    ds1 = torch.empty((m,), dtype=torch.float32, device=x.device)
+    ds2 = torch.empty((n,), dtype=torch.float32, device=x.device)
+    st = _lib.nq_lowrank_linear_bwd_scales(_ptr(x), _ptr(dy), _ptr(Upk), _ptr(Vpk), _ptr(UpkT), _ptr(VpkT), _ptr(s1),
+                                           _ptr(s2), m, n, r, batch, _ptr(ds1), _ptr(ds2), _stream(stream, x, dy))
+    _check(st, "nq_lowrank_linear_bwd_scales")
+    return ds1, ds2
 
 
 def lowrank_linear_fwd(x, Upk, Vpk, s1, s2, m: int, n: int, r: int, y=None, stream=None):

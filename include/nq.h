@@ -140,6 +140,30 @@ int nq_lowrank_linear_bwd_input(const void* dy, const uint32_t* UpkT, const uint
                                 const void* s2, int64_t m, int64_t n, int64_t r, int64_t batch, float* dx,
                                 void* stream);
 
+/*
+ * nq_lowrank_linear_bwd_scales -- the gradients with respect to the two scale vectors,
+ * for `batch` tokens of input x and output gradient dy (the refinement step tunes the
+ * scales with the factors, hardwired.dev "Krok 3"):
+ *     ds1_i = sum_b dy[b][i] * (U (V^T (s2 (.) x[b])))_i
+ *     ds2_j = sum_b x[b][j]  * (V (U^T (s1 (.) dy[b])))_j
+ *   x    : batch x n bfloat16;  dy : batch x m bfloat16
+ *   Upk, Vpk   : the forward packings;  UpkT, VpkT : their transposes (nq_transpose_signs)
+ *   s1 : m fp16;  s2 : n fp16
+ *   ds1 : m float32, ds2 : n float32 (written; either may be NULL to skip it)
+ * Every pointer in device memory, 16-byte aligned (else NQ_ERR_PTRKIND / NQ_ERR_ALIGN);
+ * shapes as nq_lowrank_linear_fwd; batch 0 writes zeros.  Each gradient is the layer
+ * evaluated without one scale (the forward pass, or the input gradient, with that scale
+ * set to 1, through the decode or prefill kernels) followed by a per-column dot product
+ * over the tokens in token order (deterministic).  Accuracy: each term carries the error
+ * of that evaluation, |error of ds1_i| <= 2e-3 * sum_b |dy[b][i]| * max_i' |z[b][i']|.
+ * Uses the workspace (not safe for concurrent calls on different streams); asynchronous
+ * on `stream`, except that the first call of a size allocates scratch.
+ */
+int nq_lowrank_linear_bwd_scales(const void* x, const void* dy, const uint32_t* Upk, const uint32_t* Vpk,
+                                 const uint32_t* UpkT, const uint32_t* VpkT, const void* s1, const void* s2,
+                                 int64_t m, int64_t n, int64_t r, int64_t batch, float* ds1, float* ds2,
+                                 void* stream);
+
 /* One factorised layer of a grouped call (same meaning and rules as the arguments of
  * nq_lowrank_linear_fwd; every pointer in device memory, 16-byte aligned). */
 typedef struct nq_linear_desc {

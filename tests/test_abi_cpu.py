@@ -135,6 +135,14 @@ def test_transpose_and_backward_argument_errors(nq):
     assert b(0, p[1], p[2], p[3], p[4], 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_NULL
     assert b(p[0] + 2, p[1], p[2], p[3], p[4], 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_ALIGN
     assert b(p[0], p[1], p[2], p[3], p[4], 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_PTRKIND
+    g = nq.nq_lowrank_linear_bwd_scales
+    q = [base + 1024 * i for i in range(10)]
+    assert g(*q[:8], 128, 128, 128, -1, q[8], q[9], 0) == nq.NQ_ERR_BATCH
+    assert g(*q[:8], 100, 128, 128, 1, q[8], q[9], 0) == nq.NQ_ERR_SHAPE
+    assert g(*q[:8], 128, 128, 128, 1, 0, 0, 0) == nq.NQ_OK  # nothing to compute
+    assert g(0, *q[1:8], 128, 128, 128, 1, q[8], q[9], 0) == nq.NQ_ERR_NULL
+    assert g(*q[:7], q[7] + 4, 128, 128, 128, 1, q[8], q[9], 0) == nq.NQ_ERR_ALIGN
+    assert g(*q[:8], 128, 128, 128, 1, q[8], q[9], 0) == nq.NQ_ERR_PTRKIND
 
 
 def test_grouped_argument_errors(nq):

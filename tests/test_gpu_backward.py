@@ -1,5 +1,6 @@
-"""The input gradient of the layer (dx = s2 * V U^T (s1 * dy)) and the packed-sign
-transpose on the GPU, through the C ABI, against the CPU oracle.
+"""The backward of the layer on the GPU, through the C ABI, against the CPU oracle: the
+input gradient (dx = s2 * V U^T (s1 * dy)), the packed-sign transpose it needs, and the
+gradients with respect to the scale vectors.
 
 Bar: the transpose bit-exact; dx within max|dx - dx_ref| / max|dx_ref| <= 2e-3, the bar of
 the forward pass it is computed with (the same kernels with the factors' roles exchanged).
@@ -129,3 +130,58 @@ def test_bwd_input_host_buffers(nq, orc):
     dx = nq.lowrank_linear_bwd_input(dy_h, layer.UpkT, layer.VpkT, layer.s1_d, layer.s2_d, m, n, r)
     assert not dx.is_cuda
     assert rel_err(dx.numpy(), layer.oracle_bwd(orc, dy)) <= TOL
+
+
+ONE_F16 = 0x3C00
+
+
+@pytest.mark.parametrize("m,n,r,batch", [
+    (512, 512, 128, 1),
+    (384, 640, 256, 5),       # decode path, two token groups
+    (1152, 384, 1664, 8),
+    (640, 384, 256, 40),      # prefill path
+    (11008, 4096, 2432, 3),   # the 7B gate projection's shape
+])
+def test_bwd_scales_match_oracle(nq, orc, m, n, r, batch):
+    """ds1 and ds2 against the oracle, within the bound that the accuracy of the layer
+    evaluations they are made of gives: |ds1_i - ref| <= 2e-3 sum_b |dy_bi| max|z_b|."""
+    layer = Layer(orc, nq, m, n, r, seed=500 + m + batch)
+    x = synth.activations_bf16(batch, n, 501 + batch)
+    dy = synth.activations_bf16(batch, m, 502 + batch, "dy")
+    x_d = torch.from_numpy(x.view(np.int16)).cuda()
+    dy_d = torch.from_numpy(dy.view(np.int16)).cuda()
+    ds1, ds2 = nq.lowrank_linear_bwd_scales(x_d, dy_d, layer.Upk, layer.Vpk, layer.UpkT, layer.VpkT,
+                                            layer.s1_d, layer.s2_d, m, n, r)
+    torch.cuda.synchronize()
+    ref1, ref2 = orc.lowrank_linear_bwd_scales(x, dy, layer.Upk_o, layer.Vpk_o, layer.s1, layer.s2, m, n, r)
+    ones_m = np.full(m, ONE_F16, dtype=np.uint16)
+    ones_n = np.full(n, ONE_F16, dtype=np.uint16)
+    z = orc.lowrank_linear_fwd(x, layer.Upk_o, layer.Vpk_o, ones_m, layer.s2, m, n, r)
+    w = orc.lowrank_linear_bwd_input(dy, layer.Upk_o, layer.Vpk_o, layer.s1, ones_n, m, n, r)
+    dyf = np.abs(synth.bf16_bits_to_f32(dy).astype(np.float64))
+    xf = np.abs(synth.bf16_bits_to_f32(x).astype(np.float64))
+    bound1 = TOL * np.sum(dyf * np.max(np.abs(z), axis=1, keepdims=True), axis=0) + 1e-12
+    bound2 = TOL * np.sum(xf * np.max(np.abs(w), axis=1, keepdims=True), axis=0) + 1e-12
+    assert np.all(np.abs(ds1.cpu().numpy() - ref1) <= bound1)
+    assert np.all(np.abs(ds2.cpu().numpy() - ref2) <= bound2)
+
+
+def test_bwd_scales_deterministic_and_skippable(nq, orc):
+    m, n, r, batch = 512, 768, 256, 4
+    layer = Layer(orc, nq, m, n, r, seed=520)
+    x_d = torch.from_numpy(synth.activations_bf16(batch, n, 521).view(np.int16)).cuda()
+    dy_d = torch.from_numpy(synth.activations_bf16(batch, m, 522, "dy").view(np.int16)).cuda()
+    a1, a2 = nq.lowrank_linear_bwd_scales(x_d, dy_d, layer.Upk, layer.Vpk, layer.UpkT, layer.VpkT,
+                                          layer.s1_d, layer.s2_d, m, n, r)
+    b1, b2 = nq.lowrank_linear_bwd_scales(x_d, dy_d, layer.Upk, layer.Vpk, layer.UpkT, layer.VpkT,
+                                          layer.s1_d, layer.s2_d, m, n, r)
+    torch.cuda.synchronize()
+    assert torch.equal(a1, b1) and torch.equal(a2, b2)
+    # ds2 alone (ds1 NULL) gives the same ds2
+    only2 = torch.empty((n,), dtype=torch.float32, device="cuda")
+    st = nq.nq_lowrank_linear_bwd_scales(x_d.data_ptr(), dy_d.data_ptr(), layer.Upk.data_ptr(), layer.Vpk.data_ptr(),
+                                         layer.UpkT.data_ptr(), layer.VpkT.data_ptr(), layer.s1_d.data_ptr(),
+                                         layer.s2_d.data_ptr(), m, n, r, batch, 0, only2.data_ptr(),
+                                         torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert st == nq.NQ_OK and torch.equal(only2, a2)
