@@ -49,6 +49,7 @@ def _load(path: str) -> ctypes.CDLL:
     L.orc_lowrank_linear_bwd_input.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p]
     L.orc_transpose_signs.argtypes = [p, i64, i64, p]
     L.orc_lowrank_linear_bwd_scales.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p, p]
+    L.orc_lowrank_linear_bwd_factors.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p, p]
     L.orc_bits_per_weight.argtypes = [i64, i64, i64]
     L.orc_bits_per_weight.restype = ctypes.c_double
     L.orc_bf16_to_double.argtypes = [ctypes.c_uint16]
@@ -140,6 +141,25 @@ class Oracle:
         if st != ORC_OK:
             raise ValueError(f"orc_lowrank_linear_bwd_scales failed with status {st}")
         return ds1, ds2
+
+    def lowrank_linear_bwd_factors(self, x_bits, dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r):
+        """(dU (m x r), dV (n x r)) float64: the straight-through gradients of the factors,
+        dU = diag(s1) dy^T t and dV = diag(s2) x^T u with t = V^T (s2 * x), u = U^T (s1 * dy)."""
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1, n)
+        dy = np.ascontiguousarray(dy_bits, dtype=np.uint16).reshape(-1, m)
+        assert x.shape[0] == dy.shape[0]
+        U = np.ascontiguousarray(Upk, dtype=np.uint32)
+        V = np.ascontiguousarray(Vpk, dtype=np.uint32)
+        a = np.ascontiguousarray(s1_bits, dtype=np.uint16)
+        b = np.ascontiguousarray(s2_bits, dtype=np.uint16)
+        assert U.shape == (m, words_per_row(r)) and V.shape == (r, words_per_row(n))
+        dU = np.zeros((m, r), dtype=np.float64)
+        dV = np.zeros((n, r), dtype=np.float64)
+        st = self.lib.orc_lowrank_linear_bwd_factors(
+            _ptr(x), _ptr(dy), _ptr(U), _ptr(V), _ptr(a), _ptr(b), m, n, r, x.shape[0], _ptr(dU), _ptr(dV))
+        if st != ORC_OK:
+            raise ValueError(f"orc_lowrank_linear_bwd_factors failed with status {st}")
+        return dU, dV
 
     def transpose_signs(self, packed: np.ndarray, rows: int, cols: int) -> np.ndarray:
         """rows x ceil(cols/32) packed words -> cols x ceil(rows/32) words of the transpose."""
@@ -303,3 +323,7 @@ def transpose_signs(packed, rows, cols):
 
 def lowrank_linear_bwd_scales(x_bits, dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r):
     return default().lowrank_linear_bwd_scales(x_bits, dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r)
+
+
+def lowrank_linear_bwd_factors(x_bits, dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r):
+    return default().lowrank_linear_bwd_factors(x_bits, dy_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r)

@@ -230,6 +230,24 @@ int orc_lowrank_linear_bwd_input(const uint16_t *dy, const uint32_t *Upk, const 
     return ORC_OK;
 }
 
+/* The two rank-r vectors of the backward pass, per token: t = V^T (s2 (.) x) and
+ * u = U^T (s1 (.) dy) (batch x r doubles each), sums in increasing index. */
+static void orc_rank_vectors(const uint16_t *x, const uint16_t *dy, const uint32_t *Upk,
+                             const uint32_t *Vpk, const uint16_t *s1, const uint16_t *s2, int64_t m,
+                             int64_t n, int64_t r, int64_t batch, double *t, double *u) {
+    const int64_t wpr_u = words_per_row(r), wpr_v = words_per_row(n);
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t k = 0; k < r; ++k) {
+            double at = 0.0, au = 0.0;
+            for (int64_t j = 0; j < n; ++j)
+                at += orc_sign_at(Vpk, wpr_v, k, j) * (orc_f16_to_double(s2[j]) * orc_bf16_to_double(x[b * n + j]));
+            for (int64_t i = 0; i < m; ++i)
+                au += orc_sign_at(Upk, wpr_u, i, k) * (orc_f16_to_double(s1[i]) * orc_bf16_to_double(dy[b * m + i]));
+            t[b * r + k] = at;
+            u[b * r + k] = au;
+        }
+}
+
 /* ---- the scale gradients ----
  *
  * The refinement step tunes the scaling factors together with the binary factors
@@ -255,17 +273,7 @@ int orc_lowrank_linear_bwd_scales(const uint16_t *x, const uint16_t *dy, const u
     double *t = (double *)malloc(sizeof(double) * (size_t)(r * batch));
     double *u = (double *)malloc(sizeof(double) * (size_t)(r * batch));
     if (!t || !u) { free(t); free(u); return ORC_ERR_ARG; }
-    /* t = V^T (s2 (.) x) and u = U^T (s1 (.) dy), sums in increasing index */
-    for (int64_t b = 0; b < batch; ++b)
-        for (int64_t k = 0; k < r; ++k) {
-            double at = 0.0, au = 0.0;
-            for (int64_t j = 0; j < n; ++j)
-                at += orc_sign_at(Vpk, wpr_v, k, j) * (orc_f16_to_double(s2[j]) * orc_bf16_to_double(x[b * n + j]));
-            for (int64_t i = 0; i < m; ++i)
-                au += orc_sign_at(Upk, wpr_u, i, k) * (orc_f16_to_double(s1[i]) * orc_bf16_to_double(dy[b * m + i]));
-            t[b * r + k] = at;
-            u[b * r + k] = au;
-        }
+    orc_rank_vectors(x, dy, Upk, Vpk, s1, s2, m, n, r, batch, t, u);
     /* ds1_i = sum_b dy_bi * (U t_b)_i ;  ds2_j = sum_b x_bj * (V u_b)_j */
     for (int64_t i = 0; i < m; ++i)
         for (int64_t b = 0; b < batch; ++b) {
@@ -279,6 +287,53 @@ int orc_lowrank_linear_bwd_scales(const uint16_t *x, const uint16_t *dy, const u
             for (int64_t k = 0; k < r; ++k) w += orc_sign_at(Vpk, wpr_v, k, j) * u[b * r + k];
             ds2[j] += orc_bf16_to_double(x[b * n + j]) * w;
         }
+    free(t);
+    free(u);
+    return ORC_OK;
+}
+
+/* ---- the gradients of the factors ----
+ *
+ * The straight-through estimator of the refinement step (hardwired.dev, section "Krok 3")
+ * passes the gradient of the sign function as the identity, so the gradient with respect
+ * to the latent factors is the gradient with respect to the +1/-1 factors themselves:
+ *     dU[i][k] = s1_i * sum_b dy[b][i] * t[b][k],   t = V^T (s2 (.) x)
+ *     dV[j][k] = s2_j * sum_b x[b][j]  * u[b][k],   u = U^T (s1 (.) dy)
+ * x: batch x n, dy: batch x m bfloat16 bit patterns; Upk, Vpk, s1, s2 as in the forward
+ * pass; dU (m x r) and dV (n x r) doubles, row-major (written).  Sums over b in increasing b.
+ */
+int orc_lowrank_linear_bwd_factors(const uint16_t *x, const uint16_t *dy, const uint32_t *Upk,
+                                   const uint32_t *Vpk, const uint16_t *s1, const uint16_t *s2,
+                                   int64_t m, int64_t n, int64_t r, int64_t batch, double *dU,
+                                   double *dV) {
+    if (m <= 0 || n <= 0 || r <= 0 || batch < 0) return ORC_ERR_ARG;
+    if (!dU || !dV) return ORC_ERR_ARG;
+    for (int64_t q = 0; q < m * r; ++q) dU[q] = 0.0;
+    for (int64_t q = 0; q < n * r; ++q) dV[q] = 0.0;
+    if (batch == 0) return ORC_OK;
+    if (!x || !dy || !Upk || !Vpk || !s1 || !s2) return ORC_ERR_ARG;
+    double *t = (double *)malloc(sizeof(double) * (size_t)(r * batch));
+    double *u = (double *)malloc(sizeof(double) * (size_t)(r * batch));
+    if (!t || !u) { free(t); free(u); return ORC_ERR_ARG; }
+    orc_rank_vectors(x, dy, Upk, Vpk, s1, s2, m, n, r, batch, t, u);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < m; ++i) {
+        const double si = orc_f16_to_double(s1[i]);
+        for (int64_t k = 0; k < r; ++k) {
+            double acc = 0.0;
+            for (int64_t b = 0; b < batch; ++b) acc += orc_bf16_to_double(dy[b * m + i]) * t[b * r + k];
+            dU[i * r + k] = si * acc;
+        }
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < n; ++j) {
+        const double s2j = orc_f16_to_double(s2[j]);
+        for (int64_t k = 0; k < r; ++k) {
+            double acc = 0.0;
+            for (int64_t b = 0; b < batch; ++b) acc += orc_bf16_to_double(x[b * n + j]) * u[b * r + k];
+            dV[j * r + k] = s2j * acc;
+        }
+    }
     free(t);
     free(u);
     return ORC_OK;

@@ -438,6 +438,51 @@ def pin_bwd_scales_dense(o):
         assert rel_err(ds2, np.sum(xf * w, axis=0)) <= 1e-12
 
 
+def pin_bwd_factors_sign_flip(o):
+    """L = sum(dy * y) is linear in every entry of U (and of V), so negating U[i][k] changes
+    L by -2 U[i][k] dU[i][k]: dU[i][k] = (L(U) - L(U with entry (i, k) negated)) / (2 U[i][k]),
+    L from the forward oracle; likewise dV."""
+    m, n, r, batch = 10, 14, 6, 3
+    x, U, V, s1, s2 = _case(m, n, r, batch, 91)
+    dy = synth.activations_bf16(batch, m, 91, "dy")
+    dyf = synth.bf16_bits_to_f32(dy).astype(np.float64)
+    dU, dV = o.lowrank_linear_bwd_factors(x, dy, o.pack_signs(U), o.pack_signs(np.ascontiguousarray(V.T)), s1, s2,
+                                          m, n, r)
+    assert dU.shape == (m, r) and dV.shape == (n, r)
+
+    def loss(Ux, Vx):
+        return float(np.sum(dyf * _fwd(o, x, Ux, Vx, s1, s2)))
+
+    L0 = loss(U, V)
+    for (i, k) in ((0, 0), (4, 3), (m - 1, r - 1)):
+        U2 = U.copy()
+        U2[i, k] *= -1
+        fd = (L0 - loss(U2, V)) / (2.0 * U[i, k])
+        assert abs(fd - dU[i, k]) <= 1e-11 * max(1.0, abs(fd)), (i, k, fd, dU[i, k])
+    for (j, k) in ((0, 1), (7, 5), (n - 1, 0)):
+        V2 = V.copy()
+        V2[j, k] *= -1
+        fd = (L0 - loss(U, V2)) / (2.0 * V[j, k])
+        assert abs(fd - dV[j, k]) <= 1e-11 * max(1.0, abs(fd)), (j, k, fd, dV[j, k])
+
+
+def pin_bwd_factors_dense(o):
+    """dU = diag(s1) dy^T (x diag(s2) V) and dV = diag(s2) x^T (dy diag(s1) U), numpy fp64."""
+    m, n, r, batch = 24, 18, 7, 4
+    x, U, V, s1, s2 = _case(m, n, r, batch, 92)
+    dy = synth.activations_bf16(batch, m, 92, "dy")
+    dU, dV = o.lowrank_linear_bwd_factors(x, dy, o.pack_signs(U), o.pack_signs(np.ascontiguousarray(V.T)), s1, s2,
+                                          m, n, r)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    dyf = synth.bf16_bits_to_f32(dy).astype(np.float64)
+    s1f = synth.f16_bits_to_f32(s1).astype(np.float64)
+    s2f = synth.f16_bits_to_f32(s2).astype(np.float64)
+    t = (xf * s2f[None, :]) @ V.astype(np.float64)   # batch x r
+    u = (dyf * s1f[None, :]) @ U.astype(np.float64)  # batch x r
+    assert rel_err(dU, s1f[:, None] * (dyf.T @ t)) <= 1e-12
+    assert rel_err(dV, s2f[:, None] * (xf.T @ u)) <= 1e-12
+
+
 def pin_transpose_signs(o):
     """The packed transpose is numpy's transpose of the unpacked signs (ragged shapes
     included), and transposing twice gives the original words back."""
@@ -474,4 +519,6 @@ ALL_PINS = [
     pin_transpose_signs,
     pin_bwd_scales_linear_in_scale,
     pin_bwd_scales_dense,
+    pin_bwd_factors_sign_flip,
+    pin_bwd_factors_dense,
 ]

@@ -47,6 +47,9 @@ MUTANTS = {
                           "for (int64_t k = 0; k < r; ++k) w += orc_sign_at(Vpk, wpr_v, k, j) * t[b * r + k];"),
     "scales_u_no_s1": ("au += orc_sign_at(Upk, wpr_u, i, k) * (orc_f16_to_double(s1[i]) * orc_bf16_to_double(dy[b * m + i]));",
                        "au += orc_sign_at(Upk, wpr_u, i, k) * orc_bf16_to_double(dy[b * m + i]);"),
+    "factors_dU_no_s1": ("dU[i * r + k] = si * acc;", "dU[i * r + k] = acc;"),
+    "factors_dV_uses_t": ("for (int64_t b = 0; b < batch; ++b) acc += orc_bf16_to_double(x[b * n + j]) * u[b * r + k];",
+                          "for (int64_t b = 0; b < batch; ++b) acc += orc_bf16_to_double(x[b * n + j]) * t[b * r + k];"),
     "transpose_msb": ("out[j * wpr_out + i / 32] |= 1u << (i % 32);", "out[j * wpr_out + i / 32] |= 1u << (31 - i % 32);"),
 }
 
