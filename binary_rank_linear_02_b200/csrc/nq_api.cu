@@ -508,6 +508,53 @@ int nq_lowrank_linear_bwd_scales(const void* x, const void* dy, const uint32_t* 
     return NQ_OK;
 }
 
+int nq_lowrank_linear_bwd_factors(const void* x, const void* dy, const uint32_t* Vpk, const uint32_t* UpkT,
+                                  const void* s1, const void* s2, int64_t m, int64_t n, int64_t r, int64_t batch,
+                                  float* dU, float* dV, void* stream) {
+    if (batch < 0) return NQ_ERR_BATCH;
+    if (m <= 0 || n <= 0 || r <= 0 || m % 128 || n % 128 || r % 128 || m > kMaxDim || n > kMaxDim ||
+        r > kMaxRank)
+        return NQ_ERR_SHAPE;
+    if (batch > (int64_t(1) << 40) / (m > n ? m : n) || (m > n ? m : n) > (int64_t(1) << 40) / r) return NQ_ERR_SHAPE;
+    if (!dU && !dV) return NQ_OK;
+    if (!x || !dy || !Vpk || !UpkT || !s1 || !s2) return NQ_ERR_NULL;
+    const void* ptrs[] = {x, dy, Vpk, UpkT, s1, s2, dU, dV};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return NQ_ERR_ALIGN;
+    for (const void* p : ptrs)
+        if (p && !pointer_kind(p)) return NQ_ERR_PTRKIND;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (batch == 0) {  // empty sums
+        if (dU && cudaMemsetAsync(dU, 0, sizeof(float) * (size_t)(m * r), s) != cudaSuccess) return NQ_ERR_CUDA;
+        if (dV && cudaMemsetAsync(dV, 0, sizeof(float) * (size_t)(n * r), s) != cudaSuccess) return NQ_ERR_CUDA;
+        return NQ_OK;
+    }
+    int st = NQ_OK;
+    const int64_t w = m > n ? m : n, bc = batch < NQ_DECODE_MAX_BATCH ? batch : NQ_DECODE_MAX_BATCH;
+    const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 128, w, r};
+    Workspace* ws = workspace_for(128, w, r, bc, decode_need(&c, 1, bc), &st);
+    if (!ws) return st;
+    st = ensure_grad_scratch(ws, 0, sizeof(float) * 2 * (size_t)batch * (size_t)r, s);
+    if (st != NQ_OK) return st;
+    float* t = ws->gstage;                       // batch x r: V^T (s2 (.) x)
+    float* u = ws->gstage + (size_t)batch * r;   // batch x r: U^T (s1 (.) dy)
+    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    const uint16_t* dyb = static_cast<const uint16_t*>(dy);
+    const uint16_t* s1b = static_cast<const uint16_t*>(s1);
+    const uint16_t* s2b = static_cast<const uint16_t*>(s2);
+    if (dU) {
+        st = decode_rank_vector(xb, Vpk, s2b, n, r, batch, t, ws, s);
+        if (st == NQ_OK) st = outer_device(dyb, s1b, t, batch, m, r, dU, s);
+        if (st != NQ_OK) return st;
+    }
+    if (dV) {
+        st = decode_rank_vector(dyb, UpkT, s1b, m, r, batch, u, ws, s);
+        if (st == NQ_OK) st = outer_device(xb, s2b, u, batch, n, r, dV, s);
+        if (st != NQ_OK) return st;
+    }
+    return NQ_OK;
+}
+
 int nq_cast_f32_to_bf16(const float* src, int64_t count, void* dst, void* stream) {
     if (count < 0 || count > kMaxElems) return NQ_ERR_SHAPE;
     if (count == 0) return NQ_OK;

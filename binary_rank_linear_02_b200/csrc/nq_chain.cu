@@ -16,6 +16,7 @@
 // Also here: the gather of pinned host inputs, and the per-column dot products over the
 // tokens that finish the scale gradients of the backward pass.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "nq_internal.cuh"
 
@@ -131,6 +132,55 @@ __global__ void fill_u16_kernel(uint16_t* p, int64_t count, uint16_t value) {
         p[i] = value;
 }
 
+// The straight-through gradients of the factors: out[i][k] = s[i] * sum_b a[b][i] * t[b][k]
+// (a bf16 batch x M, t fp32 batch x R).  A 16 x 16 thread block computes a 64 x 64 tile,
+// four by four outputs per thread, staging 32 tokens of a and t at a time in shared
+// memory; the tokens are added in order (deterministic).
+constexpr int kOuterTile = 64, kOuterTokens = 32;
+
+__global__ void __launch_bounds__(256) outer_kernel(const uint16_t* __restrict__ a, const uint16_t* __restrict__ s,
+                                                    const float* __restrict__ t, int64_t batch, int64_t M, int64_t R,
+                                                    float* __restrict__ out) {
+    __shared__ float as[kOuterTokens][kOuterTile];
+    __shared__ float ts[kOuterTokens][kOuterTile];
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const int64_t i0 = (int64_t)blockIdx.y * kOuterTile, k0 = (int64_t)blockIdx.x * kOuterTile;
+    float acc[4][4] = {};
+    for (int64_t b0 = 0; b0 < batch; b0 += kOuterTokens) {
+        for (int e = threadIdx.x; e < kOuterTokens * kOuterTile; e += 256) {
+            const int bb = e / kOuterTile, c = e % kOuterTile;
+            const int64_t b = b0 + bb;
+            as[bb][c] = (b < batch && i0 + c < M) ? __uint_as_float((uint32_t)a[b * M + i0 + c] << 16) : 0.f;
+            ts[bb][c] = (b < batch && k0 + c < R) ? t[b * R + k0 + c] : 0.f;
+        }
+        __syncthreads();
+        for (int bb = 0; bb < kOuterTokens; ++bb) {
+            float av[4], tv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                av[q] = as[bb][ty + 16 * q];
+                tv[q] = ts[bb][tx + 16 * q];
+            }
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(av[p], tv[q], acc[p][q]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int64_t i = i0 + ty + 16 * p;
+        if (i >= M) continue;
+        const float si = __half2float(__ushort_as_half(s[i]));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int64_t k = k0 + tx + 16 * q;
+            if (k < R) out[i * R + k] = si * acc[p][q];
+        }
+    }
+}
+
 }  // namespace
 
 int gather_device(const GatherList& list, cudaStream_t stream) {
@@ -175,6 +225,13 @@ int fill_u16_device(uint16_t* p, int64_t count, uint16_t value, cudaStream_t str
     if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
     if (blocks < 1) blocks = 1;
     fill_u16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(p, count, value);
+    return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
+}
+
+int outer_device(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch, int64_t M, int64_t R,
+                 float* out, cudaStream_t stream) {
+    const dim3 grid((unsigned)((R + kOuterTile - 1) / kOuterTile), (unsigned)((M + kOuterTile - 1) / kOuterTile));
+    outer_kernel<<<grid, 256, 0, stream>>>(a, s, t, batch, M, R, out);
     return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
 }
 

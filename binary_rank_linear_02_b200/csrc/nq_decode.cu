@@ -749,7 +749,7 @@ static bool set_kernel_attributes(K kernel) {
 }
 
 template <int NTG>
-int launch_group(DecGroup& grp, cudaStream_t stream, int device) {
+int launch_group(DecGroup& grp, cudaStream_t stream, int device, bool stage1_only) {
     static unsigned long long init_mask = 0;  // devices whose kernel attributes are set
     const unsigned long long bit = 1ull << (device & 63);
     if (!(__atomic_load_n(&init_mask, __ATOMIC_ACQUIRE) & bit)) {
@@ -777,6 +777,7 @@ int launch_group(DecGroup& grp, cudaStream_t stream, int device) {
         err = launch_pdl(stage1_kernel<NTG, 2>, dim3(grid1), dim3(s1_threads<2>()), smem1, stream, grp);
     }
     if (err != cudaSuccess) return NQ_ERR_CUDA;
+    if (stage1_only) return NQ_OK;
     if (launch_pdl(stage2_kernel<NTG>, dim3((unsigned)grp.s2_start[grp.count]), dim3(kThreads), smem2, stream, grp) !=
         cudaSuccess)
         return NQ_ERR_CUDA;
@@ -901,7 +902,7 @@ void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, in
 }
 
 int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Workspace* ws, cudaStream_t stream,
-                         int max_splits) {
+                         int max_splits, bool stage1_only) {
     if (count < 1 || count > kMaxGroup) return NQ_ERR_SHAPE;
     int64_t need_t, need_g, need_p, need_c;
     decode_workspace_need(calls, count, batch, max_splits, &need_t, &need_g, &need_p, &need_c);
@@ -977,8 +978,8 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
         grp.s1_start[k + 1] = grp.s1_start[k] + (L1.r / kRowsS1) * L1.nsplit;
         grp.s2_start[k + 1] = grp.s2_start[k] + L2.s2_ctas;
     }
-    if (batch <= 4) return launch_group<1>(grp, stream, ws->device);
-    return launch_group<2>(grp, stream, ws->device);
+    if (batch <= 4) return launch_group<1>(grp, stream, ws->device, stage1_only);
+    return launch_group<2>(grp, stream, ws->device, stage1_only);
 }
 
 int decode_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const uint16_t* s1,
@@ -986,6 +987,21 @@ int decode_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, 
                    Workspace* ws, cudaStream_t stream) {
     DecodeCall c{x, Upk, Vpk, s1, s2, y, m, n, r};
     return decode_forward_group(&c, 1, batch, ws, stream, kDecodeMaxSplits);
+}
+
+int decode_rank_vector(const uint16_t* x, const uint32_t* Vpk, const uint16_t* s2, int64_t n, int64_t r,
+                       int64_t batch, float* t, Workspace* ws, cudaStream_t stream) {
+    for (int64_t b0 = 0; b0 < batch; b0 += NQ_DECODE_MAX_BATCH) {
+        const int64_t bc = batch - b0 < NQ_DECODE_MAX_BATCH ? batch - b0 : NQ_DECODE_MAX_BATCH;
+        // stage 1 alone writes t of the only layer at the start of the workspace's t
+        const DecodeCall c{x + b0 * n, nullptr, Vpk, nullptr, s2, nullptr, kRowsS1, n, r};
+        int st = decode_forward_group(&c, 1, bc, ws, stream, kDecodeMaxSplits, true);
+        if (st != NQ_OK) return st;
+        if (cudaMemcpyAsync(t + b0 * r, ws->t, sizeof(float) * (size_t)(bc * r), cudaMemcpyDeviceToDevice, stream) !=
+            cudaSuccess)
+            return NQ_ERR_CUDA;
+    }
+    return NQ_OK;
 }
 
 }  // namespace nq

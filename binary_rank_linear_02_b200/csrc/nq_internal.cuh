@@ -88,7 +88,14 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 
 // ---------------------------------------------------------------- entry points of the kernels
 int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Workspace* ws, cudaStream_t stream,
-                         int max_splits = kDecodeMaxSplits);
+                         int max_splits = kDecodeMaxSplits, bool stage1_only = false);
+// t = V^T (s2 (.) x) alone (batch x r fp32, any batch: the decode stage-1 kernel, up to
+// NQ_DECODE_MAX_BATCH tokens per launch, each launch's t copied out of the workspace).
+int decode_rank_vector(const uint16_t* x, const uint32_t* Vpk, const uint16_t* s2, int64_t n, int64_t r,
+                       int64_t batch, float* t, Workspace* ws, cudaStream_t stream);
+// out[i][k] = s[i] * sum over b (increasing) of bf16(a[b][i]) * t[b][k]: M x R fp32
+int outer_device(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch, int64_t M, int64_t R,
+                 float* out, cudaStream_t stream);
 void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, int max_splits, int64_t* t_floats,
                            int64_t* tgmax_floats, int64_t* partial_floats, int64_t* counter_ints);
 

@@ -69,6 +69,7 @@ def _load() -> ctypes.CDLL:
     L.nq_transpose_signs.argtypes = [p, i64, i64, p, p]
     L.nq_lowrank_linear_bwd_input.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p]
     L.nq_lowrank_linear_bwd_scales.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p]
+    L.nq_lowrank_linear_bwd_factors.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p, p, p]
     L.nq_unpack_signs.restype = ctypes.c_int
     L.nq_lowrank_linear_fwd.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p]
     L.nq_lowrank_linear_fwd.restype = ctypes.c_int
@@ -125,6 +126,12 @@ def nq_lowrank_linear_bwd_scales(x_ptr, dy_ptr, Upk_ptr, Vpk_ptr, UpkT_ptr, VpkT
                                  ds1_ptr, ds2_ptr, stream=0) -> int:
     return _lib.nq_lowrank_linear_bwd_scales(x_ptr, dy_ptr, Upk_ptr, Vpk_ptr, UpkT_ptr, VpkT_ptr, s1_ptr, s2_ptr, m, n,
                                              r, batch, ds1_ptr, ds2_ptr, stream)
+
+
+def nq_lowrank_linear_bwd_factors(x_ptr, dy_ptr, Vpk_ptr, UpkT_ptr, s1_ptr, s2_ptr, m, n, r, batch, dU_ptr, dV_ptr,
+                                  stream=0) -> int:
+    return _lib.nq_lowrank_linear_bwd_factors(x_ptr, dy_ptr, Vpk_ptr, UpkT_ptr, s1_ptr, s2_ptr, m, n, r, batch, dU_ptr,
+                                              dV_ptr, stream)
 
 
 def nq_lowrank_linear_fwd(x_ptr, Upk_ptr, Vpk_ptr, s1_ptr, s2_ptr, m, n, r, batch, y_ptr, stream=0) -> int:
@@ -285,6 +292,20 @@ def lowrank_linear_bwd_scales(x, dy, Upk, Vpk, UpkT, VpkT, s1, s2, m: int, n: in
                                            _ptr(s2), m, n, r, batch, _ptr(ds1), _ptr(ds2), _stream(stream, x, dy))
     _check(st, "nq_lowrank_linear_bwd_scales")
     return ds1, ds2
+
+
+def lowrank_linear_bwd_factors(x, dy, Vpk, UpkT, s1, s2, m: int, n: int, r: int, stream=None):
+    """(dU (m x r), dV (n x r)) float32 device tensors: the straight-through gradients of the
+    factors for input x (batch x n bf16) and output gradient dy (batch x m bf16)."""
+    import torch
+
+    batch = x.shape[0] if x.dim() == 2 else 1
+    dU = torch.empty((m, r), dtype=torch.float32, device=x.device)
+    dV = torch.empty((n, r), dtype=torch.float32, device=x.device)
+    st = _lib.nq_lowrank_linear_bwd_factors(_ptr(x), _ptr(dy), _ptr(Vpk), _ptr(UpkT), _ptr(s1), _ptr(s2), m, n, r, batch,
+                                            _ptr(dU), _ptr(dV), _stream(stream, x, dy))
+    _check(st, "nq_lowrank_linear_bwd_factors")
+    return dU, dV
 
 
 def lowrank_linear_fwd(x, Upk, Vpk, s1, s2, m: int, n: int, r: int, y=None, stream=None):

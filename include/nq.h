@@ -164,6 +164,26 @@ int nq_lowrank_linear_bwd_scales(const void* x, const void* dy, const uint32_t* 
                                  int64_t m, int64_t n, int64_t r, int64_t batch, float* ds1, float* ds2,
                                  void* stream);
 
+/*
+ * nq_lowrank_linear_bwd_factors -- the straight-through gradients of the two factors (the
+ * refinement step passes the gradient of the sign function as the identity, hardwired.dev
+ * "Krok 3", so these are the gradients with respect to the latent real-valued factors):
+ *     dU[i][k] = s1_i * sum_b dy[b][i] * t[b][k],   t = V^T (s2 (.) x)
+ *     dV[j][k] = s2_j * sum_b x[b][j]  * u[b][k],   u = U^T (s1 (.) dy)
+ *   x  : batch x n bfloat16;  dy : batch x m bfloat16
+ *   Vpk : r x (n/32) (the forward packing of V^T);  UpkT : r x (m/32) (transpose of Upk)
+ *   s1 : m fp16;  s2 : n fp16
+ *   dU : m x r float32, dV : n x r float32, row-major (written; either may be NULL)
+ * Every pointer in device memory, 16-byte aligned; shapes as nq_lowrank_linear_fwd; batch 0
+ * writes zeros.  t and u come from the decode path's first stage (up to 8 tokens per launch,
+ * so cost grows with batch in steps of 8 tokens), the sums over the tokens from a tiled
+ * fp32 kernel in token order (deterministic).  Accuracy: |error of dU[i][k]| <=
+ * 2e-3 * |s1_i| * sum_b |dy[b][i]| * max_k' |t[b][k']| (likewise dV).  Uses the workspace.
+ */
+int nq_lowrank_linear_bwd_factors(const void* x, const void* dy, const uint32_t* Vpk, const uint32_t* UpkT,
+                                  const void* s1, const void* s2, int64_t m, int64_t n, int64_t r, int64_t batch,
+                                  float* dU, float* dV, void* stream);
+
 /* One factorised layer of a grouped call (same meaning and rules as the arguments of
  * nq_lowrank_linear_fwd; every pointer in device memory, 16-byte aligned). */
 typedef struct nq_linear_desc {

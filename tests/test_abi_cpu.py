@@ -143,6 +143,13 @@ def test_transpose_and_backward_argument_errors(nq):
     assert g(0, *q[1:8], 128, 128, 128, 1, q[8], q[9], 0) == nq.NQ_ERR_NULL
     assert g(*q[:7], q[7] + 4, 128, 128, 128, 1, q[8], q[9], 0) == nq.NQ_ERR_ALIGN
     assert g(*q[:8], 128, 128, 128, 1, q[8], q[9], 0) == nq.NQ_ERR_PTRKIND
+    f = nq.nq_lowrank_linear_bwd_factors
+    assert f(*q[:6], 128, 128, 128, -1, q[6], q[7], 0) == nq.NQ_ERR_BATCH
+    assert f(*q[:6], 128, 130, 128, 1, q[6], q[7], 0) == nq.NQ_ERR_SHAPE
+    assert f(*q[:6], 128, 128, 128, 1, 0, 0, 0) == nq.NQ_OK  # nothing to compute
+    assert f(*q[:5], 0, 128, 128, 128, 1, q[6], q[7], 0) == nq.NQ_ERR_NULL
+    assert f(*q[:6], 128, 128, 128, 1, q[6] + 8, q[7], 0) == nq.NQ_ERR_ALIGN
+    assert f(*q[:6], 128, 128, 128, 1, q[6], q[7], 0) == nq.NQ_ERR_PTRKIND
 
 
 def test_grouped_argument_errors(nq):

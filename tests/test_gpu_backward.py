@@ -1,6 +1,6 @@
 """The backward of the layer on the GPU, through the C ABI, against the CPU oracle: the
-input gradient (dx = s2 * V U^T (s1 * dy)), the packed-sign transpose it needs, and the
-gradients with respect to the scale vectors.
+input gradient (dx = s2 * V U^T (s1 * dy)), the packed-sign transpose it needs, the
+gradients with respect to the scale vectors and the straight-through gradients of the factors.
 
 Bar: the transpose bit-exact; dx within max|dx - dx_ref| / max|dx_ref| <= 2e-3, the bar of
 the forward pass it is computed with (the same kernels with the factors' roles exchanged).
@@ -185,3 +185,34 @@ def test_bwd_scales_deterministic_and_skippable(nq, orc):
                                          torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     assert st == nq.NQ_OK and torch.equal(only2, a2)
+
+
+
+@pytest.mark.parametrize("m,n,r,batch", [
+    (512, 512, 128, 1),
+    (384, 640, 256, 3),
+    (640, 384, 256, 13),      # two launches of the first stage (8 + 5 tokens)
+    (1152, 384, 1664, 8),
+    (4096, 11008, 2432, 2),   # the 7B down projection's shape
+])
+def test_bwd_factors_match_oracle(nq, orc, m, n, r, batch):
+    """dU and dV against the oracle, within the bound that the accuracy of t and u gives:
+    |dU_ik - ref| <= 2e-3 |s1_i| sum_b |dy_bi| max|t_b| (likewise dV)."""
+    layer = Layer(orc, nq, m, n, r, seed=600 + m + batch)
+    x = synth.activations_bf16(batch, n, 601 + batch)
+    dy = synth.activations_bf16(batch, m, 602 + batch, "dy")
+    x_d = torch.from_numpy(x.view(np.int16)).cuda()
+    dy_d = torch.from_numpy(dy.view(np.int16)).cuda()
+    dU, dV = nq.lowrank_linear_bwd_factors(x_d, dy_d, layer.Vpk, layer.UpkT, layer.s1_d, layer.s2_d, m, n, r)
+    torch.cuda.synchronize()
+    rU, rV = orc.lowrank_linear_bwd_factors(x, dy, layer.Upk_o, layer.Vpk_o, layer.s1, layer.s2, m, n, r)
+    t = orc.stage1(x, layer.Vpk_o, layer.s2, n, r)
+    u = orc.stage1(dy, orc.transpose_signs(layer.Upk_o, m, r), layer.s1, m, r)
+    dyf = np.abs(synth.bf16_bits_to_f32(dy).astype(np.float64))
+    xf = np.abs(synth.bf16_bits_to_f32(x).astype(np.float64))
+    s1f = np.abs(synth.f16_bits_to_f32(layer.s1).astype(np.float64))
+    s2f = np.abs(synth.f16_bits_to_f32(layer.s2).astype(np.float64))
+    bU = TOL * s1f * np.sum(dyf * np.max(np.abs(t), axis=1)[:, None], axis=0) + 1e-12
+    bV = TOL * s2f * np.sum(xf * np.max(np.abs(u), axis=1)[:, None], axis=0) + 1e-12
+    assert np.all(np.abs(dU.cpu().numpy() - rU) <= bU[:, None])
+    assert np.all(np.abs(dV.cpu().numpy() - rV) <= bV[:, None])
