@@ -20,6 +20,7 @@ constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1;  // one CTA per row
 std::mutex g_mutex;
 Workspace g_ws[kMaxDevices];
 int g_sm_count[kMaxDevices];
+uint64_t g_ws_generation = 1;  // bumped (under g_mutex) whenever a workspace buffer is replaced
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -121,6 +122,7 @@ Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, const D
     w.device = dev;
     w.bytes = off;
     w.base = base;
+    ++g_ws_generation;
     w.t = reinterpret_cast<float*>(base + o_t);
     w.tgmax = reinterpret_cast<float*>(base + o_tgmax);
     w.partials = reinterpret_cast<float*>(base + o_part);
@@ -164,6 +166,7 @@ static int ensure_staging(Workspace* w, size_t xbytes, size_t ybytes) {
         if (w->xstage) { cudaDeviceSynchronize(); cudaFree(w->xstage); w->xstage = nullptr; w->xstage_bytes = 0; }
         if (cudaMalloc(&w->xstage, xbytes) != cudaSuccess) { cudaGetLastError(); return NQ_ERR_NOMEM; }
         w->xstage_bytes = xbytes;
+        ++g_ws_generation;
     }
     if (ybytes > w->ystage_bytes) {
         if (w->ystage) { cudaDeviceSynchronize(); cudaFree(w->ystage); w->ystage = nullptr; w->ystage_bytes = 0; }
@@ -171,6 +174,7 @@ static int ensure_staging(Workspace* w, size_t xbytes, size_t ybytes) {
         if (cudaMalloc(&p, ybytes) != cudaSuccess) { cudaGetLastError(); return NQ_ERR_NOMEM; }
         w->ystage = static_cast<float*>(p);
         w->ystage_bytes = ybytes;
+        ++g_ws_generation;
     }
     return NQ_OK;
 }
@@ -186,6 +190,7 @@ static int ensure_grad_scratch(Workspace* w, size_t ones, size_t outs_bytes, cud
         w->ones = static_cast<uint16_t*>(p);
         if (fill_u16_device(w->ones, (int64_t)ones, 0x3C00, stream) != NQ_OK) return NQ_ERR_CUDA;  // fp16 1.0
         w->ones_count = ones;
+        ++g_ws_generation;
     }
     if (outs_bytes > w->gstage_bytes) {
         if (w->gstage) { cudaDeviceSynchronize(); cudaFree(w->gstage); w->gstage = nullptr; w->gstage_bytes = 0; }
@@ -193,8 +198,92 @@ static int ensure_grad_scratch(Workspace* w, size_t ones, size_t outs_bytes, cud
         if (cudaMalloc(&p, outs_bytes) != cudaSuccess) { cudaGetLastError(); return NQ_ERR_NOMEM; }
         w->gstage = static_cast<float*>(p);
         w->gstage_bytes = outs_bytes;
+        ++g_ws_generation;
     }
     return NQ_OK;
+}
+
+// ---------------------------------------------------------------- launch cache
+// A call with host x or y synchronises before it returns, so its kernels never overlap the
+// next call's, and the host cost of its launches (microseconds each) adds to its latency.
+// Such calls are replayed from an executable CUDA graph when the identical call (every
+// pointer, size and staging buffer alike, same workspace generation) was made before: its
+// first occurrence launches directly (and sizes the workspace, sets kernel attributes), the
+// second captures the same launches on a private stream into a graph that is kept, and later
+// ones launch that graph alone.  Workspace growth changes the generation, so a graph is
+// never replayed against freed scratch.  Calls on a stream that is itself being captured,
+// and calls with pageable host buffers (copies through the staging buffers), launch directly.
+constexpr size_t kGraphCacheEntries = 32;  // per device; least recently used out first
+
+struct GraphEntry {
+    std::vector<uint64_t> key;
+    cudaGraphExec_t exec = nullptr;  // nullptr: seen once, not captured yet
+    uint64_t stamp = 0;
+};
+struct GraphCache {
+    std::vector<GraphEntry> entries;
+    uint64_t clock = 0;
+    cudaStream_t capture = nullptr;  // private stream the launches are captured on
+};
+std::mutex g_graph_mutex;
+GraphCache* g_graphs[kMaxDevices];  // never freed: the driver releases the graphs at exit
+
+uint64_t ws_generation() {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    return g_ws_generation;
+}
+
+// Runs `launch` (which enqueues kernels on the stream it is given and nothing else) for the
+// call identified by `key` on stream s, through the cache as described above.
+template <typename Launch>
+int launch_cached(int dev, const std::vector<uint64_t>& key, cudaStream_t s, Launch&& launch) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (dev < 0 || dev >= kMaxDevices || cudaStreamIsCapturing(s, &cs) != cudaSuccess ||
+        cs != cudaStreamCaptureStatusNone) {
+        cudaGetLastError();
+        return launch(s);
+    }
+    std::lock_guard<std::mutex> lock(g_graph_mutex);
+    if (!g_graphs[dev]) g_graphs[dev] = new GraphCache();
+    GraphCache& c = *g_graphs[dev];
+    ++c.clock;
+    GraphEntry* e = nullptr;
+    for (GraphEntry& x : c.entries)
+        if (x.key == key) e = &x;
+    if (!e) {  // first occurrence: remember it, launch directly
+        if (c.entries.size() >= kGraphCacheEntries) {
+            auto old = std::min_element(c.entries.begin(), c.entries.end(),
+                                        [](const GraphEntry& a, const GraphEntry& b) { return a.stamp < b.stamp; });
+            if (old->exec) cudaGraphExecDestroy(old->exec);
+            c.entries.erase(old);
+        }
+        c.entries.push_back(GraphEntry{key, nullptr, c.clock});
+        return launch(s);
+    }
+    e->stamp = c.clock;
+    if (!e->exec) {  // second occurrence: capture
+        if (!c.capture && cudaStreamCreateWithFlags(&c.capture, cudaStreamNonBlocking) != cudaSuccess) {
+            cudaGetLastError();
+            c.capture = nullptr;
+            return launch(s);
+        }
+        if (cudaStreamBeginCapture(c.capture, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+            cudaGetLastError();
+            return launch(s);
+        }
+        const int st = launch(c.capture);
+        cudaGraph_t g = nullptr;
+        const cudaError_t end = cudaStreamEndCapture(c.capture, &g);
+        cudaGraphExec_t exec = nullptr;
+        const bool ok = st == NQ_OK && end == cudaSuccess && g && cudaGraphInstantiate(&exec, g, 0) == cudaSuccess;
+        if (g) cudaGraphDestroy(g);
+        if (!ok) {
+            cudaGetLastError();
+            return launch(s);
+        }
+        e->exec = exec;
+    }
+    return cudaGraphLaunch(e->exec, s) == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
 }
 
 }  // namespace nq
@@ -203,8 +292,10 @@ using namespace nq;
 
 // The grouped forward over `count` descriptors `stride` bytes apart; `ex` (may be NULL)
 // adds the optional bf16 outputs of nq_linear_desc_ex.  Without `ex`, a layer's x and y may
-// be host memory: they are staged through the workspace (one copy per buffer), the layers
-// run as usual, host y are copied back and the call synchronises the stream.
+// be host memory: pinned x are gathered into the workspace by one kernel, pinned y written
+// by the kernels through their device address, pageable x and y copied through the
+// workspace; then the call synchronises the stream.  The scratch of every launch is sized
+// before the first is enqueued, so that the launches can be captured (launch cache above).
 static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_linear_desc_ex* ex, int count,
                        int64_t batch, void* stream) {
     auto desc = [&](int i) -> const nq_linear_desc& {
@@ -256,48 +347,43 @@ static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_line
         }
     }
     const bool any_host = xbytes || std::find(y_host.begin(), y_host.end(), 1) != y_host.end();
+    bool pageable = ybytes > 0;
+    for (int i = 0; i < count; ++i) pageable = pageable || (x_host[i] && !x_pin[i]);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int st = NQ_OK;
+    // the scratch of every launch of the call, sized once before anything is enqueued
     DecodeNeed need;
-    if (batch > NQ_DECODE_MAX_BATCH) {
-        for (int i = 0; i < count; ++i) {
-            const nq_linear_desc& L = desc(i);
-            const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, L.m, L.n, L.r};
-            const DecodeNeed d = decode_need(&c, 1, batch);
-            need.partials = d.partials > need.partials ? d.partials : need.partials;
-            need.counters = d.counters > need.counters ? d.counters : need.counters;
+    for (int i0 = 0; i0 < count; i0 += (batch > NQ_DECODE_MAX_BATCH ? 1 : kMaxGroup)) {
+        const int cnt = batch > NQ_DECODE_MAX_BATCH ? 1 : (count - i0 < kMaxGroup ? count - i0 : kMaxGroup);
+        DecodeCall calls[kMaxGroup];
+        for (int i = 0; i < cnt; ++i) {
+            const nq_linear_desc& L = desc(i0 + i);
+            calls[i] = DecodeCall{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, L.m, L.n, L.r};
+            if (ex) calls[i].y_norm = static_cast<uint16_t*>(ex[i0 + i].y_rmsnorm_bf16);
         }
+        const DecodeNeed d = decode_need(calls, cnt, batch);
+        need.t = d.t > need.t ? d.t : need.t;
+        need.tgmax = d.tgmax > need.tgmax ? d.tgmax : need.tgmax;
+        need.partials = d.partials > need.partials ? d.partials : need.partials;
+        need.counters = d.counters > need.counters ? d.counters : need.counters;
     }
-    Workspace* ws = nullptr;
-    std::vector<const void*> xs(count);
-    std::vector<float*> ys(count);
+    Workspace* ws = workspace_for(m_max, n_max, r_max, batch, need, &st);
+    if (!ws) return st;
     if (xbytes || ybytes) {
-        ws = workspace_for(m_max, n_max, r_max, batch, need, &st);
-        if (!ws) return st;
         st = ensure_staging(ws, xbytes, ybytes);
         if (st != NQ_OK) return st;
     }
+    // where each layer reads x and writes y
+    std::vector<const void*> xs(count);
+    std::vector<float*> ys(count);
     size_t xo = 0, yo = 0;
-    GatherList gl;
-    gl.count = 0;
     for (int i = 0; i < count; ++i) {
         const nq_linear_desc& L = desc(i);
         xs[i] = L.x;
         ys[i] = L.y;
         if (x_host[i]) {
-            const size_t b = sizeof(uint16_t) * (size_t)batch * L.n;
-            char* dst = static_cast<char*>(ws->xstage) + xo;
-            if (x_pin[i]) {
-                gl.seg[gl.count++] = GatherSeg{x_pin[i], dst, b};
-                if (gl.count == kMaxGather) {
-                    if (gather_device(gl, s) != NQ_OK) return NQ_ERR_CUDA;
-                    gl.count = 0;
-                }
-            } else if (cudaMemcpyAsync(dst, L.x, b, cudaMemcpyHostToDevice, s) != cudaSuccess) {
-                return NQ_ERR_CUDA;
-            }
-            xs[i] = dst;
-            xo += align_up(b, 256);
+            xs[i] = static_cast<char*>(ws->xstage) + xo;
+            xo += align_up(sizeof(uint16_t) * (size_t)batch * L.n, 256);
         }
         if (y_host[i]) {
             if (y_pin[i]) {
@@ -308,38 +394,78 @@ static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_line
             }
         }
     }
-    if (gl.count > 0 && gather_device(gl, s) != NQ_OK) return NQ_ERR_CUDA;
-    if (batch > NQ_DECODE_MAX_BATCH) {
-        if (!ws) ws = workspace_for(m_max, n_max, r_max, batch, need, &st);
-        if (!ws) return st;
-        for (int i = 0; i < count && st == NQ_OK; ++i) {
+    // every launch of the call on stream q: x staging, then the layers
+    auto launch = [&](cudaStream_t q) -> int {
+        GatherList gl;
+        gl.count = 0;
+        for (int i = 0; i < count; ++i) {
+            if (!x_host[i]) continue;
             const nq_linear_desc& L = desc(i);
-            st = prefill_forward(static_cast<const uint16_t*>(xs[i]), L.Upk, L.Vpk, static_cast<const uint16_t*>(L.s1),
-                                 static_cast<const uint16_t*>(L.s2), L.m, L.n, L.r, batch, ys[i], ws, s);
-            // the optional outputs by the stand-alone kernels, after the layer
-            if (st == NQ_OK && ex && ex[i].y_bf16)
-                st = cast_f32_bf16_device(ys[i], batch * L.m, static_cast<uint16_t*>(ex[i].y_bf16), s);
-            if (st == NQ_OK && ex && ex[i].y_rmsnorm_bf16)
-                st = rms_normalize_bf16_device(ys[i], batch, L.m, static_cast<uint16_t*>(ex[i].y_rmsnorm_bf16), s);
-        }
-    } else {
-        for (int i0 = 0; i0 < count && st == NQ_OK; i0 += kMaxGroup) {
-            const int cnt = count - i0 < kMaxGroup ? count - i0 : kMaxGroup;
-            DecodeCall calls[kMaxGroup];
-            for (int i = 0; i < cnt; ++i) {
-                const nq_linear_desc& L = desc(i0 + i);
-                calls[i] = DecodeCall{static_cast<const uint16_t*>(xs[i0 + i]), L.Upk, L.Vpk,
-                                      static_cast<const uint16_t*>(L.s1), static_cast<const uint16_t*>(L.s2),
-                                      ys[i0 + i], L.m, L.n, L.r};
-                if (ex) {
-                    calls[i].y_bf16 = static_cast<uint16_t*>(ex[i0 + i].y_bf16);
-                    calls[i].y_norm = static_cast<uint16_t*>(ex[i0 + i].y_rmsnorm_bf16);
+            const size_t b = sizeof(uint16_t) * (size_t)batch * L.n;
+            void* dst = const_cast<void*>(xs[i]);
+            if (x_pin[i]) {
+                gl.seg[gl.count++] = GatherSeg{x_pin[i], dst, b};
+                if (gl.count == kMaxGather) {
+                    if (gather_device(gl, q) != NQ_OK) return NQ_ERR_CUDA;
+                    gl.count = 0;
                 }
+            } else if (cudaMemcpyAsync(dst, L.x, b, cudaMemcpyHostToDevice, q) != cudaSuccess) {
+                return NQ_ERR_CUDA;
             }
-            ws = workspace_for(m_max, n_max, r_max, batch, decode_need(calls, cnt, batch), &st);
-            if (!ws) return st;
-            st = decode_forward_group(calls, cnt, batch, ws, s);
         }
+        if (gl.count > 0 && gather_device(gl, q) != NQ_OK) return NQ_ERR_CUDA;
+        int rc = NQ_OK;
+        if (batch > NQ_DECODE_MAX_BATCH) {
+            for (int i = 0; i < count && rc == NQ_OK; ++i) {
+                const nq_linear_desc& L = desc(i);
+                rc = prefill_forward(static_cast<const uint16_t*>(xs[i]), L.Upk, L.Vpk,
+                                     static_cast<const uint16_t*>(L.s1), static_cast<const uint16_t*>(L.s2), L.m, L.n,
+                                     L.r, batch, ys[i], ws, q);
+                // the optional outputs by the stand-alone kernels, after the layer
+                if (rc == NQ_OK && ex && ex[i].y_bf16)
+                    rc = cast_f32_bf16_device(ys[i], batch * L.m, static_cast<uint16_t*>(ex[i].y_bf16), q);
+                if (rc == NQ_OK && ex && ex[i].y_rmsnorm_bf16)
+                    rc = rms_normalize_bf16_device(ys[i], batch, L.m, static_cast<uint16_t*>(ex[i].y_rmsnorm_bf16), q);
+            }
+        } else {
+            for (int i0 = 0; i0 < count && rc == NQ_OK; i0 += kMaxGroup) {
+                const int cnt = count - i0 < kMaxGroup ? count - i0 : kMaxGroup;
+                DecodeCall calls[kMaxGroup];
+                for (int i = 0; i < cnt; ++i) {
+                    const nq_linear_desc& L = desc(i0 + i);
+                    calls[i] = DecodeCall{static_cast<const uint16_t*>(xs[i0 + i]), L.Upk, L.Vpk,
+                                          static_cast<const uint16_t*>(L.s1), static_cast<const uint16_t*>(L.s2),
+                                          ys[i0 + i], L.m, L.n, L.r};
+                    if (ex) {
+                        calls[i].y_bf16 = static_cast<uint16_t*>(ex[i0 + i].y_bf16);
+                        calls[i].y_norm = static_cast<uint16_t*>(ex[i0 + i].y_rmsnorm_bf16);
+                    }
+                }
+                rc = decode_forward_group(calls, cnt, batch, ws, q);
+            }
+        }
+        return rc;
+    };
+    if (any_host && !pageable) {
+        int dev = -1;
+        if (cudaGetDevice(&dev) != cudaSuccess) {
+            cudaGetLastError();
+            return NQ_ERR_CUDA;
+        }
+        std::vector<uint64_t> key;
+        key.reserve(8 + 12 * (size_t)count);
+        auto u = [](const void* p) { return (uint64_t)reinterpret_cast<uintptr_t>(p); };
+        key.insert(key.end(), {(uint64_t)dev, ws_generation(), (uint64_t)batch, (uint64_t)count, ex ? 1ull : 0ull,
+                               u(ws->base), u(ws->xstage), u(ws->ystage)});
+        for (int i = 0; i < count; ++i) {
+            const nq_linear_desc& L = desc(i);
+            key.insert(key.end(), {u(L.x), u(L.Upk), u(L.Vpk), u(L.s1), u(L.s2), u(L.y), (uint64_t)L.m, (uint64_t)L.n,
+                                   (uint64_t)L.r, u(x_pin[i]), u(ex ? ex[i].y_bf16 : nullptr),
+                                   u(ex ? ex[i].y_rmsnorm_bf16 : nullptr)});
+        }
+        st = launch_cached(dev, key, s, launch);
+    } else {
+        st = launch(s);
     }
     if (st != NQ_OK) return st;
     if (ybytes) {

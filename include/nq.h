@@ -94,6 +94,12 @@ int nq_unpack_signs(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* 
  * address, pageable x by a copy), pinned host y is written by the kernels directly and
  * pageable host y copied back; with any host buffer the call then synchronises `stream`
  * before returning.  Device buffers are used asynchronously on `stream`.
+ * A synchronising call whose host buffers are all pinned is replayed from a CUDA graph
+ * once the identical call (same pointers, sizes and library scratch) has been made before:
+ * its second occurrence captures the launches into a graph that the library keeps (up to
+ * 32 per device, least recently used dropped first), later ones launch that graph, which
+ * costs less host time than the separate launches.  The graph reads the buffers' contents
+ * at the time of each call, like a direct launch.  Not on a stream under capture.
  * Every pointer must be 16-byte aligned.
  * Path: batch <= NQ_DECODE_MAX_BATCH runs the decode path (two binary GEMV stages on the
  * CUDA cores and integer tensor-core instructions, t kept in the workspace); larger
@@ -207,7 +213,9 @@ typedef struct nq_linear_desc {
  * (else NQ_ERR_PTRKIND).  Each layer's x and y may be device or host memory, handled as
  * in nq_lowrank_linear_fwd (pinned x gathered by one kernel for all layers, pinned y
  * written directly, pageable buffers copied); with any host buffer the call synchronises
- * `stream` before returning, with only device buffers it is asynchronous.
+ * `stream` before returning (and, with only pinned host buffers, is replayed from a kept
+ * CUDA graph when repeated, as nq_lowrank_linear_fwd), with only device buffers it is
+ * asynchronous.
  */
 int nq_lowrank_linear_fwd_grouped(const nq_linear_desc* layers, int count, int64_t batch, void* stream);
 

@@ -381,3 +381,37 @@ def test_grouped_host_buffers(nq, orc, batch):
         got = host_ys[i].cpu().numpy() if isinstance(host_ys[i], torch.Tensor) else host_ys[i]
         assert np.array_equal(got, want), i
         assert rel_err(got, c.oracle(orc)) <= TOL
+
+
+@pytest.mark.parametrize("batch", [1, 5, 20])
+def test_grouped_pinned_repeated_calls(nq, orc, batch):
+    """The same grouped call with pinned host x and y made again and again (the library
+    replays such calls from a captured CUDA graph after their first occurrence): every call
+    reads the x it is given at that moment, also after the workspace was regrown in between,
+    and returns the device-buffer call's bits."""
+    shapes = [(512, 512, 128), (384, 640, 256), (1024, 256, 384)]
+    cases = [Case(orc, nq, m, n, r, batch, seed=970 + i) for i, (m, n, r) in enumerate(shapes)]
+    xh = [torch.empty((batch, c.n), dtype=torch.int16).pin_memory() for c in cases]
+    yh = [torch.empty((batch, c.m), dtype=torch.float32).pin_memory() for c in cases]
+    host_layers = [(xh[i], c.Upk, c.Vpk, c.s1_d, c.s2_d, yh[i], c.m, c.n, c.r) for i, c in enumerate(cases)]
+    for k in range(5):
+        if k == 3:  # a call with a larger pinned x grows the staging buffer (a new generation)
+            big = Case(orc, nq, 128, 1 << 18, 128, 8, seed=990)
+            big_x = torch.from_numpy(big.x.view(np.int16)).pin_memory()
+            nq.lowrank_linear_fwd(big_x, big.Upk, big.Vpk, big.s1_d, big.s2_d, big.m, big.n, big.r)
+        xs = [synth.activations_bf16(batch, c.n, 1000 + 10 * k + i) for i, c in enumerate(cases)]
+        for i in range(len(cases)):
+            xh[i].copy_(torch.from_numpy(xs[i].view(np.int16)))
+            yh[i].fill_(float("nan"))
+        nq.lowrank_linear_fwd_grouped(host_layers, batch)
+        dev_ys = [torch.empty((batch, c.m), dtype=torch.float32, device="cuda") for c in cases]
+        nq.lowrank_linear_fwd_grouped(
+            [(torch.from_numpy(xs[i].view(np.int16)).cuda(), c.Upk, c.Vpk, c.s1_d, c.s2_d, dev_ys[i], c.m, c.n, c.r)
+             for i, c in enumerate(cases)], batch)
+        torch.cuda.synchronize()
+        for i, c in enumerate(cases):
+            assert np.array_equal(yh[i].numpy(), dev_ys[i].cpu().numpy()), (k, i)
+        if k in (0, 4):
+            for i, c in enumerate(cases):
+                want = orc.lowrank_linear_fwd(xs[i], c.Upk_o, c.Vpk_o, c.s1, c.s2, c.m, c.n, c.r)
+                assert rel_err(yh[i].numpy(), want) <= TOL, (k, i)
