@@ -351,23 +351,50 @@ static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_line
     for (int i = 0; i < count; ++i) pageable = pageable || (x_host[i] && !x_pin[i]);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int st = NQ_OK;
+    // Path.  Up to NQ_DECODE_MAX_BATCH tokens: the decode kernels, up to 16 layers per launch
+    // pair.  More tokens: each layer's prefill GEMMs, one layer after another; or, for a group
+    // of layers and a few dozen tokens, the decode kernels over token chunks of at most
+    // NQ_DECODE_MAX_BATCH, whichever a cost estimate fitted to B200 timings (microseconds)
+    // finds faster: a decode launch pair of 5..8 tokens ~ 29.4 + 0.53 per MB of the group's
+    // packed signs (1..4 tokens: half that); one layer's prefill below 64 tokens ~ 28 + 0.2
+    // per token + 1.0 per MB of its packed signs (latency-bound).
+    bool use_decode = batch <= NQ_DECODE_MAX_BATCH;
+    if (!use_decode && count > 1 && batch <= 64) {
+        double mb = 0.0, t_pre = 0.0;
+        for (int i = 0; i < count; ++i) {
+            const nq_linear_desc& L = desc(i);
+            const double mb_i = (double)L.r * (double)(L.m + L.n) / 8e6;
+            mb += mb_i;
+            t_pre += 28.0 + 0.2 * (double)batch + mb_i;
+        }
+        const double pair = 29.4 + 0.53 * mb;
+        const int64_t full = batch / NQ_DECODE_MAX_BATCH, rest = batch % NQ_DECODE_MAX_BATCH;
+        const double t_dec = (double)full * pair + (rest == 0 ? 0.0 : rest <= 4 ? 0.5 * pair : pair);
+        use_decode = t_dec < t_pre;
+    }
+    // token chunks of the decode path: full ones of NQ_DECODE_MAX_BATCH, then the rest
+    const int64_t chunk = batch < NQ_DECODE_MAX_BATCH ? batch : NQ_DECODE_MAX_BATCH;
+    const int64_t tail = batch % chunk;
     // the scratch of every launch of the call, sized once before anything is enqueued
     DecodeNeed need;
-    for (int i0 = 0; i0 < count; i0 += (batch > NQ_DECODE_MAX_BATCH ? 1 : kMaxGroup)) {
-        const int cnt = batch > NQ_DECODE_MAX_BATCH ? 1 : (count - i0 < kMaxGroup ? count - i0 : kMaxGroup);
+    for (int i0 = 0; i0 < count; i0 += (use_decode ? kMaxGroup : 1)) {
+        const int cnt = !use_decode ? 1 : (count - i0 < kMaxGroup ? count - i0 : kMaxGroup);
         DecodeCall calls[kMaxGroup];
         for (int i = 0; i < cnt; ++i) {
             const nq_linear_desc& L = desc(i0 + i);
             calls[i] = DecodeCall{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, L.m, L.n, L.r};
             if (ex) calls[i].y_norm = static_cast<uint16_t*>(ex[i0 + i].y_rmsnorm_bf16);
         }
-        const DecodeNeed d = decode_need(calls, cnt, batch);
-        need.t = d.t > need.t ? d.t : need.t;
-        need.tgmax = d.tgmax > need.tgmax ? d.tgmax : need.tgmax;
-        need.partials = d.partials > need.partials ? d.partials : need.partials;
-        need.counters = d.counters > need.counters ? d.counters : need.counters;
+        for (const int64_t b : {use_decode ? chunk : batch, use_decode ? tail : int64_t(0)}) {
+            if (b == 0) continue;
+            const DecodeNeed d = decode_need(calls, cnt, b);
+            need.t = d.t > need.t ? d.t : need.t;
+            need.tgmax = d.tgmax > need.tgmax ? d.tgmax : need.tgmax;
+            need.partials = d.partials > need.partials ? d.partials : need.partials;
+            need.counters = d.counters > need.counters ? d.counters : need.counters;
+        }
     }
-    Workspace* ws = workspace_for(m_max, n_max, r_max, batch, need, &st);
+    Workspace* ws = workspace_for(m_max, n_max, r_max, use_decode ? chunk : batch, need, &st);
     if (!ws) return st;
     if (xbytes || ybytes) {
         st = ensure_staging(ws, xbytes, ybytes);
@@ -415,7 +442,7 @@ static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_line
         }
         if (gl.count > 0 && gather_device(gl, q) != NQ_OK) return NQ_ERR_CUDA;
         int rc = NQ_OK;
-        if (batch > NQ_DECODE_MAX_BATCH) {
+        if (!use_decode) {
             for (int i = 0; i < count && rc == NQ_OK; ++i) {
                 const nq_linear_desc& L = desc(i);
                 rc = prefill_forward(static_cast<const uint16_t*>(xs[i]), L.Upk, L.Vpk,
@@ -428,20 +455,24 @@ static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_line
                     rc = rms_normalize_bf16_device(ys[i], batch, L.m, static_cast<uint16_t*>(ex[i].y_rmsnorm_bf16), q);
             }
         } else {
-            for (int i0 = 0; i0 < count && rc == NQ_OK; i0 += kMaxGroup) {
-                const int cnt = count - i0 < kMaxGroup ? count - i0 : kMaxGroup;
-                DecodeCall calls[kMaxGroup];
-                for (int i = 0; i < cnt; ++i) {
-                    const nq_linear_desc& L = desc(i0 + i);
-                    calls[i] = DecodeCall{static_cast<const uint16_t*>(xs[i0 + i]), L.Upk, L.Vpk,
-                                          static_cast<const uint16_t*>(L.s1), static_cast<const uint16_t*>(L.s2),
-                                          ys[i0 + i], L.m, L.n, L.r};
-                    if (ex) {
-                        calls[i].y_bf16 = static_cast<uint16_t*>(ex[i0 + i].y_bf16);
-                        calls[i].y_norm = static_cast<uint16_t*>(ex[i0 + i].y_rmsnorm_bf16);
+            for (int64_t b0 = 0; b0 < batch && rc == NQ_OK; b0 += chunk) {
+                const int64_t bc = batch - b0 < chunk ? batch - b0 : chunk;
+                for (int i0 = 0; i0 < count && rc == NQ_OK; i0 += kMaxGroup) {
+                    const int cnt = count - i0 < kMaxGroup ? count - i0 : kMaxGroup;
+                    DecodeCall calls[kMaxGroup];
+                    for (int i = 0; i < cnt; ++i) {
+                        const nq_linear_desc& L = desc(i0 + i);
+                        calls[i] = DecodeCall{static_cast<const uint16_t*>(xs[i0 + i]) + b0 * L.n, L.Upk, L.Vpk,
+                                              static_cast<const uint16_t*>(L.s1), static_cast<const uint16_t*>(L.s2),
+                                              ys[i0 + i] + b0 * L.m, L.m, L.n, L.r};
+                        if (ex) {
+                            if (ex[i0 + i].y_bf16) calls[i].y_bf16 = static_cast<uint16_t*>(ex[i0 + i].y_bf16) + b0 * L.m;
+                            if (ex[i0 + i].y_rmsnorm_bf16)
+                                calls[i].y_norm = static_cast<uint16_t*>(ex[i0 + i].y_rmsnorm_bf16) + b0 * L.m;
+                        }
                     }
+                    rc = decode_forward_group(calls, cnt, bc, ws, q);
                 }
-                rc = decode_forward_group(calls, cnt, batch, ws, q);
             }
         }
         return rc;

@@ -207,7 +207,12 @@ typedef struct nq_linear_desc {
  * batch, e.g. the projections of one transformer block that read the same or different
  * activations.  The result of every layer equals nq_lowrank_linear_fwd on it; the
  * decode path (batch <= NQ_DECODE_MAX_BATCH) runs up to 16 layers per launch pair, so
- * small layers share the launch and dependency latency.  No layer's y may overlap
+ * small layers share the launch and dependency latency.  With more tokens (up to 64) and
+ * more than one layer, the call runs the decode path over token chunks of at most
+ * NQ_DECODE_MAX_BATCH instead of each layer's prefill GEMMs one after another when a cost
+ * estimate (fitted to B200 timings) finds that faster: several layers and a few dozen
+ * tokens, e.g. the seven Llama-2-7B-shaped projections up to 48 tokens.  Each token's
+ * result is then that of the decode path, within the same accuracy bound.  No layer's y may overlap
  * another layer's inputs.  Argument checks as nq_lowrank_linear_fwd, plus count >= 0
  * (0 is a no-op) and `layers` non-NULL.  Weights (Upk, Vpk, s1, s2) must be device memory
  * (else NQ_ERR_PTRKIND).  Each layer's x and y may be device or host memory, handled as
