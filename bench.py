@@ -371,6 +371,15 @@ def run_ours(args):
         secondary["decode_b8_gbs"] = round(w8.step_bytes * args.steps / (ms8 * 1e-3) / 1e9, 1)
         secondary["decode_b8_tokens_per_s"] = round(8 * args.steps / (ms8 * 1e-3), 1)
         del w8
+        # 16 tokens in one grouped call of the block (the decode kernels over two token chunks)
+        w16 = DecodeWorkload(layers, 16, seed=116, device=device)
+        with torch.cuda.stream(stream):
+            w16.step(0, stream.cuda_stream)
+        torch.cuda.synchronize()
+        ms16 = timed_graphs(w16, args.steps, args.warmup, stream)
+        secondary["grouped_b16_us_per_call"] = round(ms16 * 1e3 / args.steps, 2)
+        secondary["grouped_b16_tokens_per_s"] = round(16 * args.steps / (ms16 * 1e-3), 1)
+        del w16
         # the input gradient dx = W^T dy of the same block (backward of the layers)
         for bb in (1, 8):
             wb = backward_workload(layers, bb, seed=123 + bb, device=device)
