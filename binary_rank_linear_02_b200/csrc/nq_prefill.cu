@@ -102,6 +102,28 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// orders this thread's view of global memory (generic proxy) before its later TMA loads
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Waits (one thread) until *count >= need; past kWaitLimitNs of GPU time it records
+// NQ_ERR_TIMEOUT in the status word and returns false.
+__device__ __forceinline__ bool wait_count(const int* count, int need, unsigned* status) {
+    const unsigned long long t0 = global_ns();
+    while (ld_acquire(count) < need) {
+        if (global_ns() - t0 > kWaitLimitNs) {
+            atomicExch(status, (unsigned)(-NQ_ERR_TIMEOUT));
+            return false;
+        }
+        __nanosleep(200);
+    }
+    return true;
+}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -575,11 +597,25 @@ struct TileBarriers {
 // 16).  Its epilogue does not overlap the next tile's MMAs, but neither does it compete
 // with them: with the persistent kernel's overlapped epilogue the global stores slowed the
 // main loop (27 us of 306 at 4096 tokens).
+//
+// Hand-off from GEMM 1 to GEMM 2 by token tile (`handoff`, for a GEMM 1 of more tiles than
+// one wave holds): a GEMM 1 CTA releases its dependants as soon as its own dependency wait
+// is over and, once its tile of T is stored, adds one to the counter of its token tile
+// (sync[tile]); a GEMM 2 CTA waits only for the counters of the GEMM 1 token tiles its own
+// tokens fall in (every row block of GEMM 1 done), so GEMM 2 fills the SMs that GEMM 1's
+// last wave leaves idle.  The GEMM 2 CTAs that depend on a token tile count themselves past
+// the wait in sync[ntt1 + tile]; the last one clears both counters for the next call.  The
+// waits are bounded (NQ_ERR_TIMEOUT in the status word).  Without it GEMM 1 releases GEMM 2
+// from its epilogue and GEMM 2 waits for all of GEMM 1.  Measured on the 11008 x 4096,
+// r = 2432 layer: 4096 tokens (GEMM 1: 304 tiles for 296 slots) 268 -> 256 us with it;
+// below, where GEMM 1 fits one wave, GEMM 2's early CTAs only crowd GEMM 1's SMs (1024
+// tokens 101.6 us without, 103.8 us with).
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kTileThreads, 2)
 tile_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint32_t* __restrict__ Wpk, int64_t kdim,
             int64_t mdim, int64_t batch, uint16_t* __restrict__ T_out, float* __restrict__ y_out,
-            const uint16_t* __restrict__ s1, unsigned* __restrict__ status) {
+            const uint16_t* __restrict__ s1, unsigned* __restrict__ status, int* __restrict__ sync, int bn1,
+            int ntt1, int nrb1, int handoff) {
     using G = Geometry<BN>;
     constexpr int S = G::kStages;
     extern __shared__ unsigned char smem_raw[];
@@ -622,9 +658,34 @@ tile_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint32_t* __res
     if (warp == 0) {
         // ---------------- TMA producer of the B tiles (activations)
         if (lane == 0) {
-            pdl_wait();  // B comes from the previous kernel (prescale or GEMM 1)
+            if (EPI == 0 || !handoff) {
+                pdl_wait();  // B comes from the previous kernel (prescale or GEMM 1)
+                if (handoff) pdl_trigger();  // GEMM 2 may launch: it waits on the token-tile counters
+            } else {
+                // B = T: the GEMM 1 token tiles that hold tokens n0 .. n0 + BN - 1
+                const int tt0 = (int)(n0 / bn1);
+                const int tt1 = (int)(((n0 + BN < batch ? n0 + BN : batch) - 1) / bn1);
+                bool ok = true;
+                for (int tt = tt0; tt <= tt1 && ok; ++tt) ok = wait_count(sync + tt, nrb1, status);
+                if (ok) {
+                    fence_proxy_async_global();
+                    for (int tt = tt0; tt <= tt1; ++tt) {
+                        // GEMM 2 CTAs that read token tile tt: all row blocks x the GEMM 2
+                        // token tiles overlapping it
+                        const int64_t e1 = ((int64_t)(tt + 1) * bn1 < batch ? (int64_t)(tt + 1) * bn1 : batch) - 1;
+                        const int users = (int)gridDim.x * (int)(e1 / BN - (int64_t)tt * bn1 / BN + 1);
+                        if (atomicAdd(sync + ntt1 + tt, 1) == users - 1) {
+                            sync[tt] = 0;
+                            sync[ntt1 + tt] = 0;
+                        }
+                    }
+                } else {
+                    *abort_flag = 1;
+                }
+            }
             int issued = 0;
-            for (int kb = 0; kb < nkb; ++kb) {
+            const int nkb_go = *abort_flag ? 0 : nkb;  // none after a failed wait
+            for (int kb = 0; kb < nkb_go; ++kb) {
                 const int s = kb % S;
                 const uint32_t ph = (uint32_t)(kb / S) & 1u;
                 if (!mbar_wait(smem_u32(&bar.empty[s]), ph ^ 1u, abort_flag, status)) break;
@@ -729,8 +790,17 @@ tile_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint32_t* __res
                 }
             }
         }
+        if (EPI == 0 && handoff) {  // the tile of T is stored: count it for its token tile
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (threadIdx.x == 64 && !*abort_flag) {
+                __threadfence();
+                atomicAdd(sync + blockIdx.y, 1);
+            }
+        }
     }
 
+    // GEMM 2 completes only after GEMM 1 has, so that the next kernel's dependency wait covers both
+    if (EPI == 1 && threadIdx.x == 0) pdl_wait();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -937,7 +1007,7 @@ cudaError_t launch_prescale(const uint16_t* x, const uint16_t* s2, int64_t n, in
 
 template <int BN, int EPI>
 int launch_tile_gemm(const void* bsrc, int64_t K, const uint32_t* Wpk, int64_t M, int64_t batch, uint16_t* T_out,
-                     float* y_out, const uint16_t* s1, Workspace* ws, cudaStream_t stream) {
+                     float* y_out, const uint16_t* s1, Workspace* ws, cudaStream_t stream, int bn1, int nrb1) {
     using G = Geometry<BN>;
     static unsigned long long init_mask = 0;
     const unsigned long long bit = 1ull << (ws->device & 63);
@@ -950,9 +1020,12 @@ int launch_tile_gemm(const void* bsrc, int64_t K, const uint32_t* Wpk, int64_t M
     CUtensorMap map;
     if (!make_map(&map, bsrc, batch, K, kBK, BN, false, true)) return NQ_ERR_CUDA;
     const unsigned ntiles = (unsigned)((batch + BN - 1) / BN);
+    const int ntt1 = (int)((batch + bn1 - 1) / bn1);  // GEMM 1 token tiles
+    // the hand-off when GEMM 1's tiles exceed one wave (two CTAs per SM)
+    const int handoff = (int64_t)nrb1 * ntt1 > 2 * (int64_t)sm_count() ? 1 : 0;
     return launch_pdl(tile_gemm_kernel<BN, EPI>, dim3((unsigned)(M / kBM), ntiles), dim3(kTileThreads),
-                      (size_t)G::kSmemBytes, stream, map, Wpk, K, M, batch, T_out, y_out, s1,
-                      ws->status + 1) == cudaSuccess
+                      (size_t)G::kSmemBytes, stream, map, Wpk, K, M, batch, T_out, y_out, s1, ws->status + 1,
+                      ws->counters, bn1, ntt1, nrb1, handoff) == cudaSuccess
                ? NQ_OK
                : NQ_ERR_CUDA;
 }
@@ -979,15 +1052,17 @@ int choose_bn(int64_t M, int64_t batch, int sms) {
     return best;
 }
 
+// bn1, nrb1: GEMM 1's token-tile width and row blocks (the token-tile counters' layout)
 template <int EPI>
 int launch_tile_gemm_bn(int bn, const void* bsrc, int64_t K, const uint32_t* Wpk, int64_t M, int64_t batch,
-                        uint16_t* T_out, float* y_out, const uint16_t* s1, Workspace* ws, cudaStream_t stream) {
+                        uint16_t* T_out, float* y_out, const uint16_t* s1, Workspace* ws, cudaStream_t stream,
+                        int bn1, int nrb1) {
     switch (bn) {
-        case 64: return launch_tile_gemm<64, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream);
-        case 128: return launch_tile_gemm<128, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream);
-        case 144: return launch_tile_gemm<144, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream);
-        case 176: return launch_tile_gemm<176, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream);
-        default: return launch_tile_gemm<256, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream);
+        case 64: return launch_tile_gemm<64, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream, bn1, nrb1);
+        case 128: return launch_tile_gemm<128, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream, bn1, nrb1);
+        case 144: return launch_tile_gemm<144, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream, bn1, nrb1);
+        case 176: return launch_tile_gemm<176, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream, bn1, nrb1);
+        default: return launch_tile_gemm<256, EPI>(bsrc, K, Wpk, M, batch, T_out, y_out, s1, ws, stream, bn1, nrb1);
     }
 }
 
@@ -996,10 +1071,11 @@ int run_tile_gemms(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, 
                    cudaStream_t stream) {
     if (launch_prescale(x, s2, n, batch, ws, stream) != cudaSuccess) return NQ_ERR_CUDA;
     const int sms = sm_count();
-    int st = launch_tile_gemm_bn<0>(choose_bn(r, batch, sms), ws->xprime, n, Vpk, r, batch, ws->T, nullptr, nullptr,
-                                    ws, stream);
+    const int bn1 = choose_bn(r, batch, sms), nrb1 = (int)(r / kBM);
+    int st = launch_tile_gemm_bn<0>(bn1, ws->xprime, n, Vpk, r, batch, ws->T, nullptr, nullptr, ws, stream, bn1, nrb1);
     if (st != NQ_OK) return st;
-    return launch_tile_gemm_bn<1>(choose_bn(m, batch, sms), ws->T, r, Upk, m, batch, nullptr, y, s1, ws, stream);
+    return launch_tile_gemm_bn<1>(choose_bn(m, batch, sms), ws->T, r, Upk, m, batch, nullptr, y, s1, ws, stream, bn1,
+                                  nrb1);
 }
 
 }  // namespace
@@ -1013,9 +1089,9 @@ void prefill_workspace_need(int64_t m, int64_t n, int64_t r, int64_t batch, int6
                             int64_t* counter_ints) {
     const int sms = sm_count();
     int64_t pf = 0, ci = 0;
-    if (batch > kPersistentMaxBatch) {
+    if (batch > kPersistentMaxBatch) {  // the token-tile counters of the GEMM 1 -> GEMM 2 hand-off
         *partial_floats = 0;
-        *counter_ints = 0;
+        *counter_ints = 2 * ((batch + 63) / 64);
         return;
     }
     const Plan p1 = plan_gemm(r, n, batch, sms), p2 = plan_gemm(m, r, batch, sms);
