@@ -34,7 +34,9 @@
 // before it waits on the previous kernel (programmatic dependent launch) and lets the next
 // kernel launch at once, so weight streaming overlaps the dependency chain.  Stage 1
 // splits each 128-row block's columns so that every CTA stages one chunk; the last CTA of a
-// block adds the partial sums in a fixed order (deterministic).  Stage 2 runs as one even
+// block adds the partial sums in a fixed order (deterministic), or, where all of t fits one
+// stage-2 span and the splits are few, every stage-1 CTA just stores its partial and each
+// stage-2 CTA adds the partials itself in the same order.  Stage 2 runs as one even
 // wave where it fits: each layer gets CTAs in proportion to its work, each CTA holds its
 // rows of U and the whole of t on chip.  Several independent layers share one launch, the
 // slowest first in the grid.
@@ -64,6 +66,8 @@ constexpr int kMaxK2 = 8;              // stage-2 CTAs per SM tried for a launch
 constexpr size_t kSmemPerSM = 228 * 1024;  // shared memory of one SM
 constexpr size_t kSmemReserve = 1024;      // taken by the system from it for every resident CTA
 constexpr int kWaveTiles2 = 8;         // stage-2 tiles per CTA of a launch that needs several waves
+constexpr int kSumSlots = 4;           // stage 2 adding the split partials: float4 columns per thread (r <= 4096)
+constexpr int kS2SumMaxSplits = 12;    // ... for groups whose layers have at most this many stage-1 splits
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 __device__ __forceinline__ float f16_to_f32(uint16_t h) { return __half2float(__ushort_as_half(h)); }
@@ -129,6 +133,7 @@ struct DecLayer {
     int nsplit;      // stage 1: CTAs per 128-row block (column splits)
     int cps;         // stage 1: column blocks per split
     int s2_ctas;     // stage 2: CTAs of the layer, each an even share of its 16-row tiles
+    int s2sum;       // 1: stage 2 adds up the layer's stage-1 split partials itself
 };
 
 struct DecGroup {
@@ -512,6 +517,14 @@ stage1_kernel(const __grid_constant__ DecGroup grp) {
             }
         }
     __syncthreads();
+    if (L.s2sum) {  // stage 2 adds the splits up: this CTA's sums are its split's partial of t
+        float* dst = L.nsplit > 1 ? L.partials + (int64_t)sp * batch * r : L.t;
+        for (int i = threadIdx.x; i < batch * kRowsS1; i += kThreads1) {
+            const int tok = i / kRowsS1, k = i % kRowsS1;
+            dst[(int64_t)tok * r + row0 + k] = res[tok][k];
+        }
+        return;
+    }
     const int nrb = r / kRowsS1;
     if (L.nsplit > 1) {
         for (int i = threadIdx.x; i < batch * kRowsS1; i += kThreads1) {
@@ -670,21 +683,74 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
     for (int i = threadIdx.x; i < rows * batch; i += kThreads) bq[i] = 0;  // [row][batch]
     zero_fragments<NTG, kThreads>(frag, r2 / kCB);
     pdl_trigger();
-    pdl_wait();  // t and its maxima come from stage 1
-    fetch_t(0);
-    cp_async_commit();
+    pdl_wait();  // t (or its split partials) and its maxima come from stage 1
+    if (L.s2sum) {
+        // t = the layer's stage-1 split partials added in split order (the order the reducing
+        // stage-1 CTA uses otherwise), staged as fetch_t stages it, and each token's max |t|
+        const float* src = L.nsplit > 1 ? L.partials : L.t;
+        const int nq = L.nsplit > 1 ? L.nsplit : 1;
+        const int64_t qstride = (int64_t)batch * r;
+        const int n4 = r / 4;
+        for (int tok = 0; tok < batch; ++tok) {
+            const float4* s4 = reinterpret_cast<const float4*>(src + (int64_t)tok * r);
+            float4 acc[kSumSlots];
+#pragma unroll
+            for (int j = 0; j < kSumSlots; ++j) {
+                const int p = threadIdx.x + j * kThreads;
+                acc[j] = p < n4 ? __ldcg(s4 + p) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            for (int q = 1; q < nq; ++q) {
+#pragma unroll
+                for (int j = 0; j < kSumSlots; ++j) {
+                    const int p = threadIdx.x + j * kThreads;
+                    if (p < n4) {
+                        const float4 v = __ldcg(s4 + q * qstride / 4 + p);
+                        acc[j].x += v.x;
+                        acc[j].y += v.y;
+                        acc[j].z += v.z;
+                        acc[j].w += v.w;
+                    }
+                }
+            }
+            float mx = 0.f;
+#pragma unroll
+            for (int j = 0; j < kSumSlots; ++j) {
+                const int p = threadIdx.x + j * kThreads;
+                if (p < n4) {
+                    *reinterpret_cast<float4*>(tbuf + tok * s2_t_row(r2) + 4 * p + 8 * (p >> 3)) = acc[j];
+                    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(acc[j].x), fabsf(acc[j].y)), fmaxf(fabsf(acc[j].z), fabsf(acc[j].w))));
+                }
+            }
+            mx = warp_max(mx);
+            if (lane == 0) mi.red[warp][tok] = mx;
+        }
+        __syncthreads();
+        for (int tok = warp; tok < batch; tok += kWarps) {
+            float mx = lane < kWarps ? mi.red[lane][tok] : 0.f;
+            mx = warp_max(mx);
+            if (lane == 0) {
+                const int e = range_exponent(mx);
+                mi.e[tok] = e;
+                mi.up[tok] = pow2f(kQBits - e);
+                mi.qsum[tok] = 0;
+            }
+        }
+    } else {
+        fetch_t(0);
+        cp_async_commit();
 
-    // global max |t| per token from the per-block maxima (one warp per token)
-    const int nrb = r / kRowsS1;
-    for (int tok = warp; tok < batch; tok += kWarps) {
-        float mx = 0.f;
-        for (int gi = lane; gi < nrb; gi += 32) mx = fmaxf(mx, L.tgmax[(int64_t)tok * nrb + gi]);
-        mx = warp_max(mx);
-        if (lane == 0) {
-            const int e = range_exponent(mx);
-            mi.e[tok] = e;
-            mi.up[tok] = pow2f(kQBits - e);
-            mi.qsum[tok] = 0;
+        // global max |t| per token from the per-block maxima (one warp per token)
+        const int nrb = r / kRowsS1;
+        for (int tok = warp; tok < batch; tok += kWarps) {
+            float mx = 0.f;
+            for (int gi = lane; gi < nrb; gi += 32) mx = fmaxf(mx, L.tgmax[(int64_t)tok * nrb + gi]);
+            mx = warp_max(mx);
+            if (lane == 0) {
+                const int e = range_exponent(mx);
+                mi.e[tok] = e;
+                mi.up[tok] = pow2f(kQBits - e);
+                mi.qsum[tok] = 0;
+            }
         }
     }
 
@@ -918,6 +984,17 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
     stage2_plan(calls, count, batch, ctas, &grp.w2words, &grp.rows2, &grp.per_sm2);
     const int cps = stage1_cps(calls, count, max_splits);
     grp.r2 = stage2_span(r_max, batch);
+    // Stage 2 adds up the layers' split partials itself (no hand-off between the stage-1 CTAs
+    // of a row block) when all of t fits one span and no layer has many splits: each stage-2
+    // CTA then reads nsplit x r values per token instead of r, and stage 1 ends no earlier
+    // unless every layer drops its hand-off (the layer of most splits has the longest).
+    // Measured on a B200: the seven Llama-2-7B-shaped layers at batch 1 (4 and 11 splits)
+    // 14.7 -> 13.6 us; the 70B-shaped block (8 and 28 splits) is slower with it for any
+    // subset of its layers (36.5 -> 37.0-38.8 us), so it keeps the hand-off.
+    int max_nsplit = 0;
+    for (int i = 0; i < count; ++i) max_nsplit = std::max(max_nsplit, (int)((calls[i].n / kCB + cps - 1) / cps));
+    const bool s2sum = !stage1_only && r_max <= grp.r2 && r_max <= 4 * kSumSlots * kThreads &&
+                       max_nsplit <= kS2SumMaxSplits;
     grp.depth1 = cps > kChunkCB ? 2 : 1;
     size_t toff = 0, goff = 0, poff = 0, coff = 0;
     grp.s1_start[0] = grp.s2_start[0] = 0;
@@ -951,6 +1028,7 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
         L.n = (int)c.n;
         L.r = (int)c.r;
         L.s2_ctas = ctas[i];
+        L.s2sum = s2sum ? 1 : 0;
         L.cps = cps;
         L.nsplit = (int)((c.n / kCB + cps - 1) / cps);
         L.t = ws->t + toff;
