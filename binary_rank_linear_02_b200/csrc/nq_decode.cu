@@ -249,6 +249,54 @@ __device__ __forceinline__ void build_fragments(uint4* frag, Misc& mi, Val val, 
     }
 }
 
+// The same fragments and sums for two token groups (5..8 tokens), column-major: a thread
+// forms each of its columns' scale once and quantises every token of the column, with the
+// per-token sums of q in registers and one warp reduction per token at the end (fewer
+// instructions than one pass per token).  value = val(tok, col) * scale(col).
+template <int NT, typename Val, typename Scale>
+__device__ __forceinline__ void build_fragments2(uint4* frag, Misc& mi, Val val, Scale scale, int ncb, int batch) {
+    const int tasks = ncb * 32;
+    int qs[8];
+    float up[8];
+#pragma unroll
+    for (int tok = 0; tok < 8; ++tok) {
+        qs[tok] = 0;
+        up[tok] = tok < batch ? mi.up[tok] : 0.f;
+    }
+    for (int task = threadIdx.x; task < tasks; task += NT) {
+        const int j = task & 7, t = (task >> 3) & 3, cb = task >> 5;
+        const int s4 = j >> 1, h = j & 1;
+        const int col = cb * kCB + 32 * t + s4 + 4 * h;
+        float sc[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sc[c] = scale(col + 8 * c);
+#pragma unroll
+        for (int tok = 0; tok < 8; ++tok) {
+            if (tok < batch) {
+                uint32_t wh = 0, wl = 0;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int q = quantise(val(tok, col + 8 * c) * sc[c], up[tok]);
+                    qs[tok] += q;
+                    wh |= (uint32_t)((q >> 7) & 0xFF) << (8 * c);
+                    wl |= (uint32_t)(q & 0x7F) << (8 * c);
+                }
+                const int tg = tok >> 2, ti = tok & 3;
+                reinterpret_cast<uint32_t*>(frag_ptr<2>(frag, cb, tg, j >> 2, 8 * ti + t))[j & 3] = wh;
+                reinterpret_cast<uint32_t*>(frag_ptr<2>(frag, cb, tg, j >> 2, 8 * ti + 4 + t))[j & 3] = wl;
+            }
+        }
+    }
+#pragma unroll
+    for (int tok = 0; tok < 8; ++tok) {
+        if (tok < batch) {
+            int v = qs[tok];
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if ((threadIdx.x & 31) == 0 && v != 0) atomicAdd(&mi.qsum[tok], v);
+        }
+    }
+}
+
 // One column block of a 16-row tile into accumulator set `acc`.
 template <int NTG>
 __device__ __forceinline__ void cb_mma(const uint4* frag, uint32_t wa, uint32_t wb, int cb, int lane,
@@ -455,11 +503,30 @@ stage1_kernel(const __grid_constant__ DecGroup grp) {
         // maxima are combined
         const uint16_t* ss = xchunk(buf, batch);
         auto val = [&](int tok, int c) { return bf16_to_f32(xchunk(buf, tok)[c]) * f16_to_f32(ss[c]); };
-        for (int tok = 0; tok < batch; ++tok) {
-            float mx = 0.f;
-            for (int c = threadIdx.x; c < ccols; c += kThreads1) mx = fmaxf(mx, fabsf(val(tok, c)));
-            mx = warp_max(mx);
-            if (lane == 0) mi.red[warp][tok] = mx;
+        if constexpr (NTG == 2) {  // column-major: each column's scale once for all tokens
+            float mxv[8];
+#pragma unroll
+            for (int tok = 0; tok < 8; ++tok) mxv[tok] = 0.f;
+            for (int c = threadIdx.x; c < ccols; c += kThreads1) {
+                const float sc = f16_to_f32(ss[c]);
+#pragma unroll
+                for (int tok = 0; tok < 8; ++tok)
+                    if (tok < batch) mxv[tok] = fmaxf(mxv[tok], fabsf(bf16_to_f32(xchunk(buf, tok)[c]) * sc));
+            }
+#pragma unroll
+            for (int tok = 0; tok < 8; ++tok) {
+                if (tok < batch) {
+                    const float mx = warp_max(mxv[tok]);
+                    if (lane == 0) mi.red[warp][tok] = mx;
+                }
+            }
+        } else {
+            for (int tok = 0; tok < batch; ++tok) {
+                float mx = 0.f;
+                for (int c = threadIdx.x; c < ccols; c += kThreads1) mx = fmaxf(mx, fabsf(val(tok, c)));
+                mx = warp_max(mx);
+                if (lane == 0) mi.red[warp][tok] = mx;
+            }
         }
         __syncthreads();
         if (threadIdx.x < batch) {
@@ -472,7 +539,12 @@ stage1_kernel(const __grid_constant__ DecGroup grp) {
             mi.qsum[tok] = 0;
         }
         __syncthreads();
-        build_fragments<NTG, kThreads1>(frag, mi, val, ncb, batch);
+        if constexpr (NTG == 2)
+            build_fragments2<kThreads1>(
+                frag, mi, [&](int tok, int c) { return bf16_to_f32(xchunk(buf, tok)[c]); },
+                [&](int c) { return f16_to_f32(ss[c]); }, ncb, batch);
+        else
+            build_fragments<NTG, kThreads1>(frag, mi, val, ncb, batch);
         __syncthreads();
 
         int acc[TPW][NTG][4][4];
@@ -768,8 +840,11 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
         __syncthreads();
         // every column block of the span at once: one barrier, then an uninterrupted MMA loop
         const int ncb = min(r2, r - sc * r2) / kCB;
-        build_fragments<NTG, kThreads>(
-            frag, mi, [&](int tok, int c) { return tbuf[tok * s2_t_row(r2) + c + 8 * (c >> 5)]; }, ncb, batch);
+        auto tval = [&](int tok, int c) { return tbuf[tok * s2_t_row(r2) + c + 8 * (c >> 5)]; };
+        if constexpr (NTG == 2)
+            build_fragments2<kThreads>(frag, mi, tval, [](int) { return 1.0f; }, ncb, batch);
+        else
+            build_fragments<NTG, kThreads>(frag, mi, tval, ncb, batch);
         __syncthreads();
         // the span's units (tile, column block) in tile-major order, an even run per warp;
         // a run covers the ends of up to a few tiles, each added into bq when done
