@@ -419,9 +419,9 @@ template <int TPW>
 __host__ __device__ constexpr int s1_threads() { return 32 * kRowsS1 / (16 * TPW); }
 
 // CM: the column-major fragment build (always for two token groups; for one token group the
-// host picks it from kColMajorMinBatch tokens.  Measured per 7B step: 4 tokens 23.9 -> 22.6
-// us, 70B block at 4 tokens 65.9 -> 63.1 us; 2 tokens 17.3 against 17.4 us, and a single
-// token slower with it, so those keep the token-major build)
+// host picks it from kColMajorMinBatch tokens.  Measured per 7B step: 3 tokens 21.7 -> 21.3
+// us, 4 tokens 23.9 -> 22.6 us, 70B block at 4 tokens 65.9 -> 63.1 us; 2 tokens 17.3 against
+// 17.4 us, and a single token slower with it, so those keep the token-major build)
 template <int NTG, int TPW, bool CM = false>
 __global__ void __launch_bounds__(s1_threads<TPW>(), TPW == 1 ? 4 : (NTG == 1 ? 8 : 4))
 stage1_kernel(const __grid_constant__ DecGroup grp) {
