@@ -444,3 +444,28 @@ def test_grouped_pinned_repeated_calls(nq, orc, batch):
             for i, c in enumerate(cases):
                 want = orc.lowrank_linear_fwd(xs[i], c.Upk_o, c.Vpk_o, c.s1, c.s2, c.m, c.n, c.r)
                 assert rel_err(yh[i].numpy(), want) <= TOL, (k, i)
+
+
+@pytest.mark.parametrize("batch", [2, 3, 4, 5, 8, 12])
+def test_tokens_are_independent(nq, orc, batch):
+    """Each token's result does not depend on the other tokens of the call: every row of a
+    grouped decode call of 2..12 tokens (one and two token groups, the token-major and the
+    column-major fragment builds, one and several stage-2 spans, the stage-2 sum of the
+    split partials and the stage-1 hand-off, token chunks above 8) equals, bit for bit, the
+    same grouped call on that token alone."""
+    shapes = [(512, 512, 128), (384, 640, 256), (11008, 4096, 2432)]
+    cases = [Case(orc, nq, m, n, r, batch, seed=3100 + 10 * batch + i) for i, (m, n, r) in enumerate(shapes)]
+    ys = [torch.empty((batch, c.m), dtype=torch.float32, device="cuda") for c in cases]
+    nq.lowrank_linear_fwd_grouped([(c.x_d, c.Upk, c.Vpk, c.s1_d, c.s2_d, y, c.m, c.n, c.r)
+                                   for c, y in zip(cases, ys)], batch)
+    singles = []
+    for b in range(batch):
+        y1 = [torch.empty((1, c.m), dtype=torch.float32, device="cuda") for c in cases]
+        nq.lowrank_linear_fwd_grouped([(c.x_d[b:b + 1], c.Upk, c.Vpk, c.s1_d, c.s2_d, y, c.m, c.n, c.r)
+                                       for c, y in zip(cases, y1)], 1)
+        singles.append(y1)
+    torch.cuda.synchronize()
+    for i, (c, y) in enumerate(zip(cases, ys)):
+        got = y.cpu().numpy()
+        assert np.array_equal(got, np.concatenate([s[i].cpu().numpy() for s in singles])), (i, batch)
+        assert rel_err(got, c.oracle(orc)) <= TOL
