@@ -26,16 +26,33 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Memory kind of a pointer: 1 = device-accessible (device or managed), 0 = host.
-// Without a usable device every pointer is a host pointer.
+// Memory kind of a pointer: kDeviceMem = memory this call's kernels may read (device
+// memory of the current device, or managed memory), kHostMem = host memory (pageable or
+// pinned), kForeignMem = device memory of another GPU, which a kernel launched on the
+// current device must not be given (without peer access it faults): every entry point
+// rejects it with NQ_ERR_PTRKIND before anything is enqueued.  Without a usable device
+// every pointer is a host pointer.
+constexpr int kHostMem = 0, kDeviceMem = 1, kForeignMem = -1;
+
+int classify(const cudaPointerAttributes& attr) {
+    if (attr.type == cudaMemoryTypeManaged) return kDeviceMem;
+    if (attr.type != cudaMemoryTypeDevice) return kHostMem;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return kForeignMem;
+    }
+    return attr.device == dev ? kDeviceMem : kForeignMem;
+}
+
 int pointer_kind(const void* p) {
     cudaPointerAttributes attr;
     cudaError_t err = cudaPointerGetAttributes(&attr, p);
     if (err != cudaSuccess) {
         cudaGetLastError();
-        return 0;
+        return kHostMem;
     }
-    return (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) ? 1 : 0;
+    return classify(attr);
 }
 
 // One query for x or y: the kind as pointer_kind, and for page-locked (pinned) host memory
@@ -45,11 +62,11 @@ int pointer_kind_pinned(const void* p, void** pinned) {
     cudaPointerAttributes attr;
     if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
         cudaGetLastError();
-        return 0;
+        return kHostMem;
     }
-    if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) return 1;
-    if (attr.type == cudaMemoryTypeHost) *pinned = attr.devicePointer;
-    return 0;
+    const int kind = classify(attr);
+    if (kind == kHostMem && attr.type == cudaMemoryTypeHost) *pinned = attr.devicePointer;
+    return kind;
 }
 
 }  // namespace
@@ -106,6 +123,7 @@ Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, const D
     const size_t o_status = off;   off = align_up(off + sizeof(unsigned) * 64, 256);
     const size_t o_xp = off;       off = align_up(off + sizeof(uint16_t) * (size_t)b_cap * n_cap, 256);
     const size_t o_T = off;        off = align_up(off + sizeof(uint16_t) * (size_t)b_cap * r_cap, 256);
+    const size_t o_xs = off;       off = align_up(off + sizeof(float) * (size_t)(b_cap + 1), 256);
     char* base = nullptr;
     if (cudaMalloc(&base, off) != cudaSuccess) {
         cudaGetLastError();
@@ -130,6 +148,7 @@ Workspace* workspace_for(int64_t m, int64_t n, int64_t r, int64_t batch, const D
     w.status = reinterpret_cast<unsigned*>(base + o_status);
     w.xprime = reinterpret_cast<uint16_t*>(base + o_xp);
     w.T = reinterpret_cast<uint16_t*>(base + o_T);
+    w.xscale = reinterpret_cast<float*>(base + o_xs);
     w.t_cap = t_cap;
     w.tgmax_cap = g_cap;
     w.partial_cap = p_cap;
@@ -329,13 +348,16 @@ static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_line
     size_t xbytes = 0, ybytes = 0;
     for (int i = 0; i < count; ++i) {
         const nq_linear_desc& L = desc(i);
-        if (!pointer_kind(L.Upk) || !pointer_kind(L.Vpk) || !pointer_kind(L.s1) || !pointer_kind(L.s2))
+        if (pointer_kind(L.Upk) != kDeviceMem || pointer_kind(L.Vpk) != kDeviceMem ||
+            pointer_kind(L.s1) != kDeviceMem || pointer_kind(L.s2) != kDeviceMem)
             return NQ_ERR_PTRKIND;
         void *xp = nullptr, *yp = nullptr;
-        x_host[i] = pointer_kind_pinned(L.x, &xp) == 0;
-        y_host[i] = pointer_kind_pinned(L.y, &yp) == 0;
-        if (ex && (x_host[i] || y_host[i] || (ex[i].y_bf16 && !pointer_kind(ex[i].y_bf16)) ||
-                   (ex[i].y_rmsnorm_bf16 && !pointer_kind(ex[i].y_rmsnorm_bf16))))
+        const int kx = pointer_kind_pinned(L.x, &xp), ky = pointer_kind_pinned(L.y, &yp);
+        if (kx == kForeignMem || ky == kForeignMem) return NQ_ERR_PTRKIND;
+        x_host[i] = kx == kHostMem;
+        y_host[i] = ky == kHostMem;
+        if (ex && (x_host[i] || y_host[i] || (ex[i].y_bf16 && pointer_kind(ex[i].y_bf16) != kDeviceMem) ||
+                   (ex[i].y_rmsnorm_bf16 && pointer_kind(ex[i].y_rmsnorm_bf16) != kDeviceMem)))
             return NQ_ERR_PTRKIND;
         if (x_host[i]) {
             x_pin[i] = xp;
@@ -484,14 +506,14 @@ static int grouped_run(const nq_linear_desc* first, size_t stride, const nq_line
             return NQ_ERR_CUDA;
         }
         std::vector<uint64_t> key;
-        key.reserve(8 + 12 * (size_t)count);
+        key.reserve(8 + 13 * (size_t)count);
         auto u = [](const void* p) { return (uint64_t)reinterpret_cast<uintptr_t>(p); };
         key.insert(key.end(), {(uint64_t)dev, ws_generation(), (uint64_t)batch, (uint64_t)count, ex ? 1ull : 0ull,
                                u(ws->base), u(ws->xstage), u(ws->ystage)});
         for (int i = 0; i < count; ++i) {
             const nq_linear_desc& L = desc(i);
             key.insert(key.end(), {u(L.x), u(L.Upk), u(L.Vpk), u(L.s1), u(L.s2), u(L.y), (uint64_t)L.m, (uint64_t)L.n,
-                                   (uint64_t)L.r, u(x_pin[i]), u(ex ? ex[i].y_bf16 : nullptr),
+                                   (uint64_t)L.r, u(x_pin[i]), u(y_pin[i]), u(ex ? ex[i].y_bf16 : nullptr),
                                    u(ex ? ex[i].y_rmsnorm_bf16 : nullptr)});
         }
         st = launch_cached(dev, key, s, launch);
@@ -529,7 +551,8 @@ const char* nq_status_string(int status) {
         case NQ_ERR_CUDA: return "NQ_ERR_CUDA: a CUDA call or kernel launch failed";
         case NQ_ERR_TIMEOUT: return "NQ_ERR_TIMEOUT: a bounded device-side wait gave up";
         case NQ_ERR_NOMEM: return "NQ_ERR_NOMEM: workspace allocation failed (or was needed during stream capture)";
-        case NQ_ERR_PTRKIND: return "NQ_ERR_PTRKIND: pointers of mixed or unsupported memory kinds";
+        case NQ_ERR_PTRKIND:
+            return "NQ_ERR_PTRKIND: pointers of mixed or unsupported memory kinds (or device memory of another GPU)";
         case NQ_ERR_NOALLOC_LIMIT:
             return "NQ_ERR_NOALLOC_LIMIT: nq_lowrank_linear_fwd_noalloc takes 1 <= batch <= 8 and r <= 4096 "
                    "(its scratch is a fixed array)";
@@ -549,9 +572,9 @@ int nq_pack_signs(const int8_t* signs, int64_t rows, int64_t cols, uint32_t* out
     if (!signs || !out) return NQ_ERR_NULL;
     if (rows > (int64_t(1) << 40) / cols) return NQ_ERR_SHAPE;
     const int ks = pointer_kind(signs), ko = pointer_kind(out);
-    if (ks != ko) return NQ_ERR_PTRKIND;
+    if (ks != ko || ks == kForeignMem) return NQ_ERR_PTRKIND;
     const int64_t wpr = (cols + 31) / 32;
-    if (ks == 0) {
+    if (ks == kHostMem) {
         for (int64_t i = 0; i < rows * cols; ++i)
             if (signs[i] < -1 || signs[i] > 1) return NQ_ERR_VALUE;
         for (int64_t row = 0; row < rows; ++row) {
@@ -586,9 +609,9 @@ int nq_unpack_signs(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* 
     if (!packed || !out) return NQ_ERR_NULL;
     if (rows > (int64_t(1) << 40) / cols) return NQ_ERR_SHAPE;
     const int kp = pointer_kind(packed), ko = pointer_kind(out);
-    if (kp != ko) return NQ_ERR_PTRKIND;
+    if (kp != ko || kp == kForeignMem) return NQ_ERR_PTRKIND;
     const int64_t wpr = (cols + 31) / 32;
-    if (kp == 0) {
+    if (kp == kHostMem) {
         for (int64_t row = 0; row < rows; ++row)
             for (int64_t c = 0; c < cols; ++c)
                 out[row * cols + c] = ((packed[row * wpr + c / 32] >> (c % 32)) & 1u) ? 1 : -1;
@@ -603,9 +626,9 @@ int nq_transpose_signs(const uint32_t* packed, int64_t rows, int64_t cols, uint3
     if (!packed || !out) return NQ_ERR_NULL;
     if (rows > (int64_t(1) << 40) / cols) return NQ_ERR_SHAPE;
     const int kp = pointer_kind(packed), ko = pointer_kind(out);
-    if (kp != ko) return NQ_ERR_PTRKIND;
+    if (kp != ko || kp == kForeignMem) return NQ_ERR_PTRKIND;
     const int64_t wpr_in = (cols + 31) / 32, wpr_out = (rows + 31) / 32;
-    if (kp == 0) {
+    if (kp == kHostMem) {
         memset(out, 0, sizeof(uint32_t) * (size_t)(cols * wpr_out));
         for (int64_t row = 0; row < rows; ++row)
             for (int64_t c = 0; c < cols; ++c)
@@ -637,7 +660,7 @@ int nq_lowrank_linear_bwd_scales(const void* x, const void* dy, const uint32_t* 
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return NQ_ERR_ALIGN;
     for (const void* p : ptrs)
-        if (p && !pointer_kind(p)) return NQ_ERR_PTRKIND;
+        if (p && pointer_kind(p) != kDeviceMem) return NQ_ERR_PTRKIND;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (batch == 0) {  // empty sums
         if (ds1 && cudaMemsetAsync(ds1, 0, sizeof(float) * (size_t)m, s) != cudaSuccess) return NQ_ERR_CUDA;
@@ -679,7 +702,7 @@ int nq_lowrank_linear_bwd_factors(const void* x, const void* dy, const uint32_t*
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return NQ_ERR_ALIGN;
     for (const void* p : ptrs)
-        if (p && !pointer_kind(p)) return NQ_ERR_PTRKIND;
+        if (p && pointer_kind(p) != kDeviceMem) return NQ_ERR_PTRKIND;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (batch == 0) {  // empty sums
         if (dU && cudaMemsetAsync(dU, 0, sizeof(float) * (size_t)(m * r), s) != cudaSuccess) return NQ_ERR_CUDA;
@@ -717,7 +740,7 @@ int nq_cast_f32_to_bf16(const float* src, int64_t count, void* dst, void* stream
     if (count == 0) return NQ_OK;
     if (!src || !dst) return NQ_ERR_NULL;
     if (!aligned16(src) || !aligned16(dst)) return NQ_ERR_ALIGN;
-    if (!pointer_kind(src) || !pointer_kind(dst)) return NQ_ERR_PTRKIND;
+    if (pointer_kind(src) != kDeviceMem || pointer_kind(dst) != kDeviceMem) return NQ_ERR_PTRKIND;
     return cast_f32_bf16_device(src, count, static_cast<uint16_t*>(dst), static_cast<cudaStream_t>(stream));
 }
 
@@ -726,7 +749,7 @@ int nq_rms_normalize_bf16(const float* src, int64_t rows, int64_t cols, void* ds
     if (rows == 0) return NQ_OK;
     if (!src || !dst) return NQ_ERR_NULL;
     if (!aligned16(src) || !aligned16(dst)) return NQ_ERR_ALIGN;
-    if (!pointer_kind(src) || !pointer_kind(dst)) return NQ_ERR_PTRKIND;
+    if (pointer_kind(src) != kDeviceMem || pointer_kind(dst) != kDeviceMem) return NQ_ERR_PTRKIND;
     return rms_normalize_bf16_device(src, rows, cols, static_cast<uint16_t*>(dst), static_cast<cudaStream_t>(stream));
 }
 
@@ -785,7 +808,8 @@ int nq_lowrank_linear_fwd(const void* x, const uint32_t* Upk, const uint32_t* Vp
     if (!aligned16(x) || !aligned16(Upk) || !aligned16(Vpk) || !aligned16(s1) || !aligned16(s2) ||
         !aligned16(y))
         return NQ_ERR_ALIGN;
-    if (!pointer_kind(Upk) || !pointer_kind(Vpk) || !pointer_kind(s1) || !pointer_kind(s2))
+    if (pointer_kind(Upk) != kDeviceMem || pointer_kind(Vpk) != kDeviceMem || pointer_kind(s1) != kDeviceMem ||
+        pointer_kind(s2) != kDeviceMem)
         return NQ_ERR_PTRKIND;
     // one layer of the grouped path, which also handles host x / y
     nq_linear_desc d;

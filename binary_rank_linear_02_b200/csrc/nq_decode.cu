@@ -1180,9 +1180,9 @@ int decode_rank_vector(const uint16_t* x, const uint32_t* Vpk, const uint16_t* s
 // Allocation-free decode entry point.
 //
 // Some callers cannot allocate device memory at the moment they run a layer: an inference
-// engine that sized and froze its memory pool at start-up, a process whose allocator is
-// owned by another framework, or code running under a stream capture that must not call
-// cudaMalloc.  For them nq_lowrank_linear_fwd_noalloc keeps the decode path's scratch
+// engine that sized and froze its memory pool at start-up (any later cudaMalloc competes
+// with the pool for the same HBM and may fail mid-request), or a process whose allocator is
+// owned by another framework (a side allocation bypasses its accounting).  For them nq_lowrank_linear_fwd_noalloc keeps the decode path's scratch
 // (t, the per-block maxima of |t|, the stage-1 split partials and arrival counters) in one
 // fixed array of device memory that is part of this library's module, so a call allocates
 // nothing.
@@ -1204,7 +1204,8 @@ constexpr size_t kNoAllocT = (size_t)NQ_DECODE_MAX_BATCH * kNoAllocMaxRank;
 constexpr size_t kNoAllocG = (size_t)NQ_DECODE_MAX_BATCH * (kNoAllocMaxRank / kRowsS1);
 constexpr size_t kNoAllocP = (size_t)kNoAllocMaxSplits * NQ_DECODE_MAX_BATCH * kNoAllocMaxRank;
 constexpr size_t kNoAllocC = kNoAllocMaxRank / kRowsS1;
-constexpr size_t kNoAllocBytes = 4 * (kNoAllocT + kNoAllocG + kNoAllocP + kNoAllocC);  // 1.16 MB
+constexpr size_t kNoAllocBytes = 4 * (kNoAllocT + kNoAllocG + kNoAllocP + kNoAllocC);
+static_assert(kNoAllocBytes == 1180800, "the scratch size stated in nq.h");
 
 }  // namespace
 }  // namespace nq
@@ -1231,13 +1232,17 @@ int noalloc_scratch(int dev, void** out) {
     return NQ_OK;
 }
 
-bool is_device_memory(const void* p) {
+// Memory the kernels launched on device `dev` may read: device memory of `dev` itself, or
+// managed memory.  Device memory of another GPU is refused (without peer access a kernel
+// given it faults), as is host memory.
+bool is_device_memory(const void* p, int dev) {
     cudaPointerAttributes attr;
     if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
         cudaGetLastError();
         return false;
     }
-    return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+    if (attr.type == cudaMemoryTypeManaged) return true;
+    return attr.type == cudaMemoryTypeDevice && attr.device == dev;
 }
 
 }  // namespace
@@ -1258,14 +1263,14 @@ extern "C" int nq_lowrank_linear_fwd_noalloc(const void* x, const uint32_t* Upk,
                         reinterpret_cast<uintptr_t>(Vpk) | reinterpret_cast<uintptr_t>(s1) |
                         reinterpret_cast<uintptr_t>(s2) | reinterpret_cast<uintptr_t>(y);
     if (a & 15u) return NQ_ERR_ALIGN;
-    if (!is_device_memory(x) || !is_device_memory(Upk) || !is_device_memory(Vpk) || !is_device_memory(s1) ||
-        !is_device_memory(s2) || !is_device_memory(y))
-        return NQ_ERR_PTRKIND;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
         return NQ_ERR_CUDA;
     }
+    if (!is_device_memory(x, dev) || !is_device_memory(Upk, dev) || !is_device_memory(Vpk, dev) ||
+        !is_device_memory(s1, dev) || !is_device_memory(s2, dev) || !is_device_memory(y, dev))
+        return NQ_ERR_PTRKIND;
     void* scratch = nullptr;
     int st = noalloc_scratch(dev, &scratch);
     if (st != NQ_OK) return st;
