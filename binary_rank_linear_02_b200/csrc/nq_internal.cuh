@@ -28,6 +28,7 @@ struct Workspace {
     unsigned* status = nullptr;    // [0]: pack value check, [1]: device wait timeout
     uint16_t* xprime = nullptr;    // [batch_cap][n_cap] fp16 (prefill)
     uint16_t* T = nullptr;         // [batch_cap][r_cap] fp16 (prefill)
+    float* xscale = nullptr;       // [batch_cap] (prefill: 2^e per token, the power of two x' and T carry)
     void* xstage = nullptr;        // staged host x
     float* ystage = nullptr;       // staged host y
     size_t xstage_bytes = 0, ystage_bytes = 0;

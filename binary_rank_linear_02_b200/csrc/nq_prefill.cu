@@ -1,9 +1,13 @@
 // nq_prefill.cu -- prefill path (batch > 8): the factorised linear as two dense
 // tensor-core GEMMs on tcgen05 (hardwired.dev section "Cisla": binary GEMM kernels).
 //
-//   prescale : x'[b][.] = fp16(s2 (.) x[b])                    (elementwise, K-permuted)
+//   prescale : x'[b][.] = fp16(2^-e_b s2 (.) x[b])             (per token row, K-permuted)
 //   GEMM 1   : T[b][k]  = sum_j V^T[k][j] x'[b][j]             M = r, N = batch, K = n
-//   GEMM 2   : y[b][i]  = s1_i * sum_k U[i][k] T[b][k]         M = m, N = batch, K = r
+//   GEMM 2   : y[b][i]  = 2^e_b s1_i * sum_k U[i][k] T[b][k]   M = m, N = batch, K = r
+//
+// 2^-e_b is a power of two per token that keeps x' and T inside fp16's normal range
+// (below 2^15 in magnitude) whatever the token's scale; it is undone exactly in GEMM 2's
+// epilogue.
 //
 // Weights are the MMA's A operand (M = 128 rows per CTA), tokens its B operand (N = BN
 // per CTA).  A is never stored expanded in memory: four "expander" warps read the packed
@@ -229,6 +233,7 @@ struct GemmArgs {
     uint16_t* T_out;      // EPI 0: T[b][perm(k)] fp16
     float* y_out;         // EPI 1: y[b][i] fp32
     const uint16_t* s1;   // EPI 1
+    const float* yscale;  // EPI 1: 2^e_b per token (the prescale's power of two, undone here)
     float* partials;      // split items: [row block][split][row][256 columns] fp32
     int* counters;        // split items: arrivals per row block, zero between calls
     unsigned* status;
@@ -322,7 +327,7 @@ __device__ __forceinline__ void store_out(const GemmArgs& a, int64_t b, int64_t 
     if (EPI == 0)
         a.T_out[b * a.mdim + tcol] = __half_as_ushort(__float2half_rn(d));
     else
-        a.y_out[b * a.mdim + grow] = s1v * d;
+        a.y_out[b * a.mdim + grow] = s1v * d * __ldg(a.yscale + b);
 }
 
 template <int EPI>
@@ -614,8 +619,8 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(kTileThreads, 2)
 tile_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint32_t* __restrict__ Wpk, int64_t kdim,
             int64_t mdim, int64_t batch, uint16_t* __restrict__ T_out, float* __restrict__ y_out,
-            const uint16_t* __restrict__ s1, unsigned* __restrict__ status, int* __restrict__ sync, int bn1,
-            int ntt1, int nrb1, int handoff) {
+            const uint16_t* __restrict__ s1, const float* __restrict__ yscale, unsigned* __restrict__ status,
+            int* __restrict__ sync, int bn1, int ntt1, int nrb1, int handoff) {
     using G = Geometry<BN>;
     constexpr int S = G::kStages;
     extern __shared__ unsigned char smem_raw[];
@@ -785,7 +790,7 @@ tile_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint32_t* __res
                         if (EPI == 0)
                             T_out[b * mdim + tcol] = __half_as_ushort(__float2half_rn(d));
                         else
-                            y_out[b * mdim + grow] = s1v * d;
+                            y_out[b * mdim + grow] = s1v * d * __ldg(yscale + b);
                     }
                 }
             }
@@ -824,41 +829,78 @@ __global__ void wait_selftest_kernel(unsigned long long limit_ns, unsigned* stat
     if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, status, limit_ns);
 }
 
-// x'[b][perm(j)] = fp16(bf16 x[b][j] * fp16 s2[j]); one thread per 32-column group.
-__global__ void prescale_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ s2, int64_t n,
-                                int64_t batch, uint16_t* __restrict__ xp) {
+// x'[b][perm(j)] = fp16(2^-e_b * bf16 x[b][j] * fp16 s2[j]) and xscale[b] = 2^e_b: one CTA
+// per token row at a time.  The power of two is chosen per token from the row's sum
+// L_b = sum_j |s2_j x[b][j]| (fp32) so that 2^-e_b L_b < 2^15: every |x'| and every entry
+// of T = V^T x' (each a signed sum of the x') then stays below 2^15 < 65504, so neither
+// overflows fp16, and every token uses fp16's normal range down to 2^-29 L_b whatever its
+// magnitude (without it a token of small activations falls into fp16's subnormals and a
+// token of large ones overflows T).  GEMM 2's epilogue multiplies by 2^e_b, which is exact,
+// so the result is that of the unscaled operands up to their rounding.
+constexpr int kPrescaleThreads = 128;
+
+__device__ __forceinline__ float prescale_pow2(int k) { return __int_as_float((k + 127) << 23); }  // |k| <= 126
+
+__global__ void __launch_bounds__(kPrescaleThreads)
+prescale_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ s2, int64_t n, int64_t batch,
+                uint16_t* __restrict__ xp, float* __restrict__ xscale) {
+    __shared__ float red[kPrescaleThreads / 32];
     const int64_t groups = n / 32;
-    const int64_t total = batch * groups;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
-    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
-         idx += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t b = idx / groups, g = idx % groups;
-        const uint4* xs = reinterpret_cast<const uint4*>(x + b * n + g * 32);
-        const uint4* ss = reinterpret_cast<const uint4*>(s2 + g * 32);
-        uint32_t xv[16], sv[16], out[16];
+    for (int64_t b = blockIdx.x; b < batch; b += gridDim.x) {
+        const uint16_t* xrow = x + b * n;
+        // column c of a group sits in half (c & 1) of word c / 2
+        auto load = [&](int64_t g, uint32_t (&xv)[16], uint32_t (&sv)[16]) {
+            const uint4* xs = reinterpret_cast<const uint4*>(xrow + g * 32);
+            const uint4* ss = reinterpret_cast<const uint4*>(s2 + g * 32);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint4 a = __ldg(xs + i), c = __ldg(ss + i);
-            xv[4 * i] = a.x; xv[4 * i + 1] = a.y; xv[4 * i + 2] = a.z; xv[4 * i + 3] = a.w;
-            sv[4 * i] = c.x; sv[4 * i + 1] = c.y; sv[4 * i + 2] = c.z; sv[4 * i + 3] = c.w;
-        }
-        // column c sits in half (c & 1) of word c / 2; output pair q = (column q, column q+16)
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            uint32_t pair = 0;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int c = q + 16 * h;
-                const uint16_t xb = (uint16_t)(xv[c >> 1] >> (16 * (c & 1)));
-                const uint16_t sb = (uint16_t)(sv[c >> 1] >> (16 * (c & 1)));
-                const float v = __uint_as_float((uint32_t)xb << 16) * __half2float(__ushort_as_half(sb));
-                pair |= (uint32_t)__half_as_ushort(__float2half_rn(v)) << (16 * h);
+            for (int i = 0; i < 4; ++i) {
+                const uint4 a = __ldg(xs + i), c = __ldg(ss + i);
+                xv[4 * i] = a.x; xv[4 * i + 1] = a.y; xv[4 * i + 2] = a.z; xv[4 * i + 3] = a.w;
+                sv[4 * i] = c.x; sv[4 * i + 1] = c.y; sv[4 * i + 2] = c.z; sv[4 * i + 3] = c.w;
             }
-            out[q] = pair;
-        }
-        uint4* o = reinterpret_cast<uint4*>(xp + b * n + g * 32);
+        };
+        auto value = [](const uint32_t (&xv)[16], const uint32_t (&sv)[16], int c) {
+            const uint16_t xb = (uint16_t)(xv[c >> 1] >> (16 * (c & 1)));
+            const uint16_t sb = (uint16_t)(sv[c >> 1] >> (16 * (c & 1)));
+            return __uint_as_float((uint32_t)xb << 16) * __half2float(__ushort_as_half(sb));  // exact in fp32
+        };
+        float l1 = 0.f;
+        for (int64_t g = threadIdx.x; g < groups; g += kPrescaleThreads) {
+            uint32_t xv[16], sv[16];
+            load(g, xv, sv);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) o[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+            for (int c = 0; c < 32; ++c) l1 += fabsf(value(xv, sv, c));
+        }
+        for (int o = 16; o > 0; o >>= 1) l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+        if (lane == 0) red[warp] = l1;
+        __syncthreads();
+        float total = 0.f;
+#pragma unroll
+        for (int w = 0; w < kPrescaleThreads / 32; ++w) total += red[w];
+        __syncthreads();  // red is rewritten for the next row
+        int e = 0;
+        frexpf(total, &e);  // total < 2^e (e = 0 for a zero row)
+        e = min(max(e - 15, -110), 112);
+        const float down = prescale_pow2(-e);
+        if (threadIdx.x == 0) xscale[b] = prescale_pow2(e);
+        for (int64_t g = threadIdx.x; g < groups; g += kPrescaleThreads) {
+            uint32_t xv[16], sv[16], out[16];
+            load(g, xv, sv);
+            // output pair q = (column q, column q+16)
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                uint32_t pair = 0;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    pair |= (uint32_t)__half_as_ushort(__float2half_rn(value(xv, sv, q + 16 * h) * down)) << (16 * h);
+                out[q] = pair;
+            }
+            uint4* o = reinterpret_cast<uint4*>(xp + b * n + g * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+        }
     }
     pdl_trigger();
 }
@@ -972,6 +1014,7 @@ int launch_gemm(const CUtensorMap& map, const uint32_t* Wpk, int64_t M, int64_t 
     a.T_out = T_out;
     a.y_out = y_out;
     a.s1 = s1;
+    a.yscale = ws->xscale;
     a.partials = ws->partials;
     a.counters = ws->counters;
     a.status = ws->status + 1;
@@ -999,10 +1042,10 @@ int launch_gemm(const CUtensorMap& map, const uint32_t* Wpk, int64_t M, int64_t 
 
 cudaError_t launch_prescale(const uint16_t* x, const uint16_t* s2, int64_t n, int64_t batch, Workspace* ws,
                             cudaStream_t stream) {
-    const int64_t groups = batch * (n / 32);
-    int pblocks = (int)((groups + 255) / 256);
-    if (pblocks > 4 * sm_count()) pblocks = 4 * sm_count();
-    return launch_pdl(prescale_kernel, dim3(pblocks), dim3(256), 0, stream, x, s2, n, batch, ws->xprime);
+    const int64_t cap = 8 * (int64_t)sm_count();
+    const int pblocks = (int)(batch < cap ? batch : cap);
+    return launch_pdl(prescale_kernel, dim3(pblocks), dim3(kPrescaleThreads), 0, stream, x, s2, n, batch,
+                      ws->xprime, ws->xscale);
 }
 
 template <int BN, int EPI>
@@ -1024,8 +1067,8 @@ int launch_tile_gemm(const void* bsrc, int64_t K, const uint32_t* Wpk, int64_t M
     // the hand-off when GEMM 1's tiles exceed one wave (two CTAs per SM)
     const int handoff = (int64_t)nrb1 * ntt1 > 2 * (int64_t)sm_count() ? 1 : 0;
     return launch_pdl(tile_gemm_kernel<BN, EPI>, dim3((unsigned)(M / kBM), ntiles), dim3(kTileThreads),
-                      (size_t)G::kSmemBytes, stream, map, Wpk, K, M, batch, T_out, y_out, s1, ws->status + 1,
-                      ws->counters, bn1, ntt1, nrb1, handoff) == cudaSuccess
+                      (size_t)G::kSmemBytes, stream, map, Wpk, K, M, batch, T_out, y_out, s1,
+                      (const float*)ws->xscale, ws->status + 1, ws->counters, bn1, ntt1, nrb1, handoff) == cudaSuccess
                ? NQ_OK
                : NQ_ERR_CUDA;
 }

@@ -128,3 +128,40 @@ def chain_weights(nblocks: int, layers, seed: int):
                        scales_f16(n, seed, "chain", b, name, "s2"), m, n, r)
         blocks.append(w)
     return blocks
+
+
+# Activations with the value structure of real decoder activations, for accuracy tests at
+# the edges of the kernels' number formats.  All are drawn, then rounded to bfloat16.
+
+def activations_outliers_bf16(batch: int, n: int, seed: int, *tags, per_chunk: int = 3, chunk: int = 1024,
+                              lo: float = 1e2, hi: float = 1e4) -> np.ndarray:
+    """N(0, 1) activations in which `per_chunk` columns of every `chunk`-column block carry
+    outliers of magnitude log-uniform in [lo, hi] with a random sign (the few huge
+    "massive activation" channels of decoder hidden states), as bf16 bit patterns."""
+    g = _rng(seed, "x-outliers", batch, n, per_chunk, chunk, *tags)
+    z = g.standard_normal(size=(batch, n))
+    for c0 in range(0, n, chunk):
+        width = min(chunk, n - c0)
+        for b in range(batch):
+            cols = c0 + g.choice(width, size=min(per_chunk, width), replace=False)
+            mag = 10.0 ** g.uniform(np.log10(lo), np.log10(hi), size=cols.size)
+            z[b, cols] = np.where(g.integers(0, 2, size=cols.size) == 1, mag, -mag)
+    return f32_to_bf16_bits(z.astype(np.float32))
+
+
+def activations_wide_range_bf16(batch: int, n: int, seed: int, *tags, lo_exp: float = -20.0,
+                                hi_exp: float = 10.0) -> np.ndarray:
+    """Activations of magnitude 2^u, u uniform in [lo_exp, hi_exp], random signs: every
+    column block spans the whole dynamic range.  bf16 bit patterns."""
+    g = _rng(seed, "x-wide", batch, n, *tags)
+    mag = np.exp2(g.uniform(lo_exp, hi_exp, size=(batch, n)))
+    sign = np.where(g.integers(0, 2, size=(batch, n)) == 1, 1.0, -1.0)
+    return f32_to_bf16_bits((sign * mag).astype(np.float32))
+
+
+def activations_token_scaled_bf16(n: int, seed: int, token_scales, *tags) -> np.ndarray:
+    """One row per entry of `token_scales`: N(0, 1) activations times that factor, rounded
+    to bfloat16 (tokens of very different magnitude in one call)."""
+    sc = np.asarray(token_scales, dtype=np.float64)
+    z = _rng(seed, "x-token-scaled", sc.size, n, *tags).standard_normal(size=(sc.size, n))
+    return f32_to_bf16_bits((z * sc[:, None]).astype(np.float32))

@@ -27,6 +27,9 @@
  *      Upk: U as m rows of r/32 words         (row i = U[i][0..r))
  *      Vpk: V^T as r rows of n/32 words       (row k = V[0..n)[k])
  *  - x, s1, s2 hold IEEE bit patterns: x bfloat16, s1 and s2 binary16 (fp16).
+ *  - "Device memory" means memory of the device current on the calling thread, or managed
+ *    memory; device memory of another GPU is refused with NQ_ERR_PTRKIND before anything
+ *    is enqueued (a kernel given it without peer access would fault).
  *  - The library keeps one workspace per device (intermediate t = V^T (s2 (.) x) and
  *    a few counters).  It is allocated on the first call on a device and grown when a
  *    larger shape arrives; call nq_workspace_reserve() beforehand to keep allocation out
@@ -52,7 +55,8 @@ typedef enum {
     NQ_ERR_CUDA = -6,      /* a CUDA runtime/driver call or a launch failed */
     NQ_ERR_TIMEOUT = -7,   /* a bounded device-side wait gave up */
     NQ_ERR_NOMEM = -8,     /* workspace allocation failed */
-    NQ_ERR_PTRKIND = -9,   /* pointers of mixed or unsupported memory kinds */
+    NQ_ERR_PTRKIND = -9,   /* pointers of mixed or unsupported memory kinds, or device
+                              memory of a GPU other than the current one */
     NQ_ERR_NOALLOC_LIMIT = -10 /* size beyond nq_lowrank_linear_fwd_noalloc's fixed scratch */
 } nq_status;
 
@@ -105,8 +109,15 @@ int nq_unpack_signs(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* 
  * CUDA cores and integer tensor-core instructions, t kept in the workspace); larger
  * batches run the prefill path (two tcgen05 tensor-core GEMMs with the +1/-1 operands
  * expanded on chip, fp16 operands, fp32 accumulation).
- * Accuracy: max|y - y_exact| / max|y_exact| <= 2e-3 for the documented input ranges
- * (|s2_j x_j| and |t_k| below 6.0e4).
+ * Accuracy: max|y - y_exact| / max|y_exact| <= 2e-3, over the call and over each token
+ * alone (each token's error against its own largest output), for finite inputs in these
+ * ranges.  Decode: per token the largest |s2_j x_j| of every 1024-column chunk in
+ * [2^-90, 2^100] (each chunk is quantised to 14 bits under its own power of two, t under one
+ * per token).  Prefill: per token L = sum_j |s2_j x_j| in [2^-95, 2^126] (x' and T carry a
+ * power of two per token that keeps them below 2^15, inside fp16's normal range).
+ * Tested against an fp64 reference with N(0,1) activations, three outlier channels per
+ * 1024 columns at 1e2..1e4, magnitudes 2^-20..2^10 inside every chunk, tokens of 1e-20 to
+ * 1e20 in one call, |s2_j x_j| near 6e4 and near 2e-8, and zero tokens (exact zeros out).
  * Weights (Upk, Vpk, s1, s2) may be read before the work enqueued earlier on `stream`
  * has finished (programmatic dependent launch), so they must not be produced by the
  * kernel enqueued immediately before this call on the same stream; x may be.
@@ -279,16 +290,18 @@ int nq_lowrank_linear_fwd_grouped_ex(const nq_linear_desc_ex* layers, int count,
 
 /*
  * nq_lowrank_linear_fwd_noalloc -- the decode path of nq_lowrank_linear_fwd for callers
- * that cannot allocate device memory when they run a layer (an engine whose memory pool
- * is fixed at start-up, a host framework that owns the allocator, work recorded while
- * allocation is off limits).  It has no counterpart in the NanoQuant pages: it is a
- * property of this library, not of the method.
+ * that cannot allocate device memory when they run a layer: an inference engine that
+ * reserved its memory pool at start-up (a later cudaMalloc competes with that pool and can
+ * fail in the middle of a request), or a host framework that owns the allocator (a side
+ * allocation escapes its accounting).  It has no counterpart in the NanoQuant pages: it is
+ * a property of this library, not of the method.
  *   Same arguments, layout and result as nq_lowrank_linear_fwd, restricted to
  *   1 <= batch <= NQ_NOALLOC_MAX_BATCH and r <= NQ_NOALLOC_MAX_RANK (larger sizes return
- *   NQ_ERR_NOALLOC_LIMIT; batch 0 is a no-op).  Every pointer must be device memory.
- *   Scratch: a fixed 1.16 MB array compiled into the library's device code, held by every
- *   GPU that loads the library until the process exits.  The call allocates and frees
- *   nothing, on the host or the device.
+ *   NQ_ERR_NOALLOC_LIMIT; batch 0 is a no-op).  Every pointer must be device memory of the
+ *   current device (else NQ_ERR_PTRKIND, before anything is enqueued).
+ *   Scratch: a fixed array of 1,180,800 bytes (1.18 MB) compiled into the library's device
+ *   code, held by every GPU that loads the library until the process exits.  The call
+ *   allocates and frees nothing, on the host or the device.
  *   The first call on each device resolves the array's device address (with that device
  *   current); make that first call before any stream capture that includes this entry.
  *   All calls share the one array and each call overwrites it: calls whose kernels could

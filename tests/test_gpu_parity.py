@@ -469,3 +469,22 @@ def test_tokens_are_independent(nq, orc, batch):
         got = y.cpu().numpy()
         assert np.array_equal(got, np.concatenate([s[i].cpu().numpy() for s in singles])), (i, batch)
         assert rel_err(got, c.oracle(orc)) <= TOL
+
+
+@pytest.mark.skipif(not torch.cuda.is_available() or torch.cuda.device_count() < 2,
+                    reason="needs a second GPU to hold foreign device memory")
+def test_rejects_another_gpus_memory(nq, orc):
+    """Device memory of another GPU (no peer access is assumed) is refused on the host with
+    NQ_ERR_PTRKIND, before anything is launched: as weights, as x and as y."""
+    c = Case(orc, nq, 512, 512, 128, 1, seed=4100)
+    torch.cuda.set_device(0)
+    other = {k: v.to("cuda:1") for k, v in dict(x=c.x_d, Upk=c.Upk, s1=c.s1_d).items()}
+    y = torch.empty((1, 512), dtype=torch.float32, device="cuda:0")
+    y1 = torch.empty((1, 512), dtype=torch.float32, device="cuda:1")
+    h = torch.cuda.current_stream(0).cuda_stream
+    base = dict(x=c.x_d, Upk=c.Upk, Vpk=c.Vpk, s1=c.s1_d, s2=c.s2_d, y=y)
+    for key, val in list(other.items()) + [("y", y1)]:
+        a = dict(base, **{key: val})
+        st = nq.nq_lowrank_linear_fwd(a["x"].data_ptr(), a["Upk"].data_ptr(), a["Vpk"].data_ptr(), a["s1"].data_ptr(),
+                                      a["s2"].data_ptr(), 512, 512, 128, 1, a["y"].data_ptr(), h)
+        assert st == nq.NQ_ERR_PTRKIND, key
