@@ -1,19 +1,21 @@
 #!/usr/bin/env python
 """Benchmark of the factorised binary low-rank linear, y = s1 * (U (V^T (s2 * x))).
 
-Default workload (one "step"): the seven linears of a Llama-2-7B-shaped block
-(q/k/v/o 4096x4096 r=1664, gate/up 11008x4096 r=2432, down 4096x11008 r=2432) at decode
-batch 1, each layer with its own seeded input, all through the C ABI
-(nq_lowrank_linear_fwd) on one stream, the whole run captured in CUDA graphs.
+Default workload (one "step"): the seven linears of a Llama-2-70B-shaped block
+(q/o 8192x8192 r=2432, k/v 1024x8192 r=384, gate/up 28672x8192 r=3840, down 8192x28672
+r=3840) at decode batch 1, each layer with its own seeded input, in one grouped call
+through the C ABI (nq_lowrank_linear_fwd_grouped), captured in CUDA graphs.
 Metric: packed-weight HBM GB/s = (packed sign bytes of the seven layers) x steps / time.
 The weights rotate over enough seeded copies (> 2x the 126 MB L2) that every step
-streams its signs from HBM.
+streams its signs from HBM.  The K-step region is timed `--repeats` times (CUDA events,
+synchronised on both sides) and the median is reported.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode70b|decode7b|prefill|chain7b]
     torchrun --nproc-per-node N bench.py --gpus N ...   (independent replicas, one per GPU)
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead
-(rank 0 only) on a bounded sample of the same workload.
+(rank 0 only) on a bounded sample of the same workload, with the same ``config``.
 """
 from __future__ import annotations
 
@@ -43,6 +45,31 @@ FALLBACK_BF16_TFLOPS = 1590.0
 
 def packed_bytes(m, n, r):
     return r * (m + n) // 8
+
+
+DECODE_WORKLOADS = {
+    "decode70b": ("llama2-70b", synth.LLAMA2_70B_LAYERS),
+    "decode7b": ("llama2-7b", synth.LLAMA2_7B_LAYERS),
+}
+
+
+def weight_copies(layers, min_bytes=2 * L2_BYTES):
+    """Seeded weight copies a decode step rotates over, so that the copies' packed signs
+    exceed `min_bytes` (every step then streams its weights from HBM, not L2)."""
+    step = sum(packed_bytes(m, n, r) for _, m, n, r in layers)
+    return max(1, -(-min_bytes // step))
+
+
+def decode_config(model, layers, batch):
+    """The `config` of a decode line, the same for the GPU arm and the oracle arm."""
+    step = sum(packed_bytes(m, n, r) for _, m, n, r in layers)
+    copies = weight_copies(layers)
+    return {"workload": f"{model}-shaped decode, batch {batch}: 7 factorised linears per step "
+                        f"({', '.join(f'{nm} {m}x{n} r{r}' for nm, m, n, r in layers)}), "
+                        "one nq_lowrank_linear_fwd_grouped call per step",
+            "batch": batch, "packed_bytes_per_step": step,
+            "l2": f"inputs larger than L2: weights rotate over {copies} seeded copies "
+                  f"({copies * step / 1e6:.0f} MB > 2x the 126 MB L2)"}
 
 
 def load_peaks():
@@ -132,7 +159,7 @@ class DecodeWorkload:
         self.layers = layers
         self.batch = batch
         self.step_bytes = sum(packed_bytes(m, n, r) for _, m, n, r in layers)
-        self.copies = max(1, -(-min_bytes // self.step_bytes))
+        self.copies = weight_copies(layers, min_bytes)
         gen = torch.Generator(device=device)
         gen.manual_seed(seed)
         self.sets = []
@@ -235,8 +262,10 @@ def capture(fn, stream):
     return g
 
 
-def timed_graphs(work, steps, warmup, stream, layer_filter=None, dist=None):
-    """Capture graphs covering `steps` steps (rotating copies) and time them with events."""
+def timed_graphs(work, steps, warmup, stream, layer_filter=None, dist=None, repeats=1):
+    """Capture graphs covering `steps` steps (rotating copies), then time the `steps`-step
+    region `repeats` times with CUDA events on the launching stream, each bracketed by a
+    synchronisation (and a barrier across ranks).  Returns (median ms, all ms)."""
     import torch
 
     full = capture(lambda h: [work.step(i, h, layer_filter) for i in range(work.copies)], stream)
@@ -245,23 +274,70 @@ def timed_graphs(work, steps, warmup, stream, layer_filter=None, dist=None):
     reps = steps // work.copies
     for _ in range(max(1, -(-warmup // work.copies))):
         full.replay()
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for _ in range(reps):
-            full.replay()
-        if part is not None:
-            part.replay()
-        end.record(stream)
-    torch.cuda.synchronize()
-    ms = start.elapsed_time(end)
-    if dist is not None:
-        dist.barrier()
+    times = []
+    for _ in range(repeats):
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(reps):
+                full.replay()
+            if part is not None:
+                part.replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+        times.append(start.elapsed_time(end))
+        if dist is not None:
+            dist.barrier()
     del full, part
-    return ms
+    return statistics.median(times), times
+
+
+def traffic_record(workload, batch):
+    """DRAM bytes per decode step from an ncu capture recorded in profiles/decode_traffic.json,
+    or None when there is none for this workload or the decode kernels' code has changed
+    since it was taken (the record holds a hash of the source without comments)."""
+    import hashlib
+
+    tpath = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(tpath):
+        return None
+    with open(tpath) as f:
+        recs = json.load(f)
+    for rec in recs.get("records", []):
+        if rec.get("workload_key") != f"{workload}-b{batch}":
+            continue
+        with open(os.path.join(ROOT, rec["kernel_source"])) as f:
+            code = f.read()
+        code = re.sub(r"/\*.*?\*/", "", code, flags=re.S)
+        code = "".join(re.sub(r"//[^\n]*", "", code).split())
+        if hashlib.sha256(code.encode()).hexdigest()[:16] == rec["kernel_code_sha256_16"]:
+            return rec["dram_bytes_per_step"]
+    return None
+
+
+def decode_line_numbers(work, ms, steps, peaks):
+    gbs = work.step_bytes * steps / (ms * 1e-3) / 1e9
+    return {"gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+            "us_per_step": round(ms * 1e3 / steps, 2),
+            "tokens_per_s": round(work.batch * steps / (ms * 1e-3), 1)}
+
+
+def run_secondary_decode(name, layers, batch, steps, warmup, stream, device, peaks, seed, repeats=3):
+    import torch
+
+    w = DecodeWorkload(layers, batch, seed=seed, device=device)
+    with torch.cuda.stream(stream):
+        w.step(0, stream.cuda_stream)
+    torch.cuda.synchronize()
+    st = max(w.copies, steps // w.copies * w.copies)
+    ms, _ = timed_graphs(w, st, warmup, stream, repeats=repeats)
+    out = decode_line_numbers(w, ms, st, peaks)
+    out["steps"] = st
+    del w
+    return out
 
 
 def run_ours(args):
@@ -281,15 +357,14 @@ def run_ours(args):
         dist = tdist
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    from binary_rank_linear_02_b200 import nq
+    from binary_rank_linear_02_b200 import nq  # noqa: F401  (fails loudly without libnq.so)
 
     peaks = load_peaks()
     if args.workload == "prefill":
         return run_prefill_only(args, device, peaks)
     if args.workload == "chain7b":
         return run_chain_only(args, device, peaks)
-    layers = synth.LLAMA2_70B_LAYERS if args.workload == "decode70b" else synth.LLAMA2_7B_LAYERS
-    model = "llama2-70b" if args.workload == "decode70b" else "llama2-7b"
+    model, layers = DECODE_WORKLOADS[args.workload]
     batch = args.batch
     work = DecodeWorkload(layers, batch, seed=1234 + rank, device=device)
     stream = torch.cuda.Stream(device)
@@ -300,104 +375,70 @@ def run_ours(args):
 
     sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
     sampler.start()
-    ms = timed_graphs(work, args.steps, args.warmup, stream, dist=dist)
+    ms, all_ms = timed_graphs(work, args.steps, args.warmup, stream, dist=dist, repeats=args.repeats)
     clocks = sampler.stop()
     ms_max, total_bytes = aggregate(ms, float(work.step_bytes * args.steps), dist, device)
     value = total_bytes / (ms_max * 1e-3) / 1e9
     tokens_per_s = batch * args.steps * world / (ms_max * 1e-3)
 
-    # roofline: the kernels of the headline step (the stage-1 and stage-2 kernels of one
-    # grouped call, timed live above), against the measured HBM copy bandwidth
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    if os.path.exists(tpath) and batch == 1 and args.workload == "decode7b":
-        import hashlib
-
-        with open(tpath) as f:
-            rec = json.load(f)
-        with open(os.path.join(ROOT, rec["kernel_source"])) as f:
-            code = f.read()
-        # the source with comments and white space removed: counters are only valid for the
-        # kernel code they were taken from
-        code = re.sub(r"/\*.*?\*/", "", code, flags=re.S)
-        code = "".join(re.sub(r"//[^\n]*", "", code).split())
-        if hashlib.sha256(code.encode()).hexdigest()[:16] == rec["kernel_code_sha256_16"]:
-            traffic = rec["dram_bytes_per_step_b1"]
+    # roofline: the decode kernels of the headline step (stage 1 + stage 2 of one grouped
+    # call, timed live above), against the measured HBM copy bandwidth
     achieved = value / world
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic_record(args.workload, batch),
+                "algorithmic_bytes_per_launch": work.step_bytes,
                 "kernel": f"stage1_kernel + stage2_kernel of one grouped call ({work.step_bytes} packed bytes "
-                          "per launch pair), per-GPU",
+                          "per launch pair), per GPU",
                 "peak_source": peaks["source"]}
-
-    # the largest layer (gate) alone, back to back over its own rotating copies
-    gate = [l for l in layers if l[0] == "gate"][0]
-    _, gm, gn, gr = gate
-    gwork = DecodeWorkload([gate], batch, seed=777 + rank, device=device)
-    with torch.cuda.stream(stream):
-        gwork.step(0, stream.cuda_stream)
-    torch.cuda.synchronize()
-    r_steps = max(gwork.copies * 10, 500)
-    ms_gate = timed_graphs(gwork, r_steps, args.warmup, stream)
-    del gwork
-    gate_gbs = packed_bytes(gm, gn, gr) * r_steps / (ms_gate * 1e-3) / 1e9
 
     # end to end through the public API with host buffers (pinned), synchronous per call
     e2e = run_e2e(work, stream, min(args.steps, 100), device)
 
-    # secondary: the same step as seven separate nq_lowrank_linear_fwd calls; batch 8
-    secondary = {"decode_%s_gate_alone_b%d_gbs" % (model, batch): round(gate_gbs, 1)}
+    secondary = {}
+    prefill_roofline = prefill_cpu = None
     if args.secondary and world == 1:
+        # the largest layer (gate) alone, back to back over its own rotating copies
+        gate = [l for l in layers if l[0] == "gate"][0]
+        secondary[f"decode_{model}_gate_alone_b{batch}"] = run_secondary_decode(
+            "gate", [gate], batch, max(500, args.steps), args.warmup, stream, device, peaks, seed=777)
         work.grouped = False
-        ms1 = timed_graphs(work, args.steps, args.warmup, stream)
+        ms1, _ = timed_graphs(work, args.steps, args.warmup, stream, repeats=3)
         work.grouped = True
-        secondary["decode_b%d_per_layer_calls_gbs" % batch] = round(work.step_bytes * args.steps / (ms1 * 1e-3) / 1e9, 1)
-    if args.secondary and batch == 1 and world == 1 and args.workload == "decode7b":
-        for b70 in (1, 4):  # the Llama-2-70B-shaped block, batch 1 and 4
-            w70 = DecodeWorkload(synth.LLAMA2_70B_LAYERS, b70, seed=70 + b70, device=device)
-            with torch.cuda.stream(stream):
-                w70.step(0, stream.cuda_stream)
-            torch.cuda.synchronize()
-            st70 = max(w70.copies, min(args.steps, 400) // w70.copies * w70.copies)
-            ms70 = timed_graphs(w70, st70, args.warmup, stream)
-            secondary["decode70b_b%d_gbs" % b70] = round(w70.step_bytes * st70 / (ms70 * 1e-3) / 1e9, 1)
-            secondary["decode70b_b%d_tokens_per_s" % b70] = round(b70 * st70 / (ms70 * 1e-3), 1)
-            del w70
-        w8 = DecodeWorkload(layers, 8, seed=99, device=device)
-        with torch.cuda.stream(stream):
-            w8.step(0, stream.cuda_stream)
-        torch.cuda.synchronize()
-        ms8 = timed_graphs(w8, args.steps, args.warmup, stream)
-        secondary["decode_b8_gbs"] = round(w8.step_bytes * args.steps / (ms8 * 1e-3) / 1e9, 1)
-        secondary["decode_b8_tokens_per_s"] = round(8 * args.steps / (ms8 * 1e-3), 1)
-        del w8
-        # 16 tokens in one grouped call of the block (the decode kernels over two token chunks)
-        w16 = DecodeWorkload(layers, 16, seed=116, device=device)
-        with torch.cuda.stream(stream):
-            w16.step(0, stream.cuda_stream)
-        torch.cuda.synchronize()
-        ms16 = timed_graphs(w16, args.steps, args.warmup, stream)
-        secondary["grouped_b16_us_per_call"] = round(ms16 * 1e3 / args.steps, 2)
-        secondary["grouped_b16_tokens_per_s"] = round(16 * args.steps / (ms16 * 1e-3), 1)
-        del w16
-        # the input gradient dx = W^T dy of the same block (backward of the layers)
+        secondary[f"decode_{model}_b{batch}_per_layer_calls"] = decode_line_numbers(work, ms1, args.steps, peaks)
+        others = [("decode70b", 4), ("decode7b", 1), ("decode7b", 8)]
+        if args.workload != "decode70b" or batch != 1:
+            others = [("decode70b", 1)] + others
+        for wl, b in others:
+            if wl == args.workload and b == batch:
+                continue
+            m2, l2 = DECODE_WORKLOADS[wl]
+            secondary[f"decode_{m2}_b{b}"] = run_secondary_decode(wl, l2, b, min(args.steps, 400), args.warmup,
+                                                                   stream, device, peaks, seed=70 + b)
+        # 16 tokens in one grouped call of the 7B block (the decode kernels over two token chunks)
+        g16 = run_secondary_decode("decode7b", synth.LLAMA2_7B_LAYERS, 16, min(args.steps, 400), args.warmup,
+                                   stream, device, peaks, seed=116)
+        secondary["grouped_llama2-7b_b16"] = g16
+        # the input gradient dx = W^T dy of the 7B block (backward of the layers)
         for bb in (1, 8):
-            wb = backward_workload(layers, bb, seed=123 + bb, device=device)
+            wb = backward_workload(synth.LLAMA2_7B_LAYERS, bb, seed=123 + bb, device=device)
             with torch.cuda.stream(stream):
                 wb.step(0, stream.cuda_stream)
             torch.cuda.synchronize()
-            msb = timed_graphs(wb, args.steps, args.warmup, stream)
-            secondary["backward_input_b%d_gbs" % bb] = round(wb.step_bytes * args.steps / (msb * 1e-3) / 1e9, 1)
+            msb, _ = timed_graphs(wb, args.steps, args.warmup, stream, repeats=3)
+            secondary[f"backward_input_llama2-7b_b{bb}"] = decode_line_numbers(wb, msb, args.steps, peaks)
             del wb
-
-    if args.secondary and world == 1:
-        secondary["prefill_11008x4096_r2432"] = run_prefill_sweep(device, stream, args.warmup, peaks)
-    if args.secondary and world == 1 and batch == 1 and args.workload == "decode7b":
+        sweep = run_prefill_sweep(device, stream, args.warmup, peaks)
+        secondary["prefill_11008x4096_r2432"] = sweep
+        prefill_roofline = prefill_roofline_of(sweep, peaks)
         secondary["chain_llama2-7b_32_blocks_b1"] = run_chain(device, stream, args.warmup, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = run_cpu_baseline(layers, batch, budget_s=args.cpu_seconds)
+        if args.secondary:
+            prefill_cpu = run_cpu_baseline_prefill(budget_s=max(3.0, args.cpu_seconds / 2))
+            if prefill_roofline is not None:
+                prefill_roofline["cpu_baseline"] = prefill_cpu
 
     launches = args.steps * 2  # stage-1 and stage-2 kernels of one grouped call per step
     if rank == 0:
@@ -406,15 +447,16 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in; int8x2-limb tensor-core products, int32/fp32 acc",
             "data": "synthetic",
-            "config": {"workload": f"{model}-shaped decode, batch {batch}: 7 factorised linears per step "
-                                   f"({', '.join(f'{nm} {m}x{n} r{r}' for nm, m, n, r in layers)}), "
-                                   "one nq_lowrank_linear_fwd_grouped call per step",
-                       "batch": batch, "packed_bytes_per_step": work.step_bytes,
-                       "l2": f"weights rotate over {work.copies} seeded copies "
-                             f"({work.copies * work.step_bytes / 1e6:.0f} MB > 2x L2)",
-                       "graphs": "CUDA graphs of the C-ABI calls", "parallelism": f"replicas x{world}"},
+            "config": decode_config(model, layers, batch),
+            "parallelism": f"independent replicas x{world} (no data-path collective)",
+            "timing": {"repeats": args.repeats, "reported": "median of the repeats",
+                       "ms_per_repeat": [round(t, 4) for t in all_ms],
+                       "method": "CUDA events on the launching stream around exactly `steps` steps, "
+                                 "synchronised on both sides, CUDA graphs of the C-ABI calls"},
             "tokens_per_s": round(tokens_per_s, 1),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "gpu_launches_all_repeats": launches * args.repeats, "clocks": clocks,
+            "prefill_roofline": prefill_roofline,
             "secondary": secondary,
         }
         print(json.dumps(line), flush=True)
@@ -424,7 +466,21 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_prefill_sweep(device, stream, warmup, peaks, calls=20, batches=synth.PREFILL_BATCHES):
+def prefill_roofline_of(sweep, peaks):
+    """The prefill half of the metric: config-4 sweep against the bf16 dense burst peak (the
+    two GEMMs are timed back to back in isolation), reported at the largest batch with the
+    fraction at every batch."""
+    top = str(max(int(b) for b in sweep))
+    tf = sweep[top]["tflops"]
+    return {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None,
+            "kernel": f"prescale_kernel + two tcgen05 GEMM kernels of one nq_lowrank_linear_fwd call, "
+                      f"11008x4096 r=2432 layer, {top} tokens (2*b*r*(m+n) flops per call)",
+            "frac_per_batch": {b: v["frac_of_bf16_burst"] for b, v in sweep.items()},
+            "peak_source": peaks["source"] + " (burst)"}
+
+
+def run_prefill_sweep(device, stream, warmup, peaks, calls=20, batches=synth.PREFILL_BATCHES, repeats=5):
     """Config-4 sweep: the 11008x4096 r=2432 layer at token batches 16..4096 (tcgen05 path)."""
     import torch
 
@@ -457,16 +513,17 @@ def run_prefill_sweep(device, stream, warmup, peaks, calls=20, batches=synth.PRE
         for _ in range(max(1, warmup // calls)):
             g.replay()
         torch.cuda.synchronize()
-        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 3
-        with torch.cuda.stream(stream):
-            start.record(stream)
-            for _ in range(reps):
+        times = []
+        for _ in range(repeats):
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                start.record(stream)
                 g.replay()
-            end.record(stream)
-        torch.cuda.synchronize()
+                end.record(stream)
+            torch.cuda.synchronize()
+            times.append(start.elapsed_time(end) / calls)
         nq.device_status(stream.cuda_stream)
-        ms = start.elapsed_time(end) / (reps * calls)
+        ms = statistics.median(times)
         flops = 2.0 * b * r * (m + n)
         tf = flops / (ms * 1e-3) / 1e12
         out[str(b)] = {"tflops": round(tf, 1), "us_per_call": round(ms * 1e3, 2),
@@ -476,7 +533,7 @@ def run_prefill_sweep(device, stream, warmup, peaks, calls=20, batches=synth.PRE
     return out
 
 
-def run_chain(device, stream, warmup, peaks, passes=20, batch=1, nblocks=synth.CHAIN_7B_BLOCKS):
+def run_chain(device, stream, warmup, peaks, passes=20, batch=1, nblocks=synth.CHAIN_7B_BLOCKS, repeats=3):
     """The decode chain: 32 Llama-2-7B-shaped blocks x 7 factorised linears at batch 1, per
     block two grouped forward calls, one cast and one RMS normalisation (6 kernels).  659 MB
     of packed weights per pass (> 5x L2), so every pass streams its weights from HBM."""
@@ -508,14 +565,17 @@ def run_chain(device, stream, warmup, peaks, passes=20, batch=1, nblocks=synth.C
     for _ in range(max(3, warmup // 10)):
         g.replay()
     torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for _ in range(passes):
-            g.replay()
-        end.record(stream)
-    torch.cuda.synchronize()
-    ms = start.elapsed_time(end) / passes
+    times = []
+    for _ in range(repeats):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(passes):
+                g.replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+        times.append(start.elapsed_time(end) / passes)
+    ms = statistics.median(times)
     pb = ch.packed_bytes()
     gbs = pb / (ms * 1e-3) / 1e9
     out = {"tokens_per_s": round(batch / (ms * 1e-3), 1), "us_per_pass": round(ms * 1e3, 1),
@@ -534,17 +594,21 @@ def run_chain_only(args, device, peaks):
     stream = torch.cuda.Stream(device)
     sampler = ClockSampler(torch.cuda.current_device())
     sampler.start()
-    c = run_chain(device, stream, args.warmup, peaks, passes=max(1, args.steps), batch=args.batch)
+    c = run_chain(device, stream, args.warmup, peaks, passes=max(1, args.steps), batch=args.batch,
+                  repeats=args.repeats)
     clocks = sampler.stop()
+    cpu = None if args.no_cpu_baseline else run_cpu_baseline_chain(budget_s=args.cpu_seconds)
     line = {"metric": METRIC, "value": c["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(c["us_per_pass"] / 1e3, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16 in; int8x2-limb tensor-core products, int32/fp32 acc", "data": "synthetic",
-            "config": {"workload": f"decode chain: {c['blocks']} llama2-7b-shaped blocks x 7 factorised linears, "
-                                   f"batch {c['batch']}, per-block RMS re-normalisation",
-                       "l2": "659 MB of packed weights per pass (> 5x L2)", "graphs": "one CUDA graph per pass"},
+            "config": chain_config(args.batch),
+            "timing": {"repeats": args.repeats, "reported": "median of the repeats", "graphs": "one CUDA graph per pass"},
             "roofline": {"bound": "hbm", "achieved": c["packed_gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": c["frac_of_hbm"], "traffic": None, "peak_source": peaks["source"]},
+                         "frac": c["frac_of_hbm"], "traffic": None, "peak_source": peaks["source"],
+                         "algorithmic_bytes_per_launch": c["packed_bytes_per_pass"],
+                         "kernel": "every decode kernel of one chain pass"},
+            "cpu_baseline": cpu,
             "gpu_launches": c["kernels_per_pass"] * max(1, args.steps), "clocks": clocks, "chain": c}
     print(json.dumps(line), flush=True)
 
@@ -554,13 +618,22 @@ def run_prefill_only(args, device, peaks):
     import torch
 
     stream = torch.cuda.Stream(device)
-    sweep = run_prefill_sweep(device, stream, args.warmup, peaks, calls=max(1, args.steps),
-                              batches=(args.prefill_batch,) if args.prefill_batch else synth.PREFILL_BATCHES)
+    batches = (args.prefill_batch,) if args.prefill_batch else synth.PREFILL_BATCHES
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    sweep = run_prefill_sweep(device, stream, args.warmup, peaks, calls=max(1, args.steps), batches=batches,
+                              repeats=args.repeats)
+    clocks = sampler.stop()
     top = str(max(int(b) for b in sweep))
+    cpu = None if args.no_cpu_baseline else run_cpu_baseline_prefill(budget_s=args.cpu_seconds)
     line = {"metric": METRIC, "value": sweep[top]["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "warmup": args.warmup, "ms_per_step": round(sweep[top]["us_per_call"] / 1e3, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp16 tcgen05 operands, fp32 accumulate", "data": "synthetic",
-            "config": {"workload": f"prefill 11008x4096 r=2432, token batch {top}"}, "prefill": sweep}
+            "config": prefill_config(batches),
+            "timing": {"repeats": args.repeats, "reported": "median of the repeats"},
+            "roofline": prefill_roofline_of(sweep, peaks), "cpu_baseline": cpu,
+            "gpu_launches": 3 * max(1, args.steps), "clocks": clocks, "prefill": sweep}
     print(json.dumps(line), flush=True)
 
 
@@ -624,43 +697,118 @@ def run_e2e(work, stream, steps, device):
 # ------------------------------------------------------------------ the oracle on the host
 
 def run_cpu_baseline(layers, batch, budget_s):
+    """The oracle on the host cores over the decode workload: whole steps (the seven
+    layers), rotating over the same number of seeded weight copies as the GPU arm, until
+    `budget_s` seconds have passed."""
     import oracle
 
     o = oracle.default()
+    copies = weight_copies(layers)
     data = []
-    for li, (name, m, n, r) in enumerate(layers):
-        Upk = synth.random_words(m, r // 32, 5, li, "U")
-        Vpk = synth.random_words(r, n // 32, 5, li, "V")
-        data.append((Upk, Vpk, synth.scales_f16(m, 5, li), synth.scales_f16(n, 6, li),
-                     synth.activations_bf16(batch, n, 5, li), m, n, r))
+    for c in range(copies):
+        per = []
+        for li, (name, m, n, r) in enumerate(layers):
+            per.append((synth.random_words(m, r // 32, 5, c, li, "U"), synth.random_words(r, n // 32, 5, c, li, "V"),
+                        synth.scales_f16(m, 5, c, li), synth.scales_f16(n, 6, c, li),
+                        synth.activations_bf16(batch, n, 5, li), m, n, r))
+        data.append(per)
     step_bytes = sum(packed_bytes(m, n, r) for _, m, n, r in layers)
     steps = 0
     t0 = time.perf_counter()
     while True:
-        for (Upk, Vpk, s1, s2, x, m, n, r) in data:
+        for (Upk, Vpk, s1, s2, x, m, n, r) in data[steps % copies]:
             o.lowrank_linear_fwd(x, Upk, Vpk, s1, s2, m, n, r)
         steps += 1
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
     return {"value": round(step_bytes * steps / dt / 1e9, 4), "unit": "GB/s", "cores": o.num_threads(),
-            "kind": "oracle",
-            "sample": f"{steps} step(s) of the 7-layer batch-{batch} workload on the fp64 C oracle ({dt:.1f} s)"}
+            "kind": "oracle", "steps": steps, "seconds": round(dt, 2),
+            "sample": f"{steps} step(s) of the 7-layer batch-{batch} workload ({copies} rotating weight copies) "
+                      f"on the fp64 C oracle ({dt:.1f} s)"}
+
+
+def run_cpu_baseline_prefill(budget_s, batch=16):
+    """The oracle on the host cores over the prefill layer (11008x4096, r=2432): calls of
+    `batch` tokens until `budget_s` seconds have passed; TFLOP/s over 2*b*r*(m+n)."""
+    import oracle
+
+    o = oracle.default()
+    _, m, n, r = synth.PREFILL_SHAPE
+    Upk = synth.random_words(m, r // 32, 9, "U")
+    Vpk = synth.random_words(r, n // 32, 9, "V")
+    s1, s2 = synth.scales_f16(m, 9, "s1"), synth.scales_f16(n, 9, "s2")
+    x = synth.activations_bf16(batch, n, 9)
+    calls = 0
+    t0 = time.perf_counter()
+    while True:
+        o.lowrank_linear_fwd(x, Upk, Vpk, s1, s2, m, n, r)
+        calls += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    flops = 2.0 * batch * r * (m + n) * calls
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": o.num_threads(), "kind": "oracle",
+            "sample": f"{calls} call(s) of {batch} tokens on the 11008x4096 r=2432 layer, fp64 C oracle ({dt:.1f} s)"}
+
+
+def run_cpu_baseline_chain(budget_s, nblocks=synth.CHAIN_7B_BLOCKS):
+    """The oracle's decode chain on the host cores: blocks of the 32-block chain (seeded
+    weights as the GPU arm draws them) one after another until `budget_s` seconds have
+    passed; tokens/s scaled to the whole chain."""
+    import oracle
+
+    o = oracle.default()
+    w = synth.chain_weights(1, synth.LLAMA2_7B_LAYERS, 5150)[0]
+    h = synth.activations_bf16(1, 4096, 5150, "h0")
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        h = o.chain_block(h, w)["h_next"]
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(done / nblocks / dt, 4), "unit": "tokens/s", "cores": o.num_threads(), "kind": "oracle",
+            "sample": f"{done} Llama-2-7B-shaped block(s) of the {nblocks}-block chain, batch 1, fp64 C oracle "
+                      f"({dt:.1f} s)"}
+
+
+def prefill_config(batches):
+    _, m, n, r = synth.PREFILL_SHAPE
+    return {"workload": f"prefill {m}x{n} r={r}, token batch {max(batches)} "
+                        f"(sweep {', '.join(str(b) for b in batches)})",
+            "batches": list(batches)}
+
+
+def chain_config(batch=1, nblocks=synth.CHAIN_7B_BLOCKS):
+    return {"workload": f"decode chain: {nblocks} llama2-7b-shaped blocks x 7 factorised linears, "
+                        f"batch {batch}, per-block RMS re-normalisation",
+            "l2": "inputs larger than L2: 659 MB of packed weights per pass (> 5x L2)"}
 
 
 def run_reference(args):
+    """The oracle arm: the CPU oracle as it stands, on the host cores, over a bounded sample
+    of this arm's workload, with the same config, metric and unit as the GPU arm."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    cpu = run_cpu_baseline(synth.LLAMA2_7B_LAYERS, args.batch, budget_s=args.cpu_seconds)
-    steps_done = int(cpu["sample"].split()[0])
+    if args.workload == "prefill":
+        batches = (args.prefill_batch,) if args.prefill_batch else synth.PREFILL_BATCHES
+        cpu = run_cpu_baseline_prefill(budget_s=args.cpu_seconds)
+        config = prefill_config(batches)
+    elif args.workload == "chain7b":
+        cpu = run_cpu_baseline_chain(budget_s=args.cpu_seconds)
+        config = chain_config(args.batch)
+    else:
+        model, layers = DECODE_WORKLOADS[args.workload]
+        cpu = run_cpu_baseline(layers, args.batch, budget_s=args.cpu_seconds)
+        config = decode_config(model, layers, args.batch)
     value = cpu["value"]
-    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+    line = {"metric": METRIC, "value": value, "unit": cpu["unit"], "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "impl": "reference",
-            "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"llama2-7b-shaped decode, batch {args.batch}: 7 factorised linears per step",
-                       "batch": args.batch, "steps_sampled": steps_done},
-            "cpu_baseline": cpu, "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+            "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": cpu, "e2e": {"value": value, "unit": cpu["unit"], "h2d_bytes_per_step": 0,
                                           "d2h_bytes_per_step": 0},
             "vs_baseline": None}
     print(json.dumps(line), flush=True)
@@ -676,7 +824,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", dest="secondary", action="store_false")
-    ap.add_argument("--workload", choices=["decode7b", "decode70b", "prefill", "chain7b"], default="decode7b")
+    ap.add_argument("--workload", choices=["decode70b", "decode7b", "prefill", "chain7b"], default="decode70b")
+    ap.add_argument("--repeats", type=int, default=5)
     ap.add_argument("--prefill-batch", type=int, default=0)
     args = ap.parse_args()
     if args.warmup < 3:
