@@ -94,6 +94,13 @@ def _load() -> ctypes.CDLL:
     L.nq_cast_f32_to_bf16.restype = ctypes.c_int
     L.nq_rms_normalize_bf16.argtypes = [p, i64, i64, p, p]
     L.nq_rms_normalize_bf16.restype = ctypes.c_int
+    i32, f64 = ctypes.c_int, ctypes.c_double
+    L.nq_admm_init.argtypes = [p, i64, i64, i64, p, i32, p, p, p, p, p, p, p, p, p]
+    L.nq_admm_init.restype = ctypes.c_int
+    L.nq_admm_iterate.argtypes = [p, i64, i64, i64, p, p, p, p, p, p, p, p, i32, f64, f64, p]
+    L.nq_admm_iterate.restype = ctypes.c_int
+    L.nq_admm_factorize.argtypes = [p, i64, i64, i64, p, i32, i32, f64, f64, p, p, p, p, p, p]
+    L.nq_admm_factorize.restype = ctypes.c_int
     return L
 
 
@@ -390,3 +397,56 @@ def bits_per_weight(m: int, n: int, r: int) -> float:
 
 def workspace_reserve(m: int, n: int, r: int, batch: int) -> None:
     _check(_lib.nq_workspace_reserve(m, n, r, batch), "nq_workspace_reserve")
+
+
+# ------------------------------------------------------------------ LB-ADMM initialiser
+
+class AdmmState:
+    """Device state of the ADMM iteration: latent A (m x r), B (n x r), projections Z_A, Z_B,
+    duals L_A, L_B, row scales s_A (m), s_B (n), all fp32 tensors on the current device."""
+
+    def __init__(self, m: int, n: int, r: int, device=None):
+        import torch
+
+        dev = device if device is not None else torch.device("cuda")
+        f = dict(dtype=torch.float32, device=dev)
+        self.m, self.n, self.r = m, n, r
+        self.A, self.ZA, self.LA = (torch.empty((m, r), **f) for _ in range(3))
+        self.B, self.ZB, self.LB = (torch.empty((n, r), **f) for _ in range(3))
+        self.sA, self.sB = torch.empty(m, **f), torch.empty(n, **f)
+
+    def ptrs(self):
+        return [_ptr(t) for t in (self.A, self.B, self.ZA, self.ZB, self.LA, self.LB, self.sA, self.sB)]
+
+
+def admm_init(W, m: int, n: int, r: int, Omega, power_iters: int = 1, stream=None) -> AdmmState:
+    """Start of the initialiser on W (m x n bfloat16 bits, int16/bfloat16 tensor) from Omega (n x r fp32)."""
+    st = AdmmState(m, n, r, W.device)
+    _check(_lib.nq_admm_init(_ptr(W), m, n, r, _ptr(Omega), power_iters, *st.ptrs(), _stream(stream, W)),
+           "nq_admm_init")
+    return st
+
+
+def admm_iterate(W, st: AdmmState, iters: int, lam0: float = 0.2, growth: float = 1.05, stream=None) -> AdmmState:
+    _check(_lib.nq_admm_iterate(_ptr(W), st.m, st.n, st.r, *st.ptrs(), iters, lam0, growth, _stream(stream, W)),
+           "nq_admm_iterate")
+    return st
+
+
+def admm_factorize(W, m: int, n: int, r: int, Omega, iters: int = 40, lam0: float = 0.2, growth: float = 1.05,
+                   power_iters: int = 1, stream=None):
+    """The whole initialiser: returns (Upk, Vpk, s1, s2, rel_err) with the forward pass's
+    packings (Upk m x r/32, Vpk r x n/32 int32 views of the words; s1, s2 fp16 bits as int16)."""
+    import torch
+
+    dev = W.device
+    Upk = torch.empty((m, r // 32), dtype=torch.int32, device=dev)
+    Vpk = torch.empty((r, n // 32), dtype=torch.int32, device=dev)
+    s1 = torch.empty(m, dtype=torch.int16, device=dev)
+    s2 = torch.empty(n, dtype=torch.int16, device=dev)
+    err = ctypes.c_double(0.0)
+    _check(_lib.nq_admm_factorize(_ptr(W), m, n, r, _ptr(Omega), power_iters, iters, lam0, growth, _ptr(Upk),
+                                  _ptr(Vpk), _ptr(s1), _ptr(s2), ctypes.byref(err), _stream(stream, W)),
+           "nq_admm_factorize")
+    return Upk, Vpk, s1, s2, err.value
+

@@ -165,3 +165,21 @@ def activations_token_scaled_bf16(n: int, seed: int, token_scales, *tags) -> np.
     sc = np.asarray(token_scales, dtype=np.float64)
     z = _rng(seed, "x-token-scaled", sc.size, n, *tags).standard_normal(size=(sc.size, n))
     return f32_to_bf16_bits((z * sc[:, None]).astype(np.float32))
+
+
+# Inputs of the LB-ADMM initialiser: a dense weight matrix and the start block.
+
+def weights_bf16(m: int, n: int, seed: int, *tags, spread: float = 0.5) -> np.ndarray:
+    """m x n bfloat16 weights N(0, 1) * exp(spread N(0, 1))_row * exp(spread N(0, 1))_col
+    * 0.02 (Gaussian entries with log-normal row and column magnitudes, the structure the
+    per-row and per-column scales of the factorisation capture), as bf16 bit patterns."""
+    g = _rng(seed, "weights", m, n, *tags)
+    rows = np.exp(spread * g.standard_normal(m))
+    cols = np.exp(spread * g.standard_normal(n))
+    z = g.standard_normal((m, n)) * rows[:, None] * cols[None, :] * 0.02
+    return f32_to_bf16_bits(z.astype(np.float32))
+
+
+def gaussian_f32(rows: int, cols: int, seed: int, *tags) -> np.ndarray:
+    """rows x cols float32 standard normal draws (the initialiser's start block)."""
+    return _rng(seed, "gauss", rows, cols, *tags).standard_normal(size=(rows, cols)).astype(np.float32)

@@ -313,6 +313,62 @@ int nq_lowrank_linear_fwd_noalloc(const void* x, const uint32_t* Upk, const uint
                                   int64_t batch, float* y, void* stream);
 
 /*
+ * LB-ADMM initialiser of the binary factorisation (hardwired.dev, "NanoQuant jednoduse",
+ * section "Trikrokovy pipeline", step 2 "Inicializace binarni faktorizace (LB-ADMM)": ADMM
+ * alternating a closed-form least-squares solve for the continuous parameters with a
+ * projection onto the binary constraint by the sign operation, followed by magnitude
+ * balancing of the scales).  The pages give no formula; the library's reading:
+ *   W ~= A B^T with latent A (m x r), B (n x r) constrained to row-scaled sign matrices
+ *   Z = diag(s) S, S in {+1,-1}; scaled duals L_A, L_B; iteration k with lam_k = lam0*growth^k:
+ *     rho_A = lam_k tr(B^T B)/r;  A = (W B + rho_A (Z_A - L_A)) (B^T B + rho_A I)^-1;
+ *     Z_A = Pi(A + L_A) (per row: signs, sign(0) = +1, and the scale mean |row|);
+ *     L_A = L_A + A - Z_A;  then the same for B with W^T and the new A.
+ *   Start: block power iteration from Omega (n x r): Q = orth(W Omega), power_iters times
+ *   Q = orth(W (W^T Q)), orth by Cholesky-QR; A = Q, B = W^T Q, each column pair rescaled
+ *   to equal norms; Z = Pi(A), Pi(B); L = 0.
+ *   Result: U = signs of Z_A, V = signs of Z_B; s1 = c s_A, s2 = s_B / c with
+ *   c = sqrt(rms(s_B)/rms(s_A)) (both scale vectors get the same root-mean-square).
+ * Common rules: W is m x n bfloat16, row-major, device memory; every matrix is row-major
+ * fp32 device memory of the current device, 16-byte aligned (else NQ_ERR_ALIGN /
+ * NQ_ERR_PTRKIND); m, n, r positive multiples of 128 with r <= min(m, n) and r <= 16384
+ * (else NQ_ERR_SHAPE).  The calls allocate their own scratch (cudaMalloc) and synchronise
+ * `stream` before returning (an offline step).  A Cholesky pivot that is not positive in
+ * fp32 (a start W Omega of column rank below r, or an ill-conditioned system) returns
+ * NQ_ERR_VALUE; the outputs are then unspecified.  Deterministic: every sum runs in a
+ * fixed order.  Arithmetic in fp32 (W read exactly from bf16), reductions of norms in fp64.
+ */
+
+/*
+ * nq_admm_init -- the start: A, B (latent, m x r and n x r), Z_A, Z_B (their projections),
+ * L_A, L_B (set to zero), s_A (m), s_B (n) (the projections' row scales), all written.
+ * Omega: n x r fp32, the caller's start block (e.g. Gaussian); 0 <= power_iters <= 64.
+ */
+int nq_admm_init(const void* W, int64_t m, int64_t n, int64_t r, const float* Omega, int power_iters, float* A,
+                 float* B, float* ZA, float* ZB, float* LA, float* LB, float* sA, float* sB, void* stream);
+
+/*
+ * nq_admm_iterate -- `iters` ADMM iterations on the caller's state (read and updated in
+ * place: A, B, Z_A, Z_B, L_A, L_B, s_A, s_B as written by nq_admm_init), with
+ * lam_k = lam0 * growth^k for k = 0 .. iters-1.  lam0 > 0, growth > 0, iters >= 0.
+ */
+int nq_admm_iterate(const void* W, int64_t m, int64_t n, int64_t r, float* A, float* B, float* ZA, float* ZB,
+                    float* LA, float* LB, float* sA, float* sB, int iters, double lam0, double growth, void* stream);
+
+/*
+ * nq_admm_factorize -- the whole initialiser: start, `iters` iterations, magnitude
+ * balancing, and the stored form the forward pass reads:
+ *   Upk : m x (r/32) uint32 (U, the layout of nq_pack_signs);  Vpk : r x (n/32) uint32 (V^T)
+ *   s1  : m fp16;  s2 : n fp16
+ *   rel_err : NULL, or host memory receiving ||W - diag(s1) U V^T diag(s2)||_F / ||W||_F
+ *             computed with the stored fp16 scales (sums of squares in fp64).
+ * Typical lam0 = 0.2, growth = 1.05, power_iters = 1, iters = 40 (the values the library's
+ * tests and benchmark use).
+ */
+int nq_admm_factorize(const void* W, int64_t m, int64_t n, int64_t r, const float* Omega, int power_iters, int iters,
+                      double lam0, double growth, uint32_t* Upk, uint32_t* Vpk, void* s1, void* s2, double* rel_err,
+                      void* stream);
+
+/*
  * nq_bits_per_weight -- storage cost of the factorised layer in bits per weight of the
  * dense m x n matrix it replaces: (r*(m+n) + 16*(m+n)) / (m*n)  (hardwired.dev sections
  * "Jak NanoQuant funguje" and "Co znamena sub-1-bit").  -1.0 if any argument is <= 0.

@@ -241,3 +241,29 @@ def test_grouped_ex_argument_errors(nq):
 def test_selftest_argument_errors(nq):
     assert nq.nq_selftest_wait_timeout(10, 0) == nq.NQ_ERR_VALUE
     assert nq.nq_selftest_wait_timeout(10**11, 0) == nq.NQ_ERR_VALUE
+
+
+def test_admm_argument_errors(nq):
+    """The LB-ADMM calls check shapes, values, pointers and alignment on the host, before
+    any device work (so these run without a GPU)."""
+    buf = np.zeros(1 << 16, dtype=np.uint8)
+    base = (buf.ctypes.data + 255) // 256 * 256
+    p = [base + 1024 * i for i in range(10)]
+    L = nq.lib()
+    fz = L.nq_admm_factorize
+    assert fz(p[0], 256, 256, 512, p[1], 1, 10, 0.2, 1.05, p[2], p[3], p[4], p[5], None, 0) == nq.NQ_ERR_SHAPE  # r > m
+    assert fz(p[0], 256, 200, 128, p[1], 1, 10, 0.2, 1.05, p[2], p[3], p[4], p[5], None, 0) == nq.NQ_ERR_SHAPE
+    assert fz(p[0], 256, 256, 128, p[1], 1, 10, 0.0, 1.05, p[2], p[3], p[4], p[5], None, 0) == nq.NQ_ERR_VALUE
+    assert fz(p[0], 256, 256, 128, p[1], -1, 10, 0.2, 1.05, p[2], p[3], p[4], p[5], None, 0) == nq.NQ_ERR_VALUE
+    assert fz(p[0], 256, 256, 128, p[1], 1, -3, 0.2, 1.05, p[2], p[3], p[4], p[5], None, 0) == nq.NQ_ERR_VALUE
+    assert fz(0, 256, 256, 128, p[1], 1, 10, 0.2, 1.05, p[2], p[3], p[4], p[5], None, 0) == nq.NQ_ERR_NULL
+    assert fz(p[0] + 4, 256, 256, 128, p[1], 1, 10, 0.2, 1.05, p[2], p[3], p[4], p[5], None, 0) == nq.NQ_ERR_ALIGN
+    # host memory is refused: the initialiser works on device buffers
+    assert fz(p[0], 256, 256, 128, p[1], 1, 10, 0.2, 1.05, p[2], p[3], p[4], p[5], None, 0) == nq.NQ_ERR_PTRKIND
+    st = [p[2 + i] for i in range(8)]
+    assert L.nq_admm_init(p[0], 256, 256, 128, 0, 1, *st, 0) == nq.NQ_ERR_NULL
+    assert L.nq_admm_init(p[0], 256, 256, 128, p[1], 65, *st, 0) == nq.NQ_ERR_VALUE
+    assert L.nq_admm_init(p[0], 256, 256, 128, p[1], 1, *st, 0) == nq.NQ_ERR_PTRKIND
+    assert L.nq_admm_iterate(p[0], 256, 256, 128, *st, 1, 0.2, 0.0, 0) == nq.NQ_ERR_VALUE
+    assert L.nq_admm_iterate(p[0], 256, 256, 100, *st, 1, 0.2, 1.05, 0) == nq.NQ_ERR_SHAPE
+    assert L.nq_admm_iterate(p[0], 256, 256, 128, *st, 1, 0.2, 1.05, 0) == nq.NQ_ERR_PTRKIND
