@@ -50,6 +50,9 @@ def _load(path: str) -> ctypes.CDLL:
     L.orc_transpose_signs.argtypes = [p, i64, i64, p]
     L.orc_lowrank_linear_bwd_scales.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p, p]
     L.orc_lowrank_linear_bwd_factors.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p, p]
+    L.orc_lowrank_linear_fwd_envelope.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, p]
+    L.orc_bits_per_weight_envelope.argtypes = [i64, i64, i64, i64]
+    L.orc_bits_per_weight_envelope.restype = ctypes.c_double
     L.orc_bits_per_weight.argtypes = [i64, i64, i64]
     L.orc_bits_per_weight.restype = ctypes.c_double
     L.orc_bf16_to_double.argtypes = [ctypes.c_uint16]
@@ -194,6 +197,30 @@ class Oracle:
             raise ValueError(f"orc_lowrank_linear_fwd failed with status {st}")
         return y
 
+    def lowrank_linear_fwd_envelope(self, x_bits, Upk, Vpk, a_bits, b_bits, m, n, r) -> np.ndarray:
+        """y (batch x m, float64) = sum_q a_q * (U (V^T (b_q * x))): the rank-l envelope
+        variant.  a_bits: l x m, b_bits: l x n uint16 fp16 patterns (l = 1 is the forward)."""
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1, n)
+        batch = x.shape[0]
+        a = np.ascontiguousarray(a_bits, dtype=np.uint16).reshape(-1, m)
+        b = np.ascontiguousarray(b_bits, dtype=np.uint16).reshape(-1, n)
+        l = a.shape[0]
+        assert b.shape == (l, n) and l >= 1
+        U = np.ascontiguousarray(Upk, dtype=np.uint32)
+        V = np.ascontiguousarray(Vpk, dtype=np.uint32)
+        assert U.shape == (m, words_per_row(r)) and V.shape == (r, words_per_row(n))
+        y = np.zeros((batch, m), dtype=np.float64)
+        if batch == 0:
+            return y
+        st = self.lib.orc_lowrank_linear_fwd_envelope(_ptr(x), _ptr(U), _ptr(V), _ptr(a), _ptr(b), l, m, n, r,
+                                                      batch, _ptr(y))
+        if st != ORC_OK:
+            raise ValueError(f"orc_lowrank_linear_fwd_envelope: status {st}")
+        return y
+
+    def bits_per_weight_envelope(self, m: int, n: int, r: int, l: int) -> float:
+        return self.lib.orc_bits_per_weight_envelope(m, n, r, l)
+
     def stage1(self, x_bits, Vpk, s2_bits, n, r) -> np.ndarray:
         """t (batch x r, float64) = V^T (s2 * x)."""
         x = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1, n)
@@ -283,6 +310,14 @@ def unpack_signs(packed, cols):
 
 def lowrank_linear_fwd(x_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r):
     return default().lowrank_linear_fwd(x_bits, Upk, Vpk, s1_bits, s2_bits, m, n, r)
+
+
+def lowrank_linear_fwd_envelope(x_bits, Upk, Vpk, a_bits, b_bits, m, n, r):
+    return default().lowrank_linear_fwd_envelope(x_bits, Upk, Vpk, a_bits, b_bits, m, n, r)
+
+
+def bits_per_weight_envelope(m, n, r, l):
+    return default().bits_per_weight_envelope(m, n, r, l)
 
 
 def stage1(x_bits, Vpk, s2_bits, n, r):

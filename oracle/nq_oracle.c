@@ -174,6 +174,47 @@ int orc_lowrank_linear_fwd(const uint16_t *x, const uint32_t *Upk, const uint32_
     return ORC_OK;
 }
 
+/* ---- the rank-l envelope variant of the forward pass ----
+ *
+ * MDBF ("Multi-Envelope DBF", hardwired.dev section "Kontext: co existuje kolem") replaces
+ * the simple scaling of the binary factorisation with a rank-l envelope; the same section
+ * notes that under the simple scaling all rank components share one magnitude profile.
+ * Read here as the weight
+ *     W = E (.) (U V^T),   E = sum_{q<l} a_q b_q^T   (a_q: m fp16, b_q: n fp16),
+ * whose l = 1 case is diag(s1) U V^T diag(s2) with s1 = a_0, s2 = b_0.  Since
+ * (a b^T) (.) (U V^T) = diag(a) U V^T diag(b), the output is
+ *     y = sum_{q<l} a_q (.) ( U . ( V^T . ( b_q (.) x ) ) ),
+ * each term the forward pass above with (s1, s2) = (a_q, b_q), added in increasing q.
+ *
+ * a : l rows of m fp16 bit patterns;  b : l rows of n fp16 bit patterns;  l >= 1.
+ * y : batch x m doubles (written).  Other arguments as orc_lowrank_linear_fwd.
+ */
+int orc_lowrank_linear_fwd_envelope(const uint16_t *x, const uint32_t *Upk, const uint32_t *Vpk,
+                                    const uint16_t *a, const uint16_t *b, int64_t l, int64_t m,
+                                    int64_t n, int64_t r, int64_t batch, double *y) {
+    if (l <= 0 || m <= 0 || n <= 0 || r <= 0 || batch < 0) return ORC_ERR_ARG;
+    if (batch == 0) return ORC_OK;
+    if (!a || !b) return ORC_ERR_ARG;
+    /* the first term straight into y (so that l = 1 is the forward pass bit for bit) */
+    int st = orc_lowrank_linear_fwd(x, Upk, Vpk, a, b, m, n, r, batch, y);
+    if (st != ORC_OK || l == 1) return st;
+    double *term = (double *)malloc(sizeof(double) * (size_t)(m * batch));
+    if (!term) return ORC_ERR_ARG;
+    for (int64_t q = 1; q < l && st == ORC_OK; ++q) {
+        st = orc_lowrank_linear_fwd(x, Upk, Vpk, a + q * m, b + q * n, m, n, r, batch, term);
+        for (int64_t e = 0; e < m * batch && st == ORC_OK; ++e) y[e] += term[e];
+    }
+    free(term);
+    return st;
+}
+
+/* Bits per weight of the envelope variant: r(m+n) sign bits plus l pairs of fp16 vectors,
+ * (r*(m+n) + 16*l*(m+n)) / (m*n); -1 for a non-positive argument. */
+double orc_bits_per_weight_envelope(int64_t m, int64_t n, int64_t r, int64_t l) {
+    if (m <= 0 || n <= 0 || r <= 0 || l <= 0) return -1.0;
+    return ((double)r * (double)(m + n) + 16.0 * (double)l * (double)(m + n)) / ((double)m * (double)n);
+}
+
 /* ---- the input gradient ----
  *
  * The refinement step fine-tunes the factorised components with straight-through

@@ -495,6 +495,70 @@ def pin_transpose_signs(o):
         assert np.array_equal(o.transpose_signs(t, cols, rows), p)
 
 
+def _envelope_case(m, n, r, l, batch, seed):
+    x, U, V, _, _ = _case(m, n, r, batch, seed)
+    a = np.stack([synth.scales_f16(m, seed, "env-a", q) for q in range(l)])
+    b = np.stack([synth.scales_f16(n, seed, "env-b", q) for q in range(l)])
+    return x, U, V, a, b
+
+
+def _env(o, x, U, V, a, b):
+    m, r = U.shape
+    n = V.shape[0]
+    return o.lowrank_linear_fwd_envelope(x, o.pack_signs(U), o.pack_signs(np.ascontiguousarray(V.T)), a, b, m, n, r)
+
+
+def pin_envelope_l1_is_forward(o):
+    """A rank-1 envelope is the plain s1/s2 scaling: bit for bit the forward pass."""
+    for (m, n, r, batch, seed) in ((8, 12, 3, 2, 61), (64, 96, 32, 3, 62)):
+        x, U, V, a, b = _envelope_case(m, n, r, 1, batch, seed)
+        assert np.array_equal(_env(o, x, U, V, a, b), _fwd(o, x, U, V, a[0], b[0]))
+
+
+def pin_envelope_dense(o):
+    """The envelope evaluation equals the materialised weight (sum_q a_q b_q^T) (.) (U V^T)
+    applied to x by numpy (fp64, 1e-12), for l = 2, 3, 4."""
+    for (m, n, r, l, batch, seed) in ((8, 12, 3, 2, 2, 63), (33, 40, 7, 3, 3, 64), (64, 64, 64, 4, 2, 65)):
+        x, U, V, a, b = _envelope_case(m, n, r, l, batch, seed)
+        af = a.view(np.float16).astype(np.float64)
+        bf = b.view(np.float16).astype(np.float64)
+        W = (af.T @ bf) * (U.astype(np.float64) @ V.T.astype(np.float64))
+        xd = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        y = _env(o, x, U, V, a, b)
+        assert y.shape == (batch, m)
+        assert rel_err(y, xd @ W.T) <= 1e-12, (m, n, r, l)
+
+
+def pin_envelope_repeated_term(o):
+    """Two equal envelope terms (a, b), (a, b) give exactly the single term (2a, b): doubling
+    is exact in fp16 and in double, so the two results agree bit for bit."""
+    x, U, V, a, b = _envelope_case(40, 24, 8, 1, 2, 66)
+    a2 = (a.view(np.float16) * np.float16(2)).view(np.uint16)
+    y_two = _env(o, x, U, V, np.concatenate([a, a]), np.concatenate([b, b]))
+    assert np.array_equal(y_two, _env(o, x, U, V, a2, b))
+
+
+def pin_envelope_column_negation(o):
+    """Negating column k of both U and V leaves every envelope term, and so y, bit-identical."""
+    x, U, V, a, b = _envelope_case(24, 40, 9, 3, 2, 67)
+    U2, V2 = U.copy(), V.copy()
+    U2[:, 4] *= -1
+    V2[:, 4] *= -1
+    assert np.array_equal(_env(o, x, U, V, a, b), _env(o, x, U2, V2, a, b))
+
+
+def pin_envelope_bits_per_weight(o):
+    """(r + 16 l)(m + n) / (m n), worked by hand: 4096 x 4096, r = 1664: l = 1 gives
+    1680/2048 = 0.8203125, l = 2 gives 1696/2048 = 0.828125, l = 4 gives 1728/2048 =
+    0.84375 (since (m + n)/(m n) = 8192/16777216 = 1/2048)."""
+    assert o.bits_per_weight_envelope(4096, 4096, 1664, 1) == 0.8203125
+    assert o.bits_per_weight_envelope(4096, 4096, 1664, 2) == 0.828125
+    assert o.bits_per_weight_envelope(4096, 4096, 1664, 4) == 0.84375
+    assert o.bits_per_weight_envelope(4096, 4096, 1664, 1) == o.bits_per_weight(4096, 4096, 1664)
+    for bad in ((0, 4, 4, 1), (4, 4, 4, 0)):
+        assert o.bits_per_weight_envelope(*bad) == -1.0
+
+
 def torch_bf16_to_f64(bits):
     import torch
 
@@ -521,4 +585,9 @@ ALL_PINS = [
     pin_bwd_scales_dense,
     pin_bwd_factors_sign_flip,
     pin_bwd_factors_dense,
+    pin_envelope_l1_is_forward,
+    pin_envelope_dense,
+    pin_envelope_repeated_term,
+    pin_envelope_column_negation,
+    pin_envelope_bits_per_weight,
 ]

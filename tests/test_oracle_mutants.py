@@ -50,6 +50,12 @@ MUTANTS = {
     "factors_dU_no_s1": ("dU[i * r + k] = si * acc;", "dU[i * r + k] = acc;"),
     "factors_dV_uses_t": ("for (int64_t b = 0; b < batch; ++b) acc += orc_bf16_to_double(x[b * n + j]) * u[b * r + k];",
                           "for (int64_t b = 0; b < batch; ++b) acc += orc_bf16_to_double(x[b * n + j]) * t[b * r + k];"),
+    "envelope_first_term_only": ("for (int64_t q = 1; q < l && st == ORC_OK; ++q) {",
+                                 "for (int64_t q = 1; q < 1 && st == ORC_OK; ++q) {"),
+    "envelope_b_of_first_term": ("a + q * m, b + q * n, m, n, r, batch, term", "a + q * m, b, m, n, r, batch, term"),
+    "envelope_a_of_first_term": ("a + q * m, b + q * n, m, n, r, batch, term", "a, b + q * n, m, n, r, batch, term"),
+    "envelope_subtracts": ("y[e] += term[e];", "y[e] -= term[e];"),
+    "envelope_bpw_one_pair": ("16.0 * (double)l * (double)(m + n)", "16.0 * (double)(m + n)"),
     "transpose_msb": ("out[j * wpr_out + i / 32] |= 1u << (i % 32);", "out[j * wpr_out + i / 32] |= 1u << (31 - i % 32);"),
 }
 
