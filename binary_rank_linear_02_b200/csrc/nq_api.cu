@@ -222,6 +222,20 @@ static int ensure_grad_scratch(Workspace* w, size_t ones, size_t outs_bytes, cud
     return NQ_OK;
 }
 
+// Scratch of the envelope's terms 1 .. l-1.
+static int ensure_env_scratch(Workspace* w, size_t bytes) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (bytes > w->env_bytes) {
+        if (w->env) { cudaDeviceSynchronize(); cudaFree(w->env); w->env = nullptr; w->env_bytes = 0; }
+        void* p = nullptr;
+        if (cudaMalloc(&p, bytes) != cudaSuccess) { cudaGetLastError(); return NQ_ERR_NOMEM; }
+        w->env = static_cast<float*>(p);
+        w->env_bytes = bytes;
+        ++g_ws_generation;
+    }
+    return NQ_OK;
+}
+
 // ---------------------------------------------------------------- launch cache
 // A call with host x or y synchronises before it returns, so its kernels never overlap the
 // next call's, and the host cost of its launches (microseconds each) adds to its latency.
@@ -793,6 +807,55 @@ int nq_workspace_reserve(int64_t m, int64_t n, int64_t r, int64_t batch) {
     const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, m, n, r};
     Workspace* ws = workspace_for(m, n, r, batch, decode_need(&c, 1, batch), &st);
     return ws ? NQ_OK : st;
+}
+
+double nq_bits_per_weight_envelope(int64_t m, int64_t n, int64_t r, int64_t l) {
+    if (m <= 0 || n <= 0 || r <= 0 || l <= 0) return -1.0;
+    // r(m+n) one-bit sign entries + l pairs of fp16 scale vectors (16 l (m+n) bits)
+    return ((double)r * (double)(m + n) + 16.0 * (double)l * (double)(m + n)) / ((double)m * (double)n);
+}
+
+int nq_lowrank_linear_fwd_envelope(const void* x, const uint32_t* Upk, const uint32_t* Vpk, const void* a,
+                                   const void* b, int64_t l, int64_t m, int64_t n, int64_t r, int64_t batch, float* y,
+                                   void* stream) {
+    if (batch < 0) return NQ_ERR_BATCH;
+    if (l < 1 || l > kMaxGroup) return NQ_ERR_VALUE;
+    if (m <= 0 || n <= 0 || r <= 0 || m % 128 || n % 128 || r % 128 || m > kMaxDim || n > kMaxDim ||
+        r > kMaxRank)
+        return NQ_ERR_SHAPE;
+    if (batch > (int64_t(1) << 40) / (m > n ? m : n)) return NQ_ERR_SHAPE;
+    if (batch == 0) return NQ_OK;
+    if (!x || !Upk || !Vpk || !a || !b || !y) return NQ_ERR_NULL;
+    const void* ptrs[] = {x, Upk, Vpk, a, b, y};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return NQ_ERR_ALIGN;
+    for (const void* p : ptrs)
+        if (pointer_kind(p) != kDeviceMem) return NQ_ERR_PTRKIND;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* terms = nullptr;
+    if (l > 1) {
+        int st = NQ_OK;
+        Workspace* ws = workspace_for(m, n, r, 0, DecodeNeed(), &st);
+        if (!ws) return st;
+        if ((st = ensure_env_scratch(ws, sizeof(float) * (size_t)(l - 1) * (size_t)(batch * m))) != NQ_OK) return st;
+        terms = ws->env;
+    }
+    // term q: the layer with (s1, s2) = (a_q, b_q); term 0 into y, the others into scratch
+    nq_linear_desc d[kMaxGroup];
+    for (int64_t q = 0; q < l; ++q) {
+        d[q].x = x;
+        d[q].Upk = Upk;
+        d[q].Vpk = Vpk;
+        d[q].s1 = static_cast<const uint16_t*>(a) + q * m;
+        d[q].s2 = static_cast<const uint16_t*>(b) + q * n;
+        d[q].y = q == 0 ? y : terms + (q - 1) * batch * m;
+        d[q].m = m;
+        d[q].n = n;
+        d[q].r = r;
+    }
+    int st = grouped_run(d, sizeof(nq_linear_desc), nullptr, (int)l, batch, stream);
+    if (st != NQ_OK || l == 1) return st;
+    return envelope_sum_device(y, terms, (int)(l - 1), batch * m, s);
 }
 
 int nq_lowrank_linear_fwd(const void* x, const uint32_t* Upk, const uint32_t* Vpk, const void* s1,

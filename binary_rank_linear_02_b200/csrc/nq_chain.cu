@@ -194,6 +194,32 @@ int gather_device(const GatherList& list, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
 }
 
+// The rank-l envelope's sum: y[e] += terms[q][e] for q = 0 .. nterms-1 in that order
+// (y holds the first term), four elements per thread step.
+__global__ void __launch_bounds__(256) envelope_sum_kernel(float* __restrict__ y, const float* __restrict__ terms,
+                                                           int nterms, int64_t count) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t groups = count / 4;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < groups; g += stride) {
+        float4 acc = __ldcg(reinterpret_cast<const float4*>(y) + g);
+        for (int q = 0; q < nterms; ++q) {
+            const float4 t = __ldcg(reinterpret_cast<const float4*>(terms + (int64_t)q * count) + g);
+            acc.x += t.x;
+            acc.y += t.y;
+            acc.z += t.z;
+            acc.w += t.w;
+        }
+        reinterpret_cast<float4*>(y)[g] = acc;
+    }
+    for (int64_t i = groups * 4 + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count; i += stride) {
+        float acc = __ldcg(y + i);
+        for (int q = 0; q < nterms; ++q) acc += __ldcg(terms + (int64_t)q * count + i);
+        y[i] = acc;
+    }
+}
+
 int cast_f32_bf16_device(const float* src, int64_t count, uint16_t* dst, cudaStream_t stream) {
     int64_t blocks = (count / 8 + kCastThreads - 1) / kCastThreads;
     if (blocks < 1) blocks = 1;
@@ -233,6 +259,16 @@ int outer_device(const uint16_t* a, const uint16_t* s, const float* t, int64_t b
     const dim3 grid((unsigned)((R + kOuterTile - 1) / kOuterTile), (unsigned)((M + kOuterTile - 1) / kOuterTile));
     outer_kernel<<<grid, 256, 0, stream>>>(a, s, t, batch, M, R, out);
     return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
+}
+
+int envelope_sum_device(float* y, const float* terms, int nterms, int64_t count, cudaStream_t stream) {
+    int64_t blocks = (count / 4 + 255) / 256;
+    if (blocks < 1) blocks = 1;
+    if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
+    return launch_pdl(envelope_sum_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, y, terms, nterms, count) ==
+                   cudaSuccess
+               ? NQ_OK
+               : NQ_ERR_CUDA;
 }
 
 }  // namespace nq

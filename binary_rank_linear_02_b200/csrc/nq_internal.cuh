@@ -35,6 +35,8 @@ struct Workspace {
     uint16_t* ones = nullptr;      // [ones_count] fp16 1.0 (scale gradients: the layer without a scale)
     float* gstage = nullptr;       // scale gradients: batch x max(m, n) outputs of the layer without a scale
     size_t ones_count = 0, gstage_bytes = 0;
+    float* env = nullptr;          // envelope terms 1 .. l-1: (l-1) x batch x m fp32
+    size_t env_bytes = 0;
     size_t t_cap = 0, tgmax_cap = 0, partial_cap = 0, counter_cap = 0;
     int64_t r_cap = 0, n_cap = 0, m_cap = 0, batch_cap = 0, rsum_cap = 0;
 };
@@ -132,6 +134,8 @@ struct GatherList {
 };
 int gather_device(const GatherList& list, cudaStream_t stream);
 int cast_f32_bf16_device(const float* src, int64_t count, uint16_t* dst, cudaStream_t stream);
+// y[e] += terms[q * count + e] for q = 0 .. nterms-1 in order (the envelope's sum)
+int envelope_sum_device(float* y, const float* terms, int nterms, int64_t count, cudaStream_t stream);
 int rms_normalize_bf16_device(const float* src, int64_t rows, int64_t cols, uint16_t* dst, cudaStream_t stream);
 
 }  // namespace nq

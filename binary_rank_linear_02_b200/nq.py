@@ -94,6 +94,10 @@ def _load() -> ctypes.CDLL:
     L.nq_cast_f32_to_bf16.restype = ctypes.c_int
     L.nq_rms_normalize_bf16.argtypes = [p, i64, i64, p, p]
     L.nq_rms_normalize_bf16.restype = ctypes.c_int
+    L.nq_lowrank_linear_fwd_envelope.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, p, p]
+    L.nq_lowrank_linear_fwd_envelope.restype = ctypes.c_int
+    L.nq_bits_per_weight_envelope.argtypes = [i64, i64, i64, i64]
+    L.nq_bits_per_weight_envelope.restype = ctypes.c_double
     i32, f64 = ctypes.c_int, ctypes.c_double
     L.nq_admm_init.argtypes = [p, i64, i64, i64, p, i32, p, p, p, p, p, p, p, p, p]
     L.nq_admm_init.restype = ctypes.c_int
@@ -449,4 +453,24 @@ def admm_factorize(W, m: int, n: int, r: int, Omega, iters: int = 40, lam0: floa
                                   _ptr(Vpk), _ptr(s1), _ptr(s2), ctypes.byref(err), _stream(stream, W)),
            "nq_admm_factorize")
     return Upk, Vpk, s1, s2, err.value
+
+
+# ------------------------------------------------------------------ rank-l envelope variant
+
+def lowrank_linear_fwd_envelope(x, Upk, Vpk, a, b, m: int, n: int, r: int, y=None, stream=None):
+    """y = sum_q a_q * (U (V^T (b_q * x))): a is l x m fp16 bits, b is l x n (device tensors)."""
+    import torch
+
+    batch = x.shape[0]
+    l = a.shape[0]
+    if y is None:
+        y = torch.empty((batch, m), dtype=torch.float32, device=x.device)
+    st = _lib.nq_lowrank_linear_fwd_envelope(_ptr(x), _ptr(Upk), _ptr(Vpk), _ptr(a), _ptr(b), l, m, n, r, batch,
+                                             _ptr(y), _stream(stream, x, y))
+    _check(st, "nq_lowrank_linear_fwd_envelope")
+    return y
+
+
+def bits_per_weight_envelope(m: int, n: int, r: int, l: int) -> float:
+    return _lib.nq_bits_per_weight_envelope(m, n, r, l)
 

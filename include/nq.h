@@ -284,6 +284,31 @@ typedef struct nq_linear_desc_ex {
  */
 int nq_lowrank_linear_fwd_grouped_ex(const nq_linear_desc_ex* layers, int count, int64_t batch, void* stream);
 
+/*
+ * nq_lowrank_linear_fwd_envelope -- the rank-l envelope variant of the layer (MDBF-style
+ * scaling; hardwired.dev section "Kontext: co existuje kolem": MDBF replaces the simple
+ * scaling of the binary factorisation with a rank-l envelope, since under the simple
+ * scaling all rank components share one magnitude profile).  The library's reading:
+ *     W = (sum_{q<l} a_q b_q^T) (.) (U V^T),   y = sum_{q<l} a_q (.) (U (V^T (b_q (.) x))),
+ * l = 1 being nq_lowrank_linear_fwd with s1 = a_0, s2 = b_0 (bit for bit the same result).
+ *   a : l x m fp16 (row q = a_q);  b : l x n fp16 (row q = b_q);  1 <= l <= 16
+ *   x, Upk, Vpk, y, m, n, r, batch: as nq_lowrank_linear_fwd.  Every pointer device memory
+ *   of the current device (else NQ_ERR_PTRKIND), 16-byte aligned.
+ * The l terms run as one grouped call (layers sharing U and V: one decode launch pair for
+ * up to 8 tokens, or each term's prefill GEMMs), term 0 into y and the others into library
+ * scratch (allocated on first use of a size), then one kernel adds terms 1 .. l-1 to y in
+ * increasing q.  Asynchronous on `stream`; uses the workspace like the forward.
+ * Accuracy: each term within the forward's bound, so max|y - y_exact| <= 2e-3 * sum_q
+ * max|term_q| (tested: within 2e-3 of max|y_exact|, globally and per token, for l = 2, 4).
+ */
+int nq_lowrank_linear_fwd_envelope(const void* x, const uint32_t* Upk, const uint32_t* Vpk, const void* a,
+                                   const void* b, int64_t l, int64_t m, int64_t n, int64_t r, int64_t batch,
+                                   float* y, void* stream);
+
+/* Bits per weight of the envelope variant: (r*(m+n) + 16*l*(m+n)) / (m*n); -1.0 if any
+ * argument is <= 0.  Equals nq_bits_per_weight for l = 1. */
+double nq_bits_per_weight_envelope(int64_t m, int64_t n, int64_t r, int64_t l);
+
 /* Limits of nq_lowrank_linear_fwd_noalloc. */
 #define NQ_NOALLOC_MAX_RANK 4096
 #define NQ_NOALLOC_MAX_BATCH NQ_DECODE_MAX_BATCH

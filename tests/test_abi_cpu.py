@@ -267,3 +267,23 @@ def test_admm_argument_errors(nq):
     assert L.nq_admm_iterate(p[0], 256, 256, 128, *st, 1, 0.2, 0.0, 0) == nq.NQ_ERR_VALUE
     assert L.nq_admm_iterate(p[0], 256, 256, 100, *st, 1, 0.2, 1.05, 0) == nq.NQ_ERR_SHAPE
     assert L.nq_admm_iterate(p[0], 256, 256, 128, *st, 1, 0.2, 1.05, 0) == nq.NQ_ERR_PTRKIND
+
+
+def test_envelope_bits_per_weight_and_host_errors(nq):
+    """(r + 16 l)(m + n)/(m n) by hand: 4096 x 4096, r = 1664 -> 1696/2048 at l = 2,
+    1728/2048 at l = 4; l = 1 equals nq_bits_per_weight; argument errors on the host."""
+    assert nq.lib().nq_bits_per_weight_envelope(4096, 4096, 1664, 2) == 0.828125
+    assert nq.lib().nq_bits_per_weight_envelope(4096, 4096, 1664, 4) == 0.84375
+    assert nq.lib().nq_bits_per_weight_envelope(11008, 4096, 2432, 1) == nq.nq_bits_per_weight(11008, 4096, 2432)
+    assert nq.lib().nq_bits_per_weight_envelope(4096, 4096, 1664, 0) == -1.0
+    buf = np.zeros(1 << 16, dtype=np.uint8)
+    base = (buf.ctypes.data + 255) // 256 * 256
+    p = [base + 2048 * i for i in range(6)]
+    f = nq.lib().nq_lowrank_linear_fwd_envelope
+    assert f(p[0], p[1], p[2], p[3], p[4], 2, 128, 128, 128, -1, p[5], 0) == nq.NQ_ERR_BATCH
+    assert f(p[0], p[1], p[2], p[3], p[4], 0, 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_VALUE
+    assert f(p[0], p[1], p[2], p[3], p[4], 2, 100, 128, 128, 1, p[5], 0) == nq.NQ_ERR_SHAPE
+    assert f(p[0], p[1], p[2], 0, p[4], 2, 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_NULL
+    assert f(p[0], p[1], p[2], p[3] + 2, p[4], 2, 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_ALIGN
+    assert f(p[0], p[1], p[2], p[3], p[4], 2, 128, 128, 128, 1, p[5], 0) == nq.NQ_ERR_PTRKIND
+    assert f(p[0], p[1], p[2], p[3], p[4], 2, 128, 128, 128, 0, p[5], 0) == nq.NQ_OK
