@@ -364,6 +364,8 @@ def run_ours(args):
         return run_prefill_only(args, device, peaks)
     if args.workload == "chain7b":
         return run_chain_only(args, device, peaks)
+    if args.workload == "admm":
+        return run_admm_only(args, device, peaks)
     model, layers = DECODE_WORKLOADS[args.workload]
     batch = args.batch
     work = DecodeWorkload(layers, batch, seed=1234 + rank, device=device)
@@ -431,6 +433,8 @@ def run_ours(args):
         secondary["prefill_11008x4096_r2432"] = sweep
         prefill_roofline = prefill_roofline_of(sweep, peaks)
         secondary["chain_llama2-7b_32_blocks_b1"] = run_chain(device, stream, args.warmup, peaks)
+        secondary["envelope_llama2-7b_q_l2_b1"] = run_envelope(device, stream, peaks)
+        secondary["admm_init_llama2-7b_q"] = run_admm(device, stream, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -439,6 +443,8 @@ def run_ours(args):
             prefill_cpu = run_cpu_baseline_prefill(budget_s=max(3.0, args.cpu_seconds / 2))
             if prefill_roofline is not None:
                 prefill_roofline["cpu_baseline"] = prefill_cpu
+            if "admm_init_llama2-7b_q" in secondary:
+                secondary["admm_init_llama2-7b_q"]["cpu_baseline"] = run_cpu_baseline_admm()
 
     launches = args.steps * 2  # stage-1 and stage-2 kernels of one grouped call per step
     if rank == 0:
@@ -587,6 +593,110 @@ def run_chain(device, stream, warmup, peaks, passes=20, batch=1, nblocks=synth.C
     return out
 
 
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # SMs x fp32 lanes x 2 flops (FMA) x max clock
+
+
+def admm_flops_per_iteration(m, n, r):
+    """Algorithmic flops of one ADMM iteration (both half-steps): the W products 2 x 2mnr,
+    the Gram matrices 2 x 2r^2 (m or n), the two triangular solves of each side 2 x 2r^2
+    (n or m), two Cholesky factorisations 2 x r^3/3."""
+    return 4.0 * m * n * r + 4.0 * r * r * (m + n) + 2.0 * r ** 3 / 3.0
+
+
+def run_admm(device, stream, peaks, iters=40, shape=(4096, 4096, 1664), repeats=3):
+    """The LB-ADMM initialiser on a synthetic Llama-2-7B attention-shaped weight: time of the
+    whole nq_admm_factorize call (start, iterations, balancing, packing, error), and of the
+    iterations alone from the per-iteration difference of two call lengths."""
+    import torch
+
+    from binary_rank_linear_02_b200 import nq
+
+    m, n, r = shape
+    W = torch.from_numpy(synth.weights_bf16(m, n, 8080).view(np.int16)).to(device)
+    Om = torch.from_numpy(synth.gaussian_f32(n, r, 8080, "omega")).to(device)
+
+    def one(k):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        out = nq.admm_factorize(W, m, n, r, Om, iters=k)
+        torch.cuda.synchronize()
+        return time.perf_counter() - t0, out[4]
+
+    one(2)  # warm-up (module load, first allocations)
+    t_short = statistics.median([one(2)[0] for _ in range(repeats)])
+    runs = [one(iters) for _ in range(repeats)]
+    t_full = statistics.median([t for t, _ in runs])
+    err = runs[0][1]
+    per_it = (t_full - t_short) / (iters - 2)
+    fl = admm_flops_per_iteration(m, n, r)
+    tf = fl / per_it / 1e12
+    return {"shape": f"{m}x{n} r={r}", "iters": iters, "seconds_per_call": round(t_full, 4),
+            "ms_per_iteration": round(per_it * 1e3, 3), "gflop_per_iteration": round(fl / 1e9, 1),
+            "tflops": round(tf, 2), "rel_err": round(err, 5),
+            "roofline": {"bound": "alu", "achieved": round(tf, 2), "peak": round(FP32_ALU_TFLOPS, 1),
+                         "unit": "TFLOP/s", "frac": round(tf / FP32_ALU_TFLOPS, 4),
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"},
+            "timing": "wall clock around the synchronising call (host-side allocation included), median"}
+
+
+def run_envelope(device, stream, peaks, steps=200, batch=1, l=2, shape=(4096, 4096, 1664)):
+    """The rank-l envelope forward on the Llama-2-7B q shape, back to back over rotating
+    weight copies, against the plain forward on the same copies."""
+    import torch
+
+    from binary_rank_linear_02_b200 import nq
+
+    m, n, r = shape
+    pb = packed_bytes(m, n, r)
+    copies = max(1, -(-2 * L2_BYTES // pb))
+    gen = torch.Generator(device=device)
+    gen.manual_seed(9090)
+    sets = [(torch.randint(-(1 << 31), 1 << 31, (m, r // 32), dtype=torch.int64, device=device, generator=gen).to(torch.int32),
+             torch.randint(-(1 << 31), 1 << 31, (r, n // 32), dtype=torch.int64, device=device, generator=gen).to(torch.int32))
+            for _ in range(copies)]
+    a = torch.from_numpy(np.stack([synth.scales_f16(m, 9090, "a", q) for q in range(l)]).view(np.int16)).to(device)
+    b = torch.from_numpy(np.stack([synth.scales_f16(n, 9090, "b", q) for q in range(l)]).view(np.int16)).to(device)
+    x = torch.from_numpy(synth.activations_bf16(batch, n, 9090).view(np.int16)).to(device)
+    y = torch.empty((batch, m), dtype=torch.float32, device=device)
+    env, fwd = nq.lib().nq_lowrank_linear_fwd_envelope, nq.lib().nq_lowrank_linear_fwd
+
+    def step_env(i, h):
+        U, V = sets[i % copies]
+        st = env(x.data_ptr(), U.data_ptr(), V.data_ptr(), a.data_ptr(), b.data_ptr(), l, m, n, r, batch, y.data_ptr(), h)
+        if st != 0:
+            raise RuntimeError(nq.nq_status_string(st))
+
+    def step_fwd(i, h):
+        U, V = sets[i % copies]
+        st = fwd(x.data_ptr(), U.data_ptr(), V.data_ptr(), a.data_ptr(), b.data_ptr(), m, n, r, batch, y.data_ptr(), h)
+        if st != 0:
+            raise RuntimeError(nq.nq_status_string(st))
+
+    out = {"shape": f"{m}x{n} r={r}", "l": l, "batch": batch, "packed_bytes": pb}
+    for name, fn in (("envelope", step_env), ("plain", step_fwd)):
+        with torch.cuda.stream(stream):
+            fn(0, stream.cuda_stream)
+        torch.cuda.synchronize()
+        g = capture(lambda h: [fn(i, h) for i in range(steps)], stream)
+        g.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(3):
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                start.record(stream)
+                g.replay()
+                end.record(stream)
+            torch.cuda.synchronize()
+            times.append(start.elapsed_time(end) / steps)
+        ms = statistics.median(times)
+        gbs = pb / (ms * 1e-3) / 1e9
+        out[name] = {"us_per_call": round(ms * 1e3, 2), "packed_gbs": round(gbs, 1),
+                     "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        del g
+    return out
+
+
 def run_chain_only(args, device, peaks):
     """--workload chain7b: the decode chain alone, one JSON line (tokens/s of the chain)."""
     import torch
@@ -610,6 +720,25 @@ def run_chain_only(args, device, peaks):
                          "kernel": "every decode kernel of one chain pass"},
             "cpu_baseline": cpu,
             "gpu_launches": c["kernels_per_pass"] * max(1, args.steps), "clocks": clocks, "chain": c}
+    print(json.dumps(line), flush=True)
+
+
+def run_admm_only(args, device, peaks):
+    """--workload admm: the LB-ADMM initialiser alone on the 4096x4096 r=1664 problem
+    (--admm-iters iterations per call), one JSON line, TFLOP/s of its iterations."""
+    import torch
+
+    stream = torch.cuda.Stream(device)
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    a = run_admm(device, stream, peaks, iters=args.admm_iters, repeats=args.repeats)
+    clocks = sampler.stop()
+    cpu = None if args.no_cpu_baseline else run_cpu_baseline_admm()
+    line = {"metric": METRIC, "value": a["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.admm_iters,
+            "warmup": 1, "ms_per_step": a["ms_per_iteration"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32 (W read as bf16)", "data": "synthetic",
+            "config": {"workload": f"LB-ADMM initialiser, {a['shape']}, {args.admm_iters} iterations per call"},
+            "roofline": a["roofline"], "cpu_baseline": cpu, "clocks": clocks, "admm": a}
     print(json.dumps(line), flush=True)
 
 
@@ -774,6 +903,26 @@ def run_cpu_baseline_chain(budget_s, nblocks=synth.CHAIN_7B_BLOCKS):
                       f"({dt:.1f} s)"}
 
 
+def run_cpu_baseline_admm(shape=(4096, 4096, 1664), iters=2):
+    """The oracle's ADMM iterations on the host cores (numpy fp64) for the same shape: the
+    start, then `iters` iterations timed; TFLOP/s over the same algorithmic flops."""
+    import oracle.admm as adm
+
+    m, n, r = shape
+    W = adm.decode_bf16(synth.weights_bf16(m, n, 8080))
+    Om = synth.gaussian_f32(n, r, 8080, "omega").astype(np.float64)
+    st = adm.start_state(*adm.power_iteration_init(W, Om, 1))
+    t0 = time.perf_counter()
+    for k in range(iters):
+        st = adm.admm_step(W, st, 0.2 * 1.05 ** k)
+    dt = (time.perf_counter() - t0) / iters
+    import os as _os
+
+    return {"value": round(admm_flops_per_iteration(m, n, r) / dt / 1e12, 4), "unit": "TFLOP/s",
+            "cores": _os.cpu_count(), "kind": "oracle", "seconds_per_iteration": round(dt, 3),
+            "sample": f"{iters} ADMM iteration(s) of the {m}x{n} r={r} problem on the numpy fp64 oracle"}
+
+
 def prefill_config(batches):
     _, m, n, r = synth.PREFILL_SHAPE
     return {"workload": f"prefill {m}x{n} r={r}, token batch {max(batches)} "
@@ -824,7 +973,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", dest="secondary", action="store_false")
-    ap.add_argument("--workload", choices=["decode70b", "decode7b", "prefill", "chain7b"], default="decode70b")
+    ap.add_argument("--workload", choices=["decode70b", "decode7b", "prefill", "chain7b", "admm"], default="decode70b")
+    ap.add_argument("--admm-iters", type=int, default=40)
     ap.add_argument("--repeats", type=int, default=5)
     ap.add_argument("--prefill-batch", type=int, default=0)
     args = ap.parse_args()
