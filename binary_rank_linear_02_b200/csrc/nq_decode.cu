@@ -51,6 +51,7 @@
 #include <mutex>
 
 #include "nq_internal.cuh"
+#include "nq_sm100.cuh"
 
 namespace nq {
 namespace {
@@ -76,9 +77,11 @@ constexpr int kS2SumMaxSplits = 12;    // ... for groups whose layers have at mo
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 __device__ __forceinline__ float f16_to_f32(uint16_t h) { return __half2float(__ushort_as_half(h)); }
 
+// Not volatile: the instruction only writes its registers, so the compiler may schedule it
+// freely against the loads around it.
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};\n"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
@@ -155,6 +158,11 @@ struct DecGroup {
     int s2_start[kMaxGroup + 1];
     unsigned char s1_layer[kMaxGroup];
     unsigned char s2_layer[kMaxGroup];
+    // streaming stage 2 (stage2s_kernel): prefixes over the layers in their own order of
+    // 128-row units (u_start) and of their 1024-column stages (st_start)
+    int stream2;
+    int u_start[kMaxGroup + 1];
+    int st_start[kMaxGroup + 1];
 };
 
 // The range of `block` (an index into start[]).
@@ -890,6 +898,348 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
     if (L.y_norm) rms_norm_epilogue(L, batch, rows, blk, mi, y_at);
 }
 
+// ------------------------------------------------------------------ stage 2, streaming
+// For launches whose weights do not fit on chip in one wave (the Llama-2-70B-shaped block:
+// 36.5 MB of U against ~33 MB of shared memory on all SMs), one persistent CTA per SM streams
+// an even share of all the layers' weight stages through a ring in shared memory, instead of
+// waves of CTAs that each load, then compute.  A unit is one 256-row block of a layer over
+// all r columns; a stage is 1024 columns of it (one TMA box of 256 rows x 32 words, 32 KB,
+// 128-byte swizzle).  CTA c takes stages [c S / P, (c+1) S / P) of the S stages of all units
+// in layer order, so every CTA streams the same number of bytes to within one stage.
+// The last warp issues the TMA loads (the weights do not depend on stage 1, so the ring
+// fills while the CTA waits for t); the 16 others multiply one 16-row tile each against B
+// fragments of t built once per layer (t staged into shared memory in slices with one
+// batch of asynchronous copies each; all of r, one exponent per token), loading fragment
+// words only in the lanes that hold a token.  (Templated for two token groups as two tiles
+// per warp, which measured slower than the classic kernel and is not launched.)
+// A unit cut by a CTA boundary is finished by the last of its CTAs to arrive: each writes
+// its integer row sums to its own slot, and the last adds the slots in CTA order (integer
+// sums: exact, so the result does not depend on the arrival order).  Every wait on an
+// mbarrier is bounded (NQ_ERR_TIMEOUT in the status word, then the CTA drains its loads).
+constexpr int kS2sRows = 256;                                     // rows per unit
+constexpr int kS2sBoxWords = 32;                                  // columns per stage / 32
+constexpr int kS2sStageBytes = kS2sRows * kS2sBoxWords * 4;       // 32 KB
+constexpr int kS2sStages = 4;
+constexpr int kS2sMaxRank = 4096;                                 // fragments of all of r on chip
+constexpr int kS2sMaxParts = 4;                                   // CTAs that may share a unit
+__host__ __device__ constexpr int s2s_consumers(int ntg) { return ntg == 1 ? 16 : 8; }
+__host__ __device__ constexpr int s2s_tpw(int ntg) { return ntg == 1 ? 1 : 2; }
+__host__ __device__ constexpr int s2s_threads(int ntg) { return 32 * (s2s_consumers(ntg) + 1); }
+__host__ __device__ constexpr int s2s_tstage_floats(int ntg) { return ntg == 1 ? 8192 : 4096; }
+
+struct S2sMaps {
+    CUtensorMap map[kMaxGroup];  // Upk of each layer: rows m, cols r/32 words
+};
+
+struct S2sBarriers {
+    unsigned long long full[kS2sStages], empty[kS2sStages];
+    int abort_flag;
+    int last;
+};
+
+__host__ __device__ inline size_t s2s_frag_offset() { return (size_t)kS2sStages * kS2sStageBytes; }
+__host__ __device__ inline size_t s2s_tstage_offset(int ntg) {
+    return s2s_frag_offset() + frag_bytes(kS2sMaxRank / kCB, ntg);
+}
+__host__ __device__ inline size_t s2s_misc_offset(int ntg) {
+    return s2s_tstage_offset(ntg) + (size_t)s2s_tstage_floats(ntg) * 4;
+}
+__host__ __device__ inline size_t s2s_bar_offset(int ntg) { return (s2s_misc_offset(ntg) + sizeof(Misc) + 15) / 16 * 16; }
+__host__ __device__ inline size_t s2s_bytes(int ntg) {
+    return s2s_bar_offset(ntg) + sizeof(S2sBarriers) + 1024 /*alignment slack*/;
+}
+
+template <int NTG, bool CM>
+__global__ void __launch_bounds__(s2s_threads(NTG), 1)
+stage2s_kernel(const __grid_constant__ DecGroup grp, const __grid_constant__ S2sMaps maps, unsigned* status,
+               int* part, int* part_cnt) {
+    constexpr int NC = s2s_consumers(NTG), TPW = s2s_tpw(NTG), NCT = 32 * NC;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;  // 128-byte swizzle wants 1024-byte aligned stages
+    unsigned char* gbase = smem_raw + (base - raw);
+    uint4* frag = reinterpret_cast<uint4*>(gbase + s2s_frag_offset());
+    float* tst = reinterpret_cast<float*>(gbase + s2s_tstage_offset(NTG));
+    Misc& mi = *reinterpret_cast<Misc*>(gbase + s2s_misc_offset(NTG));
+    S2sBarriers& bar = *reinterpret_cast<S2sBarriers*>(gbase + s2s_bar_offset(NTG));
+    volatile int* abort_flag = &bar.abort_flag;
+    const int batch = grp.batch;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+
+    // this CTA's stages [lo, hi) of all units' stages; unit u of layer k has stages
+    // st_start[k] + (u - u_start[k]) * nst_k ..
+    const int S = grp.st_start[grp.count];
+    const int P = gridDim.x;
+    const int lo = (int)((int64_t)blockIdx.x * S / P), hi = (int)((int64_t)(blockIdx.x + 1) * S / P);
+    auto layer_of_stage = [&](int st) {
+        int k = 0;
+        while (k + 1 < grp.count && st >= grp.st_start[k + 1]) ++k;
+        return k;
+    };
+    auto nst_of = [&](int k) { return (grp.L[k].r + 1023) / 1024; };
+    auto cta_of_stage = [&](int st) {  // the CTA whose range holds stage st
+        int c = (int)(((int64_t)st * P) / S);
+        while (c + 1 < P && (int64_t)(c + 1) * S / P <= st) ++c;
+        while (c > 0 && (int64_t)c * S / P > st) --c;
+        return c;
+    };
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < kS2sStages; ++st) {
+            mbar_init(smem_u32(&bar.full[st]), 1);
+            mbar_init(smem_u32(&bar.empty[st]), NC);
+        }
+        bar.abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == NC) {
+        // ---------------- producer: the CTA's stages, in order
+        if (lane == 0) {
+            int slot = 0, issued = 0;
+            uint32_t ph = 0;
+            for (int st = lo; st < hi && !*abort_flag; ++st) {
+                const int k = layer_of_stage(st);
+                const int off = st - grp.st_start[k], nst = nst_of(k);
+                const int rb = off / nst, c = off % nst;
+                if (!mbar_wait(smem_u32(&bar.empty[slot]), ph ^ 1u, abort_flag, status)) break;
+                mbar_expect_tx(smem_u32(&bar.full[slot]), (uint32_t)kS2sStageBytes);
+                tma_load_2d(base + (uint32_t)(slot * kS2sStageBytes), &maps.map[k], c * kS2sBoxWords, rb * kS2sRows,
+                            smem_u32(&bar.full[slot]));
+                ++issued;
+                if (++slot == kS2sStages) {
+                    slot = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (*abort_flag) {
+                // let the loads already issued land before the shared memory goes away
+                for (int q = issued - kS2sStages < 0 ? 0 : issued - kS2sStages; q < issued; ++q)
+                    mbar_drain(smem_u32(&bar.full[q % kS2sStages]), (uint32_t)(q / kS2sStages) & 1u);
+            }
+        }
+        pdl_trigger();
+        return;
+    }
+
+    // ---------------- consumers (threads 0 .. NCT-1)
+    pdl_trigger();
+    zero_fragments<NTG, NCT>(frag, kS2sMaxRank / kCB);
+    pdl_wait();  // t and its block maxima come from stage 1
+    auto consumer_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(NCT) : "memory"); };
+    int cur = -1, slot = 0;
+    uint32_t ph = 0;
+    int st = lo;
+    while (st < hi) {
+        const int k = layer_of_stage(st);
+        const DecLayer& L = grp.L[k];
+        const int r = L.r, ncb = r / kCB, nst = nst_of(k);
+        const int off = st - grp.st_start[k];
+        const int rb = off / nst, c_first = off % nst;
+        const int c_last = min(nst, c_first + (hi - st));  // stages of this unit in this CTA: [c_first, c_last)
+        if (k != cur) {
+            // the layer's exponent per token (from stage 1's block maxima) and its fragments,
+            // t staged into shared memory a slice of columns at a time
+            consumer_sync();
+            const int nrb = r / kRowsS1;
+            for (int tok = warp; tok < batch; tok += NC) {
+                float mx = 0.f;
+                for (int gi = lane; gi < nrb; gi += 32) mx = fmaxf(mx, __ldcg(L.tgmax + (int64_t)tok * nrb + gi));
+                mx = warp_max(mx);
+                if (lane == 0) {
+                    const int e = range_exponent(mx);
+                    mi.e[tok] = e;
+                    mi.up[tok] = pow2f(kQBits - e);
+                    mi.qsum[tok] = 0;
+                }
+            }
+            const int slice = min(r, s2s_tstage_floats(NTG) / batch / kCB * kCB);  // columns per slice
+            for (int c0 = 0; c0 < r; c0 += slice) {
+                const int cols = min(slice, r - c0);
+                consumer_sync();  // the previous slice is consumed (and the maxima are written)
+                for (int i = threadIdx.x; i < batch * cols / 4; i += NCT) {
+                    const int tok = i / (cols / 4), p = i % (cols / 4);
+                    cp_async16(tst + tok * slice + 4 * p, L.t + (int64_t)tok * r + c0 + 4 * p);
+                }
+                cp_async_commit();
+                cp_async_wait<0>();
+                consumer_sync();
+                auto tval = [&](int tok, int cc) { return tst[tok * slice + cc]; };
+                uint4* fslice = frag + (size_t)(c0 / kCB) * NTG * 2 * 32;
+                if constexpr (NTG == 2 || CM)
+                    build_fragments2<NTG, NCT>(fslice, mi, tval, [](int) { return 1.0f; }, cols / kCB, batch);
+                else
+                    build_fragments<NTG, NCT>(fslice, mi, tval, cols / kCB, batch);
+            }
+            consumer_sync();
+            cur = k;
+        }
+        int acc[TPW][NTG][4][4], acc2[TPW][NTG][4][4];
+#pragma unroll
+        for (int tl = 0; tl < TPW; ++tl) {
+            zero_acc<NTG>(acc[tl]);
+            zero_acc<NTG>(acc2[tl]);
+        }
+        // rows 16 TPW warp + g (+ 8, + 16, + 24) of the stage: all have row & 7 == g
+        const uint32_t row_off = (uint32_t)((16 * TPW * warp + g) * 128);
+        // B fragments: lane l carries column n = l / 4 of the MMA (token n / 2 of its group,
+        // limb n % 2); lanes of absent tokens hold zeros, so only the lanes with a token
+        // load (at batch 1: 8 of 32 lanes, a quarter of the shared-memory wavefronts)
+        auto load_frag = [&](int gcb, int tg, uint4& f0, uint4& f1) {
+            f0 = f1 = make_uint4(0u, 0u, 0u, 0u);
+            if (lane < 8 * (batch - 4 * tg)) {
+                f0 = *frag_ptr<NTG>(frag, gcb, tg, 0, lane);
+                f1 = *frag_ptr<NTG>(frag, gcb, tg, 1, lane);
+            }
+        };
+        bool ok = true;
+        for (int c = c_first; c < c_last; ++c) {
+            if (!mbar_wait(smem_u32(&bar.full[slot]), ph, abort_flag, status)) {
+                ok = false;
+                break;
+            }
+            // plain loads (not volatile asm), so that the compiler can issue the next column
+            // blocks' loads ahead of this one's MMAs; the stage's bytes are visible after the
+            // mbarrier wait (a memory clobber)
+            const uint32_t* st_row =
+                reinterpret_cast<const uint32_t*>(gbase + (size_t)slot * kS2sStageBytes + row_off);
+            const int cb_n = min(8, ncb - 8 * c);
+            // one column block into accumulator set A (an explicit function of the block, so
+            // that the two sets alternate without a run-time test)
+            auto block = [&](int cb, int (&A)[TPW][NTG][4][4]) {
+                // chunk cb of the row sits at chunk cb ^ (row & 7) = cb ^ g
+                const uint32_t* a = st_row + ((cb ^ g) << 2) + tq;
+                const int gcb = 8 * c + cb;
+                if constexpr (TPW == 1) {
+                    const uint32_t wa = a[0], wb = a[256];  // rows g and g + 8 (8 rows x 32 words apart)
+                    const uint32_t x0 = wa >> 4, y0 = wb >> 4;
+#pragma unroll
+                    for (int tg = 0; tg < NTG; ++tg) {
+                        uint4 f0, f1;
+                        load_frag(gcb, tg, f0, f1);
+                        const uint32_t bf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+#pragma unroll
+                        for (int sft = 0; sft < 4; ++sft) {
+                            const uint32_t M = 0x01010101u << sft;
+                            mma_u8s8(A[0][tg][sft], wa & M, wb & M, x0 & M, y0 & M, bf[2 * sft], bf[2 * sft + 1]);
+                        }
+                    }
+                } else {
+                    const uint32_t wa0 = a[0], wb0 = a[256], wa1 = a[512], wb1 = a[768];
+                    const uint32_t x0 = wa0 >> 4, y0 = wb0 >> 4, x1 = wa1 >> 4, y1 = wb1 >> 4;
+#pragma unroll
+                    for (int tg = 0; tg < NTG; ++tg) {
+                        uint4 f0, f1;
+                        load_frag(gcb, tg, f0, f1);
+                        const uint32_t bf[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+#pragma unroll
+                        for (int sft = 0; sft < 4; ++sft) {
+                            const uint32_t M = 0x01010101u << sft;
+                            mma_u8s8(A[0][tg][sft], wa0 & M, wb0 & M, x0 & M, y0 & M, bf[2 * sft], bf[2 * sft + 1]);
+                            mma_u8s8(A[1][tg][sft], wa1 & M, wb1 & M, x1 & M, y1 & M, bf[2 * sft], bf[2 * sft + 1]);
+                        }
+                    }
+                }
+            };
+            if (cb_n == 8) {
+#pragma unroll
+                for (int cb = 0; cb < 8; cb += 2) {
+                    block(cb, acc);
+                    block(cb + 1, acc2);
+                }
+            } else {
+                int cb = 0;
+                for (; cb + 1 < cb_n; cb += 2) {
+                    block(cb, acc);
+                    block(cb + 1, acc2);
+                }
+                if (cb < cb_n) block(cb, acc);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bar.empty[slot]));
+            if (++slot == kS2sStages) {
+                slot = 0;
+                ph ^= 1u;
+            }
+        }
+        if (!ok) break;
+        // the warp's integer row sums: bq[tl][tg][0] for row g, [1] for row g + 8
+        int bq[TPW][NTG][2];
+#pragma unroll
+        for (int tl = 0; tl < TPW; ++tl) {
+#pragma unroll
+            for (int tg = 0; tg < NTG; ++tg)
+#pragma unroll
+                for (int sft = 0; sft < 4; ++sft)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[tl][tg][sft][i] += acc2[tl][tg][sft][i];
+#pragma unroll
+            for (int tg = 0; tg < NTG; ++tg) combine<NTG>(acc[tl], tg, bq[tl][tg][0], bq[tl][tg][1]);
+        }
+        const int64_t m = L.m;
+        const int64_t row_base = (int64_t)rb * kS2sRows + 16 * TPW * warp + g;  // + 16 tl (+ 8)
+        auto store_y = [&](int tok, int64_t row, int64_t q) {  // q = 2 sum b q - sum q of (row, tok)
+            if (row >= m) return;
+            const float y = f16_to_f32(__ldg(L.s1 + row)) * ((float)q * pow2f(mi.e[tok] - kQBits));
+            L.y[tok * m + row] = y;
+            if (L.y_bf16) L.y_bf16[tok * m + row] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+        };
+        const bool whole = c_first == 0 && c_last == nst;
+        if (whole) {
+#pragma unroll
+            for (int tl = 0; tl < TPW; ++tl)
+#pragma unroll
+                for (int tg = 0; tg < NTG; ++tg) {
+                    const int tok = 4 * tg + tq;
+                    if (tok < batch) {
+                        const int64_t qs = mi.qsum[tok];
+                        store_y(tok, row_base + 16 * tl, 2 * (int64_t)bq[tl][tg][0] - qs);
+                        store_y(tok, row_base + 16 * tl + 8, 2 * (int64_t)bq[tl][tg][1] - qs);
+                    }
+                }
+        } else {
+            // a unit shared with other CTAs: this CTA's integer sums into its own slot, then
+            // the last to arrive adds the slots in CTA order and writes y.  Slot of the unit:
+            // the index of the first CTA boundary inside it (unique per shared unit).
+            const int ust = grp.st_start[k] + rb * nst;  // the unit's first stage
+            const int c0 = cta_of_stage(ust);
+            const int cnt_all = cta_of_stage(ust + nst - 1) - c0 + 1;
+            const int slotu = c0 + 1, me = blockIdx.x - c0;
+            int* mine = part + ((int64_t)slotu * kS2sMaxParts + me) * (kS2sRows * 8);
+#pragma unroll
+            for (int tl = 0; tl < TPW; ++tl)
+#pragma unroll
+                for (int tg = 0; tg < NTG; ++tg) {
+                    const int tok = 4 * tg + tq;
+                    if (tok < batch) {
+                        const int rr = 16 * TPW * warp + 16 * tl + g;
+                        mine[rr * 8 + tok] = bq[tl][tg][0];
+                        mine[(rr + 8) * 8 + tok] = bq[tl][tg][1];
+                    }
+                }
+            consumer_sync();
+            if (threadIdx.x == 0) {
+                __threadfence();
+                bar.last = atomicAdd(part_cnt + slotu, 1) == cnt_all - 1;
+                if (bar.last) __threadfence();
+            }
+            consumer_sync();
+            if (bar.last) {
+                const int* slots = part + (int64_t)slotu * kS2sMaxParts * (kS2sRows * 8);
+                for (int i = threadIdx.x; i < kS2sRows * batch; i += NCT) {
+                    const int rr = i / batch, tok = i % batch;
+                    int64_t sum = 0;
+                    for (int q = 0; q < cnt_all; ++q) sum += __ldcg(slots + q * (kS2sRows * 8) + rr * 8 + tok);
+                    store_y(tok, (int64_t)rb * kS2sRows + rr, 2 * sum - mi.qsum[tok]);
+                }
+                if (threadIdx.x == 0) part_cnt[slotu] = 0;  // ready for the next call
+            }
+        }
+        st += c_last - c_first;
+    }
+}
+
 template <typename K>
 static bool set_kernel_attributes(K kernel) {
     // the largest shared-memory carveout for every decode kernel, so that CTAs of the two
@@ -900,12 +1250,17 @@ static bool set_kernel_attributes(K kernel) {
 }
 
 template <int NTG, bool CM>
-int launch_stages(DecGroup& grp, cudaStream_t stream, int device, bool stage1_only) {
+int launch_stages(DecGroup& grp, cudaStream_t stream, int device, bool stage1_only, const S2sMaps* maps,
+                  unsigned* status, int* s2s_part, int* s2s_cnt) {
     static unsigned long long init_mask = 0;  // devices whose kernel attributes are set
     const unsigned long long bit = 1ull << (device & 63);
     if (!(__atomic_load_n(&init_mask, __ATOMIC_ACQUIRE) & bit)) {
         if (!set_kernel_attributes(stage1_kernel<NTG, 2, CM>) || !set_kernel_attributes(stage2_kernel<NTG, CM>))
             return NQ_ERR_CUDA;
+        if constexpr (NTG == 1)
+            if (cudaFuncSetAttribute(stage2s_kernel<NTG, CM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)s2s_bytes(NTG)) != cudaSuccess)
+                return NQ_ERR_CUDA;
         if constexpr (NTG == 1)
             if (!set_kernel_attributes(stage1_kernel<1, 1, CM>)) return NQ_ERR_CUDA;
         __atomic_fetch_or(&init_mask, bit, __ATOMIC_RELEASE);
@@ -929,6 +1284,16 @@ int launch_stages(DecGroup& grp, cudaStream_t stream, int device, bool stage1_on
     }
     if (err != cudaSuccess) return NQ_ERR_CUDA;
     if (stage1_only) return NQ_OK;
+    if constexpr (NTG == 1) {
+        if (grp.stream2) {
+            const int stages = grp.st_start[grp.count];
+        const int grid2 = std::min(stages, sm_count());  // every CTA has at least one stage
+            return launch_pdl(stage2s_kernel<NTG, CM>, dim3((unsigned)grid2), dim3(s2s_threads(NTG)),
+                              s2s_bytes(NTG), stream, grp, *maps, status, s2s_part, s2s_cnt) == cudaSuccess
+                       ? NQ_OK
+                       : NQ_ERR_CUDA;
+        }
+    }
     if (launch_pdl(stage2_kernel<NTG, CM>, dim3((unsigned)grp.s2_start[grp.count]), dim3(kThreads), smem2, stream,
                    grp) != cudaSuccess)
         return NQ_ERR_CUDA;
@@ -936,10 +1301,12 @@ int launch_stages(DecGroup& grp, cudaStream_t stream, int device, bool stage1_on
 }
 
 template <int NTG>
-int launch_group(DecGroup& grp, cudaStream_t stream, int device, bool stage1_only) {
+int launch_group(DecGroup& grp, cudaStream_t stream, int device, bool stage1_only, const S2sMaps* maps,
+                 unsigned* status, int* s2s_part, int* s2s_cnt) {
     if constexpr (NTG == 1)
-        if (grp.batch >= kColMajorMinBatch) return launch_stages<1, true>(grp, stream, device, stage1_only);
-    return launch_stages<NTG, false>(grp, stream, device, stage1_only);
+        if (grp.batch >= kColMajorMinBatch)
+            return launch_stages<1, true>(grp, stream, device, stage1_only, maps, status, s2s_part, s2s_cnt);
+    return launch_stages<NTG, false>(grp, stream, device, stage1_only, maps, status, s2s_part, s2s_cnt);
 }
 
 }  // namespace
@@ -1036,11 +1403,29 @@ static int stage1_cps(const DecodeCall* calls, int count, int max_splits) {
     return (int)cps;
 }
 
+// Scratch of the streaming stage 2's shared units: per CTA boundary, kS2sMaxParts slots of
+// 256 rows x 8 tokens of integer sums, and one arrival counter.
+static int64_t s2s_part_ints() { return (int64_t)(sm_count() + 1) * kS2sMaxParts * kS2sRows * 8; }
+static int64_t s2s_counter_ints() { return sm_count() + 1; }
+
+// Whether the layers' shapes take the streaming stage 2: all of r fits its fragment buffer,
+// no layer asks for the normalised output, and the classic plan finds no one-wave layout.
+static bool s2s_shapes(const DecodeCall* calls, int count, int per_sm2) {
+    int64_t r_max = 0;
+    bool any_norm = false;
+    for (int i = 0; i < count; ++i) {
+        r_max = calls[i].r > r_max ? calls[i].r : r_max;
+        any_norm = any_norm || calls[i].y_norm != nullptr;
+    }
+    return !any_norm && r_max <= kS2sMaxRank && per_sm2 == 0;
+}
+
 void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, int max_splits, int64_t* t_floats,
                            int64_t* tgmax_floats, int64_t* partial_floats, int64_t* counter_ints) {
     const int cps = stage1_cps(calls, count, max_splits);
     int ctas[kMaxGroup], w2words = 0, rows2 = 0, per_sm = 0;
     stage2_plan(calls, count, batch, ctas, &w2words, &rows2, &per_sm);
+    const bool s2s = s2s_shapes(calls, count, per_sm);
     int64_t t = 0, gm = 0, pf = 0, ci = 0;
     for (int i = 0; i < count; ++i) {
         const int64_t ncb = calls[i].n / kCB, nsplit = (ncb + cps - 1) / cps;
@@ -1055,8 +1440,10 @@ void decode_workspace_need(const DecodeCall* calls, int count, int64_t batch, in
     }
     *t_floats = t;
     *tgmax_floats = gm;
-    *partial_floats = pf;
-    *counter_ints = ci;
+    // the streaming stage 2's scratch comes last (decode_forward_group uses the stage only
+    // when the workspace holds it)
+    *partial_floats = pf + (s2s ? s2s_part_ints() : 0);
+    *counter_ints = ci + (s2s ? s2s_counter_ints() : 0);
 }
 
 int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Workspace* ws, cudaStream_t stream,
@@ -1064,6 +1451,18 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
     if (count < 1 || count > kMaxGroup) return NQ_ERR_SHAPE;
     int64_t need_t, need_g, need_p, need_c;
     decode_workspace_need(calls, count, batch, max_splits, &need_t, &need_g, &need_p, &need_c);
+    // the streaming stage 2 is optional: without room for its scratch the classic one runs
+    bool s2s_room = (size_t)need_p <= ws->partial_cap && (size_t)need_c <= ws->counter_cap;
+    {
+        int ctas0[kMaxGroup], w0 = 0, r0 = 0, ps0 = 0;
+        stage2_plan(calls, count, batch, ctas0, &w0, &r0, &ps0);
+        if (s2s_shapes(calls, count, ps0)) {
+            need_p -= s2s_part_ints();
+            need_c -= s2s_counter_ints();
+        } else {
+            s2s_room = false;
+        }
+    }
     if ((size_t)need_t > ws->t_cap || (size_t)need_g > ws->tgmax_cap || (size_t)need_p > ws->partial_cap ||
         (size_t)need_c > ws->counter_cap)
         return NQ_ERR_NOMEM;
@@ -1085,7 +1484,16 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
     // subset of its layers (36.5 -> 37.0-38.8 us), so it keeps the hand-off.
     int max_nsplit = 0;
     for (int i = 0; i < count; ++i) max_nsplit = std::max(max_nsplit, (int)((calls[i].n / kCB + cps - 1) / cps));
-    const bool s2sum = !stage1_only && r_max <= grp.r2 && r_max <= 4 * kSumSlots * kThreads &&
+    // Streaming stage 2 (stage2s_kernel) where the layers' U does not fit on chip in one wave
+    // of the classic plan (no per-SM cap found), all of r fits its fragment buffer and the
+    // workspace holds its scratch.  (It records a timed-out wait in the workspace's status
+    // word, so it needs one.)
+    // Measured on a B200, the Llama-2-70B-shaped block: 2 tokens 53.3 -> 43.4 us, 4 tokens
+    // 62.8 -> 54.8 us per step with it; 1 token 37.1 -> 38.8 us and 8 tokens (two token groups,
+    // two 16-row tiles per warp) 106 -> 112 us, so those keep the classic kernel.
+    const bool stream2 = !stage1_only && s2s_room && ws->status != nullptr && batch >= 2 && batch <= 4;
+    grp.stream2 = stream2 ? 1 : 0;
+    const bool s2sum = !stream2 && !stage1_only && r_max <= grp.r2 && r_max <= 4 * kSumSlots * kThreads &&
                        max_nsplit <= kS2SumMaxSplits;
     grp.depth1 = cps > kChunkCB ? 2 : 1;
     size_t toff = 0, goff = 0, poff = 0, coff = 0;
@@ -1148,8 +1556,22 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
         grp.s1_start[k + 1] = grp.s1_start[k] + (L1.r / kRowsS1) * L1.nsplit;
         grp.s2_start[k + 1] = grp.s2_start[k] + L2.s2_ctas;
     }
-    if (batch <= 4) return launch_group<1>(grp, stream, ws->device, stage1_only);
-    return launch_group<2>(grp, stream, ws->device, stage1_only);
+    S2sMaps maps;
+    int* s2s_part = reinterpret_cast<int*>(ws->partials + npoff);
+    int* s2s_cnt = ws->counters + ncoff;
+    if (stream2) {
+        grp.u_start[0] = grp.st_start[0] = 0;
+        for (int i = 0; i < count; ++i) {
+            const DecLayer& L = grp.L[i];
+            const int units = (L.m + kS2sRows - 1) / kS2sRows;  // a last unit of 128 rows reads zeros past m
+            grp.u_start[i + 1] = grp.u_start[i] + units;
+            grp.st_start[i + 1] = grp.st_start[i] + units * ((L.r + 1023) / 1024);
+            if (!encode_map_u32_sw128(&maps.map[i], L.Upk, L.m, L.r / 32, kS2sBoxWords, kS2sRows)) return NQ_ERR_CUDA;
+        }
+    }
+    unsigned* status = ws->status ? ws->status + 1 : nullptr;
+    if (batch <= 4) return launch_group<1>(grp, stream, ws->device, stage1_only, &maps, status, s2s_part, s2s_cnt);
+    return launch_group<2>(grp, stream, ws->device, stage1_only, &maps, status, s2s_part, s2s_cnt);
 }
 
 int decode_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const uint16_t* s1,

@@ -37,6 +37,7 @@
 #include <cudaTypedefs.h>
 
 #include "nq_internal.cuh"
+#include "nq_sm100.cuh"
 
 namespace nq {
 namespace {
@@ -44,131 +45,10 @@ namespace {
 constexpr int kBM = 128;          // rows of A per CTA (tcgen05 M)
 constexpr int kBK = 64;           // K elements per stage: one 128-byte swizzle atom of fp16
 constexpr int kUmmaK = 16;        // K per tcgen05.mma (kind::f16)
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long global_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait: false if the CTA aborted or the limit expired (then the CTA aborts).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned* status, unsigned long long limit_ns = kWaitLimitNs) {
-    if (mbar_try(bar, parity)) return true;
-    const unsigned long long t0 = global_ns();
-    while (true) {
-        if (mbar_try(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (global_ns() - t0 > limit_ns) {
-            *abort_flag = 1;
-            atomicExch(status, (unsigned)(-NQ_ERR_TIMEOUT));
-            return false;
-        }
-    }
-}
-
-// Time-bounded wait that ignores the abort flag: used to drain what this CTA issued.
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-    const unsigned long long t0 = global_ns();
-    while (!mbar_try(bar, parity) && global_ns() - t0 < kWaitLimitNs) {
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
-        : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-// orders this thread's view of global memory (generic proxy) before its later TMA loads
-__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-
-__device__ __forceinline__ int ld_acquire(const int* p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Waits (one thread) until *count >= need; past kWaitLimitNs of GPU time it records
-// NQ_ERR_TIMEOUT in the status word and returns false.
-__device__ __forceinline__ bool wait_count(const int* count, int need, unsigned* status) {
-    const unsigned long long t0 = global_ns();
-    while (ld_acquire(count) < need) {
-        if (global_ns() - t0 > kWaitLimitNs) {
-            atomicExch(status, (unsigned)(-NQ_ERR_TIMEOUT));
-            return false;
-        }
-        __nanosleep(200);
-    }
-    return true;
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// SW128 K-major shared-memory operand descriptor: 8-row groups 1024 B apart.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3FFF);
-    d |= (uint64_t)1 << 16;            // leading byte offset 16 B (unused for swizzled K-major)
-    d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset: next 8-row group
-    d |= (uint64_t)1 << 46;            // descriptor version for tcgen05
-    d |= (uint64_t)2 << 61;            // 128-byte swizzle
-    return d;
-}
 
 // kind::f16 instruction descriptor: fp16 A and B, K-major both, fp32 D, M = 128, N = bn.
 __host__ __device__ constexpr uint32_t idesc_f16(int bn) {
     return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
-    asm volatile(
-        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
-        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 // Sixteen fp16 pairs (+-1) from one packed word: pair q = (column q, column q + 16).
@@ -321,13 +201,15 @@ struct Ring {
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// ysc: the token's 2^e_b (EPI 1), passed in by the caller (one load per lane, broadcast
+// by a shuffle, instead of a load per element).
 template <int EPI>
 __device__ __forceinline__ void store_out(const GemmArgs& a, int64_t b, int64_t grow, int64_t tcol, float s1v,
-                                          float d) {
+                                          float d, float ysc) {
     if (EPI == 0)
         a.T_out[b * a.mdim + tcol] = __half_as_ushort(__float2half_rn(d));
     else
-        a.y_out[b * a.mdim + grow] = s1v * d * __ldg(a.yscale + b);
+        a.y_out[b * a.mdim + grow] = s1v * d * ysc;
 }
 
 template <int EPI>
@@ -506,10 +388,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ Ge
                 uint32_t v[32];
                 tmem_ld32(taddr + (uint32_t)c0, v);
                 if (it.tt < 0) {
+                    const float ysc_l = (EPI == 1 && c0 + lane < it.ncols) ? __ldg(a.yscale + it.col0 + c0 + lane) : 1.f;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
+                    for (int j = 0; j < 32; ++j) {
+                        const float ysc = __shfl_sync(__activemask(), ysc_l, j);
                         if (c0 + j < it.ncols)
-                            store_out<EPI>(a, it.col0 + c0 + j, grow, tcol, s1v, __uint_as_float(v[j]));
+                            store_out<EPI>(a, it.col0 + c0 + j, grow, tcol, s1v, __uint_as_float(v[j]), ysc);
+                    }
                 } else {
                     float4* q = reinterpret_cast<float4*>(part + c0);
 #pragma unroll
@@ -549,9 +434,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap bmap, const __grid_constant__ Ge
                             }
                         }
                         const float* accf = reinterpret_cast<const float*>(acc);
+                        const float ysc_l =
+                            (EPI == 1 && c0 + (lane & 15) < it.ncols) ? __ldg(a.yscale + it.col0 + c0 + (lane & 15)) : 1.f;
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            if (c0 + j < it.ncols) store_out<EPI>(a, it.col0 + c0 + j, grow, tcol, s1v, accf[j]);
+                        for (int j = 0; j < 16; ++j) {
+                            const float ysc = __shfl_sync(__activemask(), ysc_l, j);
+                            if (c0 + j < it.ncols) store_out<EPI>(a, it.col0 + c0 + j, grow, tcol, s1v, accf[j], ysc);
+                        }
                     }
                     if (et == 0) a.counters[it.tt] = 0;  // ready for the next call
                 }
@@ -782,15 +671,18 @@ tile_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint32_t* __res
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+                const int64_t bl = n0 + c0 + lane;
+                const float ysc_l = (EPI == 1 && c0 + lane < BN && bl < batch) ? __ldg(yscale + bl) : 1.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int64_t b = n0 + c0 + j;
+                    const float ysc = __shfl_sync(__activemask(), ysc_l, j);
                     if (c0 + j < BN && b < batch) {  // BN need not be a multiple of 32
                         const float d = __uint_as_float(v[j]);
                         if (EPI == 0)
                             T_out[b * mdim + tcol] = __half_as_ushort(__float2half_rn(d));
                         else
-                            y_out[b * mdim + grow] = s1v * d * __ldg(yscale + b);
+                            y_out[b * mdim + grow] = s1v * d * ysc;
                     }
                 }
             }
@@ -829,27 +721,35 @@ __global__ void wait_selftest_kernel(unsigned long long limit_ns, unsigned* stat
     if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, status, limit_ns);
 }
 
-// x'[b][perm(j)] = fp16(2^-e_b * bf16 x[b][j] * fp16 s2[j]) and xscale[b] = 2^e_b: one CTA
-// per token row at a time.  The power of two is chosen per token from the row's sum
+// x'[b][perm(j)] = fp16(2^-e_b * bf16 x[b][j] * fp16 s2[j]) and xscale[b] = 2^e_b.  The power of two is chosen per token from the row's sum
 // L_b = sum_j |s2_j x[b][j]| (fp32) so that 2^-e_b L_b < 2^15: every |x'| and every entry
 // of T = V^T x' (each a signed sum of the x') then stays below 2^15 < 65504, so neither
 // overflows fp16, and every token uses fp16's normal range down to 2^-29 L_b whatever its
 // magnitude (without it a token of small activations falls into fp16's subnormals and a
 // token of large ones overflows T).  GEMM 2's epilogue multiplies by 2^e_b, which is exact,
 // so the result is that of the unscaled operands up to their rounding.
-constexpr int kPrescaleThreads = 128;
+constexpr int kPrescaleThreads = 256;
 
 __device__ __forceinline__ float prescale_pow2(int k) { return __int_as_float((k + 127) << 23); }  // |k| <= 126
 
+// TPR threads per token row (32 .. 256, a power of two: about one 32-column group each),
+// kPrescaleThreads / TPR rows per CTA at a time; the row's sum is reduced by a warp
+// shuffle and, across the row's warps, through shared memory in warp order.
+template <int TPR>
 __global__ void __launch_bounds__(kPrescaleThreads)
 prescale_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ s2, int64_t n, int64_t batch,
                 uint16_t* __restrict__ xp, float* __restrict__ xscale) {
+    constexpr int kRows = kPrescaleThreads / TPR, kWarpsPerRow = TPR / 32;
     __shared__ float red[kPrescaleThreads / 32];
     const int64_t groups = n / 32;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = threadIdx.x / TPR, tid = threadIdx.x % TPR, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
-    for (int64_t b = blockIdx.x; b < batch; b += gridDim.x) {
-        const uint16_t* xrow = x + b * n;
+    // every CTA runs the same number of iterations (the barrier below is CTA-wide)
+    const int64_t iters = (batch + (int64_t)gridDim.x * kRows - 1) / ((int64_t)gridDim.x * kRows);
+    for (int64_t it = 0; it < iters; ++it) {
+        const int64_t b = (it * gridDim.x + blockIdx.x) * kRows + sub;
+        const bool live = b < batch;
+        const uint16_t* xrow = x + (live ? b : 0) * n;
         // column c of a group sits in half (c & 1) of word c / 2
         auto load = [&](int64_t g, uint32_t (&xv)[16], uint32_t (&sv)[16]) {
             const uint4* xs = reinterpret_cast<const uint4*>(xrow + g * 32);
@@ -867,25 +767,29 @@ prescale_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ s2,
             return __uint_as_float((uint32_t)xb << 16) * __half2float(__ushort_as_half(sb));  // exact in fp32
         };
         float l1 = 0.f;
-        for (int64_t g = threadIdx.x; g < groups; g += kPrescaleThreads) {
-            uint32_t xv[16], sv[16];
-            load(g, xv, sv);
+        if (live)
+            for (int64_t g = tid; g < groups; g += TPR) {
+                uint32_t xv[16], sv[16];
+                load(g, xv, sv);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) l1 += fabsf(value(xv, sv, c));
-        }
+                for (int c = 0; c < 32; ++c) l1 += fabsf(value(xv, sv, c));
+            }
         for (int o = 16; o > 0; o >>= 1) l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-        if (lane == 0) red[warp] = l1;
-        __syncthreads();
-        float total = 0.f;
+        if (kWarpsPerRow > 1) {
+            if (lane == 0) red[warp] = l1;
+            __syncthreads();
+            l1 = 0.f;
 #pragma unroll
-        for (int w = 0; w < kPrescaleThreads / 32; ++w) total += red[w];
-        __syncthreads();  // red is rewritten for the next row
+            for (int w = 0; w < kWarpsPerRow; ++w) l1 += red[sub * kWarpsPerRow + w];
+            __syncthreads();  // red is rewritten in the next iteration
+        }
+        if (!live) continue;
         int e = 0;
-        frexpf(total, &e);  // total < 2^e (e = 0 for a zero row)
+        frexpf(l1, &e);  // l1 < 2^e (e = 0 for a zero row)
         e = min(max(e - 15, -110), 112);
         const float down = prescale_pow2(-e);
-        if (threadIdx.x == 0) xscale[b] = prescale_pow2(e);
-        for (int64_t g = threadIdx.x; g < groups; g += kPrescaleThreads) {
+        if (tid == 0) xscale[b] = prescale_pow2(e);
+        for (int64_t g = tid; g < groups; g += TPR) {
             uint32_t xv[16], sv[16], out[16];
             load(g, xv, sv);
             // output pair q = (column q, column q+16)
@@ -1042,10 +946,19 @@ int launch_gemm(const CUtensorMap& map, const uint32_t* Wpk, int64_t M, int64_t 
 
 cudaError_t launch_prescale(const uint16_t* x, const uint16_t* s2, int64_t n, int64_t batch, Workspace* ws,
                             cudaStream_t stream) {
-    const int64_t cap = 8 * (int64_t)sm_count();
-    const int pblocks = (int)(batch < cap ? batch : cap);
-    return launch_pdl(prescale_kernel, dim3(pblocks), dim3(kPrescaleThreads), 0, stream, x, s2, n, batch,
-                      ws->xprime, ws->xscale);
+    // threads per row: the row's 32-column groups rounded up to a power of two, 32 .. 256
+    const int64_t groups = n / 32;
+    int tpr = 32;
+    while (tpr < 256 && tpr < groups) tpr *= 2;
+    const int64_t rows_per_cta = kPrescaleThreads / tpr;
+    const int64_t want = (batch + rows_per_cta - 1) / rows_per_cta, cap = 8 * (int64_t)sm_count();
+    const dim3 grid((unsigned)(want < cap ? want : cap)), block(kPrescaleThreads);
+    switch (tpr) {
+        case 32: return launch_pdl(prescale_kernel<32>, grid, block, 0, stream, x, s2, n, batch, ws->xprime, ws->xscale);
+        case 64: return launch_pdl(prescale_kernel<64>, grid, block, 0, stream, x, s2, n, batch, ws->xprime, ws->xscale);
+        case 128: return launch_pdl(prescale_kernel<128>, grid, block, 0, stream, x, s2, n, batch, ws->xprime, ws->xscale);
+        default: return launch_pdl(prescale_kernel<256>, grid, block, 0, stream, x, s2, n, batch, ws->xprime, ws->xscale);
+    }
 }
 
 template <int BN, int EPI>
@@ -1123,6 +1036,18 @@ int run_tile_gemms(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, 
 
 }  // namespace
 
+bool encode_map_u32_sw128(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * 4)};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int selftest_wait_timeout(int64_t limit_ns, Workspace* ws, cudaStream_t stream) {
     wait_selftest_kernel<<<1, 32, 0, stream>>>((unsigned long long)limit_ns, ws->status + 1);
     return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
@@ -1147,6 +1072,31 @@ void prefill_workspace_need(int64_t m, int64_t n, int64_t r, int64_t batch, int6
     }
     *partial_floats = pf;
     *counter_ints = ci;
+}
+
+// t = V^T (s2 (.) x) in fp32 (batch x r, row-major) for more than NQ_DECODE_MAX_BATCH
+// tokens: the prescale and GEMM 1 with the y epilogue (fp32, times the token's 2^e) and unit
+// scales (`ones`, r fp16 1.0) in place of s1.
+int prefill_rank_vector(const uint16_t* x, const uint32_t* Vpk, const uint16_t* s2, int64_t n, int64_t r,
+                        int64_t batch, float* t, const uint16_t* ones, Workspace* ws, cudaStream_t stream) {
+    if (batch > kPersistentMaxBatch) {
+        if (launch_prescale(x, s2, n, batch, ws, stream) != cudaSuccess) return NQ_ERR_CUDA;
+        const int bn = choose_bn(r, batch, sm_count());
+        // bn1 = bn, nrb1 = 1: no token-tile hand-off (there is no GEMM 1 to wait for)
+        return launch_tile_gemm_bn<1>(bn, ws->xprime, n, Vpk, r, batch, nullptr, t, ones, ws, stream, bn, 1);
+    }
+    static unsigned long long init_mask = 0;
+    const unsigned long long bit = 1ull << (ws->device & 63);
+    if (!(__atomic_load_n(&init_mask, __ATOMIC_ACQUIRE) & bit)) {
+        if (cudaFuncSetAttribute(gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemMax) !=
+            cudaSuccess)
+            return NQ_ERR_CUDA;
+        __atomic_fetch_or(&init_mask, bit, __ATOMIC_RELEASE);
+    }
+    CUtensorMap map_x;
+    if (!make_map(&map_x, ws->xprime, batch, n, kBK, kBox, false, true)) return NQ_ERR_CUDA;
+    if (launch_prescale(x, s2, n, batch, ws, stream) != cudaSuccess) return NQ_ERR_CUDA;
+    return launch_gemm<1>(map_x, Vpk, r, n, batch, nullptr, t, ones, ws, stream);
 }
 
 int prefill_forward(const uint16_t* x, const uint32_t* Upk, const uint32_t* Vpk, const uint16_t* s1,

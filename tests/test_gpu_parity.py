@@ -350,10 +350,12 @@ def test_grouped_mixed_sizes(nq, orc, batch):
         assert rel_err(y.cpu().numpy(), c.oracle(orc)) <= TOL
 
 
-@pytest.mark.parametrize("batch", [1, 4])
+@pytest.mark.parametrize("batch", [1, 2, 3, 4])
 def test_grouped_llama2_70b_block(nq, orc, batch):
     """The Llama-2-70B-shaped block in one grouped call (up to 28 column splits per layer,
-    a 3840-column stage-2 span), every output checked."""
+    a 3840-column stage-2 span), every output checked.  At 2-4 tokens stage 2 streams the
+    weights through one persistent CTA per SM, and 256-row units that straddle two CTAs'
+    shares are finished by the last of them."""
     cases = [Case(orc, nq, m, n, r, batch, seed=980 + i) for i, (_, m, n, r) in enumerate(synth.LLAMA2_70B_LAYERS)]
     ys = [torch.empty((batch, c.m), dtype=torch.float32, device="cuda") for c in cases]
     nq.lowrank_linear_fwd_grouped([(c.x_d, c.Upk, c.Vpk, c.s1_d, c.s2_d, y, c.m, c.n, c.r)
