@@ -16,6 +16,9 @@ constexpr int64_t kMaxDim = int64_t(1) << 20;
 constexpr int64_t kMaxRank = 65536;
 constexpr int64_t kMaxElems = int64_t(1) << 40;  // element-wise helpers: elements per call
 constexpr int64_t kMaxRows = (int64_t(1) << 31) - 1;  // one CTA per row
+// From this many tokens the factor gradients take the prefill GEMM for t and u and the
+// tensor cores for the sums over the tokens; below, the decode stage 1 and a SIMT kernel.
+constexpr int64_t kFactorTcMinBatch = 64;
 
 std::mutex g_mutex;
 Workspace g_ws[kMaxDevices];
@@ -231,6 +234,18 @@ static int ensure_env_scratch(Workspace* w, size_t bytes) {
         if (cudaMalloc(&p, bytes) != cudaSuccess) { cudaGetLastError(); return NQ_ERR_NOMEM; }
         w->env = static_cast<float*>(p);
         w->env_bytes = bytes;
+        ++g_ws_generation;
+    }
+    return NQ_OK;
+}
+
+// Scratch of the tensor-core factor gradients (the transposed, split operands).
+static int ensure_dense_scratch(Workspace* w, size_t bytes) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (bytes > w->dense_bytes) {
+        if (w->dense) { cudaDeviceSynchronize(); cudaFree(w->dense); w->dense = nullptr; w->dense_bytes = 0; }
+        if (cudaMalloc(&w->dense, bytes) != cudaSuccess) { cudaGetLastError(); w->dense = nullptr; return NQ_ERR_NOMEM; }
+        w->dense_bytes = bytes;
         ++g_ws_generation;
     }
     return NQ_OK;
@@ -724,7 +739,35 @@ int nq_lowrank_linear_bwd_factors(const void* x, const void* dy, const uint32_t*
         return NQ_OK;
     }
     int st = NQ_OK;
-    const int64_t w = m > n ? m : n, bc = batch < NQ_DECODE_MAX_BATCH ? batch : NQ_DECODE_MAX_BATCH;
+    const int64_t w = m > n ? m : n;
+    const uint16_t* xb = static_cast<const uint16_t*>(x);
+    const uint16_t* dyb = static_cast<const uint16_t*>(dy);
+    const uint16_t* s1b = static_cast<const uint16_t*>(s1);
+    const uint16_t* s2b = static_cast<const uint16_t*>(s2);
+    if (batch >= kFactorTcMinBatch) {
+        // calibration-sized batches: t and u from the prefill GEMM, the sums over the tokens on
+        // the tensor cores (nq_dense.cu)
+        const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 128, w, r};
+        Workspace* ws = workspace_for(128, w, r, batch, decode_need(&c, 1, batch), &st);
+        if (!ws) return st;
+        if ((st = ensure_grad_scratch(ws, (size_t)r, sizeof(float) * 2 * (size_t)batch * (size_t)r, s)) != NQ_OK ||
+            (st = ensure_dense_scratch(ws, (size_t)outer_tc_scratch_bytes(batch, w, r))) != NQ_OK)
+            return st;
+        float* t = ws->gstage;                       // batch x r: V^T (s2 (.) x)
+        float* u = ws->gstage + (size_t)batch * r;   // batch x r: U^T (s1 (.) dy)
+        if (dU) {
+            st = prefill_rank_vector(xb, Vpk, s2b, n, r, batch, t, ws->ones, ws, s);
+            if (st == NQ_OK) st = outer_tc(dyb, s1b, t, batch, m, r, dU, ws->dense, ws->status + 1, s);
+            if (st != NQ_OK) return st;
+        }
+        if (dV) {
+            st = prefill_rank_vector(dyb, UpkT, s1b, m, r, batch, u, ws->ones, ws, s);
+            if (st == NQ_OK) st = outer_tc(xb, s2b, u, batch, n, r, dV, ws->dense, ws->status + 1, s);
+            if (st != NQ_OK) return st;
+        }
+        return NQ_OK;
+    }
+    const int64_t bc = batch < NQ_DECODE_MAX_BATCH ? batch : NQ_DECODE_MAX_BATCH;
     const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 128, w, r};
     Workspace* ws = workspace_for(128, w, r, bc, decode_need(&c, 1, bc), &st);
     if (!ws) return st;
@@ -732,10 +775,6 @@ int nq_lowrank_linear_bwd_factors(const void* x, const void* dy, const uint32_t*
     if (st != NQ_OK) return st;
     float* t = ws->gstage;                       // batch x r: V^T (s2 (.) x)
     float* u = ws->gstage + (size_t)batch * r;   // batch x r: U^T (s1 (.) dy)
-    const uint16_t* xb = static_cast<const uint16_t*>(x);
-    const uint16_t* dyb = static_cast<const uint16_t*>(dy);
-    const uint16_t* s1b = static_cast<const uint16_t*>(s1);
-    const uint16_t* s2b = static_cast<const uint16_t*>(s2);
     if (dU) {
         st = decode_rank_vector(xb, Vpk, s2b, n, r, batch, t, ws, s);
         if (st == NQ_OK) st = outer_device(dyb, s1b, t, batch, m, r, dU, s);

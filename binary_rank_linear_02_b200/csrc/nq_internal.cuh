@@ -37,6 +37,8 @@ struct Workspace {
     size_t ones_count = 0, gstage_bytes = 0;
     float* env = nullptr;          // envelope terms 1 .. l-1: (l-1) x batch x m fp32
     size_t env_bytes = 0;
+    void* dense = nullptr;         // factor gradients on the tensor cores: transposed operands
+    size_t dense_bytes = 0;
     size_t t_cap = 0, tgmax_cap = 0, partial_cap = 0, counter_cap = 0;
     int64_t r_cap = 0, n_cap = 0, m_cap = 0, batch_cap = 0, rsum_cap = 0;
 };
@@ -96,6 +98,15 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
 // NQ_DECODE_MAX_BATCH tokens per launch, each launch's t copied out of the workspace).
 int decode_rank_vector(const uint16_t* x, const uint32_t* Vpk, const uint16_t* s2, int64_t n, int64_t r,
                        int64_t batch, float* t, Workspace* ws, cudaStream_t stream);
+// t = V^T (s2 (.) x) (batch x r fp32) by the prefill kernels, for batch > NQ_DECODE_MAX_BATCH;
+// ones: at least r fp16 1.0
+int prefill_rank_vector(const uint16_t* x, const uint32_t* Vpk, const uint16_t* s2, int64_t n, int64_t r,
+                        int64_t batch, float* t, const uint16_t* ones, Workspace* ws, cudaStream_t stream);
+// out[i][k] = s[i] * sum_b bf16(a[b][i]) * t[b][k] (M x R fp32) on the tensor cores (M, R
+// multiples of 128), t split into two bf16 halves; scratch of outer_tc_scratch_bytes.
+int64_t outer_tc_scratch_bytes(int64_t batch, int64_t M, int64_t R);
+int outer_tc(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch, int64_t M, int64_t R, float* out,
+             void* scratch, unsigned* status, cudaStream_t stream);
 // out[i][k] = s[i] * sum over b (increasing) of bf16(a[b][i]) * t[b][k]: M x R fp32
 int outer_device(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch, int64_t M, int64_t R,
                  float* out, cudaStream_t stream);

@@ -194,6 +194,11 @@ def test_bwd_scales_deterministic_and_skippable(nq, orc):
     (640, 384, 256, 13),      # two launches of the first stage (8 + 5 tokens)
     (1152, 384, 1664, 8),
     (4096, 11008, 2432, 2),   # the 7B down projection's shape
+    # calibration-sized batches: t and u from the prefill GEMM, the sums on the tensor cores
+    (512, 512, 128, 64),      # the first batch of that route (persistent split-K GEMM for t, u)
+    (384, 640, 256, 100),     # tokens padded to 128 in the transposed operands
+    (1152, 384, 1664, 257),   # one-tile-per-CTA GEMM for t, u; padded to 320
+    (11008, 4096, 2432, 128), # the 7B gate projection's shape
 ])
 def test_bwd_factors_match_oracle(nq, orc, m, n, r, batch):
     """dU and dV against the oracle, within the bound that the accuracy of t and u gives:
