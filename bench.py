@@ -435,6 +435,7 @@ def run_ours(args):
         secondary["chain_llama2-7b_32_blocks_b1"] = run_chain(device, stream, args.warmup, peaks)
         secondary["envelope_llama2-7b_q_l2_b1"] = run_envelope(device, stream, peaks)
         secondary["admm_init_llama2-7b_q"] = run_admm(device, stream, peaks)
+        secondary["backward_11008x4096_r2432"] = run_backward_calibration(device, stream, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -590,6 +591,54 @@ def run_chain(device, stream, warmup, peaks, passes=20, batch=1, nblocks=synth.C
            "kernels_per_pass": nblocks * chain.DecodeChain.launches_per_step_per_block,
            "roofline_tokens_per_s": round(batch * peaks["hbm_gbs"] * 1e9 / pb, 1)}
     del g, ch, blocks
+    return out
+
+
+def run_backward_calibration(device, stream, peaks, batches=(1024, 4096), reps=5):
+    """The refinement step's gradients of one layer (the 11008x4096 r=2432 gate shape) at
+    calibration batch sizes: nq_lowrank_linear_bwd_factors (rank vectors by the prefill
+    GEMMs, sums over the tokens on the tensor cores) and nq_lowrank_linear_bwd_scales.
+    Algorithmic flops: factors 4 b r (m + n) (t, u and the two outer products), scales
+    4 b r (m + n) (two factorised evaluations) plus 2 b (m + n)."""
+    import torch
+
+    from binary_rank_linear_02_b200 import nq
+
+    _, m, n, r = synth.PREFILL_SHAPE
+    gen = torch.Generator(device=device)
+    gen.manual_seed(777)
+    Upk = torch.randint(-(1 << 31), 1 << 31, (m, r // 32), dtype=torch.int64, device=device, generator=gen).to(torch.int32)
+    Vpk = torch.randint(-(1 << 31), 1 << 31, (r, n // 32), dtype=torch.int64, device=device, generator=gen).to(torch.int32)
+    UpkT = nq.transpose_signs(Upk, m, r)
+    VpkT = nq.transpose_signs(Vpk, r, n)
+    s1 = torch.from_numpy(synth.scales_f16(m, 777, "s1").view(np.int16)).to(device)
+    s2 = torch.from_numpy(synth.scales_f16(n, 777, "s2").view(np.int16)).to(device)
+    out = {}
+    for b in batches:
+        x = torch.from_numpy(synth.activations_bf16(b, n, 777, b).view(np.int16)).to(device)
+        dy = torch.from_numpy(synth.activations_bf16(b, m, 778, b).view(np.int16)).to(device)
+        for name, fn in (("factors", lambda: nq.lowrank_linear_bwd_factors(x, dy, Vpk, UpkT, s1, s2, m, n, r,
+                                                                           stream=stream.cuda_stream)),
+                         ("scales", lambda: nq.lowrank_linear_bwd_scales(x, dy, Upk, Vpk, UpkT, VpkT, s1, s2, m, n, r,
+                                                                         stream=stream.cuda_stream))):
+            with torch.cuda.stream(stream):
+                fn()
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(reps):
+                start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    start.record(stream)
+                    fn()
+                    end.record(stream)
+                torch.cuda.synchronize()
+                times.append(start.elapsed_time(end))
+            ms = statistics.median(times)
+            fl = 4.0 * b * r * (m + n) + (2.0 * b * (m + n) if name == "scales" else 0.0)
+            tf = fl / (ms * 1e-3) / 1e12
+            out[f"{name}_b{b}"] = {"us_per_call": round(ms * 1e3, 1), "tflops": round(tf, 1),
+                                   "frac_of_bf16_burst": round(tf / peaks["bf16_tflops"], 4)}
+        del x, dy
     return out
 
 
