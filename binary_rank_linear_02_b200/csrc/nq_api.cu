@@ -700,18 +700,22 @@ int nq_lowrank_linear_bwd_scales(const void* x, const void* dy, const uint32_t* 
     const DecodeCall c{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, m > n ? m : n, m > n ? m : n, r};
     Workspace* ws = workspace_for(m > n ? m : n, m > n ? m : n, r, batch, decode_need(&c, 1, batch), &st);
     if (!ws) return st;
-    st = ensure_grad_scratch(ws, (size_t)(m > n ? m : n), sizeof(float) * (size_t)batch * (size_t)(m > n ? m : n), s);
+    const int64_t wmax = m > n ? m : n;
+    st = ensure_grad_scratch(ws, (size_t)wmax,
+                             sizeof(float) * ((size_t)batch * (size_t)wmax + (size_t)col_dot_scratch_floats(batch, wmax)),
+                             s);
     if (st != NQ_OK) return st;
+    float* dot_scratch = ws->gstage + (size_t)batch * (size_t)wmax;
     if (ds1) {  // z = U (V^T (s2 (.) x)): the forward with s1 = 1; ds1 = sum_b dy (.) z
         st = nq_lowrank_linear_fwd(x, Upk, Vpk, ws->ones, s2, m, n, r, batch, ws->gstage, stream);
         if (st != NQ_OK) return st;
-        st = col_dot_device(static_cast<const uint16_t*>(dy), ws->gstage, batch, m, ds1, s);
+        st = col_dot_device(static_cast<const uint16_t*>(dy), ws->gstage, batch, m, ds1, dot_scratch, s);
         if (st != NQ_OK) return st;
     }
     if (ds2) {  // w = V (U^T (s1 (.) dy)): the input gradient with s2 = 1; ds2 = sum_b x (.) w
         st = nq_lowrank_linear_fwd(dy, VpkT, UpkT, ws->ones, s1, n, m, r, batch, ws->gstage, stream);
         if (st != NQ_OK) return st;
-        st = col_dot_device(static_cast<const uint16_t*>(x), ws->gstage, batch, n, ds2, s);
+        st = col_dot_device(static_cast<const uint16_t*>(x), ws->gstage, batch, n, ds2, dot_scratch, s);
         if (st != NQ_OK) return st;
     }
     return NQ_OK;

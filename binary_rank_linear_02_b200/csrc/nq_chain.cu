@@ -115,16 +115,33 @@ __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ Gat
 
 // Scale gradients: out[i] = sum_b bf16(a[b][i]) * z[b][i], one thread per i, the tokens in
 // increasing order (deterministic).  z comes from the kernel before (programmatic wait).
+// out[i] = sum_b bf16(a[b][i]) * z[b][i]: the tokens in chunks of kDotChunk, chunk c's sum
+// (tokens in order) into part[c][i] by CTA row c, or straight into out when there is one
+// chunk; then col_sum_kernel adds the chunks' sums in chunk order (a fixed order).
+constexpr int64_t kDotChunk = 64;
+
 __global__ void __launch_bounds__(256) col_dot_kernel(const uint16_t* __restrict__ a, const float* __restrict__ z,
-                                                      int64_t batch, int64_t len, float* __restrict__ out) {
+                                                      int64_t batch, int64_t len, float* __restrict__ part) {
     pdl_wait();
     pdl_trigger();
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < len; i += (int64_t)gridDim.x * blockDim.x) {
-        float acc = 0.f;
-        for (int64_t b = 0; b < batch; ++b)
-            acc = fmaf(__uint_as_float((uint32_t)a[b * len + i] << 16), z[b * len + i], acc);
-        out[i] = acc;
-    }
+    const int64_t b0 = (int64_t)blockIdx.y * kDotChunk;
+    const int64_t b1 = b0 + kDotChunk < batch ? b0 + kDotChunk : batch;
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= len) return;
+    float acc = 0.f;
+    for (int64_t b = b0; b < b1; ++b) acc = fmaf(__uint_as_float((uint32_t)a[b * len + i] << 16), z[b * len + i], acc);
+    part[(int64_t)blockIdx.y * len + i] = acc;
+}
+
+__global__ void __launch_bounds__(256) col_sum_kernel(const float* __restrict__ part, int64_t chunks, int64_t len,
+                                                      float* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= len) return;
+    float acc = 0.f;
+    for (int64_t c = 0; c < chunks; ++c) acc += __ldcg(part + c * len + i);
+    out[i] = acc;
 }
 
 __global__ void fill_u16_kernel(uint16_t* p, int64_t count, uint16_t value) {
@@ -237,11 +254,23 @@ int rms_normalize_bf16_device(const float* src, int64_t rows, int64_t cols, uint
                : NQ_ERR_CUDA;
 }
 
-int col_dot_device(const uint16_t* a, const float* z, int64_t batch, int64_t len, float* out, cudaStream_t stream) {
-    int64_t blocks = (len + 255) / 256;
-    if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
-    return launch_pdl(col_dot_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, a, z, batch, len, out) ==
-                   cudaSuccess
+int64_t col_dot_scratch_floats(int64_t batch, int64_t len) {
+    const int64_t chunks = (batch + kDotChunk - 1) / kDotChunk;
+    return chunks > 1 ? chunks * len : 0;
+}
+
+int col_dot_device(const uint16_t* a, const float* z, int64_t batch, int64_t len, float* out, float* scratch,
+                   cudaStream_t stream) {
+    const int64_t chunks = (batch + kDotChunk - 1) / kDotChunk;
+    const dim3 grid((unsigned)((len + 255) / 256), (unsigned)chunks);
+    if (chunks == 1)
+        return launch_pdl(col_dot_kernel, grid, dim3(256), 0, stream, a, z, batch, len, out) == cudaSuccess
+                   ? NQ_OK
+                   : NQ_ERR_CUDA;
+    if (launch_pdl(col_dot_kernel, grid, dim3(256), 0, stream, a, z, batch, len, scratch) != cudaSuccess)
+        return NQ_ERR_CUDA;
+    return launch_pdl(col_sum_kernel, dim3((unsigned)((len + 255) / 256)), dim3(256), 0, stream,
+                      (const float*)scratch, chunks, len, out) == cudaSuccess
                ? NQ_OK
                : NQ_ERR_CUDA;
 }

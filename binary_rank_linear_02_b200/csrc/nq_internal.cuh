@@ -130,8 +130,11 @@ int pack_device(const int8_t* signs, int64_t rows, int64_t cols, uint32_t* out, 
                 cudaStream_t stream);
 int unpack_device(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* out, cudaStream_t stream);
 int transpose_device(const uint32_t* packed, int64_t rows, int64_t cols, uint32_t* out, cudaStream_t stream);
-// out[i] = sum over b (increasing) of bf16(a[b][i]) * z[b][i], for i < len
-int col_dot_device(const uint16_t* a, const float* z, int64_t batch, int64_t len, float* out, cudaStream_t stream);
+// out[i] = sum_b bf16(a[b][i]) * z[b][i], for i < len: chunks of 64 tokens summed in token
+// order, then the chunks in order (deterministic); scratch of col_dot_scratch_floats floats
+int64_t col_dot_scratch_floats(int64_t batch, int64_t len);
+int col_dot_device(const uint16_t* a, const float* z, int64_t batch, int64_t len, float* out, float* scratch,
+                   cudaStream_t stream);
 int fill_u16_device(uint16_t* p, int64_t count, uint16_t value, cudaStream_t stream);
 constexpr int kMaxGather = 16;
 struct GatherSeg {

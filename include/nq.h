@@ -171,7 +171,9 @@ int nq_lowrank_linear_bwd_input(const void* dy, const uint32_t* UpkT, const uint
  * shapes as nq_lowrank_linear_fwd; batch 0 writes zeros.  Each gradient is the layer
  * evaluated without one scale (the forward pass, or the input gradient, with that scale
  * set to 1, through the decode or prefill kernels) followed by a per-column dot product
- * over the tokens in token order (deterministic).  Accuracy: each term carries the error
+ * over the tokens: 64-token chunks each summed in token order, then the chunks' sums in
+ * chunk order (a fixed order, so repeated calls agree bit for bit).  Accuracy: each term
+ * carries the error
  * of that evaluation, |error of ds1_i| <= 2e-3 * sum_b |dy[b][i]| * max_i' |z[b][i']|.
  * Uses the workspace (not safe for concurrent calls on different streams); asynchronous
  * on `stream`, except that the first call of a size allocates scratch.
@@ -192,10 +194,14 @@ int nq_lowrank_linear_bwd_scales(const void* x, const void* dy, const uint32_t* 
  *   s1 : m fp16;  s2 : n fp16
  *   dU : m x r float32, dV : n x r float32, row-major (written; either may be NULL)
  * Every pointer in device memory, 16-byte aligned; shapes as nq_lowrank_linear_fwd; batch 0
- * writes zeros.  t and u come from the decode path's first stage (up to 8 tokens per launch,
- * so cost grows with batch in steps of 8 tokens), the sums over the tokens from a tiled
- * fp32 kernel in token order (deterministic).  Accuracy: |error of dU[i][k]| <=
- * 2e-3 * |s1_i| * sum_b |dy[b][i]| * max_k' |t[b][k']| (likewise dV).  Uses the workspace.
+ * writes zeros.  Below 64 tokens, t and u come from the decode path's first stage (up to 8
+ * tokens per launch) and the sums over the tokens from a tiled fp32 kernel in token order.
+ * From 64 tokens, t and u come from the prefill path's first GEMM and the sums from a
+ * tensor-core GEMM: dy (or x) in bf16 against t split into two bf16 parts (t = hi + lo,
+ * the pair exact to 2^-16 relative), accumulated in fp32 on the tensor cores; the order is
+ * fixed by the tile shapes, so repeated calls agree bit for bit.  Accuracy, both routes:
+ * |error of dU[i][k]| <= 2e-3 * |s1_i| * sum_b |dy[b][i]| * max_k' |t[b][k']| (likewise
+ * dV).  Uses the workspace.
  */
 int nq_lowrank_linear_bwd_factors(const void* x, const void* dy, const uint32_t* Vpk, const uint32_t* UpkT,
                                   const void* s1, const void* s2, int64_t m, int64_t n, int64_t r, int64_t batch,

@@ -140,6 +140,7 @@ ONE_F16 = 0x3C00
     (384, 640, 256, 5),       # decode path, two token groups
     (1152, 384, 1664, 8),
     (640, 384, 256, 40),      # prefill path
+    (640, 384, 256, 130),     # token sums in three 64-token chunks, the last ragged
     (11008, 4096, 2432, 3),   # the 7B gate projection's shape
 ])
 def test_bwd_scales_match_oracle(nq, orc, m, n, r, batch):
@@ -166,8 +167,9 @@ def test_bwd_scales_match_oracle(nq, orc, m, n, r, batch):
     assert np.all(np.abs(ds2.cpu().numpy() - ref2) <= bound2)
 
 
-def test_bwd_scales_deterministic_and_skippable(nq, orc):
-    m, n, r, batch = 512, 768, 256, 4
+@pytest.mark.parametrize("batch", [4, 200])  # one token chunk; four chunks through the prefill GEMMs
+def test_bwd_scales_deterministic_and_skippable(nq, orc, batch):
+    m, n, r = 512, 768, 256
     layer = Layer(orc, nq, m, n, r, seed=520)
     x_d = torch.from_numpy(synth.activations_bf16(batch, n, 521).view(np.int16)).cuda()
     dy_d = torch.from_numpy(synth.activations_bf16(batch, m, 522, "dy").view(np.int16)).cuda()
@@ -221,3 +223,22 @@ def test_bwd_factors_match_oracle(nq, orc, m, n, r, batch):
     bV = TOL * s2f * np.sum(xf * np.max(np.abs(u), axis=1)[:, None], axis=0) + 1e-12
     assert np.all(np.abs(dU.cpu().numpy() - rU) <= bU[:, None])
     assert np.all(np.abs(dV.cpu().numpy() - rV) <= bV[:, None])
+
+
+@pytest.mark.parametrize("batch", [5, 100])  # fp32 token sums; tensor-core token sums
+def test_bwd_factors_deterministic_and_skippable(nq, orc, batch):
+    m, n, r = 384, 640, 256
+    layer = Layer(orc, nq, m, n, r, seed=530)
+    x_d = torch.from_numpy(synth.activations_bf16(batch, n, 531).view(np.int16)).cuda()
+    dy_d = torch.from_numpy(synth.activations_bf16(batch, m, 532, "dy").view(np.int16)).cuda()
+    a1, a2 = nq.lowrank_linear_bwd_factors(x_d, dy_d, layer.Vpk, layer.UpkT, layer.s1_d, layer.s2_d, m, n, r)
+    b1, b2 = nq.lowrank_linear_bwd_factors(x_d, dy_d, layer.Vpk, layer.UpkT, layer.s1_d, layer.s2_d, m, n, r)
+    torch.cuda.synchronize()
+    assert torch.equal(a1, b1) and torch.equal(a2, b2)
+    # dV alone (dU NULL) gives the same dV
+    only = torch.empty((n, r), dtype=torch.float32, device="cuda")
+    st = nq.nq_lowrank_linear_bwd_factors(x_d.data_ptr(), dy_d.data_ptr(), layer.Vpk.data_ptr(),
+                                          layer.UpkT.data_ptr(), layer.s1_d.data_ptr(), layer.s2_d.data_ptr(),
+                                          m, n, r, batch, 0, only.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert st == nq.NQ_OK and torch.equal(only, a2)
