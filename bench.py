@@ -11,7 +11,7 @@ streams its signs from HBM.  The K-step region is timed `--repeats` times (CUDA 
 synchronised on both sides) and the median is reported.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode70b|decode7b|prefill|chain7b]
+                    [--workload decode70b|decode7b|prefill|chain7b|admm|backward]
     torchrun --nproc-per-node N bench.py --gpus N ...   (independent replicas, one per GPU)
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead
@@ -366,6 +366,8 @@ def run_ours(args):
         return run_chain_only(args, device, peaks)
     if args.workload == "admm":
         return run_admm_only(args, device, peaks)
+    if args.workload == "backward":
+        return run_backward_only(args, device, peaks)
     model, layers = DECODE_WORKLOADS[args.workload]
     batch = args.batch
     work = DecodeWorkload(layers, batch, seed=1234 + rank, device=device)
@@ -791,6 +793,33 @@ def run_admm_only(args, device, peaks):
     print(json.dumps(line), flush=True)
 
 
+def run_backward_only(args, device, peaks):
+    """--workload backward: the refinement step's factor and scale gradients of the
+    11008x4096 r=2432 layer alone (--backward-batch tokens, else 1024 and 4096), one JSON line,
+    TFLOP/s of the factor gradients at the largest batch."""
+    import torch
+
+    stream = torch.cuda.Stream(device)
+    batches = (args.backward_batch,) if args.backward_batch else (1024, 4096)
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    b = run_backward_calibration(device, stream, peaks, batches=batches, reps=max(3, args.repeats))
+    clocks = sampler.stop()
+    top = max(batches)
+    f = b[f"factors_b{top}"]
+    line = {"metric": METRIC, "value": f["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": 1, "warmup": 1,
+            "ms_per_step": round(f["us_per_call"] / 1e3, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 operands (t, u split into two bf16 parts), fp32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": f"factor and scale gradients, 11008x4096 r=2432 layer, {top} tokens"},
+            "roofline": {"bound": "tensor", "achieved": f["tflops"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": f["frac_of_bf16_burst"], "traffic": None,
+                         "kernel": "nq_lowrank_linear_bwd_factors (4 b r (m + n) flops per call)",
+                         "peak_source": peaks["source"] + " (burst)"},
+            "cpu_baseline": None, "clocks": clocks, "backward": b}
+    print(json.dumps(line), flush=True)
+
+
 def run_prefill_only(args, device, peaks):
     """--workload prefill: the config-4 sweep alone (or one batch), one JSON line, TFLOP/s."""
     import torch
@@ -972,6 +1001,36 @@ def run_cpu_baseline_admm(shape=(4096, 4096, 1664), iters=2):
             "sample": f"{iters} ADMM iteration(s) of the {m}x{n} r={r} problem on the numpy fp64 oracle"}
 
 
+def run_cpu_baseline_backward(budget_s=10.0):
+    """The oracle's factor gradients of the 11008x4096 r=2432 layer on the host cores (fp64 C),
+    for growing token samples until the time budget; TFLOP/s over the same 4 b r (m + n)
+    algorithmic flops as the GPU arm."""
+    import oracle as orc
+
+    _, m, n, r = synth.PREFILL_SHAPE
+    U = synth.signs(m, r, 777, "U")
+    V = synth.signs(n, r, 777, "V")
+    Upk, Vpk = orc.pack_signs(U), orc.pack_signs(np.ascontiguousarray(V.T))  # V^T: r x n/32 words
+    s1 = synth.scales_f16(m, 777, "s1")
+    s2 = synth.scales_f16(n, 777, "s2")
+    b, spent, calls, toks = 1, 0.0, 0, 0
+    while spent < budget_s and b <= 64:
+        x = synth.activations_bf16(b, n, 777, b)
+        dy = synth.activations_bf16(b, m, 778, b)
+        t0 = time.perf_counter()
+        orc.lowrank_linear_bwd_factors(x, dy, Upk, Vpk, s1, s2, m, n, r)
+        spent += time.perf_counter() - t0
+        calls += 1
+        toks += b
+        b *= 2
+    import os as _os
+
+    return {"value": round(4.0 * toks * r * (m + n) / spent / 1e12, 6), "unit": "TFLOP/s", "cores": _os.cpu_count(),
+            "kind": "oracle", "seconds": round(spent, 2),
+            "sample": f"{calls} call(s), {toks} tokens in all, of the factor gradients of the {m}x{n} r={r} layer "
+                      f"on the fp64 C oracle ({spent:.1f} s)"}
+
+
 def prefill_config(batches):
     _, m, n, r = synth.PREFILL_SHAPE
     return {"workload": f"prefill {m}x{n} r={r}, token batch {max(batches)} "
@@ -998,6 +1057,13 @@ def run_reference(args):
     elif args.workload == "chain7b":
         cpu = run_cpu_baseline_chain(budget_s=args.cpu_seconds)
         config = chain_config(args.batch)
+    elif args.workload == "admm":
+        cpu = run_cpu_baseline_admm()
+        config = {"workload": f"LB-ADMM initialiser, 4096x4096 r=1664, {args.admm_iters} iterations per call"}
+    elif args.workload == "backward":
+        cpu = run_cpu_baseline_backward(budget_s=args.cpu_seconds)
+        top = args.backward_batch if args.backward_batch else 4096
+        config = {"workload": f"factor and scale gradients, 11008x4096 r=2432 layer, {top} tokens"}
     else:
         model, layers = DECODE_WORKLOADS[args.workload]
         cpu = run_cpu_baseline(layers, args.batch, budget_s=args.cpu_seconds)
@@ -1022,7 +1088,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", dest="secondary", action="store_false")
-    ap.add_argument("--workload", choices=["decode70b", "decode7b", "prefill", "chain7b", "admm"], default="decode70b")
+    ap.add_argument("--workload", choices=["decode70b", "decode7b", "prefill", "chain7b", "admm", "backward"],
+                    default="decode70b")
+    ap.add_argument("--backward-batch", type=int, default=0,
+                    help="--workload backward: one token batch instead of 1024 and 4096")
     ap.add_argument("--admm-iters", type=int, default=40)
     ap.add_argument("--repeats", type=int, default=5)
     ap.add_argument("--prefill-batch", type=int, default=0)
