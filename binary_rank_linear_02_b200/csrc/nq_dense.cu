@@ -57,7 +57,9 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constan
     DenseBarriers& bar = *reinterpret_cast<DenseBarriers*>(gbase + kDStages * kDStageBytes);
     volatile int* abort_flag = &bar.abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * kDM, n0 = blockIdx.y * kDN;
+    // column tiles fastest: the CTAs resident at once share a few row panels of A, and all of
+    // B (R x 2Bp bf16, 40 MB at r = 2432 and 4096 tokens) stays in L2 while A streams once
+    const int n0 = blockIdx.x * kDN, m0 = blockIdx.y * kDM;
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < kDStages; ++st) {
@@ -158,43 +160,60 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constan
 }
 
 // dst[c][b] = src[b][c] (bf16) for b < B, 0 for B <= b < Bp: the K-major A operand from
-// token-major activations.  32 x 32 tiles through shared memory.
+// token-major activations.  64 x 64 tiles through shared memory (row pitch 65 halves: the
+// column reads of the write-out fall in distinct banks), each thread moving two adjacent
+// elements per access so that a warp reads and writes 128 contiguous bytes.
+constexpr int kTT = 64;
 __global__ void __launch_bounds__(256) transpose_pad_kernel(const uint16_t* __restrict__ src, int64_t B, int64_t C,
                                                             int64_t Bp, uint16_t* __restrict__ dst) {
-    __shared__ uint16_t tile[32][33];
-    const int64_t c0 = (int64_t)blockIdx.x * 32, b0 = (int64_t)blockIdx.y * 32;
+    __shared__ uint16_t tile[kTT][kTT + 1];
+    const int64_t c0 = (int64_t)blockIdx.x * kTT, b0 = (int64_t)blockIdx.y * kTT;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
-    for (int k = ty; k < 32; k += 8) {
-        const int64_t b = b0 + k, c = c0 + tx;
-        tile[k][tx] = (b < B && c < C) ? src[b * C + c] : (uint16_t)0;
+    for (int k = ty; k < kTT; k += 8) {
+        const int64_t b = b0 + k, c = c0 + 2 * tx;
+        uint32_t v = 0;
+        if (b < B && c < C) v = *reinterpret_cast<const uint32_t*>(src + b * C + c);
+        tile[k][2 * tx] = (uint16_t)(v & 0xFFFFu);
+        tile[k][2 * tx + 1] = (uint16_t)(v >> 16);
     }
     __syncthreads();
-    for (int k = ty; k < 32; k += 8) {
-        const int64_t c = c0 + k, b = b0 + tx;
-        if (c < C && b < Bp) dst[c * Bp + b] = tile[tx][k];
+    for (int k = ty; k < kTT; k += 8) {
+        const int64_t c = c0 + k, b = b0 + 2 * tx;
+        if (c < C && b < Bp)
+            *reinterpret_cast<uint32_t*>(dst + c * Bp + b) = (uint32_t)tile[2 * tx][k] | ((uint32_t)tile[2 * tx + 1][k] << 16);
     }
 }
 
 // dst[c][b] = bf16(v), dst[c][Bp + b] = bf16(v - bf16(v)) with v = src[b][c] (fp32), zeros for
-// B <= b < Bp: the K-major B operand, each fp32 value as the sum of two bf16 numbers.
+// B <= b < Bp: the K-major B operand, each fp32 value as the sum of two bf16 numbers.  64 x 64
+// tiles as above (row pitch 65 floats).
 __global__ void __launch_bounds__(256) transpose_split_kernel(const float* __restrict__ src, int64_t B, int64_t C,
                                                               int64_t Bp, uint16_t* __restrict__ dst) {
-    __shared__ float tile[32][33];
-    const int64_t c0 = (int64_t)blockIdx.x * 32, b0 = (int64_t)blockIdx.y * 32;
+    __shared__ float tile[kTT][kTT + 1];
+    const int64_t c0 = (int64_t)blockIdx.x * kTT, b0 = (int64_t)blockIdx.y * kTT;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-    for (int k = ty; k < 32; k += 8) {
-        const int64_t b = b0 + k, c = c0 + tx;
-        tile[k][tx] = (b < B && c < C) ? src[b * C + c] : 0.f;
+    for (int k = ty; k < kTT; k += 8) {
+        const int64_t b = b0 + k, c = c0 + 2 * tx;
+        float2 v = make_float2(0.f, 0.f);
+        if (b < B && c < C) v = *reinterpret_cast<const float2*>(src + b * C + c);
+        tile[k][2 * tx] = v.x;
+        tile[k][2 * tx + 1] = v.y;
     }
     __syncthreads();
-    for (int k = ty; k < 32; k += 8) {
-        const int64_t c = c0 + k, b = b0 + tx;
+    for (int k = ty; k < kTT; k += 8) {
+        const int64_t c = c0 + k, b = b0 + 2 * tx;
         if (c < C && b < Bp) {
-            const float v = tile[tx][k];
-            const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-            dst[c * 2 * Bp + b] = __bfloat16_as_ushort(hi);
-            dst[c * 2 * Bp + Bp + b] = __bfloat16_as_ushort(lo);
+            uint32_t hi2 = 0, lo2 = 0;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float v = tile[2 * tx + e][k];
+                const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+                hi2 |= (uint32_t)__bfloat16_as_ushort(hi) << (16 * e);
+                lo2 |= (uint32_t)__bfloat16_as_ushort(lo) << (16 * e);
+            }
+            *reinterpret_cast<uint32_t*>(dst + c * 2 * Bp + b) = hi2;
+            *reinterpret_cast<uint32_t*>(dst + c * 2 * Bp + Bp + b) = lo2;
         }
     }
 }
@@ -227,13 +246,15 @@ int outer_tc(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch
             return NQ_ERR_CUDA;
         __atomic_fetch_or(&init_mask, bit, __ATOMIC_RELEASE);
     }
-    transpose_pad_kernel<<<dim3((unsigned)((M + 31) / 32), (unsigned)(Bp / 32)), 256, 0, stream>>>(a, batch, M, Bp, At);
-    transpose_split_kernel<<<dim3((unsigned)((R + 31) / 32), (unsigned)(Bp / 32)), 256, 0, stream>>>(t, batch, R, Bp, Bt);
+    transpose_pad_kernel<<<dim3((unsigned)((M + kTT - 1) / kTT), (unsigned)(Bp / kTT)), 256, 0, stream>>>(a, batch, M,
+                                                                                                       Bp, At);
+    transpose_split_kernel<<<dim3((unsigned)((R + kTT - 1) / kTT), (unsigned)(Bp / kTT)), 256, 0, stream>>>(t, batch, R,
+                                                                                                         Bp, Bt);
     if (cudaGetLastError() != cudaSuccess) return NQ_ERR_CUDA;
     CUtensorMap amap, bmap;
     if (!make_map_bf16(&amap, At, M, Bp) || !make_map_bf16(&bmap, Bt, R, 2 * Bp)) return NQ_ERR_CUDA;
     const int nkb = (int)(2 * Bp / kDK), ka_blocks = (int)(Bp / kDK);
-    return launch_pdl(dense_gemm_kernel, dim3((unsigned)(M / kDM), (unsigned)(R / kDN)), dim3(kDThreads), (size_t)kDSmem,
+    return launch_pdl(dense_gemm_kernel, dim3((unsigned)(R / kDN), (unsigned)(M / kDM)), dim3(kDThreads), (size_t)kDSmem,
                       stream, amap, bmap, nkb, ka_blocks, out, R, s, status) == cudaSuccess
                ? NQ_OK
                : NQ_ERR_CUDA;
