@@ -152,6 +152,7 @@ struct DecGroup {
     int w2words;      // stage-2 weight buffer: the most rows x words per row of one CTA
     int rows2;        // stage-2 rows held on chip: 16 x the most tiles of one CTA
     int per_sm2;      // stage-2 CTAs per SM of a one-wave plan (no more may share an SM), else 0
+    int t_global;     // stage 2 builds its B fragments from t in global memory (no staged copy)
     // CTA ranges in launch order: range k holds CTAs s1_start[k] .. s1_start[k+1]-1 of layer
     // s1_layer[k] (likewise for stage 2); the host puts the slowest layers first
     int s1_start[kMaxGroup + 1];
@@ -208,8 +209,9 @@ __host__ __device__ inline int s2_t_row(int r2) { return r2 + r2 / 4; }
 __host__ __device__ inline size_t s2_t_bytes(int batch, int r2) { return (size_t)batch * s2_t_row(r2) * 4; }
 __host__ __device__ inline size_t s2_bq_bytes(int rows2, int batch) { return ((size_t)rows2 * batch * 4 + 15) / 16 * 16; }
 __host__ __device__ inline size_t s2_s1_bytes(int rows2) { return ((size_t)rows2 * 2 + 15) / 16 * 16; }
-__host__ __device__ inline size_t s2_bytes(int w2words, int rows2, int batch, int r2, int ntg) {
-    return (size_t)w2words * 4 + s2_t_bytes(batch, r2) + frag_bytes(r2 / kCB, ntg) +
+// (t_global: no staged copy of t)
+__host__ __device__ inline size_t s2_bytes(int w2words, int rows2, int batch, int r2, int ntg, bool t_global = false) {
+    return (size_t)w2words * 4 + (t_global ? 0 : s2_t_bytes(batch, r2)) + frag_bytes(r2 / kCB, ntg) +
            s2_bq_bytes(rows2, batch) + s2_s1_bytes(rows2) + sizeof(Misc);
 }
 
@@ -305,6 +307,47 @@ __device__ __forceinline__ void build_fragments2(uint4* frag, Misc& mi, Val val,
             if ((threadIdx.x & 31) == 0 && v != 0) atomicAdd(&mi.qsum[tok], v);
         }
     }
+}
+
+// build_fragments for one token, reading t from global memory instead of a staged copy:
+// each thread takes up to four tasks per round and issues all their loads before
+// quantising, so that the round costs one L2 round trip.  Same values, layout and sums as
+// build_fragments at batch 1.
+template <int NT>
+__device__ __forceinline__ void build_fragments_t1(uint4* frag, Misc& mi, const float* __restrict__ t, int ncb) {
+    const int tasks = ncb * 32;
+    const float up = mi.up[0];
+    int qs = 0;
+    for (int t0 = threadIdx.x; t0 < tasks; t0 += 4 * NT) {
+        float v[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int task = t0 + u * NT;
+            const int j = task & 7, tt = (task >> 3) & 3, cb = task >> 5;
+            const int col = cb * kCB + 32 * tt + (j >> 1) + 4 * (j & 1);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) v[u][c] = task < tasks ? __ldcg(t + col + 8 * c) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int task = t0 + u * NT;
+            if (task < tasks) {
+                const int j = task & 7, tt = (task >> 3) & 3, cb = task >> 5;
+                uint32_t wh = 0, wl = 0;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int q = quantise(v[u][c], up);
+                    qs += q;
+                    wh |= (uint32_t)((q >> 7) & 0xFF) << (8 * c);
+                    wl |= (uint32_t)(q & 0x7F) << (8 * c);
+                }
+                reinterpret_cast<uint32_t*>(frag_ptr<1>(frag, cb, 0, j >> 2, tt))[j & 3] = wh;
+                reinterpret_cast<uint32_t*>(frag_ptr<1>(frag, cb, 0, j >> 2, 4 + tt))[j & 3] = wl;
+            }
+        }
+    }
+    for (int o = 16; o > 0; o >>= 1) qs += __shfl_xor_sync(0xffffffffu, qs, o);
+    if ((threadIdx.x & 31) == 0 && qs != 0) atomicAdd(&mi.qsum[0], qs);
 }
 
 // One column block of a 16-row tile into accumulator set `acc`.
@@ -725,7 +768,8 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
     const int batch = grp.batch, r2 = grp.r2, rows2 = grp.rows2;
     uint32_t* wbuf = reinterpret_cast<uint32_t*>(smem_raw);
     float* tbuf = reinterpret_cast<float*>(smem_raw + (size_t)grp.w2words * 4);
-    uint4* frag = reinterpret_cast<uint4*>(smem_raw + (size_t)grp.w2words * 4 + s2_t_bytes(batch, r2));
+    uint4* frag = reinterpret_cast<uint4*>(smem_raw + (size_t)grp.w2words * 4 +
+                                           (grp.t_global ? 0 : s2_t_bytes(batch, r2)));
     int* bq = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(frag) + frag_bytes(r2 / kCB, NTG));
     uint16_t* s1buf = reinterpret_cast<uint16_t*>(reinterpret_cast<unsigned char*>(bq) + s2_bq_bytes(rows2, batch));
     Misc& mi = *reinterpret_cast<Misc*>(reinterpret_cast<unsigned char*>(s1buf) + s2_s1_bytes(rows2));
@@ -826,8 +870,10 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
             }
         }
     } else {
-        fetch_t(0);
-        cp_async_commit();
+        if (!grp.t_global) {
+            fetch_t(0);
+            cp_async_commit();
+        }
 
         // global max |t| per token from the per-block maxima (one warp per token)
         const int nrb = r / kRowsS1;
@@ -858,6 +904,8 @@ __global__ void __launch_bounds__(kThreads, NTG == 1 ? 3 : 2) stage2_kernel(cons
         auto tval = [&](int tok, int c) { return tbuf[tok * s2_t_row(r2) + c + 8 * (c >> 5)]; };
         if constexpr (NTG == 2 || CM)
             build_fragments2<NTG, kThreads>(frag, mi, tval, [](int) { return 1.0f; }, ncb, batch);
+        else if (grp.t_global)
+            build_fragments_t1<kThreads>(frag, mi, L.t, ncb);
         else
             build_fragments<NTG, kThreads>(frag, mi, tval, ncb, batch);
         __syncthreads();
@@ -1266,7 +1314,7 @@ int launch_stages(DecGroup& grp, cudaStream_t stream, int device, bool stage1_on
         __atomic_fetch_or(&init_mask, bit, __ATOMIC_RELEASE);
     }
     const size_t smem1 = s1_bytes(grp.depth1, grp.batch, NTG);
-    size_t smem2 = s2_bytes(grp.w2words, grp.rows2, grp.batch, grp.r2, NTG);
+    size_t smem2 = s2_bytes(grp.w2words, grp.rows2, grp.batch, grp.r2, NTG, grp.t_global != 0);
     // a one-wave stage-2 plan gives every SM the same work only if no SM takes more than
     // per_sm2 of its CTAs: ask for enough shared memory that one more does not fit
     if (grp.per_sm2 > 0) smem2 = std::max(smem2, kSmemPerSM / (grp.per_sm2 + 1) - kSmemReserve + 16);
@@ -1386,6 +1434,32 @@ static void stage2_plan(const DecodeCall* calls, int count, int64_t batch, int* 
     measure();
 }
 
+// A several-wave stage-2 plan at batch 1 without the staged copy of t (its 19 KB at r = 3840
+// go to weight rows instead): the fewest tiles per CTA (from kWaveTiles2) for which the CTAs
+// fill at most two waves of two CTAs per SM.  false (nothing changed) if there is none.
+// Measured on a B200, the Llama-2-70B-shaped block at batch 1: 656 CTAs of 8 tiles (2.22
+// waves) -> 587 CTAs of 9 tiles (1.98 waves), 36.9 -> 36.1 us per step.
+static bool stage2_plan_t_global(const DecodeCall* calls, int count, int r2, int* ctas, int* w2words, int* rows2) {
+    const int sms = sm_count();
+    for (int tpc = kWaveTiles2; tpc <= 2 * kWaveTiles2; ++tpc) {
+        int64_t total = 0, words = 0, rows = 0;
+        for (int i = 0; i < count; ++i) {
+            const int64_t ti = calls[i].m / 16, c = (ti + tpc - 1) / tpc;
+            total += c;
+            const int64_t tl = (ti + c - 1) / c;
+            words = std::max(words, 16 * tl * s2_stride((int)calls[i].r, r2));
+            rows = std::max(rows, 16 * tl);
+        }
+        if (total > 4 * (int64_t)sms) continue;  // two waves of two CTAs per SM
+        if (2 * (s2_bytes((int)words, (int)rows, 1, r2, 1, true) + kSmemReserve) > kSmemPerSM) return false;
+        for (int i = 0; i < count; ++i) ctas[i] = (int)((calls[i].m / 16 + tpc - 1) / tpc);
+        *w2words = (int)words;
+        *rows2 = (int)rows;
+        return true;
+    }
+    return false;
+}
+
 // Column blocks per stage-1 split: about two CTAs per SM over the whole launch, at least
 // 4 and (while the split count stays <= max_splits) at most kChunkCB column blocks per CTA,
 // so that every CTA does one chunk.
@@ -1495,6 +1569,13 @@ int decode_forward_group(const DecodeCall* calls, int count, int64_t batch, Work
     grp.stream2 = stream2 ? 1 : 0;
     const bool s2sum = !stream2 && !stage1_only && r_max <= grp.r2 && r_max <= 4 * kSumSlots * kThreads &&
                        max_nsplit <= kS2SumMaxSplits;
+    // One token, a several-wave stage-2 plan, one span, t from stage 1's hand-off: stage 2
+    // builds its fragments from t in global memory, and the shared memory of the staged copy
+    // goes to CTAs of more rows that fill two waves instead of two and a fraction.
+    grp.t_global = 0;
+    if (batch == 1 && !stage1_only && !stream2 && !s2sum && grp.per_sm2 == 0 && r_max <= grp.r2 &&
+        stage2_plan_t_global(calls, count, grp.r2, ctas, &grp.w2words, &grp.rows2))
+        grp.t_global = 1;
     grp.depth1 = cps > kChunkCB ? 2 : 1;
     size_t toff = 0, goff = 0, poff = 0, coff = 0;
     grp.s1_start[0] = grp.s2_start[0] = 0;
