@@ -655,9 +655,10 @@ def admm_flops_per_iteration(m, n, r):
 
 
 def run_admm(device, stream, peaks, iters=40, shape=(4096, 4096, 1664), repeats=3):
-    """The LB-ADMM initialiser on a synthetic Llama-2-7B attention-shaped weight: time of the
-    whole nq_admm_factorize call (start, iterations, balancing, packing, error), and of the
-    iterations alone from the per-iteration difference of two call lengths."""
+    """The LB-ADMM initialiser on a synthetic Llama-2-7B attention-shaped weight: the whole
+    nq_admm_factorize call by wall clock (start, iterations, balancing, packing, error; host
+    allocation included), and the iterations by CUDA events on the call's stream around
+    nq_admm_iterate calls of `iters` iterations from one start (median of `repeats`)."""
     import torch
 
     from binary_rank_linear_02_b200 import nq
@@ -669,16 +670,25 @@ def run_admm(device, stream, peaks, iters=40, shape=(4096, 4096, 1664), repeats=
     def one(k):
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        out = nq.admm_factorize(W, m, n, r, Om, iters=k)
+        out = nq.admm_factorize(W, m, n, r, Om, iters=k, stream=stream.cuda_stream)
         torch.cuda.synchronize()
         return time.perf_counter() - t0, out[4]
 
     one(2)  # warm-up (module load, first allocations)
-    t_short = statistics.median([one(2)[0] for _ in range(repeats)])
     runs = [one(iters) for _ in range(repeats)]
     t_full = statistics.median([t for t, _ in runs])
     err = runs[0][1]
-    per_it = (t_full - t_short) / (iters - 2)
+    st = nq.admm_init(W, m, n, r, Om, 1, stream=stream.cuda_stream)
+    nq.admm_iterate(W, st, 2, stream=stream.cuda_stream)
+    times = []
+    for _ in range(repeats):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        nq.admm_iterate(W, st, iters, stream=stream.cuda_stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+        times.append(start.elapsed_time(end) / 1e3)
+    per_it = statistics.median(times) / iters
     fl = admm_flops_per_iteration(m, n, r)
     tf = fl / per_it / 1e12
     return {"shape": f"{m}x{n} r={r}", "iters": iters, "seconds_per_call": round(t_full, 4),
@@ -687,7 +697,8 @@ def run_admm(device, stream, peaks, iters=40, shape=(4096, 4096, 1664), repeats=
             "roofline": {"bound": "alu", "achieved": round(tf, 2), "peak": round(FP32_ALU_TFLOPS, 1),
                          "unit": "TFLOP/s", "frac": round(tf / FP32_ALU_TFLOPS, 4),
                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"},
-            "timing": "wall clock around the synchronising call (host-side allocation included), median"}
+            "timing": "iterations: CUDA events on the launching stream around nq_admm_iterate calls "
+                      "(median); seconds_per_call: wall clock around the whole synchronising call"}
 
 
 def run_envelope(device, stream, peaks, steps=200, batch=1, l=2, shape=(4096, 4096, 1664)):

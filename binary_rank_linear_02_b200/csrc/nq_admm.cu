@@ -468,6 +468,10 @@ struct AdmmState {
     float* H;     // r x r
     float* rho;   // device scalar
     int* flag;    // device: a Cholesky pivot was not positive
+    // the iterations' products of W on the tensor cores (set when the call iterates)
+    const uint16_t* Wt = nullptr;  // W^T: n x m bf16
+    void* dscr = nullptr;          // a factor split into three bf16 parts: r x 3 max(m, n)
+    unsigned* status = nullptr;    // bounded-wait timeouts of those products
 };
 
 int project(float* X, float* L, float* Z, float* sc, int64_t rows, int64_t r, int dual, cudaStream_t s) {
@@ -487,18 +491,11 @@ int half_step(AdmmState& st, const float* F, int64_t frows, float* X, int64_t xr
     add_penalty_kernel<<<1, 256, 0, s>>>(st.H, r, lam, st.rho);
     int rc = cholesky(st.H, r, st.flag, s);
     if (rc != NQ_OK) return rc;
-    // R = Wop F + rho (Zx - Lx)
+    // R = Wop F + rho (Zx - Lx), on the tensor cores: W in bf16 as given (exact), F as the
+    // sum of three bf16 parts (fp32's precision), fp32 accumulation in a fixed order
     const int64_t K = TRANS ? st.m : st.n;
-    GemmF32<__nv_bfloat16> w = gemm_args<__nv_bfloat16>(xrows, r, K, st.W, st.n, F, r, X, r);
-    w.beta = 1.f;
-    w.D = Zx;
-    w.ldd = r;
-    w.gamma = -1.f;
-    w.E = Lx;
-    w.lde = r;
-    w.scale = st.rho;
-    if ((TRANS ? gemm<__nv_bfloat16, true, false>(w, s) : gemm<__nv_bfloat16, false, false>(w, s)) != NQ_OK)
-        return NQ_ERR_CUDA;
+    const uint16_t* Wop = TRANS ? st.Wt : reinterpret_cast<const uint16_t*>(st.W);
+    if ((rc = dense_af(Wop, xrows, K, F, r, X, Zx, Lx, st.rho, st.dscr, st.status, s)) != NQ_OK) return rc;
     if ((rc = solve_lower_T(X, xrows, st.H, r, s)) != NQ_OK) return rc;
     if ((rc = solve_lower(X, xrows, st.H, r, s)) != NQ_OK) return rc;
     return project(X, Lx, Zx, sx, xrows, r, 1, s);
@@ -576,9 +573,14 @@ struct Scratch {
     }
 };
 
-int bind_scratch(AdmmState& st, Scratch& sc) {
+// dense: also W^T and the split-factor buffer of the iterations' tensor-core products
+// (W^T made here, on stream s).
+int bind_scratch(AdmmState& st, Scratch& sc, bool dense = false, cudaStream_t s = nullptr) {
     const int64_t rows = st.m > st.n ? st.m : st.n;
-    const size_t bytes = sizeof(float) * (size_t)(rows * st.r + st.r * st.r) + 256;
+    const size_t base_bytes = sizeof(float) * (size_t)(rows * st.r + st.r * st.r) + 256;
+    const size_t wt_bytes = dense ? (size_t)(st.m * st.n) * 2 : 0;
+    const size_t d_bytes = dense ? (size_t)dense_af_scratch_bytes(rows, st.r) : 0;
+    const size_t bytes = base_bytes + 256 + wt_bytes + 256 + d_bytes;
     if (cudaMalloc(&sc.base, bytes) != cudaSuccess) {
         cudaGetLastError();
         sc.base = nullptr;
@@ -588,15 +590,25 @@ int bind_scratch(AdmmState& st, Scratch& sc) {
     st.H = st.R + rows * st.r;
     st.rho = st.H + st.r * st.r;
     st.flag = reinterpret_cast<int*>(st.rho + 4);
-    return cudaMemset(st.flag, 0, sizeof(int)) == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
+    st.status = reinterpret_cast<unsigned*>(st.flag + 1);
+    if (cudaMemset(st.flag, 0, 2 * sizeof(int)) != cudaSuccess) return NQ_ERR_CUDA;  // flag and status
+    if (dense) {
+        char* p = sc.base + (base_bytes + 255) / 256 * 256;
+        uint16_t* wt = reinterpret_cast<uint16_t*>(p);
+        st.Wt = wt;
+        st.dscr = p + (wt_bytes + 255) / 256 * 256;
+        return transpose_bf16_device(reinterpret_cast<const uint16_t*>(st.W), st.m, st.n, wt, s);
+    }
+    return NQ_OK;
 }
 
 int finish_flag(AdmmState& st, cudaStream_t s) {
-    int flag = 0;
-    if (cudaMemcpyAsync(&flag, st.flag, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+    int flag[2] = {0, 0};  // the Cholesky flag, then the dense products' timeout word
+    if (cudaMemcpyAsync(flag, st.flag, sizeof(flag), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
         return NQ_ERR_CUDA;
-    return flag ? NQ_ERR_VALUE : NQ_OK;
+    if (flag[1]) return NQ_ERR_TIMEOUT;
+    return flag[0] ? NQ_ERR_VALUE : NQ_OK;
 }
 
 }  // namespace
@@ -619,7 +631,7 @@ extern "C" int nq_admm_iterate(const void* W, int64_t m, int64_t n, int64_t r, f
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     AdmmState st{m, n, r, static_cast<const __nv_bfloat16*>(W), A, B, ZA, ZB, LA, LB, sA, sB, nullptr, nullptr, nullptr, nullptr};
     Scratch sc;
-    if ((rc = bind_scratch(st, sc)) != NQ_OK) return rc;
+    if ((rc = bind_scratch(st, sc, true, s)) != NQ_OK) return rc;
     if ((rc = iterate(st, iters, lam0, growth, s)) != NQ_OK) return rc;
     return finish_flag(st, s);
 }
@@ -682,7 +694,7 @@ extern "C" int nq_admm_factorize(const void* W, int64_t m, int64_t n, int64_t r,
     double* part = reinterpret_cast<double*>(sB + n);
     AdmmState st{m, n, r, static_cast<const __nv_bfloat16*>(W), A, B, ZA, ZB, LA, LB, sA, sB, nullptr, nullptr, nullptr, nullptr};
     Scratch sc;
-    if ((rc = bind_scratch(st, sc)) != NQ_OK) return rc;
+    if ((rc = bind_scratch(st, sc, true, s)) != NQ_OK) return rc;
     if ((rc = init(st, Omega, power_iters, s)) != NQ_OK) return rc;
     if ((rc = iterate(st, iters, lam0, growth, s)) != NQ_OK) return rc;
     balance_scales_kernel<<<1, 256, 0, s>>>(sA, m, sB, n, static_cast<uint16_t*>(s1), static_cast<uint16_t*>(s2));

@@ -14,6 +14,9 @@
 // K-major), warp 1 issues tcgen05.mma kind::f16 (bf16 operands, fp32 accumulators in tensor
 // memory), warps 2-5 read the accumulators back (tcgen05.ld) and write s_i * acc.  Every
 // mbarrier wait is bounded (NQ_ERR_TIMEOUT in the status word; the CTA drains and exits).
+// The same kernel serves the LB-ADMM initialiser's products of W (bf16 input, exact) with a
+// factor F (fp32, split into three bf16 parts: fp32's precision), out = W F + rho (D - E),
+// the penalty term of the least-squares step folded into the epilogue.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -49,6 +52,7 @@ struct DenseBarriers {
 __global__ void __launch_bounds__(kDThreads, 2)
 dense_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap, int nkb,
                   int ka_blocks, float* __restrict__ out, int64_t ldo, const uint16_t* __restrict__ s,
+                  const float* __restrict__ D, const float* __restrict__ E, const float* __restrict__ rho,
                   unsigned* __restrict__ status) {
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -137,17 +141,32 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constan
             pdl_trigger();
             const int quad = warp & 3;
             const int row = m0 + quad * 32 + lane;
-            const float sv = __half2float(__ushort_as_half(s[row]));
+            const float sv = s ? __half2float(__ushort_as_half(s[row])) : 1.f;
             float* orow = out + (int64_t)row * ldo + n0;
 #pragma unroll 1
             for (int c0 = 0; c0 < kDN; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+                if (D) {  // + rho (D - E), D and E laid out as out
+                    const float rv = *rho;
+                    const float* drow = D + (int64_t)row * ldo + n0 + c0;
+                    const float* erow = E + (int64_t)row * ldo + n0 + c0;
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4*>(orow + c0 + j) =
-                        make_float4(sv * __uint_as_float(v[j]), sv * __uint_as_float(v[j + 1]),
-                                    sv * __uint_as_float(v[j + 2]), sv * __uint_as_float(v[j + 3]));
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 d = *reinterpret_cast<const float4*>(drow + j);
+                        const float4 e = *reinterpret_cast<const float4*>(erow + j);
+                        *reinterpret_cast<float4*>(orow + c0 + j) = make_float4(
+                            fmaf(rv, d.x - e.x, sv * __uint_as_float(v[j])), fmaf(rv, d.y - e.y, sv * __uint_as_float(v[j + 1])),
+                            fmaf(rv, d.z - e.z, sv * __uint_as_float(v[j + 2])),
+                            fmaf(rv, d.w - e.w, sv * __uint_as_float(v[j + 3])));
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4*>(orow + c0 + j) =
+                            make_float4(sv * __uint_as_float(v[j]), sv * __uint_as_float(v[j + 1]),
+                                        sv * __uint_as_float(v[j + 2]), sv * __uint_as_float(v[j + 3]));
+                }
             }
         }
     }
@@ -218,6 +237,43 @@ __global__ void __launch_bounds__(256) transpose_split_kernel(const float* __res
     }
 }
 
+// dst[c][b], dst[c][K + b], dst[c][2K + b] = the three bf16 parts of v = src[b][c] (fp32):
+// hi = bf16(v), mid = bf16(v - hi), lo = bf16(v - hi - mid), whose sum carries v to ~2^-25
+// relative (fp32's own precision): for the ADMM products, whose sign projections and
+// small-penalty solves amplify the two-part error.  B rows (K) a multiple of 64.
+__global__ void __launch_bounds__(256) transpose_split3_kernel(const float* __restrict__ src, int64_t K, int64_t C,
+                                                               uint16_t* __restrict__ dst) {
+    __shared__ float tile[kTT][kTT + 1];
+    const int64_t c0 = (int64_t)blockIdx.x * kTT, b0 = (int64_t)blockIdx.y * kTT;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    for (int k = ty; k < kTT; k += 8) {
+        const int64_t b = b0 + k, c = c0 + 2 * tx;
+        float2 v = make_float2(0.f, 0.f);
+        if (c < C) v = *reinterpret_cast<const float2*>(src + b * C + c);
+        tile[k][2 * tx] = v.x;
+        tile[k][2 * tx + 1] = v.y;
+    }
+    __syncthreads();
+    for (int k = ty; k < kTT; k += 8) {
+        const int64_t c = c0 + k, b = b0 + 2 * tx;
+        if (c < C) {
+            uint32_t p[3] = {0u, 0u, 0u};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float v = tile[2 * tx + e][k];
+#pragma unroll
+                for (int q = 0; q < 3; ++q) {
+                    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+                    p[q] |= (uint32_t)__bfloat16_as_ushort(h) << (16 * e);
+                    v -= __bfloat162float(h);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 3; ++q) *reinterpret_cast<uint32_t*>(dst + c * 3 * K + q * K + b) = p[q];
+        }
+    }
+}
+
 bool make_map_bf16(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols) {
     // encode_map_u32_sw128 takes 32-bit words: a bf16 row of `cols` is cols / 2 words, the
     // 64-element box 32 words; TMA copies bytes, so the element type only sets the units
@@ -231,12 +287,8 @@ int64_t outer_tc_scratch_bytes(int64_t batch, int64_t M, int64_t R) {
     return 2 * (M * Bp + R * 2 * Bp) + 256;
 }
 
-int outer_tc(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch, int64_t M, int64_t R, float* out,
-             void* scratch, unsigned* status, cudaStream_t stream) {
-    if (M % kDM || R % kDN || batch <= 0) return NQ_ERR_SHAPE;
-    const int64_t Bp = (batch + kDPad - 1) / kDPad * kDPad;
-    uint16_t* At = static_cast<uint16_t*>(scratch);                      // M x Bp
-    uint16_t* Bt = At + ((M * Bp + 127) / 128) * 128;                    // R x 2 Bp (hi | lo)
+namespace {
+int dense_prepare() {
     static unsigned long long init_mask = 0;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NQ_ERR_CUDA;
@@ -246,18 +298,58 @@ int outer_tc(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch
             return NQ_ERR_CUDA;
         __atomic_fetch_or(&init_mask, bit, __ATOMIC_RELEASE);
     }
+    return NQ_OK;
+}
+
+// out (M x R, pitch R) = diag(s) A (sum of the parts of Bt)^T [+ rho (D - E)]: A is M x Kp
+// bf16 (K-major), Bt is R x parts Kp bf16 (the parts side by side), Kp a multiple of kDK.
+int dense_launch(const uint16_t* A, const uint16_t* Bt, int parts, int64_t M, int64_t Kp, int64_t R, float* out,
+                 const uint16_t* s, const float* D, const float* E, const float* rho, unsigned* status,
+                 cudaStream_t stream) {
+    CUtensorMap amap, bmap;
+    if (!make_map_bf16(&amap, A, M, Kp) || !make_map_bf16(&bmap, Bt, R, parts * Kp)) return NQ_ERR_CUDA;
+    const int nkb = (int)(parts * Kp / kDK), ka_blocks = (int)(Kp / kDK);
+    return launch_pdl(dense_gemm_kernel, dim3((unsigned)(R / kDN), (unsigned)(M / kDM)), dim3(kDThreads), (size_t)kDSmem,
+                      stream, amap, bmap, nkb, ka_blocks, out, R, s, D, E, rho, status) == cudaSuccess
+               ? NQ_OK
+               : NQ_ERR_CUDA;
+}
+}  // namespace
+
+int outer_tc(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch, int64_t M, int64_t R, float* out,
+             void* scratch, unsigned* status, cudaStream_t stream) {
+    if (M % kDM || R % kDN || batch <= 0) return NQ_ERR_SHAPE;
+    const int64_t Bp = (batch + kDPad - 1) / kDPad * kDPad;
+    uint16_t* At = static_cast<uint16_t*>(scratch);                      // M x Bp
+    uint16_t* Bt = At + ((M * Bp + 127) / 128) * 128;                    // R x 2 Bp (hi | lo)
+    int rc = dense_prepare();
+    if (rc != NQ_OK) return rc;
     transpose_pad_kernel<<<dim3((unsigned)((M + kTT - 1) / kTT), (unsigned)(Bp / kTT)), 256, 0, stream>>>(a, batch, M,
                                                                                                        Bp, At);
     transpose_split_kernel<<<dim3((unsigned)((R + kTT - 1) / kTT), (unsigned)(Bp / kTT)), 256, 0, stream>>>(t, batch, R,
                                                                                                          Bp, Bt);
     if (cudaGetLastError() != cudaSuccess) return NQ_ERR_CUDA;
-    CUtensorMap amap, bmap;
-    if (!make_map_bf16(&amap, At, M, Bp) || !make_map_bf16(&bmap, Bt, R, 2 * Bp)) return NQ_ERR_CUDA;
-    const int nkb = (int)(2 * Bp / kDK), ka_blocks = (int)(Bp / kDK);
-    return launch_pdl(dense_gemm_kernel, dim3((unsigned)(R / kDN), (unsigned)(M / kDM)), dim3(kDThreads), (size_t)kDSmem,
-                      stream, amap, bmap, nkb, ka_blocks, out, R, s, status) == cudaSuccess
-               ? NQ_OK
-               : NQ_ERR_CUDA;
+    return dense_launch(At, Bt, 2, M, Bp, R, out, s, nullptr, nullptr, nullptr, status, stream);
+}
+
+int64_t dense_af_scratch_bytes(int64_t K, int64_t R) { return 2 * (R * 3 * K) + 256; }
+
+int dense_af(const uint16_t* A, int64_t M, int64_t K, const float* F, int64_t R, float* out, const float* D,
+             const float* E, const float* rho, void* scratch, unsigned* status, cudaStream_t stream) {
+    if (M % kDM || R % kDN || K % kDK || K <= 0) return NQ_ERR_SHAPE;
+    uint16_t* Bt = static_cast<uint16_t*>(scratch);  // R x 3K (hi | mid | lo)
+    int rc = dense_prepare();
+    if (rc != NQ_OK) return rc;
+    transpose_split3_kernel<<<dim3((unsigned)((R + kTT - 1) / kTT), (unsigned)(K / kTT)), 256, 0, stream>>>(F, K, R, Bt);
+    if (cudaGetLastError() != cudaSuccess) return NQ_ERR_CUDA;
+    return dense_launch(A, Bt, 3, M, K, R, out, nullptr, D, E, rho, status, stream);
+}
+
+int transpose_bf16_device(const uint16_t* src, int64_t rows, int64_t cols, uint16_t* dst, cudaStream_t stream) {
+    if (rows % kTT || cols % kTT) return NQ_ERR_SHAPE;
+    transpose_pad_kernel<<<dim3((unsigned)(cols / kTT), (unsigned)(rows / kTT)), 256, 0, stream>>>(src, rows, cols, rows,
+                                                                                                dst);
+    return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
 }
 
 }  // namespace nq

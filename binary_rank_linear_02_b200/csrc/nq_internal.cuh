@@ -107,6 +107,14 @@ int prefill_rank_vector(const uint16_t* x, const uint32_t* Vpk, const uint16_t* 
 int64_t outer_tc_scratch_bytes(int64_t batch, int64_t M, int64_t R);
 int outer_tc(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch, int64_t M, int64_t R, float* out,
              void* scratch, unsigned* status, cudaStream_t stream);
+// out (M x R fp32) = A F + rho (D - E) on the tensor cores: A is M x K bfloat16 (row pitch K,
+// K a multiple of 64), F is K x R fp32 split into three bfloat16 parts (scratch of
+// dense_af_scratch_bytes), D and E laid out as out, rho a device scalar; M, R multiples of 128.
+int64_t dense_af_scratch_bytes(int64_t K, int64_t R);
+int dense_af(const uint16_t* A, int64_t M, int64_t K, const float* F, int64_t R, float* out, const float* D,
+             const float* E, const float* rho, void* scratch, unsigned* status, cudaStream_t stream);
+// dst (cols x rows) = src^T for a rows x cols bfloat16 matrix (both multiples of 64)
+int transpose_bf16_device(const uint16_t* src, int64_t rows, int64_t cols, uint16_t* dst, cudaStream_t stream);
 // out[i][k] = s[i] * sum over b (increasing) of bf16(a[b][i]) * t[b][k]: M x R fp32
 int outer_device(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch, int64_t M, int64_t R,
                  float* out, cudaStream_t stream);
