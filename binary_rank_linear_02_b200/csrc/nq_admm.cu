@@ -469,8 +469,7 @@ struct AdmmState {
     float* rho;   // device scalar
     int* flag;    // device: a Cholesky pivot was not positive
     // the iterations' products of W on the tensor cores (set when the call iterates)
-    const uint16_t* Wt = nullptr;  // W^T: n x m bf16
-    void* dscr = nullptr;          // a factor split into three bf16 parts: r x 3 max(m, n)
+    void* dscr = nullptr;          // a factor split into three bf16 parts: 3 max(m, n) x r
     unsigned* status = nullptr;    // bounded-wait timeouts of those products
 };
 
@@ -493,9 +492,11 @@ int half_step(AdmmState& st, const float* F, int64_t frows, float* X, int64_t xr
     if (rc != NQ_OK) return rc;
     // R = Wop F + rho (Zx - Lx), on the tensor cores: W in bf16 as given (exact), F as the
     // sum of three bf16 parts (fp32's precision), fp32 accumulation in a fixed order
+    // (W^T read in place: W's rows are its columns)
     const int64_t K = TRANS ? st.m : st.n;
-    const uint16_t* Wop = TRANS ? st.Wt : reinterpret_cast<const uint16_t*>(st.W);
-    if ((rc = dense_af(Wop, xrows, K, F, r, X, Zx, Lx, st.rho, st.dscr, st.status, s)) != NQ_OK) return rc;
+    if ((rc = dense_af(reinterpret_cast<const uint16_t*>(st.W), !TRANS, xrows, K, F, r, X, Zx, Lx, st.rho, st.dscr,
+                       st.status, s)) != NQ_OK)
+        return rc;
     if ((rc = solve_lower_T(X, xrows, st.H, r, s)) != NQ_OK) return rc;
     if ((rc = solve_lower(X, xrows, st.H, r, s)) != NQ_OK) return rc;
     return project(X, Lx, Zx, sx, xrows, r, 1, s);
@@ -573,14 +574,12 @@ struct Scratch {
     }
 };
 
-// dense: also W^T and the split-factor buffer of the iterations' tensor-core products
-// (W^T made here, on stream s).
-int bind_scratch(AdmmState& st, Scratch& sc, bool dense = false, cudaStream_t s = nullptr) {
+// dense: also the split-factor buffer of the iterations' tensor-core products.
+int bind_scratch(AdmmState& st, Scratch& sc, bool dense = false) {
     const int64_t rows = st.m > st.n ? st.m : st.n;
     const size_t base_bytes = sizeof(float) * (size_t)(rows * st.r + st.r * st.r) + 256;
-    const size_t wt_bytes = dense ? (size_t)(st.m * st.n) * 2 : 0;
     const size_t d_bytes = dense ? (size_t)dense_af_scratch_bytes(rows, st.r) : 0;
-    const size_t bytes = base_bytes + 256 + wt_bytes + 256 + d_bytes;
+    const size_t bytes = base_bytes + 256 + d_bytes;
     if (cudaMalloc(&sc.base, bytes) != cudaSuccess) {
         cudaGetLastError();
         sc.base = nullptr;
@@ -591,15 +590,8 @@ int bind_scratch(AdmmState& st, Scratch& sc, bool dense = false, cudaStream_t s 
     st.rho = st.H + st.r * st.r;
     st.flag = reinterpret_cast<int*>(st.rho + 4);
     st.status = reinterpret_cast<unsigned*>(st.flag + 1);
-    if (cudaMemset(st.flag, 0, 2 * sizeof(int)) != cudaSuccess) return NQ_ERR_CUDA;  // flag and status
-    if (dense) {
-        char* p = sc.base + (base_bytes + 255) / 256 * 256;
-        uint16_t* wt = reinterpret_cast<uint16_t*>(p);
-        st.Wt = wt;
-        st.dscr = p + (wt_bytes + 255) / 256 * 256;
-        return transpose_bf16_device(reinterpret_cast<const uint16_t*>(st.W), st.m, st.n, wt, s);
-    }
-    return NQ_OK;
+    if (dense) st.dscr = sc.base + (base_bytes + 255) / 256 * 256;
+    return cudaMemset(st.flag, 0, 2 * sizeof(int)) == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;  // flag and status
 }
 
 int finish_flag(AdmmState& st, cudaStream_t s) {
@@ -631,7 +623,7 @@ extern "C" int nq_admm_iterate(const void* W, int64_t m, int64_t n, int64_t r, f
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     AdmmState st{m, n, r, static_cast<const __nv_bfloat16*>(W), A, B, ZA, ZB, LA, LB, sA, sB, nullptr, nullptr, nullptr, nullptr};
     Scratch sc;
-    if ((rc = bind_scratch(st, sc, true, s)) != NQ_OK) return rc;
+    if ((rc = bind_scratch(st, sc, true)) != NQ_OK) return rc;
     if ((rc = iterate(st, iters, lam0, growth, s)) != NQ_OK) return rc;
     return finish_flag(st, s);
 }
@@ -694,7 +686,7 @@ extern "C" int nq_admm_factorize(const void* W, int64_t m, int64_t n, int64_t r,
     double* part = reinterpret_cast<double*>(sB + n);
     AdmmState st{m, n, r, static_cast<const __nv_bfloat16*>(W), A, B, ZA, ZB, LA, LB, sA, sB, nullptr, nullptr, nullptr, nullptr};
     Scratch sc;
-    if ((rc = bind_scratch(st, sc, true, s)) != NQ_OK) return rc;
+    if ((rc = bind_scratch(st, sc, true)) != NQ_OK) return rc;
     if ((rc = init(st, Omega, power_iters, s)) != NQ_OK) return rc;
     if ((rc = iterate(st, iters, lam0, growth, s)) != NQ_OK) return rc;
     balance_scales_kernel<<<1, 256, 0, s>>>(sA, m, sB, n, static_cast<uint16_t*>(s1), static_cast<uint16_t*>(s2));

@@ -10,13 +10,16 @@
 // the sum of two bfloat16 numbers, hi = bf16(v) and lo = bf16(v - hi), in the two halves of
 // a doubled K (the A tile is the same for both halves: its TMA coordinate wraps): a
 // bf16 x bf16 product is exact in fp32, so the products carry ~2^-17 relative error of v.
-// One CTA per 128 x 128 output tile: warp 0 loads A and B tiles by TMA (128-byte swizzle,
-// K-major), warp 1 issues tcgen05.mma kind::f16 (bf16 operands, fp32 accumulators in tensor
-// memory), warps 2-5 read the accumulators back (tcgen05.ld) and write s_i * acc.  Every
-// mbarrier wait is bounded (NQ_ERR_TIMEOUT in the status word; the CTA drains and exits).
-// The same kernel serves the LB-ADMM initialiser's products of W (bf16 input, exact) with a
-// factor F (fp32, split into three bf16 parts: fp32's precision), out = W F + rho (D - E),
-// the penalty term of the least-squares step folded into the epilogue.
+// Both operands are read where they lie, token-major ([K][M] and [K][R] rows): the tensor
+// cores take MN-major shared-memory tiles (rows of 64 M or R elements along K), so neither
+// a nor the split rank vectors are transposed.
+// One CTA per 128 x 128 output tile: warp 0 loads A and B tiles by TMA (128-byte swizzle),
+// warp 1 issues tcgen05.mma kind::f16 (bf16 operands, fp32 accumulators in tensor memory),
+// warps 2-5 read the accumulators back (tcgen05.ld) and write s_i * acc.  Every mbarrier
+// wait is bounded (NQ_ERR_TIMEOUT in the status word; the CTA drains and exits).
+// The same kernel serves the LB-ADMM initialiser's products of W (bf16 input, exact; K-major
+// for W F, MN-major for W^T F) with a factor F (fp32, split into three bf16 parts: fp32's
+// precision), out = Wop F + rho (D - E), the penalty term folded into the epilogue.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -34,10 +37,26 @@ constexpr int kDStageBytes = 2 * kDTileBytes;
 constexpr int kDThreads = 192;
 constexpr int kDSmem = kDStages * kDStageBytes + 1024 /*barriers*/ + 1024 /*alignment slack*/;
 constexpr int kDPad = 64;                         // tokens are padded to a multiple of this
+constexpr int kDHalf = kDTileBytes / 2;           // one TMA box of an MN-major tile: 64 rows x 64 elements
 
-// kind::f16 instruction descriptor: bf16 A and B (format 1), K-major both, fp32 D, M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+// kind::f16 instruction descriptor: bf16 A and B (format 1), fp32 D, M x N; A and B K-major
+// (0) or MN-major (1, bits 15 and 16).
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool amn, bool bmn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((amn ? 1u : 0u) << 15) | ((bmn ? 1u : 0u) << 16) |
+           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// SW128 MN-major shared-memory operand descriptor: rows of 64 elements (128 B) along K,
+// 8-row groups 1024 B apart (stride byte offset), the second 64-element block of the tile's
+// 128 M (or N) elements one TMA box (8 KB) further (leading byte offset).
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFF);
+    d |= (uint64_t)(kDHalf >> 4) << 16;  // leading byte offset: next 64-element block
+    d |= (uint64_t)(1024 >> 4) << 32;    // stride byte offset: next 8-row group
+    d |= (uint64_t)1 << 46;              // descriptor version for tcgen05
+    d |= (uint64_t)2 << 61;              // 128-byte swizzle
+    return d;
 }
 
 struct DenseBarriers {
@@ -48,7 +67,10 @@ struct DenseBarriers {
 };
 
 // out[(m0 + i) * ldo + n0 + j] = s[m0 + i] * sum_k A[m0 + i][k] B[n0 + j][k] over nkb stages;
-// A's stage kb reads K block kb % ka_blocks.
+// A's stage kb reads K block kb % ka_blocks.  AMN / BMN: the operand's map is over [K][M]
+// ([K][N]) rows, each stage two 64 x 64 boxes (MN-major), else over [M][K] ([N][K]) rows,
+// one 128 x 64 box (K-major).
+template <bool AMN, bool BMN>
 __global__ void __launch_bounds__(kDThreads, 2)
 dense_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap, int nkb,
                   int ka_blocks, float* __restrict__ out, int64_t ldo, const uint16_t* __restrict__ s,
@@ -100,8 +122,19 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constan
                 mbar_expect_tx(full, (uint32_t)kDStageBytes);
                 const uint32_t dst = base + (uint32_t)(st * kDStageBytes);
                 // x coordinates in 32-bit words of the maps (two bf16 each)
-                tma_load_2d(dst, &amap, (kb % ka_blocks) * (kDK / 2), m0, full);
-                tma_load_2d(dst + kDTileBytes, &bmap, kb * (kDK / 2), n0, full);
+                const int ka = kb % ka_blocks;
+                if constexpr (AMN) {
+                    tma_load_2d(dst, &amap, m0 / 2, ka * kDK, full);
+                    tma_load_2d(dst + kDHalf, &amap, m0 / 2 + kDK / 2, ka * kDK, full);
+                } else {
+                    tma_load_2d(dst, &amap, ka * (kDK / 2), m0, full);
+                }
+                if constexpr (BMN) {
+                    tma_load_2d(dst + kDTileBytes, &bmap, n0 / 2, kb * kDK, full);
+                    tma_load_2d(dst + kDTileBytes + kDHalf, &bmap, n0 / 2 + kDK / 2, kb * kDK, full);
+                } else {
+                    tma_load_2d(dst + kDTileBytes, &bmap, kb * (kDK / 2), n0, full);
+                }
                 ++issued;
             }
             if (*abort_flag) {
@@ -112,19 +145,21 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constan
     } else if (warp == 1) {
         // ---------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(kDM, kDN);
+            constexpr uint32_t idesc = idesc_bf16(kDM, kDN, AMN, BMN);
             int kb = 0;
             for (; kb < nkb; ++kb) {
                 const int st = kb % kDStages;
                 const uint32_t ph = (uint32_t)(kb / kDStages) & 1u;
                 if (!mbar_wait(smem_u32(&bar.full[st]), ph, abort_flag, status)) break;
                 tc_fence_after();
-                const uint64_t ad = sw128_desc(base + (uint32_t)(st * kDStageBytes));
-                const uint64_t bd = sw128_desc(base + (uint32_t)(st * kDStageBytes + kDTileBytes));
+                const uint32_t aaddr = base + (uint32_t)(st * kDStageBytes), baddr = aaddr + kDTileBytes;
+                const uint64_t ad = AMN ? sw128_desc_mn(aaddr) : sw128_desc(aaddr);
+                const uint64_t bd = BMN ? sw128_desc_mn(baddr) : sw128_desc(baddr);
+                // a K step of 16: 32 bytes along a K-major row, 16 rows (2 KB) of an MN-major tile
+                constexpr uint64_t astep = AMN ? 2048 / 16 : 32 / 16, bstep = BMN ? 2048 / 16 : 32 / 16;
 #pragma unroll
                 for (int k = 0; k < kDK / 16; ++k)
-                    umma_f16(tmem, ad + (uint64_t)(k * 16 * 2 / 16), bd + (uint64_t)(k * 16 * 2 / 16), idesc,
-                             (kb > 0 || k > 0) ? 1u : 0u);
+                    umma_f16(tmem, ad + (uint64_t)k * astep, bd + (uint64_t)k * bstep, idesc, (kb > 0 || k > 0) ? 1u : 0u);
                 umma_commit(smem_u32(&bar.empty[st]));
             }
             if (kb == nkb) {
@@ -178,141 +213,103 @@ dense_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constan
     }
 }
 
-// dst[c][b] = src[b][c] (bf16) for b < B, 0 for B <= b < Bp: the K-major A operand from
-// token-major activations.  64 x 64 tiles through shared memory (row pitch 65 halves: the
-// column reads of the write-out fall in distinct banks), each thread moving two adjacent
-// elements per access so that a warp reads and writes 128 contiguous bytes.
-constexpr int kTT = 64;
-__global__ void __launch_bounds__(256) transpose_pad_kernel(const uint16_t* __restrict__ src, int64_t B, int64_t C,
-                                                            int64_t Bp, uint16_t* __restrict__ dst) {
-    __shared__ uint16_t tile[kTT][kTT + 1];
-    const int64_t c0 = (int64_t)blockIdx.x * kTT, b0 = (int64_t)blockIdx.y * kTT;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
-    for (int k = ty; k < kTT; k += 8) {
-        const int64_t b = b0 + k, c = c0 + 2 * tx;
-        uint32_t v = 0;
-        if (b < B && c < C) v = *reinterpret_cast<const uint32_t*>(src + b * C + c);
-        tile[k][2 * tx] = (uint16_t)(v & 0xFFFFu);
-        tile[k][2 * tx + 1] = (uint16_t)(v >> 16);
-    }
-    __syncthreads();
-    for (int k = ty; k < kTT; k += 8) {
-        const int64_t c = c0 + k, b = b0 + 2 * tx;
-        if (c < C && b < Bp)
-            *reinterpret_cast<uint32_t*>(dst + c * Bp + b) = (uint32_t)tile[2 * tx][k] | ((uint32_t)tile[2 * tx + 1][k] << 16);
+// The rank vectors (batch x R fp32, token-major) as the B operand's rows: dst[b][c] =
+// bf16(v), dst[Bp + b][c] = bf16(v - bf16(v)) with v = src[b][c], zero rows for
+// B <= b < Bp.  Two columns per thread.
+__global__ void __launch_bounds__(256) split2_kernel(const float* __restrict__ src, int64_t B, int64_t C, int64_t Bp,
+                                                     uint16_t* __restrict__ dst) {
+    const int64_t pairs = Bp * C / 2;
+    for (int64_t p = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; p < pairs; p += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t b = p / (C / 2), c = 2 * (p % (C / 2));
+        const float2 v = b < B ? *reinterpret_cast<const float2*>(src + b * C + c) : make_float2(0.f, 0.f);
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(v.x), h1 = __float2bfloat16_rn(v.y);
+        const __nv_bfloat16 l0 = __float2bfloat16_rn(v.x - __bfloat162float(h0));
+        const __nv_bfloat16 l1 = __float2bfloat16_rn(v.y - __bfloat162float(h1));
+        *reinterpret_cast<uint32_t*>(dst + b * C + c) =
+            (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+        *reinterpret_cast<uint32_t*>(dst + (Bp + b) * C + c) =
+            (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
     }
 }
 
-// dst[c][b] = bf16(v), dst[c][Bp + b] = bf16(v - bf16(v)) with v = src[b][c] (fp32), zeros for
-// B <= b < Bp: the K-major B operand, each fp32 value as the sum of two bf16 numbers.  64 x 64
-// tiles as above (row pitch 65 floats).
-__global__ void __launch_bounds__(256) transpose_split_kernel(const float* __restrict__ src, int64_t B, int64_t C,
-                                                              int64_t Bp, uint16_t* __restrict__ dst) {
-    __shared__ float tile[kTT][kTT + 1];
-    const int64_t c0 = (int64_t)blockIdx.x * kTT, b0 = (int64_t)blockIdx.y * kTT;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-    for (int k = ty; k < kTT; k += 8) {
-        const int64_t b = b0 + k, c = c0 + 2 * tx;
-        float2 v = make_float2(0.f, 0.f);
-        if (b < B && c < C) v = *reinterpret_cast<const float2*>(src + b * C + c);
-        tile[k][2 * tx] = v.x;
-        tile[k][2 * tx + 1] = v.y;
-    }
-    __syncthreads();
-    for (int k = ty; k < kTT; k += 8) {
-        const int64_t c = c0 + k, b = b0 + 2 * tx;
-        if (c < C && b < Bp) {
-            uint32_t hi2 = 0, lo2 = 0;
+// A factor (K x C fp32, row-major) as the B operand's rows in three bf16 parts: dst[q K + k][c]
+// for q = 0, 1, 2 holds hi = bf16(v), mid = bf16(v - hi), lo = bf16(v - hi - mid), whose sum
+// carries v to ~2^-25 relative (fp32's own precision): for the ADMM products, whose sign
+// projections and small-penalty solves amplify a two-part error.  Two columns per thread.
+__global__ void __launch_bounds__(256) split3_kernel(const float* __restrict__ src, int64_t K, int64_t C,
+                                                     uint16_t* __restrict__ dst) {
+    const int64_t pairs = K * C / 2;
+    for (int64_t p = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; p < pairs; p += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t k = p / (C / 2), c = 2 * (p % (C / 2));
+        float2 v = *reinterpret_cast<const float2*>(src + k * C + c);
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float v = tile[2 * tx + e][k];
-                const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-                const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
-                hi2 |= (uint32_t)__bfloat16_as_ushort(hi) << (16 * e);
-                lo2 |= (uint32_t)__bfloat16_as_ushort(lo) << (16 * e);
-            }
-            *reinterpret_cast<uint32_t*>(dst + c * 2 * Bp + b) = hi2;
-            *reinterpret_cast<uint32_t*>(dst + c * 2 * Bp + Bp + b) = lo2;
+        for (int q = 0; q < 3; ++q) {
+            const __nv_bfloat16 h0 = __float2bfloat16_rn(v.x), h1 = __float2bfloat16_rn(v.y);
+            *reinterpret_cast<uint32_t*>(dst + ((int64_t)q * K + k) * C + c) =
+                (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+            v.x -= __bfloat162float(h0);
+            v.y -= __bfloat162float(h1);
         }
     }
 }
 
-// dst[c][b], dst[c][K + b], dst[c][2K + b] = the three bf16 parts of v = src[b][c] (fp32):
-// hi = bf16(v), mid = bf16(v - hi), lo = bf16(v - hi - mid), whose sum carries v to ~2^-25
-// relative (fp32's own precision): for the ADMM products, whose sign projections and
-// small-penalty solves amplify the two-part error.  B rows (K) a multiple of 64.
-__global__ void __launch_bounds__(256) transpose_split3_kernel(const float* __restrict__ src, int64_t K, int64_t C,
-                                                               uint16_t* __restrict__ dst) {
-    __shared__ float tile[kTT][kTT + 1];
-    const int64_t c0 = (int64_t)blockIdx.x * kTT, b0 = (int64_t)blockIdx.y * kTT;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-    for (int k = ty; k < kTT; k += 8) {
-        const int64_t b = b0 + k, c = c0 + 2 * tx;
-        float2 v = make_float2(0.f, 0.f);
-        if (c < C) v = *reinterpret_cast<const float2*>(src + b * C + c);
-        tile[k][2 * tx] = v.x;
-        tile[k][2 * tx + 1] = v.y;
-    }
-    __syncthreads();
-    for (int k = ty; k < kTT; k += 8) {
-        const int64_t c = c0 + k, b = b0 + 2 * tx;
-        if (c < C) {
-            uint32_t p[3] = {0u, 0u, 0u};
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float v = tile[2 * tx + e][k];
-#pragma unroll
-                for (int q = 0; q < 3; ++q) {
-                    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-                    p[q] |= (uint32_t)__bfloat16_as_ushort(h) << (16 * e);
-                    v -= __bfloat162float(h);
-                }
-            }
-#pragma unroll
-            for (int q = 0; q < 3; ++q) *reinterpret_cast<uint32_t*>(dst + c * 3 * K + q * K + b) = p[q];
-        }
-    }
-}
-
+// Maps over bf16 matrices (rows x cols elements, row pitch cols): encode_map_u32_sw128 takes
+// 32-bit words (a row is cols / 2 words); TMA copies bytes, so the element type only sets
+// the units.  K-major operand ([M][K] rows): boxes of 64 elements x 128 rows.  MN-major
+// operand ([K][M] rows): boxes of 64 elements x 64 rows.
 bool make_map_bf16(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols) {
-    // encode_map_u32_sw128 takes 32-bit words: a bf16 row of `cols` is cols / 2 words, the
-    // 64-element box 32 words; TMA copies bytes, so the element type only sets the units
     return encode_map_u32_sw128(map, ptr, rows, cols / 2, kDK / 2, kDM);
+}
+bool make_map_bf16_mn(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols) {
+    return encode_map_u32_sw128(map, ptr, rows, cols / 2, kDK / 2, kDK);
 }
 
 }  // namespace
 
 int64_t outer_tc_scratch_bytes(int64_t batch, int64_t M, int64_t R) {
     const int64_t Bp = (batch + kDPad - 1) / kDPad * kDPad;
-    return 2 * (M * Bp + R * 2 * Bp) + 256;
+    return 2 * (2 * Bp * R) + 256;
 }
 
 namespace {
+template <bool AMN, bool BMN>
 int dense_prepare() {
     static unsigned long long init_mask = 0;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NQ_ERR_CUDA;
     const unsigned long long bit = 1ull << (dev & 63);
     if (!(__atomic_load_n(&init_mask, __ATOMIC_ACQUIRE) & bit)) {
-        if (cudaFuncSetAttribute(dense_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDSmem) != cudaSuccess)
+        if (cudaFuncSetAttribute(dense_gemm_kernel<AMN, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDSmem) !=
+            cudaSuccess)
             return NQ_ERR_CUDA;
         __atomic_fetch_or(&init_mask, bit, __ATOMIC_RELEASE);
     }
     return NQ_OK;
 }
 
-// out (M x R, pitch R) = diag(s) A (sum of the parts of Bt)^T [+ rho (D - E)]: A is M x Kp
-// bf16 (K-major), Bt is R x parts Kp bf16 (the parts side by side), Kp a multiple of kDK.
-int dense_launch(const uint16_t* A, const uint16_t* Bt, int parts, int64_t M, int64_t Kp, int64_t R, float* out,
-                 const uint16_t* s, const float* D, const float* E, const float* rho, unsigned* status,
+// out (M x R, pitch R) = diag(s) A (sum of the parts of B)^T [+ rho (D - E)] over K = Kp per
+// part.  A: AMN ? rows_a x M ([K][M], rows_a >= 1, rows past it read as zeros) : M x Kp
+// ([M][K]); B: parts Kp x R ([K][R]) bf16.  M, R multiples of 128, Kp of 64.
+template <bool AMN>
+int dense_launch(const uint16_t* A, int64_t rows_a, const uint16_t* B, int parts, int64_t M, int64_t Kp, int64_t R,
+                 float* out, const uint16_t* s, const float* D, const float* E, const float* rho, unsigned* status,
                  cudaStream_t stream) {
+    int rc = dense_prepare<AMN, true>();
+    if (rc != NQ_OK) return rc;
     CUtensorMap amap, bmap;
-    if (!make_map_bf16(&amap, A, M, Kp) || !make_map_bf16(&bmap, Bt, R, parts * Kp)) return NQ_ERR_CUDA;
+    if (!(AMN ? make_map_bf16_mn(&amap, A, rows_a, M) : make_map_bf16(&amap, A, M, Kp)) ||
+        !make_map_bf16_mn(&bmap, B, parts * Kp, R))
+        return NQ_ERR_CUDA;
     const int nkb = (int)(parts * Kp / kDK), ka_blocks = (int)(Kp / kDK);
-    return launch_pdl(dense_gemm_kernel, dim3((unsigned)(R / kDN), (unsigned)(M / kDM)), dim3(kDThreads), (size_t)kDSmem,
-                      stream, amap, bmap, nkb, ka_blocks, out, R, s, D, E, rho, status) == cudaSuccess
+    return launch_pdl(dense_gemm_kernel<AMN, true>, dim3((unsigned)(R / kDN), (unsigned)(M / kDM)), dim3(kDThreads),
+                      (size_t)kDSmem, stream, amap, bmap, nkb, ka_blocks, out, R, s, D, E, rho, status) == cudaSuccess
                ? NQ_OK
                : NQ_ERR_CUDA;
+}
+
+unsigned split_grid(int64_t pairs) {
+    const int64_t g = (pairs + 255) / 256, cap = 8 * (int64_t)sm_count();
+    return (unsigned)(g < cap ? g : cap);
 }
 }  // namespace
 
@@ -320,36 +317,24 @@ int outer_tc(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch
              void* scratch, unsigned* status, cudaStream_t stream) {
     if (M % kDM || R % kDN || batch <= 0) return NQ_ERR_SHAPE;
     const int64_t Bp = (batch + kDPad - 1) / kDPad * kDPad;
-    uint16_t* At = static_cast<uint16_t*>(scratch);                      // M x Bp
-    uint16_t* Bt = At + ((M * Bp + 127) / 128) * 128;                    // R x 2 Bp (hi | lo)
-    int rc = dense_prepare();
-    if (rc != NQ_OK) return rc;
-    transpose_pad_kernel<<<dim3((unsigned)((M + kTT - 1) / kTT), (unsigned)(Bp / kTT)), 256, 0, stream>>>(a, batch, M,
-                                                                                                       Bp, At);
-    transpose_split_kernel<<<dim3((unsigned)((R + kTT - 1) / kTT), (unsigned)(Bp / kTT)), 256, 0, stream>>>(t, batch, R,
-                                                                                                         Bp, Bt);
+    uint16_t* Bs = static_cast<uint16_t*>(scratch);  // 2 Bp x R: rows of hi, then rows of lo
+    split2_kernel<<<split_grid(Bp * R / 2), 256, 0, stream>>>(t, batch, R, Bp, Bs);
     if (cudaGetLastError() != cudaSuccess) return NQ_ERR_CUDA;
-    return dense_launch(At, Bt, 2, M, Bp, R, out, s, nullptr, nullptr, nullptr, status, stream);
+    // a (batch x M, token-major) read in place: the token rows from batch to Bp are outside
+    // the map and read as zeros
+    return dense_launch<true>(a, batch, Bs, 2, M, Bp, R, out, s, nullptr, nullptr, nullptr, status, stream);
 }
 
-int64_t dense_af_scratch_bytes(int64_t K, int64_t R) { return 2 * (R * 3 * K) + 256; }
+int64_t dense_af_scratch_bytes(int64_t K, int64_t R) { return 2 * (3 * K * R) + 256; }
 
-int dense_af(const uint16_t* A, int64_t M, int64_t K, const float* F, int64_t R, float* out, const float* D,
-             const float* E, const float* rho, void* scratch, unsigned* status, cudaStream_t stream) {
+int dense_af(const uint16_t* A, bool a_kmajor_rows, int64_t M, int64_t K, const float* F, int64_t R, float* out,
+             const float* D, const float* E, const float* rho, void* scratch, unsigned* status, cudaStream_t stream) {
     if (M % kDM || R % kDN || K % kDK || K <= 0) return NQ_ERR_SHAPE;
-    uint16_t* Bt = static_cast<uint16_t*>(scratch);  // R x 3K (hi | mid | lo)
-    int rc = dense_prepare();
-    if (rc != NQ_OK) return rc;
-    transpose_split3_kernel<<<dim3((unsigned)((R + kTT - 1) / kTT), (unsigned)(K / kTT)), 256, 0, stream>>>(F, K, R, Bt);
+    uint16_t* Bs = static_cast<uint16_t*>(scratch);  // 3K x R: rows of hi, mid, lo
+    split3_kernel<<<split_grid(K * R / 2), 256, 0, stream>>>(F, K, R, Bs);
     if (cudaGetLastError() != cudaSuccess) return NQ_ERR_CUDA;
-    return dense_launch(A, Bt, 3, M, K, R, out, nullptr, D, E, rho, status, stream);
-}
-
-int transpose_bf16_device(const uint16_t* src, int64_t rows, int64_t cols, uint16_t* dst, cudaStream_t stream) {
-    if (rows % kTT || cols % kTT) return NQ_ERR_SHAPE;
-    transpose_pad_kernel<<<dim3((unsigned)(cols / kTT), (unsigned)(rows / kTT)), 256, 0, stream>>>(src, rows, cols, rows,
-                                                                                                dst);
-    return cudaGetLastError() == cudaSuccess ? NQ_OK : NQ_ERR_CUDA;
+    return a_kmajor_rows ? dense_launch<false>(A, M, Bs, 3, M, K, R, out, nullptr, D, E, rho, status, stream)
+                         : dense_launch<true>(A, K, Bs, 3, M, K, R, out, nullptr, D, E, rho, status, stream);
 }
 
 }  // namespace nq

@@ -37,7 +37,7 @@ struct Workspace {
     size_t ones_count = 0, gstage_bytes = 0;
     float* env = nullptr;          // envelope terms 1 .. l-1: (l-1) x batch x m fp32
     size_t env_bytes = 0;
-    void* dense = nullptr;         // factor gradients on the tensor cores: transposed operands
+    void* dense = nullptr;         // factor gradients on the tensor cores: the split rank vectors
     size_t dense_bytes = 0;
     size_t t_cap = 0, tgmax_cap = 0, partial_cap = 0, counter_cap = 0;
     int64_t r_cap = 0, n_cap = 0, m_cap = 0, batch_cap = 0, rsum_cap = 0;
@@ -107,14 +107,13 @@ int prefill_rank_vector(const uint16_t* x, const uint32_t* Vpk, const uint16_t* 
 int64_t outer_tc_scratch_bytes(int64_t batch, int64_t M, int64_t R);
 int outer_tc(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch, int64_t M, int64_t R, float* out,
              void* scratch, unsigned* status, cudaStream_t stream);
-// out (M x R fp32) = A F + rho (D - E) on the tensor cores: A is M x K bfloat16 (row pitch K,
-// K a multiple of 64), F is K x R fp32 split into three bfloat16 parts (scratch of
-// dense_af_scratch_bytes), D and E laid out as out, rho a device scalar; M, R multiples of 128.
+// out (M x R fp32) = Aop F + rho (D - E) on the tensor cores: Aop is M x K with A bfloat16
+// given as M x K rows (a_kmajor_rows) or as K x M rows (Aop = A^T: read in place), K a
+// multiple of 64; F is K x R fp32 split into three bfloat16 parts (scratch of
+// dense_af_scratch_bytes); D and E laid out as out, rho a device scalar; M, R multiples of 128.
 int64_t dense_af_scratch_bytes(int64_t K, int64_t R);
-int dense_af(const uint16_t* A, int64_t M, int64_t K, const float* F, int64_t R, float* out, const float* D,
-             const float* E, const float* rho, void* scratch, unsigned* status, cudaStream_t stream);
-// dst (cols x rows) = src^T for a rows x cols bfloat16 matrix (both multiples of 64)
-int transpose_bf16_device(const uint16_t* src, int64_t rows, int64_t cols, uint16_t* dst, cudaStream_t stream);
+int dense_af(const uint16_t* A, bool a_kmajor_rows, int64_t M, int64_t K, const float* F, int64_t R, float* out,
+             const float* D, const float* E, const float* rho, void* scratch, unsigned* status, cudaStream_t stream);
 // out[i][k] = s[i] * sum over b (increasing) of bf16(a[b][i]) * t[b][k]: M x R fp32
 int outer_device(const uint16_t* a, const uint16_t* s, const float* t, int64_t batch, int64_t M, int64_t R,
                  float* out, cudaStream_t stream);

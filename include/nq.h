@@ -369,8 +369,8 @@ int nq_lowrank_linear_fwd_noalloc(const void* x, const uint32_t* Upk, const uint
  * fixed order.  Arithmetic in fp32 (W read exactly from bf16), reductions of norms in fp64;
  * the iterations' products W B and W^T A run on the tensor cores with W in bf16 and the
  * fp32 factor as the sum of three bf16 parts (fp32's precision), accumulated in fp32 (the
- * iterating calls also hold a transposed copy of W and the split factor in their scratch:
- * 2mn + 6 max(m, n) r bytes more).  A bounded wait that gives up returns NQ_ERR_TIMEOUT.
+ * iterating calls hold the split factor in their scratch: 6 max(m, n) r bytes more).  A
+ * bounded wait that gives up returns NQ_ERR_TIMEOUT.
  */
 
 /*
