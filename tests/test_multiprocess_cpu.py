@@ -79,3 +79,21 @@ def test_reference_arm_rank0_json_line():
     assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["value"] > 0
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] >= 1
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_backward_workload():
+    """The oracle arm of `--workload backward`: one JSON line in TFLOP/s with the workload
+    string the GPU arm prints for the same token batch."""
+    import json
+
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                          "backward", "--backward-batch", "1024", "--cpu-seconds", "0.1"], env=env,
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["unit"] == "TFLOP/s" and rec["value"] > 0
+    assert rec["config"]["workload"] == "factor and scale gradients, 11008x4096 r=2432 layer, 1024 tokens"
+    assert rec["cpu_baseline"]["kind"] == "oracle"
